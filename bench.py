@@ -1,0 +1,427 @@
+"""Benchmark of the block-sparse video attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload wan13b] [--order hilbert]
+    python bench.py --impl reference ...      # the fp64 CPU oracle as the reference arm
+
+One step = the whole path over one synthetic layer already resident in HBM:
+svsa_build_perm, svsa_reorder x3 (Q, K, V), svsa_build_mask, svsa_attn_fwd,
+svsa_inverse_reorder.  Each timed step is bracketed by CUDA events on the
+launching stream, with an L2 flush (a 512 MiB write) between steps, outside
+the events.  `value` = kept-block attention FLOPs of all ranks / the slowest
+rank's time (TFLOP/s).  Ranks run independent layers (weak scaling, no
+collective on the data path; only the timing max is reduced).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "block-sparse attn fwd ms & kept-FLOP TFLOP/s (% BF16 peak); speedup vs dense"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+ATTN_KERNEL_SRC = os.path.join(ROOT, "block_sparse_attention_hilbert_b200", "csrc", "attn_mma.cu")
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="svsa", choices=["svsa", "reference"])
+    ap.add_argument("--workload", default="wan13b", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--order", default=None, choices=["raster", "hilbert"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws == 1:
+        return 0, 1, 0
+    import datetime
+    import torch.distributed as dist
+    rank = int(os.environ["RANK"])
+    local = int(os.environ.get("LOCAL_RANK", rank))
+    backend = "nccl" if torch.cuda.is_available() else "gloo"
+    if torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, ws, local
+
+
+def _barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _workload(args):
+    w = workloads.WORKLOADS[args.workload]
+    if args.order:
+        w = w.with_(order=args.order)
+    return w
+
+
+def kept_flops_from_lists(kv_idx: np.ndarray, kv_cnt: np.ndarray, nvalid: np.ndarray, d: int) -> float:
+    """4 * d * sum over kept (I, J) of n_I * n_J, from the compacted lists."""
+    nb = nvalid.shape[0]
+    cap = kv_idx.shape[-1]
+    idx = kv_idx.reshape(-1, nb, cap)
+    cnt = kv_cnt.reshape(-1, nb)
+    mask = np.arange(cap)[None, None, :] < cnt[..., None]
+    nJ = np.where(mask, nvalid[np.clip(idx, 0, nb - 1)], 0).sum(-1)       # [BH, nb]
+    return 4.0 * d * float((nJ * nvalid[None, :]).sum())
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"svsa_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for n, flag in zip(names, r[3][1:]):
+                if flag.lower().startswith("active"):
+                    reasons.add(n)
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows), "samples": len(rows), "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------------------- traffic
+def _attn_traffic(workload: str):
+    """dram bytes per attention launch from the committed ncu summary, if it was
+    taken on the current kernel source (else null)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"attn_{workload}.traffic")
+    if not os.path.exists(path):
+        return None
+    kv = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                a, b = line.split(":", 1)
+                kv[a.strip()] = b.strip()
+    with open(ATTN_KERNEL_SRC, "rb") as f:
+        h = hashlib.sha256(f.read()).hexdigest()[:16]
+    if kv.get("kernel_sha256_16") != h:
+        return None
+    try:
+        return float(kv["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# --------------------------------------------------------------------------- oracle arm
+def _oracle_sample(w, q, k, v, seconds: float, perm_cache=None):
+    """Time the fp64 oracle on a bounded sample of the layer: the full permutation,
+    then head by head the pooling, the mask rows and the attention of query
+    blocks until `seconds` elapse.  Returns (kept_flops, elapsed, description)."""
+    import oracle
+    from threadpoolctl import threadpool_info
+    t0 = time.perf_counter()
+    perm, _ = perm_cache if perm_cache is not None else oracle.build_perm(w.T, w.H, w.W, w.order)
+    flops = 0.0
+    blocks = 0
+    heads_done = 0
+    nb = w.nb
+    k_keep = oracle.topk_count(w.keep_frac, nb)
+    for eta in range(w.heads):
+        qp, kp, vp = (oracle.reorder(t[0, eta].float().cpu().numpy().astype(np.float64), perm) for t in (q, k, v))
+        qb, nv = oracle.pool(qp, w.N)
+        kb, _ = oracle.pool(kp, w.N)
+        heads_done += 1
+        for I in range(nb):
+            if w.select == "structured":
+                keep_row = oracle.structured_mask(perm, w.T, w.H, w.W, win_t=w.win_t, win_rows=w.win_rows,
+                                                  n_anchors=w.n_anchors, anchor_offset=0)[I]
+            else:
+                if w.sub_block == 64:
+                    S = oracle.block_scores(qb[I:I + 1], kb)[0]
+                else:
+                    S = oracle.subblock_scores(qp, kp, w.N, w.sub_block, rows=[I])[0]
+                if w.select == "topk":
+                    keep_row, _ = oracle.select_topk(S, k_keep)
+                else:
+                    keep_row, _ = oracle.select_threshold(S, w.tau)
+            keep = np.zeros((nb, nb), dtype=bool)
+            keep[I] = keep_row
+            oracle.masked_attention(qp, kp, vp, w.N, keep, q_blocks=[I])
+            flops += oracle.kept_flops(keep, nv, w.d)
+            blocks += 1
+            if time.perf_counter() - t0 >= seconds:
+                break
+        if time.perf_counter() - t0 >= seconds:
+            break
+    elapsed = time.perf_counter() - t0
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    desc = (f"{w.name}: full {w.order} permutation, then per head pooling + mask row + exact attention "
+            f"of {blocks} query blocks over {heads_done} head(s) (of {w.heads} x {nb}); "
+            f"{flops / 1e12:.4f} kept TFLOP in {elapsed:.1f} s")
+    return flops, elapsed, desc, threads
+
+
+def run_reference(args):
+    rank, ws, _ = int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), 0
+    if rank != 0:
+        return
+    import oracle
+    w = _workload(args)
+    q, k, v = workloads.make_qkv(w, device="cpu")
+    perm_cache = oracle.build_perm(w.T, w.H, w.W, w.order)
+    per_step = max(0.5, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        _oracle_sample(w, q, k, v, per_step, perm_cache)
+    tot_f, tot_t, desc, threads = 0.0, 0.0, "", 1
+    for _ in range(args.steps):
+        f, t, desc, threads = _oracle_sample(w, q, k, v, per_step, perm_cache)
+        tot_f += f
+        tot_t += t
+    value = tot_f / tot_t / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "heads": w.heads, "d": w.d, "grid": [w.T, w.H, w.W],
+                       "N": w.N, "order": w.order, "select": w.select},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": f"each step: {desc}"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- GPU arm
+def run_svsa(args):
+    rank, ws, local = _dist()
+    import block_sparse_attention_hilbert_b200 as svsa
+    assert torch.cuda.is_available(), "bench.py needs a GPU"
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    svsa.lib()
+    w = _workload(args)
+    stream = torch.cuda.current_stream()
+    q, k, v = workloads.make_qkv(w, seed=rank, device=dev)
+    attn = svsa.SparseVideoAttention(w.B, w.heads, w.T, w.H, w.W, w.d, order=w.order, select=w.select,
+                                     tau=w.tau, keep_frac=w.keep_frac, sub_block=w.sub_block,
+                                     win_t=w.win_t, win_rows=w.win_rows,
+                                     n_anchors=w.n_anchors if w.select == "structured" else 0,
+                                     routing=w.routing, compensate=w.compensate, device=dev)
+    out = torch.empty_like(q)
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    off = workloads.anchor_offset(seed=0, step=0, nkb=w.nb, n_anchors=w.n_anchors) if w.select == "structured" else 0
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record(stream)
+        attn.build_perm()
+        if evs is not None:
+            evs[1].record(stream)
+        attn.reorder(q, k, v)
+        if evs is not None:
+            evs[2].record(stream)
+        attn.build_mask(off)
+        if evs is not None:
+            evs[3].record(stream)
+        attn.attend()
+        if evs is not None:
+            evs[4].record(stream)
+        attn.inverse(out)
+        if evs is not None:
+            evs[5].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    nvalid = np.minimum(64, w.N - 64 * np.arange(w.nb)).astype(np.int64)
+    kflops = kept_flops_from_lists(attn.buf.kv_idx.cpu().numpy(), attn.buf.kv_cnt.cpu().numpy(), nvalid, w.d)
+    dense_flops = 4.0 * w.d * float(w.N) ** 2 * w.heads * w.B
+    density = kflops / dense_flops
+
+    phases = ["perm", "reorder", "mask", "attn", "inverse"]
+    times = {p: [] for p in phases}
+    launches0 = svsa.svsa_launch_count()
+    _barrier(ws)
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        for _ in range(args.steps):
+            flush.fill_(1.0)
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+            step(evs)
+            torch.cuda.synchronize()
+            for i, p in enumerate(phases):
+                times[p].append(evs[i].elapsed_time(evs[i + 1]))
+    torch.cuda.synchronize()
+    _barrier(ws)
+    launches = svsa.svsa_launch_count() - launches0
+    step_ms_local = sum(sum(times[p]) for p in phases) / args.steps
+    step_ms = _max_over_ranks(step_ms_local, ws)
+    attn_ms_local = statistics.mean(times["attn"])
+    attn_ms = _max_over_ranks(attn_ms_local, ws)
+
+    # dense denominator: same arithmetic over every key block
+    dtimes = []
+    for i in range(args.warmup + args.steps):
+        flush.fill_(1.0)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        attn.attend_dense()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            dtimes.append(e0.elapsed_time(e1))
+    dense_ms = _max_over_ranks(statistics.mean(dtimes), ws)
+
+    # end to end through the public API: pinned host Q, K, V in, O back to the host
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    dq, dk, dv = (torch.empty_like(t) for t in (q, k, v))
+    e2e_times = []
+    for i in range(args.warmup + args.steps):
+        flush.fill_(1.0)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for h, d_ in ((hq, dq), (hk, dk), (hv, dv)):
+            d_.copy_(h, non_blocking=True)
+        attn(dq, dk, dv, out=out, anchor_offset=off)
+        hout.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            e2e_times.append(e0.elapsed_time(e1))
+    e2e_ms = _max_over_ranks(statistics.mean(e2e_times), ws)
+    h2d = 3 * q.numel() * q.element_size()
+    d2h = out.numel() * out.element_size()
+
+    peaks, peak_src = _peaks()
+    peak = float(peaks["bf16_tflops"])
+    attn_tflops = kflops / (attn_ms * 1e-3) / 1e12
+    value = ws * kflops / (step_ms * 1e-3) / 1e12
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        f, t, desc, threads = _oracle_sample(w, q, k, v, args.cpu_seconds)
+        cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        reorder_bytes = 3 * (w.B * w.heads * (w.N + w.Npad) * w.d * 2)
+        inverse_bytes = w.B * w.heads * (w.N + w.Npad) * w.d * 2
+        reorder_ms = statistics.mean(times["reorder"])
+        inverse_ms = statistics.mean(times["inverse"])
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "heads": w.heads, "d": w.d, "grid": [w.T, w.H, w.W],
+                       "N": w.N, "order": w.order, "select": w.select, "keep_frac": w.keep_frac,
+                       "tau": w.tau, "sub_block": w.sub_block, "routing": w.routing,
+                       "compensate": w.compensate, "l2": "flushed (512 MiB write) between timed steps",
+                       "parallelism": f"independent layer per GPU x{ws}"},
+            "attn_ms": attn_ms, "attn_tflops": attn_tflops, "attn_frac_of_peak": attn_tflops / peak,
+            "dense_ms": dense_ms, "dense_tflops": dense_flops / (dense_ms * 1e-3) / 1e12,
+            "speedup_vs_dense": dense_ms / attn_ms, "density": density,
+            "kept_tflop_per_step": kflops / 1e12,
+            "phase_ms": {p: statistics.mean(times[p]) for p in phases},
+            "reorder_gbs": reorder_bytes / (reorder_ms * 1e-3) / 1e9,
+            "inverse_gbs": inverse_bytes / (inverse_ms * 1e-3) / 1e9,
+            "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
+                         "frac": attn_tflops / peak, "traffic": _attn_traffic(w.name),
+                         "kernel": "svsa attention (kept-block FLOPs / launch time)",
+                         "peak_source": f"{peak_src} bf16_tflops (burst)"},
+            "e2e": {"value": ws * kflops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "clocks": clk.summary(),
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    args = _args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_svsa(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,180 @@
+"""Python binding of libsvsa, the B200 block-sparse video attention library.
+
+Argument marshalling only: each function passes raw device pointers, sizes and
+the current CUDA stream to the C entry point of the same name (see
+include/svsa.h) and raises SvsaError on a non-zero status.  Every step of the
+computation runs in the library's CUDA kernels; torch supplies device memory
+and streams.  If the shared library is missing, importing works but every
+call raises -- there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "lib", "libsvsa.so")
+
+ORDER_RASTER, ORDER_HILBERT = 0, 1
+SEL_THRESHOLD, SEL_TOPK, SEL_STRUCTURED = 0, 1, 2
+BLOCK = 64
+
+STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: "CUDA", 5: "TIMEOUT"}
+
+
+class SvsaError(RuntimeError):
+    def __init__(self, status: int, fn: str, msg: str):
+        super().__init__(f"{fn}: {STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("heads", ctypes.c_int32), ("T", ctypes.c_int32),
+                ("H", ctypes.c_int32), ("W", ctypes.c_int32), ("d", ctypes.c_int32)]
+
+
+class MaskParams(ctypes.Structure):
+    _fields_ = [("select", ctypes.c_int32), ("tau", ctypes.c_float), ("keep_frac", ctypes.c_float),
+                ("sub_block", ctypes.c_int32), ("win_t", ctypes.c_int32), ("win_rows", ctypes.c_int32),
+                ("n_anchors", ctypes.c_int32), ("anchor_offset", ctypes.c_int32),
+                ("routing", ctypes.c_int32)]
+
+
+class Mask(ctypes.Structure):
+    _fields_ = [("kv_idx", ctypes.c_void_p), ("kv_cnt", ctypes.c_void_p), ("cap", ctypes.c_int32),
+                ("bits", ctypes.c_void_p), ("kbar", ctypes.c_void_p), ("vbar", ctypes.c_void_p),
+                ("nvalid", ctypes.c_void_p)]
+
+
+_lib = None
+
+_SIGS = {
+    "svsa_perm_workspace_bytes": (ctypes.c_size_t, [Shape, ctypes.c_int32]),
+    "svsa_build_perm": (ctypes.c_int, [Shape, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                                       ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "svsa_reorder": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, Shape,
+                                    ctypes.c_void_p]),
+    "svsa_mask_workspace_bytes": (ctypes.c_size_t, [Shape, ctypes.POINTER(MaskParams)]),
+    "svsa_build_mask": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                       ctypes.c_void_p, Shape, ctypes.POINTER(MaskParams),
+                                       ctypes.POINTER(Mask), ctypes.c_void_p, ctypes.c_size_t,
+                                       ctypes.c_void_p]),
+    "svsa_attn_fwd": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                     ctypes.POINTER(Mask), ctypes.c_int32, ctypes.c_void_p,
+                                     ctypes.c_void_p, Shape, ctypes.c_void_p]),
+    "svsa_attn_dense_fwd": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                           ctypes.c_void_p, ctypes.c_void_p, Shape, ctypes.c_void_p]),
+    "svsa_inverse_reorder": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, Shape,
+                                            ctypes.c_void_p]),
+    "svsa_sync_status": (ctypes.c_int, [ctypes.c_void_p]),
+    "svsa_last_error": (ctypes.c_char_p, []),
+    "svsa_version": (ctypes.c_char_p, []),
+    "svsa_launch_count": (ctypes.c_ulonglong, []),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libsvsa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m block_sparse_attention_hilbert_b200.build`")
+        h = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(h, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = h
+    return _lib
+
+
+def exported_symbols():
+    return list(_SIGS)
+
+
+def _check(status: int, fn: str) -> None:
+    if status != 0:
+        raise SvsaError(status, fn, lib().svsa_last_error().decode())
+
+
+def _p(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream=None) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def shape(B: int, heads: int, T: int, H: int, W: int, d: int) -> Shape:
+    return Shape(B, heads, T, H, W, d)
+
+
+def mask_params(select: int = SEL_THRESHOLD, tau: float = 0.9, keep_frac: float = 0.25,
+                sub_block: int = 64, win_t: int = 2, win_rows: int = 1, n_anchors: int = 0,
+                anchor_offset: int = 0, routing: bool = False) -> MaskParams:
+    return MaskParams(select, tau, keep_frac, sub_block, win_t, win_rows, n_anchors, anchor_offset,
+                      int(routing))
+
+
+def make_mask(kv_idx, kv_cnt, cap: int, bits=None, kbar=None, vbar=None, nvalid=None) -> Mask:
+    return Mask(_p(kv_idx), _p(kv_cnt), cap, _p(bits), _p(kbar), _p(vbar), _p(nvalid))
+
+
+def version() -> str:
+    return lib().svsa_version().decode()
+
+
+def svsa_perm_workspace_bytes(s: Shape, order: int) -> int:
+    return int(lib().svsa_perm_workspace_bytes(s, order))
+
+
+def svsa_build_perm(s: Shape, order: int, perm, iperm, ws=None, ws_bytes: int = 0, stream=None) -> None:
+    _check(lib().svsa_build_perm(s, order, _p(perm), _p(iperm), _p(ws), ws_bytes, _stream(stream)),
+           "svsa_build_perm")
+
+
+def svsa_reorder(x, xp, perm, s: Shape, stream=None) -> None:
+    _check(lib().svsa_reorder(_p(x), _p(xp), _p(perm), s, _stream(stream)), "svsa_reorder")
+
+
+def svsa_mask_workspace_bytes(s: Shape, p: MaskParams) -> int:
+    return int(lib().svsa_mask_workspace_bytes(s, ctypes.byref(p)))
+
+
+def svsa_build_mask(qp, kp, vp, perm, s: Shape, p: MaskParams, m: Mask, ws=None, ws_bytes: int = 0,
+                    stream=None) -> None:
+    _check(lib().svsa_build_mask(_p(qp), _p(kp), _p(vp), _p(perm), s, ctypes.byref(p), ctypes.byref(m),
+                                 _p(ws), ws_bytes, _stream(stream)), "svsa_build_mask")
+
+
+def svsa_attn_fwd(qp, kp, vp, m: Mask, compensate: bool, op, lse, s: Shape, stream=None) -> None:
+    _check(lib().svsa_attn_fwd(_p(qp), _p(kp), _p(vp), ctypes.byref(m), int(compensate), _p(op), _p(lse),
+                               s, _stream(stream)), "svsa_attn_fwd")
+
+
+def svsa_attn_dense_fwd(qp, kp, vp, op, lse, s: Shape, stream=None) -> None:
+    _check(lib().svsa_attn_dense_fwd(_p(qp), _p(kp), _p(vp), _p(op), _p(lse), s, _stream(stream)),
+           "svsa_attn_dense_fwd")
+
+
+def svsa_inverse_reorder(op, o, iperm, s: Shape, stream=None) -> None:
+    _check(lib().svsa_inverse_reorder(_p(op), _p(o), _p(iperm), s, _stream(stream)), "svsa_inverse_reorder")
+
+
+def svsa_launch_count() -> int:
+    return int(lib().svsa_launch_count())
+
+
+def svsa_sync_status(stream=None) -> None:
+    _check(lib().svsa_sync_status(_stream(stream)), "svsa_sync_status")
+
+
+from .pipeline import SparseVideoAttention, LayerBuffers  # noqa: E402,F401

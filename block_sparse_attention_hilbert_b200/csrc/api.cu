@@ -1,0 +1,369 @@
+// C ABI of libsvsa: argument validation, workspace layout, kernel launches.
+// Every entry point validates before launching anything, returns a status
+// and never throws across the boundary.
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "common.cuh"
+#include "svsa.h"
+
+namespace svsa {
+// kernels (one translation unit each)
+cudaError_t launch_build_perm(int T, int H, int W, int hilbert, int32_t* perm, int32_t* iperm,
+                              void* ws, cudaStream_t st);
+size_t perm_workspace_bytes(int T, int H, int W);
+int hilbert_order_bits(int T, int H, int W);
+cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* map, long long BH,
+                               long long rows_dst, long long rows_src, int d, cudaStream_t st);
+cudaError_t launch_pool(const void* xp, float* out, int32_t* nvalid, long long BH, long long N,
+                        long long Npad, int d, int size, cudaStream_t st);
+cudaError_t launch_nvalid(int32_t* nvalid, long long N, int nb, cudaStream_t st);
+cudaError_t launch_scores(const float* qs, const float* ks, float* S, long long BH, long long N,
+                          int ng, int nb, int d, int size, cudaStream_t st);
+cudaError_t launch_select(const float* S, const float* R, long long rows, int nb, int mode, float tau,
+                          int k, int cap, int32_t* kv_idx, int32_t* kv_cnt, uint32_t* bits,
+                          cudaStream_t st);
+cudaError_t launch_structured(const int32_t* perm, long long rows, int nb, int H, int W, int win_t,
+                              int R, int n_anchors, int anchor_offset, int cap, int32_t* kv_idx,
+                              int32_t* kv_cnt, uint32_t* bits, cudaStream_t st);
+cudaError_t launch_route(const float* qbar, const void* kp, const void* vp, const float* kbar,
+                         const float* vbar, float* R, float* Rm, long long BH, long long N, int nb,
+                         int d, cudaStream_t st);
+cudaError_t launch_attn_mma(const void* q, const void* k, const void* v, const int32_t* kv_idx,
+                            const int32_t* kv_cnt, int cap, const float* kbar, const float* vbar,
+                            const int32_t* nvalid, void* o, float* lse, long long BH, long long N,
+                            int nb, int d, bool dense, bool comp, cudaStream_t st);
+}  // namespace svsa
+
+using namespace svsa;
+
+namespace {
+
+thread_local std::string g_last_error;
+std::atomic<unsigned long long> g_launches{0};
+
+// Count `n` kernel launches once a launch helper reported success.
+cudaError_t counted(cudaError_t e, int n) {
+  if (e == cudaSuccess) g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed);
+  return e;
+}
+
+svsa_status fail(svsa_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+svsa_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return SVSA_OK;
+  return fail(SVSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int kMaxBlocks = 16384;
+
+svsa_status check_shape(const svsa_shape& s, bool need_heads) {
+  if (s.T < 1 || s.H < 1 || s.W < 1)
+    return fail(SVSA_ERR_INVALID_ARG, "grid dims must be >= 1 (T=%d H=%d W=%d)", s.T, s.H, s.W);
+  const long long N = (long long)s.T * s.H * s.W;
+  if (N >= (1LL << 31)) return fail(SVSA_ERR_UNSUPPORTED, "N = T*H*W = %lld exceeds int32", N);
+  if (need_heads) {
+    if (s.B < 1 || s.heads < 1)
+      return fail(SVSA_ERR_INVALID_ARG, "B and heads must be >= 1 (B=%d heads=%d)", s.B, s.heads);
+    if (s.d != 64 && s.d != 128) return fail(SVSA_ERR_UNSUPPORTED, "head dim d=%d (supported: 64, 128)", s.d);
+    const Dims g = make_dims(s.B, s.heads, s.T, s.H, s.W, s.d);
+    if (g.BH * g.Npad * s.d >= (1LL << 31))
+      return fail(SVSA_ERR_UNSUPPORTED, "B*heads*Npad*d = %lld exceeds int32", g.BH * g.Npad * s.d);
+  }
+  return SVSA_OK;
+}
+
+#define SVSA_TRY(expr)                   \
+  do {                                   \
+    svsa_status _s = (expr);             \
+    if (_s != SVSA_OK) return _s;        \
+  } while (0)
+
+#define SVSA_PTR(p, name)                                                                      \
+  do {                                                                                         \
+    if ((p) == nullptr) return fail(SVSA_ERR_INVALID_ARG, "%s is NULL", name);                 \
+    if (!aligned16(p)) return fail(SVSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);   \
+  } while (0)
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Workspace layout of svsa_build_mask.
+struct MaskWs {
+  size_t qpool, kpool, S, R, Rm, qbar64, total;
+};
+
+MaskWs mask_ws_layout(const Dims& g, const svsa_mask_params& p, bool have_kbar) {
+  MaskWs w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off += align256(bytes); return o; };
+  const size_t f = sizeof(float);
+  if (p.select == SVSA_SEL_STRUCTURED) {
+    w.total = 0;
+    return w;
+  }
+  const int sub = p.sub_block;
+  const long long ng = g.Npad / sub;
+  w.qpool = take((size_t)g.BH * ng * g.d * f);
+  // key pooling can go straight into the caller's kbar when block-level
+  w.kpool = (sub == kBlock && have_kbar) ? SIZE_MAX : take((size_t)g.BH * ng * g.d * f);
+  w.S = take((size_t)g.BH * g.nb * g.nb * f);
+  w.R = w.Rm = w.qbar64 = SIZE_MAX;
+  if (p.routing) {
+    w.R = take((size_t)g.BH * g.nb * g.nb * f);
+    w.Rm = take((size_t)g.BH * g.nb * g.nb * f);
+    if (sub != kBlock) w.qbar64 = take((size_t)g.BH * g.nb * g.d * f);
+  }
+  w.total = off;
+  return w;
+}
+
+svsa_status check_params(const svsa_mask_params* p, const Dims& g) {
+  if (p == nullptr) return fail(SVSA_ERR_INVALID_ARG, "params is NULL");
+  if (p->select < 0 || p->select > 2) return fail(SVSA_ERR_INVALID_ARG, "select=%d unknown", p->select);
+  if (p->select != SVSA_SEL_STRUCTURED && p->sub_block != 64 && p->sub_block != 16)
+    return fail(SVSA_ERR_UNSUPPORTED, "sub_block=%d (supported: 64, 16)", p->sub_block);
+  if (p->select == SVSA_SEL_THRESHOLD && !(p->tau >= 0.f))
+    return fail(SVSA_ERR_INVALID_ARG, "tau=%g must be >= 0", (double)p->tau);
+  if (p->select == SVSA_SEL_TOPK && !(p->keep_frac >= 0.f))
+    return fail(SVSA_ERR_INVALID_ARG, "keep_frac=%g must be >= 0", (double)p->keep_frac);
+  if (p->routing && p->select != SVSA_SEL_THRESHOLD)
+    return fail(SVSA_ERR_INVALID_ARG, "routing needs select = THRESHOLD (its budget)");
+  if (p->select == SVSA_SEL_STRUCTURED) {
+    if (p->win_t < 0 || p->win_rows < 0 || p->n_anchors < 0 || p->n_anchors > g.nb)
+      return fail(SVSA_ERR_INVALID_ARG, "structured window/anchors out of range");
+    if (p->n_anchors > 0) {
+      const int stride = std::max(g.nb / p->n_anchors, 1);
+      if (p->anchor_offset < 0 || p->anchor_offset >= stride)
+        return fail(SVSA_ERR_INVALID_ARG, "anchor_offset=%d not in [0, %d)", p->anchor_offset, stride);
+    }
+  }
+  if (g.nb > kMaxBlocks) return fail(SVSA_ERR_UNSUPPORTED, "nb=%d blocks exceeds %d", g.nb, kMaxBlocks);
+  return SVSA_OK;
+}
+
+int topk_count(float keep_frac, int nb) {
+  double k = std::ceil((double)keep_frac * (double)nb);
+  if (k < 1.0) k = 1.0;
+  if (k > nb) k = nb;
+  return (int)k;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* svsa_last_error(void) { return g_last_error.c_str(); }
+
+const char* svsa_version(void) { return "svsa 0.1.0 (sm_100a)"; }
+
+unsigned long long svsa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+size_t svsa_perm_workspace_bytes(svsa_shape s, int32_t order) {
+  if (order != SVSA_ORDER_HILBERT || s.T < 1 || s.H < 1 || s.W < 1) return 0;
+  if (hilbert_order_bits(s.T, s.H, s.W) > 10) return 0;
+  return perm_workspace_bytes(s.T, s.H, s.W);
+}
+
+svsa_status svsa_build_perm(svsa_shape s, int32_t order, int32_t* perm, int32_t* iperm, void* ws,
+                            size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  SVSA_TRY(check_shape(s, false));
+  if (order != SVSA_ORDER_RASTER && order != SVSA_ORDER_HILBERT)
+    return fail(SVSA_ERR_INVALID_ARG, "order=%d unknown", order);
+  SVSA_PTR(perm, "perm");
+  SVSA_PTR(iperm, "iperm");
+  if (order == SVSA_ORDER_HILBERT) {
+    if (hilbert_order_bits(s.T, s.H, s.W) > 10)
+      return fail(SVSA_ERR_UNSUPPORTED, "Hilbert order needs max(T,H,W) <= 1024");
+    const size_t need = perm_workspace_bytes(s.T, s.H, s.W);
+    SVSA_PTR(ws, "ws");
+    if (ws_bytes < need) return fail(SVSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need);
+  }
+  return cuda_status(counted(launch_build_perm(s.T, s.H, s.W, order == SVSA_ORDER_HILBERT, perm, iperm, ws,
+                                               (cudaStream_t)stream),
+                             order == SVSA_ORDER_HILBERT ? 5 : 1),
+                     "build_perm launch");
+}
+
+svsa_status svsa_reorder(const void* x, void* xp, const int32_t* perm, svsa_shape s, void* stream) {
+  g_last_error.clear();
+  SVSA_TRY(check_shape(s, true));
+  SVSA_PTR(x, "x");
+  SVSA_PTR(xp, "xp");
+  SVSA_PTR(perm, "perm");
+  if (x == xp) return fail(SVSA_ERR_INVALID_ARG, "x and xp must not alias");
+  const Dims g = make_dims(s.B, s.heads, s.T, s.H, s.W, s.d);
+  return cuda_status(counted(launch_gather_rows(x, xp, perm, g.BH, g.Npad, g.N, g.d, (cudaStream_t)stream), 1),
+                     "reorder launch");
+}
+
+svsa_status svsa_inverse_reorder(const void* op, void* o, const int32_t* iperm, svsa_shape s, void* stream) {
+  g_last_error.clear();
+  SVSA_TRY(check_shape(s, true));
+  SVSA_PTR(op, "op");
+  SVSA_PTR(o, "o");
+  SVSA_PTR(iperm, "iperm");
+  if (op == o) return fail(SVSA_ERR_INVALID_ARG, "op and o must not alias");
+  const Dims g = make_dims(s.B, s.heads, s.T, s.H, s.W, s.d);
+  return cuda_status(counted(launch_gather_rows(op, o, iperm, g.BH, g.N, g.Npad, g.d, (cudaStream_t)stream), 1),
+                     "inverse_reorder launch");
+}
+
+size_t svsa_mask_workspace_bytes(svsa_shape s, const svsa_mask_params* p) {
+  if (p == nullptr || s.T < 1 || s.H < 1 || s.W < 1 || s.B < 1 || s.heads < 1) return 0;
+  if (p->select != SVSA_SEL_STRUCTURED && p->sub_block != 64 && p->sub_block != 16) return 0;
+  const Dims g = make_dims(s.B, s.heads, s.T, s.H, s.W, s.d);
+  // sized for the worst case (caller's kbar/vbar absent)
+  return mask_ws_layout(g, *p, false).total;
+}
+
+svsa_status svsa_build_mask(const void* qp, const void* kp, const void* vp, const int32_t* perm,
+                            svsa_shape s, const svsa_mask_params* p, const svsa_mask* m, void* ws,
+                            size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  SVSA_TRY(check_shape(s, true));
+  const Dims g = make_dims(s.B, s.heads, s.T, s.H, s.W, s.d);
+  SVSA_TRY(check_params(p, g));
+  if (m == nullptr) return fail(SVSA_ERR_INVALID_ARG, "mask is NULL");
+  SVSA_PTR(m->kv_idx, "mask.kv_idx");
+  SVSA_PTR(m->kv_cnt, "mask.kv_cnt");
+  if (m->bits != nullptr && !aligned16(m->bits)) return fail(SVSA_ERR_INVALID_ARG, "mask.bits misaligned");
+  if (m->kbar != nullptr && !aligned16(m->kbar)) return fail(SVSA_ERR_INVALID_ARG, "mask.kbar misaligned");
+  if (m->vbar != nullptr && !aligned16(m->vbar)) return fail(SVSA_ERR_INVALID_ARG, "mask.vbar misaligned");
+  if (m->nvalid != nullptr && !aligned16(m->nvalid)) return fail(SVSA_ERR_INVALID_ARG, "mask.nvalid misaligned");
+  const int k = topk_count(p->keep_frac, g.nb);
+  const int need_cap = p->select == SVSA_SEL_TOPK ? k : g.nb;
+  if (m->cap < need_cap) return fail(SVSA_ERR_INVALID_ARG, "mask.cap=%d < %d", m->cap, need_cap);
+  const bool structured = p->select == SVSA_SEL_STRUCTURED;
+  if (!structured) {
+    SVSA_PTR(qp, "qp");
+    SVSA_PTR(kp, "kp");
+  }
+  if (structured) SVSA_PTR(perm, "perm");
+  if (p->routing) {
+    SVSA_PTR(vp, "vp");
+    SVSA_PTR(m->kbar, "mask.kbar (routing)");
+    SVSA_PTR(m->vbar, "mask.vbar (routing)");
+    SVSA_PTR(m->nvalid, "mask.nvalid (routing)");
+  }
+  if (m->vbar != nullptr) SVSA_PTR(vp, "vp (mask.vbar requested)");
+  if (m->kbar != nullptr) SVSA_PTR(kp, "kp (mask.kbar requested)");
+  const MaskWs w = mask_ws_layout(g, *p, m->kbar != nullptr);
+  if (w.total > 0) {
+    SVSA_PTR(ws, "ws");
+    if (ws_bytes < w.total) return fail(SVSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, w.total);
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  char* base = reinterpret_cast<char*>(ws);
+  auto at = [&](size_t off) { return off == SIZE_MAX ? nullptr : reinterpret_cast<float*>(base + off); };
+  const long long rows = g.BH * g.nb;
+  int32_t* nvalid = m->nvalid;
+
+  // block-level outputs the caller asked for (compensation / routing inputs)
+  if (nvalid != nullptr) SVSA_TRY(cuda_status(counted(launch_nvalid(nvalid, g.N, g.nb, st), 1), "nvalid"));
+  if (m->kbar != nullptr && (structured || p->sub_block != kBlock))
+    SVSA_TRY(cuda_status(counted(launch_pool(kp, m->kbar, nullptr, g.BH, g.N, g.Npad, g.d, kBlock, st), 1), "pool K"));
+  if (m->vbar != nullptr)
+    SVSA_TRY(cuda_status(counted(launch_pool(vp, m->vbar, nullptr, g.BH, g.N, g.Npad, g.d, kBlock, st), 1), "pool V"));
+
+  if (structured) {
+    const int R = p->win_rows * ((kBlock + g.W - 1) / g.W);
+    return cuda_status(counted(launch_structured(perm, rows, g.nb, g.H, g.W, p->win_t, R, p->n_anchors,
+                                                 p->anchor_offset, m->cap, m->kv_idx, m->kv_cnt, m->bits,
+                                                 st), 1),
+                       "structured mask");
+  }
+
+  const int sub = p->sub_block;
+  const int ng = (int)(g.Npad / sub);
+  float* qpool = at(w.qpool);
+  float* kpool = w.kpool == SIZE_MAX ? m->kbar : at(w.kpool);
+  float* S = at(w.S);
+  SVSA_TRY(cuda_status(counted(launch_pool(qp, qpool, nullptr, g.BH, g.N, g.Npad, g.d, sub, st), 1), "pool Q"));
+  SVSA_TRY(cuda_status(counted(launch_pool(kp, kpool, nullptr, g.BH, g.N, g.Npad, g.d, sub, st), 1), "pool K"));
+  SVSA_TRY(cuda_status(counted(launch_scores(qpool, kpool, S, g.BH, g.N, ng, g.nb, g.d, sub, st), 1), "scores"));
+  const float* Rr = nullptr;
+  int mode = p->select == SVSA_SEL_TOPK ? 1 : 0;
+  if (p->routing) {
+    const float* qbar = qpool;
+    if (sub != kBlock) {
+      SVSA_TRY(cuda_status(counted(launch_pool(qp, at(w.qbar64), nullptr, g.BH, g.N, g.Npad, g.d, kBlock,
+                                               st), 1),
+                           "pool Q (blocks)"));
+      qbar = at(w.qbar64);
+    }
+    SVSA_TRY(cuda_status(counted(launch_route(qbar, kp, vp, m->kbar, m->vbar, at(w.R), at(w.Rm), g.BH,
+                                              g.N, g.nb, g.d, st), 1), "route"));
+    Rr = at(w.R);
+    mode = 3;
+  }
+  return cuda_status(counted(launch_select(S, Rr, rows, g.nb, mode, p->tau, k, m->cap, m->kv_idx,
+                                           m->kv_cnt, m->bits, st), 1), "select");
+}
+
+svsa_status svsa_attn_fwd(const void* qp, const void* kp, const void* vp, const svsa_mask* m,
+                          int32_t compensate, void* op, float* lse, svsa_shape s, void* stream) {
+  g_last_error.clear();
+  SVSA_TRY(check_shape(s, true));
+  const Dims g = make_dims(s.B, s.heads, s.T, s.H, s.W, s.d);
+  SVSA_PTR(qp, "qp");
+  SVSA_PTR(kp, "kp");
+  SVSA_PTR(vp, "vp");
+  SVSA_PTR(op, "op");
+  if (m == nullptr) return fail(SVSA_ERR_INVALID_ARG, "mask is NULL");
+  SVSA_PTR(m->kv_idx, "mask.kv_idx");
+  SVSA_PTR(m->kv_cnt, "mask.kv_cnt");
+  if (m->cap < 1) return fail(SVSA_ERR_INVALID_ARG, "mask.cap=%d", m->cap);
+  if (lse != nullptr && !aligned16(lse)) return fail(SVSA_ERR_INVALID_ARG, "lse misaligned");
+  if (g.nb > kMaxBlocks) return fail(SVSA_ERR_UNSUPPORTED, "nb=%d exceeds %d", g.nb, kMaxBlocks);
+  if (compensate) {
+    SVSA_PTR(m->kbar, "mask.kbar (compensation)");
+    SVSA_PTR(m->vbar, "mask.vbar (compensation)");
+    SVSA_PTR(m->nvalid, "mask.nvalid (compensation)");
+  }
+  if (op == qp || op == kp || op == vp) return fail(SVSA_ERR_INVALID_ARG, "op must not alias an input");
+  return cuda_status(counted(launch_attn_mma(qp, kp, vp, m->kv_idx, m->kv_cnt, m->cap, m->kbar, m->vbar,
+                                             m->nvalid, op, lse, g.BH, g.N, g.nb, g.d, false,
+                                             compensate != 0, (cudaStream_t)stream), 1),
+                     "attn_fwd launch");
+}
+
+svsa_status svsa_attn_dense_fwd(const void* qp, const void* kp, const void* vp, void* op, float* lse,
+                                svsa_shape s, void* stream) {
+  g_last_error.clear();
+  SVSA_TRY(check_shape(s, true));
+  const Dims g = make_dims(s.B, s.heads, s.T, s.H, s.W, s.d);
+  SVSA_PTR(qp, "qp");
+  SVSA_PTR(kp, "kp");
+  SVSA_PTR(vp, "vp");
+  SVSA_PTR(op, "op");
+  if (lse != nullptr && !aligned16(lse)) return fail(SVSA_ERR_INVALID_ARG, "lse misaligned");
+  if (op == qp || op == kp || op == vp) return fail(SVSA_ERR_INVALID_ARG, "op must not alias an input");
+  return cuda_status(counted(launch_attn_mma(qp, kp, vp, nullptr, nullptr, 1, nullptr, nullptr, nullptr,
+                                             op, lse, g.BH, g.N, g.nb, g.d, true, false,
+                                             (cudaStream_t)stream), 1),
+                     "attn_dense_fwd launch");
+}
+
+svsa_status svsa_sync_status(void* stream) {
+  g_last_error.clear();
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_status(e, "stream synchronize");
+  e = cudaGetLastError();
+  return cuda_status(e, "asynchronous error");
+}
+
+}  // extern "C"

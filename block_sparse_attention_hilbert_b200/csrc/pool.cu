@@ -1,0 +1,99 @@
+// Block / sub-block means of a reordered tensor.
+//
+// "DFSAttn", trick 2 (the block "average" stands for the block) and "SVG-EAR"
+// 2.A (a cluster centroid is its mean).  out[bh, g, :] = mean of the valid
+// rows (position < N) of group g = rows [g*SIZE, g*SIZE + SIZE); 0 if none.
+//
+// One CTA reads one 64-row block (d*128 bytes) with 16-byte loads: 16 (d=128)
+// or 32 (d=64) row lanes x CPR chunk lanes; each thread keeps fp32 partial
+// sums of its rows per group, and the row lanes are added in a fixed order
+// through shared memory, so the result is deterministic.
+#include "common.cuh"
+
+namespace svsa {
+
+constexpr int kPoolThreads = 256;
+
+template <int D, int SIZE>
+__global__ void __launch_bounds__(kPoolThreads) pool_kernel(
+    const __nv_bfloat16* __restrict__ xp, float* __restrict__ out, int32_t* __restrict__ nvalid,
+    long long N, long long Npad) {
+  constexpr int CPR = D / 8;                 // 16-byte chunks per row
+  constexpr int RL = kPoolThreads / CPR;     // row lanes
+  constexpr int RPT = kBlock / RL;           // rows per thread
+  constexpr int G = kBlock / SIZE;           // groups per 64-row block
+  __shared__ float red[RL][G][D];
+
+  const int blk = blockIdx.x;
+  const long long bh = blockIdx.y;
+  const int ch = threadIdx.x % CPR, rl = threadIdx.x / CPR;
+  const long long row0 = (long long)blk * kBlock;
+  const __nv_bfloat16* base = xp + (bh * Npad + row0) * D;
+
+  float acc[G][8];
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
+
+#pragma unroll
+  for (int u = 0; u < RPT; ++u) {
+    const int r = rl + RL * u;
+    if (row0 + r < N) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(base + (long long)r * D) + ch);
+      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+      const int g = r / SIZE;
+#pragma unroll
+      for (int gg = 0; gg < G; ++gg) {
+        if (gg == g) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(p[e]);
+            acc[gg][2 * e] += f.x;
+            acc[gg][2 * e + 1] += f.y;
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[rl][g][ch * 8 + e] = acc[g][e];
+  __syncthreads();
+  for (int o = threadIdx.x; o < G * D; o += kPoolThreads) {
+    const int g = o / D, c = o % D;
+    float s = 0.f;
+#pragma unroll 8
+    for (int l = 0; l < RL; ++l) s += red[l][g][c];
+    const long long grow = row0 + (long long)g * SIZE;
+    const long long n = std::max<long long>(0, std::min<long long>(SIZE, N - grow));
+    const long long gidx = (long long)blk * G + g;
+    out[(bh * (Npad / SIZE) + gidx) * D + c] = n > 0 ? s / (float)n : 0.f;
+    if (nvalid != nullptr && bh == 0 && c == 0) nvalid[gidx] = (int32_t)n;
+  }
+}
+
+__global__ void nvalid_kernel(int32_t* __restrict__ nvalid, long long N, int nb) {
+  for (int J = blockIdx.x * blockDim.x + threadIdx.x; J < nb; J += gridDim.x * blockDim.x)
+    nvalid[J] = (int32_t)std::max<long long>(0, std::min<long long>(kBlock, N - (long long)J * kBlock));
+}
+
+cudaError_t launch_nvalid(int32_t* nvalid, long long N, int nb, cudaStream_t st) {
+  nvalid_kernel<<<(nb + 255) / 256, 256, 0, st>>>(nvalid, N, nb);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pool(const void* xp, float* out, int32_t* nvalid, long long BH, long long N,
+                        long long Npad, int d, int size, cudaStream_t st) {
+  dim3 grid((unsigned)(Npad / kBlock), (unsigned)BH);
+  const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(xp);
+  if (d == 128 && size == 64) pool_kernel<128, 64><<<grid, kPoolThreads, 0, st>>>(x, out, nvalid, N, Npad);
+  else if (d == 128 && size == 16) pool_kernel<128, 16><<<grid, kPoolThreads, 0, st>>>(x, out, nvalid, N, Npad);
+  else if (d == 64 && size == 64) pool_kernel<64, 64><<<grid, kPoolThreads, 0, st>>>(x, out, nvalid, N, Npad);
+  else if (d == 64 && size == 16) pool_kernel<64, 16><<<grid, kPoolThreads, 0, st>>>(x, out, nvalid, N, Npad);
+  else return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+}  // namespace svsa

@@ -1,0 +1,76 @@
+// Row gathers between raster order and the reordered, padded layout.
+//
+// Forward  ("DFSAttn", trick 1):  xp[bh, i, :] = x[bh, perm[i], :]   (zeros where perm[i] < 0)
+// Inverse:                        o[bh, r, :]  = op[bh, iperm[r], :]
+//
+// Both are pure data movement (HBM-bound): every thread moves 16-byte chunks,
+// consecutive threads cover consecutive bytes of the destination (coalesced
+// stores) and a source row (128 or 256 bytes) is read whole by 8 or 16
+// neighbouring threads.  Each thread issues kUnroll independent loads before
+// its stores to keep enough bytes in flight.
+#include "common.cuh"
+
+namespace svsa {
+
+constexpr int kGatherThreads = 256;
+constexpr int kUnroll = 4;
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+
+// grid.y = bh; grid.x covers rows_dst * chunks-per-row in tiles of
+// kGatherThreads * kUnroll chunks.
+template <int CPR>
+__global__ void __launch_bounds__(kGatherThreads) gather_rows_kernel(
+    const uint4* __restrict__ src, uint4* __restrict__ dst, const int32_t* __restrict__ map,
+    long long rows_dst, long long rows_src) {
+  const long long bh = blockIdx.y;
+  const long long total = rows_dst * CPR;
+  const uint4* s_base = src + bh * rows_src * CPR;
+  uint4* d_base = dst + bh * rows_dst * CPR;
+  const long long tile = (long long)kGatherThreads * kUnroll;
+  for (long long base = (long long)blockIdx.x * tile; base < total; base += (long long)gridDim.x * tile) {
+    uint4 v[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const long long c = base + u * kGatherThreads + threadIdx.x;
+      v[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (c < total) {
+        const int32_t srow = __ldg(map + c / CPR);
+        if (srow >= 0) v[u] = ld_stream(s_base + (long long)srow * CPR + (c % CPR));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const long long c = base + u * kGatherThreads + threadIdx.x;
+      if (c < total) d_base[c] = v[u];
+    }
+  }
+}
+
+cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* map, long long BH,
+                               long long rows_dst, long long rows_src, int d, cudaStream_t st) {
+  const int cpr = d * 2 / 16;
+  const long long total = rows_dst * cpr;
+  const long long tile = (long long)kGatherThreads * kUnroll;
+  long long gx = (total + tile - 1) / tile;
+  // enough CTAs to fill the GPU several times over, as a multiple of the SM count
+  const long long want = std::max<long long>(1, (kNumSMs * 8LL + BH - 1) / BH);
+  gx = std::max<long long>(1, std::min<long long>(gx, std::max<long long>(want, gx)));
+  dim3 grid((unsigned)gx, (unsigned)BH);
+  if (cpr == 16)
+    gather_rows_kernel<16><<<grid, kGatherThreads, 0, st>>>(
+        (const uint4*)src, (uint4*)dst, map, rows_dst, rows_src);
+  else if (cpr == 8)
+    gather_rows_kernel<8><<<grid, kGatherThreads, 0, st>>>(
+        (const uint4*)src, (uint4*)dst, map, rows_dst, rows_src);
+  else
+    return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+}  // namespace svsa

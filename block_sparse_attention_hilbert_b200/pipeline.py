@@ -1,0 +1,122 @@
+"""One attention layer through the four library calls, with its device buffers.
+
+    attn = SparseVideoAttention(B, heads, T, H, W, d, order="hilbert", select="topk", keep_frac=0.25)
+    o = attn(q, k, v)               # q, k, v: bf16 [B, heads, T*H*W, d] on the GPU, raster order
+
+A call runs svsa_reorder (x3), svsa_build_mask (unless the cached mask is
+reused across denoising steps -- "DFSAttn" trick 3), svsa_attn_fwd and
+svsa_inverse_reorder on the current stream.  The permutation is built once per
+object.  Buffers are allocated once with torch (the library allocates nothing).
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import (ORDER_HILBERT, ORDER_RASTER, SEL_STRUCTURED, SEL_THRESHOLD, SEL_TOPK, BLOCK,
+               make_mask, mask_params, shape, svsa_attn_dense_fwd, svsa_attn_fwd, svsa_build_mask,
+               svsa_build_perm, svsa_inverse_reorder, svsa_mask_workspace_bytes,
+               svsa_perm_workspace_bytes, svsa_reorder)
+
+_ORDERS = {"raster": ORDER_RASTER, "hilbert": ORDER_HILBERT}
+_SELECTS = {"threshold": SEL_THRESHOLD, "topk": SEL_TOPK, "structured": SEL_STRUCTURED}
+
+
+class LayerBuffers:
+    """Device buffers of one layer shape (all caller-owned, as the ABI requires)."""
+
+    def __init__(self, B, heads, T, H, W, d, *, cap, need_means, keep_bits, ws_bytes, perm_ws_bytes,
+                 device):
+        N = T * H * W
+        nb = -(-N // BLOCK)
+        Npad = nb * BLOCK
+        dev = torch.device(device)
+        bf = torch.bfloat16
+        self.perm = torch.empty(Npad, dtype=torch.int32, device=dev)
+        self.iperm = torch.empty(N, dtype=torch.int32, device=dev)
+        self.perm_ws = torch.empty(max(perm_ws_bytes, 16), dtype=torch.uint8, device=dev)
+        self.qp = torch.empty(B, heads, Npad, d, dtype=bf, device=dev)
+        self.kp = torch.empty_like(self.qp)
+        self.vp = torch.empty_like(self.qp)
+        self.op = torch.empty_like(self.qp)
+        self.kv_idx = torch.empty(B, heads, nb, cap, dtype=torch.int32, device=dev)
+        self.kv_cnt = torch.empty(B, heads, nb, dtype=torch.int32, device=dev)
+        self.bits = (torch.empty(B, heads, nb, -(-nb // 32), dtype=torch.int32, device=dev)
+                     if keep_bits else None)
+        self.kbar = torch.empty(B, heads, nb, d, dtype=torch.float32, device=dev) if need_means else None
+        self.vbar = torch.empty_like(self.kbar) if need_means else None
+        self.nvalid = torch.empty(nb, dtype=torch.int32, device=dev) if need_means else None
+        self.ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+        self.cap = cap
+
+    def mask(self):
+        return make_mask(self.kv_idx, self.kv_cnt, self.cap, self.bits, self.kbar, self.vbar, self.nvalid)
+
+
+class SparseVideoAttention:
+    def __init__(self, B, heads, T, H, W, d, *, order="hilbert", select="threshold", tau=0.9,
+                 keep_frac=0.25, sub_block=64, win_t=2, win_rows=1, n_anchors=0, routing=False,
+                 compensate=False, keep_bits=False, device="cuda"):
+        self.B, self.heads, self.T, self.H, self.W, self.d = B, heads, T, H, W, d
+        self.N = T * H * W
+        self.nb = -(-self.N // BLOCK)
+        self.Npad = self.nb * BLOCK
+        self.order = _ORDERS[order]
+        self.select = _SELECTS[select]
+        self.compensate = bool(compensate)
+        self.routing = bool(routing)
+        self.shape = shape(B, heads, T, H, W, d)
+        self.params = mask_params(self.select, tau, keep_frac, sub_block, win_t, win_rows, n_anchors, 0,
+                                  routing)
+        k = max(1, min(self.nb, math.ceil(float(torch.tensor(keep_frac, dtype=torch.float32)) * self.nb)))
+        cap = k if self.select == SEL_TOPK else self.nb
+        self.buf = LayerBuffers(B, heads, T, H, W, d, cap=cap, need_means=self.compensate or self.routing,
+                                keep_bits=keep_bits, ws_bytes=svsa_mask_workspace_bytes(self.shape, self.params),
+                                perm_ws_bytes=svsa_perm_workspace_bytes(self.shape, self.order),
+                                device=device)
+        self._mask = self.buf.mask()
+        self._perm_ready = False
+        self.mask_ready = False
+
+    # ---- the four steps -------------------------------------------------
+    def build_perm(self, stream=None):
+        b = self.buf
+        svsa_build_perm(self.shape, self.order, b.perm, b.iperm, b.perm_ws, b.perm_ws.numel(), stream)
+        self._perm_ready = True
+
+    def reorder(self, q, k, v, stream=None):
+        if not self._perm_ready:
+            self.build_perm(stream)
+        b = self.buf
+        for x, xp in ((q, b.qp), (k, b.kp), (v, b.vp)):
+            svsa_reorder(x, xp, b.perm, self.shape, stream)
+
+    def build_mask(self, anchor_offset: int = 0, stream=None):
+        b = self.buf
+        self.params.anchor_offset = int(anchor_offset)
+        svsa_build_mask(b.qp, b.kp, b.vp, b.perm, self.shape, self.params, self._mask, b.ws, b.ws.numel(),
+                        stream)
+        self.mask_ready = True
+
+    def attend(self, lse=None, stream=None):
+        b = self.buf
+        svsa_attn_fwd(b.qp, b.kp, b.vp, self._mask, self.compensate, b.op, lse, self.shape, stream)
+
+    def attend_dense(self, lse=None, stream=None):
+        b = self.buf
+        svsa_attn_dense_fwd(b.qp, b.kp, b.vp, b.op, lse, self.shape, stream)
+
+    def inverse(self, out, stream=None):
+        svsa_inverse_reorder(self.buf.op, out, self.buf.iperm, self.shape, stream)
+
+    # ---- whole layer ----------------------------------------------------
+    def __call__(self, q, k, v, *, out=None, anchor_offset: int = 0, reuse_mask: bool = False, stream=None):
+        if out is None:
+            out = torch.empty_like(q)
+        self.reorder(q, k, v, stream)
+        if not (reuse_mask and self.mask_ready):
+            self.build_mask(anchor_offset, stream)
+        self.attend(stream=stream)
+        self.inverse(out, stream)
+        return out

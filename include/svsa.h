@@ -1,0 +1,209 @@
+/*
+ * svsa.h -- C ABI of the B200 block-sparse video attention library (libsvsa.so).
+ *
+ * The library computes training-free block-sparse self-attention for video
+ * diffusion transformers in four steps, each an entry point below:
+ *
+ *   1. svsa_build_perm / svsa_reorder -- put the (T, H, W) latent tokens in
+ *      raster or 3D Hilbert order ("DFSAttn: Dynamic Fine-grained Sparse
+ *      Attention for Efficient Video Generation", trick 1: a Hilbert curve
+ *      threads the tokens so that sequence neighbours are space-time
+ *      neighbours and every block is coherent).
+ *   2. svsa_build_mask -- choose, for every 64-token query block, the key
+ *      blocks computed exactly (DFSAttn trick 2: block scores from block
+ *      averages, optionally from 16-token sub-blocks summed per block; SVOO
+ *      "Training-Free Sparse Attention for Fast Video Generation via Offline
+ *      Layer-Wise Sparsity Profiling and Online Bidirectional Co-Clustering",
+ *      technical summary 2.A: keep the blocks that cover a cumulative
+ *      attention mass; "LVSA: Training-Free Sparse Attention for Long Video
+ *      Diffusion", abstract: structured window pattern with rotating global
+ *      anchors; "SVG-EAR: Parameter-Free Linear Compensation for Sparse Video
+ *      Generation via Error-aware Routing", 2.B: error-aware routing).
+ *   3. svsa_attn_fwd -- exact softmax attention over the kept block pairs only
+ *      (SVG-EAR, problem statement: sparse attention computes a subset of the
+ *      attention blocks), optionally with centroid compensation of the skipped
+ *      blocks (SVG-EAR 2.A: skipped keys and values are replaced by their
+ *      block centroid).
+ *   4. svsa_inverse_reorder -- put the output back in raster order.
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are row-major and contiguous.  Q, K, V and O in raster order are
+ *     bf16 [B, heads, N, d] with N = T*H*W; the reordered ("p") tensors are
+ *     bf16 [B, heads, Npad, d] with Npad = 64 * nb, nb = ceil(N / 64).  Rows
+ *     N..Npad-1 of a reordered tensor are zero pads; they never count in a
+ *     mean, a softmax or an output.
+ *   - Every pointer is a device pointer owned by the caller, and must be
+ *     16-byte aligned.  The library allocates no memory and keeps no state.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and returns after enqueueing its kernels.
+ *   - Arguments are validated before anything is launched.  A failed
+ *     validation returns SVSA_ERR_INVALID_ARG (or SVSA_ERR_UNSUPPORTED /
+ *     SVSA_ERR_WORKSPACE) and launches nothing; a launch failure returns
+ *     SVSA_ERR_CUDA.  svsa_last_error() gives a message for the last failure
+ *     on the calling thread.  No entry point throws or aborts.
+ *   - Supported: d in {64, 128}; B*heads*Npad*d < 2^31; nb <= 16384;
+ *     Hilbert order needs max(T, H, W) <= 1024.
+ */
+#ifndef SVSA_H_
+#define SVSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SVSA_OK = 0,
+  SVSA_ERR_INVALID_ARG = 1,   /* bad pointer, size, alignment or parameter */
+  SVSA_ERR_UNSUPPORTED = 2,   /* valid request outside the supported range */
+  SVSA_ERR_WORKSPACE = 3,     /* workspace smaller than the *_workspace_bytes query */
+  SVSA_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed */
+  SVSA_ERR_TIMEOUT = 5        /* a bounded device-side wait gave up (svsa_sync_status) */
+} svsa_status;
+
+typedef enum { SVSA_ORDER_RASTER = 0, SVSA_ORDER_HILBERT = 1 } svsa_order;
+
+typedef enum {
+  SVSA_SEL_THRESHOLD = 0,     /* cumulative score mass >= tau */
+  SVSA_SEL_TOPK = 1,          /* k = ceil(keep_frac * nb) highest scores */
+  SVSA_SEL_STRUCTURED = 2     /* temporal/spatial window OR rotating anchors */
+} svsa_select;
+
+/* One attention layer: batch, heads, latent grid (frames T, rows H, columns W)
+ * and head dimension d.  N = T*H*W tokens. */
+typedef struct {
+  int32_t B, heads, T, H, W, d;
+} svsa_shape;
+
+/* Mask rule.  Fields a rule does not use are ignored. */
+typedef struct {
+  int32_t select;         /* svsa_select */
+  float tau;              /* THRESHOLD: mass to reach; >= 1 keeps every block */
+  float keep_frac;        /* TOPK: k = ceil(keep_frac * nb) clamped to [1, nb] */
+  int32_t sub_block;      /* THRESHOLD/TOPK: 64 = block means, 16 = sub-block
+                             scores summed per block (DFSAttn trick 2) */
+  int32_t win_t;          /* STRUCTURED: keep |t_I - t_J| <= win_t (frames) */
+  int32_t win_rows;       /* STRUCTURED: or |h_I - h_J| <= win_rows * ceil(64 / W) */
+  int32_t n_anchors;      /* STRUCTURED: anchor key-block columns kept for all rows */
+  int32_t anchor_offset;  /* STRUCTURED: this step's rotation, in [0, nb / n_anchors);
+                             anchors are (anchor_offset + m * floor(nb / n_anchors)) mod nb */
+  int32_t routing;        /* THRESHOLD only: 1 = keep, per row, as many blocks as the
+                             threshold rule would, chosen by largest estimated
+                             compensation error per token (SVG-EAR 2.B); needs vp,
+                             mask.kbar, mask.vbar and mask.nvalid */
+} svsa_mask_params;
+
+/* Block mask, written by svsa_build_mask and read by svsa_attn_fwd.  All
+ * buffers are caller-owned device memory. */
+typedef struct {
+  int32_t* kv_idx;        /* [B, heads, nb, cap] kept key blocks of each query
+                             block, ascending; entries past kv_cnt are unspecified */
+  int32_t* kv_cnt;        /* [B, heads, nb] number of kept key blocks */
+  int32_t cap;            /* row capacity: >= nb (>= k for TOPK) */
+  uint32_t* bits;         /* nullable [B, heads, nb, ceil(nb/32)]: bit J%32 of word
+                             J/32 set iff block J is kept */
+  float* kbar;            /* nullable [B, heads, nb, d] fp32 key block means */
+  float* vbar;            /* nullable [B, heads, nb, d] fp32 value block means */
+  int32_t* nvalid;        /* nullable [nb] valid (non-pad) tokens per block */
+} svsa_mask;
+
+/* ---- step 1: token order ------------------------------------------------ */
+
+/* Workspace bytes svsa_build_perm needs (0 for raster order). */
+size_t svsa_perm_workspace_bytes(svsa_shape s, int32_t order);
+
+/* Build the permutation of the latent grid.
+ *   perm  [Npad] int32 out: position i -> raster token id (t*H + h)*W + w, or
+ *         -1 for the pad positions N..Npad-1.
+ *   iperm [N]    int32 out: raster token id -> position.
+ * Raster order is the identity.  Hilbert order (DFSAttn trick 1) sorts the
+ * cells by their index on the Hilbert curve of the enclosing 2^k cube,
+ * k = ceil(log2(max(T, H, W))), computed with Skilling's transpose method
+ * (axes t, h, w); the sort is a rank by bitmap and prefix count, so the result
+ * is deterministic.  ws: svsa_perm_workspace_bytes(s, order) bytes of device
+ * scratch (may be NULL when that is 0).  B, heads and d are ignored. */
+svsa_status svsa_build_perm(svsa_shape s, int32_t order, int32_t* perm, int32_t* iperm,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* Gather one tensor into the reordered layout:
+ *   xp[b, h, i, :] = x[b, h, perm[i], :] for i < Npad (zeros where perm[i] = -1).
+ * x: bf16 [B, heads, N, d]; xp: bf16 [B, heads, Npad, d]; perm from
+ * svsa_build_perm.  Call once per tensor (Q, K, V). */
+svsa_status svsa_reorder(const void* x, void* xp, const int32_t* perm, svsa_shape s, void* stream);
+
+/* ---- step 2: block mask ------------------------------------------------- */
+
+/* Workspace bytes svsa_build_mask needs for this shape and rule. */
+size_t svsa_mask_workspace_bytes(svsa_shape s, const svsa_mask_params* p);
+
+/* Build the block mask from reordered Q and K (and V for routing).
+ * THRESHOLD / TOPK: pooled block scores P_IJ = softmax_J(qbar_I . kbar_J /
+ *   sqrt(d)) over all key blocks (means over valid tokens; with sub_block = 16
+ *   the per-sub-block softmax probabilities are summed over the 16 sub-pairs
+ *   of (I, J) and averaged over the non-empty query sub-blocks of I); each row
+ *   is ordered by (score desc, block index asc) and keeps the shortest prefix
+ *   whose fp64 cumulative sum reaches tau, or the first k.
+ * STRUCTURED: keep (I, J) iff |t_I - t_J| <= win_t or |h_I - h_J| <=
+ *   win_rows * ceil(64 / W) or J is an anchor column, where (t, h) is the
+ *   coordinate of the block's first token (perm required).
+ * routing = 1: with the threshold rule's count m_I as the budget, keep the
+ *   m_I blocks with the largest r_IJ = e_IJ / Z_I * 64 / n_J, where e_IJ is the
+ *   l2 norm of the change of the un-normalised output of the proxy query
+ *   qbar_I when block J's keys/values are replaced by their means (SVG-EAR 2.B).
+ * Outputs: m->kv_idx, m->kv_cnt, and m->bits / kbar / vbar / nvalid when those
+ * are non-NULL (kbar, vbar, nvalid required for routing).  perm may be NULL
+ * unless select = STRUCTURED.  vp may be NULL unless routing = 1. */
+svsa_status svsa_build_mask(const void* qp, const void* kp, const void* vp, const int32_t* perm,
+                            svsa_shape s, const svsa_mask_params* p, const svsa_mask* m,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* ---- step 3: attention -------------------------------------------------- */
+
+/* Block-sparse attention over the reordered tensors:
+ *   O_i = sum_{J kept for block(i)} sum_{j in J, j < N} softmax(q_i . k_j / sqrt(d)) v_j
+ * computed with an online softmax (fp32 statistics and accumulators, bf16
+ * tensor-core products, P rounded to bf16).  compensate = 1 adds, for every
+ * skipped block J, n_J copies of (kbar_J, vbar_J) to the same softmax
+ * (SVG-EAR 2.A); that needs m->kbar, m->vbar and m->nvalid.
+ * op: bf16 [B, heads, Npad, d] (pad rows are written as zeros).
+ * lse: nullable fp32 [B, heads, Npad]: natural-log sum-exp of each row's
+ * scaled scores (0 for pad rows). */
+svsa_status svsa_attn_fwd(const void* qp, const void* kp, const void* vp, const svsa_mask* m,
+                          int32_t compensate, void* op, float* lse, svsa_shape s, void* stream);
+
+/* Dense attention over all N keys, same arithmetic and layout as
+ * svsa_attn_fwd; the denominator of the speedup the benchmark reports. */
+svsa_status svsa_attn_dense_fwd(const void* qp, const void* kp, const void* vp, void* op,
+                                float* lse, svsa_shape s, void* stream);
+
+/* ---- step 4: back to raster order --------------------------------------- */
+
+/* o[b, h, r, :] = op[b, h, iperm[r], :] for r < N.
+ * op: bf16 [B, heads, Npad, d]; o: bf16 [B, heads, N, d]. */
+svsa_status svsa_inverse_reorder(const void* op, void* o, const int32_t* iperm, svsa_shape s,
+                                 void* stream);
+
+/* ---- status ------------------------------------------------------------- */
+
+/* Synchronise `stream` and report device-side failures recorded by the
+ * kernels since the last call (a bounded wait that gave up -> SVSA_ERR_TIMEOUT;
+ * an asynchronous CUDA error -> SVSA_ERR_CUDA).  Clears the recorded flags. */
+svsa_status svsa_sync_status(void* stream);
+
+/* Message for the last failure on the calling thread ("" if none). */
+const char* svsa_last_error(void);
+
+/* Library version string. */
+const char* svsa_version(void);
+
+/* Number of kernels this process has launched through the library (all
+ * threads, all devices); a diagnostic for benchmarks and tests. */
+unsigned long long svsa_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVSA_H_ */

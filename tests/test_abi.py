@@ -1,0 +1,130 @@
+"""C ABI checks that need no GPU: the library loads, exports every entry point
+that include/svsa.h declares, and rejects bad arguments before launching."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_attention_hilbert_b200 as svsa
+from block_sparse_attention_hilbert_b200 import Shape, MaskParams, Mask
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(svsa_\w+)\s*\(", text))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = svsa.lib()
+    declared = _declared()
+    assert {"svsa_reorder", "svsa_build_mask", "svsa_attn_fwd", "svsa_inverse_reorder"} <= declared
+    for name in declared:
+        assert hasattr(lib, name), name
+    # the binding wraps every declared entry point
+    assert declared <= set(svsa.exported_symbols())
+
+
+def test_struct_sizes_match_header():
+    assert ctypes.sizeof(Shape) == 24
+    assert ctypes.sizeof(MaskParams) == 36
+    assert ctypes.sizeof(Mask) == 56
+
+
+def test_version():
+    assert "sm_100a" in svsa.version()
+
+
+def test_workspace_queries():
+    s = svsa.shape(1, 12, 21, 30, 52, 128)
+    assert svsa.svsa_perm_workspace_bytes(s, svsa.ORDER_RASTER) == 0
+    # 64^3 cube -> 2^18 bits
+    assert svsa.svsa_perm_workspace_bytes(s, svsa.ORDER_HILBERT) >= 2 * (1 << 18) // 8
+    nb = 512
+    p = svsa.mask_params(svsa.SEL_TOPK)
+    assert svsa.svsa_mask_workspace_bytes(s, p) >= 12 * nb * nb * 4
+    assert svsa.svsa_mask_workspace_bytes(s, svsa.mask_params(svsa.SEL_STRUCTURED)) == 0
+    p16 = svsa.mask_params(svsa.SEL_THRESHOLD, sub_block=16)
+    assert svsa.svsa_mask_workspace_bytes(s, p16) > svsa.svsa_mask_workspace_bytes(s, p)
+    assert svsa.svsa_mask_workspace_bytes(s, svsa.mask_params(sub_block=32)) == 0
+
+
+def _raw():
+    return svsa.lib()
+
+
+def _err():
+    return _raw().svsa_last_error().decode()
+
+
+def test_build_perm_rejects_before_launch():
+    lib = _raw()
+    s = svsa.shape(1, 1, 4, 8, 8, 64)
+    assert lib.svsa_build_perm(s, 1, None, None, None, 0, None) == 1
+    assert "perm" in _err()
+    assert lib.svsa_build_perm(s, 7, 16, 32, None, 0, None) == 1
+    assert lib.svsa_build_perm(svsa.shape(1, 1, 0, 8, 8, 64), 0, 16, 32, None, 0, None) == 1
+    assert lib.svsa_build_perm(s, 0, 17, 32, None, 0, None) == 1          # misaligned
+    assert "aligned" in _err()
+    assert lib.svsa_build_perm(s, 1, 16, 32, 48, 8, None) == 3            # workspace too small
+    assert lib.svsa_build_perm(svsa.shape(1, 1, 2000, 2, 2, 64), 1, 16, 32, 48, 1 << 30, None) == 2
+
+
+def test_reorder_and_attention_reject_before_launch():
+    lib = _raw()
+    s = svsa.shape(1, 2, 4, 8, 8, 96)                                     # d = 96 unsupported
+    assert lib.svsa_reorder(16, 32, 48, s, None) == 2
+    s = svsa.shape(1, 2, 4, 8, 8, 128)
+    assert lib.svsa_reorder(16, 16, 48, s, None) == 1                     # aliasing
+    assert lib.svsa_inverse_reorder(None, 32, 48, s, None) == 1
+    m = Mask(None, None, 4, None, None, None, None)
+    assert lib.svsa_attn_fwd(16, 32, 48, ctypes.byref(m), 0, 64, None, s, None) == 1
+    m = Mask(16, 32, 4, None, None, None, None)
+    assert lib.svsa_attn_fwd(16, 32, 48, ctypes.byref(m), 1, 64, None, s, None) == 1   # comp w/o means
+    assert "kbar" in _err()
+    assert lib.svsa_attn_dense_fwd(16, 32, 48, 16, None, s, None) == 1    # output aliases input
+    assert lib.svsa_attn_fwd(16, 32, 48, None, 0, 64, None, s, None) == 1
+
+
+def test_build_mask_rejects_before_launch():
+    lib = _raw()
+    s = svsa.shape(1, 2, 4, 8, 8, 128)                                    # nb = 4
+    m = Mask(16, 32, 4, None, None, None, None)
+    ok = svsa.mask_params(svsa.SEL_THRESHOLD)
+    # capacity below nb for a threshold rule
+    small = Mask(16, 32, 3, None, None, None, None)
+    assert lib.svsa_build_mask(16, 32, None, None, s, ctypes.byref(ok), ctypes.byref(small), 64, 1 << 20, None) == 1
+    # routing without V / means
+    r = svsa.mask_params(svsa.SEL_THRESHOLD, routing=True)
+    assert lib.svsa_build_mask(16, 32, None, None, s, ctypes.byref(r), ctypes.byref(m), 64, 1 << 20, None) == 1
+    # routing with a non-threshold rule
+    r2 = svsa.mask_params(svsa.SEL_TOPK, routing=True)
+    assert lib.svsa_build_mask(16, 32, 48, None, s, ctypes.byref(r2), ctypes.byref(m), 64, 1 << 20, None) == 1
+    # structured without perm
+    st = svsa.mask_params(svsa.SEL_STRUCTURED, n_anchors=2, anchor_offset=0)
+    assert lib.svsa_build_mask(None, None, None, None, s, ctypes.byref(st), ctypes.byref(m), None, 0, None) == 1
+    # anchor offset outside [0, nb / n_anchors)
+    st2 = svsa.mask_params(svsa.SEL_STRUCTURED, n_anchors=2, anchor_offset=5)
+    assert lib.svsa_build_mask(None, None, None, 16, s, ctypes.byref(st2), ctypes.byref(m), None, 0, None) == 1
+    # workspace too small
+    assert lib.svsa_build_mask(16, 32, None, None, s, ctypes.byref(ok), ctypes.byref(m), 64, 16, None) == 3
+    # unknown selection rule / sub-block size
+    bad = svsa.mask_params(5)
+    assert lib.svsa_build_mask(16, 32, None, None, s, ctypes.byref(bad), ctypes.byref(m), 64, 1 << 20, None) == 1
+    bad = svsa.mask_params(svsa.SEL_THRESHOLD, sub_block=32)
+    assert lib.svsa_build_mask(16, 32, None, None, s, ctypes.byref(bad), ctypes.byref(m), 64, 1 << 20, None) == 2
+
+
+def test_status_codes_are_stable():
+    # values are part of the ABI
+    text = open(os.path.join(ROOT, "include", "svsa.h")).read()
+    for name, val in [("SVSA_OK", 0), ("SVSA_ERR_INVALID_ARG", 1), ("SVSA_ERR_UNSUPPORTED", 2),
+                      ("SVSA_ERR_WORKSPACE", 3), ("SVSA_ERR_CUDA", 4), ("SVSA_ERR_TIMEOUT", 5)]:
+        assert re.search(rf"{name}\s*=\s*{val}\b", text)

@@ -1,0 +1,226 @@
+"""GPU path vs the fp64 oracle on small shapes that still span several tiles and
+a ragged tail.  Every GPU step runs through the C ABI (libsvsa.so)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+import block_sparse_attention_hilbert_b200 as svsa
+from _parity import (check_attention, compare_mask_rows, gpu_keep, gpu_layer, oracle_rows, to_np)
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [(4, 8, 8), (3, 5, 7), (5, 7, 9), (1, 1, 1), (1, 3, 50), (2, 9, 13), (6, 12, 20)]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    svsa.lib()
+
+
+@pytest.mark.parametrize("order", ["raster", "hilbert"])
+@pytest.mark.parametrize("grid", SHAPES + [(21, 30, 52), (126, 30, 52), (62, 45, 80), (17, 64, 3)])
+def test_perm_bit_exact(order, grid):
+    T, H, W = grid
+    s = svsa.shape(1, 1, T, H, W, 64)
+    N = T * H * W
+    nb = -(-N // 64)
+    perm = torch.full((nb * 64,), 12345, dtype=torch.int32, device="cuda")
+    iperm = torch.full((N,), 12345, dtype=torch.int32, device="cuda")
+    o = svsa.ORDER_HILBERT if order == "hilbert" else svsa.ORDER_RASTER
+    ws = torch.empty(max(svsa.svsa_perm_workspace_bytes(s, o), 16), dtype=torch.uint8, device="cuda")
+    svsa.svsa_build_perm(s, o, perm, iperm, ws, ws.numel())
+    svsa.svsa_sync_status()
+    ep, ei = oracle.build_perm(T, H, W, order)
+    assert np.array_equal(perm.cpu().numpy(), ep)
+    assert np.array_equal(iperm.cpu().numpy(), ei)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("grid", [(3, 5, 7), (4, 8, 8), (2, 9, 13)])
+def test_reorder_inverse_bit_exact(d, grid):
+    T, H, W = grid
+    B, h = 2, 3
+    N = T * H * W
+    x = torch.randn(B, h, N, d, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16).cuda()
+    attn = svsa.SparseVideoAttention(B, h, T, H, W, d, order="hilbert", select="topk")
+    attn.build_perm()
+    b = attn.buf
+    b.qp.fill_(7.0)
+    svsa.svsa_reorder(x, b.qp, b.perm, attn.shape)
+    out = torch.zeros_like(x)
+    svsa.svsa_inverse_reorder(b.qp, out, b.iperm, attn.shape)
+    svsa.svsa_sync_status()
+    perm, _ = oracle.build_perm(T, H, W, "hilbert")
+    expect = oracle.reorder(x.cpu().view(torch.int16).numpy(), perm)
+    assert np.array_equal(b.qp.cpu().view(torch.int16).numpy(), expect)
+    assert torch.equal(out.view(torch.int16), x.view(torch.int16))
+
+
+def _small(select, sub=64, grid=(5, 7, 9), heads=2, d=128, **kw):
+    T, H, W = grid
+    return workloads.Workload("small", 1, heads, d, T, H, W, select=select, sub_block=sub, **kw)
+
+
+def _run_and_compare_masks(w, anchor_offset=0, seed=0):
+    q, k, v = (t.cuda() for t in workloads.make_qkv(w, seed=seed))
+    attn = gpu_layer(w, q, k, v, anchor_offset=anchor_offset)
+    keep = gpu_keep(attn)
+    perm, _ = oracle.build_perm(w.T, w.H, w.W, w.order)
+    qp, kp, vp = (oracle.reorder(to_np(t)[0].astype(np.float64), perm) for t in (q, k, v))
+    near_total = 0
+    rows = list(range(attn.nb))
+    for eta in range(w.heads):
+        kept, near = oracle_rows(w, qp[eta], kp[eta], vp[eta], perm, rows, anchor_offset)
+        n, _ = compare_mask_rows(keep[eta], kept, near)
+        near_total += n
+    return attn, keep, (q, k, v), (qp, kp, vp), perm, near_total
+
+
+@pytest.mark.parametrize("order", ["raster", "hilbert"])
+@pytest.mark.parametrize("select,sub", [("topk", 64), ("threshold", 64), ("threshold", 16), ("topk", 16)])
+@pytest.mark.parametrize("grid", [(5, 7, 9), (6, 12, 20)])
+def test_mask_and_attention_small(order, select, sub, grid):
+    w = _small(select, sub, grid=grid, order=order, tau=0.9, keep_frac=0.3)
+    attn, keep, _, (qp, kp, vp), _, near = _run_and_compare_masks(w)
+    op = to_np(attn.buf.op)[0]
+    for eta in range(w.heads):
+        ref = oracle.masked_attention(qp[eta], kp[eta], vp[eta], w.N, keep[eta])
+        gout = np.concatenate([op[eta][I * 64:min(I * 64 + 64, w.N)] for I in range(attn.nb)])
+        check_attention(gout, np.concatenate([ref[I] for I in range(attn.nb)]), f"head {eta}")
+        assert np.all(op[eta][w.N:] == 0)
+
+
+@pytest.mark.parametrize("tau", [0.5, 0.95, 1.0])
+def test_threshold_extremes(tau):
+    w = _small("threshold", 64, grid=(6, 12, 20), tau=tau)
+    _, keep, *_ = _run_and_compare_masks(w)
+    if tau >= 1.0:
+        assert keep.all()
+
+
+def test_structured_bit_exact():
+    w = workloads.Workload("s", 1, 2, 64, 12, 10, 20, order="raster", select="structured",
+                           win_t=2, win_rows=1, n_anchors=4)
+    for off in (0, 3, 7):
+        _, keep, *_ = _run_and_compare_masks(w, anchor_offset=off)
+        assert np.array_equal(keep[0], keep[1])          # structure is per layer, not per head
+    w0 = w.with_(win_t=0, win_rows=0, n_anchors=0, T=3, H=8, W=16)
+    _run_and_compare_masks(w0)
+
+
+def test_routing_and_compensation_small():
+    w = _small("threshold", 64, grid=(6, 12, 20), tau=0.9, routing=True, compensate=True)
+    attn, keep, _, (qp, kp, vp), _, near = _run_and_compare_masks(w)
+    b = attn.buf
+    op = to_np(b.op)[0]
+    kbar_g = to_np(b.kbar)[0]
+    vbar_g = to_np(b.vbar)[0]
+    assert np.array_equal(b.nvalid.cpu().numpy(), oracle.pool(kp[0], w.N)[1])
+    for eta in range(w.heads):
+        kb, n = oracle.pool(kp[eta], w.N)
+        vb, _ = oracle.pool(vp[eta], w.N)
+        assert np.allclose(kbar_g[eta], kb, rtol=1e-5, atol=1e-6)
+        assert np.allclose(vbar_g[eta], vb, rtol=1e-5, atol=1e-6)
+        ref = oracle.compensated_attention(qp[eta], kp[eta], vp[eta], w.N, keep[eta], kb, vb, n)
+        gout = np.concatenate([op[eta][I * 64:min(I * 64 + 64, w.N)] for I in range(attn.nb)])
+        check_attention(gout, np.concatenate([ref[I] for I in range(attn.nb)]), f"comp head {eta}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_dense_and_random_masks(d):
+    T, H, W = 5, 7, 9
+    w = _small("topk", 64, grid=(T, H, W), heads=2, d=d)
+    q, k, v = (t.cuda() for t in workloads.make_qkv(w, seed=4))
+    attn = svsa.SparseVideoAttention(1, 2, T, H, W, d, order="hilbert", select="threshold", tau=1.0)
+    attn.reorder(q, k, v)
+    b = attn.buf
+    perm, _ = oracle.build_perm(T, H, W, "hilbert")
+    qp, kp, vp = (oracle.reorder(to_np(t)[0].astype(np.float64), perm) for t in (q, k, v))
+    # dense
+    attn.attend_dense()
+    torch.cuda.synchronize()
+    op = to_np(b.op)[0]
+    for eta in range(2):
+        ref = oracle.dense_attention(qp[eta][:w.N], kp[eta][:w.N], vp[eta][:w.N])
+        check_attention(op[eta][:w.N], ref, "dense")
+    # random masks fed straight into the kv lists
+    nb = attn.nb
+    keep = np.stack([workloads.random_mask_lists(nb, nb, density=0.4, seed=s) for s in range(2)])
+    idx = np.zeros((1, 2, nb, nb), dtype=np.int32)
+    cnt = keep.sum(-1).astype(np.int32)[None]
+    for eta in range(2):
+        for I in range(nb):
+            lst = np.nonzero(keep[eta, I])[0]
+            idx[0, eta, I, :len(lst)] = lst
+    b.kv_idx.copy_(torch.from_numpy(idx))
+    b.kv_cnt.copy_(torch.from_numpy(cnt))
+    attn.attend()
+    torch.cuda.synchronize()
+    op = to_np(b.op)[0]
+    for eta in range(2):
+        ref = oracle.masked_attention(qp[eta], kp[eta], vp[eta], w.N, keep[eta])
+        gout = np.concatenate([op[eta][I * 64:min(I * 64 + 64, w.N)] for I in range(nb)])
+        check_attention(gout, np.concatenate([ref[I] for I in range(nb)]), "random mask")
+
+
+def test_single_token_and_single_block():
+    for grid in [(1, 1, 1), (1, 3, 5)]:
+        w = _small("threshold", 64, grid=grid, heads=1, tau=0.9)
+        q, k, v = (t.cuda() for t in workloads.make_qkv(w, seed=1))
+        attn = gpu_layer(w, q, k, v)
+        out = attn.out
+        if w.N == 1:
+            assert torch.allclose(out.float(), v.float(), atol=0, rtol=0)
+        perm, _ = oracle.build_perm(*grid, "hilbert")
+        ref = oracle.dense_attention(to_np(q)[0, 0], to_np(k)[0, 0], to_np(v)[0, 0])
+        check_attention(to_np(out)[0, 0], ref, "single block")
+
+
+def test_layer_end_to_end_raster_in_raster_out():
+    w = _small("topk", 64, grid=(6, 12, 20), heads=2, keep_frac=0.4, order="hilbert")
+    q, k, v = (t.cuda() for t in workloads.make_qkv(w, seed=5))
+    attn = gpu_layer(w, q, k, v)
+    keep = gpu_keep(attn)
+    perm, _ = oracle.build_perm(w.T, w.H, w.W, w.order)
+    qp, kp, vp = (oracle.reorder(to_np(t)[0].astype(np.float64), perm) for t in (q, k, v))
+    out = to_np(attn.out)[0]
+    for eta in range(2):
+        ref = oracle.masked_attention(qp[eta], kp[eta], vp[eta], w.N, keep[eta])
+        refp = np.zeros((attn.Npad, w.d))
+        for I in range(attn.nb):
+            refp[I * 64:min(I * 64 + 64, w.N)] = ref[I]
+        check_attention(out[eta], oracle.inverse_reorder(refp, perm, w.N), "raster out")
+
+
+def test_masks_are_deterministic():
+    w = _small("threshold", 16, grid=(6, 12, 20), tau=0.9)
+    q, k, v = (t.cuda() for t in workloads.make_qkv(w, seed=6))
+    a1 = gpu_layer(w, q, k, v)
+    a2 = gpu_layer(w, q, k, v)
+    assert torch.equal(a1.buf.kv_cnt, a2.buf.kv_cnt)
+    assert np.array_equal(gpu_keep(a1), gpu_keep(a2))
+    assert torch.equal(a1.out.view(torch.int16), a2.out.view(torch.int16))
+
+
+def test_lse_output():
+    w = _small("topk", 64, grid=(5, 7, 9), heads=1, keep_frac=0.5)
+    q, k, v = (t.cuda() for t in workloads.make_qkv(w, seed=7))
+    attn = gpu_layer(w, q, k, v)
+    keep = gpu_keep(attn)
+    lse = torch.full((1, 1, attn.Npad), 99.0, device="cuda")
+    attn.attend(lse=lse)
+    torch.cuda.synchronize()
+    perm, _ = oracle.build_perm(w.T, w.H, w.W, w.order)
+    qp, kp = (oracle.reorder(to_np(t)[0, 0].astype(np.float64), perm) for t in (q, k))
+    g = lse.cpu().numpy()[0, 0]
+    for I in range(attn.nb):
+        lo, hi = I * 64, min(I * 64 + 64, w.N)
+        pos = np.concatenate([np.arange(J * 64, min(J * 64 + 64, w.N)) for J in np.nonzero(keep[0, I])[0]])
+        s = qp[lo:hi] @ kp[pos].T / np.sqrt(w.d)
+        ref = np.log(np.exp(s - s.max(1, keepdims=True)).sum(1)) + s.max(1)
+        assert np.abs(g[lo:hi] - ref).max() < 1e-3
+    assert np.all(g[w.N:] == 0)

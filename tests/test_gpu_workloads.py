@@ -1,0 +1,140 @@
+"""GPU path vs the fp64 oracle at the full layer sizes of the five workloads.
+
+Permutations are compared whole; masks and outputs on seeded samples of query
+blocks (always including the first and the ragged last block) of two heads,
+which the oracle computes one block at a time.  Inputs are generated on the
+GPU by `workloads` and copied to the host, so both sides read the same bf16
+bits.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+import block_sparse_attention_hilbert_b200 as svsa
+from _parity import check_attention, compare_mask_rows, gpu_layer, oracle_rows, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    svsa.lib()
+
+
+def _sample_rows(nb, n, seed):
+    rng = np.random.default_rng(seed)
+    rows = set(rng.choice(nb, size=min(n, nb), replace=False).tolist()) | {0, nb - 1}
+    return sorted(rows)
+
+
+def _head_np(t, eta):
+    return t[0, eta].float().cpu().numpy().astype(np.float64)
+
+
+def _gpu_rows(attn, eta, rows):
+    b = attn.buf
+    idx = b.kv_idx[0, eta].cpu().numpy()
+    cnt = b.kv_cnt[0, eta].cpu().numpy()
+    keep = np.zeros((attn.nb, attn.nb), dtype=bool)
+    for I in range(attn.nb):
+        lst = idx[I, :cnt[I]]
+        assert np.all(np.diff(lst) > 0) and lst.min() >= 0 and lst.max() < attn.nb
+        keep[I, lst] = True
+    return keep
+
+
+def _check_layer(w, q, k, v, *, anchor_offset=0, n_rows=12, heads=None, seed=0):
+    attn = gpu_layer(w, q, k, v, anchor_offset=anchor_offset, keep_bits=False)
+    perm, iperm = oracle.build_perm(w.T, w.H, w.W, w.order)
+    assert np.array_equal(attn.buf.perm.cpu().numpy(), perm)
+    assert np.array_equal(attn.buf.iperm.cpu().numpy(), iperm)
+    heads = heads or [0, w.heads - 1]
+    rows = _sample_rows(attn.nb, n_rows, seed)
+    report = {"near": 0, "rows": 0, "max_abs": 0.0, "mean_abs": 0.0}
+    for eta in heads:
+        qp, kp, vp = (_head_np(t, eta) for t in (attn.buf.qp, attn.buf.kp, attn.buf.vp))
+        # reorder is a bit-exact gather of the raster rows
+        assert np.array_equal(qp, oracle.reorder(_head_np(q, eta), perm))
+        keep = _gpu_rows(attn, eta, rows)
+        kept, near = oracle_rows(w, qp, kp, vp, perm, rows, anchor_offset)
+        n, _ = compare_mask_rows(keep[rows], kept, near)
+        report["near"] += n
+        report["rows"] += len(rows)
+        op = _head_np(attn.buf.op, eta)
+        if w.compensate:
+            kb, nv = oracle.pool(kp, w.N)
+            vb, _ = oracle.pool(vp, w.N)
+            ref = oracle.compensated_attention(qp, kp, vp, w.N, keep, kb, vb, nv, q_blocks=rows)
+        else:
+            ref = oracle.masked_attention(qp, kp, vp, w.N, keep, q_blocks=rows)
+        for I in rows:
+            mx, mn = check_attention(op[I * 64:min(I * 64 + 64, w.N)], ref[I], f"head {eta} block {I}")
+            report["max_abs"] = max(report["max_abs"], mx)
+        # the raster-order output is the inverse gather of op
+        out = _head_np(attn.out, eta)
+        assert np.array_equal(out, op[iperm])
+    print(f"{w.name}: near-threshold blocks {report['near']} over {report['rows']} sampled rows; "
+          f"max-abs {report['max_abs']:.3e}")
+    return attn
+
+
+@pytest.mark.parametrize("order", ["raster", "hilbert"])
+def test_wan13b_topk(order):
+    w = workloads.WORKLOADS["wan13b"].with_(order=order)
+    q, k, v = workloads.make_qkv(w, device="cuda")
+    attn = _check_layer(w, q, k, v)
+    k_keep = oracle.topk_count(w.keep_frac, attn.nb)
+    assert torch.all(attn.buf.kv_cnt == k_keep)
+
+
+def test_tiny_threshold():
+    w = workloads.WORKLOADS["tiny"]
+    q, k, v = workloads.make_qkv(w, device="cuda")
+    _check_layer(w, q, k, v, n_rows=4, heads=[0])
+
+
+def test_wan13b_6x_structured():
+    w = workloads.WORKLOADS["wan13b_6x"]
+    q, k, v = workloads.make_qkv(w, device="cuda")
+    nb = w.nb
+    for step in (0, 1):
+        off = workloads.anchor_offset(seed=0, step=step, nkb=nb, n_anchors=w.n_anchors)
+        attn = _check_layer(w, q, k, v, anchor_offset=off, n_rows=8, seed=step)
+        # the whole structured mask is bit-exact, every head
+        perm, _ = oracle.build_perm(w.T, w.H, w.W, w.order)
+        full = oracle.structured_mask(perm, w.T, w.H, w.W, win_t=w.win_t, win_rows=w.win_rows,
+                                      n_anchors=w.n_anchors, anchor_offset=off)
+        cnt = attn.buf.kv_cnt.cpu().numpy()
+        assert np.array_equal(cnt[0, 0], full.sum(1))
+        assert np.all(cnt == cnt[:, :1])
+        del attn
+
+
+def test_wan14b_routing_compensation():
+    w = workloads.WORKLOADS["wan14b"]
+    q, k, v = workloads.make_qkv(w, device="cuda")
+    _check_layer(w, q, k, v, n_rows=8)
+
+
+def test_hunyuan_2x_subblock_mask_reuse():
+    w = workloads.WORKLOADS["hunyuan_2x"]
+    q0, k0, v = workloads.make_qkv(w, device="cuda")
+    attn = _check_layer(w, q0, k0, v, n_rows=6, heads=[0])
+    keep0 = _gpu_rows(attn, 0, None)
+    perm, _ = oracle.build_perm(w.T, w.H, w.W, w.order)
+    rows = _sample_rows(attn.nb, 4, 11)
+    for step in range(1, w.reuse_steps):
+        qs, ks = workloads.qk_at_step(q0, k0, sigma=w.sigma, seed=0, step=step)
+        out = attn(qs, ks, v, reuse_mask=True)
+        torch.cuda.synchronize()
+        assert np.array_equal(_gpu_rows(attn, 0, None), keep0)       # mask not rebuilt
+        qp, kp, vp = (oracle.reorder(_head_np(t, 0), perm) for t in (qs, ks, v))
+        ref = oracle.masked_attention(qp, kp, vp, w.N, keep0, q_blocks=rows)
+        op = _head_np(attn.buf.op, 0)
+        for I in rows:
+            check_attention(op[I * 64:min(I * 64 + 64, w.N)], ref[I], f"step {step} block {I}")
+        del out
