@@ -56,6 +56,8 @@ _SIGS = {
                                        ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "svsa_reorder": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, Shape,
                                     ctypes.c_void_p]),
+    "svsa_reorder_values": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, Shape,
+                                           ctypes.c_void_p]),
     "svsa_mask_workspace_bytes": (ctypes.c_size_t, [Shape, ctypes.POINTER(MaskParams)]),
     "svsa_build_mask": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                        ctypes.c_void_p, Shape, ctypes.POINTER(MaskParams),
@@ -143,6 +145,10 @@ def svsa_build_perm(s: Shape, order: int, perm, iperm, ws=None, ws_bytes: int = 
 
 def svsa_reorder(x, xp, perm, s: Shape, stream=None) -> None:
     _check(lib().svsa_reorder(_p(x), _p(xp), _p(perm), s, _stream(stream)), "svsa_reorder")
+
+
+def svsa_reorder_values(v, vp, perm, s: Shape, stream=None) -> None:
+    _check(lib().svsa_reorder_values(_p(v), _p(vp), _p(perm), s, _stream(stream)), "svsa_reorder_values")
 
 
 def svsa_mask_workspace_bytes(s: Shape, p: MaskParams) -> int:

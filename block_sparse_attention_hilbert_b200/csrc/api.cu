@@ -18,8 +18,12 @@ size_t perm_workspace_bytes(int T, int H, int W);
 int hilbert_order_bits(int T, int H, int W);
 cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* map, long long BH,
                                long long rows_dst, long long rows_src, int d, cudaStream_t st);
+cudaError_t launch_gather_rows_f16(const void* src, void* dst, const int32_t* map, long long BH,
+                                   long long rows_dst, long long rows_src, int d, cudaStream_t st);
 cudaError_t launch_pool(const void* xp, float* out, int32_t* nvalid, long long BH, long long N,
                         long long Npad, int d, int size, cudaStream_t st);
+cudaError_t launch_pool_f16(const void* xp, float* out, int32_t* nvalid, long long BH, long long N,
+                            long long Npad, int d, int size, cudaStream_t st);
 cudaError_t launch_nvalid(int32_t* nvalid, long long N, int nb, cudaStream_t st);
 cudaError_t launch_scores(const float* qs, const float* ks, float* S, long long BH, long long N,
                           int ng, int nb, int d, int size, cudaStream_t st);
@@ -36,6 +40,10 @@ cudaError_t launch_attn_mma(const void* q, const void* k, const void* v, const i
                             const int32_t* kv_cnt, int cap, const float* kbar, const float* vbar,
                             const int32_t* nvalid, void* o, float* lse, long long BH, long long N,
                             int nb, int d, bool dense, bool comp, cudaStream_t st);
+cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, const int32_t* kv_idx,
+                           const int32_t* kv_cnt, int cap, void* o, float* lse, long long BH, long long N, int nb,
+                           int d, bool dense, cudaStream_t st);
+cudaError_t attn_tc_error(unsigned int* code, cudaStream_t st);
 }  // namespace svsa
 
 using namespace svsa;
@@ -210,6 +218,18 @@ svsa_status svsa_reorder(const void* x, void* xp, const int32_t* perm, svsa_shap
                      "reorder launch");
 }
 
+svsa_status svsa_reorder_values(const void* v, void* vp, const int32_t* perm, svsa_shape s, void* stream) {
+  g_last_error.clear();
+  SVSA_TRY(check_shape(s, true));
+  SVSA_PTR(v, "v");
+  SVSA_PTR(vp, "vp");
+  SVSA_PTR(perm, "perm");
+  if (v == vp) return fail(SVSA_ERR_INVALID_ARG, "v and vp must not alias");
+  const Dims g = make_dims(s.B, s.heads, s.T, s.H, s.W, s.d);
+  return cuda_status(counted(launch_gather_rows_f16(v, vp, perm, g.BH, g.Npad, g.N, g.d, (cudaStream_t)stream), 1),
+                     "reorder_values launch");
+}
+
 svsa_status svsa_inverse_reorder(const void* op, void* o, const int32_t* iperm, svsa_shape s, void* stream) {
   g_last_error.clear();
   SVSA_TRY(check_shape(s, true));
@@ -277,7 +297,8 @@ svsa_status svsa_build_mask(const void* qp, const void* kp, const void* vp, cons
   if (m->kbar != nullptr && (structured || p->sub_block != kBlock))
     SVSA_TRY(cuda_status(counted(launch_pool(kp, m->kbar, nullptr, g.BH, g.N, g.Npad, g.d, kBlock, st), 1), "pool K"));
   if (m->vbar != nullptr)
-    SVSA_TRY(cuda_status(counted(launch_pool(vp, m->vbar, nullptr, g.BH, g.N, g.Npad, g.d, kBlock, st), 1), "pool V"));
+    SVSA_TRY(cuda_status(counted(launch_pool_f16(vp, m->vbar, nullptr, g.BH, g.N, g.Npad, g.d, kBlock, st), 1),
+                         "pool V"));
 
   if (structured) {
     const int R = p->win_rows * ((kBlock + g.W - 1) / g.W);
@@ -335,9 +356,13 @@ svsa_status svsa_attn_fwd(const void* qp, const void* kp, const void* vp, const 
     SVSA_PTR(m->nvalid, "mask.nvalid (compensation)");
   }
   if (op == qp || op == kp || op == vp) return fail(SVSA_ERR_INVALID_ARG, "op must not alias an input");
-  return cuda_status(counted(launch_attn_mma(qp, kp, vp, m->kv_idx, m->kv_cnt, m->cap, m->kbar, m->vbar,
-                                             m->nvalid, op, lse, g.BH, g.N, g.nb, g.d, false,
-                                             compensate != 0, (cudaStream_t)stream), 1),
+  if (compensate)
+    return cuda_status(counted(launch_attn_mma(qp, kp, vp, m->kv_idx, m->kv_cnt, m->cap, m->kbar, m->vbar,
+                                               m->nvalid, op, lse, g.BH, g.N, g.nb, g.d, false, true,
+                                               (cudaStream_t)stream), 1),
+                       "attn_fwd (compensated) launch");
+  return cuda_status(counted(launch_attn_tc(qp, kp, vp, m->kv_idx, m->kv_cnt, m->cap, op, lse, g.BH, g.N,
+                                            g.nb, g.d, false, (cudaStream_t)stream), 1),
                      "attn_fwd launch");
 }
 
@@ -352,9 +377,8 @@ svsa_status svsa_attn_dense_fwd(const void* qp, const void* kp, const void* vp, 
   SVSA_PTR(op, "op");
   if (lse != nullptr && !aligned16(lse)) return fail(SVSA_ERR_INVALID_ARG, "lse misaligned");
   if (op == qp || op == kp || op == vp) return fail(SVSA_ERR_INVALID_ARG, "op must not alias an input");
-  return cuda_status(counted(launch_attn_mma(qp, kp, vp, nullptr, nullptr, 1, nullptr, nullptr, nullptr,
-                                             op, lse, g.BH, g.N, g.nb, g.d, true, false,
-                                             (cudaStream_t)stream), 1),
+  return cuda_status(counted(launch_attn_tc(qp, kp, vp, nullptr, nullptr, 1, op, lse, g.BH, g.N, g.nb, g.d,
+                                            true, (cudaStream_t)stream), 1),
                      "attn_dense_fwd launch");
 }
 
@@ -363,7 +387,13 @@ svsa_status svsa_sync_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_status(e, "stream synchronize");
   e = cudaGetLastError();
-  return cuda_status(e, "asynchronous error");
+  if (e != cudaSuccess) return cuda_status(e, "asynchronous error");
+  unsigned int code = 0u;
+  e = attn_tc_error(&code, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_status(e, "reading the device error word");
+  if (code != 0u)
+    return fail(SVSA_ERR_TIMEOUT, "attention kernel: a bounded wait gave up (site %u)", code);
+  return SVSA_OK;
 }
 
 }  // extern "C"

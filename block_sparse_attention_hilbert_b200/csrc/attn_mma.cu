@@ -4,14 +4,20 @@
 // the attention blocks; 2.A: with compensation every skipped block J enters
 // the same softmax as n_J copies of its centroid (kbar_J, vbar_J).
 //
+// Q and K are bf16, the reordered values fp16 (P is rounded to fp16 for the
+// P.V product, whose 11-bit significand keeps the softmax weights 8x more
+// precise than bf16 would).
+//
 // One CTA = one 64-row query block (the mask's granularity, so no tile is
 // wasted), 4 warps x 16 query rows.  The kept key blocks are streamed through
 // a double-buffered, XOR-swizzled shared-memory ring with cp.async; S = Q K^T
 // and O += P V run on mma.sync with fp32 accumulators; the online softmax
-// keeps a running max / sum per row in the log2 domain; P is rounded to bf16
+// keeps a running max / sum per row in the log2 domain; P is rounded to fp16
 // in registers and fed straight back as the A operand.  Compensation appends
 // ceil(nb / 64) centroid tiles whose columns carry the bias log2(n_J) for
 // skipped blocks and -inf for kept ones.  DENSE visits every key block.
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 
 namespace svsa {
@@ -44,6 +50,17 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+__device__ __forceinline__ void mma16816_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
+  __half2 v = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
 __device__ __forceinline__ float fast_ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
@@ -61,7 +78,7 @@ __device__ __forceinline__ int clamp_block(int J, int nb) { return J < 0 ? 0 : (
 struct AttnArgs {
   const __nv_bfloat16* q;
   const __nv_bfloat16* k;
-  const __nv_bfloat16* v;
+  const __half* v;
   const int32_t* kv_idx;
   const int32_t* kv_cnt;
   int cap;
@@ -86,8 +103,8 @@ __device__ __forceinline__ void load_tile_async(__nv_bfloat16* dst, const __nv_b
   }
 }
 
-// Centroid rows J0 .. J0+63 (fp32) -> bf16 tile; rows past nb are zero.
-template <int D>
+// Centroid rows J0 .. J0+63 (fp32) -> bf16 (keys) or fp16 (values) tile; rows past nb are zero.
+template <int D, bool F16>
 __device__ __forceinline__ void load_centroid_tile(__nv_bfloat16* dst, const float* src, int J0, int nb, int tid) {
   constexpr int CPR = D / 8;
 #pragma unroll
@@ -98,8 +115,13 @@ __device__ __forceinline__ void load_centroid_tile(__nv_bfloat16* dst, const flo
     if (J0 + r < nb) {
       const float4 a = *reinterpret_cast<const float4*>(src + (long long)(J0 + r) * D + c * 8);
       const float4 b = *reinterpret_cast<const float4*>(src + (long long)(J0 + r) * D + c * 8 + 4);
-      packed.x = pack_bf16x2(a.x, a.y); packed.y = pack_bf16x2(a.z, a.w);
-      packed.z = pack_bf16x2(b.x, b.y); packed.w = pack_bf16x2(b.z, b.w);
+      if (F16) {
+        packed.x = pack_f16x2(a.x, a.y); packed.y = pack_f16x2(a.z, a.w);
+        packed.z = pack_f16x2(b.x, b.y); packed.w = pack_f16x2(b.z, b.w);
+      } else {
+        packed.x = pack_bf16x2(a.x, a.y); packed.y = pack_bf16x2(a.z, a.w);
+        packed.z = pack_bf16x2(b.x, b.y); packed.w = pack_bf16x2(b.z, b.w);
+      }
     }
     *reinterpret_cast<uint4*>(dst + swz<D>(r, c)) = packed;
   }
@@ -124,7 +146,7 @@ __global__ void __launch_bounds__(kMmaThreads, 2) attn_mma_kernel(const AttnArgs
   const long long rowbase = bh * a.Npad;
   const __nv_bfloat16* qg = a.q + (rowbase + (long long)I * kBlock) * D;
   const __nv_bfloat16* kg = a.k + rowbase * D;
-  const __nv_bfloat16* vg = a.v + rowbase * D;
+  const __nv_bfloat16* vg = reinterpret_cast<const __nv_bfloat16*>(a.v) + rowbase * D;   // fp16 bits
   const int32_t* list = DENSE ? nullptr : a.kv_idx + (bh * nb + I) * (long long)a.cap;
   // a caller-supplied list is trusted for order, not for range: the count is
   // clamped to the row capacity and entries outside [0, nb) are masked out
@@ -150,8 +172,8 @@ __global__ void __launch_bounds__(kMmaThreads, 2) attn_mma_kernel(const AttnArgs
       load_tile_async<D>(Vs + buf * TILE, vg + (long long)J * kBlock * D, tid);
     } else if (COMP) {
       const int J0 = (t - cnt) * kBlock;
-      load_centroid_tile<D>(Ks + buf * TILE, kbar_h, J0, nb, tid);
-      load_centroid_tile<D>(Vs + buf * TILE, vbar_h, J0, nb, tid);
+      load_centroid_tile<D, false>(Ks + buf * TILE, kbar_h, J0, nb, tid);
+      load_centroid_tile<D, true>(Vs + buf * TILE, vbar_h, J0, nb, tid);
     }
   };
 
@@ -252,8 +274,8 @@ __global__ void __launch_bounds__(kMmaThreads, 2) attn_mma_kernel(const AttnArgs
       const float p2 = fast_ex2(s[n][2] - mu1), p3 = fast_ex2(s[n][3] - mu1);
       rs0 += p0 + p1;
       rs1 += p2 + p3;
-      pa[n >> 1][(n & 1) * 2 + 0] = pack_bf16x2(p0, p1);
-      pa[n >> 1][(n & 1) * 2 + 1] = pack_bf16x2(p2, p3);
+      pa[n >> 1][(n & 1) * 2 + 0] = pack_f16x2(p0, p1);
+      pa[n >> 1][(n & 1) * 2 + 1] = pack_f16x2(p2, p3);
     }
     l0 = l0 * c0 + rs0;
     l1 = l1 * c1 + rs1;
@@ -270,8 +292,8 @@ __global__ void __launch_bounds__(kMmaThreads, 2) attn_mma_kernel(const AttnArgs
         const int r = 16 * kk + (lane & 7) + (((lane >> 3) & 1) << 3);
         const int c = 2 * dp + (lane >> 4);
         ldsm_x4_t(smem_u32(Vt + swz<D>(r, c)), b0, b1, b2, b3);
-        mma16816(o[2 * dp], pa[kk], b0, b1);
-        mma16816(o[2 * dp + 1], pa[kk], b2, b3);
+        mma16816_f16(o[2 * dp], pa[kk], b0, b1);
+        mma16816_f16(o[2 * dp + 1], pa[kk], b2, b3);
       }
     }
     __syncthreads();
@@ -331,7 +353,7 @@ cudaError_t launch_attn_mma(const void* q, const void* k, const void* v, const i
                             const int32_t* nvalid, void* o, float* lse, long long BH, long long N,
                             int nb, int d, bool dense, bool comp, cudaStream_t st) {
   AttnArgs a;
-  a.q = (const __nv_bfloat16*)q; a.k = (const __nv_bfloat16*)k; a.v = (const __nv_bfloat16*)v;
+  a.q = (const __nv_bfloat16*)q; a.k = (const __nv_bfloat16*)k; a.v = (const __half*)v;
   a.kv_idx = kv_idx; a.kv_cnt = kv_cnt; a.cap = cap;
   a.kbar = kbar; a.vbar = vbar; a.nvalid = nvalid;
   a.o = (__nv_bfloat16*)o; a.lse = lse;

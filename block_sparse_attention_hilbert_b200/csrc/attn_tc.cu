@@ -1,0 +1,698 @@
+// Block-sparse attention on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// "SVG-EAR", problem statement: only the kept (query block, key block) pairs
+// are computed; "SPADE" part 3: a per-head sparse engine built for the
+// hardware.  Exact online-softmax attention over each 64-row query block's
+// kept key blocks.
+//
+// Design (sm_100a):
+//   * Work item = one 64-query block of one head; a persistent grid walks the
+//     items.  Tiles are PAIRS of kept key blocks (128 keys), taken in list
+//     order, so every MMA row does useful work whatever the mask looks like.
+//   * Transposed products keep M = 128 on the tensor core although the mask
+//     granularity is 64 queries:
+//        S^T [128 keys x 64 queries] = K_pair [128 x d] . Q^T      (A, B: K-major)
+//        O^T [d x 64 queries]       += V_pair^T [d x 128] . P^T    (A, B: MN-major)
+//     Both accumulate in TMEM (S^T double-buffered, O^T resident).
+//   * Warp roles: warp 0 issues TMA copies (Q once per item; K and V of each
+//     pair into 2-stage rings, 64-row boxes with 128-byte swizzle), warp 1
+//     issues the MMAs from one thread and owns the TMEM allocation, warps 2-5
+//     (one thread per key / per head-dim lane) run the softmax and the
+//     epilogue.  All hand-offs are mbarriers; every wait is bounded in time
+//     and a timeout sets an error word read by svsa_sync_status.
+//   * Softmax: thread k holds key k's 64 scores.  A column (query) maximum
+//     needs all 128 threads, so the running maximum is lazy: a tile only
+//     updates it (warp transpose-reduction + shared memory, then an in-TMEM
+//     rescale of O^T and of the partial sums) when some score exceeds the
+//     current maximum by more than 2^8; otherwise exp2(x - m) is taken against
+//     the stale maximum, which is exact up to the final normalisation.  The
+//     row sums stay per-thread partial sums until the epilogue.
+//   * P^T is rounded to fp16 and written to shared memory in the MN-major
+//     128-byte-swizzled layout the second MMA reads; the values arrive as
+//     fp16 (the reordered V), so the second product is fp16 x fp16.  With the
+//     lazy maximum the weights reach 2^8 and the dominant one is no longer
+//     exactly 1, so fp16's 11-bit significand (vs bf16's 8) is what keeps
+//     their rounding well inside the output tolerance.
+#include <cuda.h>
+
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+
+namespace svsa {
+namespace tc {
+
+constexpr int kThreads = 192;
+constexpr int kSoftmaxThreads = 128;
+constexpr uint32_t kBox = 8192;                  // one 64-row x 128-byte TMA box
+constexpr float kLazyTh = 8.0f;                  // log2 headroom before a rescale
+constexpr unsigned long long kWaitNs = 2000000000ull;   // 2 s per wait
+
+// shared memory map (offsets from a 1024-byte aligned base)
+constexpr uint32_t kOffQ = 0;                    // 2 x 8 KB (head-dim chunks)
+constexpr uint32_t kOffK = 16384;                // 2 stages x 32 KB
+constexpr uint32_t kOffV = kOffK + 2 * 32768;    // 2 stages x 32 KB
+constexpr uint32_t kOffP = kOffV + 2 * 32768;    // 2 x 16 KB
+constexpr uint32_t kOffO = kOffP + 2 * 16384;    // 16 KB output staging
+constexpr uint32_t kOffMisc = kOffO + 16384;
+constexpr uint32_t kSmemBytes = kOffMisc + 4096 + 1024;   // + alignment slack
+
+// TMEM columns
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColS0 = 0, kColO = 128;
+
+__device__ unsigned int g_tc_error;              // first failure code, 0 = none
+
+enum : uint32_t {
+  BAR_Q_FULL = 0, BAR_Q_EMPTY, BAR_K_FULL, BAR_K_EMPTY = BAR_K_FULL + 2, BAR_V_FULL = BAR_K_EMPTY + 2,
+  BAR_V_EMPTY = BAR_V_FULL + 2, BAR_S_FULL = BAR_V_EMPTY + 2, BAR_S_EMPTY = BAR_S_FULL + 2,
+  BAR_P_FULL = BAR_S_EMPTY + 2, BAR_P_EMPTY = BAR_P_FULL + 2, BAR_O_FULL = BAR_P_EMPTY + 2,
+  BAR_O_EMPTY, BAR_FINAL, NUM_BARS
+};
+
+struct Misc {
+  uint64_t bar[NUM_BARS];
+  uint32_t tmem_base;
+  uint32_t abort;
+  float m[64];          // running maximum per query (log2 domain)
+  float alpha[64];      // rescale factors of the current tile
+  float fin[64];        // combined column result (max or 1 / sum)
+  float red[4][64];     // per-warp partial column results
+};
+
+struct Args {
+  const int32_t* kv_idx;
+  const int32_t* kv_cnt;
+  int cap;
+  __nv_bfloat16* o;
+  float* lse;
+  long long N, Npad;
+  int nb;
+  long long items;
+  float scale_log2;
+  int dense;
+};
+
+// ---------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0u;
+}
+__device__ __forceinline__ unsigned long long gtimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
+  return t;
+}
+
+// Bounded wait: false on timeout (error word + abort flag set) or abort.
+__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
+                                      uint32_t where) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = gtimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63u) == 0u) {
+      if (*abort_flag) return false;
+      if (gtimer() - t0 > kWaitNs) {
+        atomicCAS(&g_tc_error, 0u, where);
+        *abort_flag = 1u;
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+
+__device__ __forceinline__ void named_bar(uint32_t id, uint32_t n) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ bool named_bar_or(uint32_t id, uint32_t n, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r) : "r"((uint32_t)pred), "r"(id), "r"(n) : "memory");
+  return r != 0u;
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
+               : "memory");
+}
+
+#define SVSA_R8(i) "=f"(r[i]), "=f"(r[i + 1]), "=f"(r[i + 2]), "=f"(r[i + 3]), "=f"(r[i + 4]), \
+                   "=f"(r[i + 5]), "=f"(r[i + 6]), "=f"(r[i + 7])
+#define SVSA_W8(i) "f"(r[i]), "f"(r[i + 1]), "f"(r[i + 2]), "f"(r[i + 3]), "f"(r[i + 4]), \
+                   "f"(r[i + 5]), "f"(r[i + 6]), "f"(r[i + 7])
+
+// 32 consecutive TMEM columns of this thread's lane (32x32b shape).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+      : SVSA_R8(0), SVSA_R8(8), SVSA_R8(16), SVSA_R8(24)
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n"
+      ::"r"(taddr), SVSA_W8(0), SVSA_W8(8), SVSA_W8(16), SVSA_W8(24)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
+  __half2 v = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 format, version 1).
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor, kind::f16 with f32 accumulation, M = 128, N = 64.
+// bf16 = 1 / fp16 = 0 in the A and B format fields (A and B always match).
+constexpr uint32_t idesc_f16(bool bf16, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) | ((a_mn_major ? 1u : 0u) << 15) |
+         ((b_mn_major ? 1u : 0u) << 16) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
+}
+
+// Column reduction of v[0..31] across the 32 lanes of a warp by halving
+// exchanges (31 shuffles); lane l ends with the result for column l.
+template <bool MAX>
+__device__ __forceinline__ float warp_colreduce32(float* v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1) {
+    const bool hi = (lane & w) != 0;
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      const float keep = hi ? v[i + w] : v[i];
+      const float send = hi ? v[i] : v[i + w];
+      const float other = __shfl_xor_sync(0xffffffffu, send, w);
+      v[i] = MAX ? fmaxf(keep, other) : keep + other;
+    }
+  }
+  return v[0];
+}
+
+// ---------------------------------------------------------------- the kernel
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                                                              const __grid_constant__ CUtensorMap tmK,
+                                                              const __grid_constant__ CUtensorMap tmV,
+                                                              const Args a) {
+  constexpr int NCH = D / 64;                    // 128-byte chunks of the head dim
+  constexpr int KSTEPS = D / 16;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  Misc* ms = reinterpret_cast<Misc*>(smem + kOffMisc);
+  const uint32_t sbase = su32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  volatile uint32_t* abort_flag = &ms->abort;
+  auto bar = [&](int i) { return su32(&ms->bar[i]); };
+
+  if (tid == 0) {
+    mbar_init(bar(BAR_Q_FULL), 1);
+    mbar_init(bar(BAR_Q_EMPTY), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(BAR_K_FULL + s), 1);
+      mbar_init(bar(BAR_K_EMPTY + s), 1);
+      mbar_init(bar(BAR_V_FULL + s), 1);
+      mbar_init(bar(BAR_V_EMPTY + s), 1);
+      mbar_init(bar(BAR_S_FULL + s), 1);
+      mbar_init(bar(BAR_S_EMPTY + s), 4);
+      mbar_init(bar(BAR_P_FULL + s), 4);
+      mbar_init(bar(BAR_P_EMPTY + s), 1);
+    }
+    mbar_init(bar(BAR_O_FULL), 1);
+    mbar_init(bar(BAR_O_EMPTY), 4);
+    mbar_init(bar(BAR_FINAL), 1);
+    ms->abort = 0u;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  if (D < 128) {
+    // the second head-dim chunk of every V stage stays zero: the MMA reads a
+    // 128-row V^T, rows d >= D contribute nothing
+    for (int s = 0; s < 2; ++s)
+      for (int i = tid; i < 16384 / 16; i += kThreads)
+        reinterpret_cast<uint4*>(smem + kOffV + s * 32768 + 16384)[i] = make_uint4(0u, 0u, 0u, 0u);
+    fence_async_smem();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(su32(&ms->tmem_base)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ms->tmem_base;
+  const long long items = a.items;
+  const int nb = a.nb;
+
+  auto item_count = [&](long long it) -> int {
+    if (a.dense) return nb;
+    const int c = a.kv_cnt[it];
+    return c < 0 ? 0 : (c > a.cap ? a.cap : c);
+  };
+  auto item_block = [&](long long it, int j) -> int {
+    if (a.dense) return j;
+    const int J = a.kv_idx[it * a.cap + j];
+    return J < 0 ? 0 : (J >= nb ? nb - 1 : J);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t qit = 0, kit = 0, vit = 0;
+      bool ok = true;
+      for (long long it = blockIdx.x; it < items && ok; it += gridDim.x) {
+        const int cnt = item_count(it);
+        if (cnt == 0) continue;
+        const long long bh = it / nb;
+        const int I = (int)(it % nb);
+        const int row_q = (int)(bh * a.Npad + (long long)I * kBlock);
+        ok = wait_bar(bar(BAR_Q_EMPTY), (qit & 1u) ^ 1u, abort_flag, 1);
+        if (!ok) break;
+        mbar_expect_tx(bar(BAR_Q_FULL), NCH * kBox);
+        for (int c = 0; c < NCH; ++c) tma_load_2d(sbase + kOffQ + c * kBox, &tmQ, c * 64, row_q, bar(BAR_Q_FULL));
+        ++qit;
+        const int npairs = (cnt + 1) >> 1;
+        for (int t = 0; t < npairs && ok; ++t) {
+          const int J1 = item_block(it, 2 * t);
+          const int J2 = (2 * t + 1 < cnt) ? item_block(it, 2 * t + 1) : J1;
+          const int r1 = (int)(bh * a.Npad + (long long)J1 * kBlock);
+          const int r2 = (int)(bh * a.Npad + (long long)J2 * kBlock);
+          const uint32_t ks = kit & 1u;
+          ok = wait_bar(bar(BAR_K_EMPTY + ks), ((kit >> 1) & 1u) ^ 1u, abort_flag, 2);
+          if (!ok) break;
+          mbar_expect_tx(bar(BAR_K_FULL + ks), 2 * NCH * kBox);
+          for (int c = 0; c < NCH; ++c) {
+            const uint32_t dst = sbase + kOffK + ks * 32768 + c * 16384;
+            tma_load_2d(dst, &tmK, c * 64, r1, bar(BAR_K_FULL + ks));
+            tma_load_2d(dst + kBox, &tmK, c * 64, r2, bar(BAR_K_FULL + ks));
+          }
+          ++kit;
+          const uint32_t vs = vit & 1u;
+          ok = wait_bar(bar(BAR_V_EMPTY + vs), ((vit >> 1) & 1u) ^ 1u, abort_flag, 3);
+          if (!ok) break;
+          mbar_expect_tx(bar(BAR_V_FULL + vs), 2 * NCH * kBox);
+          for (int c = 0; c < NCH; ++c) {
+            const uint32_t dst = sbase + kOffV + vs * 32768 + c * 16384;
+            tma_load_2d(dst, &tmV, c * 64, r1, bar(BAR_V_FULL + vs));
+            tma_load_2d(dst + kBox, &tmV, c * 64, r2, bar(BAR_V_FULL + vs));
+          }
+          ++vit;
+        }
+      }
+      // never leave with copies in flight: wait (bounded) for the last fill of each ring
+      volatile uint32_t no_abort = 0u;
+      if (qit > 0) wait_bar(bar(BAR_Q_FULL), (qit - 1) & 1u, &no_abort, 20);
+      for (uint32_t s = 0; s < 2; ++s) {
+        if (kit > s) wait_bar(bar(BAR_K_FULL + ((kit - 1 - s) & 1u)), ((kit - 1 - s) >> 1) & 1u, &no_abort, 21);
+        if (vit > s) wait_bar(bar(BAR_V_FULL + ((vit - 1 - s) & 1u)), ((vit - 1 - s) >> 1) & 1u, &no_abort, 22);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t ID_S = idesc_f16(true, false, false);    // bf16 K . Q^T
+      constexpr uint32_t ID_O = idesc_f16(false, true, true);     // fp16 V^T . P^T
+      uint32_t qit = 0, kit = 0, vit = 0, sit = 0, pit = 0, oit = 0;
+      bool ok = true;
+      for (long long it = blockIdx.x; it < items && ok; it += gridDim.x) {
+        const int cnt = item_count(it);
+        if (cnt == 0) continue;
+        const int npairs = (cnt + 1) >> 1;
+        ok = wait_bar(bar(BAR_Q_FULL), qit & 1u, abort_flag, 4);
+        if (!ok) break;
+        ++qit;
+        for (int t = 0; t <= npairs && ok; ++t) {
+          if (t < npairs) {
+            const uint32_t ks = kit & 1u, sb = sit & 1u;
+            ok = wait_bar(bar(BAR_K_FULL + ks), (kit >> 1) & 1u, abort_flag, 5) &&
+                 wait_bar(bar(BAR_S_EMPTY + sb), ((sit >> 1) & 1u) ^ 1u, abort_flag, 6);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t kbase = sbase + kOffK + ks * 32768;
+#pragma unroll
+            for (int kk = 0; kk < KSTEPS; ++kk) {
+              const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+              const uint32_t qoff = (kk >> 2) * kBox + (kk & 3) * 32;
+              umma_f16(tmem + kColS0 + sb * 64, sdesc(kbase + off, 16, 1024), sdesc(sbase + kOffQ + qoff, 16, 1024),
+                       ID_S, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(bar(BAR_K_EMPTY + ks));
+            umma_commit(bar(BAR_S_FULL + sb));
+            if (t == npairs - 1) umma_commit(bar(BAR_Q_EMPTY));
+            ++kit;
+            ++sit;
+          }
+          if (t >= 1) {
+            const int u = t - 1;
+            const uint32_t vs = vit & 1u, pb = pit & 1u;
+            ok = wait_bar(bar(BAR_V_FULL + vs), (vit >> 1) & 1u, abort_flag, 7) &&
+                 wait_bar(bar(BAR_P_FULL + pb), (pit >> 1) & 1u, abort_flag, 8) &&
+                 (u > 0 || wait_bar(bar(BAR_O_EMPTY), (oit & 1u) ^ 1u, abort_flag, 9));
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t vbase = sbase + kOffV + vs * 32768;
+            const uint32_t pbase = sbase + kOffP + pb * 16384;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              umma_f16(tmem + kColO, sdesc(vbase + kk * 2048, 16384, 1024), sdesc(pbase + kk * 2048, 16384, 1024),
+                       ID_O, (u > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(bar(BAR_V_EMPTY + vs));
+            umma_commit(bar(BAR_P_EMPTY + pb));
+            if (u == npairs - 1) {
+              umma_commit(bar(BAR_O_FULL));
+              ++oit;
+            }
+            ++vit;
+            ++pit;
+          }
+        }
+      }
+      // every issued MMA has finished before TMEM is released
+      umma_commit(bar(BAR_FINAL));
+      volatile uint32_t no_abort = 0u;
+      wait_bar(bar(BAR_FINAL), 0u, &no_abort, 23);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    // The 128 threads of this group meet at named barrier 1 in lock step.  A
+    // failed wait never makes one thread leave alone: it only sets the abort
+    // flag; the group leaves together after an OR-reduction over that flag.
+    const int sw = warp - 2;                       // 0..3
+    const int quad = warp & 3;                     // TMEM lane quadrant of this warp
+    const int k = quad * 32 + lane;                // key row (S^T) / head-dim row (O^T)
+    const int st = tid - 64;                       // 0..127 within the softmax group
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const float sl2 = a.scale_log2;
+    uint32_t sit = 0, oit = 0;
+    bool stop = false;
+    for (long long it = blockIdx.x; it < items && !stop; it += gridDim.x) {
+      const int cnt = item_count(it);
+      const long long bh = it / nb;
+      const int I = (int)(it % nb);
+      const long long q0 = (long long)I * kBlock;
+      __nv_bfloat16* og = a.o + (bh * a.Npad + q0) * D;
+      if (cnt == 0) {
+        for (int i = st; i < kBlock * D / 8; i += kSoftmaxThreads)
+          reinterpret_cast<uint4*>(og)[i] = make_uint4(0u, 0u, 0u, 0u);
+        if (a.lse != nullptr && st < 64) a.lse[bh * a.Npad + q0 + st] = 0.f;
+        continue;
+      }
+      const int npairs = (cnt + 1) >> 1;
+      if (st < 64) ms->m[st] = -INFINITY;
+      named_bar(1, kSoftmaxThreads);
+      float lp[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) lp[c] = 0.f;
+
+      for (int t = 0; t < npairs; ++t) {
+        const uint32_t sb = sit & 1u;
+        wait_bar(bar(BAR_S_FULL + sb), (sit >> 1) & 1u, abort_flag, 10);
+        tc_fence_after();
+        float s[64];
+        tmem_ld32(tmem + lane_off + kColS0 + sb * 64, s);
+        tmem_ld32(tmem + lane_off + kColS0 + sb * 64 + 32, s + 32);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(BAR_S_EMPTY + sb));
+
+        // this thread's key: slot 0 = first block of the pair, 1 = second
+        const int slot = k >> 6;
+        bool valid = 2 * t + slot < cnt;
+        if (valid) {
+          const int J = item_block(it, 2 * t + slot);
+          valid = (long long)J * kBlock + (k & 63) < a.N;
+        }
+        // x = scaled score (log2 domain); excess over the running maximum
+        float excess = -INFINITY;
+#pragma unroll
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 m4 = reinterpret_cast<const float4*>(ms->m)[c4];
+          const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * c4 + e;
+            const float x = valid ? s[c] * sl2 : -INFINITY;
+            s[c] = x;
+            excess = fmaxf(excess, x - mm[e]);
+          }
+        }
+        if (named_bar_or(1, kSoftmaxThreads, (*abort_flag != 0u) || excess > kLazyTh)) {
+          if (named_bar_or(1, kSoftmaxThreads, *abort_flag != 0u)) {
+            stop = true;
+            break;
+          }
+          // exact column maxima of this tile, 32 columns at a time
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            float v[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) v[c] = s[32 * h + c];
+            ms->red[sw][32 * h + lane] = warp_colreduce32<true>(v);
+          }
+          named_bar(1, kSoftmaxThreads);
+          if (st < 64) {
+            const float tmax = fmaxf(fmaxf(ms->red[0][st], ms->red[1][st]), fmaxf(ms->red[2][st], ms->red[3][st]));
+            const float m_old = ms->m[st];
+            const float m_new = fmaxf(m_old, tmax);
+            ms->m[st] = m_new;
+            ms->alpha[st] = (m_old == -INFINITY) ? 0.f : ex2(m_old - m_new);
+          }
+          named_bar(1, kSoftmaxThreads);
+#pragma unroll
+          for (int c = 0; c < 64; ++c) lp[c] *= ms->alpha[c];
+          if (t > 0) {
+            // O^T holds the previous tiles' sum once their MMA has finished
+            const uint32_t pprev = (sit - 1) & 1u;
+            wait_bar(bar(BAR_P_EMPTY + pprev), ((sit - 1) >> 1) & 1u, abort_flag, 11);
+            tc_fence_after();
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              float o[32];
+              tmem_ld32(tmem + lane_off + kColO + 32 * h, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 32; ++c) o[c] *= ms->alpha[32 * h + c];
+              tmem_st32(tmem + lane_off + kColO + 32 * h, o);
+            }
+            tmem_wait_st();
+          }
+        }
+        // P^T row k: exp2(x - m), fp16, in the 128-byte swizzled MN-major layout
+        uint32_t pk[32];
+#pragma unroll
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 m4 = reinterpret_cast<const float4*>(ms->m)[c4];
+          const float p0 = ex2(s[4 * c4] - m4.x), p1 = ex2(s[4 * c4 + 1] - m4.y);
+          const float p2 = ex2(s[4 * c4 + 2] - m4.z), p3 = ex2(s[4 * c4 + 3] - m4.w);
+          lp[4 * c4] += p0;
+          lp[4 * c4 + 1] += p1;
+          lp[4 * c4 + 2] += p2;
+          lp[4 * c4 + 3] += p3;
+          pk[2 * c4] = pack_f16x2(p0, p1);
+          pk[2 * c4 + 1] = pack_f16x2(p2, p3);
+        }
+        wait_bar(bar(BAR_P_EMPTY + sb), ((sit >> 1) & 1u) ^ 1u, abort_flag, 12);
+        unsigned char* prow = smem + kOffP + sb * 16384 + (k >> 3) * 1024 + (k & 7) * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<uint4*>(prow + ((j ^ (k & 7)) << 4)) =
+              make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        fence_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(BAR_P_FULL + sb));
+        ++sit;
+      }
+      if (stop) break;
+
+      // ---- epilogue: column sums, normalise O^T, stage as [query][d], store
+#pragma unroll
+      for (int h = 0; h < 2; ++h) ms->red[sw][32 * h + lane] = warp_colreduce32<false>(lp + 32 * h);
+      named_bar(1, kSoftmaxThreads);
+      if (st < 64) {
+        const float l = ms->red[0][st] + ms->red[1][st] + ms->red[2][st] + ms->red[3][st];
+        ms->fin[st] = l > 0.f ? 1.f / l : 0.f;
+        if (a.lse != nullptr) {
+          const float ln2 = 0.6931471805599453f;
+          a.lse[bh * a.Npad + q0 + st] = (q0 + st < a.N && l > 0.f) ? (ms->m[st] + __log2f(l)) * ln2 : 0.f;
+        }
+      }
+      wait_bar(bar(BAR_O_FULL), oit & 1u, abort_flag, 13);
+      ++oit;
+      tc_fence_after();
+      named_bar(1, kSoftmaxThreads);
+      unsigned char* ost = smem + kOffO;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float o[32];
+        tmem_ld32(tmem + lane_off + kColO + 32 * h, o);
+        tmem_wait_ld();
+        if (k < D) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const int qc = 32 * h + c;
+            reinterpret_cast<__nv_bfloat16*>(ost)[qc * D + k] = __float2bfloat16_rn(o[c] * ms->fin[qc]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_O_EMPTY));
+      named_bar(1, kSoftmaxThreads);
+      constexpr int CPR = D / 8;
+      for (int i = st; i < kBlock * CPR; i += kSoftmaxThreads) {
+        const int r = i / CPR;
+        uint4 val = reinterpret_cast<const uint4*>(ost)[i];
+        if (q0 + r >= a.N) val = make_uint4(0u, 0u, 0u, 0u);
+        reinterpret_cast<uint4*>(og)[i] = val;
+      }
+      stop = named_bar_or(1, kSoftmaxThreads, *abort_flag != 0u);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kTmemCols));
+  }
+}
+
+}  // namespace tc
+
+// ---------------------------------------------------------------- host side
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2D view [rows, d] of a 16-bit tensor, 64 x 64 boxes, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, long long rows, int d, bool f16) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+             const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = kNumSMs;
+  }
+  return n;
+}
+
+}  // namespace
+
+cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, const int32_t* kv_idx,
+                           const int32_t* kv_cnt, int cap, void* o, float* lse, long long BH, long long N, int nb,
+                           int d, bool dense, cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
+  const long long rows = BH * (long long)nb * kBlock;
+  if (!make_map(&mq, q, rows, d, false) || !make_map(&mk, k, rows, d, false) || !make_map(&mv, v, rows, d, true))
+    return cudaErrorInvalidValue;
+  tc::Args a;
+  a.kv_idx = kv_idx; a.kv_cnt = kv_cnt; a.cap = cap;
+  a.o = (__nv_bfloat16*)o; a.lse = lse;
+  a.N = N; a.nb = nb; a.Npad = (long long)nb * kBlock;
+  a.items = BH * nb;
+  a.scale_log2 = 1.4426950408889634f / sqrtf((float)d);
+  a.dense = dense ? 1 : 0;
+  const long long grid = std::min<long long>(a.items, sm_count());
+  cudaError_t e;
+  if (d == 128) {
+    e = cudaFuncSetAttribute(tc::attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    tc::attn_tc_kernel<128><<<(unsigned)grid, tc::kThreads, tc::kSmemBytes, st>>>(mq, mk, mv, a);
+  } else if (d == 64) {
+    e = cudaFuncSetAttribute(tc::attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    tc::attn_tc_kernel<64><<<(unsigned)grid, tc::kThreads, tc::kSmemBytes, st>>>(mq, mk, mv, a);
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+// Read and clear the device error word (0 = no failure).
+cudaError_t attn_tc_error(unsigned int* code, cudaStream_t st) {
+  unsigned int zero = 0u;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(code, tc::g_tc_error, sizeof(unsigned int), 0,
+                                            cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return e;
+  e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return e;
+  if (*code != 0u) e = cudaMemcpyToSymbolAsync(tc::g_tc_error, &zero, sizeof(unsigned int), 0, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return e;
+  return cudaStreamSynchronize(st);
+}
+
+}  // namespace svsa

@@ -8,15 +8,21 @@
 // or 32 (d=64) row lanes x CPR chunk lanes; each thread keeps fp32 partial
 // sums of its rows per group, and the row lanes are added in a fixed order
 // through shared memory, so the result is deterministic.
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 
 namespace svsa {
 
 constexpr int kPoolThreads = 256;
 
-template <int D, int SIZE>
+__device__ __forceinline__ float2 pair_to_float2(const __nv_bfloat162& v) { return __bfloat1622float2(v); }
+__device__ __forceinline__ float2 pair_to_float2(const __half2& v) { return __half22float2(v); }
+
+// T2 = __nv_bfloat162 (queries, keys) or __half2 (values)
+template <int D, int SIZE, typename T2>
 __global__ void __launch_bounds__(kPoolThreads) pool_kernel(
-    const __nv_bfloat16* __restrict__ xp, float* __restrict__ out, int32_t* __restrict__ nvalid,
+    const T2* __restrict__ xp, float* __restrict__ out, int32_t* __restrict__ nvalid,
     long long N, long long Npad) {
   constexpr int CPR = D / 8;                 // 16-byte chunks per row
   constexpr int RL = kPoolThreads / CPR;     // row lanes
@@ -28,7 +34,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(
   const long long bh = blockIdx.y;
   const int ch = threadIdx.x % CPR, rl = threadIdx.x / CPR;
   const long long row0 = (long long)blk * kBlock;
-  const __nv_bfloat16* base = xp + (bh * Npad + row0) * D;
+  const T2* base = xp + (bh * Npad + row0) * (D / 2);
 
   float acc[G][8];
 #pragma unroll
@@ -40,15 +46,15 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(
   for (int u = 0; u < RPT; ++u) {
     const int r = rl + RL * u;
     if (row0 + r < N) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(base + (long long)r * D) + ch);
-      const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(base + (long long)r * (D / 2)) + ch);
+      const T2* p = reinterpret_cast<const T2*>(&v);
       const int g = r / SIZE;
 #pragma unroll
       for (int gg = 0; gg < G; ++gg) {
         if (gg == g) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(p[e]);
+            const float2 f = pair_to_float2(p[e]);
             acc[gg][2 * e] += f.x;
             acc[gg][2 * e + 1] += f.y;
           }
@@ -84,16 +90,29 @@ cudaError_t launch_nvalid(int32_t* nvalid, long long N, int nb, cudaStream_t st)
   return cudaGetLastError();
 }
 
-cudaError_t launch_pool(const void* xp, float* out, int32_t* nvalid, long long BH, long long N,
-                        long long Npad, int d, int size, cudaStream_t st) {
+template <typename T2>
+static cudaError_t launch_pool_t(const void* xp, float* out, int32_t* nvalid, long long BH, long long N,
+                                 long long Npad, int d, int size, cudaStream_t st) {
   dim3 grid((unsigned)(Npad / kBlock), (unsigned)BH);
-  const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(xp);
-  if (d == 128 && size == 64) pool_kernel<128, 64><<<grid, kPoolThreads, 0, st>>>(x, out, nvalid, N, Npad);
-  else if (d == 128 && size == 16) pool_kernel<128, 16><<<grid, kPoolThreads, 0, st>>>(x, out, nvalid, N, Npad);
-  else if (d == 64 && size == 64) pool_kernel<64, 64><<<grid, kPoolThreads, 0, st>>>(x, out, nvalid, N, Npad);
-  else if (d == 64 && size == 16) pool_kernel<64, 16><<<grid, kPoolThreads, 0, st>>>(x, out, nvalid, N, Npad);
+  const T2* x = reinterpret_cast<const T2*>(xp);
+  if (d == 128 && size == 64) pool_kernel<128, 64, T2><<<grid, kPoolThreads, 0, st>>>(x, out, nvalid, N, Npad);
+  else if (d == 128 && size == 16) pool_kernel<128, 16, T2><<<grid, kPoolThreads, 0, st>>>(x, out, nvalid, N, Npad);
+  else if (d == 64 && size == 64) pool_kernel<64, 64, T2><<<grid, kPoolThreads, 0, st>>>(x, out, nvalid, N, Npad);
+  else if (d == 64 && size == 16) pool_kernel<64, 16, T2><<<grid, kPoolThreads, 0, st>>>(x, out, nvalid, N, Npad);
   else return cudaErrorInvalidValue;
   return cudaGetLastError();
+}
+
+// bf16 input (queries, keys)
+cudaError_t launch_pool(const void* xp, float* out, int32_t* nvalid, long long BH, long long N,
+                        long long Npad, int d, int size, cudaStream_t st) {
+  return launch_pool_t<__nv_bfloat162>(xp, out, nvalid, BH, N, Npad, d, size, st);
+}
+
+// fp16 input (reordered values)
+cudaError_t launch_pool_f16(const void* xp, float* out, int32_t* nvalid, long long BH, long long N,
+                            long long Npad, int d, int size, cudaStream_t st) {
+  return launch_pool_t<__half2>(xp, out, nvalid, BH, N, Npad, d, size, st);
 }
 
 }  // namespace svsa

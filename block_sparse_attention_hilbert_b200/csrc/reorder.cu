@@ -2,6 +2,8 @@
 //
 // Forward  ("DFSAttn", trick 1):  xp[bh, i, :] = x[bh, perm[i], :]   (zeros where perm[i] < 0)
 // Inverse:                        o[bh, r, :]  = op[bh, iperm[r], :]
+// The value tensor's forward gather also converts bf16 -> fp16 (the P.V
+// product runs in fp16).
 //
 // Both are pure data movement (HBM-bound): every thread moves 16-byte chunks,
 // consecutive threads cover consecutive bytes of the destination (coalesced
@@ -52,15 +54,72 @@ __global__ void __launch_bounds__(kGatherThreads) gather_rows_kernel(
   }
 }
 
+// bf16 -> fp16 conversion of one 16-byte chunk (8 values), saturating at
+// +-65504; exact for every bf16 value in fp16's normal range.
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
+  const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&v);
+  uint4 out;
+  uint32_t* o = reinterpret_cast<uint32_t*>(&out);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __bfloat1622float2(b[e]);
+    uint32_t h;
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;\n" : "=r"(h) : "f"(f.y), "f"(f.x));
+    o[e] = h;
+  }
+  return out;
+}
+
+template <int CPR>
+__global__ void __launch_bounds__(kGatherThreads) gather_rows_f16_kernel(
+    const uint4* __restrict__ src, uint4* __restrict__ dst, const int32_t* __restrict__ map,
+    long long rows_dst, long long rows_src) {
+  const long long bh = blockIdx.y;
+  const long long total = rows_dst * CPR;
+  const uint4* s_base = src + bh * rows_src * CPR;
+  uint4* d_base = dst + bh * rows_dst * CPR;
+  const long long tile = (long long)kGatherThreads * kUnroll;
+  for (long long base = (long long)blockIdx.x * tile; base < total; base += (long long)gridDim.x * tile) {
+    uint4 v[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const long long c = base + u * kGatherThreads + threadIdx.x;
+      v[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (c < total) {
+        const int32_t srow = __ldg(map + c / CPR);
+        if (srow >= 0) v[u] = ld_stream(s_base + (long long)srow * CPR + (c % CPR));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const long long c = base + u * kGatherThreads + threadIdx.x;
+      if (c < total) d_base[c] = bf16x8_to_f16x8(v[u]);
+    }
+  }
+}
+
+cudaError_t launch_gather_rows_f16(const void* src, void* dst, const int32_t* map, long long BH,
+                                   long long rows_dst, long long rows_src, int d, cudaStream_t st) {
+  const int cpr = d * 2 / 16;
+  const long long total = rows_dst * cpr;
+  const long long tile = (long long)kGatherThreads * kUnroll;
+  const long long gx = std::max<long long>(1, (total + tile - 1) / tile);
+  dim3 grid((unsigned)gx, (unsigned)BH);
+  if (cpr == 16)
+    gather_rows_f16_kernel<16><<<grid, kGatherThreads, 0, st>>>((const uint4*)src, (uint4*)dst, map, rows_dst, rows_src);
+  else if (cpr == 8)
+    gather_rows_f16_kernel<8><<<grid, kGatherThreads, 0, st>>>((const uint4*)src, (uint4*)dst, map, rows_dst, rows_src);
+  else
+    return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* map, long long BH,
                                long long rows_dst, long long rows_src, int d, cudaStream_t st) {
   const int cpr = d * 2 / 16;
   const long long total = rows_dst * cpr;
   const long long tile = (long long)kGatherThreads * kUnroll;
-  long long gx = (total + tile - 1) / tile;
-  // enough CTAs to fill the GPU several times over, as a multiple of the SM count
-  const long long want = std::max<long long>(1, (kNumSMs * 8LL + BH - 1) / BH);
-  gx = std::max<long long>(1, std::min<long long>(gx, std::max<long long>(want, gx)));
+  const long long gx = std::max<long long>(1, (total + tile - 1) / tile);
   dim3 grid((unsigned)gx, (unsigned)BH);
   if (cpr == 16)
     gather_rows_kernel<16><<<grid, kGatherThreads, 0, st>>>(

@@ -13,6 +13,8 @@
 // tiles arrive, so each e_IJ is first taken against the maximum m_J known at
 // tile J and stored with m_J; a final sweep turns it into
 // e * exp(m_J - M) / Z * 64 / n_J.  fp32 throughout.
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 
 namespace svsa {
@@ -23,13 +25,13 @@ constexpr int kRouteRows = 16;
 template <int D>
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(
     const float* __restrict__ qbar, const __nv_bfloat16* __restrict__ kp,
-    const __nv_bfloat16* __restrict__ vp, const float* __restrict__ kbar,
+    const __half* __restrict__ vp, const float* __restrict__ kbar,
     const float* __restrict__ vbar, float* __restrict__ R, float* __restrict__ Rm, long long N, int nb,
     float scale) {
   constexpr int CH = D / 16;                          // channels per thread in the value phase
   __shared__ float q_s[kRouteRows][D];
   __shared__ __nv_bfloat16 k_s[kBlock][D + 8];
-  __shared__ __nv_bfloat16 v_s[kBlock][D];
+  __shared__ __half v_s[kBlock][D];
   __shared__ float e_s[kRouteRows][kBlock];
   __shared__ float m_s[kRouteRows], z_s[kRouteRows];
 
@@ -51,7 +53,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(
   for (int J = 0; J < nb; ++J) {
     __syncthreads();
     const __nv_bfloat16* kb = kp + (bh * Npad + (long long)J * kBlock) * D;
-    const __nv_bfloat16* vb = vp + (bh * Npad + (long long)J * kBlock) * D;
+    const __half* vb = vp + (bh * Npad + (long long)J * kBlock) * D;
     for (int o = tid; o < kBlock * D / 8; o += kRouteThreads) {
       const int r = o / (D / 8), c = (o % (D / 8)) * 8;
       const uint4 kv = *reinterpret_cast<const uint4*>(kb + (long long)r * D + c);
@@ -108,7 +110,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(
       const int c = sub * CH + u;
       float a = 0.f;
 #pragma unroll 8
-      for (int j = 0; j < kBlock; ++j) a = fmaf(e_s[row][j], __bfloat162float(v_s[j][c]), a);
+      for (int j = 0; j < kBlock; ++j) a = fmaf(e_s[row][j], __half2float(v_s[j][c]), a);
       const float diff = a - cw * vbJ[c];
       err2 = fmaf(diff, diff, err2);
     }
@@ -137,7 +139,7 @@ cudaError_t launch_route(const float* qbar, const void* kp, const void* vp, cons
   dim3 grid((unsigned)((nb + kRouteRows - 1) / kRouteRows), (unsigned)BH);
   const float scale = 1.0f / sqrtf((float)d);
   const __nv_bfloat16* k = reinterpret_cast<const __nv_bfloat16*>(kp);
-  const __nv_bfloat16* v = reinterpret_cast<const __nv_bfloat16*>(vp);
+  const __half* v = reinterpret_cast<const __half*>(vp);
   if (d == 128) route_kernel<128><<<grid, kRouteThreads, 0, st>>>(qbar, k, v, kbar, vbar, R, Rm, N, nb, scale);
   else if (d == 64) route_kernel<64><<<grid, kRouteThreads, 0, st>>>(qbar, k, v, kbar, vbar, R, Rm, N, nb, scale);
   else return cudaErrorInvalidValue;

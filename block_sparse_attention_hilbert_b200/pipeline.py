@@ -3,7 +3,7 @@
     attn = SparseVideoAttention(B, heads, T, H, W, d, order="hilbert", select="topk", keep_frac=0.25)
     o = attn(q, k, v)               # q, k, v: bf16 [B, heads, T*H*W, d] on the GPU, raster order
 
-A call runs svsa_reorder (x3), svsa_build_mask (unless the cached mask is
+A call runs svsa_reorder (Q, K), svsa_reorder_values (V), svsa_build_mask (unless the cached mask is
 reused across denoising steps -- "DFSAttn" trick 3), svsa_attn_fwd and
 svsa_inverse_reorder on the current stream.  The permutation is built once per
 object.  Buffers are allocated once with torch (the library allocates nothing).
@@ -17,7 +17,7 @@ import torch
 from . import (ORDER_HILBERT, ORDER_RASTER, SEL_STRUCTURED, SEL_THRESHOLD, SEL_TOPK, BLOCK,
                make_mask, mask_params, shape, svsa_attn_dense_fwd, svsa_attn_fwd, svsa_build_mask,
                svsa_build_perm, svsa_inverse_reorder, svsa_mask_workspace_bytes,
-               svsa_perm_workspace_bytes, svsa_reorder)
+               svsa_perm_workspace_bytes, svsa_reorder, svsa_reorder_values)
 
 _ORDERS = {"raster": ORDER_RASTER, "hilbert": ORDER_HILBERT}
 _SELECTS = {"threshold": SEL_THRESHOLD, "topk": SEL_TOPK, "structured": SEL_STRUCTURED}
@@ -38,7 +38,7 @@ class LayerBuffers:
         self.perm_ws = torch.empty(max(perm_ws_bytes, 16), dtype=torch.uint8, device=dev)
         self.qp = torch.empty(B, heads, Npad, d, dtype=bf, device=dev)
         self.kp = torch.empty_like(self.qp)
-        self.vp = torch.empty_like(self.qp)
+        self.vp = torch.empty(B, heads, Npad, d, dtype=torch.float16, device=dev)   # values in fp16
         self.op = torch.empty_like(self.qp)
         self.kv_idx = torch.empty(B, heads, nb, cap, dtype=torch.int32, device=dev)
         self.kv_cnt = torch.empty(B, heads, nb, dtype=torch.int32, device=dev)
@@ -89,8 +89,9 @@ class SparseVideoAttention:
         if not self._perm_ready:
             self.build_perm(stream)
         b = self.buf
-        for x, xp in ((q, b.qp), (k, b.kp), (v, b.vp)):
-            svsa_reorder(x, xp, b.perm, self.shape, stream)
+        svsa_reorder(q, b.qp, b.perm, self.shape, stream)
+        svsa_reorder(k, b.kp, b.perm, self.shape, stream)
+        svsa_reorder_values(v, b.vp, b.perm, self.shape, stream)
 
     def build_mask(self, anchor_offset: int = 0, stream=None):
         b = self.buf

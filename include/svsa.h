@@ -127,18 +127,28 @@ size_t svsa_perm_workspace_bytes(svsa_shape s, int32_t order);
 svsa_status svsa_build_perm(svsa_shape s, int32_t order, int32_t* perm, int32_t* iperm,
                             void* ws, size_t ws_bytes, void* stream);
 
-/* Gather one tensor into the reordered layout:
+/* Gather the queries or the keys into the reordered layout:
  *   xp[b, h, i, :] = x[b, h, perm[i], :] for i < Npad (zeros where perm[i] = -1).
  * x: bf16 [B, heads, N, d]; xp: bf16 [B, heads, Npad, d]; perm from
- * svsa_build_perm.  Call once per tensor (Q, K, V). */
+ * svsa_build_perm.  Call once for Q and once for K. */
 svsa_status svsa_reorder(const void* x, void* xp, const int32_t* perm, svsa_shape s, void* stream);
+
+/* The same gather for the values, converting bf16 to fp16:
+ *   vp[b, h, i, :] = fp16(v[b, h, perm[i], :]) (zeros where perm[i] = -1).
+ * v: bf16 [B, heads, N, d]; vp: fp16 [B, heads, Npad, d].  The conversion is
+ * exact for every bf16 value of magnitude in [2^-14, 65504] (smaller ones keep
+ * fp16's 2^-24 absolute resolution, larger ones saturate to +-65504).  The
+ * attention's P.V product runs in fp16 so that the softmax weights keep an
+ * 11-bit significand. */
+svsa_status svsa_reorder_values(const void* v, void* vp, const int32_t* perm, svsa_shape s, void* stream);
 
 /* ---- step 2: block mask ------------------------------------------------- */
 
 /* Workspace bytes svsa_build_mask needs for this shape and rule. */
 size_t svsa_mask_workspace_bytes(svsa_shape s, const svsa_mask_params* p);
 
-/* Build the block mask from reordered Q and K (and V for routing).
+/* Build the block mask from reordered Q and K (bf16) and V (fp16, from
+ * svsa_reorder_values; needed for routing and for mask.vbar).
  * THRESHOLD / TOPK: pooled block scores P_IJ = softmax_J(qbar_I . kbar_J /
  *   sqrt(d)) over all key blocks (means over valid tokens; with sub_block = 16
  *   the per-sub-block softmax probabilities are summed over the 16 sub-pairs
@@ -161,10 +171,11 @@ svsa_status svsa_build_mask(const void* qp, const void* kp, const void* vp, cons
 
 /* ---- step 3: attention -------------------------------------------------- */
 
-/* Block-sparse attention over the reordered tensors:
+/* Block-sparse attention over the reordered tensors (qp, kp bf16 from
+ * svsa_reorder, vp fp16 from svsa_reorder_values):
  *   O_i = sum_{J kept for block(i)} sum_{j in J, j < N} softmax(q_i . k_j / sqrt(d)) v_j
- * computed with an online softmax (fp32 statistics and accumulators, bf16
- * tensor-core products, P rounded to bf16).  compensate = 1 adds, for every
+ * computed with an online softmax on the tensor cores (Q.K^T in bf16, P.V in
+ * fp16, fp32 statistics and accumulators, P rounded to fp16).  compensate = 1 adds, for every
  * skipped block J, n_J copies of (kbar_J, vbar_J) to the same softmax
  * (SVG-EAR 2.A); that needs m->kbar, m->vbar and m->nvalid.
  * op: bf16 [B, heads, Npad, d] (pad rows are written as zeros).
@@ -173,7 +184,7 @@ svsa_status svsa_build_mask(const void* qp, const void* kp, const void* vp, cons
 svsa_status svsa_attn_fwd(const void* qp, const void* kp, const void* vp, const svsa_mask* m,
                           int32_t compensate, void* op, float* lse, svsa_shape s, void* stream);
 
-/* Dense attention over all N keys, same arithmetic and layout as
+/* Dense attention over all N keys, same arithmetic and layouts as
  * svsa_attn_fwd; the denominator of the speedup the benchmark reports. */
 svsa_status svsa_attn_dense_fwd(const void* qp, const void* kp, const void* vp, void* op,
                                 float* lse, svsa_shape s, void* stream);

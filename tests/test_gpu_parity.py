@@ -60,6 +60,26 @@ def test_reorder_inverse_bit_exact(d, grid):
     assert torch.equal(out.view(torch.int16), x.view(torch.int16))
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_reorder_values_fp16_bit_exact(d):
+    T, H, W = 2, 9, 13
+    B, h = 1, 2
+    N = T * H * W
+    g = torch.Generator().manual_seed(9)
+    v = (torch.randn(B, h, N, d, generator=g) * 3.0)
+    v[0, 0, :5, 0] = torch.tensor([1e-6, -3e-7, 6.1e-5, 70000.0, -1e5])     # subnormal and saturating cases
+    v = v.to(torch.bfloat16).cuda()
+    attn = svsa.SparseVideoAttention(B, h, T, H, W, d, order="hilbert", select="topk")
+    attn.build_perm()
+    b = attn.buf
+    svsa.svsa_reorder_values(v, b.vp, b.perm, attn.shape)
+    svsa.svsa_sync_status()
+    perm, _ = oracle.build_perm(T, H, W, "hilbert")
+    vf16 = v.float().clamp(-65504, 65504).to(torch.float16).cpu()
+    expect = oracle.reorder(vf16.view(torch.int16).numpy(), perm)
+    assert np.array_equal(b.vp.cpu().view(torch.int16).numpy(), expect)
+
+
 def _small(select, sub=64, grid=(5, 7, 9), heads=2, d=128, **kw):
     T, H, W = grid
     return workloads.Workload("small", 1, heads, d, T, H, W, select=select, sub_block=sub, **kw)
