@@ -16,9 +16,9 @@
 //     Both accumulate in TMEM (S^T double-buffered, O^T resident).
 //   * Warp roles: warp 0 issues TMA copies (Q once per item; K and V of each
 //     pair into 2-stage rings, 64-row boxes with 128-byte swizzle), warp 1
-//     issues the MMAs from one thread and owns the TMEM allocation, warps 2-5
-//     (one thread per key / per head-dim lane) run the softmax and the
-//     epilogue.  All hand-offs are mbarriers; every wait is bounded in time
+//     issues the MMAs from one thread and owns the TMEM allocation, warps 2-9
+//     (two warpgroups, one thread per key / head-dim lane, 32 query columns
+//     per group) run the softmax and the epilogue.  All hand-offs are mbarriers; every wait is bounded in time
 //     and a timeout sets an error word read by svsa_sync_status.
 //   * Softmax: thread k holds key k's 64 scores.  A column (query) maximum
 //     needs all 128 threads, so the running maximum is lazy: a tile only
@@ -35,6 +35,8 @@
 //     their rounding well inside the output tolerance.
 #include <cuda.h>
 
+#include <cstddef>
+
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -42,43 +44,52 @@
 namespace svsa {
 namespace tc {
 
-constexpr int kThreads = 192;
-constexpr int kSoftmaxThreads = 128;
+#ifndef SVSA_TC_GROUPS
+#define SVSA_TC_GROUPS 4
+#endif
+// warp 0 Q/K TMA, 1 S-MMA (and TMEM owner), 2 V TMA, 3 O-MMA, 4.. softmax warpgroups
+constexpr int kGroups = SVSA_TC_GROUPS;          // softmax warpgroups; each owns 64 / kGroups query columns
+constexpr int kCols = 64 / kGroups;
+constexpr int kThreads = 32 * (4 + 4 * kGroups);
+constexpr int kKStages = 3, kVStages = 2, kSBufs = 3, kPBufs = 2;
+constexpr int kSoftmaxThreads = 128;             // one softmax warpgroup
 constexpr uint32_t kBox = 8192;                  // one 64-row x 128-byte TMA box
 constexpr float kLazyTh = 8.0f;                  // log2 headroom before a rescale
 constexpr unsigned long long kWaitNs = 2000000000ull;   // 2 s per wait
 
 // shared memory map (offsets from a 1024-byte aligned base)
-constexpr uint32_t kOffQ = 0;                    // 2 x 8 KB (head-dim chunks)
-constexpr uint32_t kOffK = 16384;                // 2 stages x 32 KB
-constexpr uint32_t kOffV = kOffK + 2 * 32768;    // 2 stages x 32 KB
-constexpr uint32_t kOffP = kOffV + 2 * 32768;    // 2 x 16 KB
-constexpr uint32_t kOffO = kOffP + 2 * 16384;    // 16 KB output staging
-constexpr uint32_t kOffMisc = kOffO + 16384;
-constexpr uint32_t kSmemBytes = kOffMisc + 4096 + 1024;   // + alignment slack
+constexpr uint32_t kOffQ = 0;                               // 2 x 8 KB (head-dim chunks)
+constexpr uint32_t kOffK = 16384;                           // kKStages x 32 KB
+constexpr uint32_t kOffV = kOffK + kKStages * 32768;        // kVStages x 32 KB
+constexpr uint32_t kOffP = kOffV + kVStages * 32768;        // kPBufs x 16 KB
+constexpr uint32_t kOffMisc = kOffP + kPBufs * 16384;
+constexpr uint32_t kSmemBytes = kOffMisc + 2048 + 1024;     // + alignment slack
 
-// TMEM columns
+// TMEM columns: three S^T buffers and O^T
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS0 = 0, kColO = 128;
+constexpr uint32_t kColS0 = 0, kColO = 192;
 
 __device__ unsigned int g_tc_error;              // first failure code, 0 = none
 
 enum : uint32_t {
-  BAR_Q_FULL = 0, BAR_Q_EMPTY, BAR_K_FULL, BAR_K_EMPTY = BAR_K_FULL + 2, BAR_V_FULL = BAR_K_EMPTY + 2,
-  BAR_V_EMPTY = BAR_V_FULL + 2, BAR_S_FULL = BAR_V_EMPTY + 2, BAR_S_EMPTY = BAR_S_FULL + 2,
-  BAR_P_FULL = BAR_S_EMPTY + 2, BAR_P_EMPTY = BAR_P_FULL + 2, BAR_O_FULL = BAR_P_EMPTY + 2,
-  BAR_O_EMPTY, BAR_FINAL, NUM_BARS
+  BAR_Q_FULL = 0, BAR_Q_EMPTY, BAR_K_FULL, BAR_K_EMPTY = BAR_K_FULL + kKStages,
+  BAR_V_FULL = BAR_K_EMPTY + kKStages, BAR_V_EMPTY = BAR_V_FULL + kVStages,
+  BAR_S_FULL = BAR_V_EMPTY + kVStages, BAR_S_EMPTY = BAR_S_FULL + kSBufs,
+  BAR_P_FULL = BAR_S_EMPTY + kSBufs, BAR_P_EMPTY = BAR_P_FULL + kPBufs, BAR_O_FULL = BAR_P_EMPTY + kPBufs,
+  BAR_O_EMPTY, BAR_FINAL, BAR_FINAL2, NUM_BARS
 };
 
 struct Misc {
   uint64_t bar[NUM_BARS];
   uint32_t tmem_base;
   uint32_t abort;
-  float m[64];          // running maximum per query (log2 domain)
-  float alpha[64];      // rescale factors of the current tile
-  float fin[64];        // combined column result (max or 1 / sum)
-  float red[4][64];     // per-warp partial column results
+  alignas(16) float m[64];          // running maximum per query (log2 domain); read as float4
+  alignas(16) float alpha[64];      // rescale factors of the current tile
+  alignas(16) float fin[64];        // shift of this tile's scores, then 1 / row sum
+  alignas(16) float red[kGroups][4][kCols];  // per-warp partial column results of each warpgroup
 };
+static_assert(offsetof(Misc, m) % 16 == 0 && offsetof(Misc, alpha) % 16 == 0, "float4 access");
+static_assert(sizeof(Misc) <= 2048, "misc region");
 
 struct Args {
   const int32_t* kv_idx;
@@ -112,6 +123,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
   return ok != 0u;
 }
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0u;
+}
 __device__ __forceinline__ unsigned long long gtimer() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
@@ -119,9 +137,8 @@ __device__ __forceinline__ unsigned long long gtimer() {
 }
 
 // Bounded wait: false on timeout (error word + abort flag set) or abort.
-__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
-                                      uint32_t where) {
-  if (mbar_try_wait(bar, parity)) return true;
+__device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
+                                           uint32_t where) {
   const unsigned long long t0 = gtimer();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -134,6 +151,11 @@ __device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile ui
       }
     }
   }
+}
+
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
+                                         uint32_t where) {
+  return mbar_try_wait(bar, parity) || wait_bar_slow(bar, parity, abort_flag, where);
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
@@ -189,6 +211,28 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* r) {
       ::"r"(taddr), SVSA_W8(0), SVSA_W8(8), SVSA_W8(16), SVSA_W8(24)
       : "memory");
 }
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+      : SVSA_R8(0), SVSA_R8(8)
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n"
+      ::"r"(taddr), SVSA_W8(0), SVSA_W8(8)
+      : "memory");
+}
+template <int NC>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float* r) {
+  if constexpr (NC == 32) tmem_ld32(taddr, r);
+  else tmem_ld16(taddr, r);
+}
+template <int NC>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const float* r) {
+  if constexpr (NC == 32) tmem_st32(taddr, r);
+  else tmem_st16(taddr, r);
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
 
@@ -216,13 +260,15 @@ constexpr uint32_t idesc_f16(bool bf16, bool a_mn_major, bool b_mn_major) {
          ((b_mn_major ? 1u : 0u) << 16) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
 }
 
-// Column reduction of v[0..31] across the 32 lanes of a warp by halving
-// exchanges (31 shuffles); lane l ends with the result for column l.
-template <bool MAX>
-__device__ __forceinline__ float warp_colreduce32(float* v) {
+// Column reduction of v[0..NC-1] across the 32 lanes of a warp: halving
+// exchanges over lane bits log2(NC)-1 .. 0 leave lane l with column l % NC
+// summed over the lanes that share its upper bits; xor-shuffles over those
+// upper bits finish the reduction (31 shuffles for NC = 32, 16 for NC = 16).
+template <bool MAX, int NC>
+__device__ __forceinline__ float warp_colreduce(float* v) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int w = 16; w >= 1; w >>= 1) {
+  for (int w = NC / 2; w >= 1; w >>= 1) {
     const bool hi = (lane & w) != 0;
 #pragma unroll
     for (int i = 0; i < w; ++i) {
@@ -232,7 +278,13 @@ __device__ __forceinline__ float warp_colreduce32(float* v) {
       v[i] = MAX ? fmaxf(keep, other) : keep + other;
     }
   }
-  return v[0];
+  float r = v[0];
+#pragma unroll
+  for (int o = NC; o < 32; o <<= 1) {
+    const float other = __shfl_xor_sync(0xffffffffu, r, o);
+    r = MAX ? fmaxf(r, other) : r + other;
+  }
+  return r;
 }
 
 // ---------------------------------------------------------------- the kernel
@@ -254,26 +306,33 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   if (tid == 0) {
     mbar_init(bar(BAR_Q_FULL), 1);
     mbar_init(bar(BAR_Q_EMPTY), 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(BAR_K_FULL + s), 1);
-      mbar_init(bar(BAR_K_EMPTY + s), 1);
-      mbar_init(bar(BAR_V_FULL + s), 1);
-      mbar_init(bar(BAR_V_EMPTY + s), 1);
-      mbar_init(bar(BAR_S_FULL + s), 1);
-      mbar_init(bar(BAR_S_EMPTY + s), 4);
-      mbar_init(bar(BAR_P_FULL + s), 4);
-      mbar_init(bar(BAR_P_EMPTY + s), 1);
+    for (int i = 0; i < kKStages; ++i) {
+      mbar_init(bar(BAR_K_FULL + i), 1);
+      mbar_init(bar(BAR_K_EMPTY + i), 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(bar(BAR_V_FULL + i), 1);
+      mbar_init(bar(BAR_V_EMPTY + i), 1);
+    }
+    for (int i = 0; i < kSBufs; ++i) {
+      mbar_init(bar(BAR_S_FULL + i), 1);
+      mbar_init(bar(BAR_S_EMPTY + i), 4 * kGroups);
+    }
+    for (int i = 0; i < kPBufs; ++i) {
+      mbar_init(bar(BAR_P_FULL + i), 4 * kGroups);
+      mbar_init(bar(BAR_P_EMPTY + i), 1);
     }
     mbar_init(bar(BAR_O_FULL), 1);
-    mbar_init(bar(BAR_O_EMPTY), 4);
+    mbar_init(bar(BAR_O_EMPTY), 4 * kGroups);
     mbar_init(bar(BAR_FINAL), 1);
+    mbar_init(bar(BAR_FINAL2), 1);
     ms->abort = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
   if (D < 128) {
     // the second head-dim chunk of every V stage stays zero: the MMA reads a
     // 128-row V^T, rows d >= D contribute nothing
-    for (int s = 0; s < 2; ++s)
+    for (int s = 0; s < kVStages; ++s)
       for (int i = tid; i < 16384 / 16; i += kThreads)
         reinterpret_cast<uint4*>(smem + kOffV + s * 32768 + 16384)[i] = make_uint4(0u, 0u, 0u, 0u);
     fence_async_smem();
@@ -301,134 +360,154 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     return J < 0 ? 0 : (J >= nb ? nb - 1 : J);
   };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp == 0 || warp == 2) {
+    // ------------------------------------------------------------ TMA producers
+    // warp 0: Q of each item and the K pair tiles; warp 2: the V pair tiles.
+    // Separate producers keep a K load from queueing behind a V slot that only
+    // frees after the (later) second MMA of an older tile.
     if (lane == 0) {
-      uint32_t qit = 0, kit = 0, vit = 0;
+      const bool is_k = warp == 0;
+      uint32_t qit = 0, it_n = 0;
       bool ok = true;
       for (long long it = blockIdx.x; it < items && ok; it += gridDim.x) {
         const int cnt = item_count(it);
         if (cnt == 0) continue;
         const long long bh = it / nb;
         const int I = (int)(it % nb);
-        const int row_q = (int)(bh * a.Npad + (long long)I * kBlock);
-        ok = wait_bar(bar(BAR_Q_EMPTY), (qit & 1u) ^ 1u, abort_flag, 1);
-        if (!ok) break;
-        mbar_expect_tx(bar(BAR_Q_FULL), NCH * kBox);
-        for (int c = 0; c < NCH; ++c) tma_load_2d(sbase + kOffQ + c * kBox, &tmQ, c * 64, row_q, bar(BAR_Q_FULL));
-        ++qit;
+        if (is_k) {
+          const int row_q = (int)(bh * a.Npad + (long long)I * kBlock);
+          ok = wait_bar(bar(BAR_Q_EMPTY), (qit & 1u) ^ 1u, abort_flag, 1);
+          if (!ok) break;
+          mbar_expect_tx(bar(BAR_Q_FULL), NCH * kBox);
+          for (int c = 0; c < NCH; ++c) tma_load_2d(sbase + kOffQ + c * kBox, &tmQ, c * 64, row_q, bar(BAR_Q_FULL));
+          ++qit;
+        }
         const int npairs = (cnt + 1) >> 1;
+        const int stages = is_k ? kKStages : kVStages;
+        const uint32_t full0 = is_k ? BAR_K_FULL : BAR_V_FULL;
+        const uint32_t empty0 = is_k ? BAR_K_EMPTY : BAR_V_EMPTY;
+        const uint32_t region = is_k ? kOffK : kOffV;
+        const CUtensorMap* map = is_k ? &tmK : &tmV;
         for (int t = 0; t < npairs && ok; ++t) {
           const int J1 = item_block(it, 2 * t);
           const int J2 = (2 * t + 1 < cnt) ? item_block(it, 2 * t + 1) : J1;
           const int r1 = (int)(bh * a.Npad + (long long)J1 * kBlock);
           const int r2 = (int)(bh * a.Npad + (long long)J2 * kBlock);
-          const uint32_t ks = kit & 1u;
-          ok = wait_bar(bar(BAR_K_EMPTY + ks), ((kit >> 1) & 1u) ^ 1u, abort_flag, 2);
+          const uint32_t stg = it_n % stages;
+          ok = wait_bar(bar(empty0 + stg), ((it_n / stages) & 1u) ^ 1u, abort_flag, is_k ? 2 : 3);
           if (!ok) break;
-          mbar_expect_tx(bar(BAR_K_FULL + ks), 2 * NCH * kBox);
+          mbar_expect_tx(bar(full0 + stg), 2 * NCH * kBox);
           for (int c = 0; c < NCH; ++c) {
-            const uint32_t dst = sbase + kOffK + ks * 32768 + c * 16384;
-            tma_load_2d(dst, &tmK, c * 64, r1, bar(BAR_K_FULL + ks));
-            tma_load_2d(dst + kBox, &tmK, c * 64, r2, bar(BAR_K_FULL + ks));
+            const uint32_t dst = sbase + region + stg * 32768 + c * 16384;
+            tma_load_2d(dst, map, c * 64, r1, bar(full0 + stg));
+            tma_load_2d(dst + kBox, map, c * 64, r2, bar(full0 + stg));
           }
-          ++kit;
-          const uint32_t vs = vit & 1u;
-          ok = wait_bar(bar(BAR_V_EMPTY + vs), ((vit >> 1) & 1u) ^ 1u, abort_flag, 3);
-          if (!ok) break;
-          mbar_expect_tx(bar(BAR_V_FULL + vs), 2 * NCH * kBox);
-          for (int c = 0; c < NCH; ++c) {
-            const uint32_t dst = sbase + kOffV + vs * 32768 + c * 16384;
-            tma_load_2d(dst, &tmV, c * 64, r1, bar(BAR_V_FULL + vs));
-            tma_load_2d(dst + kBox, &tmV, c * 64, r2, bar(BAR_V_FULL + vs));
-          }
-          ++vit;
+          ++it_n;
         }
       }
-      // never leave with copies in flight: wait (bounded) for the last fill of each ring
+      // never leave with copies in flight: wait (bounded) for the last fill of every stage
       volatile uint32_t no_abort = 0u;
-      if (qit > 0) wait_bar(bar(BAR_Q_FULL), (qit - 1) & 1u, &no_abort, 20);
-      for (uint32_t s = 0; s < 2; ++s) {
-        if (kit > s) wait_bar(bar(BAR_K_FULL + ((kit - 1 - s) & 1u)), ((kit - 1 - s) >> 1) & 1u, &no_abort, 21);
-        if (vit > s) wait_bar(bar(BAR_V_FULL + ((vit - 1 - s) & 1u)), ((vit - 1 - s) >> 1) & 1u, &no_abort, 22);
+      if (is_k && qit > 0) wait_bar(bar(BAR_Q_FULL), (qit - 1) & 1u, &no_abort, 20);
+      const uint32_t stages = is_k ? kKStages : kVStages;
+      for (uint32_t j = 1; j <= stages && j <= it_n; ++j) {
+        const uint32_t n = it_n - j;
+        wait_bar(bar((is_k ? BAR_K_FULL : BAR_V_FULL) + n % stages), (n / stages) & 1u, &no_abort, 21);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 3) {
+    // ------------------------------------------------------------ MMA issuers
+    // Warp 1 issues the first product S^T = K_pair . Q^T of every tile into
+    // the kSBufs-deep S ring (it runs ahead as far as the softmax frees S
+    // buffers); warp 3 issues the second product O^T += V^T . P^T.  Two
+    // issuing threads keep the tensor core fed, and each commits (hence
+    // waits for) only its own MMAs.  Descriptors are base values plus
+    // compile-time offsets (the 14-bit address field never carries).
     if (lane == 0) {
+      const bool first_mma = warp == 1;
       constexpr uint32_t ID_S = idesc_f16(true, false, false);    // bf16 K . Q^T
       constexpr uint32_t ID_O = idesc_f16(false, true, true);     // fp16 V^T . P^T
-      uint32_t qit = 0, kit = 0, vit = 0, sit = 0, pit = 0, oit = 0;
+      const uint64_t dK = sdesc(sbase + kOffK, 16, 1024);
+      const uint64_t dQ = sdesc(sbase + kOffQ, 16, 1024);
+      const uint64_t dV = sdesc(sbase + kOffV, 16384, 1024);
+      const uint64_t dP = sdesc(sbase + kOffP, 16384, 1024);
+      uint32_t ring = 0, tiles = 0, qit = 0, oit = 0;
       bool ok = true;
       for (long long it = blockIdx.x; it < items && ok; it += gridDim.x) {
         const int cnt = item_count(it);
         if (cnt == 0) continue;
         const int npairs = (cnt + 1) >> 1;
-        ok = wait_bar(bar(BAR_Q_FULL), qit & 1u, abort_flag, 4);
-        if (!ok) break;
-        ++qit;
-        for (int t = 0; t <= npairs && ok; ++t) {
-          if (t < npairs) {
-            const uint32_t ks = kit & 1u, sb = sit & 1u;
-            ok = wait_bar(bar(BAR_K_FULL + ks), (kit >> 1) & 1u, abort_flag, 5) &&
-                 wait_bar(bar(BAR_S_EMPTY + sb), ((sit >> 1) & 1u) ^ 1u, abort_flag, 6);
+        if (first_mma) {
+          ok = wait_bar(bar(BAR_Q_FULL), qit & 1u, abort_flag, 4);
+          ++qit;
+          for (int t = 0; t < npairs && ok; ++t) {
+            const uint32_t ks = ring % kKStages, sb = tiles % kSBufs;
+            ok = wait_bar(bar(BAR_K_FULL + ks), (ring / kKStages) & 1u, abort_flag, 5) &&
+                 wait_bar(bar(BAR_S_EMPTY + sb), ((tiles / kSBufs) & 1u) ^ 1u, abort_flag, 6);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t kbase = sbase + kOffK + ks * 32768;
+            const uint64_t a0 = dK + ((ks * 32768u) >> 4);
 #pragma unroll
-            for (int kk = 0; kk < KSTEPS; ++kk) {
-              const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-              const uint32_t qoff = (kk >> 2) * kBox + (kk & 3) * 32;
-              umma_f16(tmem + kColS0 + sb * 64, sdesc(kbase + off, 16, 1024), sdesc(sbase + kOffQ + qoff, 16, 1024),
-                       ID_S, kk > 0 ? 1u : 0u);
-            }
+            for (int kk = 0; kk < KSTEPS; ++kk)
+              umma_f16(tmem + kColS0 + sb * 64, a0 + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                       dQ + (((kk >> 2) * kBox + (kk & 3) * 32) >> 4), ID_S, kk > 0 ? 1u : 0u);
             umma_commit(bar(BAR_K_EMPTY + ks));
             umma_commit(bar(BAR_S_FULL + sb));
-            if (t == npairs - 1) umma_commit(bar(BAR_Q_EMPTY));
-            ++kit;
-            ++sit;
+            ++ring;
+            ++tiles;
           }
-          if (t >= 1) {
-            const int u = t - 1;
-            const uint32_t vs = vit & 1u, pb = pit & 1u;
-            ok = wait_bar(bar(BAR_V_FULL + vs), (vit >> 1) & 1u, abort_flag, 7) &&
-                 wait_bar(bar(BAR_P_FULL + pb), (pit >> 1) & 1u, abort_flag, 8) &&
-                 (u > 0 || wait_bar(bar(BAR_O_EMPTY), (oit & 1u) ^ 1u, abort_flag, 9));
+          if (ok) umma_commit(bar(BAR_Q_EMPTY));
+        } else {
+          for (int t = 0; t < npairs && ok; ++t) {
+            const uint32_t vs = ring % kVStages, pb = tiles % kPBufs;
+            ok = wait_bar(bar(BAR_V_FULL + vs), (ring / kVStages) & 1u, abort_flag, 7) &&
+                 wait_bar(bar(BAR_P_FULL + pb), (tiles / kPBufs) & 1u, abort_flag, 8) &&
+                 (t > 0 || wait_bar(bar(BAR_O_EMPTY), (oit & 1u) ^ 1u, abort_flag, 9));
             if (!ok) break;
             tc_fence_after();
-            const uint32_t vbase = sbase + kOffV + vs * 32768;
-            const uint32_t pbase = sbase + kOffP + pb * 16384;
+            const uint64_t a0 = dV + ((vs * 32768u) >> 4);
+            const uint64_t b0 = dP + ((pb * 16384u) >> 4);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              umma_f16(tmem + kColO, sdesc(vbase + kk * 2048, 16384, 1024), sdesc(pbase + kk * 2048, 16384, 1024),
-                       ID_O, (u > 0 || kk > 0) ? 1u : 0u);
+              umma_f16(tmem + kColO, a0 + ((kk * 2048) >> 4), b0 + ((kk * 2048) >> 4), ID_O,
+                       (t > 0 || kk > 0) ? 1u : 0u);
             umma_commit(bar(BAR_V_EMPTY + vs));
             umma_commit(bar(BAR_P_EMPTY + pb));
-            if (u == npairs - 1) {
-              umma_commit(bar(BAR_O_FULL));
-              ++oit;
-            }
-            ++vit;
-            ++pit;
+            ++ring;
+            ++tiles;
+          }
+          if (ok) {
+            umma_commit(bar(BAR_O_FULL));
+            ++oit;
           }
         }
       }
-      // every issued MMA has finished before TMEM is released
-      umma_commit(bar(BAR_FINAL));
+      // every MMA this thread issued has finished before TMEM is released
+      const uint32_t fin = first_mma ? BAR_FINAL : BAR_FINAL2;
+      umma_commit(bar(fin));
       volatile uint32_t no_abort = 0u;
-      wait_bar(bar(BAR_FINAL), 0u, &no_abort, 23);
+      wait_bar(bar(fin), 0u, &no_abort, 23);
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    // The 128 threads of this group meet at named barrier 1 in lock step.  A
-    // failed wait never makes one thread leave alone: it only sets the abort
-    // flag; the group leaves together after an OR-reduction over that flag.
-    const int sw = warp - 2;                       // 0..3
+    // kGroups warpgroups (warps 4.., four consecutive warps each) split the
+    // 64 query columns of every tile: each covers all 128 TMEM lanes (one key /
+    // head-dim row per thread) for its own kCols columns, with its own running
+    // maxima, rescales and partial sums, so groups never wait for each other.
+    // Inside a group the 128 threads meet at their named barrier in lock
+    // step; a failed wait only sets the abort flag, and the group leaves
+    // together after an OR-reduction over that flag.
+    const int wg = (warp - 4) >> 2;                // warpgroup
+    const int sw = (warp - 4) & 3;                 // warp within the group
     const int quad = warp & 3;                     // TMEM lane quadrant of this warp
     const int k = quad * 32 + lane;                // key row (S^T) / head-dim row (O^T)
-    const int st = tid - 64;                       // 0..127 within the softmax group
+    const int st = sw * 32 + lane;                 // 0..127 within the group
+    const uint32_t gbar = 1u + (uint32_t)wg;       // named barrier of this group
+    const int cb = kCols * wg;                     // first query column of this group
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const float sl2 = a.scale_log2;
+    float* mcol = ms->m + cb;
+    float* acol = ms->alpha + cb;
+    float* fcol = ms->fin + cb;
     uint32_t sit = 0, oit = 0;
     bool stop = false;
     for (long long it = blockIdx.x; it < items && !stop; it += gridDim.x) {
@@ -436,164 +515,158 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const long long bh = it / nb;
       const int I = (int)(it % nb);
       const long long q0 = (long long)I * kBlock;
-      __nv_bfloat16* og = a.o + (bh * a.Npad + q0) * D;
+      __nv_bfloat16* og = a.o + (bh * a.Npad + q0 + cb) * D;       // this group's kCols rows
+      constexpr int CPR = D / 8;
       if (cnt == 0) {
-        for (int i = st; i < kBlock * D / 8; i += kSoftmaxThreads)
+        for (int i = st; i < kCols * CPR; i += kSoftmaxThreads)
           reinterpret_cast<uint4*>(og)[i] = make_uint4(0u, 0u, 0u, 0u);
-        if (a.lse != nullptr && st < 64) a.lse[bh * a.Npad + q0 + st] = 0.f;
+        if (a.lse != nullptr && st < kCols) a.lse[bh * a.Npad + q0 + cb + st] = 0.f;
         continue;
       }
       const int npairs = (cnt + 1) >> 1;
-      if (st < 64) ms->m[st] = -INFINITY;
-      named_bar(1, kSoftmaxThreads);
-      float lp[64];
+      float lp[kCols], mref[kCols];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) lp[c] = 0.f;
+      for (int c = 0; c < kCols; ++c) {
+        lp[c] = 0.f;
+        mref[c] = 0.f;                             // reference maxima; set by the first tile
+      }
+      // this thread's key block for the current pair (prefetched one tile ahead)
+      const int slot = k >> 6;
+      int jcur = (slot < cnt) ? item_block(it, slot) : -1;
 
       for (int t = 0; t < npairs; ++t) {
-        const uint32_t sb = sit & 1u;
-        wait_bar(bar(BAR_S_FULL + sb), (sit >> 1) & 1u, abort_flag, 10);
+        const int jnext = (2 * t + 2 + slot < cnt) ? item_block(it, 2 * t + 2 + slot) : -1;
+        const uint32_t sb = sit % kSBufs, pb = sit % kPBufs;
+        wait_bar(bar(BAR_S_FULL + sb), (sit / kSBufs) & 1u, abort_flag, 10);
         tc_fence_after();
-        float s[64];
-        tmem_ld32(tmem + lane_off + kColS0 + sb * 64, s);
-        tmem_ld32(tmem + lane_off + kColS0 + sb * 64 + 32, s + 32);
+        float y[kCols];
+        tmem_ld_cols<kCols>(tmem + lane_off + kColS0 + sb * 64 + cb, y);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(BAR_S_EMPTY + sb));
 
-        // this thread's key: slot 0 = first block of the pair, 1 = second
-        const int slot = k >> 6;
-        bool valid = 2 * t + slot < cnt;
-        if (valid) {
-          const int J = item_block(it, 2 * t + slot);
-          valid = (long long)J * kBlock + (k & 63) < a.N;
-        }
-        // x = scaled score (log2 domain); excess over the running maximum
+        const bool valid = jcur >= 0 && (long long)jcur * kBlock + (k & 63) < a.N;
+        const bool first = t == 0;
+        // y = scaled score (log2 domain) minus the reference of its column
         float excess = -INFINITY;
+        if (valid) {
 #pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
-          const float4 m4 = reinterpret_cast<const float4*>(ms->m)[c4];
-          const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = 4 * c4 + e;
-            const float x = valid ? s[c] * sl2 : -INFINITY;
-            s[c] = x;
-            excess = fmaxf(excess, x - mm[e]);
+          for (int c = 0; c < kCols; ++c) {
+            y[c] = fmaf(y[c], sl2, -mref[c]);
+            excess = fmaxf(excess, y[c]);
           }
+        } else {
+#pragma unroll
+          for (int c = 0; c < kCols; ++c) y[c] = -INFINITY;
         }
-        if (named_bar_or(1, kSoftmaxThreads, (*abort_flag != 0u) || excess > kLazyTh)) {
-          if (named_bar_or(1, kSoftmaxThreads, *abort_flag != 0u)) {
+        if (named_bar_or(gbar, kSoftmaxThreads, first || (*abort_flag != 0u) || excess > kLazyTh)) {
+          if (named_bar_or(gbar, kSoftmaxThreads, *abort_flag != 0u)) {
             stop = true;
             break;
           }
-          // exact column maxima of this tile, 32 columns at a time
+          // exact column maxima of this tile (in y units), then a new reference
+          {
+            float v[kCols];
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            float v[32];
-#pragma unroll
-            for (int c = 0; c < 32; ++c) v[c] = s[32 * h + c];
-            ms->red[sw][32 * h + lane] = warp_colreduce32<true>(v);
+            for (int c = 0; c < kCols; ++c) v[c] = y[c];
+            const float r = warp_colreduce<true, kCols>(v);
+            if (lane < kCols) ms->red[wg][sw][lane] = r;
           }
-          named_bar(1, kSoftmaxThreads);
-          if (st < 64) {
-            const float tmax = fmaxf(fmaxf(ms->red[0][st], ms->red[1][st]), fmaxf(ms->red[2][st], ms->red[3][st]));
-            const float m_old = ms->m[st];
-            const float m_new = fmaxf(m_old, tmax);
-            ms->m[st] = m_new;
-            ms->alpha[st] = (m_old == -INFINITY) ? 0.f : ex2(m_old - m_new);
+          named_bar(gbar, kSoftmaxThreads);
+          if (st < kCols) {
+            const float ty = fmaxf(fmaxf(ms->red[wg][0][st], ms->red[wg][1][st]),
+                                   fmaxf(ms->red[wg][2][st], ms->red[wg][3][st]));
+            const float m_used = first ? 0.f : mcol[st];
+            const float m_new = first ? ty : fmaxf(mcol[st], ty + m_used);
+            mcol[st] = m_new;
+            acol[st] = first ? 0.f : ex2(m_used - m_new);
+            fcol[st] = m_new - m_used;              // shift to apply to this tile's y
           }
-          named_bar(1, kSoftmaxThreads);
+          named_bar(gbar, kSoftmaxThreads);
 #pragma unroll
-          for (int c = 0; c < 64; ++c) lp[c] *= ms->alpha[c];
-          if (t > 0) {
+          for (int c = 0; c < kCols; ++c) {
+            y[c] -= fcol[c];
+            lp[c] *= acol[c];
+            mref[c] = mcol[c];
+          }
+          if (!first) {
             // O^T holds the previous tiles' sum once their MMA has finished
-            const uint32_t pprev = (sit - 1) & 1u;
-            wait_bar(bar(BAR_P_EMPTY + pprev), ((sit - 1) >> 1) & 1u, abort_flag, 11);
+            const uint32_t pprev = (sit - 1) % kPBufs;
+            wait_bar(bar(BAR_P_EMPTY + pprev), ((sit - 1) / kPBufs) & 1u, abort_flag, 11);
             tc_fence_after();
+            float o[kCols];
+            tmem_ld_cols<kCols>(tmem + lane_off + kColO + cb, o);
+            tmem_wait_ld();
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              float o[32];
-              tmem_ld32(tmem + lane_off + kColO + 32 * h, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int c = 0; c < 32; ++c) o[c] *= ms->alpha[32 * h + c];
-              tmem_st32(tmem + lane_off + kColO + 32 * h, o);
-            }
+            for (int c = 0; c < kCols; ++c) o[c] *= acol[c];
+            tmem_st_cols<kCols>(tmem + lane_off + kColO + cb, o);
             tmem_wait_st();
           }
         }
-        // P^T row k: exp2(x - m), fp16, in the 128-byte swizzled MN-major layout
-        uint32_t pk[32];
+        // P^T row k, this group's columns: exp2(y), fp16, 128-byte swizzled MN-major layout
+        uint32_t pk[kCols / 2];
 #pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
-          const float4 m4 = reinterpret_cast<const float4*>(ms->m)[c4];
-          const float p0 = ex2(s[4 * c4] - m4.x), p1 = ex2(s[4 * c4 + 1] - m4.y);
-          const float p2 = ex2(s[4 * c4 + 2] - m4.z), p3 = ex2(s[4 * c4 + 3] - m4.w);
-          lp[4 * c4] += p0;
-          lp[4 * c4 + 1] += p1;
-          lp[4 * c4 + 2] += p2;
-          lp[4 * c4 + 3] += p3;
-          pk[2 * c4] = pack_f16x2(p0, p1);
-          pk[2 * c4 + 1] = pack_f16x2(p2, p3);
+        for (int c = 0; c < kCols; c += 2) {
+          const float p0 = ex2(y[c]), p1 = ex2(y[c + 1]);
+          lp[c] += p0;
+          lp[c + 1] += p1;
+          pk[c >> 1] = pack_f16x2(p0, p1);
         }
-        wait_bar(bar(BAR_P_EMPTY + sb), ((sit >> 1) & 1u) ^ 1u, abort_flag, 12);
-        unsigned char* prow = smem + kOffP + sb * 16384 + (k >> 3) * 1024 + (k & 7) * 128;
+        wait_bar(bar(BAR_P_EMPTY + pb), ((sit / kPBufs) & 1u) ^ 1u, abort_flag, 12);
+        unsigned char* prow = smem + kOffP + pb * 16384 + (k >> 3) * 1024 + (k & 7) * 128;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int jj = 0; jj < kCols / 8; ++jj) {
+          const int j = cb / 8 + jj;
           *reinterpret_cast<uint4*>(prow + ((j ^ (k & 7)) << 4)) =
-              make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+              make_uint4(pk[4 * jj], pk[4 * jj + 1], pk[4 * jj + 2], pk[4 * jj + 3]);
+        }
         fence_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(BAR_P_FULL + sb));
+        if (lane == 0) mbar_arrive(bar(BAR_P_FULL + pb));
         ++sit;
+        jcur = jnext;
       }
       if (stop) break;
 
-      // ---- epilogue: column sums, normalise O^T, stage as [query][d], store
-#pragma unroll
-      for (int h = 0; h < 2; ++h) ms->red[sw][32 * h + lane] = warp_colreduce32<false>(lp + 32 * h);
-      named_bar(1, kSoftmaxThreads);
-      if (st < 64) {
-        const float l = ms->red[0][st] + ms->red[1][st] + ms->red[2][st] + ms->red[3][st];
-        ms->fin[st] = l > 0.f ? 1.f / l : 0.f;
+      // ---- epilogue: column sums, normalise O^T, store
+      {
+        const float r = warp_colreduce<false, kCols>(lp);
+        if (lane < kCols) ms->red[wg][sw][lane] = r;
+      }
+      named_bar(gbar, kSoftmaxThreads);
+      if (st < kCols) {
+        const float l = ms->red[wg][0][st] + ms->red[wg][1][st] + ms->red[wg][2][st] + ms->red[wg][3][st];
+        fcol[st] = l > 0.f ? 1.f / l : 0.f;
         if (a.lse != nullptr) {
           const float ln2 = 0.6931471805599453f;
-          a.lse[bh * a.Npad + q0 + st] = (q0 + st < a.N && l > 0.f) ? (ms->m[st] + __log2f(l)) * ln2 : 0.f;
+          const long long q = q0 + cb + st;
+          a.lse[bh * a.Npad + q] = (q < a.N && l > 0.f) ? (mcol[st] + __log2f(l)) * ln2 : 0.f;
         }
       }
       wait_bar(bar(BAR_O_FULL), oit & 1u, abort_flag, 13);
       ++oit;
       tc_fence_after();
-      named_bar(1, kSoftmaxThreads);
-      unsigned char* ost = smem + kOffO;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float o[32];
-        tmem_ld32(tmem + lane_off + kColO + 32 * h, o);
+      named_bar(gbar, kSoftmaxThreads);
+      {
+        // thread k holds O^T[k][kCols queries]: row q of O gets element k; a
+        // warp writes 64 contiguous bytes per query row
+        float o[kCols];
+        tmem_ld_cols<kCols>(tmem + lane_off + kColO + cb, o);
         tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(BAR_O_EMPTY));
         if (k < D) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int qc = 32 * h + c;
-            reinterpret_cast<__nv_bfloat16*>(ost)[qc * D + k] = __float2bfloat16_rn(o[c] * ms->fin[qc]);
+          for (int c = 0; c < kCols; ++c) {
+            const bool row_ok = q0 + cb + c < a.N;
+            og[(long long)c * D + k] = __float2bfloat16_rn(row_ok ? o[c] * fcol[c] : 0.f);
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(BAR_O_EMPTY));
-      named_bar(1, kSoftmaxThreads);
-      constexpr int CPR = D / 8;
-      for (int i = st; i < kBlock * CPR; i += kSoftmaxThreads) {
-        const int r = i / CPR;
-        uint4 val = reinterpret_cast<const uint4*>(ost)[i];
-        if (q0 + r >= a.N) val = make_uint4(0u, 0u, 0u, 0u);
-        reinterpret_cast<uint4*>(og)[i] = val;
-      }
-      stop = named_bar_or(1, kSoftmaxThreads, *abort_flag != 0u);
+      stop = named_bar_or(gbar, kSoftmaxThreads, *abort_flag != 0u);
     }
   }
 
