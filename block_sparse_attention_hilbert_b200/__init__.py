@@ -54,6 +54,8 @@ _SIGS = {
     "svsa_perm_workspace_bytes": (ctypes.c_size_t, [Shape, ctypes.c_int32]),
     "svsa_build_perm": (ctypes.c_int, [Shape, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
                                        ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "svsa_build_perm_noalloc": (ctypes.c_int, [Shape, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                                               ctypes.c_void_p]),
     "svsa_reorder": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, Shape,
                                     ctypes.c_void_p]),
     "svsa_reorder_values": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, Shape,
@@ -141,6 +143,12 @@ def svsa_perm_workspace_bytes(s: Shape, order: int) -> int:
 def svsa_build_perm(s: Shape, order: int, perm, iperm, ws=None, ws_bytes: int = 0, stream=None) -> None:
     _check(lib().svsa_build_perm(s, order, _p(perm), _p(iperm), _p(ws), ws_bytes, _stream(stream)),
            "svsa_build_perm")
+
+
+def svsa_build_perm_noalloc(s: Shape, order: int, perm, iperm, stream=None) -> None:
+    """svsa_build_perm with the library's fixed scratch (no allocation; max side 128 for Hilbert)."""
+    _check(lib().svsa_build_perm_noalloc(s, order, _p(perm), _p(iperm), _stream(stream)),
+           "svsa_build_perm_noalloc")
 
 
 def svsa_reorder(x, xp, perm, s: Shape, stream=None) -> None:

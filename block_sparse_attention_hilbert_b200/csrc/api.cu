@@ -16,6 +16,9 @@ cudaError_t launch_build_perm(int T, int H, int W, int hilbert, int32_t* perm, i
                               void* ws, cudaStream_t st);
 size_t perm_workspace_bytes(int T, int H, int W);
 int hilbert_order_bits(int T, int H, int W);
+int perm_noalloc_max_bits();
+size_t perm_noalloc_scratch_bytes();
+cudaError_t perm_noalloc_scratch(void** out);
 cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* map, long long BH,
                                long long rows_dst, long long rows_src, int d, cudaStream_t st);
 cudaError_t launch_gather_rows_f16(const void* src, void* dst, const int32_t* map, long long BH,
@@ -204,6 +207,28 @@ svsa_status svsa_build_perm(svsa_shape s, int32_t order, int32_t* perm, int32_t*
                                                (cudaStream_t)stream),
                              order == SVSA_ORDER_HILBERT ? 5 : 1),
                      "build_perm launch");
+}
+
+svsa_status svsa_build_perm_noalloc(svsa_shape s, int32_t order, int32_t* perm, int32_t* iperm, void* stream) {
+  g_last_error.clear();
+  SVSA_TRY(check_shape(s, false));
+  if (order != SVSA_ORDER_RASTER && order != SVSA_ORDER_HILBERT)
+    return fail(SVSA_ERR_INVALID_ARG, "order=%d unknown", order);
+  SVSA_PTR(perm, "perm");
+  SVSA_PTR(iperm, "iperm");
+  void* scratch = nullptr;
+  if (order == SVSA_ORDER_HILBERT) {
+    if (hilbert_order_bits(s.T, s.H, s.W) > perm_noalloc_max_bits())
+      return fail(SVSA_ERR_UNSUPPORTED,
+                  "no-allocation permutation build supports max(T,H,W) <= %d (got T=%d H=%d W=%d); "
+                  "use svsa_build_perm with a workspace",
+                  1 << perm_noalloc_max_bits(), s.T, s.H, s.W);
+    SVSA_TRY(cuda_status(perm_noalloc_scratch(&scratch), "resolving the static scratch address"));
+  }
+  return cuda_status(counted(launch_build_perm(s.T, s.H, s.W, order == SVSA_ORDER_HILBERT, perm, iperm, scratch,
+                                               (cudaStream_t)stream),
+                             order == SVSA_ORDER_HILBERT ? 5 : 1),
+                     "build_perm_noalloc launch");
 }
 
 svsa_status svsa_reorder(const void* x, void* xp, const int32_t* perm, svsa_shape s, void* stream) {

@@ -10,6 +10,8 @@
 // The sort of the N valid cells by curve index is a rank by bitmap: one bit
 // per cube cell, a per-word prefix count and a per-chunk prefix count give
 // each cell its rank with no comparison sort, deterministically.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace svsa {
@@ -200,6 +202,44 @@ cudaError_t launch_build_perm(int T, int H, int W, int hilbert, int32_t* perm, i
   const int g3 = (int)std::min<long long>((Npad + threads - 1) / threads, kNumSMs * 16LL);
   hilbert_assign_kernel<<<g3, threads, 0, st>>>(T, H, W, k, bits, word_prefix, chunk_prefix, perm, iperm, Npad);
   return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- no-allocation variant
+// Scratch of svsa_build_perm_noalloc, for callers that cannot allocate device
+// memory: one file-scope array per device that loads the library, sized for
+// grids whose longest side is at most 2^kNoAllocMaxBits (128).  Layout as in
+// perm_workspace_bytes: bitmap | word prefix | chunk prefix.
+constexpr int kNoAllocMaxBits = 7;
+constexpr long long kNoAllocWords = (1LL << (3 * kNoAllocMaxBits)) / 32;
+constexpr long long kNoAllocChunks = (kNoAllocWords + kChunkWords - 1) / kChunkWords;
+constexpr size_t kNoAllocScratchBytes = (size_t)(kNoAllocWords * 4 * 2 + kNoAllocChunks * 4 + 256);
+static __device__ __align__(256) unsigned char g_perm_scratch[kNoAllocScratchBytes];
+
+int perm_noalloc_max_bits() { return kNoAllocMaxBits; }
+size_t perm_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+namespace {
+std::mutex g_scratch_mu;
+void* g_scratch_addr[128] = {};   // per device ordinal, resolved once
+}  // namespace
+
+// Device address of g_perm_scratch on the current device.  The first call on
+// a device resolves it (cudaGetSymbolAddress, with that device current); later
+// calls reuse the cached value.
+cudaError_t perm_noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_perm_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
 }
 
 }  // namespace svsa

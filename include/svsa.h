@@ -127,6 +127,31 @@ size_t svsa_perm_workspace_bytes(svsa_shape s, int32_t order);
 svsa_status svsa_build_perm(svsa_shape s, int32_t order, int32_t* perm, int32_t* iperm,
                             void* ws, size_t ws_bytes, void* stream);
 
+/* Permutation build for callers that cannot allocate device memory.
+ * (An addition of this library with no counterpart on the pages.)  Some
+ * callers have no way to provide the scratch svsa_build_perm needs: code that
+ * runs where cudaMalloc is not allowed or not reachable -- a plain-C host
+ * that owns no allocator, or a component whose device memory is entirely
+ * managed by a framework pool it cannot call into.  This variant computes
+ * exactly what svsa_build_perm computes, but its scratch (the Hilbert
+ * bitmap and prefix counts) is a fixed array inside the library, so it
+ * allocates nothing and calls no allocating routine.
+ *   - Limit: Hilbert order needs max(T, H, W) <= 128 (the array holds
+ *     524,800 bytes; every GPU that loads the library keeps it until the
+ *     process exits).  Larger grids return SVSA_ERR_UNSUPPORTED with a
+ *     message; use svsa_build_perm with a workspace for them.  Raster order
+ *     needs no scratch and has no limit.
+ *   - The first call on a device looks up the array's device address once
+ *     (with that device current); make that first call before any stream
+ *     capture.
+ *   - Every call shares the one array: two calls whose kernels overlap on
+ *     the GPU (different streams, no ordering between them) race and may both
+ *     produce wrong permutations.  Order them on one stream or with events.
+ *     The array keeps the last call's contents; each call clears what must
+ *     start at zero itself.
+ * perm, iperm, order, shape and errors are as for svsa_build_perm. */
+svsa_status svsa_build_perm_noalloc(svsa_shape s, int32_t order, int32_t* perm, int32_t* iperm, void* stream);
+
 /* Gather the queries or the keys into the reordered layout:
  *   xp[b, h, i, :] = x[b, h, perm[i], :] for i < Npad (zeros where perm[i] = -1).
  * x: bf16 [B, heads, N, d]; xp: bf16 [B, heads, Npad, d]; perm from
