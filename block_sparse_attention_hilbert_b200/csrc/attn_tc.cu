@@ -123,6 +123,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
   return ok != 0u;
 }
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes (or the hint expires) instead of spinning on the issue slots.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok) : "r"(bar), "r"(parity), "r"(1000000u) : "memory");
+  return ok != 0u;
+}
 __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -141,8 +150,8 @@ __device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, volati
                                            uint32_t where) {
   const unsigned long long t0 = gtimer();
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 0u) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if ((i & 7u) == 0u) {
       if (*abort_flag) return false;
       if (gtimer() - t0 > kWaitNs) {
         atomicCAS(&g_tc_error, 0u, where);
@@ -508,7 +517,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     float* mcol = ms->m + cb;
     float* acol = ms->alpha + cb;
     float* fcol = ms->fin + cb;
-    uint32_t sit = 0, oit = 0;
+    static_assert(kPBufs == 2, "the softmax walks the P ring as a pair");
+    uint32_t sb = 0, sph = 0, pb = 0, pph = 0, oit = 0;      // ring slots and phases
+    // this thread's P^T row (key k) and its swizzled 16-byte chunks for the group's columns
+    unsigned char* const prow0 = smem + kOffP + (k >> 3) * 1024 + (k & 7) * 128;
+    uint32_t pchunk[kCols / 8];
+#pragma unroll
+    for (int jj = 0; jj < kCols / 8; ++jj) pchunk[jj] = (uint32_t)(((cb / 8 + jj) ^ (k & 7)) << 4);
     bool stop = false;
     for (long long it = blockIdx.x; it < items && !stop; it += gridDim.x) {
       const int cnt = item_count(it);
@@ -524,6 +539,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         continue;
       }
       const int npairs = (cnt + 1) >> 1;
+      const int32_t* lst = a.dense ? nullptr : a.kv_idx + it * a.cap;
+      const int n_in_last = (int)(a.N - (long long)(nb - 1) * kBlock);   // valid keys of block nb-1
       float lp[kCols], mref[kCols];
 #pragma unroll
       for (int c = 0; c < kCols; ++c) {
@@ -532,12 +549,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       }
       // this thread's key block for the current pair (prefetched one tile ahead)
       const int slot = k >> 6;
-      int jcur = (slot < cnt) ? item_block(it, slot) : -1;
+      auto block_at = [&](int j) -> int {
+        if (j >= cnt) return -1;
+        if (a.dense) return j;
+        const int J = lst[j];
+        return J < 0 ? 0 : (J >= nb ? nb - 1 : J);
+      };
+      int jcur = block_at(slot);
 
       for (int t = 0; t < npairs; ++t) {
-        const int jnext = (2 * t + 2 + slot < cnt) ? item_block(it, 2 * t + 2 + slot) : -1;
-        const uint32_t sb = sit % kSBufs, pb = sit % kPBufs;
-        wait_bar(bar(BAR_S_FULL + sb), (sit / kSBufs) & 1u, abort_flag, 10);
+        const int jnext = block_at(2 * t + 2 + slot);
+        wait_bar(bar(BAR_S_FULL + sb), sph, abort_flag, 10);
         tc_fence_after();
         float y[kCols];
         tmem_ld_cols<kCols>(tmem + lane_off + kColS0 + sb * 64 + cb, y);
@@ -546,7 +568,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(BAR_S_EMPTY + sb));
 
-        const bool valid = jcur >= 0 && (long long)jcur * kBlock + (k & 63) < a.N;
+        const bool valid = jcur >= 0 && (jcur < nb - 1 || (k & 63) < n_in_last);
         const bool first = t == 0;
         // y = scaled score (log2 domain) minus the reference of its column
         float excess = -INFINITY;
@@ -560,6 +582,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 #pragma unroll
           for (int c = 0; c < kCols; ++c) y[c] = -INFINITY;
         }
+        // exponentials against the current reference before the group vote, so
+        // the wait for the slowest warp overlaps with this warp's MUFU work;
+        // only a rescale tile (rare after the first) recomputes them
+        float pv[kCols];
+#pragma unroll
+        for (int c = 0; c < kCols; ++c) pv[c] = ex2(y[c]);
         if (named_bar_or(gbar, kSoftmaxThreads, first || (*abort_flag != 0u) || excess > kLazyTh)) {
           if (named_bar_or(gbar, kSoftmaxThreads, *abort_flag != 0u)) {
             stop = true;
@@ -589,11 +617,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             y[c] -= fcol[c];
             lp[c] *= acol[c];
             mref[c] = mcol[c];
+            pv[c] = ex2(y[c]);
           }
           if (!first) {
             // O^T holds the previous tiles' sum once their MMA has finished
-            const uint32_t pprev = (sit - 1) % kPBufs;
-            wait_bar(bar(BAR_P_EMPTY + pprev), ((sit - 1) / kPBufs) & 1u, abort_flag, 11);
+            // tile sit-1 used the other P buffer (kPBufs == 2)
+            const uint32_t pprev = pb ^ 1u;
+            wait_bar(bar(BAR_P_EMPTY + pprev), pb == 0u ? pph ^ 1u : pph, abort_flag, 11);
             tc_fence_after();
             float o[kCols];
             tmem_ld_cols<kCols>(tmem + lane_off + kColO + cb, o);
@@ -608,24 +638,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         uint32_t pk[kCols / 2];
 #pragma unroll
         for (int c = 0; c < kCols; c += 2) {
-          const float p0 = ex2(y[c]), p1 = ex2(y[c + 1]);
-          lp[c] += p0;
-          lp[c + 1] += p1;
-          pk[c >> 1] = pack_f16x2(p0, p1);
+          lp[c] += pv[c];
+          lp[c + 1] += pv[c + 1];
+          pk[c >> 1] = pack_f16x2(pv[c], pv[c + 1]);
         }
-        wait_bar(bar(BAR_P_EMPTY + pb), ((sit / kPBufs) & 1u) ^ 1u, abort_flag, 12);
-        unsigned char* prow = smem + kOffP + pb * 16384 + (k >> 3) * 1024 + (k & 7) * 128;
+        wait_bar(bar(BAR_P_EMPTY + pb), pph ^ 1u, abort_flag, 12);
+        unsigned char* prow = prow0 + pb * 16384;
 #pragma unroll
-        for (int jj = 0; jj < kCols / 8; ++jj) {
-          const int j = cb / 8 + jj;
-          *reinterpret_cast<uint4*>(prow + ((j ^ (k & 7)) << 4)) =
+        for (int jj = 0; jj < kCols / 8; ++jj)
+          *reinterpret_cast<uint4*>(prow + pchunk[jj]) =
               make_uint4(pk[4 * jj], pk[4 * jj + 1], pk[4 * jj + 2], pk[4 * jj + 3]);
-        }
         fence_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(BAR_P_FULL + pb));
-        ++sit;
+        // advance the S ring (kSBufs) and the P ring (kPBufs == 2) and their phases
+        if (++sb == (uint32_t)kSBufs) { sb = 0u; sph ^= 1u; }
+        if (++pb == 2u) { pb = 0u; pph ^= 1u; }
         jcur = jnext;
       }
       if (stop) break;
