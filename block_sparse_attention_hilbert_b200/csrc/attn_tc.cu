@@ -51,7 +51,13 @@ namespace tc {
 constexpr int kGroups = SVSA_TC_GROUPS;          // softmax warpgroups; each owns 64 / kGroups query columns
 constexpr int kCols = 64 / kGroups;
 constexpr int kThreads = 32 * (4 + 4 * kGroups);
-constexpr int kKStages = 3, kVStages = 2, kSBufs = 3, kPBufs = 2;
+#ifndef SVSA_TC_KSTAGES
+#define SVSA_TC_KSTAGES 2
+#endif
+#ifndef SVSA_TC_PBUFS
+#define SVSA_TC_PBUFS 3
+#endif
+constexpr int kKStages = SVSA_TC_KSTAGES, kVStages = 2, kSBufs = 3, kPBufs = SVSA_TC_PBUFS;
 constexpr int kSoftmaxThreads = 128;             // one softmax warpgroup
 constexpr uint32_t kBox = 8192;                  // one 64-row x 128-byte TMA box
 constexpr float kLazyTh = 8.0f;                  // log2 headroom before a rescale
@@ -64,6 +70,7 @@ constexpr uint32_t kOffV = kOffK + kKStages * 32768;        // kVStages x 32 KB
 constexpr uint32_t kOffP = kOffV + kVStages * 32768;        // kPBufs x 16 KB
 constexpr uint32_t kOffMisc = kOffP + kPBufs * 16384;
 constexpr uint32_t kSmemBytes = kOffMisc + 2048 + 1024;     // + alignment slack
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 // TMEM columns: three S^T buffers and O^T
 constexpr uint32_t kTmemCols = 256;
@@ -517,7 +524,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     float* mcol = ms->m + cb;
     float* acol = ms->alpha + cb;
     float* fcol = ms->fin + cb;
-    static_assert(kPBufs == 2, "the softmax walks the P ring as a pair");
     uint32_t sb = 0, sph = 0, pb = 0, pph = 0, oit = 0;      // ring slots and phases
     // this thread's P^T row (key k) and its swizzled 16-byte chunks for the group's columns
     unsigned char* const prow0 = smem + kOffP + (k >> 3) * 1024 + (k & 7) * 128;
@@ -621,8 +627,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           }
           if (!first) {
             // O^T holds the previous tiles' sum once their MMA has finished
-            // tile sit-1 used the other P buffer (kPBufs == 2)
-            const uint32_t pprev = pb ^ 1u;
+            // the previous tile used the previous slot of the P ring
+            const uint32_t pprev = pb == 0u ? (uint32_t)kPBufs - 1u : pb - 1u;
             wait_bar(bar(BAR_P_EMPTY + pprev), pb == 0u ? pph ^ 1u : pph, abort_flag, 11);
             tc_fence_after();
             float o[kCols];
@@ -652,9 +658,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(BAR_P_FULL + pb));
-        // advance the S ring (kSBufs) and the P ring (kPBufs == 2) and their phases
+        // advance the S and P rings and their phases
         if (++sb == (uint32_t)kSBufs) { sb = 0u; sph ^= 1u; }
-        if (++pb == 2u) { pb = 0u; pph ^= 1u; }
+        if (++pb == (uint32_t)kPBufs) { pb = 0u; pph ^= 1u; }
         jcur = jnext;
       }
       if (stop) break;
