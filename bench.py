@@ -4,7 +4,7 @@
     python bench.py --impl reference ...      # the fp64 CPU oracle as the reference arm
 
 One step = the whole path over one synthetic layer already resident in HBM:
-svsa_build_perm, svsa_reorder x3 (Q, K, V), svsa_build_mask, svsa_attn_fwd,
+svsa_build_perm, svsa_reorder (Q, K), svsa_reorder_values (V), svsa_build_mask, svsa_attn_fwd,
 svsa_inverse_reorder.  Each timed step is bracketed by CUDA events on the
 launching stream, with an L2 flush (a 512 MiB write) between steps, outside
 the events.  `value` = kept-block attention FLOPs of all ranks / the slowest
@@ -32,7 +32,7 @@ import workloads  # noqa: E402
 
 METRIC = "block-sparse attn fwd ms & kept-FLOP TFLOP/s (% BF16 peak); speedup vs dense"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-ATTN_KERNEL_SRC = os.path.join(ROOT, "block_sparse_attention_hilbert_b200", "csrc", "attn_mma.cu")
+ATTN_KERNEL_SRC = os.path.join(ROOT, "block_sparse_attention_hilbert_b200", "csrc", "attn_tc.cu")
 
 
 def _args():
@@ -170,7 +170,7 @@ def _attn_traffic(workload: str):
     """dram bytes per attention launch from the committed ncu summary, if it was
     taken on the current kernel source (else null)."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", f"attn_{workload}.traffic")
+    path = os.path.join(ROOT, "profiles", f"attn_{workload}.traffic.txt")
     if not os.path.exists(path):
         return None
     kv = {}
