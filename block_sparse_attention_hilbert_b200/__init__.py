@@ -45,7 +45,7 @@ class MaskParams(ctypes.Structure):
 class Mask(ctypes.Structure):
     _fields_ = [("kv_idx", ctypes.c_void_p), ("kv_cnt", ctypes.c_void_p), ("cap", ctypes.c_int32),
                 ("bits", ctypes.c_void_p), ("kbar", ctypes.c_void_p), ("vbar", ctypes.c_void_p),
-                ("nvalid", ctypes.c_void_p)]
+                ("nvalid", ctypes.c_void_p), ("cbar", ctypes.c_void_p)]
 
 
 _lib = None
@@ -128,8 +128,8 @@ def mask_params(select: int = SEL_THRESHOLD, tau: float = 0.9, keep_frac: float 
                       int(routing))
 
 
-def make_mask(kv_idx, kv_cnt, cap: int, bits=None, kbar=None, vbar=None, nvalid=None) -> Mask:
-    return Mask(_p(kv_idx), _p(kv_cnt), cap, _p(bits), _p(kbar), _p(vbar), _p(nvalid))
+def make_mask(kv_idx, kv_cnt, cap: int, bits=None, kbar=None, vbar=None, nvalid=None, cbar=None) -> Mask:
+    return Mask(_p(kv_idx), _p(kv_cnt), cap, _p(bits), _p(kbar), _p(vbar), _p(nvalid), _p(cbar))
 
 
 def version() -> str:

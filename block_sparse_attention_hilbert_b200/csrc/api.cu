@@ -39,13 +39,11 @@ cudaError_t launch_structured(const int32_t* perm, long long rows, int nb, int H
 cudaError_t launch_route(const float* qbar, const void* kp, const void* vp, const float* kbar,
                          const float* vbar, float* R, float* Rm, long long BH, long long N, int nb,
                          int d, cudaStream_t st);
-cudaError_t launch_attn_mma(const void* q, const void* k, const void* v, const int32_t* kv_idx,
-                            const int32_t* kv_cnt, int cap, const float* kbar, const float* vbar,
-                            const int32_t* nvalid, void* o, float* lse, long long BH, long long N,
-                            int nb, int d, bool dense, bool comp, cudaStream_t st);
+cudaError_t launch_centroid16(const float* kbar, const float* vbar, void* cbar, long long rows, int d,
+                              cudaStream_t st);
 cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, const int32_t* kv_idx,
-                           const int32_t* kv_cnt, int cap, void* o, float* lse, long long BH, long long N, int nb,
-                           int d, bool dense, cudaStream_t st);
+                           const int32_t* kv_cnt, int cap, const uint32_t* bits, const void* cbar, void* o,
+                           float* lse, long long BH, long long N, int nb, int d, bool dense, cudaStream_t st);
 cudaError_t attn_tc_error(unsigned int* code, cudaStream_t st);
 }  // namespace svsa
 
@@ -378,16 +376,17 @@ svsa_status svsa_attn_fwd(const void* qp, const void* kp, const void* vp, const 
   if (compensate) {
     SVSA_PTR(m->kbar, "mask.kbar (compensation)");
     SVSA_PTR(m->vbar, "mask.vbar (compensation)");
-    SVSA_PTR(m->nvalid, "mask.nvalid (compensation)");
+    SVSA_PTR(m->bits, "mask.bits (compensation)");
+    SVSA_PTR(m->cbar, "mask.cbar (compensation)");
   }
   if (op == qp || op == kp || op == vp) return fail(SVSA_ERR_INVALID_ARG, "op must not alias an input");
   if (compensate)
-    return cuda_status(counted(launch_attn_mma(qp, kp, vp, m->kv_idx, m->kv_cnt, m->cap, m->kbar, m->vbar,
-                                               m->nvalid, op, lse, g.BH, g.N, g.nb, g.d, false, true,
-                                               (cudaStream_t)stream), 1),
-                       "attn_fwd (compensated) launch");
-  return cuda_status(counted(launch_attn_tc(qp, kp, vp, m->kv_idx, m->kv_cnt, m->cap, op, lse, g.BH, g.N,
-                                            g.nb, g.d, false, (cudaStream_t)stream), 1),
+    SVSA_TRY(cuda_status(counted(launch_centroid16(m->kbar, m->vbar, m->cbar, g.BH * g.nb, g.d,
+                                                   (cudaStream_t)stream), 1),
+                         "centroid copies"));
+  return cuda_status(counted(launch_attn_tc(qp, kp, vp, m->kv_idx, m->kv_cnt, m->cap, compensate ? m->bits : nullptr,
+                                            compensate ? m->cbar : nullptr, op, lse, g.BH, g.N, g.nb, g.d, false,
+                                            (cudaStream_t)stream), 1),
                      "attn_fwd launch");
 }
 
@@ -402,8 +401,8 @@ svsa_status svsa_attn_dense_fwd(const void* qp, const void* kp, const void* vp, 
   SVSA_PTR(op, "op");
   if (lse != nullptr && !aligned16(lse)) return fail(SVSA_ERR_INVALID_ARG, "lse misaligned");
   if (op == qp || op == kp || op == vp) return fail(SVSA_ERR_INVALID_ARG, "op must not alias an input");
-  return cuda_status(counted(launch_attn_tc(qp, kp, vp, nullptr, nullptr, 1, op, lse, g.BH, g.N, g.nb, g.d,
-                                            true, (cudaStream_t)stream), 1),
+  return cuda_status(counted(launch_attn_tc(qp, kp, vp, nullptr, nullptr, 1, nullptr, nullptr, op, lse, g.BH, g.N,
+                                            g.nb, g.d, true, (cudaStream_t)stream), 1),
                      "attn_dense_fwd launch");
 }
 

@@ -27,6 +27,12 @@
 //     current maximum by more than 2^8; otherwise exp2(x - m) is taken against
 //     the stale maximum, which is exact up to the final normalisation.  The
 //     row sums stay per-thread partial sums until the epilogue.
+//   * Compensation ("SVG-EAR" 2.A): after the kept pairs, an item walks
+//     ceil(nb / 128) centroid tiles -- 128 key-block means as keys and value
+//     means as values (16-bit copies of the fp32 means) -- through the same
+//     two products.  The softmax gives centroid row J the bias log2(n_J)
+//     (n_J identical keys) when block J is skipped and -inf when it is kept,
+//     so the skipped blocks enter the same softmax as the exact ones.
 //   * P^T is rounded to fp16 and written to shared memory in the MN-major
 //     128-byte-swizzled layout the second MMA reads; the values arrive as
 //     fp16 (the reordered V), so the second product is fp16 x fp16.  With the
@@ -101,7 +107,10 @@ static_assert(sizeof(Misc) <= 2048, "misc region");
 struct Args {
   const int32_t* kv_idx;
   const int32_t* kv_cnt;
+  const uint32_t* bits;   // kept-block bitmap rows (compensation only)
   int cap;
+  int nwords;             // words per bitmap row
+  int ncent;              // centroid tiles per item (0 = no compensation)
   __nv_bfloat16* o;
   float* lse;
   long long N, Npad;
@@ -304,10 +313,11 @@ __device__ __forceinline__ float warp_colreduce(float* v) {
 }
 
 // ---------------------------------------------------------------- the kernel
-template <int D>
+template <int D, bool COMP>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                               const __grid_constant__ CUtensorMap tmK,
                                                               const __grid_constant__ CUtensorMap tmV,
+                                                              const __grid_constant__ CUtensorMap tmC,
                                                               const Args a) {
   constexpr int NCH = D / 64;                    // 128-byte chunks of the head dim
   constexpr int KSTEPS = D / 16;
@@ -364,6 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   const uint32_t tmem = ms->tmem_base;
   const long long items = a.items;
   const int nb = a.nb;
+  const int ncent = COMP ? a.ncent : 0;          // centroid tiles per item
 
   auto item_count = [&](long long it) -> int {
     if (a.dense) return nb;
@@ -387,7 +398,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       bool ok = true;
       for (long long it = blockIdx.x; it < items && ok; it += gridDim.x) {
         const int cnt = item_count(it);
-        if (cnt == 0) continue;
+        const int npairs = (cnt + 1) >> 1;
+        const int ntiles = npairs + ncent;
+        if (ntiles == 0) continue;
         const long long bh = it / nb;
         const int I = (int)(it % nb);
         if (is_k) {
@@ -398,25 +411,34 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           for (int c = 0; c < NCH; ++c) tma_load_2d(sbase + kOffQ + c * kBox, &tmQ, c * 64, row_q, bar(BAR_Q_FULL));
           ++qit;
         }
-        const int npairs = (cnt + 1) >> 1;
         const int stages = is_k ? kKStages : kVStages;
         const uint32_t full0 = is_k ? BAR_K_FULL : BAR_V_FULL;
         const uint32_t empty0 = is_k ? BAR_K_EMPTY : BAR_V_EMPTY;
         const uint32_t region = is_k ? kOffK : kOffV;
-        const CUtensorMap* map = is_k ? &tmK : &tmV;
-        for (int t = 0; t < npairs && ok; ++t) {
-          const int J1 = item_block(it, 2 * t);
-          const int J2 = (2 * t + 1 < cnt) ? item_block(it, 2 * t + 1) : J1;
-          const int r1 = (int)(bh * a.Npad + (long long)J1 * kBlock);
-          const int r2 = (int)(bh * a.Npad + (long long)J2 * kBlock);
+        for (int t = 0; t < ntiles && ok; ++t) {
+          // kept pairs first, then the centroid tiles (128 block means each;
+          // rows past this head's nb blocks are masked by the softmax)
+          const CUtensorMap* map = is_k ? &tmK : &tmV;
+          int r1, r2, x0 = 0;
+          if (!COMP || t < npairs) {
+            const int J1 = item_block(it, 2 * t);
+            const int J2 = (2 * t + 1 < cnt) ? item_block(it, 2 * t + 1) : J1;
+            r1 = (int)(bh * a.Npad + (long long)J1 * kBlock);
+            r2 = (int)(bh * a.Npad + (long long)J2 * kBlock);
+          } else {
+            map = &tmC;
+            r1 = (int)(bh * nb + (long long)(t - npairs) * 128);
+            r2 = r1 + 64;
+            x0 = is_k ? 0 : D;
+          }
           const uint32_t stg = it_n % stages;
           ok = wait_bar(bar(empty0 + stg), ((it_n / stages) & 1u) ^ 1u, abort_flag, is_k ? 2 : 3);
           if (!ok) break;
           mbar_expect_tx(bar(full0 + stg), 2 * NCH * kBox);
           for (int c = 0; c < NCH; ++c) {
             const uint32_t dst = sbase + region + stg * 32768 + c * 16384;
-            tma_load_2d(dst, map, c * 64, r1, bar(full0 + stg));
-            tma_load_2d(dst + kBox, map, c * 64, r2, bar(full0 + stg));
+            tma_load_2d(dst, map, x0 + c * 64, r1, bar(full0 + stg));
+            tma_load_2d(dst + kBox, map, x0 + c * 64, r2, bar(full0 + stg));
           }
           ++it_n;
         }
@@ -450,8 +472,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       bool ok = true;
       for (long long it = blockIdx.x; it < items && ok; it += gridDim.x) {
         const int cnt = item_count(it);
-        if (cnt == 0) continue;
-        const int npairs = (cnt + 1) >> 1;
+        const int npairs = ((cnt + 1) >> 1) + ncent;       // pair tiles, then centroid tiles
+        if (npairs == 0) continue;
         if (first_mma) {
           ok = wait_bar(bar(BAR_Q_FULL), qit & 1u, abort_flag, 4);
           ++qit;
@@ -538,13 +560,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const long long q0 = (long long)I * kBlock;
       __nv_bfloat16* og = a.o + (bh * a.Npad + q0 + cb) * D;       // this group's kCols rows
       constexpr int CPR = D / 8;
-      if (cnt == 0) {
+      const int npairs = (cnt + 1) >> 1;
+      const int ntiles = npairs + ncent;
+      if (ntiles == 0) {
         for (int i = st; i < kCols * CPR; i += kSoftmaxThreads)
           reinterpret_cast<uint4*>(og)[i] = make_uint4(0u, 0u, 0u, 0u);
         if (a.lse != nullptr && st < kCols) a.lse[bh * a.Npad + q0 + cb + st] = 0.f;
         continue;
       }
-      const int npairs = (cnt + 1) >> 1;
       const int32_t* lst = a.dense ? nullptr : a.kv_idx + it * a.cap;
       const int n_in_last = (int)(a.N - (long long)(nb - 1) * kBlock);   // valid keys of block nb-1
       float lp[kCols], mref[kCols];
@@ -563,8 +586,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       };
       int jcur = block_at(slot);
 
-      for (int t = 0; t < npairs; ++t) {
+      for (int t = 0; t < ntiles; ++t) {
         const int jnext = block_at(2 * t + 2 + slot);
+        // centroid tile: this thread's block J and its kept bit (read before the wait)
+        const bool cent = COMP && t >= npairs;
+        const int Jc = (t - npairs) * 128 + k;
+        uint32_t kept_word = ~0u;
+        if (cent && Jc < nb) kept_word = a.bits[it * a.nwords + (Jc >> 5)];
         wait_bar(bar(BAR_S_FULL + sb), sph, abort_flag, 10);
         tc_fence_after();
         float y[kCols];
@@ -574,14 +602,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(BAR_S_EMPTY + sb));
 
-        const bool valid = jcur >= 0 && (jcur < nb - 1 || (k & 63) < n_in_last);
+        const bool valid = cent ? ((kept_word >> (Jc & 31)) & 1u) == 0u
+                                : jcur >= 0 && (jcur < nb - 1 || (k & 63) < n_in_last);
         const bool first = t == 0;
-        // y = scaled score (log2 domain) minus the reference of its column
+        // y = scaled score (log2 domain) minus the reference of its column; a
+        // skipped block's centroid enters n_J times: + log2(n_J)
         float excess = -INFINITY;
         if (valid) {
+          const float bias = cent ? (Jc == nb - 1 ? __log2f((float)n_in_last) : 6.0f) : 0.f;
 #pragma unroll
           for (int c = 0; c < kCols; ++c) {
-            y[c] = fmaf(y[c], sl2, -mref[c]);
+            y[c] = COMP ? fmaf(y[c], sl2, bias - mref[c]) : fmaf(y[c], sl2, -mref[c]);
             excess = fmaxf(excess, y[c]);
           }
         } else {
@@ -612,7 +643,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const float ty = fmaxf(fmaxf(ms->red[wg][0][st], ms->red[wg][1][st]),
                                    fmaxf(ms->red[wg][2][st], ms->red[wg][3][st]));
             const float m_used = first ? 0.f : mcol[st];
-            const float m_new = first ? ty : fmaxf(mcol[st], ty + m_used);
+            // (a first tile with no valid key keeps the reference at 0)
+            const float m_new = first ? (COMP && ty == -INFINITY ? 0.f : ty) : fmaxf(mcol[st], ty + m_used);
             mcol[st] = m_new;
             acol[st] = first ? 0.f : ex2(m_used - m_new);
             fcol[st] = m_new - m_used;              // shift to apply to this tile's y
@@ -761,33 +793,35 @@ int sm_count() {
 }  // namespace
 
 cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, const int32_t* kv_idx,
-                           const int32_t* kv_cnt, int cap, void* o, float* lse, long long BH, long long N, int nb,
-                           int d, bool dense, cudaStream_t st) {
-  CUtensorMap mq, mk, mv;
+                           const int32_t* kv_cnt, int cap, const uint32_t* bits, const void* cbar, void* o,
+                           float* lse, long long BH, long long N, int nb, int d, bool dense, cudaStream_t st) {
+  CUtensorMap mq, mk, mv, mc;
   const long long rows = BH * (long long)nb * kBlock;
   if (!make_map(&mq, q, rows, d, false) || !make_map(&mk, k, rows, d, false) || !make_map(&mv, v, rows, d, true))
     return cudaErrorInvalidValue;
+  // centroid rows [BH * nb, 2d]: bf16 key means, then fp16 value means (raw 16-bit copies)
+  if (cbar != nullptr ? !make_map(&mc, cbar, BH * (long long)nb, 2 * d, false) : !make_map(&mc, k, rows, d, false))
+    return cudaErrorInvalidValue;
   tc::Args a;
   a.kv_idx = kv_idx; a.kv_cnt = kv_cnt; a.cap = cap;
+  a.bits = bits; a.nwords = (nb + 31) / 32;
+  a.ncent = cbar != nullptr ? (nb + 127) / 128 : 0;
   a.o = (__nv_bfloat16*)o; a.lse = lse;
   a.N = N; a.nb = nb; a.Npad = (long long)nb * kBlock;
   a.items = BH * nb;
   a.scale_log2 = 1.4426950408889634f / sqrtf((float)d);
   a.dense = dense ? 1 : 0;
   const long long grid = std::min<long long>(a.items, sm_count());
-  cudaError_t e;
-  if (d == 128) {
-    e = cudaFuncSetAttribute(tc::attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kSmemBytes);
+  const bool comp = a.ncent > 0;
+  auto go = [&](auto kernel) -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kSmemBytes);
     if (e != cudaSuccess) return e;
-    tc::attn_tc_kernel<128><<<(unsigned)grid, tc::kThreads, tc::kSmemBytes, st>>>(mq, mk, mv, a);
-  } else if (d == 64) {
-    e = cudaFuncSetAttribute(tc::attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    tc::attn_tc_kernel<64><<<(unsigned)grid, tc::kThreads, tc::kSmemBytes, st>>>(mq, mk, mv, a);
-  } else {
-    return cudaErrorInvalidValue;
-  }
-  return cudaGetLastError();
+    kernel<<<(unsigned)grid, tc::kThreads, tc::kSmemBytes, st>>>(mq, mk, mv, mc, a);
+    return cudaGetLastError();
+  };
+  if (d == 128) return comp ? go(tc::attn_tc_kernel<128, true>) : go(tc::attn_tc_kernel<128, false>);
+  if (d == 64) return comp ? go(tc::attn_tc_kernel<64, true>) : go(tc::attn_tc_kernel<64, false>);
+  return cudaErrorInvalidValue;
 }
 
 // Read and clear the device error word (0 = no failure).

@@ -115,4 +115,31 @@ cudaError_t launch_pool_f16(const void* xp, float* out, int32_t* nvalid, long lo
   return launch_pool_t<__half2>(xp, out, nvalid, BH, N, Npad, d, size, st);
 }
 
+// 16-bit centroid rows for the tensor-core compensation: row r of cbar is
+// [kbar_r as bf16 (d) | vbar_r as fp16 (d)], both rounded to nearest even.
+__global__ void centroid16_kernel(const float4* __restrict__ kbar, const float4* __restrict__ vbar,
+                                  uint2* __restrict__ cbar, long long rows, int d4) {
+  const long long total = rows * d4;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long r = i / d4;
+    const int c = (int)(i % d4);
+    const float4 kv = kbar[i], vv = vbar[i];
+    __nv_bfloat162 k01 = __floats2bfloat162_rn(kv.x, kv.y), k23 = __floats2bfloat162_rn(kv.z, kv.w);
+    __half2 v01 = __floats2half2_rn(vv.x, vv.y), v23 = __floats2half2_rn(vv.z, vv.w);
+    cbar[r * 2 * d4 + c] = make_uint2(*reinterpret_cast<uint32_t*>(&k01), *reinterpret_cast<uint32_t*>(&k23));
+    cbar[r * 2 * d4 + d4 + c] = make_uint2(*reinterpret_cast<uint32_t*>(&v01), *reinterpret_cast<uint32_t*>(&v23));
+  }
+}
+
+cudaError_t launch_centroid16(const float* kbar, const float* vbar, void* cbar, long long rows, int d,
+                              cudaStream_t st) {
+  const long long total = rows * (d / 4);
+  const int blocks = (int)std::min<long long>((total + 255) / 256, 148LL * 16);
+  centroid16_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(kbar),
+                                            reinterpret_cast<const float4*>(vbar), reinterpret_cast<uint2*>(cbar),
+                                            rows, d / 4);
+  return cudaGetLastError();
+}
+
 }  // namespace svsa

@@ -27,7 +27,7 @@ class LayerBuffers:
     """Device buffers of one layer shape (all caller-owned, as the ABI requires)."""
 
     def __init__(self, B, heads, T, H, W, d, *, cap, need_means, keep_bits, ws_bytes, perm_ws_bytes,
-                 device):
+                 device, compensate=False):
         N = T * H * W
         nb = -(-N // BLOCK)
         Npad = nb * BLOCK
@@ -42,16 +42,21 @@ class LayerBuffers:
         self.op = torch.empty_like(self.qp)
         self.kv_idx = torch.empty(B, heads, nb, cap, dtype=torch.int32, device=dev)
         self.kv_cnt = torch.empty(B, heads, nb, dtype=torch.int32, device=dev)
-        self.bits = (torch.empty(B, heads, nb, -(-nb // 32), dtype=torch.int32, device=dev)
-                     if keep_bits else None)
         self.kbar = torch.empty(B, heads, nb, d, dtype=torch.float32, device=dev) if need_means else None
         self.vbar = torch.empty_like(self.kbar) if need_means else None
         self.nvalid = torch.empty(nb, dtype=torch.int32, device=dev) if need_means else None
+        # compensation: kept-block bitmap and the 16-bit centroid scratch of the attention
+        if compensate:
+            keep_bits = True
+        self.bits = (torch.empty(B, heads, nb, -(-nb // 32), dtype=torch.int32, device=dev)
+                     if keep_bits else None)
+        self.cbar = torch.empty(B, heads, nb, 2 * d, dtype=torch.int16, device=dev) if compensate else None
         self.ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
         self.cap = cap
 
     def mask(self):
-        return make_mask(self.kv_idx, self.kv_cnt, self.cap, self.bits, self.kbar, self.vbar, self.nvalid)
+        return make_mask(self.kv_idx, self.kv_cnt, self.cap, self.bits, self.kbar, self.vbar, self.nvalid,
+                         self.cbar)
 
 
 class SparseVideoAttention:
@@ -74,7 +79,7 @@ class SparseVideoAttention:
         self.buf = LayerBuffers(B, heads, T, H, W, d, cap=cap, need_means=self.compensate or self.routing,
                                 keep_bits=keep_bits, ws_bytes=svsa_mask_workspace_bytes(self.shape, self.params),
                                 perm_ws_bytes=svsa_perm_workspace_bytes(self.shape, self.order),
-                                device=device)
+                                device=device, compensate=self.compensate)
         self._mask = self.buf.mask()
         self._perm_ready = False
         self.mask_ready = False

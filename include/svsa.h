@@ -107,6 +107,10 @@ typedef struct {
   float* kbar;            /* nullable [B, heads, nb, d] fp32 key block means */
   float* vbar;            /* nullable [B, heads, nb, d] fp32 value block means */
   int32_t* nvalid;        /* nullable [nb] valid (non-pad) tokens per block */
+  void* cbar;             /* nullable [B, heads, nb, 2*d] 16-bit scratch, required by
+                             svsa_attn_fwd(compensate = 1), which first writes each
+                             block's kbar (bf16, first d) and vbar (fp16, last d)
+                             there; 16-byte aligned; not read by svsa_build_mask */
 } svsa_mask;
 
 /* ---- step 1: token order ------------------------------------------------ */
@@ -202,7 +206,10 @@ svsa_status svsa_build_mask(const void* qp, const void* kp, const void* vp, cons
  * computed with an online softmax on the tensor cores (Q.K^T in bf16, P.V in
  * fp16, fp32 statistics and accumulators, P rounded to fp16).  compensate = 1 adds, for every
  * skipped block J, n_J copies of (kbar_J, vbar_J) to the same softmax
- * (SVG-EAR 2.A); that needs m->kbar, m->vbar and m->nvalid.
+ * (SVG-EAR 2.A), n_J = the valid tokens of block J.  That needs m->kbar and
+ * m->vbar (fp32 means, as svsa_build_mask writes them), m->bits (the kept
+ * set; it must agree with kv_idx / kv_cnt) and m->cbar (scratch, overwritten:
+ * the means rounded to bf16 keys / fp16 values for the tensor cores).
  * op: bf16 [B, heads, Npad, d] (pad rows are written as zeros).
  * lse: nullable fp32 [B, heads, Npad]: natural-log sum-exp of each row's
  * scaled scores (0 for pad rows). */

@@ -35,7 +35,7 @@ def test_library_exports_every_declared_symbol():
 def test_struct_sizes_match_header():
     assert ctypes.sizeof(Shape) == 24
     assert ctypes.sizeof(MaskParams) == 36
-    assert ctypes.sizeof(Mask) == 56
+    assert ctypes.sizeof(Mask) == 64
 
 
 def test_version():
@@ -84,11 +84,18 @@ def test_reorder_and_attention_reject_before_launch():
     s = svsa.shape(1, 2, 4, 8, 8, 128)
     assert lib.svsa_reorder(16, 16, 48, s, None) == 1                     # aliasing
     assert lib.svsa_inverse_reorder(None, 32, 48, s, None) == 1
-    m = Mask(None, None, 4, None, None, None, None)
+    m = Mask(None, None, 4, None, None, None, None, None)
     assert lib.svsa_attn_fwd(16, 32, 48, ctypes.byref(m), 0, 64, None, s, None) == 1
-    m = Mask(16, 32, 4, None, None, None, None)
+    m = Mask(16, 32, 4, None, None, None, None, None)
     assert lib.svsa_attn_fwd(16, 32, 48, ctypes.byref(m), 1, 64, None, s, None) == 1   # comp w/o means
     assert "kbar" in _err()
+    kb = 80
+    m = Mask(16, 32, 4, None, kb, kb + 16, None, None)
+    assert lib.svsa_attn_fwd(16, 32, 48, ctypes.byref(m), 1, 64, None, s, None) == 1   # comp w/o bits
+    assert "bits" in _err()
+    m = Mask(16, 32, 4, 96, kb, kb + 16, None, None)
+    assert lib.svsa_attn_fwd(16, 32, 48, ctypes.byref(m), 1, 64, None, s, None) == 1   # comp w/o scratch
+    assert "cbar" in _err()
     assert lib.svsa_attn_dense_fwd(16, 32, 48, 16, None, s, None) == 1    # output aliases input
     assert lib.svsa_attn_fwd(16, 32, 48, None, 0, 64, None, s, None) == 1
 
@@ -96,10 +103,10 @@ def test_reorder_and_attention_reject_before_launch():
 def test_build_mask_rejects_before_launch():
     lib = _raw()
     s = svsa.shape(1, 2, 4, 8, 8, 128)                                    # nb = 4
-    m = Mask(16, 32, 4, None, None, None, None)
+    m = Mask(16, 32, 4, None, None, None, None, None)
     ok = svsa.mask_params(svsa.SEL_THRESHOLD)
     # capacity below nb for a threshold rule
-    small = Mask(16, 32, 3, None, None, None, None)
+    small = Mask(16, 32, 3, None, None, None, None, None)
     assert lib.svsa_build_mask(16, 32, None, None, s, ctypes.byref(ok), ctypes.byref(small), 64, 1 << 20, None) == 1
     # routing without V / means
     r = svsa.mask_params(svsa.SEL_THRESHOLD, routing=True)
