@@ -23,12 +23,12 @@ cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* map, l
                                long long rows_dst, long long rows_src, int d, cudaStream_t st);
 cudaError_t launch_gather_rows_f16(const void* src, void* dst, const int32_t* map, long long BH,
                                    long long rows_dst, long long rows_src, int d, cudaStream_t st);
-cudaError_t launch_pool(const void* xp, float* out, int32_t* nvalid, long long BH, long long N,
+cudaError_t launch_pool(const void* xp, float* out, void* split, int32_t* nvalid, long long BH, long long N,
                         long long Npad, int d, int size, cudaStream_t st);
 cudaError_t launch_pool_f16(const void* xp, float* out, int32_t* nvalid, long long BH, long long N,
                             long long Npad, int d, int size, cudaStream_t st);
 cudaError_t launch_nvalid(int32_t* nvalid, long long N, int nb, cudaStream_t st);
-cudaError_t launch_scores(const float* qs, const float* ks, float* S, long long BH, long long N,
+cudaError_t launch_scores(const void* qsplit, const void* ksplit, float* S, long long BH, long long N,
                           int ng, int nb, int d, int size, cudaStream_t st);
 cudaError_t launch_select(const float* S, const float* R, long long rows, int nb, int mode, float tau,
                           int k, int cap, int32_t* kv_idx, int32_t* kv_cnt, uint32_t* bits,
@@ -45,6 +45,7 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, const in
                            const int32_t* kv_cnt, int cap, const uint32_t* bits, const void* cbar, void* o,
                            float* lse, long long BH, long long N, int nb, int d, bool dense, cudaStream_t st);
 cudaError_t attn_tc_error(unsigned int* code, cudaStream_t st);
+cudaError_t scores_tc_error(unsigned int* code, cudaStream_t st);
 }  // namespace svsa
 
 using namespace svsa;
@@ -111,7 +112,7 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // Workspace layout of svsa_build_mask.
 struct MaskWs {
-  size_t qpool, kpool, S, R, Rm, qbar64, total;
+  size_t qsplit, ksplit, S, R, Rm, qbar64, total;
 };
 
 MaskWs mask_ws_layout(const Dims& g, const svsa_mask_params& p, bool have_kbar) {
@@ -125,15 +126,16 @@ MaskWs mask_ws_layout(const Dims& g, const svsa_mask_params& p, bool have_kbar) 
   }
   const int sub = p.sub_block;
   const long long ng = g.Npad / sub;
-  w.qpool = take((size_t)g.BH * ng * g.d * f);
-  // key pooling can go straight into the caller's kbar when block-level
-  w.kpool = (sub == kBlock && have_kbar) ? SIZE_MAX : take((size_t)g.BH * ng * g.d * f);
+  (void)have_kbar;
+  // pooled Q and K as fp16 hi | lo pairs for the tensor-core scores
+  w.qsplit = take((size_t)g.BH * ng * 2 * g.d * 2);
+  w.ksplit = take((size_t)g.BH * ng * 2 * g.d * 2);
   w.S = take((size_t)g.BH * g.nb * g.nb * f);
   w.R = w.Rm = w.qbar64 = SIZE_MAX;
   if (p.routing) {
     w.R = take((size_t)g.BH * g.nb * g.nb * f);
     w.Rm = take((size_t)g.BH * g.nb * g.nb * f);
-    if (sub != kBlock) w.qbar64 = take((size_t)g.BH * g.nb * g.d * f);
+    w.qbar64 = take((size_t)g.BH * g.nb * g.d * f);      // fp32 query block means
   }
   w.total = off;
   return w;
@@ -318,7 +320,8 @@ svsa_status svsa_build_mask(const void* qp, const void* kp, const void* vp, cons
   // block-level outputs the caller asked for (compensation / routing inputs)
   if (nvalid != nullptr) SVSA_TRY(cuda_status(counted(launch_nvalid(nvalid, g.N, g.nb, st), 1), "nvalid"));
   if (m->kbar != nullptr && (structured || p->sub_block != kBlock))
-    SVSA_TRY(cuda_status(counted(launch_pool(kp, m->kbar, nullptr, g.BH, g.N, g.Npad, g.d, kBlock, st), 1), "pool K"));
+    SVSA_TRY(cuda_status(counted(launch_pool(kp, m->kbar, nullptr, nullptr, g.BH, g.N, g.Npad, g.d, kBlock, st), 1),
+                         "pool K"));
   if (m->vbar != nullptr)
     SVSA_TRY(cuda_status(counted(launch_pool_f16(vp, m->vbar, nullptr, g.BH, g.N, g.Npad, g.d, kBlock, st), 1),
                          "pool V"));
@@ -333,21 +336,25 @@ svsa_status svsa_build_mask(const void* qp, const void* kp, const void* vp, cons
 
   const int sub = p->sub_block;
   const int ng = (int)(g.Npad / sub);
-  float* qpool = at(w.qpool);
-  float* kpool = w.kpool == SIZE_MAX ? m->kbar : at(w.kpool);
+  void* qsplit = base + w.qsplit;
+  void* ksplit = base + w.ksplit;
   float* S = at(w.S);
-  SVSA_TRY(cuda_status(counted(launch_pool(qp, qpool, nullptr, g.BH, g.N, g.Npad, g.d, sub, st), 1), "pool Q"));
-  SVSA_TRY(cuda_status(counted(launch_pool(kp, kpool, nullptr, g.BH, g.N, g.Npad, g.d, sub, st), 1), "pool K"));
-  SVSA_TRY(cuda_status(counted(launch_scores(qpool, kpool, S, g.BH, g.N, ng, g.nb, g.d, sub, st), 1), "scores"));
+  // block-level fp32 means ride along with the split when the rule works on blocks
+  float* qbar = p->routing ? at(w.qbar64) : nullptr;
+  float* kbar_here = (sub == kBlock) ? m->kbar : nullptr;
+  SVSA_TRY(cuda_status(counted(launch_pool(qp, sub == kBlock ? qbar : nullptr, qsplit, nullptr, g.BH, g.N, g.Npad,
+                                           g.d, sub, st), 1),
+                       "pool Q"));
+  SVSA_TRY(cuda_status(counted(launch_pool(kp, kbar_here, ksplit, nullptr, g.BH, g.N, g.Npad, g.d, sub, st), 1),
+                       "pool K"));
+  SVSA_TRY(cuda_status(counted(launch_scores(qsplit, ksplit, S, g.BH, g.N, ng, g.nb, g.d, sub, st), 1), "scores"));
   const float* Rr = nullptr;
   int mode = p->select == SVSA_SEL_TOPK ? 1 : 0;
   if (p->routing) {
-    const float* qbar = qpool;
     if (sub != kBlock) {
-      SVSA_TRY(cuda_status(counted(launch_pool(qp, at(w.qbar64), nullptr, g.BH, g.N, g.Npad, g.d, kBlock,
+      SVSA_TRY(cuda_status(counted(launch_pool(qp, qbar, nullptr, nullptr, g.BH, g.N, g.Npad, g.d, kBlock,
                                                st), 1),
                            "pool Q (blocks)"));
-      qbar = at(w.qbar64);
     }
     SVSA_TRY(cuda_status(counted(launch_route(qbar, kp, vp, m->kbar, m->vbar, at(w.R), at(w.Rm), g.BH,
                                               g.N, g.nb, g.d, st), 1), "route"));
@@ -412,11 +419,15 @@ svsa_status svsa_sync_status(void* stream) {
   if (e != cudaSuccess) return cuda_status(e, "stream synchronize");
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_status(e, "asynchronous error");
-  unsigned int code = 0u;
+  unsigned int code = 0u, code_scores = 0u;
   e = attn_tc_error(&code, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_status(e, "reading the device error word");
+  e = scores_tc_error(&code_scores, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_status(e, "reading the device error word");
   if (code != 0u)
     return fail(SVSA_ERR_TIMEOUT, "attention kernel: a bounded wait gave up (site %u)", code);
+  if (code_scores != 0u)
+    return fail(SVSA_ERR_TIMEOUT, "scores kernel: a bounded wait gave up (site %u)", code_scores);
   return SVSA_OK;
 }
 

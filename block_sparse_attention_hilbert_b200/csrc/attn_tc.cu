@@ -39,13 +39,9 @@
 //     lazy maximum the weights reach 2^8 and the dominant one is no longer
 //     exactly 1, so fp16's 11-bit significand (vs bf16's 8) is what keeps
 //     their rounding well inside the output tolerance.
-#include <cuda.h>
-
 #include <cstddef>
 
-#include <cuda_fp16.h>
-
-#include "common.cuh"
+#include "tcgen05.cuh"
 
 namespace svsa {
 namespace tc {
@@ -67,7 +63,6 @@ constexpr int kKStages = SVSA_TC_KSTAGES, kVStages = 2, kSBufs = 3, kPBufs = SVS
 constexpr int kSoftmaxThreads = 128;             // one softmax warpgroup
 constexpr uint32_t kBox = 8192;                  // one 64-row x 128-byte TMA box
 constexpr float kLazyTh = 8.0f;                  // log2 headroom before a rescale
-constexpr unsigned long long kWaitNs = 2000000000ull;   // 2 s per wait
 
 // shared memory map (offsets from a 1024-byte aligned base)
 constexpr uint32_t kOffQ = 0;                               // 2 x 8 KB (head-dim chunks)
@@ -82,7 +77,6 @@ static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColS0 = 0, kColO = 192;
 
-__device__ unsigned int g_tc_error;              // first failure code, 0 = none
 
 enum : uint32_t {
   BAR_Q_FULL = 0, BAR_Q_EMPTY, BAR_K_FULL, BAR_K_EMPTY = BAR_K_FULL + kKStages,
@@ -119,171 +113,6 @@ struct Args {
   float scale_log2;
   int dense;
 };
-
-// ---------------------------------------------------------------- PTX wrappers
-__device__ __forceinline__ uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-  return ok != 0u;
-}
-// try_wait with a suspend-time hint: the thread sleeps until the phase
-// completes (or the hint expires) instead of spinning on the issue slots.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok) : "r"(bar), "r"(parity), "r"(1000000u) : "memory");
-  return ok != 0u;
-}
-__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-  return ok != 0u;
-}
-__device__ __forceinline__ unsigned long long gtimer() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
-  return t;
-}
-
-// Bounded wait: false on timeout (error word + abort flag set) or abort.
-__device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
-                                           uint32_t where) {
-  const unsigned long long t0 = gtimer();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait_sleep(bar, parity)) return true;
-    if ((i & 7u) == 0u) {
-      if (*abort_flag) return false;
-      if (gtimer() - t0 > kWaitNs) {
-        atomicCAS(&g_tc_error, 0u, where);
-        *abort_flag = 1u;
-        return false;
-      }
-    }
-  }
-}
-
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
-                                         uint32_t where) {
-  return mbar_try_wait(bar, parity) || wait_bar_slow(bar, parity, abort_flag, where);
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n"
-      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar) : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
-
-__device__ __forceinline__ void named_bar(uint32_t id, uint32_t n) {
-  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
-}
-__device__ __forceinline__ bool named_bar_or(uint32_t id, uint32_t n, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
-      : "=r"(r) : "r"((uint32_t)pred), "r"(id), "r"(n) : "memory");
-  return r != 0u;
-}
-
-__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                         uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
-      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
-}
-__device__ __forceinline__ void umma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
-               : "memory");
-}
-
-#define SVSA_R8(i) "=f"(r[i]), "=f"(r[i + 1]), "=f"(r[i + 2]), "=f"(r[i + 3]), "=f"(r[i + 4]), \
-                   "=f"(r[i + 5]), "=f"(r[i + 6]), "=f"(r[i + 7])
-#define SVSA_W8(i) "f"(r[i]), "f"(r[i + 1]), "f"(r[i + 2]), "f"(r[i + 3]), "f"(r[i + 4]), \
-                   "f"(r[i + 5]), "f"(r[i + 6]), "f"(r[i + 7])
-
-// 32 consecutive TMEM columns of this thread's lane (32x32b shape).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* r) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
-      : SVSA_R8(0), SVSA_R8(8), SVSA_R8(16), SVSA_R8(24)
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* r) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n"
-      ::"r"(taddr), SVSA_W8(0), SVSA_W8(8), SVSA_W8(16), SVSA_W8(24)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* r) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
-      : SVSA_R8(0), SVSA_R8(8)
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* r) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n"
-      ::"r"(taddr), SVSA_W8(0), SVSA_W8(8)
-      : "memory");
-}
-template <int NC>
-__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float* r) {
-  if constexpr (NC == 32) tmem_ld32(taddr, r);
-  else tmem_ld16(taddr, r);
-}
-template <int NC>
-__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const float* r) {
-  if constexpr (NC == 32) tmem_st32(taddr, r);
-  else tmem_st16(taddr, r);
-}
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
-
-__device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
-  __half2 v = __floats2half2_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 format, version 1).
-__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-
-// Instruction descriptor, kind::f16 with f32 accumulation, M = 128, N = 64.
-// bf16 = 1 / fp16 = 0 in the A and B format fields (A and B always match).
-constexpr uint32_t idesc_f16(bool bf16, bool a_mn_major, bool b_mn_major) {
-  return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) | ((a_mn_major ? 1u : 0u) << 15) |
-         ((b_mn_major ? 1u : 0u) << 16) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
-}
 
 // Column reduction of v[0..NC-1] across the 32 lanes of a warp: halving
 // exchanges over lane bits log2(NC)-1 .. 0 leave lane l with column l % NC
@@ -750,44 +579,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 // ---------------------------------------------------------------- host side
 namespace {
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
 // 2D view [rows, d] of a 16-bit tensor, 64 x 64 boxes, 128-byte swizzle.
 bool make_map(CUtensorMap* m, const void* base, long long rows, int d, bool f16) {
-  EncodeTiledFn enc = encode_fn();
-  if (enc == nullptr) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-  cuuint32_t box[2] = {64, 64};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-             const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-int sm_count() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = kNumSMs;
-  }
-  return n;
+  return tc::make_map_2d(m, base, rows, d, 64, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
 }
 
 }  // namespace
@@ -811,7 +605,7 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, const in
   a.items = BH * nb;
   a.scale_log2 = 1.4426950408889634f / sqrtf((float)d);
   a.dense = dense ? 1 : 0;
-  const long long grid = std::min<long long>(a.items, sm_count());
+  const long long grid = std::min<long long>(a.items, tc::sm_count());
   const bool comp = a.ncent > 0;
   auto go = [&](auto kernel) -> cudaError_t {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kSmemBytes);
@@ -824,17 +618,7 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, const in
   return cudaErrorInvalidValue;
 }
 
-// Read and clear the device error word (0 = no failure).
-cudaError_t attn_tc_error(unsigned int* code, cudaStream_t st) {
-  unsigned int zero = 0u;
-  cudaError_t e = cudaMemcpyFromSymbolAsync(code, tc::g_tc_error, sizeof(unsigned int), 0,
-                                            cudaMemcpyDeviceToHost, st);
-  if (e != cudaSuccess) return e;
-  e = cudaStreamSynchronize(st);
-  if (e != cudaSuccess) return e;
-  if (*code != 0u) e = cudaMemcpyToSymbolAsync(tc::g_tc_error, &zero, sizeof(unsigned int), 0, cudaMemcpyHostToDevice, st);
-  if (e != cudaSuccess) return e;
-  return cudaStreamSynchronize(st);
-}
+// Read and clear this kernel's device error word (0 = no failure).
+cudaError_t attn_tc_error(unsigned int* code, cudaStream_t st) { return tc::read_error(code, st); }
 
 }  // namespace svsa

@@ -8,6 +8,11 @@
 // or 32 (d=64) row lanes x CPR chunk lanes; each thread keeps fp32 partial
 // sums of its rows per group, and the row lanes are added in a fixed order
 // through shared memory, so the result is deterministic.
+//
+// Optional second output for the tensor-core scores: each mean m as an fp16
+// pair, split[bh, g, :] = [hi (d) | lo (d)] with hi = fp16(m) and
+// lo = fp16(m - hi) (m - hi is exact in fp32), so hi + lo carries m to ~22
+// bits.  Means beyond the fp16 range saturate.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -22,8 +27,8 @@ __device__ __forceinline__ float2 pair_to_float2(const __half2& v) { return __ha
 // T2 = __nv_bfloat162 (queries, keys) or __half2 (values)
 template <int D, int SIZE, typename T2>
 __global__ void __launch_bounds__(kPoolThreads) pool_kernel(
-    const T2* __restrict__ xp, float* __restrict__ out, int32_t* __restrict__ nvalid,
-    long long N, long long Npad) {
+    const T2* __restrict__ xp, float* __restrict__ out, __half* __restrict__ split,
+    int32_t* __restrict__ nvalid, long long N, long long Npad) {
   constexpr int CPR = D / 8;                 // 16-byte chunks per row
   constexpr int RL = kPoolThreads / CPR;     // row lanes
   constexpr int RPT = kBlock / RL;           // rows per thread
@@ -75,7 +80,14 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(
     const long long grow = row0 + (long long)g * SIZE;
     const long long n = std::max<long long>(0, std::min<long long>(SIZE, N - grow));
     const long long gidx = (long long)blk * G + g;
-    out[(bh * (Npad / SIZE) + gidx) * D + c] = n > 0 ? s / (float)n : 0.f;
+    const float mean = n > 0 ? s / (float)n : 0.f;
+    const long long row = bh * (Npad / SIZE) + gidx;
+    if (out != nullptr) out[row * D + c] = mean;
+    if (split != nullptr) {
+      const __half hi = __float2half_rn(fminf(fmaxf(mean, -65504.f), 65504.f));
+      split[row * 2 * D + c] = hi;
+      split[row * 2 * D + D + c] = __float2half_rn(fminf(fmaxf(mean - __half2float(hi), -65504.f), 65504.f));
+    }
     if (nvalid != nullptr && bh == 0 && c == 0) nvalid[gidx] = (int32_t)n;
   }
 }
@@ -91,28 +103,29 @@ cudaError_t launch_nvalid(int32_t* nvalid, long long N, int nb, cudaStream_t st)
 }
 
 template <typename T2>
-static cudaError_t launch_pool_t(const void* xp, float* out, int32_t* nvalid, long long BH, long long N,
+static cudaError_t launch_pool_t(const void* xp, float* out, void* split, int32_t* nvalid, long long BH, long long N,
                                  long long Npad, int d, int size, cudaStream_t st) {
   dim3 grid((unsigned)(Npad / kBlock), (unsigned)BH);
   const T2* x = reinterpret_cast<const T2*>(xp);
-  if (d == 128 && size == 64) pool_kernel<128, 64, T2><<<grid, kPoolThreads, 0, st>>>(x, out, nvalid, N, Npad);
-  else if (d == 128 && size == 16) pool_kernel<128, 16, T2><<<grid, kPoolThreads, 0, st>>>(x, out, nvalid, N, Npad);
-  else if (d == 64 && size == 64) pool_kernel<64, 64, T2><<<grid, kPoolThreads, 0, st>>>(x, out, nvalid, N, Npad);
-  else if (d == 64 && size == 16) pool_kernel<64, 16, T2><<<grid, kPoolThreads, 0, st>>>(x, out, nvalid, N, Npad);
+  __half* sp = reinterpret_cast<__half*>(split);
+  if (d == 128 && size == 64) pool_kernel<128, 64, T2><<<grid, kPoolThreads, 0, st>>>(x, out, sp, nvalid, N, Npad);
+  else if (d == 128 && size == 16) pool_kernel<128, 16, T2><<<grid, kPoolThreads, 0, st>>>(x, out, sp, nvalid, N, Npad);
+  else if (d == 64 && size == 64) pool_kernel<64, 64, T2><<<grid, kPoolThreads, 0, st>>>(x, out, sp, nvalid, N, Npad);
+  else if (d == 64 && size == 16) pool_kernel<64, 16, T2><<<grid, kPoolThreads, 0, st>>>(x, out, sp, nvalid, N, Npad);
   else return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
 
-// bf16 input (queries, keys)
-cudaError_t launch_pool(const void* xp, float* out, int32_t* nvalid, long long BH, long long N,
+// bf16 input (queries, keys); `out` (fp32 means) and `split` (fp16 hi | lo) nullable
+cudaError_t launch_pool(const void* xp, float* out, void* split, int32_t* nvalid, long long BH, long long N,
                         long long Npad, int d, int size, cudaStream_t st) {
-  return launch_pool_t<__nv_bfloat162>(xp, out, nvalid, BH, N, Npad, d, size, st);
+  return launch_pool_t<__nv_bfloat162>(xp, out, split, nvalid, BH, N, Npad, d, size, st);
 }
 
 // fp16 input (reordered values)
 cudaError_t launch_pool_f16(const void* xp, float* out, int32_t* nvalid, long long BH, long long N,
                             long long Npad, int d, int size, cudaStream_t st) {
-  return launch_pool_t<__half2>(xp, out, nvalid, BH, N, Npad, d, size, st);
+  return launch_pool_t<__half2>(xp, out, nullptr, nvalid, BH, N, Npad, d, size, st);
 }
 
 // 16-bit centroid rows for the tensor-core compensation: row r of cbar is

@@ -1,4 +1,4 @@
-// Pooled block scores S[bh, I, J] (fp32), one row per 64-token query block.
+// Pooled block scores S[bh, I, J] (fp32) on the tensor cores.
 //
 // SIZE = 64 ("DFSAttn" trick 2, block averages):
 //   S_IJ = softmax_J(qbar_I . kbar_J / sqrt(d)) over all key blocks.
@@ -7,182 +7,319 @@
 //   S_IJ = (1 / m_I) * sum_{i in I} sum_{j in J} p_ij over the m_I non-empty
 //   query sub-blocks i of I.
 //
-// fp32 SIMT products (the selection needs scores to ~1e-7, far below what a
-// bf16 product gives).  A CTA owns 32 pooled query rows of one head and
-// streams the pooled keys through shared memory in 64-row tiles, twice: pass
-// 1 keeps each row's running max and sum of exponentials, pass 2 recomputes
-// the identical logits, normalises, and (SIZE = 16) adds the 4 x 4 sub-pairs
-// of every block pair with warp shuffles before one store per (I, J).
-#include "common.cuh"
+// The selection needs the scores to ~1e-7, far below what one bf16 or fp16
+// product gives, so each fp32 mean arrives split as fp16 hi + lo (the pooling
+// kernel writes the split) and every logit is the fp32 accumulation of three
+// fp16 products, hi.hi + hi.lo + lo.hi (the dropped lo.lo term and the
+// rounding of lo are ~2^-22 of |q||k|).
+//
+// Work item = 128 pooled query rows of one head (M = 128); the pooled keys
+// stream through in 128-row tiles (N = 128), twice: pass 1 keeps each row's
+// running maximum and sum of exponentials, pass 2 recomputes the identical
+// logits, normalises, and writes S (SIZE = 16: the 4 x 4 sub-pairs of each
+// block pair are added first, columns in-thread and rows by warp shuffles).
+// Warp 0 issues the TMA copies (Q tile once per item, K tiles into a 2-stage
+// ring), warp 1 issues the MMAs into a 2-deep TMEM ring and owns the TMEM
+// allocation, warps 2-5 hold one query row per thread.  Every wait is bounded.
+#include "tcgen05.cuh"
 
 namespace svsa {
+namespace tc {
+namespace scores {
 
-constexpr int kScoreThreads = 256;
-constexpr int kQRows = 32;     // pooled query rows per CTA
-constexpr int kKRows = 64;     // pooled key rows per tile
+constexpr int kThreads = 192;
+constexpr int kRows = 128;                  // pooled query rows per item
+constexpr int kKeys = 128;                  // pooled keys per tile
+constexpr int kKStages = 2, kSBufs = 2;
+constexpr uint32_t kChunk = kRows * 128;    // 128 rows x 64 fp16 (one swizzled column chunk)
+constexpr uint32_t kTmemCols = kSBufs * kKeys;
+
+template <int D>
+struct Smem {
+  static constexpr int NCH = D / 64;
+  static constexpr uint32_t kTile = 2 * NCH * kChunk;          // hi and lo chunks of 128 rows
+  static constexpr uint32_t kOffQ = 0;
+  static constexpr uint32_t kOffK = kTile;
+  static constexpr uint32_t kOffMisc = kOffK + kKStages * kTile;
+  static constexpr uint32_t kBytes = kOffMisc + 256 + 1024;    // + alignment slack
+  static_assert(kBytes <= 232448, "shared memory per CTA");
+};
+
+enum : uint32_t {
+  BAR_Q_FULL = 0, BAR_Q_EMPTY, BAR_K_FULL, BAR_K_EMPTY = BAR_K_FULL + kKStages,
+  BAR_S_FULL = BAR_K_EMPTY + kKStages, BAR_S_EMPTY = BAR_S_FULL + kSBufs, BAR_FINAL = BAR_S_EMPTY + kSBufs,
+  NUM_BARS
+};
+
+struct Misc {
+  uint64_t bar[NUM_BARS];
+  uint32_t tmem_base;
+  uint32_t abort;
+};
+
+struct Args {
+  float* S;
+  long long N;
+  int ng;              // pooled rows per head
+  int nvc;             // non-empty pooled rows per head (the rest are padding)
+  int nb;
+  int nqt, nkt;        // query / key tiles per head
+  long long items;
+  float scale_log2;
+};
 
 template <int D, int SIZE>
-__global__ void __launch_bounds__(kScoreThreads) scores_kernel(
-    const float* __restrict__ qs, const float* __restrict__ ks, float* __restrict__ S,
-    long long N, int ng, int nb, float scale) {
-  constexpr int PER = kBlock / SIZE;          // sub-rows per block (1 or 4)
-  constexpr int LD = D + 4;                   // padded smem row (floats)
-  extern __shared__ float smem[];
-  float* q_s = smem;                          // [kQRows][LD]
-  float* k_s = smem + kQRows * LD;            // [kKRows][LD]
+__global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                                                                const __grid_constant__ CUtensorMap tmK,
+                                                                const Args a) {
+  constexpr int NCH = D / 64;
+  constexpr int KSTEPS = D / 16;
+  using L = Smem<D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  Misc* ms = reinterpret_cast<Misc*>(smem + L::kOffMisc);
+  const uint32_t sbase = su32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  volatile uint32_t* abort_flag = &ms->abort;
+  auto bar = [&](int i) { return su32(&ms->bar[i]); };
 
-  const long long bh = blockIdx.y;
-  const int row0 = blockIdx.x * kQRows;       // first pooled query row
-  const int tid = threadIdx.x;
-  const int tx = tid & 15, ty = tid >> 4;     // 16 x 16 threads; ty pairs of rows, tx columns
-  const float* qb = qs + bh * (long long)ng * D;
-  const float* kb = ks + bh * (long long)ng * D;
-
-  for (int o = tid; o < kQRows * D / 4; o += kScoreThreads) {
-    const int r = o / (D / 4), c = (o % (D / 4)) * 4;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (row0 + r < ng) v = *reinterpret_cast<const float4*>(qb + (long long)(row0 + r) * D + c);
-    *reinterpret_cast<float4*>(q_s + r * LD + c) = v;
+  if (tid == 0) {
+    mbar_init(bar(BAR_Q_FULL), 1);
+    mbar_init(bar(BAR_Q_EMPTY), 1);
+    for (int i = 0; i < kKStages; ++i) {
+      mbar_init(bar(BAR_K_FULL + i), 1);
+      mbar_init(bar(BAR_K_EMPTY + i), 1);
+    }
+    for (int i = 0; i < kSBufs; ++i) {
+      mbar_init(bar(BAR_S_FULL + i), 1);
+      mbar_init(bar(BAR_S_EMPTY + i), 4);
+    }
+    mbar_init(bar(BAR_FINAL), 1);
+    ms->abort = 0u;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(su32(&ms->tmem_base)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ms->tmem_base;
+  const int ntiles = 2 * a.nkt;                   // two passes over the key tiles
 
-  // valid rows: a pooled row is empty when its first position is >= N
-  auto row_ok = [&](int g) { return g < ng && (long long)g * SIZE < N; };
-  const int r_a = row0 + 2 * ty, r_b = r_a + 1;
-  const bool ok_a = row_ok(r_a), ok_b = row_ok(r_b);
-
-  float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
-  const int ntiles = (ng + kKRows - 1) / kKRows;
-
-  for (int pass = 0; pass < 2; ++pass) {
-    for (int kt = 0; kt < ntiles; ++kt) {
-      __syncthreads();
-      for (int o = tid; o < kKRows * D / 4; o += kScoreThreads) {
-        const int r = o / (D / 4), c = (o % (D / 4)) * 4;
-        const int g = kt * kKRows + r;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (g < ng) v = *reinterpret_cast<const float4*>(kb + (long long)g * D + c);
-        *reinterpret_cast<float4*>(k_s + r * LD + c) = v;
-      }
-      __syncthreads();
-      float acc[2][4];
-#pragma unroll
-      for (int i = 0; i < 2; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-      const float* qa = q_s + (2 * ty) * LD;
-      const float* qbp = qa + LD;
-#pragma unroll 4
-      for (int c = 0; c < D; c += 4) {
-        const float4 a0 = *reinterpret_cast<const float4*>(qa + c);
-        const float4 a1 = *reinterpret_cast<const float4*>(qbp + c);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float4 b = *reinterpret_cast<const float4*>(k_s + (tx + 16 * j) * LD + c);
-          acc[0][j] = fmaf(a0.x, b.x, acc[0][j]); acc[0][j] = fmaf(a0.y, b.y, acc[0][j]);
-          acc[0][j] = fmaf(a0.z, b.z, acc[0][j]); acc[0][j] = fmaf(a0.w, b.w, acc[0][j]);
-          acc[1][j] = fmaf(a1.x, b.x, acc[1][j]); acc[1][j] = fmaf(a1.y, b.y, acc[1][j]);
-          acc[1][j] = fmaf(a1.z, b.z, acc[1][j]); acc[1][j] = fmaf(a1.w, b.w, acc[1][j]);
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t qit = 0, kn = 0;
+      bool ok = true;
+      for (long long it = blockIdx.x; it < a.items && ok; it += gridDim.x) {
+        const long long bh = it / a.nqt;
+        const int qt = (int)(it % a.nqt);
+        ok = wait_bar(bar(BAR_Q_EMPTY), (qit & 1u) ^ 1u, abort_flag, 31);
+        if (!ok) break;
+        mbar_expect_tx(bar(BAR_Q_FULL), L::kTile);
+        const int yq = (int)(bh * a.ng + (long long)qt * kRows);
+        for (int c = 0; c < 2 * NCH; ++c) tma_load_2d(sbase + L::kOffQ + c * kChunk, &tmQ, c * 64, yq, bar(BAR_Q_FULL));
+        ++qit;
+        for (int t = 0; t < ntiles && ok; ++t) {
+          const int kt = t % a.nkt;
+          const uint32_t stg = kn % kKStages;
+          ok = wait_bar(bar(BAR_K_EMPTY + stg), ((kn / kKStages) & 1u) ^ 1u, abort_flag, 32);
+          if (!ok) break;
+          mbar_expect_tx(bar(BAR_K_FULL + stg), L::kTile);
+          const int yk = (int)(bh * a.ng + (long long)kt * kKeys);
+          for (int c = 0; c < 2 * NCH; ++c)
+            tma_load_2d(sbase + L::kOffK + stg * L::kTile + c * kChunk, &tmK, c * 64, yk, bar(BAR_K_FULL + stg));
+          ++kn;
         }
       }
-      // scaled logits; empty key rows -> -inf
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int g = kt * kKRows + tx + 16 * j;
-        const bool kok = row_ok(g);
-        acc[0][j] = kok ? acc[0][j] * scale : -INFINITY;
-        acc[1][j] = kok ? acc[1][j] * scale : -INFINITY;
+      // never leave with copies in flight
+      volatile uint32_t no_abort = 0u;
+      if (qit > 0) wait_bar(bar(BAR_Q_FULL), (qit - 1) & 1u, &no_abort, 40);
+      for (uint32_t j = 1; j <= (uint32_t)kKStages && j <= kn; ++j) {
+        const uint32_t n = kn - j;
+        wait_bar(bar(BAR_K_FULL + n % kKStages), (n / kKStages) & 1u, &no_abort, 41);
       }
-      if (pass == 0) {
-        float ta = fmaxf(fmaxf(acc[0][0], acc[0][1]), fmaxf(acc[0][2], acc[0][3]));
-        float tb = fmaxf(fmaxf(acc[1][0], acc[1][1]), fmaxf(acc[1][2], acc[1][3]));
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t ID = idesc_f16(false, false, false, kKeys, kRows);   // fp16, K-major A and B
+      const uint64_t dQ = sdesc(sbase + L::kOffQ, 16, 1024);
+      const uint64_t dK = sdesc(sbase + L::kOffK, 16, 1024);
+      uint32_t qit = 0, kn = 0, sn = 0;
+      bool ok = true;
+      for (long long it = blockIdx.x; it < a.items && ok; it += gridDim.x) {
+        ok = wait_bar(bar(BAR_Q_FULL), qit & 1u, abort_flag, 33);
+        ++qit;
+        for (int t = 0; t < ntiles && ok; ++t) {
+          const uint32_t ks = kn % kKStages, sb = sn % kSBufs;
+          ok = wait_bar(bar(BAR_K_FULL + ks), (kn / kKStages) & 1u, abort_flag, 34) &&
+               wait_bar(bar(BAR_S_EMPTY + sb), ((sn / kSBufs) & 1u) ^ 1u, abort_flag, 35);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t k0 = dK + ((ks * L::kTile) >> 4);
+          // chunk c of the hi part at c * kChunk, of the lo part at (NCH + c) * kChunk
 #pragma unroll
-        for (int o = 8; o > 0; o >>= 1) {
-          ta = fmaxf(ta, __shfl_xor_sync(0xffffffffu, ta, o));
-          tb = fmaxf(tb, __shfl_xor_sync(0xffffffffu, tb, o));
-        }
-        const float na = fmaxf(m_a, ta), nbm = fmaxf(m_b, tb);
-        float sa = 0.f, sb = 0.f;
+          for (int term = 0; term < 3; ++term) {
+            const uint32_t qpart = term == 2 ? NCH : 0;      // hi.hi, hi.lo, lo.hi
+            const uint32_t kpart = term == 1 ? NCH : 0;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          sa += (acc[0][j] == -INFINITY) ? 0.f : expf(acc[0][j] - na);
-          sb += (acc[1][j] == -INFINITY) ? 0.f : expf(acc[1][j] - nbm);
-        }
-#pragma unroll
-        for (int o = 8; o > 0; o >>= 1) {
-          sa += __shfl_xor_sync(0xffffffffu, sa, o);
-          sb += __shfl_xor_sync(0xffffffffu, sb, o);
-        }
-        l_a = (m_a == -INFINITY ? 0.f : l_a * expf(m_a - na)) + sa;
-        l_b = (m_b == -INFINITY ? 0.f : l_b * expf(m_b - nbm)) + sb;
-        m_a = na; m_b = nbm;
-      } else {
-        const float ia = ok_a ? 1.f / l_a : 0.f, ib = ok_b ? 1.f / l_b : 0.f;
-        float p[2][4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          p[0][j] = (ok_a && acc[0][j] != -INFINITY) ? expf(acc[0][j] - m_a) * ia : 0.f;
-          p[1][j] = (ok_b && acc[1][j] != -INFINITY) ? expf(acc[1][j] - m_b) * ib : 0.f;
-        }
-        if constexpr (SIZE == kBlock) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int J = kt * kKRows + tx + 16 * j;
-            if (J < nb) {
-              if (r_a < nb) S[(bh * nb + r_a) * (long long)nb + J] = p[0][j];
-              if (r_b < nb) S[(bh * nb + r_b) * (long long)nb + J] = p[1][j];
+            for (int kk = 0; kk < KSTEPS; ++kk) {
+              const uint32_t off_in = (kk & 3) * 32;
+              umma_f16(tmem + sb * kKeys, dQ + (((qpart + (kk >> 2)) * kChunk + off_in) >> 4),
+                       k0 + (((kpart + (kk >> 2)) * kChunk + off_in) >> 4), ID, (term > 0 || kk > 0) ? 1u : 0u);
             }
           }
-        } else {
-          // rows 2ty, 2ty+1 and the partner half-warp's two rows form one query
-          // block; columns tx..tx^3 (same j) form one key block
-          float v[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            v[j] = p[0][j] + p[1][j];
-            v[j] += __shfl_xor_sync(0xffffffffu, v[j], 1);
-            v[j] += __shfl_xor_sync(0xffffffffu, v[j], 2);
-            v[j] += __shfl_xor_sync(0xffffffffu, v[j], 16);
+          umma_commit(bar(BAR_K_EMPTY + ks));
+          umma_commit(bar(BAR_S_FULL + sb));
+          ++kn;
+          ++sn;
+        }
+        if (ok) umma_commit(bar(BAR_Q_EMPTY));
+      }
+      umma_commit(bar(BAR_FINAL));
+      volatile uint32_t no_abort = 0u;
+      wait_bar(bar(BAR_FINAL), 0u, &no_abort, 42);
+    }
+  } else {
+    // ------------------------------------------------------------ one pooled query row per thread
+    const int quad = warp & 3;                      // TMEM lane quadrant of this warp
+    const int row = quad * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const float sl2 = a.scale_log2;
+    uint32_t sn = 0;
+    bool stop = false;
+    for (long long it = blockIdx.x; it < a.items && !stop; it += gridDim.x) {
+      const long long bh = it / a.nqt;
+      const int qt = (int)(it % a.nqt);
+      const int g = qt * kRows + row;               // pooled query row within the head
+      const bool row_ok = g < a.nvc;
+      float m = -INFINITY, l = 0.f, inv = 0.f;
+      // SIZE = 16: block I = g / 4 and its non-empty sub-row count
+      const int I = g / (kBlock / SIZE);
+      float inv_m = 0.f;
+      if (SIZE != kBlock) {
+        const long long nval = std::max<long long>(0, std::min<long long>(kBlock, a.N - (long long)I * kBlock));
+        const int m_sub = (int)((nval + SIZE - 1) / SIZE);
+        inv_m = m_sub > 0 ? 1.f / (float)m_sub : 0.f;
+      }
+      float* srow = a.S + (bh * a.nb + (I < a.nb ? I : 0)) * (long long)a.nb;
+      for (int t = 0; t < ntiles; ++t) {
+        const uint32_t sb = sn % kSBufs;
+        if (!wait_bar(bar(BAR_S_FULL + sb), (sn / kSBufs) & 1u, abort_flag, 36)) { stop = true; break; }
+        tc_fence_after();
+        const bool pass2 = t >= a.nkt;
+        const int kt = pass2 ? t - a.nkt : t;
+        const int c0 = kt * kKeys;
+        if (pass2 && t == a.nkt) inv = (row_ok && l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll 1
+        for (int ch = 0; ch < kKeys / 32; ++ch) {
+          float x[32];
+          tmem_ld32(tmem + lane_off + sb * kKeys + ch * 32, x);
+          tmem_wait_ld();
+          if (ch == kKeys / 32 - 1) {
+            // the whole S tile is in registers: hand the buffer back
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(BAR_S_EMPTY + sb));
           }
-          // number of non-empty sub-rows of this query block
-          const int I = (row0 + 2 * ty) / PER;
-          const long long first = (long long)I * kBlock;
-          const long long nval = std::max<long long>(0, std::min<long long>(kBlock, N - first));
-          const int m_sub = (int)((nval + SIZE - 1) / SIZE);
-          if ((tx & 3) == 0 && (ty & 1) == 0 && I < nb && m_sub > 0) {
-            const float inv = 1.f / (float)m_sub;
+          const int cb = c0 + ch * 32;              // first pooled key of this chunk
+          const int nvalid = a.nvc - cb;            // keys >= nvc are padding
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int J = (kt * kKRows + tx + 16 * j) / PER;
-              if (J < nb) S[(bh * nb + I) * (long long)nb + J] = v[j] * inv;
+          for (int c = 0; c < 32; ++c) x[c] = c < nvalid ? x[c] * sl2 : -INFINITY;
+          if (!pass2) {
+            float cm = x[0];
+#pragma unroll
+            for (int c = 1; c < 32; ++c) cm = fmaxf(cm, x[c]);
+            const float mn = fmaxf(m, cm);
+            if (mn > -INFINITY) {
+              float sum = 0.f;
+#pragma unroll
+              for (int c = 0; c < 32; ++c) sum += ex2(x[c] - mn);
+              l = (m == -INFINITY ? 0.f : l * ex2(m - mn)) + sum;
+              m = mn;
+            }
+          } else if (SIZE == kBlock) {
+            if (row_ok && I < a.nb) {
+#pragma unroll
+              for (int c = 0; c < 32; ++c) {
+                const float p = ex2(x[c] - m) * inv;
+                if (cb + c < a.nb) srow[cb + c] = p;
+              }
+            }
+          } else {
+            // 8 key blocks of 4 sub-columns each; then the 4 sub-rows of the block (lanes 4i .. 4i+3)
+            float v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              v[j] = 0.f;
+#pragma unroll
+              for (int u = 0; u < 4; ++u) v[j] += ex2(x[4 * j + u] - m);
+              v[j] *= inv;
+              v[j] += __shfl_xor_sync(0xffffffffu, v[j], 1);
+              v[j] += __shfl_xor_sync(0xffffffffu, v[j], 2);
+            }
+            const int q = lane & 3;
+            const int J0 = cb / 4 + 2 * q;
+            if (I < a.nb) {
+              const float w0 = q == 0 ? v[0] : q == 1 ? v[2] : q == 2 ? v[4] : v[6];
+              const float w1 = q == 0 ? v[1] : q == 1 ? v[3] : q == 2 ? v[5] : v[7];
+              if (J0 < a.nb) srow[J0] = w0 * inv_m;
+              if (J0 + 1 < a.nb) srow[J0 + 1] = w1 * inv_m;
             }
           }
         }
+        ++sn;
       }
     }
   }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kTmemCols));
+  }
 }
 
-size_t scores_smem_bytes(int d) { return (size_t)(kQRows + kKRows) * (d + 4) * sizeof(float); }
+}  // namespace scores
+}  // namespace tc
 
-cudaError_t launch_scores(const float* qs, const float* ks, float* S, long long BH, long long N,
-                          int ng, int nb, int d, int size, cudaStream_t st) {
-  dim3 grid((unsigned)((ng + kQRows - 1) / kQRows), (unsigned)BH);
-  const size_t smem = scores_smem_bytes(d);
-  const float scale = 1.0f / sqrtf((float)d);
-#define SVSA_SCORES(DD, SS)                                                                      \
-  do {                                                                                           \
-    cudaError_t e = cudaFuncSetAttribute(scores_kernel<DD, SS>,                                  \
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
-    if (e != cudaSuccess) return e;                                                              \
-    scores_kernel<DD, SS><<<grid, kScoreThreads, smem, st>>>(qs, ks, S, N, ng, nb, scale);       \
-  } while (0)
-  if (d == 128 && size == 64) SVSA_SCORES(128, 64);
-  else if (d == 128 && size == 16) SVSA_SCORES(128, 16);
-  else if (d == 64 && size == 64) SVSA_SCORES(64, 64);
-  else if (d == 64 && size == 16) SVSA_SCORES(64, 16);
-  else return cudaErrorInvalidValue;
-#undef SVSA_SCORES
-  return cudaGetLastError();
+// qsplit, ksplit: fp16 [BH, ng, 2d] (hi | lo of each pooled row), ng = Npad / size.
+cudaError_t launch_scores(const void* qsplit, const void* ksplit, float* S, long long BH, long long N, int ng,
+                          int nb, int d, int size, cudaStream_t st) {
+  using namespace tc::scores;
+  CUtensorMap mq, mk;
+  if (!tc::make_map_2d(&mq, qsplit, BH * ng, 2 * d, kRows, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+      !tc::make_map_2d(&mk, ksplit, BH * ng, 2 * d, kKeys, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+    return cudaErrorInvalidValue;
+  Args a;
+  a.S = S;
+  a.N = N;
+  a.ng = ng;
+  a.nvc = (int)std::min<long long>(ng, (N + size - 1) / size);
+  a.nb = nb;
+  a.nqt = (ng + kRows - 1) / kRows;
+  a.nkt = (ng + kKeys - 1) / kKeys;
+  a.items = BH * a.nqt;
+  a.scale_log2 = 1.4426950408889634f / sqrtf((float)d);
+  const long long grid = std::min<long long>(a.items, tc::sm_count());
+  auto go = [&](auto kernel, uint32_t smem) -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kernel<<<(unsigned)grid, kThreads, smem, st>>>(mq, mk, a);
+    return cudaGetLastError();
+  };
+  if (d == 128 && size == 64) return go(scores_tc_kernel<128, 64>, Smem<128>::kBytes);
+  if (d == 128 && size == 16) return go(scores_tc_kernel<128, 16>, Smem<128>::kBytes);
+  if (d == 64 && size == 64) return go(scores_tc_kernel<64, 64>, Smem<64>::kBytes);
+  if (d == 64 && size == 16) return go(scores_tc_kernel<64, 16>, Smem<64>::kBytes);
+  return cudaErrorInvalidValue;
 }
+
+cudaError_t scores_tc_error(unsigned int* code, cudaStream_t st) { return tc::read_error(code, st); }
 
 }  // namespace svsa
