@@ -23,12 +23,12 @@ cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* map, l
                                long long rows_dst, long long rows_src, int d, cudaStream_t st);
 cudaError_t launch_gather_rows_f16(const void* src, void* dst, const int32_t* map, long long BH,
                                    long long rows_dst, long long rows_src, int d, cudaStream_t st);
-cudaError_t launch_pool(const void* xp, float* out, void* split, int32_t* nvalid, long long BH, long long N,
-                        long long Npad, int d, int size, cudaStream_t st);
+cudaError_t launch_pool(const void* xp, float* out, void* split, void* split_bf, int32_t* nvalid, long long BH,
+                        long long N, long long Npad, int d, int size, cudaStream_t st);
 cudaError_t launch_pool_f16(const void* xp, float* out, int32_t* nvalid, long long BH, long long N,
                             long long Npad, int d, int size, cudaStream_t st);
 cudaError_t launch_nvalid(int32_t* nvalid, long long N, int nb, cudaStream_t st);
-cudaError_t launch_scores(const void* qsplit, const void* ksplit, float* S, long long BH, long long N,
+cudaError_t launch_scores(const void* qsplit, const void* ksplit, float* S, float* L, long long BH, long long N,
                           int ng, int nb, int d, int size, cudaStream_t st);
 cudaError_t launch_select(const float* S, const float* R, long long rows, int nb, int mode, float tau,
                           int k, int cap, int32_t* kv_idx, int32_t* kv_cnt, uint32_t* bits,
@@ -36,9 +36,11 @@ cudaError_t launch_select(const float* S, const float* R, long long rows, int nb
 cudaError_t launch_structured(const int32_t* perm, long long rows, int nb, int H, int W, int win_t,
                               int R, int n_anchors, int anchor_offset, int cap, int32_t* kv_idx,
                               int32_t* kv_cnt, uint32_t* bits, cudaStream_t st);
-cudaError_t launch_route(const float* qbar, const void* kp, const void* vp, const float* kbar,
-                         const float* vbar, float* R, float* Rm, long long BH, long long N, int nb,
+int route_nsplit(int nb);
+cudaError_t launch_route(const void* qsplit_bf, const void* kp, const void* vp, const float* L, const float* vbar,
+                         float* R, float* Rm, float* Mp, float* Zp, int nsplit, long long BH, long long N, int nb,
                          int d, cudaStream_t st);
+cudaError_t route_tc_error(unsigned int* code, cudaStream_t st);
 cudaError_t launch_centroid16(const float* kbar, const float* vbar, void* cbar, long long rows, int d,
                               cudaStream_t st);
 cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, const int32_t* kv_idx,
@@ -112,7 +114,7 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // Workspace layout of svsa_build_mask.
 struct MaskWs {
-  size_t qsplit, ksplit, S, R, Rm, qbar64, total;
+  size_t qsplit, ksplit, S, R, Rm, qbf, L, Mp, Zp, q64, k64, total;
 };
 
 MaskWs mask_ws_layout(const Dims& g, const svsa_mask_params& p, bool have_kbar) {
@@ -131,11 +133,20 @@ MaskWs mask_ws_layout(const Dims& g, const svsa_mask_params& p, bool have_kbar) 
   w.qsplit = take((size_t)g.BH * ng * 2 * g.d * 2);
   w.ksplit = take((size_t)g.BH * ng * 2 * g.d * 2);
   w.S = take((size_t)g.BH * g.nb * g.nb * f);
-  w.R = w.Rm = w.qbar64 = SIZE_MAX;
+  w.R = w.Rm = w.qbf = w.L = w.Mp = w.Zp = w.q64 = w.k64 = SIZE_MAX;
   if (p.routing) {
-    w.R = take((size_t)g.BH * g.nb * g.nb * f);
-    w.Rm = take((size_t)g.BH * g.nb * g.nb * f);
-    w.qbar64 = take((size_t)g.BH * g.nb * g.d * f);      // fp32 query block means
+    const size_t nn = (size_t)g.BH * g.nb * g.nb * f;
+    const size_t part = (size_t)g.BH * g.nb * route_nsplit(g.nb) * f;
+    w.R = take(nn);
+    w.Rm = take(nn);
+    w.L = take(nn);                                        // centroid logits
+    w.Mp = take(part);
+    w.Zp = take(part);
+    w.qbf = take((size_t)g.BH * g.nb * 2 * g.d * 2);       // query block means, bf16 hi | lo
+    if (sub != kBlock) {                                   // block-level splits for the centroid logits
+      w.q64 = take((size_t)g.BH * g.nb * 2 * g.d * 2);
+      w.k64 = take((size_t)g.BH * g.nb * 2 * g.d * 2);
+    }
   }
   w.total = off;
   return w;
@@ -320,7 +331,7 @@ svsa_status svsa_build_mask(const void* qp, const void* kp, const void* vp, cons
   // block-level outputs the caller asked for (compensation / routing inputs)
   if (nvalid != nullptr) SVSA_TRY(cuda_status(counted(launch_nvalid(nvalid, g.N, g.nb, st), 1), "nvalid"));
   if (m->kbar != nullptr && (structured || p->sub_block != kBlock))
-    SVSA_TRY(cuda_status(counted(launch_pool(kp, m->kbar, nullptr, nullptr, g.BH, g.N, g.Npad, g.d, kBlock, st), 1),
+    SVSA_TRY(cuda_status(counted(launch_pool(kp, m->kbar, nullptr, nullptr, nullptr, g.BH, g.N, g.Npad, g.d, kBlock, st), 1),
                          "pool K"));
   if (m->vbar != nullptr)
     SVSA_TRY(cuda_status(counted(launch_pool_f16(vp, m->vbar, nullptr, g.BH, g.N, g.Npad, g.d, kBlock, st), 1),
@@ -339,25 +350,36 @@ svsa_status svsa_build_mask(const void* qp, const void* kp, const void* vp, cons
   void* qsplit = base + w.qsplit;
   void* ksplit = base + w.ksplit;
   float* S = at(w.S);
-  // block-level fp32 means ride along with the split when the rule works on blocks
-  float* qbar = p->routing ? at(w.qbar64) : nullptr;
-  float* kbar_here = (sub == kBlock) ? m->kbar : nullptr;
-  SVSA_TRY(cuda_status(counted(launch_pool(qp, sub == kBlock ? qbar : nullptr, qsplit, nullptr, g.BH, g.N, g.Npad,
-                                           g.d, sub, st), 1),
+  // the routing proxies (bf16 split of the query block means) ride along when the rule works on blocks
+  void* qbf = p->routing ? base + w.qbf : nullptr;
+  float* L = p->routing ? at(w.L) : nullptr;
+  SVSA_TRY(cuda_status(counted(launch_pool(qp, nullptr, qsplit, sub == kBlock ? qbf : nullptr, nullptr, g.BH, g.N,
+                                           g.Npad, g.d, sub, st), 1),
                        "pool Q"));
-  SVSA_TRY(cuda_status(counted(launch_pool(kp, kbar_here, ksplit, nullptr, g.BH, g.N, g.Npad, g.d, sub, st), 1),
+  SVSA_TRY(cuda_status(counted(launch_pool(kp, sub == kBlock ? m->kbar : nullptr, ksplit, nullptr, nullptr, g.BH,
+                                           g.N, g.Npad, g.d, sub, st), 1),
                        "pool K"));
-  SVSA_TRY(cuda_status(counted(launch_scores(qsplit, ksplit, S, g.BH, g.N, ng, g.nb, g.d, sub, st), 1), "scores"));
+  SVSA_TRY(cuda_status(counted(launch_scores(qsplit, ksplit, S, sub == kBlock ? L : nullptr, g.BH, g.N, ng, g.nb,
+                                             g.d, sub, st), 1),
+                       "scores"));
   const float* Rr = nullptr;
   int mode = p->select == SVSA_SEL_TOPK ? 1 : 0;
   if (p->routing) {
     if (sub != kBlock) {
-      SVSA_TRY(cuda_status(counted(launch_pool(qp, qbar, nullptr, nullptr, g.BH, g.N, g.Npad, g.d, kBlock,
-                                               st), 1),
+      // block-level means for the proxies and the centroid logits
+      SVSA_TRY(cuda_status(counted(launch_pool(qp, nullptr, base + w.q64, qbf, nullptr, g.BH, g.N, g.Npad, g.d,
+                                               kBlock, st), 1),
                            "pool Q (blocks)"));
+      SVSA_TRY(cuda_status(counted(launch_pool(kp, nullptr, base + w.k64, nullptr, nullptr, g.BH, g.N, g.Npad, g.d,
+                                               kBlock, st), 1),
+                           "pool K (blocks)"));
+      SVSA_TRY(cuda_status(counted(launch_scores(base + w.q64, base + w.k64, nullptr, L, g.BH, g.N, g.nb, g.nb, g.d,
+                                                 kBlock, st), 1),
+                           "centroid logits"));
     }
-    SVSA_TRY(cuda_status(counted(launch_route(qbar, kp, vp, m->kbar, m->vbar, at(w.R), at(w.Rm), g.BH,
-                                              g.N, g.nb, g.d, st), 1), "route"));
+    SVSA_TRY(cuda_status(counted(launch_route(qbf, kp, vp, L, m->vbar, at(w.R), at(w.Rm), at(w.Mp), at(w.Zp),
+                                              route_nsplit(g.nb), g.BH, g.N, g.nb, g.d, st), 2),
+                         "route"));
     Rr = at(w.R);
     mode = 3;
   }
@@ -419,15 +441,22 @@ svsa_status svsa_sync_status(void* stream) {
   if (e != cudaSuccess) return cuda_status(e, "stream synchronize");
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_status(e, "asynchronous error");
-  unsigned int code = 0u, code_scores = 0u;
-  e = attn_tc_error(&code, (cudaStream_t)stream);
-  if (e != cudaSuccess) return cuda_status(e, "reading the device error word");
-  e = scores_tc_error(&code_scores, (cudaStream_t)stream);
-  if (e != cudaSuccess) return cuda_status(e, "reading the device error word");
-  if (code != 0u)
-    return fail(SVSA_ERR_TIMEOUT, "attention kernel: a bounded wait gave up (site %u)", code);
-  if (code_scores != 0u)
-    return fail(SVSA_ERR_TIMEOUT, "scores kernel: a bounded wait gave up (site %u)", code_scores);
+  // every tensor-core translation unit keeps its own error word; read (and clear) all of them
+  cudaError_t (*readers[3])(unsigned int*, cudaStream_t) = {attn_tc_error, scores_tc_error, route_tc_error};
+  const char* names[3] = {"attention", "scores", "routing"};
+  unsigned int first_code = 0u;
+  const char* first_name = nullptr;
+  for (int i = 0; i < 3; ++i) {
+    unsigned int code = 0u;
+    e = readers[i](&code, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_status(e, "reading the device error word");
+    if (code != 0u && first_name == nullptr) {
+      first_code = code;
+      first_name = names[i];
+    }
+  }
+  if (first_name != nullptr)
+    return fail(SVSA_ERR_TIMEOUT, "%s kernel: a bounded wait gave up (site %u)", first_name, first_code);
   return SVSA_OK;
 }
 

@@ -12,7 +12,9 @@
 // Optional second output for the tensor-core scores: each mean m as an fp16
 // pair, split[bh, g, :] = [hi (d) | lo (d)] with hi = fp16(m) and
 // lo = fp16(m - hi) (m - hi is exact in fp32), so hi + lo carries m to ~22
-// bits.  Means beyond the fp16 range saturate.
+// bits.  Means beyond the fp16 range saturate.  A third optional output holds
+// the same split in bf16 (hi = bf16(m), lo = bf16(m - hi): ~16 bits, fp32
+// range) for products against raw bf16 keys.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -28,7 +30,7 @@ __device__ __forceinline__ float2 pair_to_float2(const __half2& v) { return __ha
 template <int D, int SIZE, typename T2>
 __global__ void __launch_bounds__(kPoolThreads) pool_kernel(
     const T2* __restrict__ xp, float* __restrict__ out, __half* __restrict__ split,
-    int32_t* __restrict__ nvalid, long long N, long long Npad) {
+    __nv_bfloat16* __restrict__ split_bf, int32_t* __restrict__ nvalid, long long N, long long Npad) {
   constexpr int CPR = D / 8;                 // 16-byte chunks per row
   constexpr int RL = kPoolThreads / CPR;     // row lanes
   constexpr int RPT = kBlock / RL;           // rows per thread
@@ -88,6 +90,11 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(
       split[row * 2 * D + c] = hi;
       split[row * 2 * D + D + c] = __float2half_rn(fminf(fmaxf(mean - __half2float(hi), -65504.f), 65504.f));
     }
+    if (split_bf != nullptr) {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(mean);
+      split_bf[row * 2 * D + c] = hi;
+      split_bf[row * 2 * D + D + c] = __float2bfloat16_rn(mean - __bfloat162float(hi));
+    }
     if (nvalid != nullptr && bh == 0 && c == 0) nvalid[gidx] = (int32_t)n;
   }
 }
@@ -103,29 +110,33 @@ cudaError_t launch_nvalid(int32_t* nvalid, long long N, int nb, cudaStream_t st)
 }
 
 template <typename T2>
-static cudaError_t launch_pool_t(const void* xp, float* out, void* split, int32_t* nvalid, long long BH, long long N,
-                                 long long Npad, int d, int size, cudaStream_t st) {
+static cudaError_t launch_pool_t(const void* xp, float* out, void* split, void* split_bf, int32_t* nvalid,
+                                 long long BH, long long N, long long Npad, int d, int size, cudaStream_t st) {
   dim3 grid((unsigned)(Npad / kBlock), (unsigned)BH);
   const T2* x = reinterpret_cast<const T2*>(xp);
   __half* sp = reinterpret_cast<__half*>(split);
-  if (d == 128 && size == 64) pool_kernel<128, 64, T2><<<grid, kPoolThreads, 0, st>>>(x, out, sp, nvalid, N, Npad);
-  else if (d == 128 && size == 16) pool_kernel<128, 16, T2><<<grid, kPoolThreads, 0, st>>>(x, out, sp, nvalid, N, Npad);
-  else if (d == 64 && size == 64) pool_kernel<64, 64, T2><<<grid, kPoolThreads, 0, st>>>(x, out, sp, nvalid, N, Npad);
-  else if (d == 64 && size == 16) pool_kernel<64, 16, T2><<<grid, kPoolThreads, 0, st>>>(x, out, sp, nvalid, N, Npad);
+  __nv_bfloat16* sb = reinterpret_cast<__nv_bfloat16*>(split_bf);
+#define SVSA_POOL(DD, SS) pool_kernel<DD, SS, T2><<<grid, kPoolThreads, 0, st>>>(x, out, sp, sb, nvalid, N, Npad)
+  if (d == 128 && size == 64) SVSA_POOL(128, 64);
+  else if (d == 128 && size == 16) SVSA_POOL(128, 16);
+  else if (d == 64 && size == 64) SVSA_POOL(64, 64);
+  else if (d == 64 && size == 16) SVSA_POOL(64, 16);
   else return cudaErrorInvalidValue;
+#undef SVSA_POOL
   return cudaGetLastError();
 }
 
-// bf16 input (queries, keys); `out` (fp32 means) and `split` (fp16 hi | lo) nullable
-cudaError_t launch_pool(const void* xp, float* out, void* split, int32_t* nvalid, long long BH, long long N,
-                        long long Npad, int d, int size, cudaStream_t st) {
-  return launch_pool_t<__nv_bfloat162>(xp, out, split, nvalid, BH, N, Npad, d, size, st);
+// bf16 input (queries, keys); `out` (fp32 means), `split` (fp16 hi | lo) and
+// `split_bf` (bf16 hi | lo) are each nullable
+cudaError_t launch_pool(const void* xp, float* out, void* split, void* split_bf, int32_t* nvalid, long long BH,
+                        long long N, long long Npad, int d, int size, cudaStream_t st) {
+  return launch_pool_t<__nv_bfloat162>(xp, out, split, split_bf, nvalid, BH, N, Npad, d, size, st);
 }
 
 // fp16 input (reordered values)
 cudaError_t launch_pool_f16(const void* xp, float* out, int32_t* nvalid, long long BH, long long N,
                             long long Npad, int d, int size, cudaStream_t st) {
-  return launch_pool_t<__half2>(xp, out, nullptr, nvalid, BH, N, Npad, d, size, st);
+  return launch_pool_t<__half2>(xp, out, nullptr, nullptr, nvalid, BH, N, Npad, d, size, st);
 }
 
 // 16-bit centroid rows for the tensor-core compensation: row r of cbar is

@@ -1,4 +1,5 @@
-// Error-aware routing ratios ("SVG-EAR", technical summary 2.B).
+// Error-aware routing ratios ("SVG-EAR", technical summary 2.B) on the tensor
+// cores.
 //
 // The query centroid qbar_I stands in for the queries of block I.  With
 // s_j = qbar_I . k_j / sqrt(d) over all valid keys, M = max_j s_j and
@@ -8,142 +9,436 @@
 // replaced by their means) and the routed ratio is r_IJ = e_IJ / Z * 64 / n_J
 // (error per unit of block size).
 //
-// One CTA owns 16 query blocks of one head and streams the key/value blocks
-// once (O(C_q N_k d) work, as the page states).  The running maximum grows as
-// tiles arrive, so each e_IJ is first taken against the maximum m_J known at
-// tile J and stored with m_J; a final sweep turns it into
-// e * exp(m_J - M) / Z * 64 / n_J.  fp32 throughout.
-#include <cuda_fp16.h>
-
-#include "common.cuh"
+// Work item = 128 proxies (query blocks) of one head and a contiguous range
+// of key blocks.  Per key block J (one 64-key tile):
+//   S [128 x 64]  = Qbar . K_J^T   qbar split as bf16 hi + lo against the exact
+//                                   bf16 keys (two MMA passes, ~16-bit qbar);
+//   E = 2^(S log2e - m)             m = the proxy's running maximum, E <= 1;
+//   O [128 x d]   = E . V_J         E split as fp16 hi + lo against the fp16
+//                                   values (two MMA passes, ~22-bit weights);
+//   e_IJ(m)       = || O_I - n_J 2^(L_IJ - m) vbar_J ||, stored with m,
+// where L_IJ is the log2-domain centroid logit from the scores kernel.  The
+// running maximum only grows, so each e_IJ is exact for the m it was taken
+// against; per item the proxies' (m, Z) partials are stored and a fix-up
+// kernel combines the key ranges and rescales: r_IJ = e_IJ 2^(m_IJ - M) / Z
+// * 64 / n_J.
+//
+// Warp 0 issues the TMA copies (qbar tile per item; K_J and V_J per tile into
+// a 2-stage ring), warp 1 issues the MMAs (S of tile t+1 ahead of the E.V of
+// tile t) and owns TMEM, warps 2-5 hold one proxy per thread: exponentials,
+// the E split into shared memory, and the error epilogue of the previous
+// tile while the tensor core works on the next one.  Every wait is bounded.
+#include "tcgen05.cuh"
 
 namespace svsa {
+namespace tc {
+namespace route {
 
-constexpr int kRouteThreads = 256;
-constexpr int kRouteRows = 16;
+constexpr int kThreads = 192;
+constexpr int kRows = 128;                   // proxies per item
+constexpr int kStages = 2, kSBufs = 2, kEBufs = 2, kOBufs = 2;
+constexpr uint32_t kBoxQ = kRows * 128;      // 128 rows x 64 bf16 (16 KB)
+constexpr uint32_t kBoxK = kBlock * 128;     // 64 rows x 64 elements (8 KB)
+constexpr uint32_t kEPart = kRows * 128;     // E hi or lo: 128 proxies x 64 fp16 (16 KB)
 
 template <int D>
-__global__ void __launch_bounds__(kRouteThreads) route_kernel(
-    const float* __restrict__ qbar, const __nv_bfloat16* __restrict__ kp,
-    const __half* __restrict__ vp, const float* __restrict__ kbar,
-    const float* __restrict__ vbar, float* __restrict__ R, float* __restrict__ Rm, long long N, int nb,
-    float scale) {
-  constexpr int CH = D / 16;                          // channels per thread in the value phase
-  __shared__ float q_s[kRouteRows][D];
-  __shared__ __nv_bfloat16 k_s[kBlock][D + 8];
-  __shared__ __half v_s[kBlock][D];
-  __shared__ float e_s[kRouteRows][kBlock];
-  __shared__ float m_s[kRouteRows], z_s[kRouteRows];
+struct Smem {
+  static constexpr int NCH = D / 64;
+  static constexpr uint32_t kQ = 2 * NCH * kBoxQ;          // qbar hi and lo
+  static constexpr uint32_t kStage = 2 * NCH * kBoxK;      // K_J then V_J
+  static constexpr uint32_t kOffQ = 0;
+  static constexpr uint32_t kOffKV = kQ;
+  static constexpr uint32_t kOffE = kOffKV + kStages * kStage;
+  static constexpr uint32_t kOffMisc = kOffE + kEBufs * 2 * kEPart;
+  static constexpr uint32_t kBytes = kOffMisc + 512 + 1024;
+  static_assert(kBytes <= 232448, "shared memory per CTA");
+  // TMEM: S buffers (64 columns each), then O buffers (D columns each)
+  static constexpr uint32_t kColS = 0, kColO = kSBufs * 64;
+  static constexpr uint32_t kCols = kColO + kOBufs * D <= 256 ? 256 : 512;
+};
 
-  const long long bh = blockIdx.y;
-  const int I0 = blockIdx.x * kRouteRows;
-  const int tid = threadIdx.x;
-  const int row = tid >> 4, sub = tid & 15;           // 16 threads per proxy row
-  const long long Npad = (long long)nb * kBlock;
+enum : uint32_t {
+  BAR_Q_FULL = 0, BAR_Q_EMPTY, BAR_KV_FULL, BAR_KV_EMPTY = BAR_KV_FULL + kStages,
+  BAR_S_FULL = BAR_KV_EMPTY + kStages, BAR_S_EMPTY = BAR_S_FULL + kSBufs,
+  BAR_E_FULL = BAR_S_EMPTY + kSBufs, BAR_E_EMPTY = BAR_E_FULL + kEBufs,
+  BAR_O_FULL = BAR_E_EMPTY + kEBufs, BAR_O_EMPTY = BAR_O_FULL + kOBufs, BAR_FINAL = BAR_O_EMPTY + kOBufs,
+  NUM_BARS
+};
 
-  for (int o = tid; o < kRouteRows * D; o += kRouteThreads) {
-    const int r = o / D, c = o % D;
-    q_s[r][c] = (I0 + r < nb) ? qbar[(bh * nb + I0 + r) * (long long)D + c] : 0.f;
+struct Misc {
+  uint64_t bar[NUM_BARS];
+  uint32_t tmem_base;
+  uint32_t abort;
+};
+
+struct Args {
+  const float* L;       // [BH, nb, nb] centroid logits, log2 domain
+  const float* vbar;    // [BH, nb, d]
+  float* R;             // [BH, nb, nb] e_IJ against m_IJ
+  float* Rm;            // [BH, nb, nb] m_IJ (log2 domain)
+  float* Mp;            // [BH, nb, nsplit] partial maxima
+  float* Zp;            // [BH, nb, nsplit] partial sums against Mp
+  long long N, Npad;
+  int nb, nqt, nsplit, per;   // proxy tiles per head, key ranges, key blocks per range
+  long long items;
+  float scale_log2;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                                                               const __grid_constant__ CUtensorMap tmK,
+                                                               const __grid_constant__ CUtensorMap tmV,
+                                                               const Args a) {
+  constexpr int NCH = D / 64;
+  constexpr int KSTEPS = D / 16;
+  using L = Smem<D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  Misc* ms = reinterpret_cast<Misc*>(smem + L::kOffMisc);
+  const uint32_t sbase = su32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  volatile uint32_t* abort_flag = &ms->abort;
+  auto bar = [&](int i) { return su32(&ms->bar[i]); };
+
+  if (tid == 0) {
+    mbar_init(bar(BAR_Q_FULL), 1);
+    mbar_init(bar(BAR_Q_EMPTY), 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(bar(BAR_KV_FULL + i), 1);
+      mbar_init(bar(BAR_KV_EMPTY + i), 1);
+    }
+    for (int i = 0; i < kSBufs; ++i) {
+      mbar_init(bar(BAR_S_FULL + i), 1);
+      mbar_init(bar(BAR_S_EMPTY + i), 4);
+    }
+    for (int i = 0; i < kEBufs; ++i) {
+      mbar_init(bar(BAR_E_FULL + i), 4);
+      mbar_init(bar(BAR_E_EMPTY + i), 1);
+    }
+    for (int i = 0; i < kOBufs; ++i) {
+      mbar_init(bar(BAR_O_FULL + i), 1);
+      mbar_init(bar(BAR_O_EMPTY + i), 4);
+    }
+    mbar_init(bar(BAR_FINAL), 1);
+    ms->abort = 0u;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
-  if (tid < kRouteRows) { m_s[tid] = -INFINITY; z_s[tid] = 0.f; }
-  const bool row_ok = I0 + row < nb;
-  float* rrow = R + (bh * nb + (row_ok ? I0 + row : 0)) * (long long)nb;
-  float* mrow = Rm + (bh * nb + (row_ok ? I0 + row : 0)) * (long long)nb;
-
-  for (int J = 0; J < nb; ++J) {
-    __syncthreads();
-    const __nv_bfloat16* kb = kp + (bh * Npad + (long long)J * kBlock) * D;
-    const __half* vb = vp + (bh * Npad + (long long)J * kBlock) * D;
-    for (int o = tid; o < kBlock * D / 8; o += kRouteThreads) {
-      const int r = o / (D / 8), c = (o % (D / 8)) * 8;
-      const uint4 kv = *reinterpret_cast<const uint4*>(kb + (long long)r * D + c);
-      const uint4 vv = *reinterpret_cast<const uint4*>(vb + (long long)r * D + c);
-      *reinterpret_cast<uint4*>(&k_s[r][c]) = kv;
-      *reinterpret_cast<uint4*>(&v_s[r][c]) = vv;
-    }
-    __syncthreads();
-    const long long key0 = (long long)J * kBlock;
-    const int nJ = (int)std::max<long long>(0, std::min<long long>(kBlock, N - key0));
-    // logits: row `row`, keys sub + 16*u
-    float s[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) s[u] = 0.f;
-    for (int c = 0; c < D; ++c) {
-      const float q = q_s[row][c];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) s[u] = fmaf(q, __bfloat162float(k_s[sub + 16 * u][c]), s[u]);
-    }
-    float tmax = -INFINITY;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      s[u] = (sub + 16 * u < nJ) ? s[u] * scale : -INFINITY;
-      tmax = fmaxf(tmax, s[u]);
-    }
-#pragma unroll
-    for (int o = 8; o > 0; o >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
-    const float m_old = m_s[row];
-    const float m_new = fmaxf(m_old, tmax);
-    float zs = 0.f;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float e = s[u] == -INFINITY ? 0.f : expf(s[u] - m_new);
-      e_s[row][sub + 16 * u] = e;
-      zs += e;
-    }
-#pragma unroll
-    for (int o = 8; o > 0; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
-    __syncwarp();
-    // centroid logit qbar_I . kbar_J (fp32 mean of block J)
-    const float* kbJ = kbar + (bh * nb + J) * (long long)D;
-    const float* vbJ = vbar + (bh * nb + J) * (long long)D;
-    float lc = 0.f;
-#pragma unroll
-    for (int u = 0; u < CH; ++u) lc = fmaf(q_s[row][sub * CH + u], kbJ[sub * CH + u], lc);
-#pragma unroll
-    for (int o = 8; o > 0; o >>= 1) lc += __shfl_xor_sync(0xffffffffu, lc, o);
-    const float cw = nJ > 0 ? (float)nJ * expf(lc * scale - m_new) : 0.f;
-    __syncthreads();                                  // e_s complete
-    // exact weighted value sum minus centroid term, channels sub*CH .. +CH
-    float err2 = 0.f;
-#pragma unroll
-    for (int u = 0; u < CH; ++u) {
-      const int c = sub * CH + u;
-      float a = 0.f;
-#pragma unroll 8
-      for (int j = 0; j < kBlock; ++j) a = fmaf(e_s[row][j], __half2float(v_s[j][c]), a);
-      const float diff = a - cw * vbJ[c];
-      err2 = fmaf(diff, diff, err2);
-    }
-#pragma unroll
-    for (int o = 8; o > 0; o >>= 1) err2 += __shfl_xor_sync(0xffffffffu, err2, o);
-    if (sub == 0) {
-      m_s[row] = m_new;
-      z_s[row] = (m_old == -INFINITY ? 0.f : z_s[row] * expf(m_old - m_new)) + zs;
-      if (row_ok) { rrow[J] = sqrtf(err2); mrow[J] = m_new; }
-    }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(su32(&ms->tmem_base)),
+                 "r"(L::kCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::);
   }
+  tc_fence_before();
   __syncthreads();
-  if (!row_ok) return;
-  const float M = m_s[row], Z = z_s[row];
-  for (int J = sub; J < nb; J += 16) {
-    const long long key0 = (long long)J * kBlock;
-    const int nJ = (int)std::max<long long>(1, std::min<long long>(kBlock, N - key0));
-    const float e = rrow[J];
-    rrow[J] = e > 0.f ? e * expf(mrow[J] - M) / Z * ((float)kBlock / (float)nJ) : 0.f;
+  tc_fence_after();
+  const uint32_t tmem = ms->tmem_base;
+  const int nb = a.nb;
+  // item -> (head, proxy tile, key range)
+  auto decode = [&](long long it, long long& bh, int& qt, int& j0, int& j1) {
+    const int sp = (int)(it % a.nsplit);
+    const long long r = it / a.nsplit;
+    qt = (int)(r % a.nqt);
+    bh = r / a.nqt;
+    j0 = sp * a.per;
+    j1 = min(nb, j0 + a.per);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t qit = 0, kn = 0;
+      bool ok = true;
+      for (long long it = blockIdx.x; it < a.items && ok; it += gridDim.x) {
+        long long bh;
+        int qt, j0, j1;
+        decode(it, bh, qt, j0, j1);
+        if (j0 >= j1) continue;
+        ok = wait_bar(bar(BAR_Q_EMPTY), (qit & 1u) ^ 1u, abort_flag, 51);
+        if (!ok) break;
+        mbar_expect_tx(bar(BAR_Q_FULL), L::kQ);
+        const int yq = (int)(bh * nb + (long long)qt * kRows);
+        for (int c = 0; c < 2 * NCH; ++c) tma_load_2d(sbase + L::kOffQ + c * kBoxQ, &tmQ, c * 64, yq, bar(BAR_Q_FULL));
+        ++qit;
+        for (int J = j0; J < j1 && ok; ++J) {
+          const uint32_t stg = kn % kStages;
+          ok = wait_bar(bar(BAR_KV_EMPTY + stg), ((kn / kStages) & 1u) ^ 1u, abort_flag, 52);
+          if (!ok) break;
+          mbar_expect_tx(bar(BAR_KV_FULL + stg), L::kStage);
+          const int yk = (int)(bh * a.Npad + (long long)J * kBlock);
+          const uint32_t dst = sbase + L::kOffKV + stg * L::kStage;
+          for (int c = 0; c < NCH; ++c) {
+            tma_load_2d(dst + c * kBoxK, &tmK, c * 64, yk, bar(BAR_KV_FULL + stg));
+            tma_load_2d(dst + (NCH + c) * kBoxK, &tmV, c * 64, yk, bar(BAR_KV_FULL + stg));
+          }
+          ++kn;
+        }
+      }
+      volatile uint32_t no_abort = 0u;
+      if (qit > 0) wait_bar(bar(BAR_Q_FULL), (qit - 1) & 1u, &no_abort, 60);
+      for (uint32_t j = 1; j <= (uint32_t)kStages && j <= kn; ++j) {
+        const uint32_t n = kn - j;
+        wait_bar(bar(BAR_KV_FULL + n % kStages), (n / kStages) & 1u, &no_abort, 61);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t ID_S = idesc_f16(true, false, false, 64, kRows);     // bf16 Qbar . K^T
+      constexpr uint32_t ID_O = idesc_f16(false, false, true, D, kRows);      // fp16 E . V (V MN-major)
+      const uint64_t dQ = sdesc(sbase + L::kOffQ, 16, 1024);
+      const uint64_t dKV = sdesc(sbase + L::kOffKV, 16, 1024);
+      const uint64_t dVm = sdesc(sbase + L::kOffKV + NCH * kBoxK, kBoxK, 1024);
+      const uint64_t dE = sdesc(sbase + L::kOffE, 16, 1024);
+      uint32_t qit = 0, kn = 0, pn = 0;     // K/V ring position of the next S, of the next E.V
+      bool ok = true;
+      auto issue_s = [&](uint32_t n) -> bool {
+        const uint32_t stg = n % kStages, sb = n % kSBufs;
+        if (!wait_bar(bar(BAR_KV_FULL + stg), (n / kStages) & 1u, abort_flag, 53) ||
+            !wait_bar(bar(BAR_S_EMPTY + sb), ((n / kSBufs) & 1u) ^ 1u, abort_flag, 54))
+          return false;
+        tc_fence_after();
+        const uint64_t k0 = dKV + ((stg * L::kStage) >> 4);
+#pragma unroll
+        for (int part = 0; part < 2; ++part)
+#pragma unroll
+          for (int kk = 0; kk < KSTEPS; ++kk)
+            umma_f16(tmem + L::kColS + sb * 64, dQ + ((((part * NCH) + (kk >> 2)) * kBoxQ + (kk & 3) * 32) >> 4),
+                     k0 + ((((kk >> 2)) * kBoxK + (kk & 3) * 32) >> 4), ID_S, (part > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(bar(BAR_S_FULL + sb));
+        return true;
+      };
+      auto issue_o = [&](uint32_t n) -> bool {
+        const uint32_t stg = n % kStages, eb = n % kEBufs, ob = n % kOBufs;
+        if (!wait_bar(bar(BAR_E_FULL + eb), (n / kEBufs) & 1u, abort_flag, 55) ||
+            !wait_bar(bar(BAR_O_EMPTY + ob), ((n / kOBufs) & 1u) ^ 1u, abort_flag, 56))
+          return false;
+        tc_fence_after();
+        const uint64_t v0 = dVm + ((stg * L::kStage) >> 4);
+        const uint64_t e0 = dE + ((eb * 2 * kEPart) >> 4);
+#pragma unroll
+        for (int part = 0; part < 2; ++part)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_f16(tmem + L::kColO + ob * D, e0 + ((part * kEPart + kk * 32) >> 4), v0 + ((kk * 2048) >> 4), ID_O,
+                     (part > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(bar(BAR_KV_EMPTY + stg));
+        umma_commit(bar(BAR_E_EMPTY + eb));
+        umma_commit(bar(BAR_O_FULL + ob));
+        return true;
+      };
+      for (long long it = blockIdx.x; it < a.items && ok; it += gridDim.x) {
+        long long bh;
+        int qt, j0, j1;
+        decode(it, bh, qt, j0, j1);
+        if (j0 >= j1) continue;
+        ok = wait_bar(bar(BAR_Q_FULL), qit & 1u, abort_flag, 57);
+        ++qit;
+        const uint32_t first = kn;
+        for (int J = j0; J < j1 && ok; ++J) {
+          ok = issue_s(kn);
+          ++kn;
+          if (ok && kn - first >= 2) ok = issue_o(pn++);    // E.V of the previous tile
+        }
+        if (ok) ok = issue_o(pn++);                         // the last tile of the item
+        if (ok) umma_commit(bar(BAR_Q_EMPTY));
+      }
+      umma_commit(bar(BAR_FINAL));
+      volatile uint32_t no_abort = 0u;
+      wait_bar(bar(BAR_FINAL), 0u, &no_abort, 62);
+    }
+  } else {
+    // ------------------------------------------------------------ one proxy per thread
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const float sl2 = a.scale_log2;
+    const int n_in_last = (int)(a.N - (long long)(nb - 1) * kBlock);
+    // this thread's E row in the K-major 128-byte-swizzled layout
+    unsigned char* const erow0 = smem + L::kOffE + (row >> 3) * 1024 + (row & 7) * 128;
+    uint32_t sn = 0;
+    bool stop = false;
+    for (long long it = blockIdx.x; it < a.items && !stop; it += gridDim.x) {
+      long long bh;
+      int qt, j0, j1;
+      decode(it, bh, qt, j0, j1);
+      const int I = qt * kRows + row;
+      const bool row_ok = I < nb;
+      if (j0 >= j1) {
+        // an empty key range contributes nothing to the proxy's max and sum
+        if (row_ok) {
+          const long long p = (bh * nb + I) * (long long)a.nsplit + it % a.nsplit;
+          a.Mp[p] = -INFINITY;
+          a.Zp[p] = 0.f;
+        }
+        continue;
+      }
+      const long long rbase = (bh * nb + (row_ok ? I : 0)) * (long long)nb;
+      float m = -INFINITY, Z = 0.f;
+      float m_prev = 0.f;
+      int J_prev = -1;
+      // error epilogue of tile n (block J, weights against m_used)
+      auto epilogue = [&](uint32_t n, int J, float m_used) -> bool {
+        const uint32_t ob = n % kOBufs;
+        if (!wait_bar(bar(BAR_O_FULL + ob), (n / kOBufs) & 1u, abort_flag, 58)) return false;
+        tc_fence_after();
+        const int nJ = J == nb - 1 ? n_in_last : kBlock;
+        const float cw = row_ok ? (float)nJ * ex2(a.L[rbase + J] - m_used) : 0.f;
+        const float4* vb = reinterpret_cast<const float4*>(a.vbar + (bh * nb + J) * (long long)D);
+        float err2 = 0.f;
+#pragma unroll 1
+        for (int ch = 0; ch < D / 32; ++ch) {
+          float o[32];
+          tmem_ld32(tmem + lane_off + L::kColO + ob * D + ch * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; c += 4) {
+            const float4 v4 = __ldg(vb + ch * 8 + c / 4);
+            const float d0 = fmaf(-cw, v4.x, o[c]), d1 = fmaf(-cw, v4.y, o[c + 1]);
+            const float d2 = fmaf(-cw, v4.z, o[c + 2]), d3 = fmaf(-cw, v4.w, o[c + 3]);
+            err2 = fmaf(d0, d0, fmaf(d1, d1, fmaf(d2, d2, fmaf(d3, d3, err2))));
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(BAR_O_EMPTY + ob));
+        if (row_ok) {
+          a.R[rbase + J] = sqrtf(err2);
+          a.Rm[rbase + J] = m_used;
+        }
+        return true;
+      };
+      for (int J = j0; J < j1; ++J) {
+        const uint32_t sb = sn % kSBufs, eb = sn % kEBufs;
+        if (!wait_bar(bar(BAR_S_FULL + sb), (sn / kSBufs) & 1u, abort_flag, 59)) { stop = true; break; }
+        tc_fence_after();
+        float x[64];
+        tmem_ld32(tmem + lane_off + L::kColS + sb * 64, x);
+        tmem_ld32(tmem + lane_off + L::kColS + sb * 64 + 32, x + 32);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(BAR_S_EMPTY + sb));
+        const int nval = J == nb - 1 ? n_in_last : kBlock;
+        float tmax = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          x[c] = c < nval ? x[c] * sl2 : -INFINITY;
+          tmax = fmaxf(tmax, x[c]);
+        }
+        const float mn = fmaxf(m, tmax);
+        float sum = 0.f;
+        uint32_t hi[32], lo[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const float e0 = ex2(x[c] - mn), e1 = ex2(x[c + 1] - mn);
+          sum += e0 + e1;
+          const __half2 h = __floats2half2_rn(e0, e1);
+          const float2 hf = __half22float2(h);
+          const __half2 l = __floats2half2_rn(e0 - hf.x, e1 - hf.y);
+          hi[c / 2] = *reinterpret_cast<const uint32_t*>(&h);
+          lo[c / 2] = *reinterpret_cast<const uint32_t*>(&l);
+        }
+        Z = (m == -INFINITY ? 0.f : Z * ex2(m - mn)) + sum;
+        m = mn;
+        if (!wait_bar(bar(BAR_E_EMPTY + eb), ((sn / kEBufs) & 1u) ^ 1u, abort_flag, 63)) { stop = true; break; }
+        unsigned char* erow = erow0 + eb * 2 * kEPart;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint32_t off = (uint32_t)((ch ^ (row & 7)) << 4);
+          *reinterpret_cast<uint4*>(erow + off) = make_uint4(hi[4 * ch], hi[4 * ch + 1], hi[4 * ch + 2], hi[4 * ch + 3]);
+          *reinterpret_cast<uint4*>(erow + kEPart + off) =
+              make_uint4(lo[4 * ch], lo[4 * ch + 1], lo[4 * ch + 2], lo[4 * ch + 3]);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(BAR_E_FULL + eb));
+        if (J_prev >= 0 && !epilogue(sn - 1, J_prev, m_prev)) { stop = true; break; }
+        J_prev = J;
+        m_prev = m;
+        ++sn;
+      }
+      if (stop) break;
+      if (J_prev >= 0 && !epilogue(sn - 1, J_prev, m_prev)) break;
+      if (row_ok) {
+        const long long p = (bh * nb + I) * (long long)a.nsplit + it % a.nsplit;
+        a.Mp[p] = m;
+        a.Zp[p] = Z;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(L::kCols));
   }
 }
 
-cudaError_t launch_route(const float* qbar, const void* kp, const void* vp, const float* kbar,
-                         const float* vbar, float* R, float* Rm, long long BH, long long N, int nb,
+// r_IJ = e_IJ 2^(m_IJ - M) / Z * 64 / n_J with M, Z combined over the key ranges.
+__global__ void route_fixup_kernel(float* __restrict__ R, const float* __restrict__ Rm, const float* __restrict__ Mp,
+                                   const float* __restrict__ Zp, long long N, int nb, int nsplit) {
+  const long long rowi = blockIdx.x;                 // (bh, I)
+  float M = -INFINITY;
+  for (int s = 0; s < nsplit; ++s) M = fmaxf(M, Mp[rowi * nsplit + s]);
+  float Z = 0.f;
+  for (int s = 0; s < nsplit; ++s) {
+    const float mp = Mp[rowi * nsplit + s];
+    if (mp > -INFINITY) Z += Zp[rowi * nsplit + s] * ex2(mp - M);
+  }
+  const float iz = Z > 0.f ? 1.f / Z : 0.f;
+  for (int J = threadIdx.x; J < nb; J += blockDim.x) {
+    const long long i = rowi * nb + J;
+    const int nJ = (int)std::max<long long>(1, std::min<long long>(kBlock, N - (long long)J * kBlock));
+    const float e = R[i];
+    R[i] = e > 0.f ? e * ex2(Rm[i] - M) * iz * ((float)kBlock / (float)nJ) : 0.f;
+  }
+}
+
+}  // namespace route
+}  // namespace tc
+
+// Key ranges per (head, proxy tile): 8 gives the persistent grid several
+// items per SM on every configuration, at a small per-item cost.
+int route_nsplit(int nb) { return std::max(1, std::min(nb, 8)); }
+
+// qsplit_bf: bf16 [BH, nb, 2d] (hi | lo of each query block mean); kp bf16 and vp fp16 [BH, Npad, d];
+// L: [BH, nb, nb] log2-domain centroid logits; R, Rm: [BH, nb, nb]; Mp, Zp: [BH, nb, nsplit].
+cudaError_t launch_route(const void* qsplit_bf, const void* kp, const void* vp, const float* L, const float* vbar,
+                         float* R, float* Rm, float* Mp, float* Zp, int nsplit, long long BH, long long N, int nb,
                          int d, cudaStream_t st) {
-  dim3 grid((unsigned)((nb + kRouteRows - 1) / kRouteRows), (unsigned)BH);
-  const float scale = 1.0f / sqrtf((float)d);
-  const __nv_bfloat16* k = reinterpret_cast<const __nv_bfloat16*>(kp);
-  const __half* v = reinterpret_cast<const __half*>(vp);
-  if (d == 128) route_kernel<128><<<grid, kRouteThreads, 0, st>>>(qbar, k, v, kbar, vbar, R, Rm, N, nb, scale);
-  else if (d == 64) route_kernel<64><<<grid, kRouteThreads, 0, st>>>(qbar, k, v, kbar, vbar, R, Rm, N, nb, scale);
+  using namespace tc::route;
+  const long long Npad = (long long)nb * kBlock;
+  CUtensorMap mq, mk, mv;
+  if (!tc::make_map_2d(&mq, qsplit_bf, BH * nb, 2 * d, kRows, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) ||
+      !tc::make_map_2d(&mk, kp, BH * Npad, d, 64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) ||
+      !tc::make_map_2d(&mv, vp, BH * Npad, d, 64, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+    return cudaErrorInvalidValue;
+  Args a;
+  a.L = L; a.vbar = vbar; a.R = R; a.Rm = Rm; a.Mp = Mp; a.Zp = Zp;
+  a.N = N; a.Npad = Npad; a.nb = nb;
+  a.nqt = (nb + kRows - 1) / kRows;
+  a.nsplit = nsplit;
+  a.per = (nb + nsplit - 1) / nsplit;
+  a.items = BH * a.nqt * nsplit;
+  a.scale_log2 = 1.4426950408889634f / sqrtf((float)d);
+  const long long grid = std::min<long long>(a.items, tc::sm_count());
+  auto go = [&](auto kernel, uint32_t smem) -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kernel<<<(unsigned)grid, kThreads, smem, st>>>(mq, mk, mv, a);
+    return cudaGetLastError();
+  };
+  cudaError_t e;
+  if (d == 128) e = go(route_tc_kernel<128>, Smem<128>::kBytes);
+  else if (d == 64) e = go(route_tc_kernel<64>, Smem<64>::kBytes);
   else return cudaErrorInvalidValue;
+  if (e != cudaSuccess) return e;
+  route_fixup_kernel<<<(unsigned)(BH * nb), 128, 0, st>>>(R, Rm, Mp, Zp, N, nb, nsplit);
   return cudaGetLastError();
 }
+
+cudaError_t route_tc_error(unsigned int* code, cudaStream_t st) { return tc::read_error(code, st); }
 
 }  // namespace svsa

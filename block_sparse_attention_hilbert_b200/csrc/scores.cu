@@ -21,6 +21,10 @@
 // Warp 0 issues the TMA copies (Q tile once per item, K tiles into a 2-stage
 // ring), warp 1 issues the MMAs into a 2-deep TMEM ring and owns the TMEM
 // allocation, warps 2-5 hold one query row per thread.  Every wait is bounded.
+//
+// SIZE = 64 can also write the raw logits L_IJ = qbar_I . kbar_J / sqrt(d) *
+// log2(e) (the centroid logits of the error-aware routing); with S = NULL
+// the kernel makes that single pass only.
 #include "tcgen05.cuh"
 
 namespace svsa {
@@ -58,7 +62,9 @@ struct Misc {
 };
 
 struct Args {
-  float* S;
+  float* S;            // nullable: normalised scores
+  float* L;            // nullable: raw log2-domain logits (SIZE = 64)
+  int passes;          // 2 (scores), or 1 (logits only)
   long long N;
   int ng;              // pooled rows per head
   int nvc;             // non-empty pooled rows per head (the rest are padding)
@@ -107,7 +113,7 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ms->tmem_base;
-  const int ntiles = 2 * a.nkt;                   // two passes over the key tiles
+  const int ntiles = a.passes * a.nkt;            // one or two passes over the key tiles
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -206,13 +212,14 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
         const int m_sub = (int)((nval + SIZE - 1) / SIZE);
         inv_m = m_sub > 0 ? 1.f / (float)m_sub : 0.f;
       }
-      float* srow = a.S + (bh * a.nb + (I < a.nb ? I : 0)) * (long long)a.nb;
+      const long long roff = (bh * a.nb + (I < a.nb ? I : 0)) * (long long)a.nb;   // row I of S / L
+      float* srow = a.S != nullptr ? a.S + roff : nullptr;
       for (int t = 0; t < ntiles; ++t) {
         const uint32_t sb = sn % kSBufs;
         if (!wait_bar(bar(BAR_S_FULL + sb), (sn / kSBufs) & 1u, abort_flag, 36)) { stop = true; break; }
         tc_fence_after();
-        const bool pass2 = t >= a.nkt;
-        const int kt = pass2 ? t - a.nkt : t;
+        const bool pass2 = t >= a.nkt || a.passes == 1;
+        const int kt = t >= a.nkt ? t - a.nkt : t;
         const int c0 = kt * kKeys;
         if (pass2 && t == a.nkt) inv = (row_ok && l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll 1
@@ -244,10 +251,18 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
             }
           } else if (SIZE == kBlock) {
             if (row_ok && I < a.nb) {
+              if (a.L != nullptr) {
+                float* lrow = a.L + roff;
 #pragma unroll
-              for (int c = 0; c < 32; ++c) {
-                const float p = ex2(x[c] - m) * inv;
-                if (cb + c < a.nb) srow[cb + c] = p;
+                for (int c = 0; c < 32; ++c)
+                  if (cb + c < a.nb) lrow[cb + c] = x[c];
+              }
+              if (a.S != nullptr) {
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                  const float p = ex2(x[c] - m) * inv;
+                  if (cb + c < a.nb) srow[cb + c] = p;
+                }
               }
             }
           } else {
@@ -289,8 +304,9 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
 }  // namespace tc
 
 // qsplit, ksplit: fp16 [BH, ng, 2d] (hi | lo of each pooled row), ng = Npad / size.
-cudaError_t launch_scores(const void* qsplit, const void* ksplit, float* S, long long BH, long long N, int ng,
-                          int nb, int d, int size, cudaStream_t st) {
+cudaError_t launch_scores(const void* qsplit, const void* ksplit, float* S, float* L, long long BH, long long N,
+                          int ng, int nb, int d, int size, cudaStream_t st) {
+  if (S == nullptr && (L == nullptr || size != kBlock)) return cudaErrorInvalidValue;
   using namespace tc::scores;
   CUtensorMap mq, mk;
   if (!tc::make_map_2d(&mq, qsplit, BH * ng, 2 * d, kRows, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
@@ -298,6 +314,8 @@ cudaError_t launch_scores(const void* qsplit, const void* ksplit, float* S, long
     return cudaErrorInvalidValue;
   Args a;
   a.S = S;
+  a.L = size == kBlock ? L : nullptr;
+  a.passes = S != nullptr ? 2 : 1;
   a.N = N;
   a.ng = ng;
   a.nvc = (int)std::min<long long>(ng, (N + size - 1) / size);

@@ -150,6 +150,17 @@ def test_routing_and_compensation_small():
         check_attention(gout, np.concatenate([ref[I] for I in range(attn.nb)]), f"comp head {eta}")
 
 
+@pytest.mark.parametrize("sub,d,grid,heads", [
+    (64, 128, (4, 10, 16), 2),      # nb = 10: key ranges of the routing kernel past nb are empty
+    (64, 64, (5, 7, 9), 2),         # head dim 64, ragged last block
+    (16, 128, (6, 12, 20), 2),      # budget from 16-token sub-block scores, ratios from block means
+    (64, 128, (10, 30, 52), 1),     # nb = 244: two tiles of 128 proxies, the second one ragged
+])
+def test_routing_masks(sub, d, grid, heads):
+    w = _small("threshold", sub, grid=grid, heads=heads, d=d, tau=0.9, routing=True)
+    _run_and_compare_masks(w)
+
+
 @pytest.mark.parametrize("d", [64, 128])
 def test_dense_and_random_masks(d):
     T, H, W = 5, 7, 9
