@@ -4,7 +4,7 @@
 // abstract: structured window with rotating anchors; "SVG-EAR" 2.B: routing by
 // estimated error under the threshold rule's budget):
 //   THRESHOLD  order the row by (score desc, index asc) and keep the shortest
-//              prefix whose fp64 cumulative sum reaches tau;
+//              prefix whose cumulative sum reaches tau;
 //   TOPK       keep the first k of that order;
 //   ROUTING    m = count THRESHOLD keeps on the score row, then the first m of
 //              the (ratio desc, index asc) order of the ratio row;
@@ -13,12 +13,13 @@
 // The ordered prefix is found without sorting: scores are non-negative
 // floats, so their bit patterns order like the values.  A most-significant-
 // digit-first radix select over the 32 bits (4 passes of 8 bits) histograms
-// the candidates' counts and fp64 masses per digit, and a suffix scan over the
-// 256 digits locates the digit holding the crossing element.  After the 4th
-// pass the crossing value v* is known exactly; everything above v* is kept,
-// and of the elements equal to v* the first t in index order.  One CTA per
-// row; the row lives in shared memory; output lists are ascending by
-// construction (a block-wide prefix count in index order).
+// the candidates' counts and masses per digit, and a suffix scan over the 256
+// digits locates the digit holding the crossing element.  After the 4th pass
+// the crossing value v* is known exactly; everything above v* is kept, and of
+// the elements equal to v* the first t in index order.  One warp per row
+// (histogram updates aggregated over the lanes that share a digit, so the
+// shared-memory atomics do not contend); output lists are ascending by
+// construction (ballot-based compaction in index order).
 #include "common.cuh"
 
 namespace svsa {
@@ -28,13 +29,8 @@ constexpr int kSelThreads = 256;
 enum { SEL_THRESHOLD = 0, SEL_TOPK = 1, SEL_STRUCTURED = 2, SEL_ROUTING = 3 };
 
 struct SelShared {
-  uint32_t cnt[256];
-  double mass[256];
   uint32_t scan_cnt[kSelThreads / 32];
   double scan_mass[kSelThreads / 32];
-  uint32_t prefix, above_cnt, eq_cnt, take;
-  uint32_t found, min_dg;
-  double above_mass, total;
   uint32_t run;                     // running output position (compaction)
 };
 
@@ -54,73 +50,6 @@ __device__ __forceinline__ void block_scan2(uint32_t& c, double& m, SelShared& s
   uint32_t oc = 0; double om = 0.0;
   for (int w = 0; w < wid; ++w) { oc += sh.scan_cnt[w]; om += sh.scan_mass[w]; }
   c += oc; m += om;
-  __syncthreads();
-}
-
-// Radix select over keys[0..n): on return sh.prefix = v* (bits), sh.above_cnt /
-// sh.above_mass = count / mass strictly above v*, sh.eq_cnt = elements equal to
-// v*, sh.take = how many of those (first in index order) are kept.
-// by_mass: reach `tau` in mass; else reach `k` in count.  Requires a reachable
-// target (caller handles "keep all").
-__device__ void radix_cut(const uint32_t* keys, int n, bool by_mass, double tau, uint32_t k,
-                          SelShared& sh) {
-  const int tid = threadIdx.x;
-  if (tid == 0) { sh.prefix = 0u; sh.above_cnt = 0u; sh.above_mass = 0.0; }
-  uint32_t pmask = 0u;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    sh.cnt[tid] = 0u;
-    sh.mass[tid] = 0.0;
-    if (tid == 0) { sh.found = 0u; sh.min_dg = 256u; }
-    __syncthreads();
-    const uint32_t prefix = sh.prefix;
-    for (int j = tid; j < n; j += kSelThreads) {
-      const uint32_t key = keys[j];
-      if ((key & pmask) == prefix) {
-        const uint32_t dg = (key >> shift) & 255u;
-        atomicAdd(&sh.cnt[dg], 1u);
-        if (by_mass) atomicAdd(&sh.mass[dg], (double)__uint_as_float(key));
-      }
-    }
-    __syncthreads();
-    // thread t owns digit 255 - t; inclusive scan = suffix sums over digits
-    const uint32_t dg = 255u - (uint32_t)tid;
-    uint32_t c = sh.cnt[dg];
-    double m = sh.mass[dg];
-    const uint32_t own_c = c;
-    const double own_m = m;
-    block_scan2(c, m, sh);
-    const uint32_t above_c = sh.above_cnt;
-    const double above_m = sh.above_mass;
-    bool hit;
-    if (by_mass) hit = (above_m + m >= tau) && (above_m + (m - own_m) < tau);
-    else hit = (above_c + c >= k) && (above_c + (c - own_c) < k);
-    if (own_c > 0u) atomicMin(&sh.min_dg, dg);
-    if (hit) sh.found = 1u;
-    __syncthreads();
-    // fp64 sums taken in a different order in this pass can miss the target by
-    // an ulp when the cumulative mass sits on tau; the crossing is then the
-    // last candidate, i.e. the smallest non-empty digit.
-    if (!sh.found && dg == sh.min_dg) hit = true;
-    if (hit) {
-      sh.prefix = prefix | (dg << shift);
-      sh.above_cnt = above_c + (c - own_c);
-      sh.above_mass = above_m + (m - own_m);
-      sh.eq_cnt = own_c;
-    }
-    pmask |= 255u << shift;
-    __syncthreads();
-  }
-  if (tid == 0) {
-    uint32_t t = 1;
-    if (by_mass) {
-      const double v = (double)__uint_as_float(sh.prefix);
-      double acc = sh.above_mass + v;
-      while (acc < tau && t < sh.eq_cnt) { acc += v; ++t; }
-    } else {
-      t = k - sh.above_cnt;
-    }
-    sh.take = t;
-  }
   __syncthreads();
 }
 
@@ -150,93 +79,200 @@ __device__ void compact_row(int n, KeepFn keep, int32_t* idx_out, int32_t* cnt_o
   if (tid == 0) *cnt_out = (int32_t)sh.run;
 }
 
-// Prefix rank among the elements equal to v* (in index order) is needed to
-// keep only the first `take` of them; computed on the fly during compaction.
-__global__ void __launch_bounds__(kSelThreads) select_kernel(
-    const float* __restrict__ S, const float* __restrict__ R, int nb, int mode, float tau, int k,
+// ---------------------------------------------------------------- one warp per row
+// Masses are exact 48-bit fixed-point integers (x * 2^48 truncated; scores are
+// probabilities, x <= 1, so a row of up to 16384 sums below 2^62): every
+// partial sum is exact and independent of the order it is taken in, so the
+// crossing digit found in one pass is consistent with the next, and the sums
+// differ from fp64 cumulative sums by < nb * 2^-48.
+constexpr int kSelWarps = 8;                 // rows per CTA
+constexpr double kFix = 281474976710656.0;   // 2^48
+
+__device__ __forceinline__ unsigned long long fix48(uint32_t key) {
+  return (unsigned long long)((double)__uint_as_float(key) * kFix);
+}
+
+struct WarpHist {
+  uint32_t cnt[256];
+  unsigned long long mass[256];
+};
+
+struct Cut {
+  uint32_t vstar;       // the crossing key
+  uint32_t take;        // how many keys equal to vstar (first in index order) are kept
+};
+
+// Radix select over one row by a single warp: keys are re-read from `row`
+// (through `key_of`) in every pass.  by_mass: the shortest prefix of the
+// (key desc, index asc) order whose mass reaches tau_fx; else the first k.
+// The target must be reachable (the caller handles "keep all").
+template <typename KeyOf>
+__device__ Cut warp_radix_cut(KeyOf key_of, int n, bool by_mass, unsigned long long tau_fx, uint32_t k,
+                              WarpHist& h) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t prefix = 0u, pmask = 0u, above_c = 0u, eq_c = 0u;
+  unsigned long long above_m = 0ull;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      h.cnt[lane * 8 + i] = 0u;
+      h.mass[lane * 8 + i] = 0ull;
+    }
+    __syncwarp();
+    for (int base = 0; base < n; base += 32) {
+      const int j = base + lane;
+      const uint32_t key = j < n ? key_of(j) : 0u;
+      const bool cand = j < n && (key & pmask) == prefix;
+      const uint32_t cmask = __ballot_sync(0xffffffffu, cand);
+      if (cand) {
+        const uint32_t dg = (key >> shift) & 255u;
+        const uint32_t peers = __match_any_sync(cmask, dg);
+        const bool leader = (peers & lt) == 0u;
+        if (by_mass) {
+          const unsigned long long m = fix48(key);
+          const uint32_t hi = __reduce_add_sync(peers, (uint32_t)(m >> 24));
+          const uint32_t lo = __reduce_add_sync(peers, (uint32_t)(m & 0xFFFFFFull));
+          if (leader) atomicAdd(&h.mass[dg], ((unsigned long long)hi << 24) + lo);
+        }
+        if (leader) atomicAdd(&h.cnt[dg], (uint32_t)__popc(peers));
+      }
+    }
+    __syncwarp();
+    // lane L owns digits 255 - 8L .. 248 - 8L (descending); exclusive scan over lanes
+    uint32_t c8[8];
+    unsigned long long m8[8];
+    uint32_t lc = 0u;
+    unsigned long long lm = 0ull;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int dg = 255 - (lane * 8 + i);
+      c8[i] = h.cnt[dg];
+      m8[i] = h.mass[dg];
+      lc += c8[i];
+      lm += m8[i];
+    }
+    uint32_t sc = lc;
+    unsigned long long sm = lm;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t yc = __shfl_up_sync(0xffffffffu, sc, o);
+      const unsigned long long ym = __shfl_up_sync(0xffffffffu, sm, o);
+      if (lane >= o) { sc += yc; sm += ym; }
+    }
+    uint32_t acc_c = above_c + sc - lc;           // everything above this lane's first digit
+    unsigned long long acc_m = above_m + sm - lm;
+    int hit = -1;
+    uint32_t hit_above_c = 0u, hit_c = 0u;
+    unsigned long long hit_above_m = 0ull;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const bool reach = by_mass ? (acc_m + m8[i] >= tau_fx && acc_m < tau_fx) : (acc_c + c8[i] >= k && acc_c < k);
+      if (hit < 0 && reach && c8[i] > 0u) {
+        hit = 255 - (lane * 8 + i);
+        hit_above_c = acc_c;
+        hit_above_m = acc_m;
+        hit_c = c8[i];
+      }
+      acc_c += c8[i];
+      acc_m += m8[i];
+    }
+    const uint32_t hb = __ballot_sync(0xffffffffu, hit >= 0);
+    const int src = hb ? __ffs(hb) - 1 : 31;     // exact sums: exactly one lane hits
+    const int dg = __shfl_sync(0xffffffffu, hit, src);
+    above_c = __shfl_sync(0xffffffffu, hit_above_c, src);
+    above_m = __shfl_sync(0xffffffffu, hit_above_m, src);
+    eq_c = __shfl_sync(0xffffffffu, hit_c, src);
+    prefix |= (uint32_t)(dg < 0 ? 0 : dg) << shift;
+    pmask |= 255u << shift;
+    __syncwarp();
+  }
+  Cut cut;
+  cut.vstar = prefix;
+  if (by_mass) {
+    const unsigned long long v = fix48(prefix);
+    const unsigned long long need = tau_fx - above_m;           // > 0 by construction
+    unsigned long long t = v > 0ull ? (need + v - 1ull) / v : (unsigned long long)eq_c;
+    if (t < 1ull) t = 1ull;
+    if (t > eq_c) t = eq_c;
+    cut.take = (uint32_t)t;
+  } else {
+    cut.take = k - above_c;
+  }
+  return cut;
+}
+
+__global__ void __launch_bounds__(kSelWarps * 32) select_kernel(
+    const float* __restrict__ S, const float* __restrict__ R, long long rows, int nb, int mode, float tau, int k,
     int cap, int32_t* __restrict__ kv_idx, int32_t* __restrict__ kv_cnt, uint32_t* __restrict__ bits) {
-  extern __shared__ uint32_t keys[];                   // [nb]
-  __shared__ SelShared sh;
-  const long long row = blockIdx.x;
-  const int tid = threadIdx.x;
+  __shared__ WarpHist hist[kSelWarps];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const long long row = (long long)blockIdx.x * kSelWarps + wid;
+  if (row >= rows) return;
+  WarpHist& h = hist[wid];
+  const uint32_t lt = (1u << lane) - 1u;
   const int words = (nb + 31) / 32;
   const float* srow = S + row * (long long)nb;
-
-  // --- score row: total mass (fp64), keys
-  double part = 0.0;
-  for (int j = tid; j < nb; j += kSelThreads) {
-    const uint32_t key = score_key(srow[j]);
-    keys[j] = key;
-    part += (double)__uint_as_float(key);
-  }
-  {
-    uint32_t dc = 0;
-    block_scan2(dc, part, sh);
-    if (tid == kSelThreads - 1) sh.total = part;
-    __syncthreads();
-  }
-  const double total = sh.total;
+  auto skey = [&](int j) { return score_key(__ldg(srow + j)); };
 
   bool keep_all = false;
-  uint32_t budget = 0;
+  uint32_t budget = 0u;
+  Cut cut{0u, 0u};
   if (mode == SEL_THRESHOLD || mode == SEL_ROUTING) {
-    if ((double)tau >= 1.0 || total < (double)tau) {
+    unsigned long long part = 0ull;
+    for (int j = lane; j < nb; j += 32) part += fix48(skey(j));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    const unsigned long long tau_fx = (unsigned long long)((double)tau * kFix);
+    if ((double)tau >= 1.0 || part < tau_fx) {
       keep_all = true;
       budget = (uint32_t)nb;
+    } else if (tau_fx == 0ull) {
+      cut = warp_radix_cut(skey, nb, false, 0ull, 1u, h);       // the shortest prefix is one block
+      budget = 1u;
     } else {
-      radix_cut(keys, nb, true, (double)tau, 0u, sh);
-      budget = sh.above_cnt + sh.take;
+      cut = warp_radix_cut(skey, nb, true, tau_fx, 0u, h);
+      // budget = kept count: keys above vstar plus `take`
+      uint32_t above = 0u;
+      for (int j = lane; j < nb; j += 32) above += skey(j) > cut.vstar ? 1u : 0u;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
+      budget = above + cut.take;
     }
   } else {  // TOPK
     budget = (uint32_t)k;
     if (k >= nb) keep_all = true;
-    else radix_cut(keys, nb, false, 0.0, (uint32_t)k, sh);
+    else cut = warp_radix_cut(skey, nb, false, 0ull, (uint32_t)k, h);
   }
-
-  if (mode == SEL_ROUTING && !keep_all) {
-    // rank by the ratio row instead, same budget
-    __syncthreads();
-    const float* rrow = R + row * (long long)nb;
-    for (int j = tid; j < nb; j += kSelThreads) keys[j] = score_key(rrow[j]);
-    __syncthreads();
+  const float* rrow = R != nullptr ? R + row * (long long)nb : nullptr;
+  auto rkey = [&](int j) { return score_key(__ldg(rrow + j)); };
+  const bool by_ratio = mode == SEL_ROUTING && !keep_all;
+  if (by_ratio) {
     if (budget >= (uint32_t)nb) keep_all = true;
-    else radix_cut(keys, nb, false, 0.0, budget, sh);
+    else cut = warp_radix_cut(rkey, nb, false, 0ull, budget, h);
   }
 
   int32_t* idx_out = kv_idx + row * (long long)cap;
   uint32_t* bits_out = bits ? bits + row * (long long)words : nullptr;
-  if (keep_all) {
-    compact_row(nb, [](int) { return true; }, idx_out, kv_cnt + row, bits_out, sh);
-    return;
+  uint32_t run = 0u, eq_run = 0u;
+  for (int base = 0; base < nb; base += 32) {
+    const int j = base + lane;
+    bool f = j < nb;
+    bool eq = false;
+    if (!keep_all && f) {
+      const uint32_t key = by_ratio ? rkey(j) : skey(j);
+      eq = key == cut.vstar;
+      f = key > cut.vstar;
+    }
+    const uint32_t eb = __ballot_sync(0xffffffffu, eq);
+    if (eq) f = eq_run + (uint32_t)__popc(eb & lt) < cut.take;
+    eq_run += (uint32_t)__popc(eb);
+    const uint32_t fb = __ballot_sync(0xffffffffu, f);
+    if (bits_out != nullptr && lane == 0) bits_out[base >> 5] = fb;
+    if (f) idx_out[run + (uint32_t)__popc(fb & lt)] = j;
+    run += (uint32_t)__popc(fb);
   }
-  // elements equal to v*: keep the first `take` in index order.  A running
-  // count of equal elements seen in earlier chunks plus an in-chunk scan.
-  const uint32_t vstar = sh.prefix;
-  const uint32_t take = sh.take;
-  __shared__ uint32_t eq_run;
-  if (tid == 0) { eq_run = 0u; sh.run = 0u; }
-  __syncthreads();
-  for (int base = 0; base < nb; base += kSelThreads) {
-    const int j = base + tid;
-    const uint32_t key = j < nb ? keys[j] : 0u;
-    const bool eq = j < nb && key == vstar;
-    uint32_t ce = eq ? 1u : 0u;
-    double dz = 0.0;
-    block_scan2(ce, dz, sh);
-    const uint32_t eq_rank = eq_run + ce - (eq ? 1u : 0u);
-    const bool f = j < nb && (key > vstar || (eq && eq_rank < take));
-    const uint32_t ballot = __ballot_sync(0xffffffffu, f);
-    if (bits_out != nullptr && (tid & 31) == 0 && base + (tid & ~31) < nb)
-      bits_out[(base + tid) >> 5] = ballot;
-    uint32_t c = f ? 1u : 0u;
-    double dz2 = 0.0;
-    block_scan2(c, dz2, sh);
-    if (f) idx_out[sh.run + c - 1u] = j;
-    __syncthreads();
-    if (tid == kSelThreads - 1) { sh.run += c; eq_run += ce; }
-    __syncthreads();
-  }
-  if (tid == 0) kv_cnt[row] = (int32_t)sh.run;
+  if (lane == 0) kv_cnt[row] = (int32_t)run;
 }
 
 // STRUCTURED: block coordinates from the raster id of each block's first token.
@@ -273,12 +309,9 @@ __global__ void __launch_bounds__(kSelThreads) structured_kernel(
 cudaError_t launch_select(const float* S, const float* R, long long rows, int nb, int mode, float tau,
                           int k, int cap, int32_t* kv_idx, int32_t* kv_cnt, uint32_t* bits,
                           cudaStream_t st) {
-  const size_t smem = (size_t)nb * sizeof(uint32_t);
-  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)std::max<size_t>(smem, 1));
-  if (e != cudaSuccess) return e;
-  select_kernel<<<(unsigned)rows, kSelThreads, smem, st>>>(S, R, nb, mode, tau, k, cap, kv_idx,
-                                                            kv_cnt, bits);
+  const long long blocks = (rows + kSelWarps - 1) / kSelWarps;
+  select_kernel<<<(unsigned)blocks, kSelWarps * 32, 0, st>>>(S, R, rows, nb, mode, tau, k, cap, kv_idx, kv_cnt,
+                                                             bits);
   return cudaGetLastError();
 }
 
