@@ -32,7 +32,8 @@ import workloads  # noqa: E402
 
 METRIC = "block-sparse attn fwd ms & kept-FLOP TFLOP/s (% BF16 peak); speedup vs dense"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-ATTN_KERNEL_SRC = os.path.join(ROOT, "block_sparse_attention_hilbert_b200", "csrc", "attn_tc.cu")
+ATTN_KERNEL_SRCS = [os.path.join(ROOT, "block_sparse_attention_hilbert_b200", "csrc", f)
+                    for f in ("attn_tc.cu", "tcgen05.cuh")]
 
 
 def _args():
@@ -168,7 +169,8 @@ class ClockSampler:
 # --------------------------------------------------------------------------- traffic
 def _attn_traffic(workload: str):
     """dram bytes per attention launch from the committed ncu summary, if it was
-    taken on the current kernel source (else null)."""
+    taken on the current kernel source -- attn_tc.cu and tcgen05.cuh, hashed
+    together -- (else null)."""
     import hashlib
     path = os.path.join(ROOT, "profiles", f"attn_{workload}.traffic.txt")
     if not os.path.exists(path):
@@ -179,8 +181,11 @@ def _attn_traffic(workload: str):
             if ":" in line and not line.startswith("#"):
                 a, b = line.split(":", 1)
                 kv[a.strip()] = b.strip()
-    with open(ATTN_KERNEL_SRC, "rb") as f:
-        h = hashlib.sha256(f.read()).hexdigest()[:16]
+    sha = hashlib.sha256()
+    for src in ATTN_KERNEL_SRCS:
+        with open(src, "rb") as f:
+            sha.update(f.read())
+    h = sha.hexdigest()[:16]
     if kv.get("kernel_sha256_16") != h:
         return None
     try:
