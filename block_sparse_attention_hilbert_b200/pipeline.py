@@ -7,6 +7,13 @@ A call runs svsa_reorder (Q, K), svsa_reorder_values (V), svsa_build_mask (unles
 reused across denoising steps -- "DFSAttn" trick 3), svsa_attn_fwd and
 svsa_inverse_reorder on the current stream.  The permutation is built once per
 object.  Buffers are allocated once with torch (the library allocates nothing).
+
+    attn.forward_host(q_h, k_h, v_h, o_h)   # pinned host tensors in and out
+
+runs the same calls on groups of (batch, head) rows, with the host->device
+copies of one group, the library calls of the previous group and the
+device->host copy of the one before overlapping on three streams (every
+(batch, head) row is independent in all four steps).
 """
 from __future__ import annotations
 
@@ -115,6 +122,71 @@ class SparseVideoAttention:
 
     def inverse(self, out, stream=None):
         svsa_inverse_reorder(self.buf.op, out, self.buf.iperm, self.shape, stream)
+
+    # ---- a group of (batch, head) rows, as a layer of its own -------------
+    def _rows(self, t, r0, r1):
+        """rows r0..r1 of the flattened (batch, head) dimension of a layer-shaped buffer"""
+        return t.reshape((self.B * self.heads,) + tuple(t.shape[2:]))[r0:r1] if t is not None else None
+
+    def _group(self, r0, r1):
+        b = self.buf
+        sh = shape(1, r1 - r0, self.T, self.H, self.W, self.d)
+        m = make_mask(self._rows(b.kv_idx, r0, r1), self._rows(b.kv_cnt, r0, r1), b.cap,
+                      self._rows(b.bits, r0, r1), self._rows(b.kbar, r0, r1), self._rows(b.vbar, r0, r1),
+                      b.nvalid, self._rows(b.cbar, r0, r1))
+        return sh, m
+
+    def forward_host(self, q, k, v, out, *, anchor_offset: int = 0, reuse_mask: bool = False, groups: int = 8):
+        """q, k, v, out: pinned host bf16 [B, heads, N, d] (raster order).  The rows
+        are processed in `groups` groups; each group's inputs are copied in on one
+        stream, its four library calls run on the current stream once they have
+        arrived, and its output is copied out on a third stream.  The current
+        stream waits for the last copy, so synchronising it covers the layer."""
+        b = self.buf
+        rows = self.B * self.heads
+        if getattr(self, "_stage", None) is None:
+            dev = b.qp.device
+            self._stage = tuple(torch.empty(rows, self.N, self.d, dtype=torch.bfloat16, device=dev)
+                                for _ in range(4))
+            self._h2d, self._d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        dq, dk, dv, dout = self._stage
+        hq, hk, hv, hout = (t.reshape(rows, self.N, self.d) for t in (q, k, v, out))
+        compute = torch.cuda.current_stream()
+        if not self._perm_ready:
+            self.build_perm()
+        build = not (reuse_mask and self.mask_ready)
+        if build:
+            self.params.anchor_offset = int(anchor_offset)
+        # group bounds keep every per-row mask slice 16-byte aligned (the ABI's
+        # pointer rule): rows of nb int32 counts must start at a multiple of 4 words
+        unit = 4 // math.gcd(self.nb, 4)
+        groups = max(1, min(groups, rows))
+        bounds = sorted({min(rows, (rows * g // groups) // unit * unit) for g in range(groups)} | {rows})
+        # the copy streams start after what the current stream has already queued
+        self._h2d.wait_stream(compute)
+        self._d2h.wait_stream(compute)
+        for r0, r1 in zip(bounds[:-1], bounds[1:]):
+            with torch.cuda.stream(self._h2d):
+                for h, d_ in ((hq, dq), (hk, dk), (hv, dv)):
+                    d_[r0:r1].copy_(h[r0:r1], non_blocking=True)
+            compute.wait_stream(self._h2d)
+            sh, m = self._group(r0, r1)
+            svsa_reorder(dq[r0:r1], self._rows(b.qp, r0, r1), b.perm, sh, compute)
+            svsa_reorder(dk[r0:r1], self._rows(b.kp, r0, r1), b.perm, sh, compute)
+            svsa_reorder_values(dv[r0:r1], self._rows(b.vp, r0, r1), b.perm, sh, compute)
+            if build:
+                svsa_build_mask(self._rows(b.qp, r0, r1), self._rows(b.kp, r0, r1), self._rows(b.vp, r0, r1),
+                                b.perm, sh, self.params, m, b.ws, b.ws.numel(), compute)
+            svsa_attn_fwd(self._rows(b.qp, r0, r1), self._rows(b.kp, r0, r1), self._rows(b.vp, r0, r1), m,
+                          self.compensate, self._rows(b.op, r0, r1), None, sh, compute)
+            svsa_inverse_reorder(self._rows(b.op, r0, r1), dout[r0:r1], b.iperm, sh, compute)
+            self._d2h.wait_stream(compute)
+            with torch.cuda.stream(self._d2h):
+                hout[r0:r1].copy_(dout[r0:r1], non_blocking=True)
+        if build:
+            self.mask_ready = True
+        compute.wait_stream(self._d2h)
+        return out
 
     # ---- whole layer ----------------------------------------------------
     def __call__(self, q, k, v, *, out=None, anchor_offset: int = 0, reuse_mask: bool = False, stream=None):

@@ -161,6 +161,33 @@ def test_routing_masks(sub, d, grid, heads):
     _run_and_compare_masks(w)
 
 
+@pytest.mark.parametrize("select,groups,kw", [
+    ("topk", 3, {}),
+    ("threshold", 5, {"routing": True, "compensate": True}),
+    ("structured", 2, {"n_anchors": 2}),
+])
+def test_forward_host_matches_device_call(select, groups, kw):
+    """The streamed host-to-host layer (groups of heads on three streams) gives
+    bit for bit the output of the device call on the same inputs."""
+    w = _small(select, 64, grid=(6, 12, 20), heads=8, tau=0.9, keep_frac=0.3, **kw)   # nb = 23: groups of 4 rows
+    q, k, v = (t.cuda() for t in workloads.make_qkv(w, seed=3))
+    mk = lambda: svsa.SparseVideoAttention(w.B, w.heads, w.T, w.H, w.W, w.d, order=w.order, select=w.select,
+                                           tau=w.tau, keep_frac=w.keep_frac, n_anchors=w.n_anchors,
+                                           routing=w.routing, compensate=w.compensate, device="cuda")
+    ref = mk()(q, k, v, anchor_offset=1)
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    hout = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    attn = mk()
+    attn.forward_host(hq, hk, hv, hout, anchor_offset=1, groups=groups)
+    torch.cuda.synchronize()
+    assert torch.equal(hout, ref.cpu())
+    # a second call reusing the cached mask gives the same output again
+    hout2 = torch.empty_like(hout).pin_memory()
+    attn.forward_host(hq, hk, hv, hout2, reuse_mask=True, groups=groups)
+    torch.cuda.synchronize()
+    assert torch.equal(hout2, hout)
+
+
 @pytest.mark.parametrize("d", [64, 128])
 def test_dense_and_random_masks(d):
     T, H, W = 5, 7, 9
