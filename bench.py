@@ -32,6 +32,7 @@ import workloads  # noqa: E402
 
 METRIC = "block-sparse attn fwd ms & kept-FLOP TFLOP/s (% BF16 peak); speedup vs dense"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+LONG_STEP_MS = 100.0
 ATTN_KERNEL_SRCS = [os.path.join(ROOT, "block_sparse_attention_hilbert_b200", "csrc", f)
                     for f in ("attn_tc.cu", "tcgen05.cuh")]
 
@@ -372,7 +373,10 @@ def run_svsa(args):
     d2h = out.numel() * out.element_size()
 
     peaks, peak_src = _peaks()
-    peak = float(peaks["bf16_tflops"])
+    # a kernel inside steps of 100 ms or more runs seconds-long loops under the
+    # power cap: its denominator is the sustained GEMM rate, else the burst one
+    sustained = step_ms >= LONG_STEP_MS
+    peak = float(peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"])
     attn_tflops = kflops / (attn_ms * 1e-3) / 1e12
     value = ws * kflops / (step_ms * 1e-3) / 1e12
     cpu = None
@@ -404,7 +408,8 @@ def run_svsa(args):
             "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
                          "frac": attn_tflops / peak, "traffic": _attn_traffic(w.name),
                          "kernel": "svsa attention (kept-block FLOPs / launch time)",
-                         "peak_source": f"{peak_src} bf16_tflops (burst)"},
+                         "peak_source": f"{peak_src} " + ("bf16_tflops_sustained (step >= 100 ms)" if sustained
+                                                           else "bf16_tflops (burst)")},
             "e2e": {"value": ws * kflops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
