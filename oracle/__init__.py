@@ -24,6 +24,9 @@ Sources (page title, section):
     attention mass such as 95%).
   * "LVSA: Training-Free Sparse Attention for Long Video Diffusion" --
     abstract (structured window pattern with rotating global anchors).
+  * DFSAttn trick 3 and SVOO 2.B -- a step schedule: dense early steps, a
+    sparser rule as the video clears, the mask rebuilt every few steps
+    (`schedule.py`).
 
 Pins: every function here is checked in `tests/test_oracle_*.py` against
 something other than itself (brute force, closed forms, invariants, library
@@ -37,11 +40,12 @@ from .mask import (pool, block_scores, subblock_scores, select_threshold, select
                    mask_from_rows)
 from .attention import (masked_attention, compensated_attention, dense_attention,
                         online_block_attention, kept_flops)
+from .schedule import step_param, rebuilds, mask_steps
 
 __all__ = [
     "hilbert_key_3d", "perm_raster", "perm_hilbert", "build_perm", "reorder", "inverse_reorder",
     "locality_stats", "pool", "block_scores", "subblock_scores", "select_threshold", "select_topk",
     "topk_count", "select_rows", "structured_mask", "anchor_blocks", "route_ratios",
     "select_routing", "mask_from_rows", "masked_attention", "compensated_attention",
-    "dense_attention", "online_block_attention", "kept_flops",
+    "dense_attention", "online_block_attention", "kept_flops", "step_param", "rebuilds", "mask_steps",
 ]
