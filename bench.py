@@ -47,6 +47,10 @@ def _args():
     ap.add_argument("--order", default=None, choices=["raster", "hilbert"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--schedule", default=None, metavar="N,DENSE,START,END,EVERY",
+                    help="time whole denoising runs of the layer under the step schedule "
+                         "(svsa_schedule_step): N steps, DENSE dense ones, the rule parameter "
+                         "from START to END, the mask rebuilt every EVERY steps")
     return ap.parse_args()
 
 
@@ -422,10 +426,105 @@ def run_svsa(args):
         dist.destroy_process_group()
 
 
+# --------------------------------------------------------------------------- schedule mode
+def run_schedule(args):
+    """One bench step = one whole denoising run of the layer under the step
+    schedule: every step reorders, builds its mask only on the schedule's
+    rebuild steps, attends and reorders back (same inputs every step)."""
+    rank, ws, local = _dist()
+    import block_sparse_attention_hilbert_b200 as svsa
+    assert torch.cuda.is_available(), "bench.py needs a GPU"
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    svsa.lib()
+    w = _workload(args)
+    n, dense, start, end, every = args.schedule.split(",")
+    sched = (int(n), int(dense), float(start), float(end), int(every))
+    n = sched[0]
+    stream = torch.cuda.current_stream()
+    q, k, v = workloads.make_qkv(w, seed=rank, device=dev)
+    attn = svsa.SparseVideoAttention(w.B, w.heads, w.T, w.H, w.W, w.d, order=w.order, select=w.select,
+                                     tau=w.tau, keep_frac=w.keep_frac, sub_block=w.sub_block,
+                                     routing=w.routing, compensate=w.compensate, schedule=sched, device=dev)
+    out = torch.empty_like(q)
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    nvalid = np.minimum(64, w.N - 64 * np.arange(w.nb)).astype(np.int64)
+    # untimed pass: the kept FLOPs of every step's mask
+    kf, builds = [], 0
+    for st in range(n):
+        _, rebuilt = attn.step(q, k, v, st, out=out)
+        if rebuilt:
+            builds += 1
+            torch.cuda.synchronize()
+            cur = kept_flops_from_lists(attn.buf.kv_idx.cpu().numpy(), attn.buf.kv_cnt.cpu().numpy(), nvalid, w.d)
+        kf.append(cur)
+    kflops = float(sum(kf))
+    dense_flops = 4.0 * w.d * float(w.N) ** 2 * w.heads * w.B * n
+
+    def run():
+        for st in range(n):
+            attn.step(q, k, v, st, out=out)
+
+    for _ in range(max(args.warmup, 3)):
+        run()
+    torch.cuda.synchronize()
+    launches0 = svsa.svsa_launch_count()
+    times = []
+    _barrier(ws)
+    with ClockSampler(dev.index) as clk:
+        for _ in range(args.steps):
+            flush.fill_(1.0)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            run()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+    _barrier(ws)
+    launches = svsa.svsa_launch_count() - launches0
+    run_ms = _max_over_ranks(statistics.mean(times), ws)
+    # the same run with dense attention on every step: the denominator of the speedup
+    dtimes = []
+    for i in range(2):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for st in range(n):
+            attn.reorder(q, k, v)
+            attn.attend_dense()
+            attn.inverse(out)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dtimes.append(e0.elapsed_time(e1))
+    dense_run_ms = _max_over_ranks(min(dtimes), ws)
+    if rank == 0:
+        line = {
+            "metric": "block-sparse attn fwd, whole denoising run under the step schedule: kept TFLOP/s",
+            "value": ws * kflops / (run_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": run_ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "heads": w.heads, "d": w.d, "grid": [w.T, w.H, w.W], "select": w.select,
+                       "schedule": {"n_steps": sched[0], "dense_steps": sched[1], "start": sched[2],
+                                    "end": sched[3], "refresh_every": sched[4]},
+                       "l2": "flushed (512 MiB write) between timed runs",
+                       "step": "one bench step = one whole denoising run of the layer"},
+            "ms_per_denoising_step": run_ms / n, "mask_builds_per_run": builds,
+            "density_per_run": kflops / dense_flops, "dense_run_ms": dense_run_ms,
+            "speedup_vs_dense": dense_run_ms / run_ms, "gpu_launches": launches,
+            "clocks": clk.summary(),
+            "e2e": None, "cpu_baseline": None,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     args = _args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.schedule is not None:
+        run_schedule(args)
     else:
         run_svsa(args)
 

@@ -48,6 +48,11 @@ class Mask(ctypes.Structure):
                 ("nvalid", ctypes.c_void_p), ("cbar", ctypes.c_void_p)]
 
 
+class Schedule(ctypes.Structure):
+    _fields_ = [("n_steps", ctypes.c_int32), ("dense_steps", ctypes.c_int32), ("start", ctypes.c_float),
+                ("end", ctypes.c_float), ("refresh_every", ctypes.c_int32)]
+
+
 _lib = None
 
 _SIGS = {
@@ -72,6 +77,8 @@ _SIGS = {
                                            ctypes.c_void_p, ctypes.c_void_p, Shape, ctypes.c_void_p]),
     "svsa_inverse_reorder": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, Shape,
                                             ctypes.c_void_p]),
+    "svsa_schedule_step": (ctypes.c_int, [ctypes.POINTER(Schedule), ctypes.c_int32, ctypes.POINTER(MaskParams),
+                                          ctypes.POINTER(MaskParams), ctypes.POINTER(ctypes.c_int32)]),
     "svsa_sync_status": (ctypes.c_int, [ctypes.c_void_p]),
     "svsa_last_error": (ctypes.c_char_p, []),
     "svsa_version": (ctypes.c_char_p, []),
@@ -149,6 +156,19 @@ def svsa_build_perm_noalloc(s: Shape, order: int, perm, iperm, stream=None) -> N
     """svsa_build_perm with the library's fixed scratch (no allocation; max side 128 for Hilbert)."""
     _check(lib().svsa_build_perm_noalloc(s, order, _p(perm), _p(iperm), _stream(stream)),
            "svsa_build_perm_noalloc")
+
+
+def schedule(n_steps: int, dense_steps: int, start: float, end: float, refresh_every: int) -> Schedule:
+    return Schedule(n_steps, dense_steps, start, end, refresh_every)
+
+
+def svsa_schedule_step(sch: Schedule, step: int, base: MaskParams):
+    """(mask params of `step`, True if the step builds its mask)."""
+    out = MaskParams()
+    rebuild = ctypes.c_int32(0)
+    _check(lib().svsa_schedule_step(ctypes.byref(sch), step, ctypes.byref(base), ctypes.byref(out),
+                                    ctypes.byref(rebuild)), "svsa_schedule_step")
+    return out, bool(rebuild.value)
 
 
 def svsa_reorder(x, xp, perm, s: Shape, stream=None) -> None:

@@ -435,6 +435,37 @@ svsa_status svsa_attn_dense_fwd(const void* qp, const void* kp, const void* vp, 
                      "attn_dense_fwd launch");
 }
 
+svsa_status svsa_schedule_step(const svsa_schedule* sch, int32_t step, const svsa_mask_params* base,
+                               svsa_mask_params* out, int32_t* rebuild) {
+  g_last_error.clear();
+  if (sch == nullptr || base == nullptr || out == nullptr || rebuild == nullptr)
+    return fail(SVSA_ERR_INVALID_ARG, "schedule, base, out and rebuild must not be NULL");
+  if (sch->n_steps < 1 || sch->dense_steps < 0 || sch->dense_steps > sch->n_steps || sch->refresh_every < 1)
+    return fail(SVSA_ERR_INVALID_ARG, "schedule n_steps=%d dense_steps=%d refresh_every=%d out of range",
+                sch->n_steps, sch->dense_steps, sch->refresh_every);
+  if (!(sch->start >= 0.f) || !(sch->end >= 0.f) || !std::isfinite(sch->start) || !std::isfinite(sch->end))
+    return fail(SVSA_ERR_INVALID_ARG, "schedule start/end must be finite and >= 0");
+  if (step < 0 || step >= sch->n_steps)
+    return fail(SVSA_ERR_INVALID_ARG, "step=%d outside [0, %d)", step, sch->n_steps);
+  if (base->select != SVSA_SEL_THRESHOLD && base->select != SVSA_SEL_TOPK)
+    return fail(SVSA_ERR_UNSUPPORTED, "only THRESHOLD and TOPK rules have a density to schedule");
+  float p = 1.0f;
+  if (step >= sch->dense_steps) {
+    const int span = sch->n_steps - 1 - sch->dense_steps;
+    const double u = span > 0 ? (double)(step - sch->dense_steps) / (double)span : 0.0;
+    p = (float)((double)sch->start + ((double)sch->end - (double)sch->start) * u);
+  }
+  const int32_t r = (step == 0 || step == sch->dense_steps ||
+                     (step > sch->dense_steps && (step - sch->dense_steps) % sch->refresh_every == 0))
+                        ? 1 : 0;
+  svsa_mask_params o = *base;
+  if (o.select == SVSA_SEL_THRESHOLD) o.tau = p;
+  else o.keep_frac = p;
+  *out = o;
+  *rebuild = r;
+  return SVSA_OK;
+}
+
 svsa_status svsa_sync_status(void* stream) {
   g_last_error.clear();
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);

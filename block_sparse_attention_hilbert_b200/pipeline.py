@@ -22,9 +22,9 @@ import math
 import torch
 
 from . import (ORDER_HILBERT, ORDER_RASTER, SEL_STRUCTURED, SEL_THRESHOLD, SEL_TOPK, BLOCK,
-               make_mask, mask_params, shape, svsa_attn_dense_fwd, svsa_attn_fwd, svsa_build_mask,
-               svsa_build_perm, svsa_inverse_reorder, svsa_mask_workspace_bytes,
-               svsa_perm_workspace_bytes, svsa_reorder, svsa_reorder_values)
+               make_mask, mask_params, schedule as make_schedule, shape, svsa_attn_dense_fwd, svsa_attn_fwd,
+               svsa_build_mask, svsa_build_perm, svsa_inverse_reorder, svsa_mask_workspace_bytes,
+               svsa_perm_workspace_bytes, svsa_reorder, svsa_reorder_values, svsa_schedule_step)
 
 _ORDERS = {"raster": ORDER_RASTER, "hilbert": ORDER_HILBERT}
 _SELECTS = {"threshold": SEL_THRESHOLD, "topk": SEL_TOPK, "structured": SEL_STRUCTURED}
@@ -69,7 +69,9 @@ class LayerBuffers:
 class SparseVideoAttention:
     def __init__(self, B, heads, T, H, W, d, *, order="hilbert", select="threshold", tau=0.9,
                  keep_frac=0.25, sub_block=64, win_t=2, win_rows=1, n_anchors=0, routing=False,
-                 compensate=False, keep_bits=False, device="cuda"):
+                 compensate=False, keep_bits=False, schedule=None, device="cuda"):
+        """schedule: optional (n_steps, dense_steps, start, end, refresh_every) -- a
+        timestep-adaptive rule for `step()` (svsa_schedule_step)."""
         self.B, self.heads, self.T, self.H, self.W, self.d = B, heads, T, H, W, d
         self.N = T * H * W
         self.nb = -(-self.N // BLOCK)
@@ -82,7 +84,9 @@ class SparseVideoAttention:
         self.params = mask_params(self.select, tau, keep_frac, sub_block, win_t, win_rows, n_anchors, 0,
                                   routing)
         k = max(1, min(self.nb, math.ceil(float(torch.tensor(keep_frac, dtype=torch.float32)) * self.nb)))
-        cap = k if self.select == SEL_TOPK else self.nb
+        self.schedule = make_schedule(*schedule) if schedule is not None else None
+        # a scheduled top-k rule reaches keep_frac = 1 on its dense steps
+        cap = k if (self.select == SEL_TOPK and self.schedule is None) else self.nb
         self.buf = LayerBuffers(B, heads, T, H, W, d, cap=cap, need_means=self.compensate or self.routing,
                                 keep_bits=keep_bits, ws_bytes=svsa_mask_workspace_bytes(self.shape, self.params),
                                 perm_ws_bytes=svsa_perm_workspace_bytes(self.shape, self.order),
@@ -122,6 +126,26 @@ class SparseVideoAttention:
 
     def inverse(self, out, stream=None):
         svsa_inverse_reorder(self.buf.op, out, self.buf.iperm, self.shape, stream)
+
+    # ---- one denoising step under the schedule ----------------------------
+    def step(self, q, k, v, step: int, *, out=None, anchor_offset: int = 0, stream=None):
+        """The layer at denoising step `step` of the schedule: the step's rule
+        parameter, and a new mask only on the schedule's rebuild steps (the
+        others reuse the last mask).  Returns (out, rebuilt)."""
+        if self.schedule is None:
+            raise ValueError("no schedule given to this layer")
+        base = self.params
+        p, rebuild = svsa_schedule_step(self.schedule, step, base)
+        self.params = p
+        if out is None:
+            out = torch.empty_like(q)
+        build = rebuild or not self.mask_ready
+        self.reorder(q, k, v, stream)
+        if build:
+            self.build_mask(anchor_offset, stream)
+        self.attend(stream=stream)
+        self.inverse(out, stream)
+        return out, build
 
     # ---- a group of (batch, head) rows, as a layer of its own -------------
     def _rows(self, t, r0, r1):

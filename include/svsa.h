@@ -228,6 +228,36 @@ svsa_status svsa_attn_dense_fwd(const void* qp, const void* kp, const void* vp, 
 svsa_status svsa_inverse_reorder(const void* op, void* o, const int32_t* iperm, svsa_shape s,
                                  void* stream);
 
+/* ---- step schedule -------------------------------------------------------- */
+
+/* Timestep-adaptive sparsity with a cached mask ("DFSAttn: Dynamic Fine-grained
+ * Sparse Attention for Efficient Video Generation", trick 3: look at nearly
+ * everything while the latent is noise, skip more as the video clears, and
+ * reuse a decided mask for the following steps; "SVOO" 2.B reuses its block
+ * structure every N diffusion steps).  The pages give the shape, not the
+ * numbers; this reading:
+ *   steps [0, dense_steps) keep every block (tau = 1 or keep_frac = 1);
+ *   from step dense_steps to n_steps - 1 the rule parameter (tau for
+ *   THRESHOLD, keep_frac for TOPK) moves linearly from start to end:
+ *   p = start + (end - start) * (step - dense_steps) / (n_steps - 1 - dense_steps)
+ *   in double, rounded to float (p = start when that span is empty);
+ *   a mask is built at step 0, at step dense_steps and every refresh_every
+ *   steps after it; the steps in between reuse the last one. */
+typedef struct {
+  int32_t n_steps;        /* denoising steps of the run, >= 1 */
+  int32_t dense_steps;    /* in [0, n_steps] */
+  float start, end;       /* rule parameter at step dense_steps and at the last step, >= 0 */
+  int32_t refresh_every;  /* >= 1 */
+} svsa_schedule;
+
+/* Mask parameters of `step` (in [0, n_steps)): *out = *base with tau
+ * (THRESHOLD) or keep_frac (TOPK) replaced by the step's value; *rebuild = 1
+ * when this step builds its mask, 0 when it reuses the last one.  Host-only,
+ * no device work.  STRUCTURED has no density parameter: SVSA_ERR_UNSUPPORTED.
+ * out may alias base. */
+svsa_status svsa_schedule_step(const svsa_schedule* sch, int32_t step, const svsa_mask_params* base,
+                               svsa_mask_params* out, int32_t* rebuild);
+
 /* ---- status ------------------------------------------------------------- */
 
 /* Synchronise `stream` and report device-side failures recorded by the

@@ -16,8 +16,8 @@ reading, used here and by the library:
     (tau for the threshold rule, keep_frac for top-k) moves linearly from
     `start` to `end`: p(s) = start + (end - start) * u, with
     u = (s - dense_steps) / (n_steps - 1 - dense_steps) (u = 0 when that
-    span is empty), evaluated in fp64 and rounded to float32 (the rule's
-    parameter type);
+    span is empty), with start and end taken as float32 values, evaluated in
+    fp64 and rounded to float32 (the rule's parameter type);
   * a mask is built at step 0, at step dense_steps, and every refresh_every
     steps after it; every other step reuses the last mask built (with that
     step's parameter and inputs).
@@ -32,6 +32,7 @@ def step_param(n_steps: int, dense_steps: int, start: float, end: float, step: i
     """The rule parameter of `step` (a float32 value, returned as a Python float)."""
     if step < dense_steps:
         return 1.0
+    start, end = float(np.float32(start)), float(np.float32(end))
     span = n_steps - 1 - dense_steps
     u = (step - dense_steps) / span if span > 0 else 0.0
     return float(np.float32(start + (end - start) * u))

@@ -4,6 +4,8 @@ import ctypes
 import os
 import re
 
+import numpy as np
+
 import pytest
 
 import block_sparse_attention_hilbert_b200 as svsa
@@ -135,3 +137,37 @@ def test_status_codes_are_stable():
     for name, val in [("SVSA_OK", 0), ("SVSA_ERR_INVALID_ARG", 1), ("SVSA_ERR_UNSUPPORTED", 2),
                       ("SVSA_ERR_WORKSPACE", 3), ("SVSA_ERR_CUDA", 4), ("SVSA_ERR_TIMEOUT", 5)]:
         assert re.search(rf"{name}\s*=\s*{val}\b", text)
+
+
+@pytest.mark.parametrize("n,dense,start,end,every", [
+    (50, 5, 0.97, 0.85, 5), (12, 0, 0.5, 0.2, 3), (7, 7, 0.9, 0.1, 2), (3, 2, 0.9, 0.1, 1), (1, 0, 0.3, 0.3, 4)])
+@pytest.mark.parametrize("select", [svsa.SEL_THRESHOLD, svsa.SEL_TOPK])
+def test_schedule_step_matches_the_oracle(n, dense, start, end, every, select):
+    """Host-only entry point: the step's rule parameter is the oracle's float32
+    value bit for bit, and the rebuild flags are the oracle's pattern."""
+    import oracle
+    sch = svsa.schedule(n, dense, start, end, every)
+    base = svsa.mask_params(select, tau=0.5, keep_frac=0.5)
+    flags = oracle.rebuilds(n, dense, every)
+    for s in range(n):
+        p, rebuild = svsa.svsa_schedule_step(sch, s, base)
+        got = p.tau if select == svsa.SEL_THRESHOLD else p.keep_frac
+        other = p.keep_frac if select == svsa.SEL_THRESHOLD else p.tau
+        assert got == oracle.step_param(n, dense, start, end, s)
+        assert other == np.float32(0.5)                       # the other field is untouched
+        assert rebuild == flags[s]
+
+
+def test_schedule_step_rejects():
+    lib = _raw()
+    sch = svsa.schedule(10, 2, 0.9, 0.5, 3)
+    out = svsa.MaskParams()
+    r = ctypes.c_int32(0)
+    base = svsa.mask_params(svsa.SEL_STRUCTURED)
+    assert lib.svsa_schedule_step(ctypes.byref(sch), 0, ctypes.byref(base), ctypes.byref(out), ctypes.byref(r)) == 2
+    base = svsa.mask_params(svsa.SEL_THRESHOLD)
+    assert lib.svsa_schedule_step(ctypes.byref(sch), 10, ctypes.byref(base), ctypes.byref(out), ctypes.byref(r)) == 1
+    bad = svsa.schedule(10, 11, 0.9, 0.5, 3)
+    assert lib.svsa_schedule_step(ctypes.byref(bad), 0, ctypes.byref(base), ctypes.byref(out), ctypes.byref(r)) == 1
+    bad = svsa.schedule(10, 2, 0.9, 0.5, 0)
+    assert lib.svsa_schedule_step(ctypes.byref(bad), 0, ctypes.byref(base), ctypes.byref(out), ctypes.byref(r)) == 1

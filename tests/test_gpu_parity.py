@@ -161,6 +161,46 @@ def test_routing_masks(sub, d, grid, heads):
     _run_and_compare_masks(w)
 
 
+@pytest.mark.parametrize("select,start,end", [("threshold", 0.97, 0.7), ("topk", 0.6, 0.25)])
+def test_schedule_run_matches_oracle(select, start, end):
+    """An 8-step run under the step schedule (2 dense steps, mask rebuilt every 3
+    steps, Q and K drifting between steps): each rebuilt mask is the oracle's
+    for that step's parameter and inputs, each reused mask is bit-identical to
+    the last built one, and every step's output is the oracle's attention over
+    the step's inputs with the mask in use."""
+    n, dense, every = 8, 2, 3
+    w = _small(select, 64, grid=(6, 12, 20), heads=2)
+    q0, k0, v = (t.cuda() for t in workloads.make_qkv(w, seed=5))
+    attn = svsa.SparseVideoAttention(w.B, w.heads, w.T, w.H, w.W, w.d, order=w.order, select=select,
+                                     schedule=(n, dense, start, end, every), keep_bits=True, device="cuda")
+    perm, _ = oracle.build_perm(w.T, w.H, w.W, w.order)
+    flags = oracle.rebuilds(n, dense, every)
+    last = None
+    for s in range(n):
+        q, k = workloads.qk_at_step(q0, k0, sigma=0.05, seed=5, step=s)
+        out, rebuilt = attn.step(q, k, v, s)
+        torch.cuda.synchronize()
+        assert rebuilt == flags[s]
+        keep = gpu_keep(attn)
+        qp, kp, vp = (oracle.reorder(to_np(t)[0].astype(np.float64), perm) for t in (q, k, v))
+        if rebuilt:
+            p = oracle.step_param(n, dense, start, end, s)
+            ws = w.with_(tau=p) if select == "threshold" else w.with_(keep_frac=p)
+            for eta in range(w.heads):
+                kept, near = oracle_rows(ws, qp[eta], kp[eta], vp[eta], perm, list(range(attn.nb)))
+                compare_mask_rows(keep[eta], kept, near)
+            if s < dense:
+                assert keep.all()
+            last = keep
+        else:
+            assert np.array_equal(keep, last)
+        op = to_np(attn.buf.op)[0]
+        for eta in range(w.heads):
+            ref = oracle.masked_attention(qp[eta], kp[eta], vp[eta], w.N, keep[eta])
+            gout = np.concatenate([op[eta][I * 64:min(I * 64 + 64, w.N)] for I in range(attn.nb)])
+            check_attention(gout, np.concatenate([ref[I] for I in range(attn.nb)]), f"step {s} head {eta}")
+
+
 @pytest.mark.parametrize("select,groups,kw", [
     ("topk", 3, {}),
     ("threshold", 5, {"routing": True, "compensate": True}),
