@@ -27,6 +27,8 @@ Sources (page title, section):
   * DFSAttn trick 3 and SVOO 2.B -- a step schedule: dense early steps, a
     sparser rule as the video clears, the mask rebuilt every few steps
     (`schedule.py`).
+  * SVOO 2.B and SVG-EAR 2.A -- bidirectional query-key co-clustering and the
+    semantic token order it gives (`cluster.py`).
 
 Pins: every function here is checked in `tests/test_oracle_*.py` against
 something other than itself (brute force, closed forms, invariants, library
@@ -41,6 +43,7 @@ from .mask import (pool, block_scores, subblock_scores, select_threshold, select
 from .attention import (masked_attention, compensated_attention, dense_attention,
                         online_block_attention, kept_flops)
 from .schedule import step_param, rebuilds, mask_steps
+from .cluster import cocluster, perm_from_clusters, initial_centroids
 
 __all__ = [
     "hilbert_key_3d", "perm_raster", "perm_hilbert", "build_perm", "reorder", "inverse_reorder",
@@ -48,4 +51,5 @@ __all__ = [
     "topk_count", "select_rows", "structured_mask", "anchor_blocks", "route_ratios",
     "select_routing", "mask_from_rows", "masked_attention", "compensated_attention",
     "dense_attention", "online_block_attention", "kept_flops", "step_param", "rebuilds", "mask_steps",
+    "cocluster", "perm_from_clusters", "initial_centroids",
 ]
