@@ -44,7 +44,7 @@ def _args():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="svsa", choices=["svsa", "reference"])
     ap.add_argument("--workload", default="wan13b", choices=sorted(workloads.WORKLOADS))
-    ap.add_argument("--order", default=None, choices=["raster", "hilbert"])
+    ap.add_argument("--order", default=None, choices=["raster", "hilbert", "cocluster"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--schedule", default=None, metavar="N,DENSE,START,END,EVERY",
@@ -255,6 +255,8 @@ def run_reference(args):
     import oracle
     w = _workload(args)
     q, k, v = workloads.make_qkv(w, device="cpu")
+    if w.order not in ("raster", "hilbert"):
+        raise SystemExit("the oracle arm samples the geometric orders (raster, hilbert) only")
     perm_cache = oracle.build_perm(w.T, w.H, w.W, w.order)
     per_step = max(0.5, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
@@ -300,7 +302,7 @@ def run_svsa(args):
     def step(evs=None):
         if evs is not None:
             evs[0].record(stream)
-        attn.build_perm()
+        attn.build_perm(q=q, k=k)
         if evs is not None:
             evs[1].record(stream)
         attn.reorder(q, k, v)

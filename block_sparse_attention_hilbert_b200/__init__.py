@@ -77,6 +77,16 @@ _SIGS = {
                                            ctypes.c_void_p, ctypes.c_void_p, Shape, ctypes.c_void_p]),
     "svsa_inverse_reorder": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, Shape,
                                             ctypes.c_void_p]),
+    "svsa_cocluster_workspace_bytes": (ctypes.c_size_t, [Shape]),
+    "svsa_build_perm_cocluster": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, Shape, ctypes.c_int32,
+                                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                                 ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "svsa_reorder_heads": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, Shape,
+                                          ctypes.c_void_p]),
+    "svsa_reorder_values_heads": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, Shape,
+                                                 ctypes.c_void_p]),
+    "svsa_inverse_reorder_heads": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, Shape,
+                                                  ctypes.c_void_p]),
     "svsa_schedule_step": (ctypes.c_int, [ctypes.POINTER(Schedule), ctypes.c_int32, ctypes.POINTER(MaskParams),
                                           ctypes.POINTER(MaskParams), ctypes.POINTER(ctypes.c_int32)]),
     "svsa_sync_status": (ctypes.c_int, [ctypes.c_void_p]),
@@ -169,6 +179,30 @@ def svsa_schedule_step(sch: Schedule, step: int, base: MaskParams):
     _check(lib().svsa_schedule_step(ctypes.byref(sch), step, ctypes.byref(base), ctypes.byref(out),
                                     ctypes.byref(rebuild)), "svsa_schedule_step")
     return out, bool(rebuild.value)
+
+
+def svsa_cocluster_workspace_bytes(s: Shape) -> int:
+    return int(lib().svsa_cocluster_workspace_bytes(s))
+
+
+def svsa_build_perm_cocluster(q, k, s: Shape, rounds: int, perm_q, iperm_q, perm_k, iperm_k, ws, ws_bytes: int,
+                              stream=None) -> None:
+    _check(lib().svsa_build_perm_cocluster(_p(q), _p(k), s, rounds, _p(perm_q), _p(iperm_q), _p(perm_k),
+                                           _p(iperm_k), _p(ws), ws_bytes, _stream(stream)),
+           "svsa_build_perm_cocluster")
+
+
+def svsa_reorder_heads(x, xp, perm, s: Shape, stream=None) -> None:
+    _check(lib().svsa_reorder_heads(_p(x), _p(xp), _p(perm), s, _stream(stream)), "svsa_reorder_heads")
+
+
+def svsa_reorder_values_heads(v, vp, perm, s: Shape, stream=None) -> None:
+    _check(lib().svsa_reorder_values_heads(_p(v), _p(vp), _p(perm), s, _stream(stream)), "svsa_reorder_values_heads")
+
+
+def svsa_inverse_reorder_heads(op, o, iperm, s: Shape, stream=None) -> None:
+    _check(lib().svsa_inverse_reorder_heads(_p(op), _p(o), _p(iperm), s, _stream(stream)),
+           "svsa_inverse_reorder_heads")
 
 
 def svsa_reorder(x, xp, perm, s: Shape, stream=None) -> None:

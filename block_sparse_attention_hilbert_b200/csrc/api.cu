@@ -19,10 +19,15 @@ int hilbert_order_bits(int T, int H, int W);
 int perm_noalloc_max_bits();
 size_t perm_noalloc_scratch_bytes();
 cudaError_t perm_noalloc_scratch(void** out);
-cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* map, long long BH,
+cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* map, long long map_stride, long long BH,
                                long long rows_dst, long long rows_src, int d, cudaStream_t st);
-cudaError_t launch_gather_rows_f16(const void* src, void* dst, const int32_t* map, long long BH,
-                                   long long rows_dst, long long rows_src, int d, cudaStream_t st);
+cudaError_t launch_gather_rows_f16(const void* src, void* dst, const int32_t* map, long long map_stride,
+                                   long long BH, long long rows_dst, long long rows_src, int d, cudaStream_t st);
+size_t cocluster_workspace_bytes(long long BH, long long N, int nb, int d);
+cudaError_t launch_cocluster(const void* q, const void* k, long long BH, long long N, int nb, int d, int rounds,
+                             int32_t* perm_q, int32_t* iperm_q, int32_t* perm_k, int32_t* iperm_k, void* ws,
+                             cudaStream_t st, int* launches);
+cudaError_t cocluster_tc_error(unsigned int* code, cudaStream_t st);
 cudaError_t launch_pool(const void* xp, float* out, void* split, void* split_bf, int32_t* nvalid, long long BH,
                         long long N, long long Npad, int d, int size, cudaStream_t st);
 cudaError_t launch_pool_f16(const void* xp, float* out, int32_t* nvalid, long long BH, long long N,
@@ -185,6 +190,27 @@ int topk_count(float keep_frac, int nb) {
 
 }  // namespace
 
+namespace {
+// The row gathers of steps 2 and 4; per_head: the map holds one row per (batch, head).
+svsa_status gather(const void* src, void* dst, const int32_t* map, svsa_shape s, bool forward, bool to_f16,
+                   bool per_head, void* stream, const char* what) {
+  g_last_error.clear();
+  SVSA_TRY(check_shape(s, true));
+  SVSA_PTR(src, "input");
+  SVSA_PTR(dst, "output");
+  SVSA_PTR(map, forward ? "perm" : "iperm");
+  if (src == dst) return fail(SVSA_ERR_INVALID_ARG, "input and output must not alias");
+  const Dims g = make_dims(s.B, s.heads, s.T, s.H, s.W, s.d);
+  const long long rows_dst = forward ? g.Npad : g.N, rows_src = forward ? g.N : g.Npad;
+  const long long stride = per_head ? rows_dst : 0;
+  cudaError_t e = to_f16 ? launch_gather_rows_f16(src, dst, map, stride, g.BH, rows_dst, rows_src, g.d,
+                                                  (cudaStream_t)stream)
+                         : launch_gather_rows(src, dst, map, stride, g.BH, rows_dst, rows_src, g.d,
+                                              (cudaStream_t)stream);
+  return cuda_status(counted(e, 1), what);
+}
+}  // namespace
+
 extern "C" {
 
 const char* svsa_last_error(void) { return g_last_error.c_str(); }
@@ -243,39 +269,56 @@ svsa_status svsa_build_perm_noalloc(svsa_shape s, int32_t order, int32_t* perm, 
 }
 
 svsa_status svsa_reorder(const void* x, void* xp, const int32_t* perm, svsa_shape s, void* stream) {
-  g_last_error.clear();
-  SVSA_TRY(check_shape(s, true));
-  SVSA_PTR(x, "x");
-  SVSA_PTR(xp, "xp");
-  SVSA_PTR(perm, "perm");
-  if (x == xp) return fail(SVSA_ERR_INVALID_ARG, "x and xp must not alias");
-  const Dims g = make_dims(s.B, s.heads, s.T, s.H, s.W, s.d);
-  return cuda_status(counted(launch_gather_rows(x, xp, perm, g.BH, g.Npad, g.N, g.d, (cudaStream_t)stream), 1),
-                     "reorder launch");
+  return gather(x, xp, perm, s, true, false, false, stream, "reorder launch");
 }
 
 svsa_status svsa_reorder_values(const void* v, void* vp, const int32_t* perm, svsa_shape s, void* stream) {
-  g_last_error.clear();
-  SVSA_TRY(check_shape(s, true));
-  SVSA_PTR(v, "v");
-  SVSA_PTR(vp, "vp");
-  SVSA_PTR(perm, "perm");
-  if (v == vp) return fail(SVSA_ERR_INVALID_ARG, "v and vp must not alias");
-  const Dims g = make_dims(s.B, s.heads, s.T, s.H, s.W, s.d);
-  return cuda_status(counted(launch_gather_rows_f16(v, vp, perm, g.BH, g.Npad, g.N, g.d, (cudaStream_t)stream), 1),
-                     "reorder_values launch");
+  return gather(v, vp, perm, s, true, true, false, stream, "reorder_values launch");
 }
 
 svsa_status svsa_inverse_reorder(const void* op, void* o, const int32_t* iperm, svsa_shape s, void* stream) {
+  return gather(op, o, iperm, s, false, false, false, stream, "inverse_reorder launch");
+}
+
+svsa_status svsa_reorder_heads(const void* x, void* xp, const int32_t* perm, svsa_shape s, void* stream) {
+  return gather(x, xp, perm, s, true, false, true, stream, "reorder_heads launch");
+}
+
+svsa_status svsa_reorder_values_heads(const void* v, void* vp, const int32_t* perm, svsa_shape s, void* stream) {
+  return gather(v, vp, perm, s, true, true, true, stream, "reorder_values_heads launch");
+}
+
+svsa_status svsa_inverse_reorder_heads(const void* op, void* o, const int32_t* iperm, svsa_shape s, void* stream) {
+  return gather(op, o, iperm, s, false, false, true, stream, "inverse_reorder_heads launch");
+}
+
+size_t svsa_cocluster_workspace_bytes(svsa_shape s) {
+  if (s.T < 1 || s.H < 1 || s.W < 1 || s.B < 1 || s.heads < 1 || (s.d != 64 && s.d != 128)) return 0;
+  const Dims g = make_dims(s.B, s.heads, s.T, s.H, s.W, s.d);
+  return cocluster_workspace_bytes(g.BH, g.N, g.nb, g.d);
+}
+
+svsa_status svsa_build_perm_cocluster(const void* q, const void* k, svsa_shape s, int32_t rounds, int32_t* perm_q,
+                                      int32_t* iperm_q, int32_t* perm_k, int32_t* iperm_k, void* ws, size_t ws_bytes,
+                                      void* stream) {
   g_last_error.clear();
   SVSA_TRY(check_shape(s, true));
-  SVSA_PTR(op, "op");
-  SVSA_PTR(o, "o");
-  SVSA_PTR(iperm, "iperm");
-  if (op == o) return fail(SVSA_ERR_INVALID_ARG, "op and o must not alias");
+  SVSA_PTR(q, "q");
+  SVSA_PTR(k, "k");
+  SVSA_PTR(perm_q, "perm_q");
+  SVSA_PTR(iperm_q, "iperm_q");
+  SVSA_PTR(perm_k, "perm_k");
+  SVSA_PTR(iperm_k, "iperm_k");
+  SVSA_PTR(ws, "ws");
+  if (rounds < 1 || rounds > 64) return fail(SVSA_ERR_INVALID_ARG, "rounds=%d outside [1, 64]", rounds);
   const Dims g = make_dims(s.B, s.heads, s.T, s.H, s.W, s.d);
-  return cuda_status(counted(launch_gather_rows(op, o, iperm, g.BH, g.N, g.Npad, g.d, (cudaStream_t)stream), 1),
-                     "inverse_reorder launch");
+  if (g.nb > kMaxBlocks) return fail(SVSA_ERR_UNSUPPORTED, "nb=%d exceeds %d", g.nb, kMaxBlocks);
+  const size_t need = cocluster_workspace_bytes(g.BH, g.N, g.nb, g.d);
+  if (ws_bytes < need) return fail(SVSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need);
+  int launches = 0;
+  cudaError_t e = launch_cocluster(q, k, g.BH, g.N, g.nb, g.d, rounds, perm_q, iperm_q, perm_k, iperm_k, ws,
+                                   (cudaStream_t)stream, &launches);
+  return cuda_status(counted(e, launches), "cocluster launch");
 }
 
 size_t svsa_mask_workspace_bytes(svsa_shape s, const svsa_mask_params* p) {
@@ -473,11 +516,12 @@ svsa_status svsa_sync_status(void* stream) {
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_status(e, "asynchronous error");
   // every tensor-core translation unit keeps its own error word; read (and clear) all of them
-  cudaError_t (*readers[3])(unsigned int*, cudaStream_t) = {attn_tc_error, scores_tc_error, route_tc_error};
-  const char* names[3] = {"attention", "scores", "routing"};
+  cudaError_t (*readers[4])(unsigned int*, cudaStream_t) = {attn_tc_error, scores_tc_error, route_tc_error,
+                                                           cocluster_tc_error};
+  const char* names[4] = {"attention", "scores", "routing", "co-clustering"};
   unsigned int first_code = 0u;
   const char* first_name = nullptr;
-  for (int i = 0; i < 3; ++i) {
+  for (int i = 0; i < 4; ++i) {
     unsigned int code = 0u;
     e = readers[i](&code, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_status(e, "reading the device error word");

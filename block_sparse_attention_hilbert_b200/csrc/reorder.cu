@@ -2,6 +2,8 @@
 //
 // Forward  ("DFSAttn", trick 1):  xp[bh, i, :] = x[bh, perm[i], :]   (zeros where perm[i] < 0)
 // Inverse:                        o[bh, r, :]  = op[bh, iperm[r], :]
+// The map is shared by all (batch, head) rows (map_stride = 0) or given per
+// row (map_stride = its length), as the semantic orders are.
 // The value tensor's forward gather also converts bf16 -> fp16 (the P.V
 // product runs in fp16).
 //
@@ -28,9 +30,10 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
 // kGatherThreads * kUnroll chunks.
 template <int CPR>
 __global__ void __launch_bounds__(kGatherThreads) gather_rows_kernel(
-    const uint4* __restrict__ src, uint4* __restrict__ dst, const int32_t* __restrict__ map,
-    long long rows_dst, long long rows_src) {
+    const uint4* __restrict__ src, uint4* __restrict__ dst, const int32_t* __restrict__ map_all,
+    long long map_stride, long long rows_dst, long long rows_src) {
   const long long bh = blockIdx.y;
+  const int32_t* map = map_all + bh * map_stride;
   const long long total = rows_dst * CPR;
   const uint4* s_base = src + bh * rows_src * CPR;
   uint4* d_base = dst + bh * rows_dst * CPR;
@@ -72,9 +75,10 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
 
 template <int CPR>
 __global__ void __launch_bounds__(kGatherThreads) gather_rows_f16_kernel(
-    const uint4* __restrict__ src, uint4* __restrict__ dst, const int32_t* __restrict__ map,
-    long long rows_dst, long long rows_src) {
+    const uint4* __restrict__ src, uint4* __restrict__ dst, const int32_t* __restrict__ map_all,
+    long long map_stride, long long rows_dst, long long rows_src) {
   const long long bh = blockIdx.y;
+  const int32_t* map = map_all + bh * map_stride;
   const long long total = rows_dst * CPR;
   const uint4* s_base = src + bh * rows_src * CPR;
   uint4* d_base = dst + bh * rows_dst * CPR;
@@ -98,23 +102,23 @@ __global__ void __launch_bounds__(kGatherThreads) gather_rows_f16_kernel(
   }
 }
 
-cudaError_t launch_gather_rows_f16(const void* src, void* dst, const int32_t* map, long long BH,
-                                   long long rows_dst, long long rows_src, int d, cudaStream_t st) {
+cudaError_t launch_gather_rows_f16(const void* src, void* dst, const int32_t* map, long long map_stride,
+                                   long long BH, long long rows_dst, long long rows_src, int d, cudaStream_t st) {
   const int cpr = d * 2 / 16;
   const long long total = rows_dst * cpr;
   const long long tile = (long long)kGatherThreads * kUnroll;
   const long long gx = std::max<long long>(1, (total + tile - 1) / tile);
   dim3 grid((unsigned)gx, (unsigned)BH);
   if (cpr == 16)
-    gather_rows_f16_kernel<16><<<grid, kGatherThreads, 0, st>>>((const uint4*)src, (uint4*)dst, map, rows_dst, rows_src);
+    gather_rows_f16_kernel<16><<<grid, kGatherThreads, 0, st>>>((const uint4*)src, (uint4*)dst, map, map_stride, rows_dst, rows_src);
   else if (cpr == 8)
-    gather_rows_f16_kernel<8><<<grid, kGatherThreads, 0, st>>>((const uint4*)src, (uint4*)dst, map, rows_dst, rows_src);
+    gather_rows_f16_kernel<8><<<grid, kGatherThreads, 0, st>>>((const uint4*)src, (uint4*)dst, map, map_stride, rows_dst, rows_src);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
 
-cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* map, long long BH,
+cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* map, long long map_stride, long long BH,
                                long long rows_dst, long long rows_src, int d, cudaStream_t st) {
   const int cpr = d * 2 / 16;
   const long long total = rows_dst * cpr;
@@ -123,10 +127,10 @@ cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* map, l
   dim3 grid((unsigned)gx, (unsigned)BH);
   if (cpr == 16)
     gather_rows_kernel<16><<<grid, kGatherThreads, 0, st>>>(
-        (const uint4*)src, (uint4*)dst, map, rows_dst, rows_src);
+        (const uint4*)src, (uint4*)dst, map, map_stride, rows_dst, rows_src);
   else if (cpr == 8)
     gather_rows_kernel<8><<<grid, kGatherThreads, 0, st>>>(
-        (const uint4*)src, (uint4*)dst, map, rows_dst, rows_src);
+        (const uint4*)src, (uint4*)dst, map, map_stride, rows_dst, rows_src);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();

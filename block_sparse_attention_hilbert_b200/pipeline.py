@@ -23,8 +23,10 @@ import torch
 
 from . import (ORDER_HILBERT, ORDER_RASTER, SEL_STRUCTURED, SEL_THRESHOLD, SEL_TOPK, BLOCK,
                make_mask, mask_params, schedule as make_schedule, shape, svsa_attn_dense_fwd, svsa_attn_fwd,
-               svsa_build_mask, svsa_build_perm, svsa_inverse_reorder, svsa_mask_workspace_bytes,
-               svsa_perm_workspace_bytes, svsa_reorder, svsa_reorder_values, svsa_schedule_step)
+               svsa_build_mask, svsa_build_perm, svsa_build_perm_cocluster, svsa_cocluster_workspace_bytes,
+               svsa_inverse_reorder, svsa_inverse_reorder_heads, svsa_mask_workspace_bytes,
+               svsa_perm_workspace_bytes, svsa_reorder, svsa_reorder_heads, svsa_reorder_values,
+               svsa_reorder_values_heads, svsa_schedule_step)
 
 _ORDERS = {"raster": ORDER_RASTER, "hilbert": ORDER_HILBERT}
 _SELECTS = {"threshold": SEL_THRESHOLD, "topk": SEL_TOPK, "structured": SEL_STRUCTURED}
@@ -69,14 +71,20 @@ class LayerBuffers:
 class SparseVideoAttention:
     def __init__(self, B, heads, T, H, W, d, *, order="hilbert", select="threshold", tau=0.9,
                  keep_frac=0.25, sub_block=64, win_t=2, win_rows=1, n_anchors=0, routing=False,
-                 compensate=False, keep_bits=False, schedule=None, device="cuda"):
-        """schedule: optional (n_steps, dense_steps, start, end, refresh_every) -- a
-        timestep-adaptive rule for `step()` (svsa_schedule_step)."""
+                 compensate=False, keep_bits=False, schedule=None, cluster_rounds=3, device="cuda"):
+        """order: "raster", "hilbert" or "cocluster" (a per-head semantic order from
+        bidirectional query-key co-clustering, built from the first inputs and
+        kept until `rebuild_order()`).  schedule: optional (n_steps, dense_steps,
+        start, end, refresh_every) -- a timestep-adaptive rule for `step()`."""
         self.B, self.heads, self.T, self.H, self.W, self.d = B, heads, T, H, W, d
         self.N = T * H * W
         self.nb = -(-self.N // BLOCK)
         self.Npad = self.nb * BLOCK
-        self.order = _ORDERS[order]
+        self.cocluster = order == "cocluster"
+        self.cluster_rounds = int(cluster_rounds)
+        self.order = ORDER_RASTER if self.cocluster else _ORDERS[order]
+        if self.cocluster and select == "structured":
+            raise ValueError("the structured rule needs a geometric order (raster or hilbert)")
         self.select = _SELECTS[select]
         self.compensate = bool(compensate)
         self.routing = bool(routing)
@@ -92,19 +100,42 @@ class SparseVideoAttention:
                                 perm_ws_bytes=svsa_perm_workspace_bytes(self.shape, self.order),
                                 device=device, compensate=self.compensate)
         self._mask = self.buf.mask()
+        if self.cocluster:
+            rows, dev = B * heads, self.buf.qp.device
+            b = self.buf
+            b.perm_q = torch.empty(rows, self.Npad, dtype=torch.int32, device=dev)
+            b.iperm_q = torch.empty(rows, self.N, dtype=torch.int32, device=dev)
+            b.perm_k = torch.empty_like(b.perm_q)
+            b.iperm_k = torch.empty_like(b.iperm_q)
+            b.clu_ws = torch.empty(max(svsa_cocluster_workspace_bytes(self.shape), 16), dtype=torch.uint8, device=dev)
         self._perm_ready = False
         self.mask_ready = False
 
     # ---- the four steps -------------------------------------------------
-    def build_perm(self, stream=None):
+    def build_perm(self, stream=None, q=None, k=None):
         b = self.buf
-        svsa_build_perm(self.shape, self.order, b.perm, b.iperm, b.perm_ws, b.perm_ws.numel(), stream)
+        if self.cocluster:
+            if q is None or k is None:
+                raise ValueError("the co-clustering order is built from the layer's raster q and k")
+            svsa_build_perm_cocluster(q, k, self.shape, self.cluster_rounds, b.perm_q, b.iperm_q, b.perm_k,
+                                      b.iperm_k, b.clu_ws, b.clu_ws.numel(), stream)
+        else:
+            svsa_build_perm(self.shape, self.order, b.perm, b.iperm, b.perm_ws, b.perm_ws.numel(), stream)
         self._perm_ready = True
+
+    def rebuild_order(self):
+        """Re-cluster at the next call (the co-clustering order is reused until then)."""
+        self._perm_ready = False
 
     def reorder(self, q, k, v, stream=None):
         if not self._perm_ready:
-            self.build_perm(stream)
+            self.build_perm(stream, q, k)
         b = self.buf
+        if self.cocluster:
+            svsa_reorder_heads(q, b.qp, b.perm_q, self.shape, stream)
+            svsa_reorder_heads(k, b.kp, b.perm_k, self.shape, stream)
+            svsa_reorder_values_heads(v, b.vp, b.perm_k, self.shape, stream)
+            return
         svsa_reorder(q, b.qp, b.perm, self.shape, stream)
         svsa_reorder(k, b.kp, b.perm, self.shape, stream)
         svsa_reorder_values(v, b.vp, b.perm, self.shape, stream)
@@ -112,8 +143,8 @@ class SparseVideoAttention:
     def build_mask(self, anchor_offset: int = 0, stream=None):
         b = self.buf
         self.params.anchor_offset = int(anchor_offset)
-        svsa_build_mask(b.qp, b.kp, b.vp, b.perm, self.shape, self.params, self._mask, b.ws, b.ws.numel(),
-                        stream)
+        svsa_build_mask(b.qp, b.kp, b.vp, None if self.cocluster else b.perm, self.shape, self.params, self._mask,
+                        b.ws, b.ws.numel(), stream)
         self.mask_ready = True
 
     def attend(self, lse=None, stream=None):
@@ -125,7 +156,10 @@ class SparseVideoAttention:
         svsa_attn_dense_fwd(b.qp, b.kp, b.vp, b.op, lse, self.shape, stream)
 
     def inverse(self, out, stream=None):
-        svsa_inverse_reorder(self.buf.op, out, self.buf.iperm, self.shape, stream)
+        if self.cocluster:
+            svsa_inverse_reorder_heads(self.buf.op, out, self.buf.iperm_q, self.shape, stream)
+        else:
+            svsa_inverse_reorder(self.buf.op, out, self.buf.iperm, self.shape, stream)
 
     # ---- one denoising step under the schedule ----------------------------
     def step(self, q, k, v, step: int, *, out=None, anchor_offset: int = 0, stream=None):
@@ -177,6 +211,8 @@ class SparseVideoAttention:
         hq, hk, hv, hout = (t.reshape(rows, self.N, self.d) for t in (q, k, v, out))
         compute = torch.cuda.current_stream()
         if not self._perm_ready:
+            if self.cocluster:
+                raise ValueError("forward_host needs the co-clustering order built first (a device call)")
             self.build_perm()
         build = not (reuse_mask and self.mask_ready)
         if build:
@@ -195,15 +231,24 @@ class SparseVideoAttention:
                     d_[r0:r1].copy_(h[r0:r1], non_blocking=True)
             compute.wait_stream(self._h2d)
             sh, m = self._group(r0, r1)
-            svsa_reorder(dq[r0:r1], self._rows(b.qp, r0, r1), b.perm, sh, compute)
-            svsa_reorder(dk[r0:r1], self._rows(b.kp, r0, r1), b.perm, sh, compute)
-            svsa_reorder_values(dv[r0:r1], self._rows(b.vp, r0, r1), b.perm, sh, compute)
+            if self.cocluster:
+                svsa_reorder_heads(dq[r0:r1], self._rows(b.qp, r0, r1), b.perm_q[r0:r1], sh, compute)
+                svsa_reorder_heads(dk[r0:r1], self._rows(b.kp, r0, r1), b.perm_k[r0:r1], sh, compute)
+                svsa_reorder_values_heads(dv[r0:r1], self._rows(b.vp, r0, r1), b.perm_k[r0:r1], sh, compute)
+            else:
+                svsa_reorder(dq[r0:r1], self._rows(b.qp, r0, r1), b.perm, sh, compute)
+                svsa_reorder(dk[r0:r1], self._rows(b.kp, r0, r1), b.perm, sh, compute)
+                svsa_reorder_values(dv[r0:r1], self._rows(b.vp, r0, r1), b.perm, sh, compute)
             if build:
                 svsa_build_mask(self._rows(b.qp, r0, r1), self._rows(b.kp, r0, r1), self._rows(b.vp, r0, r1),
-                                b.perm, sh, self.params, m, b.ws, b.ws.numel(), compute)
+                                None if self.cocluster else b.perm, sh, self.params, m, b.ws, b.ws.numel(),
+                                compute)
             svsa_attn_fwd(self._rows(b.qp, r0, r1), self._rows(b.kp, r0, r1), self._rows(b.vp, r0, r1), m,
                           self.compensate, self._rows(b.op, r0, r1), None, sh, compute)
-            svsa_inverse_reorder(self._rows(b.op, r0, r1), dout[r0:r1], b.iperm, sh, compute)
+            if self.cocluster:
+                svsa_inverse_reorder_heads(self._rows(b.op, r0, r1), dout[r0:r1], b.iperm_q[r0:r1], sh, compute)
+            else:
+                svsa_inverse_reorder(self._rows(b.op, r0, r1), dout[r0:r1], b.iperm, sh, compute)
             self._d2h.wait_stream(compute)
             with torch.cuda.stream(self._d2h):
                 hout[r0:r1].copy_(dout[r0:r1], non_blocking=True)

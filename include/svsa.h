@@ -228,6 +228,37 @@ svsa_status svsa_attn_dense_fwd(const void* qp, const void* kp, const void* vp, 
 svsa_status svsa_inverse_reorder(const void* op, void* o, const int32_t* iperm, svsa_shape s,
                                  void* stream);
 
+/* ---- step 1, data-dependent alternative: co-clustering order ------------- */
+
+/* Semantic token order by bidirectional query-key co-clustering ("Training-
+ * Free Sparse Attention for Fast Video Generation via Offline Layer-Wise
+ * Sparsity Profiling and Online Bidirectional Co-Clustering" (SVOO), 2.B:
+ * alternately group the keys by affinity to the query centroids and the
+ * queries by affinity to the updated key centroids; "SVG-EAR" 2.A: permute so
+ * that a cluster is contiguous).  Reading: per (batch, head), C = nb
+ * clusters; initial query centroids = means of the raster 64-token blocks;
+ * affinity = q . k, decided exactly (bf16 tokens, float32 centroids, fp64
+ * value; ties to the lower cluster index); a centroid is the float32 mean of
+ * its tokens, an empty cluster takes the centroid it was matched against;
+ * one round = key assignment, key centroids, query assignment, query
+ * centroids; tokens sorted by (cluster, raster index).
+ * q, k: raster bf16 [B, heads, N, d].  Writes the query order
+ * perm_q [B, heads, Npad] (raster id or -1 for a pad) / iperm_q [B, heads, N]
+ * and the key order perm_k / iperm_k (same shapes), for the *_heads gathers:
+ * Q with perm_q, K and V with perm_k, O back with iperm_q.  rounds in [1, 64];
+ * ws: svsa_cocluster_workspace_bytes(s) bytes of device memory. */
+size_t svsa_cocluster_workspace_bytes(svsa_shape s);
+svsa_status svsa_build_perm_cocluster(const void* q, const void* k, svsa_shape s, int32_t rounds,
+                                      int32_t* perm_q, int32_t* iperm_q, int32_t* perm_k, int32_t* iperm_k,
+                                      void* ws, size_t ws_bytes, void* stream);
+
+/* svsa_reorder / svsa_reorder_values / svsa_inverse_reorder with one map per
+ * (batch, head) row: perm [B, heads, Npad], iperm [B, heads, N]. */
+svsa_status svsa_reorder_heads(const void* x, void* xp, const int32_t* perm, svsa_shape s, void* stream);
+svsa_status svsa_reorder_values_heads(const void* v, void* vp, const int32_t* perm, svsa_shape s, void* stream);
+svsa_status svsa_inverse_reorder_heads(const void* op, void* o, const int32_t* iperm, svsa_shape s,
+                                       void* stream);
+
 /* ---- step schedule -------------------------------------------------------- */
 
 /* Timestep-adaptive sparsity with a cached mask ("DFSAttn: Dynamic Fine-grained

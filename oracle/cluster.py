@@ -32,6 +32,8 @@ Readings where the pages leave a step open (also listed in the design doc):
 """
 from __future__ import annotations
 
+import math
+
 import numpy as np
 
 from .order import _pad, BLOCK
@@ -49,9 +51,21 @@ def _means(x: np.ndarray, assign: np.ndarray, C: int, fallback: np.ndarray) -> n
 
 
 def _assign(x: np.ndarray, cent: np.ndarray):
-    """argmax_j x . c_j in float64 (first index on ties) and the top-2 gap."""
-    a = x @ cent.astype(np.float64).T
+    """argmax_j x . c_j (first index on ties) and the top-2 gap.  The products
+    of a bf16 and a float32 value are exact in float64; rows whose best
+    candidates lie within 1e-9 of each other (relative) are re-decided on the
+    correctly rounded exact sums (math.fsum), so that equal centroids always
+    give equal affinities."""
+    c64 = cent.astype(np.float64)
+    a = x @ c64.T
     best = np.argmax(a, axis=1)
+    top = a[np.arange(a.shape[0]), best]
+    close = a >= (top - 1e-9 * np.maximum(np.abs(top), 1.0))[:, None]
+    for t in np.nonzero(close.sum(axis=1) > 1)[0]:
+        cand = np.nonzero(close[t])[0]
+        exact = [math.fsum(x[t] * c64[j]) for j in cand]
+        a[t, cand] = exact
+        best[t] = cand[int(np.argmax(exact))]
     top = a[np.arange(a.shape[0]), best]
     if a.shape[1] > 1:
         a2 = a.copy()

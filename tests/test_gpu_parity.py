@@ -322,3 +322,68 @@ def test_lse_output():
         ref = np.log(np.exp(s - s.max(1, keepdims=True)).sum(1)) + s.max(1)
         assert np.abs(g[lo:hi] - ref).max() < 1e-3
     assert np.all(g[w.N:] == 0)
+
+
+def _cocluster_case(w, q, k, rounds=3):
+    """GPU co-clustering orders next to the oracle's, head by head."""
+    attn = svsa.SparseVideoAttention(w.B, w.heads, w.T, w.H, w.W, w.d, order="cocluster", select=w.select,
+                                     tau=w.tau, keep_frac=w.keep_frac, cluster_rounds=rounds, device="cuda")
+    attn.build_perm(q=q, k=k)
+    torch.cuda.synchronize()
+    b = attn.buf
+    qn, kn = to_np(q)[0].astype(np.float64), to_np(k)[0].astype(np.float64)
+    for eta in range(w.heads):
+        aq, ak, gq, gk = oracle.cocluster(qn[eta], kn[eta], w.N, rounds=rounds)
+        pq, ipq = oracle.perm_from_clusters(aq, w.N)
+        pk, ipk = oracle.perm_from_clusters(ak, w.N)
+        got_pq, got_pk = b.perm_q[eta].cpu().numpy(), b.perm_k[eta].cpu().numpy()
+        assert np.array_equal(got_pq, pq), f"head {eta}: query order differs at {np.nonzero(got_pq != pq)[0][:8]}"
+        assert np.array_equal(got_pk, pk), f"head {eta}: key order differs at {np.nonzero(got_pk != pk)[0][:8]}"
+        assert np.array_equal(b.iperm_q[eta].cpu().numpy(), ipq)
+        assert np.array_equal(b.iperm_k[eta].cpu().numpy(), ipk)
+    return attn
+
+
+@pytest.mark.parametrize("d,grid,heads", [(128, (6, 12, 20), 2), (64, (5, 7, 9), 2), (128, (8, 30, 52), 1)])
+def test_cocluster_order_bit_exact(d, grid, heads):
+    """Both orders (queries; keys and values) equal the oracle's bit for bit."""
+    w = _small("topk", 64, grid=grid, heads=heads, d=d, keep_frac=0.3)
+    q, k, _ = (t.cuda() for t in workloads.make_qkv(w, seed=6))
+    _cocluster_case(w, q, k)
+
+
+def test_cocluster_exact_ties_take_the_lower_cluster():
+    """Repeated tokens make equal centroids and exactly tied affinities: the
+    fp64 fix-up must give the lower cluster index, as the oracle does."""
+    w = _small("topk", 64, grid=(4, 8, 16), heads=1, d=128, keep_frac=0.3)
+    g = torch.Generator().manual_seed(7)
+    base = (torch.randn(6, 128, generator=g) * 2).to(torch.bfloat16)
+    idx = torch.randint(0, 6, (w.N,), generator=g)
+    q = base[idx][None, None].cuda()
+    k = base[torch.roll(idx, 5)][None, None].cuda()
+    _cocluster_case(w, q, k, rounds=2)
+
+
+@pytest.mark.parametrize("select", ["topk", "threshold"])
+def test_cocluster_layer_matches_oracle(select):
+    """The whole layer on the co-clustering order: masks bit-exact outside the
+    near set, outputs within tolerance, against the oracle on its own orders."""
+    w = _small(select, 64, grid=(6, 12, 20), heads=2, tau=0.9, keep_frac=0.3)
+    q, k, v = (t.cuda() for t in workloads.make_qkv(w, seed=8))
+    attn = _cocluster_case(w, q, k)
+    out = attn(q, k, v)
+    torch.cuda.synchronize()
+    keep = gpu_keep(attn)
+    qn, kn, vn = (to_np(t)[0].astype(np.float64) for t in (q, k, v))
+    on = to_np(out)[0]
+    for eta in range(w.heads):
+        aq, ak, _, _ = oracle.cocluster(qn[eta], kn[eta], w.N)
+        pq, _ = oracle.perm_from_clusters(aq, w.N)
+        pk, _ = oracle.perm_from_clusters(ak, w.N)
+        qp, kp, vp = oracle.reorder(qn[eta], pq), oracle.reorder(kn[eta], pk), oracle.reorder(vn[eta], pk)
+        kept, near = oracle_rows(w, qp, kp, vp, None, list(range(attn.nb)))
+        compare_mask_rows(keep[eta], kept, near)
+        ref = oracle.masked_attention(qp, kp, vp, w.N, keep[eta])
+        ref_raster = oracle.inverse_reorder(np.concatenate([ref[I] for I in range(attn.nb)] +
+                                                           [np.zeros((attn.Npad - w.N, w.d))]), pq, w.N)
+        check_attention(on[eta], ref_raster, f"head {eta}")
