@@ -387,3 +387,45 @@ def test_cocluster_layer_matches_oracle(select):
         ref_raster = oracle.inverse_reorder(np.concatenate([ref[I] for I in range(attn.nb)] +
                                                            [np.zeros((attn.Npad - w.N, w.d))]), pq, w.N)
         check_attention(on[eta], ref_raster, f"head {eta}")
+
+
+@pytest.mark.parametrize("grid", [(1, 1, 1), (1, 1, 64), (1, 1, 65), (2, 3, 5), (1, 8, 8)])
+@pytest.mark.parametrize("case", ["topk", "threshold", "threshold16", "routing_comp", "cocluster"])
+def test_degenerate_grids(grid, case):
+    """One token, exactly one block, one token past a block, tiny ragged grids:
+    the whole layer through every rule, masks and outputs against the oracle."""
+    d = 64 if case == "threshold16" else 128
+    sel = "topk" if case in ("topk", "cocluster") else "threshold"
+    kw = {"routing": True, "compensate": True} if case == "routing_comp" else {}
+    w = _small(sel, 16 if case == "threshold16" else 64, grid=grid, heads=2, d=d, tau=0.9, keep_frac=0.3, **kw)
+    q, k, v = (t.cuda() for t in workloads.make_qkv(w, seed=9))
+    if case == "cocluster":
+        attn = _cocluster_case(w, q, k)
+        out = attn(q, k, v)
+    else:
+        attn = gpu_layer(w, q, k, v)
+        out = attn.out
+    torch.cuda.synchronize()
+    keep = gpu_keep(attn)
+    qn, kn, vn = (to_np(t)[0].astype(np.float64) for t in (q, k, v))
+    on = to_np(out)[0]
+    b = attn.buf
+    for eta in range(w.heads):
+        if case == "cocluster":
+            aq, ak, _, _ = oracle.cocluster(qn[eta], kn[eta], w.N)
+            pq, _ = oracle.perm_from_clusters(aq, w.N)
+            pk, _ = oracle.perm_from_clusters(ak, w.N)
+        else:
+            pq, _ = oracle.build_perm(w.T, w.H, w.W, w.order)
+            pk = pq
+        qp, kp, vp = oracle.reorder(qn[eta], pq), oracle.reorder(kn[eta], pk), oracle.reorder(vn[eta], pk)
+        kept, near = oracle_rows(w, qp, kp, vp, pq, list(range(attn.nb)))
+        compare_mask_rows(keep[eta], kept, near)
+        if w.compensate:
+            kb, n = oracle.pool(kp, w.N)
+            vb, _ = oracle.pool(vp, w.N)
+            ref = oracle.compensated_attention(qp, kp, vp, w.N, keep[eta], kb, vb, n)
+        else:
+            ref = oracle.masked_attention(qp, kp, vp, w.N, keep[eta])
+        full = np.concatenate([ref[I] for I in range(attn.nb)] + [np.zeros((attn.Npad - w.N, w.d))])
+        check_attention(on[eta], oracle.inverse_reorder(full, pq, w.N), f"{case} {grid} head {eta}")
