@@ -45,6 +45,7 @@ def _args():
     ap.add_argument("--impl", default="svsa", choices=["svsa", "reference"])
     ap.add_argument("--workload", default="wan13b", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--order", default=None, choices=["raster", "hilbert", "cocluster"])
+    ap.add_argument("--heads", type=int, default=None, help="override the layer's head count (profiling captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--schedule", default=None, metavar="N,DENSE,START,END,EVERY",
@@ -97,6 +98,8 @@ def _workload(args):
     w = workloads.WORKLOADS[args.workload]
     if args.order:
         w = w.with_(order=args.order)
+    if args.heads:
+        w = w.with_(heads=args.heads)
     return w
 
 
