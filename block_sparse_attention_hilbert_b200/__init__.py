@@ -89,6 +89,7 @@ _SIGS = {
                                                   ctypes.c_void_p]),
     "svsa_schedule_step": (ctypes.c_int, [ctypes.POINTER(Schedule), ctypes.c_int32, ctypes.POINTER(MaskParams),
                                           ctypes.POINTER(MaskParams), ctypes.POINTER(ctypes.c_int32)]),
+    "svsa_selftest_timeout": (ctypes.c_int, [ctypes.c_int32, ctypes.c_void_p]),
     "svsa_sync_status": (ctypes.c_int, [ctypes.c_void_p]),
     "svsa_last_error": (ctypes.c_char_p, []),
     "svsa_version": (ctypes.c_char_p, []),

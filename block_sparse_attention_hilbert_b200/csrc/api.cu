@@ -7,6 +7,8 @@
 #include <cstdio>
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 #include "svsa.h"
 
@@ -52,6 +54,7 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, const in
                            const int32_t* kv_cnt, int cap, const uint32_t* bits, const void* cbar, void* o,
                            float* lse, long long BH, long long N, int nb, int d, bool dense, cudaStream_t st);
 cudaError_t attn_tc_error(unsigned int* code, cudaStream_t st);
+cudaError_t launch_selftest_timeout(unsigned long long budget_ns, cudaStream_t st);
 cudaError_t scores_tc_error(unsigned int* code, cudaStream_t st);
 }  // namespace svsa
 
@@ -191,9 +194,17 @@ int topk_count(float keep_frac, int nb) {
 }  // namespace
 
 namespace {
+// NVTX range around a public call: the calls appear by name in a timeline
+// profiler; without one attached the push / pop cost nothing measurable.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+
 // The row gathers of steps 2 and 4; per_head: the map holds one row per (batch, head).
 svsa_status gather(const void* src, void* dst, const int32_t* map, svsa_shape s, bool forward, bool to_f16,
                    bool per_head, void* stream, const char* what) {
+  NvtxRange nvtx_(what);
   g_last_error.clear();
   SVSA_TRY(check_shape(s, true));
   SVSA_PTR(src, "input");
@@ -227,6 +238,7 @@ size_t svsa_perm_workspace_bytes(svsa_shape s, int32_t order) {
 
 svsa_status svsa_build_perm(svsa_shape s, int32_t order, int32_t* perm, int32_t* iperm, void* ws,
                             size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_("svsa_build_perm");
   g_last_error.clear();
   SVSA_TRY(check_shape(s, false));
   if (order != SVSA_ORDER_RASTER && order != SVSA_ORDER_HILBERT)
@@ -247,6 +259,7 @@ svsa_status svsa_build_perm(svsa_shape s, int32_t order, int32_t* perm, int32_t*
 }
 
 svsa_status svsa_build_perm_noalloc(svsa_shape s, int32_t order, int32_t* perm, int32_t* iperm, void* stream) {
+  NvtxRange nvtx_("svsa_build_perm_noalloc");
   g_last_error.clear();
   SVSA_TRY(check_shape(s, false));
   if (order != SVSA_ORDER_RASTER && order != SVSA_ORDER_HILBERT)
@@ -301,6 +314,7 @@ size_t svsa_cocluster_workspace_bytes(svsa_shape s) {
 svsa_status svsa_build_perm_cocluster(const void* q, const void* k, svsa_shape s, int32_t rounds, int32_t* perm_q,
                                       int32_t* iperm_q, int32_t* perm_k, int32_t* iperm_k, void* ws, size_t ws_bytes,
                                       void* stream) {
+  NvtxRange nvtx_("svsa_build_perm_cocluster");
   g_last_error.clear();
   SVSA_TRY(check_shape(s, true));
   SVSA_PTR(q, "q");
@@ -332,6 +346,7 @@ size_t svsa_mask_workspace_bytes(svsa_shape s, const svsa_mask_params* p) {
 svsa_status svsa_build_mask(const void* qp, const void* kp, const void* vp, const int32_t* perm,
                             svsa_shape s, const svsa_mask_params* p, const svsa_mask* m, void* ws,
                             size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_("svsa_build_mask");
   g_last_error.clear();
   SVSA_TRY(check_shape(s, true));
   const Dims g = make_dims(s.B, s.heads, s.T, s.H, s.W, s.d);
@@ -432,6 +447,7 @@ svsa_status svsa_build_mask(const void* qp, const void* kp, const void* vp, cons
 
 svsa_status svsa_attn_fwd(const void* qp, const void* kp, const void* vp, const svsa_mask* m,
                           int32_t compensate, void* op, float* lse, svsa_shape s, void* stream) {
+  NvtxRange nvtx_("svsa_attn_fwd");
   g_last_error.clear();
   SVSA_TRY(check_shape(s, true));
   const Dims g = make_dims(s.B, s.heads, s.T, s.H, s.W, s.d);
@@ -464,6 +480,7 @@ svsa_status svsa_attn_fwd(const void* qp, const void* kp, const void* vp, const 
 
 svsa_status svsa_attn_dense_fwd(const void* qp, const void* kp, const void* vp, void* op, float* lse,
                                 svsa_shape s, void* stream) {
+  NvtxRange nvtx_("svsa_attn_dense_fwd");
   g_last_error.clear();
   SVSA_TRY(check_shape(s, true));
   const Dims g = make_dims(s.B, s.heads, s.T, s.H, s.W, s.d);
@@ -509,7 +526,16 @@ svsa_status svsa_schedule_step(const svsa_schedule* sch, int32_t step, const svs
   return SVSA_OK;
 }
 
+svsa_status svsa_selftest_timeout(int32_t wait_us, void* stream) {
+  NvtxRange nvtx_("svsa_selftest_timeout");
+  g_last_error.clear();
+  if (wait_us < 1 || wait_us > 1000000) return fail(SVSA_ERR_INVALID_ARG, "wait_us=%d outside [1, 1e6]", wait_us);
+  return cuda_status(counted(launch_selftest_timeout((unsigned long long)wait_us * 1000ull, (cudaStream_t)stream), 1),
+                     "selftest launch");
+}
+
 svsa_status svsa_sync_status(void* stream) {
+  NvtxRange nvtx_("svsa_sync_status");
   g_last_error.clear();
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_status(e, "stream synchronize");

@@ -618,6 +618,28 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, const in
   return cudaErrorInvalidValue;
 }
 
+// Self-test of the failure path: one thread waits on a barrier that nothing
+// arrives at, gives up after `budget_ns` and records site 90 in the error
+// word, as every bounded wait of the kernels does.  No fault, no trap.
+__global__ void selftest_wait_kernel(unsigned long long budget_ns) {
+  __shared__ uint64_t b;
+  const uint32_t bar = tc::su32(&b);
+  tc::mbar_init(bar, 1);
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  const unsigned long long t0 = tc::gtimer();
+  while (!tc::mbar_try_wait(bar, 0u)) {
+    if (tc::gtimer() - t0 > budget_ns) {
+      atomicCAS(&tc::g_tc_error, 0u, 90u);
+      return;
+    }
+  }
+}
+
+cudaError_t launch_selftest_timeout(unsigned long long budget_ns, cudaStream_t st) {
+  selftest_wait_kernel<<<1, 1, 0, st>>>(budget_ns);
+  return cudaGetLastError();
+}
+
 // Read and clear this kernel's device error word (0 = no failure).
 cudaError_t attn_tc_error(unsigned int* code, cudaStream_t st) { return tc::read_error(code, st); }
 

@@ -296,6 +296,13 @@ svsa_status svsa_schedule_step(const svsa_schedule* sch, int32_t step, const svs
  * an asynchronous CUDA error -> SVSA_ERR_CUDA).  Clears the recorded flags. */
 svsa_status svsa_sync_status(void* stream);
 
+/* Self-test of the failure path: launches a one-thread kernel whose bounded
+ * wait on a barrier that nothing arrives at gives up after wait_us
+ * microseconds (in [1, 1e6]) and records the failure the way every bounded
+ * wait of the library does; the next svsa_sync_status then reports
+ * SVSA_ERR_TIMEOUT (and clears it).  Nothing faults, traps or hangs. */
+svsa_status svsa_selftest_timeout(int32_t wait_us, void* stream);
+
 /* Message for the last failure on the calling thread ("" if none). */
 const char* svsa_last_error(void);
 
