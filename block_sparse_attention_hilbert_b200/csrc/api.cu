@@ -52,7 +52,12 @@ cudaError_t launch_centroid16(const float* kbar, const float* vbar, void* cbar, 
                               cudaStream_t st);
 cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, const int32_t* kv_idx,
                            const int32_t* kv_cnt, int cap, const uint32_t* bits, const void* cbar, void* o,
-                           float* lse, long long BH, long long N, int nb, int d, bool dense, cudaStream_t st);
+                           float* lse, long long BH, long long N, int nb, int d, bool dense, cudaStream_t st,
+                           float* o32 = nullptr, float lse_empty = 0.f);
+cudaError_t launch_split_mask(const int32_t* kv_idx, const int32_t* kv_cnt, int cap, long long rows, int nb, int P,
+                              int R, int32_t* idx_p, int32_t* cnt_p, cudaStream_t st);
+cudaError_t launch_combine(const float* o_p, const float* lse_p, long long rows, int P, int d, void* out,
+                           float* lse_out, cudaStream_t st);
 cudaError_t attn_tc_error(unsigned int* code, cudaStream_t st);
 cudaError_t launch_selftest_timeout(unsigned long long budget_ns, cudaStream_t st);
 cudaError_t scores_tc_error(unsigned int* code, cudaStream_t st);
@@ -476,6 +481,87 @@ svsa_status svsa_attn_fwd(const void* qp, const void* kp, const void* vp, const 
                                             compensate ? m->cbar : nullptr, op, lse, g.BH, g.N, g.nb, g.d, false,
                                             (cudaStream_t)stream), 1),
                      "attn_fwd launch");
+}
+
+namespace {
+struct SplitWs {
+  size_t idx, cnt, o, lse, total;
+};
+SplitWs split_layout(const Dims& g, int P) {
+  SplitWs w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off += (bytes + 255) & ~(size_t)255; return o; };
+  const long long rows = g.BH * g.nb;
+  const int R = (g.nb + P - 1) / P;
+  w.idx = take((size_t)P * rows * R * 4);
+  w.cnt = take((size_t)P * rows * 4);
+  w.o = take((size_t)P * g.BH * g.Npad * g.d * 4);
+  w.lse = take((size_t)P * g.BH * g.Npad * 4);
+  w.total = off;
+  return w;
+}
+}  // namespace
+
+size_t svsa_attn_split_workspace_bytes(svsa_shape s, int32_t passes) {
+  if (passes < 2 || passes > 8 || s.T < 1 || s.H < 1 || s.W < 1 || s.B < 1 || s.heads < 1) return 0;
+  const Dims g = make_dims(s.B, s.heads, s.T, s.H, s.W, s.d);
+  return split_layout(g, passes).total;
+}
+
+svsa_status svsa_attn_fwd_split(const void* qp, const void* kp, const void* vp, const svsa_mask* m,
+                                int32_t compensate, void* op, float* lse, svsa_shape s, int32_t passes, void* ws,
+                                size_t ws_bytes, void* stream) {
+  if (passes == 1) return svsa_attn_fwd(qp, kp, vp, m, compensate, op, lse, s, stream);
+  NvtxRange nvtx_("svsa_attn_fwd_split");
+  g_last_error.clear();
+  if (passes < 1 || passes > 8) return fail(SVSA_ERR_INVALID_ARG, "passes=%d outside [1, 8]", passes);
+  SVSA_TRY(check_shape(s, true));
+  const Dims g = make_dims(s.B, s.heads, s.T, s.H, s.W, s.d);
+  SVSA_PTR(qp, "qp");
+  SVSA_PTR(kp, "kp");
+  SVSA_PTR(vp, "vp");
+  SVSA_PTR(op, "op");
+  SVSA_PTR(ws, "ws");
+  if (m == nullptr) return fail(SVSA_ERR_INVALID_ARG, "mask is NULL");
+  SVSA_PTR(m->kv_idx, "mask.kv_idx");
+  SVSA_PTR(m->kv_cnt, "mask.kv_cnt");
+  if (m->cap < 1) return fail(SVSA_ERR_INVALID_ARG, "mask.cap=%d", m->cap);
+  if (lse != nullptr && !aligned16(lse)) return fail(SVSA_ERR_INVALID_ARG, "lse misaligned");
+  if (g.nb > kMaxBlocks) return fail(SVSA_ERR_UNSUPPORTED, "nb=%d exceeds %d", g.nb, kMaxBlocks);
+  if (compensate) {
+    SVSA_PTR(m->kbar, "mask.kbar (compensation)");
+    SVSA_PTR(m->vbar, "mask.vbar (compensation)");
+    SVSA_PTR(m->bits, "mask.bits (compensation)");
+    SVSA_PTR(m->cbar, "mask.cbar (compensation)");
+  }
+  if (op == qp || op == kp || op == vp) return fail(SVSA_ERR_INVALID_ARG, "op must not alias an input");
+  const SplitWs w = split_layout(g, passes);
+  if (ws_bytes < w.total) return fail(SVSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, w.total);
+  cudaStream_t st = (cudaStream_t)stream;
+  char* base = reinterpret_cast<char*>(ws);
+  int32_t* idx_p = reinterpret_cast<int32_t*>(base + w.idx);
+  int32_t* cnt_p = reinterpret_cast<int32_t*>(base + w.cnt);
+  float* o_p = reinterpret_cast<float*>(base + w.o);
+  float* lse_p = reinterpret_cast<float*>(base + w.lse);
+  const long long rows = g.BH * g.nb;
+  const int R = (g.nb + passes - 1) / passes;
+  if (compensate)
+    SVSA_TRY(cuda_status(counted(launch_centroid16(m->kbar, m->vbar, m->cbar, g.BH * g.nb, g.d, st), 1),
+                         "centroid copies"));
+  SVSA_TRY(cuda_status(counted(launch_split_mask(m->kv_idx, m->kv_cnt, m->cap, rows, g.nb, passes, R, idx_p, cnt_p,
+                                                 st), 1),
+                       "split mask"));
+  for (int p = 0; p < passes; ++p) {
+    // the centroid tiles of the skipped blocks go with the last pass
+    const bool comp = compensate && p + 1 == passes;
+    SVSA_TRY(cuda_status(counted(launch_attn_tc(qp, kp, vp, idx_p + (long long)p * rows * R, cnt_p + (long long)p * rows,
+                                                 R, comp ? m->bits : nullptr, comp ? m->cbar : nullptr, nullptr,
+                                                 lse_p + (long long)p * g.BH * g.Npad, g.BH, g.N, g.nb, g.d, false, st,
+                                                 o_p + (long long)p * g.BH * g.Npad * g.d, -INFINITY), 1),
+                         "attn_fwd pass launch"));
+  }
+  return cuda_status(counted(launch_combine(o_p, lse_p, g.BH * g.Npad, passes, g.d, op, lse, st), 1),
+                     "combine launch");
 }
 
 svsa_status svsa_attn_dense_fwd(const void* qp, const void* kp, const void* vp, void* op, float* lse,

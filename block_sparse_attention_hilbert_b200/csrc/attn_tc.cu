@@ -106,7 +106,9 @@ struct Args {
   int nwords;             // words per bitmap row
   int ncent;              // centroid tiles per item (0 = no compensation)
   __nv_bfloat16* o;
+  float* o32;              // non-null: fp32 output (a key-range pass of a split launch) instead of bf16
   float* lse;
+  float lse_empty;         // lse of a row with no kept key: 0, or -inf for a split pass
   long long N, Npad;
   int nb;
   long long items;
@@ -142,7 +144,7 @@ __device__ __forceinline__ float warp_colreduce(float* v) {
 }
 
 // ---------------------------------------------------------------- the kernel
-template <int D, bool COMP>
+template <int D, bool COMP, bool O32>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                               const __grid_constant__ CUtensorMap tmK,
                                                               const __grid_constant__ CUtensorMap tmV,
@@ -392,9 +394,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const int npairs = (cnt + 1) >> 1;
       const int ntiles = npairs + ncent;
       if (ntiles == 0) {
-        for (int i = st; i < kCols * CPR; i += kSoftmaxThreads)
-          reinterpret_cast<uint4*>(og)[i] = make_uint4(0u, 0u, 0u, 0u);
-        if (a.lse != nullptr && st < kCols) a.lse[bh * a.Npad + q0 + cb + st] = 0.f;
+        if (O32) {
+          float* og32 = a.o32 + (bh * a.Npad + q0 + cb) * D;
+          for (int i = st; i < kCols * D / 4; i += kSoftmaxThreads)
+            reinterpret_cast<float4*>(og32)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        } else {
+          for (int i = st; i < kCols * CPR; i += kSoftmaxThreads)
+            reinterpret_cast<uint4*>(og)[i] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        if (a.lse != nullptr && st < kCols) a.lse[bh * a.Npad + q0 + cb + st] = a.lse_empty;
         continue;
       }
       const int32_t* lst = a.dense ? nullptr : a.kv_idx + it * a.cap;
@@ -538,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         if (a.lse != nullptr) {
           const float ln2 = 0.6931471805599453f;
           const long long q = q0 + cb + st;
-          a.lse[bh * a.Npad + q] = (q < a.N && l > 0.f) ? (mcol[st] + __log2f(l)) * ln2 : 0.f;
+          a.lse[bh * a.Npad + q] = (q < a.N && l > 0.f) ? (mcol[st] + __log2f(l)) * ln2 : a.lse_empty;
         }
       }
       wait_bar(bar(BAR_O_FULL), oit & 1u, abort_flag, 13);
@@ -555,10 +563,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(BAR_O_EMPTY));
         if (k < D) {
+          if (O32) {
+            float* og32 = a.o32 + (bh * a.Npad + q0 + cb) * D;
 #pragma unroll
-          for (int c = 0; c < kCols; ++c) {
-            const bool row_ok = q0 + cb + c < a.N;
-            og[(long long)c * D + k] = __float2bfloat16_rn(row_ok ? o[c] * fcol[c] : 0.f);
+            for (int c = 0; c < kCols; ++c) {
+              const bool row_ok = q0 + cb + c < a.N;
+              og32[(long long)c * D + k] = row_ok ? o[c] * fcol[c] : 0.f;
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < kCols; ++c) {
+              const bool row_ok = q0 + cb + c < a.N;
+              og[(long long)c * D + k] = __float2bfloat16_rn(row_ok ? o[c] * fcol[c] : 0.f);
+            }
           }
         }
       }
@@ -588,7 +605,8 @@ bool make_map(CUtensorMap* m, const void* base, long long rows, int d, bool f16)
 
 cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, const int32_t* kv_idx,
                            const int32_t* kv_cnt, int cap, const uint32_t* bits, const void* cbar, void* o,
-                           float* lse, long long BH, long long N, int nb, int d, bool dense, cudaStream_t st) {
+                           float* lse, long long BH, long long N, int nb, int d, bool dense, cudaStream_t st,
+                           float* o32, float lse_empty) {
   CUtensorMap mq, mk, mv, mc;
   const long long rows = BH * (long long)nb * kBlock;
   if (!make_map(&mq, q, rows, d, false) || !make_map(&mk, k, rows, d, false) || !make_map(&mv, v, rows, d, true))
@@ -601,6 +619,7 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, const in
   a.bits = bits; a.nwords = (nb + 31) / 32;
   a.ncent = cbar != nullptr ? (nb + 127) / 128 : 0;
   a.o = (__nv_bfloat16*)o; a.lse = lse;
+  a.o32 = o32; a.lse_empty = lse_empty;
   a.N = N; a.nb = nb; a.Npad = (long long)nb * kBlock;
   a.items = BH * nb;
   a.scale_log2 = 1.4426950408889634f / sqrtf((float)d);
@@ -613,8 +632,15 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, const in
     kernel<<<(unsigned)grid, tc::kThreads, tc::kSmemBytes, st>>>(mq, mk, mv, mc, a);
     return cudaGetLastError();
   };
-  if (d == 128) return comp ? go(tc::attn_tc_kernel<128, true>) : go(tc::attn_tc_kernel<128, false>);
-  if (d == 64) return comp ? go(tc::attn_tc_kernel<64, true>) : go(tc::attn_tc_kernel<64, false>);
+  const bool split = o32 != nullptr;
+  if (d == 128) {
+    if (split) return comp ? go(tc::attn_tc_kernel<128, true, true>) : go(tc::attn_tc_kernel<128, false, true>);
+    return comp ? go(tc::attn_tc_kernel<128, true, false>) : go(tc::attn_tc_kernel<128, false, false>);
+  }
+  if (d == 64) {
+    if (split) return comp ? go(tc::attn_tc_kernel<64, true, true>) : go(tc::attn_tc_kernel<64, false, true>);
+    return comp ? go(tc::attn_tc_kernel<64, true, false>) : go(tc::attn_tc_kernel<64, false, false>);
+  }
   return cudaErrorInvalidValue;
 }
 

@@ -1,0 +1,114 @@
+// Key-range passes for layers whose keys and values outgrow L2.
+//
+// The attention of a query block over its kept key blocks is split into P
+// passes over the key-block ranges [p * R, (p + 1) * R), R = ceil(nb / P):
+// each pass is an exact attention over the kept blocks of its range and
+// yields O_p (fp32, normalised within the pass) and its log-sum-exp lse_p;
+// then
+//     lse = log sum_p exp(lse_p),    O = sum_p exp(lse_p - lse) O_p
+// is the attention over all kept blocks (the softmax over a union of
+// disjoint key sets).  A pass touches 1 / P of a head's keys and values, so
+// that working set stays in L2 while the query blocks stream.
+//
+// split_mask_kernel cuts every ascending kept list into its P range lists
+// (each at most R long, so the P masks together take the room of one);
+// combine_kernel merges the passes.
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+
+namespace svsa {
+namespace {
+
+constexpr int kWarps = 8;
+
+// One warp per (bh, query block) row.  Lists are ascending: the entries of
+// range p are a contiguous run starting at the count of entries below p * R.
+__global__ void split_mask_kernel(const int32_t* __restrict__ kv_idx, const int32_t* __restrict__ kv_cnt, int cap,
+                                  long long rows, int nb, int P, int R, int32_t* __restrict__ idx_p,
+                                  int32_t* __restrict__ cnt_p) {
+  const long long row = (long long)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const int c0 = kv_cnt[row];
+  const int cnt = c0 < 0 ? 0 : (c0 > cap ? cap : c0);
+  const int32_t* lst = kv_idx + row * (long long)cap;
+  // start[p] = entries with J < p * R (ascending lists)
+  int below[9];
+#pragma unroll
+  for (int p = 0; p <= 8; ++p) below[p] = 0;
+  for (int e = lane; e < cnt; e += 32) {
+    int J = lst[e];
+    J = J < 0 ? 0 : (J >= nb ? nb - 1 : J);
+    const int pe = J / R;
+#pragma unroll
+    for (int p = 1; p <= 8; ++p)
+      if (p <= P && pe < p) ++below[p];
+  }
+#pragma unroll
+  for (int p = 1; p <= 8; ++p) below[p] = (int)warp_sum((float)below[p]);
+  for (int p = 0; p < P; ++p) {
+    const int s = p == 0 ? 0 : below[p];
+    const int t = p + 1 == P ? cnt : below[p + 1];
+    if (lane == 0) cnt_p[(long long)p * rows + row] = t - s;
+    for (int e = s + lane; e < t; e += 32) {
+      int J = lst[e];
+      J = J < 0 ? 0 : (J >= nb ? nb - 1 : J);
+      const int pos = e - s;
+      if (pos < R) idx_p[((long long)p * rows + row) * R + pos] = J;
+    }
+  }
+}
+
+// One warp per output row: O = sum_p exp(lse_p - lse) O_p, lse = log sum exp(lse_p).
+template <int D>
+__global__ void combine_kernel(const float* __restrict__ o_p, const float* __restrict__ lse_p, long long rows, int P,
+                               __nv_bfloat16* __restrict__ out, float* __restrict__ lse_out) {
+  const long long row = (long long)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  float m = -INFINITY;
+  for (int p = 0; p < P; ++p) m = fmaxf(m, lse_p[(long long)p * rows + row]);
+  constexpr int U = D / 32;
+  float acc[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) acc[u] = 0.f;
+  float wsum = 0.f;
+  if (m > -INFINITY) {
+    for (int p = 0; p < P; ++p) {
+      const float l = lse_p[(long long)p * rows + row];
+      if (l == -INFINITY) continue;
+      const float w = __expf(l - m);
+      wsum += w;
+      const float* src = o_p + ((long long)p * rows + row) * D;
+#pragma unroll
+      for (int u = 0; u < U; ++u) acc[u] = fmaf(w, src[lane + 32 * u], acc[u]);
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+  for (int u = 0; u < U; ++u) out[row * D + lane + 32 * u] = __float2bfloat16_rn(acc[u] * inv);
+  if (lse_out != nullptr && lane == 0) lse_out[row] = wsum > 0.f ? m + __logf(wsum) : 0.f;
+}
+
+}  // namespace
+
+cudaError_t launch_split_mask(const int32_t* kv_idx, const int32_t* kv_cnt, int cap, long long rows, int nb, int P,
+                              int R, int32_t* idx_p, int32_t* cnt_p, cudaStream_t st) {
+  if (P < 1 || P > 8) return cudaErrorInvalidValue;
+  split_mask_kernel<<<(unsigned)((rows + kWarps - 1) / kWarps), 32 * kWarps, 0, st>>>(kv_idx, kv_cnt, cap, rows, nb,
+                                                                                       P, R, idx_p, cnt_p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const float* o_p, const float* lse_p, long long rows, int P, int d, void* out,
+                           float* lse_out, cudaStream_t st) {
+  const unsigned blocks = (unsigned)((rows + kWarps - 1) / kWarps);
+  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
+  if (d == 128) combine_kernel<128><<<blocks, 32 * kWarps, 0, st>>>(o_p, lse_p, rows, P, o, lse_out);
+  else if (d == 64) combine_kernel<64><<<blocks, 32 * kWarps, 0, st>>>(o_p, lse_p, rows, P, o, lse_out);
+  else return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+}  // namespace svsa

@@ -26,7 +26,8 @@ from . import (ORDER_HILBERT, ORDER_RASTER, SEL_STRUCTURED, SEL_THRESHOLD, SEL_T
                svsa_build_mask, svsa_build_perm, svsa_build_perm_cocluster, svsa_cocluster_workspace_bytes,
                svsa_inverse_reorder, svsa_inverse_reorder_heads, svsa_mask_workspace_bytes,
                svsa_perm_workspace_bytes, svsa_reorder, svsa_reorder_heads, svsa_reorder_values,
-               svsa_reorder_values_heads, svsa_schedule_step)
+               svsa_reorder_values_heads, svsa_schedule_step, svsa_attn_fwd_split,
+               svsa_attn_split_workspace_bytes)
 
 _ORDERS = {"raster": ORDER_RASTER, "hilbert": ORDER_HILBERT}
 _SELECTS = {"threshold": SEL_THRESHOLD, "topk": SEL_TOPK, "structured": SEL_STRUCTURED}
@@ -71,11 +72,15 @@ class LayerBuffers:
 class SparseVideoAttention:
     def __init__(self, B, heads, T, H, W, d, *, order="hilbert", select="threshold", tau=0.9,
                  keep_frac=0.25, sub_block=64, win_t=2, win_rows=1, n_anchors=0, routing=False,
-                 compensate=False, keep_bits=False, schedule=None, cluster_rounds=3, device="cuda"):
+                 compensate=False, keep_bits=False, schedule=None, cluster_rounds=3, attn_passes=None,
+                 device="cuda"):
         """order: "raster", "hilbert" or "cocluster" (a per-head semantic order from
         bidirectional query-key co-clustering, built from the first inputs and
         kept until `rebuild_order()`).  schedule: optional (n_steps, dense_steps,
-        start, end, refresh_every) -- a timestep-adaptive rule for `step()`."""
+        start, end, refresh_every) -- a timestep-adaptive rule for `step()`.
+        attn_passes: key-range passes of the attention (svsa_attn_fwd_split); by
+        default 1 while a head's reordered K and V (Npad * d * 4 bytes) fit in
+        48 MB of L2, else enough passes for at most 64 MB each (at most 8)."""
         self.B, self.heads, self.T, self.H, self.W, self.d = B, heads, T, H, W, d
         self.N = T * H * W
         self.nb = -(-self.N // BLOCK)
@@ -100,6 +105,13 @@ class SparseVideoAttention:
                                 perm_ws_bytes=svsa_perm_workspace_bytes(self.shape, self.order),
                                 device=device, compensate=self.compensate)
         self._mask = self.buf.mask()
+        kv_bytes = self.Npad * d * 4
+        if attn_passes is None:
+            attn_passes = 1 if kv_bytes <= 48 * 2**20 else min(8, -(-kv_bytes // (64 * 2**20)))
+        self.attn_passes = int(attn_passes)
+        self.buf.split_ws = (torch.empty(svsa_attn_split_workspace_bytes(self.shape, self.attn_passes),
+                                         dtype=torch.uint8, device=self.buf.qp.device)
+                             if self.attn_passes > 1 else None)
         if self.cocluster:
             rows, dev = B * heads, self.buf.qp.device
             b = self.buf
@@ -149,7 +161,11 @@ class SparseVideoAttention:
 
     def attend(self, lse=None, stream=None):
         b = self.buf
-        svsa_attn_fwd(b.qp, b.kp, b.vp, self._mask, self.compensate, b.op, lse, self.shape, stream)
+        if self.attn_passes > 1:
+            svsa_attn_fwd_split(b.qp, b.kp, b.vp, self._mask, self.compensate, b.op, lse, self.shape,
+                                self.attn_passes, b.split_ws, b.split_ws.numel(), stream)
+        else:
+            svsa_attn_fwd(b.qp, b.kp, b.vp, self._mask, self.compensate, b.op, lse, self.shape, stream)
 
     def attend_dense(self, lse=None, stream=None):
         b = self.buf
@@ -243,8 +259,13 @@ class SparseVideoAttention:
                 svsa_build_mask(self._rows(b.qp, r0, r1), self._rows(b.kp, r0, r1), self._rows(b.vp, r0, r1),
                                 None if self.cocluster else b.perm, sh, self.params, m, b.ws, b.ws.numel(),
                                 compute)
-            svsa_attn_fwd(self._rows(b.qp, r0, r1), self._rows(b.kp, r0, r1), self._rows(b.vp, r0, r1), m,
-                          self.compensate, self._rows(b.op, r0, r1), None, sh, compute)
+            if self.attn_passes > 1:
+                svsa_attn_fwd_split(self._rows(b.qp, r0, r1), self._rows(b.kp, r0, r1), self._rows(b.vp, r0, r1), m,
+                                    self.compensate, self._rows(b.op, r0, r1), None, sh, self.attn_passes,
+                                    b.split_ws, b.split_ws.numel(), compute)
+            else:
+                svsa_attn_fwd(self._rows(b.qp, r0, r1), self._rows(b.kp, r0, r1), self._rows(b.vp, r0, r1), m,
+                              self.compensate, self._rows(b.op, r0, r1), None, sh, compute)
             if self.cocluster:
                 svsa_inverse_reorder_heads(self._rows(b.op, r0, r1), dout[r0:r1], b.iperm_q[r0:r1], sh, compute)
             else:

@@ -216,6 +216,21 @@ svsa_status svsa_build_mask(const void* qp, const void* kp, const void* vp, cons
 svsa_status svsa_attn_fwd(const void* qp, const void* kp, const void* vp, const svsa_mask* m,
                           int32_t compensate, void* op, float* lse, svsa_shape s, void* stream);
 
+/* svsa_attn_fwd in `passes` key-range passes, for layers whose keys and
+ * values outgrow L2: pass p attends over the kept key blocks in
+ * [p * R, (p + 1) * R), R = ceil(nb / passes), and yields an fp32 output
+ * normalised within the pass with its log-sum-exp; the passes are merged as
+ * O = sum_p exp(lse_p - lse) O_p, lse = log sum_p exp(lse_p) (the softmax over
+ * the union of disjoint key sets), so the result is svsa_attn_fwd's up to
+ * rounding.  Compensation terms go with the last pass.  kv_idx rows must be
+ * ascending (as svsa_build_mask writes them).  passes in [1, 8] (1 = a plain
+ * svsa_attn_fwd call, no workspace needed); ws: device memory of
+ * svsa_attn_split_workspace_bytes(s, passes) bytes. */
+size_t svsa_attn_split_workspace_bytes(svsa_shape s, int32_t passes);
+svsa_status svsa_attn_fwd_split(const void* qp, const void* kp, const void* vp, const svsa_mask* m,
+                                int32_t compensate, void* op, float* lse, svsa_shape s, int32_t passes, void* ws,
+                                size_t ws_bytes, void* stream);
+
 /* Dense attention over all N keys, same arithmetic and layouts as
  * svsa_attn_fwd; the denominator of the speedup the benchmark reports. */
 svsa_status svsa_attn_dense_fwd(const void* qp, const void* kp, const void* vp, void* op,

@@ -429,3 +429,43 @@ def test_degenerate_grids(grid, case):
             ref = oracle.masked_attention(qp, kp, vp, w.N, keep[eta])
         full = np.concatenate([ref[I] for I in range(attn.nb)] + [np.zeros((attn.Npad - w.N, w.d))])
         check_attention(on[eta], oracle.inverse_reorder(full, pq, w.N), f"{case} {grid} head {eta}")
+
+
+@pytest.mark.parametrize("passes,select,kw", [
+    (2, "topk", {}),
+    (3, "threshold", {"routing": True, "compensate": True}),
+    (5, "threshold", {"sub": 16}),
+])
+def test_split_attention_matches_single_pass_and_oracle(passes, select, kw):
+    """Key-range passes merged by log-sum-exp: the output and the lse agree with
+    the single-pass call (up to rounding) and with the oracle."""
+    sub = kw.pop("sub", 64)
+    w = _small(select, sub, grid=(6, 12, 20), heads=2, tau=0.9, keep_frac=0.3, **kw)
+    q, k, v = (t.cuda() for t in workloads.make_qkv(w, seed=12))
+    mk = lambda p: svsa.SparseVideoAttention(w.B, w.heads, w.T, w.H, w.W, w.d, order=w.order, select=select,
+                                             tau=w.tau, keep_frac=w.keep_frac, sub_block=sub, routing=w.routing,
+                                             compensate=w.compensate, keep_bits=True, attn_passes=p, device="cuda")
+    one, many = mk(1), mk(passes)
+    one.reorder(q, k, v); one.build_mask()
+    many.reorder(q, k, v); many.build_mask()
+    lse1 = torch.empty(1, w.heads, one.Npad, dtype=torch.float32, device="cuda")
+    lsep = torch.empty_like(lse1)
+    one.attend(lse=lse1); many.attend(lse=lsep)
+    torch.cuda.synchronize()
+    assert np.array_equal(gpu_keep(one), gpu_keep(many))
+    a1, ap = to_np(one.buf.op)[0], to_np(many.buf.op)[0]
+    assert np.abs(a1 - ap).max() <= 2 * 2 ** -8 * max(1.0, np.abs(a1).max())       # two bf16 roundings apart at most
+    valid = np.arange(one.Npad) < w.N
+    assert np.allclose(to_np(lse1)[0][:, valid], to_np(lsep)[0][:, valid], atol=1e-4)
+    keep = gpu_keep(many)
+    perm, _ = oracle.build_perm(w.T, w.H, w.W, w.order)
+    qp, kp, vp = (oracle.reorder(to_np(t)[0].astype(np.float64), perm) for t in (q, k, v))
+    for eta in range(w.heads):
+        if w.compensate:
+            kb, n = oracle.pool(kp[eta], w.N)
+            vb, _ = oracle.pool(vp[eta], w.N)
+            ref = oracle.compensated_attention(qp[eta], kp[eta], vp[eta], w.N, keep[eta], kb, vb, n)
+        else:
+            ref = oracle.masked_attention(qp[eta], kp[eta], vp[eta], w.N, keep[eta])
+        gout = np.concatenate([ap[eta][I * 64:min(I * 64 + 64, w.N)] for I in range(many.nb)])
+        check_attention(gout, np.concatenate([ref[I] for I in range(many.nb)]), f"passes={passes} head {eta}")
