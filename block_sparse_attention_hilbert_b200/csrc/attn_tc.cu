@@ -24,7 +24,7 @@
 //     needs all 128 threads, so the running maximum is lazy: a tile only
 //     updates it (warp transpose-reduction + shared memory, then an in-TMEM
 //     rescale of O^T and of the partial sums) when some score exceeds the
-//     current maximum by more than 2^8; otherwise exp2(x - m) is taken against
+//     current maximum by more than 2^12; otherwise exp2(x - m) is taken against
 //     the stale maximum, which is exact up to the final normalisation.  The
 //     row sums stay per-thread partial sums until the epilogue.
 //   * Compensation ("SVG-EAR" 2.A): after the kept pairs, an item walks
@@ -36,7 +36,7 @@
 //   * P^T is rounded to fp16 and written to shared memory in the MN-major
 //     128-byte-swizzled layout the second MMA reads; the values arrive as
 //     fp16 (the reordered V), so the second product is fp16 x fp16.  With the
-//     lazy maximum the weights reach 2^8 and the dominant one is no longer
+//     lazy maximum the weights reach 2^12 and the dominant one is no longer
 //     exactly 1, so fp16's 11-bit significand (vs bf16's 8) is what keeps
 //     their rounding well inside the output tolerance.
 #include <cstddef>
@@ -62,7 +62,7 @@ constexpr int kThreads = 32 * (4 + 4 * kGroups);
 constexpr int kKStages = SVSA_TC_KSTAGES, kVStages = 2, kSBufs = 3, kPBufs = SVSA_TC_PBUFS;
 constexpr int kSoftmaxThreads = 128;             // one softmax warpgroup
 constexpr uint32_t kBox = 8192;                  // one 64-row x 128-byte TMA box
-constexpr float kLazyTh = 8.0f;                  // log2 headroom before a rescale
+constexpr float kLazyTh = 12.0f;                 // log2 headroom before a rescale (fp16 P <= 2^12)
 
 // shared memory map (offsets from a 1024-byte aligned base)
 constexpr uint32_t kOffQ = 0;                               // 2 x 8 KB (head-dim chunks)
