@@ -421,10 +421,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         const int J = lst[j];
         return J < 0 ? 0 : (J >= nb ? nb - 1 : J);
       };
-      int jcur = block_at(slot);
 
       for (int t = 0; t < ntiles; ++t) {
-        const int jnext = block_at(2 * t + 2 + slot);
+        // kept lists are ascending: only the last pair can hold block nb - 1
+        // (ragged) or a missing second block, so only it needs the list entry
+        const bool tail = t >= npairs - 1;
+        const int jcur = tail ? block_at(2 * t + slot) : 0;
         // centroid tile: this thread's block J and its kept bit (read before the wait)
         const bool cent = COMP && t >= npairs;
         const int Jc = (t - npairs) * 128 + k;
@@ -440,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         if (lane == 0) mbar_arrive(bar(BAR_S_EMPTY + sb));
 
         const bool valid = cent ? ((kept_word >> (Jc & 31)) & 1u) == 0u
-                                : jcur >= 0 && (jcur < nb - 1 || (k & 63) < n_in_last);
+                                : !tail || (jcur >= 0 && (jcur < nb - 1 || (k & 63) < n_in_last));
         const bool first = t == 0;
         // y = scaled score (log2 domain) minus the reference of its column; a
         // skipped block's centroid enters n_J times: + log2(n_J)
@@ -530,7 +532,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         // advance the S and P rings and their phases
         if (++sb == (uint32_t)kSBufs) { sb = 0u; sph ^= 1u; }
         if (++pb == (uint32_t)kPBufs) { pb = 0u; pph ^= 1u; }
-        jcur = jnext;
       }
       if (stop) break;
 

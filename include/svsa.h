@@ -99,7 +99,9 @@ typedef struct {
  * buffers are caller-owned device memory. */
 typedef struct {
   int32_t* kv_idx;        /* [B, heads, nb, cap] kept key blocks of each query
-                             block, ascending; entries past kv_cnt are unspecified */
+                             block, strictly ascending (required: the attention
+                             checks only a row's last pair for the ragged block
+                             nb - 1); entries past kv_cnt are unspecified */
   int32_t* kv_cnt;        /* [B, heads, nb] number of kept key blocks */
   int32_t cap;            /* row capacity: >= nb (>= k for TOPK) */
   uint32_t* bits;         /* nullable [B, heads, nb, ceil(nb/32)]: bit J%32 of word
