@@ -422,116 +422,123 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         return J < 0 ? 0 : (J >= nb ? nb - 1 : J);
       };
 
-      for (int t = 0; t < ntiles; ++t) {
-        // kept lists are ascending: only the last pair can hold block nb - 1
-        // (ragged) or a missing second block, so only it needs the list entry
-        const bool tail = t >= npairs - 1;
-        const int jcur = tail ? block_at(2 * t + slot) : 0;
-        // centroid tile: this thread's block J and its kept bit (read before the wait)
-        const bool cent = COMP && t >= npairs;
-        const int Jc = (t - npairs) * 128 + k;
-        uint32_t kept_word = ~0u;
-        if (cent && Jc < nb) kept_word = a.bits[it * a.nwords + (Jc >> 5)];
-        wait_bar(bar(BAR_S_FULL + sb), sph, abort_flag, 10);
-        tc_fence_after();
-        float y[kCols];
-        tmem_ld_cols<kCols>(tmem + lane_off + kColS0 + sb * 64 + cb, y);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(BAR_S_EMPTY + sb));
+      // kept-pair tiles, then (with compensation) the centroid tiles; the
+      // phase loop is unrolled so that each phase's tile loop is compiled for
+      // its own kind of tile and the pair loop carries no centroid code
+#pragma unroll
+      for (int phase = 0; phase < (COMP ? 2 : 1); ++phase) {
+        const bool cent = phase == 1;
+        for (int t = cent ? npairs : 0; t < (cent ? ntiles : npairs); ++t) {
+          // kept lists are ascending: only the last pair can hold block nb - 1
+          // (ragged) or a missing second block, so only it needs the list entry
+          const bool tail = !cent && t >= npairs - 1;
+          const int jcur = tail ? block_at(2 * t + slot) : 0;
+          // centroid tile: this thread's block J and its kept bit (read before the wait)
+          const int Jc = (t - npairs) * 128 + k;
+          uint32_t kept_word = ~0u;
+          if (cent && Jc < nb) kept_word = a.bits[it * a.nwords + (Jc >> 5)];
+          wait_bar(bar(BAR_S_FULL + sb), sph, abort_flag, 10);
+          tc_fence_after();
+          float y[kCols];
+          tmem_ld_cols<kCols>(tmem + lane_off + kColS0 + sb * 64 + cb, y);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(BAR_S_EMPTY + sb));
 
-        const bool valid = cent ? ((kept_word >> (Jc & 31)) & 1u) == 0u
-                                : !tail || (jcur >= 0 && (jcur < nb - 1 || (k & 63) < n_in_last));
-        const bool first = t == 0;
-        // y = scaled score (log2 domain) minus the reference of its column; a
-        // skipped block's centroid enters n_J times: + log2(n_J)
-        float excess = -INFINITY;
-        if (valid) {
-          const float bias = cent ? (Jc == nb - 1 ? __log2f((float)n_in_last) : 6.0f) : 0.f;
+          const bool valid = cent ? ((kept_word >> (Jc & 31)) & 1u) == 0u
+                                  : !tail || (jcur >= 0 && (jcur < nb - 1 || (k & 63) < n_in_last));
+          const bool first = t == 0;
+          // y = scaled score (log2 domain) minus the reference of its column; a
+          // skipped block's centroid enters n_J times: + log2(n_J)
+          float excess = -INFINITY;
+          if (valid) {
+            const float bias = cent ? (Jc == nb - 1 ? __log2f((float)n_in_last) : 6.0f) : 0.f;
 #pragma unroll
-          for (int c = 0; c < kCols; ++c) {
-            y[c] = COMP ? fmaf(y[c], sl2, bias - mref[c]) : fmaf(y[c], sl2, -mref[c]);
-            excess = fmaxf(excess, y[c]);
+            for (int c = 0; c < kCols; ++c) {
+              y[c] = cent ? fmaf(y[c], sl2, bias - mref[c]) : fmaf(y[c], sl2, -mref[c]);
+              excess = fmaxf(excess, y[c]);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < kCols; ++c) y[c] = -INFINITY;
           }
-        } else {
+          // exponentials against the current reference before the group vote, so
+          // the wait for the slowest warp overlaps with this warp's MUFU work;
+          // only a rescale tile (rare after the first) recomputes them
+          float pv[kCols];
 #pragma unroll
-          for (int c = 0; c < kCols; ++c) y[c] = -INFINITY;
+          for (int c = 0; c < kCols; ++c) pv[c] = ex2(y[c]);
+          if (named_bar_or(gbar, kSoftmaxThreads, first || (*abort_flag != 0u) || excess > kLazyTh)) {
+            if (named_bar_or(gbar, kSoftmaxThreads, *abort_flag != 0u)) {
+              stop = true;
+              break;
+            }
+            // exact column maxima of this tile (in y units), then a new reference
+            {
+              float v[kCols];
+#pragma unroll
+              for (int c = 0; c < kCols; ++c) v[c] = y[c];
+              const float r = warp_colreduce<true, kCols>(v);
+              if (lane < kCols) ms->red[wg][sw][lane] = r;
+            }
+            named_bar(gbar, kSoftmaxThreads);
+            if (st < kCols) {
+              const float ty = fmaxf(fmaxf(ms->red[wg][0][st], ms->red[wg][1][st]),
+                                     fmaxf(ms->red[wg][2][st], ms->red[wg][3][st]));
+              const float m_used = first ? 0.f : mcol[st];
+              // (a first tile with no valid key keeps the reference at 0)
+              const float m_new = first ? (cent && ty == -INFINITY ? 0.f : ty) : fmaxf(mcol[st], ty + m_used);
+              mcol[st] = m_new;
+              acol[st] = first ? 0.f : ex2(m_used - m_new);
+              fcol[st] = m_new - m_used;              // shift to apply to this tile's y
+            }
+            named_bar(gbar, kSoftmaxThreads);
+#pragma unroll
+            for (int c = 0; c < kCols; ++c) {
+              y[c] -= fcol[c];
+              lp[c] *= acol[c];
+              mref[c] = mcol[c];
+              pv[c] = ex2(y[c]);
+            }
+            if (!first) {
+              // O^T holds the previous tiles' sum once their MMA has finished
+              // the previous tile used the previous slot of the P ring
+              const uint32_t pprev = pb == 0u ? (uint32_t)kPBufs - 1u : pb - 1u;
+              wait_bar(bar(BAR_P_EMPTY + pprev), pb == 0u ? pph ^ 1u : pph, abort_flag, 11);
+              tc_fence_after();
+              float o[kCols];
+              tmem_ld_cols<kCols>(tmem + lane_off + kColO + cb, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < kCols; ++c) o[c] *= acol[c];
+              tmem_st_cols<kCols>(tmem + lane_off + kColO + cb, o);
+              tmem_wait_st();
+            }
+          }
+          // P^T row k, this group's columns: exp2(y), fp16, 128-byte swizzled MN-major layout
+          uint32_t pk[kCols / 2];
+#pragma unroll
+          for (int c = 0; c < kCols; c += 2) {
+            lp[c] += pv[c];
+            lp[c + 1] += pv[c + 1];
+            pk[c >> 1] = pack_f16x2(pv[c], pv[c + 1]);
+          }
+          wait_bar(bar(BAR_P_EMPTY + pb), pph ^ 1u, abort_flag, 12);
+          unsigned char* prow = prow0 + pb * 16384;
+#pragma unroll
+          for (int jj = 0; jj < kCols / 8; ++jj)
+            *reinterpret_cast<uint4*>(prow + pchunk[jj]) =
+                make_uint4(pk[4 * jj], pk[4 * jj + 1], pk[4 * jj + 2], pk[4 * jj + 3]);
+          fence_async_smem();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(BAR_P_FULL + pb));
+          // advance the S and P rings and their phases
+          if (++sb == (uint32_t)kSBufs) { sb = 0u; sph ^= 1u; }
+          if (++pb == (uint32_t)kPBufs) { pb = 0u; pph ^= 1u; }
         }
-        // exponentials against the current reference before the group vote, so
-        // the wait for the slowest warp overlaps with this warp's MUFU work;
-        // only a rescale tile (rare after the first) recomputes them
-        float pv[kCols];
-#pragma unroll
-        for (int c = 0; c < kCols; ++c) pv[c] = ex2(y[c]);
-        if (named_bar_or(gbar, kSoftmaxThreads, first || (*abort_flag != 0u) || excess > kLazyTh)) {
-          if (named_bar_or(gbar, kSoftmaxThreads, *abort_flag != 0u)) {
-            stop = true;
-            break;
-          }
-          // exact column maxima of this tile (in y units), then a new reference
-          {
-            float v[kCols];
-#pragma unroll
-            for (int c = 0; c < kCols; ++c) v[c] = y[c];
-            const float r = warp_colreduce<true, kCols>(v);
-            if (lane < kCols) ms->red[wg][sw][lane] = r;
-          }
-          named_bar(gbar, kSoftmaxThreads);
-          if (st < kCols) {
-            const float ty = fmaxf(fmaxf(ms->red[wg][0][st], ms->red[wg][1][st]),
-                                   fmaxf(ms->red[wg][2][st], ms->red[wg][3][st]));
-            const float m_used = first ? 0.f : mcol[st];
-            // (a first tile with no valid key keeps the reference at 0)
-            const float m_new = first ? (COMP && ty == -INFINITY ? 0.f : ty) : fmaxf(mcol[st], ty + m_used);
-            mcol[st] = m_new;
-            acol[st] = first ? 0.f : ex2(m_used - m_new);
-            fcol[st] = m_new - m_used;              // shift to apply to this tile's y
-          }
-          named_bar(gbar, kSoftmaxThreads);
-#pragma unroll
-          for (int c = 0; c < kCols; ++c) {
-            y[c] -= fcol[c];
-            lp[c] *= acol[c];
-            mref[c] = mcol[c];
-            pv[c] = ex2(y[c]);
-          }
-          if (!first) {
-            // O^T holds the previous tiles' sum once their MMA has finished
-            // the previous tile used the previous slot of the P ring
-            const uint32_t pprev = pb == 0u ? (uint32_t)kPBufs - 1u : pb - 1u;
-            wait_bar(bar(BAR_P_EMPTY + pprev), pb == 0u ? pph ^ 1u : pph, abort_flag, 11);
-            tc_fence_after();
-            float o[kCols];
-            tmem_ld_cols<kCols>(tmem + lane_off + kColO + cb, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < kCols; ++c) o[c] *= acol[c];
-            tmem_st_cols<kCols>(tmem + lane_off + kColO + cb, o);
-            tmem_wait_st();
-          }
-        }
-        // P^T row k, this group's columns: exp2(y), fp16, 128-byte swizzled MN-major layout
-        uint32_t pk[kCols / 2];
-#pragma unroll
-        for (int c = 0; c < kCols; c += 2) {
-          lp[c] += pv[c];
-          lp[c + 1] += pv[c + 1];
-          pk[c >> 1] = pack_f16x2(pv[c], pv[c + 1]);
-        }
-        wait_bar(bar(BAR_P_EMPTY + pb), pph ^ 1u, abort_flag, 12);
-        unsigned char* prow = prow0 + pb * 16384;
-#pragma unroll
-        for (int jj = 0; jj < kCols / 8; ++jj)
-          *reinterpret_cast<uint4*>(prow + pchunk[jj]) =
-              make_uint4(pk[4 * jj], pk[4 * jj + 1], pk[4 * jj + 2], pk[4 * jj + 3]);
-        fence_async_smem();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(BAR_P_FULL + pb));
-        // advance the S and P rings and their phases
-        if (++sb == (uint32_t)kSBufs) { sb = 0u; sph ^= 1u; }
-        if (++pb == (uint32_t)kPBufs) { pb = 0u; pph ^= 1u; }
+        if (stop) break;
       }
       if (stop) break;
 
