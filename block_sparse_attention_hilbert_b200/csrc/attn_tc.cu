@@ -377,7 +377,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     float* mcol = ms->m + cb;
     float* acol = ms->alpha + cb;
     float* fcol = ms->fin + cb;
-    uint32_t sb = 0, sph = 0, pb = 0, pph = 0, oit = 0;      // ring slots and phases
+    // S and P rings have the same depth and advance together here: one slot
+    // index and phase serve both
+    static_assert(kSBufs == kPBufs, "S and P rings share the softmax slot counter");
+    uint32_t sb = 0, sph = 0, oit = 0;
     // this thread's P^T row (key k) and its swizzled 16-byte chunks for the group's columns
     unsigned char* const prow0 = smem + kOffP + (k >> 3) * 1024 + (k & 7) * 128;
     uint32_t pchunk[kCols / 8];
@@ -407,11 +410,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       }
       const int32_t* lst = a.dense ? nullptr : a.kv_idx + it * a.cap;
       const int n_in_last = (int)(a.N - (long long)(nb - 1) * kBlock);   // valid keys of block nb-1
-      float lp[kCols], mref[kCols];
+      float lp[kCols], nmref[kCols];
 #pragma unroll
       for (int c = 0; c < kCols; ++c) {
         lp[c] = 0.f;
-        mref[c] = 0.f;                             // reference maxima; set by the first tile
+        nmref[c] = 0.f;                            // negated reference maxima; set by the first tile
       }
       // this thread's key block for the current pair (prefetched one tile ahead)
       const int slot = k >> 6;
@@ -425,6 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       // kept-pair tiles, then (with compensation) the centroid tiles; the
       // phase loop is unrolled so that each phase's tile loop is compiled for
       // its own kind of tile and the pair loop carries no centroid code
+      bool badp = false;                           // the last P-ring wait failed
 #pragma unroll
       for (int phase = 0; phase < (COMP ? 2 : 1); ++phase) {
         const bool cent = phase == 1;
@@ -437,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           const int Jc = (t - npairs) * 128 + k;
           uint32_t kept_word = ~0u;
           if (cent && Jc < nb) kept_word = a.bits[it * a.nwords + (Jc >> 5)];
-          wait_bar(bar(BAR_S_FULL + sb), sph, abort_flag, 10);
+          const bool bad = !wait_bar(bar(BAR_S_FULL + sb), sph, abort_flag, 10);
           tc_fence_after();
           float y[kCols];
           tmem_ld_cols<kCols>(tmem + lane_off + kColS0 + sb * 64 + cb, y);
@@ -455,10 +459,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           if (valid) {
             const float bias = cent ? (Jc == nb - 1 ? __log2f((float)n_in_last) : 6.0f) : 0.f;
 #pragma unroll
-            for (int c = 0; c < kCols; ++c) {
-              y[c] = cent ? fmaf(y[c], sl2, bias - mref[c]) : fmaf(y[c], sl2, -mref[c]);
-              excess = fmaxf(excess, y[c]);
+            for (int c = 0; c < kCols; c += 2) {
+              if (cent) fma2(y[c], y[c + 1], sl2, bias + nmref[c], bias + nmref[c + 1]);
+              else fma2(y[c], y[c + 1], sl2, nmref[c], nmref[c + 1]);
             }
+#pragma unroll
+            for (int c = 0; c < kCols; c += 2) excess = max3(excess, y[c], y[c + 1]);
           } else {
 #pragma unroll
             for (int c = 0; c < kCols; ++c) y[c] = -INFINITY;
@@ -469,7 +475,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           float pv[kCols];
 #pragma unroll
           for (int c = 0; c < kCols; ++c) pv[c] = ex2(y[c]);
-          if (named_bar_or(gbar, kSoftmaxThreads, first || (*abort_flag != 0u) || excess > kLazyTh)) {
+          // (a failed wait of this thread, here or at the P ring of the previous
+          // tile, takes the slow path, whose second vote sees the abort flag)
+          if (named_bar_or(gbar, kSoftmaxThreads, first || bad || badp || excess > kLazyTh)) {
             if (named_bar_or(gbar, kSoftmaxThreads, *abort_flag != 0u)) {
               stop = true;
               break;
@@ -498,14 +506,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             for (int c = 0; c < kCols; ++c) {
               y[c] -= fcol[c];
               lp[c] *= acol[c];
-              mref[c] = mcol[c];
+              nmref[c] = -mcol[c];
               pv[c] = ex2(y[c]);
             }
             if (!first) {
               // O^T holds the previous tiles' sum once their MMA has finished
               // the previous tile used the previous slot of the P ring
-              const uint32_t pprev = pb == 0u ? (uint32_t)kPBufs - 1u : pb - 1u;
-              wait_bar(bar(BAR_P_EMPTY + pprev), pb == 0u ? pph ^ 1u : pph, abort_flag, 11);
+              const uint32_t pprev = sb == 0u ? (uint32_t)kPBufs - 1u : sb - 1u;
+              wait_bar(bar(BAR_P_EMPTY + pprev), sb == 0u ? sph ^ 1u : sph, abort_flag, 11);
               tc_fence_after();
               float o[kCols];
               tmem_ld_cols<kCols>(tmem + lane_off + kColO + cb, o);
@@ -520,12 +528,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           uint32_t pk[kCols / 2];
 #pragma unroll
           for (int c = 0; c < kCols; c += 2) {
-            lp[c] += pv[c];
-            lp[c + 1] += pv[c + 1];
+            add2(lp[c], lp[c + 1], pv[c], pv[c + 1]);
             pk[c >> 1] = pack_f16x2(pv[c], pv[c + 1]);
           }
-          wait_bar(bar(BAR_P_EMPTY + pb), pph ^ 1u, abort_flag, 12);
-          unsigned char* prow = prow0 + pb * 16384;
+          badp = !wait_bar(bar(BAR_P_EMPTY + sb), sph ^ 1u, abort_flag, 12);
+          unsigned char* prow = prow0 + sb * 16384;
 #pragma unroll
           for (int jj = 0; jj < kCols / 8; ++jj)
             *reinterpret_cast<uint4*>(prow + pchunk[jj]) =
@@ -533,10 +540,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           fence_async_smem();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar(BAR_P_FULL + pb));
-          // advance the S and P rings and their phases
+          if (lane == 0) mbar_arrive(bar(BAR_P_FULL + sb));
+          // advance the S and P rings and their phase
           if (++sb == (uint32_t)kSBufs) { sb = 0u; sph ^= 1u; }
-          if (++pb == (uint32_t)kPBufs) { pb = 0u; pph ^= 1u; }
         }
         if (stop) break;
       }

@@ -168,6 +168,27 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Packed fp32 pairs (sm_100): one instruction for two lanes of the same
+// operation, each rounded exactly as its scalar form.
+// (a, b) = (a * s + c0, b * s + c1)
+__device__ __forceinline__ void fma2(float& a, float& b, float s, float c0, float c1) {
+  asm("{\n .reg .b64 x, m, c, r;\n mov.b64 x, {%0, %1};\n mov.b64 m, {%2, %2};\n mov.b64 c, {%3, %4};\n"
+      " fma.rn.f32x2 r, x, m, c;\n mov.b64 {%0, %1}, r;\n}\n"
+      : "+f"(a), "+f"(b) : "f"(s), "f"(c0), "f"(c1));
+}
+// (a, b) += (x, y)
+__device__ __forceinline__ void add2(float& a, float& b, float x, float y) {
+  asm("{\n .reg .b64 p, q;\n mov.b64 p, {%0, %1};\n mov.b64 q, {%2, %3};\n add.rn.f32x2 p, p, q;\n"
+      " mov.b64 {%0, %1}, p;\n}\n"
+      : "+f"(a), "+f"(b) : "f"(x), "f"(y));
+}
+// max(a, b, c) in one instruction
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;\n" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle (sm_100 format, version 1).
 __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
   return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
