@@ -381,11 +381,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     // index and phase serve both
     static_assert(kSBufs == kPBufs, "S and P rings share the softmax slot counter");
     uint32_t sb = 0, sph = 0, oit = 0;
-    // this thread's P^T row (key k) and its swizzled 16-byte chunks for the group's columns
-    unsigned char* const prow0 = smem + kOffP + (k >> 3) * 1024 + (k & 7) * 128;
-    uint32_t pchunk[kCols / 8];
-#pragma unroll
-    for (int jj = 0; jj < kCols / 8; ++jj) pchunk[jj] = (uint32_t)(((cb / 8 + jj) ^ (k & 7)) << 4);
+    // shared address of this thread's first 16-byte chunk of its P^T row (key
+    // k) for the group's columns, 128-byte swizzle; the row starts on a
+    // 128-byte boundary and the group's two chunks are 16-byte slots 2 wg and
+    // 2 wg + 1 before the swizzle, so the second chunk is the first ^ 16
+    static_assert(kCols == 16, "two 16-byte chunks of fp16 P per row and group");
+    const uint32_t pa0 = sbase + kOffP + (uint32_t)((k >> 3) * 1024 + (k & 7) * 128) +
+                         (uint32_t)(((2 * wg) ^ (k & 7)) << 4);
     bool stop = false;
     for (long long it = blockIdx.x; it < items && !stop; it += gridDim.x) {
       const int cnt = item_count(it);
@@ -443,38 +445,41 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           if (cent && Jc < nb) kept_word = a.bits[it * a.nwords + (Jc >> 5)];
           const bool bad = !wait_bar(bar(BAR_S_FULL + sb), sph, abort_flag, 10);
           tc_fence_after();
-          float y[kCols];
-          tmem_ld_cols<kCols>(tmem + lane_off + kColS0 + sb * 64 + cb, y);
-          tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(BAR_S_EMPTY + sb));
-
           const bool valid = cent ? ((kept_word >> (Jc & 31)) & 1u) == 0u
                                   : !tail || (jcur >= 0 && (jcur < nb - 1 || (k & 63) < n_in_last));
           const bool first = t == 0;
+          const float bias = cent ? (Jc == nb - 1 ? __log2f((float)n_in_last) : 6.0f) : 0.f;
           // y = scaled score (log2 domain) minus the reference of its column; a
-          // skipped block's centroid enters n_J times: + log2(n_J)
-          float excess = -INFINITY;
-          if (valid) {
-            const float bias = cent ? (Jc == nb - 1 ? __log2f((float)n_in_last) : 6.0f) : 0.f;
+          // skipped block's centroid enters n_J times: + log2(n_J).  The S slot
+          // is held until after the vote, so the rare rescale path reads it
+          // again instead of keeping y live next to the exponentials.
+          auto load_y = [&](float (&y)[kCols]) {
+            tmem_ld_cols<kCols>(tmem + lane_off + kColS0 + sb * 64 + cb, y);
+            tmem_wait_ld();
+            if (valid) {
 #pragma unroll
-            for (int c = 0; c < kCols; c += 2) {
-              if (cent) fma2(y[c], y[c + 1], sl2, bias + nmref[c], bias + nmref[c + 1]);
-              else fma2(y[c], y[c + 1], sl2, nmref[c], nmref[c + 1]);
+              for (int c = 0; c < kCols; c += 2) {
+                if (cent) fma2(y[c], y[c + 1], sl2, bias + nmref[c], bias + nmref[c + 1]);
+                else fma2(y[c], y[c + 1], sl2, nmref[c], nmref[c + 1]);
+              }
+            } else {
+#pragma unroll
+              for (int c = 0; c < kCols; ++c) y[c] = -INFINITY;
             }
-#pragma unroll
-            for (int c = 0; c < kCols; c += 2) excess = max3(excess, y[c], y[c + 1]);
-          } else {
-#pragma unroll
-            for (int c = 0; c < kCols; ++c) y[c] = -INFINITY;
-          }
+          };
           // exponentials against the current reference before the group vote, so
           // the wait for the slowest warp overlaps with this warp's MUFU work;
           // only a rescale tile (rare after the first) recomputes them
           float pv[kCols];
+          float excess = -INFINITY;
+          {
+            float y[kCols];
+            load_y(y);
 #pragma unroll
-          for (int c = 0; c < kCols; ++c) pv[c] = ex2(y[c]);
+            for (int c = 0; c < kCols; c += 2) excess = max3(excess, y[c], y[c + 1]);
+#pragma unroll
+            for (int c = 0; c < kCols; ++c) pv[c] = ex2(y[c]);
+          }
           // (a failed wait of this thread, here or at the P ring of the previous
           // tile, takes the slow path, whose second vote sees the abort flag)
           if (named_bar_or(gbar, kSoftmaxThreads, first || bad || badp || excess > kLazyTh)) {
@@ -483,6 +488,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
               break;
             }
             // exact column maxima of this tile (in y units), then a new reference
+            float y[kCols];
+            load_y(y);
             {
               float v[kCols];
 #pragma unroll
@@ -524,6 +531,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
               tmem_wait_st();
             }
           }
+          // S slot free (this warp's reads of it are done)
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(BAR_S_EMPTY + sb));
           // P^T row k, this group's columns: exp2(y), fp16, 128-byte swizzled MN-major layout
           uint32_t pk[kCols / 2];
 #pragma unroll
@@ -532,11 +543,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             pk[c >> 1] = pack_f16x2(pv[c], pv[c + 1]);
           }
           badp = !wait_bar(bar(BAR_P_EMPTY + sb), sph ^ 1u, abort_flag, 12);
-          unsigned char* prow = prow0 + sb * 16384;
-#pragma unroll
-          for (int jj = 0; jj < kCols / 8; ++jj)
-            *reinterpret_cast<uint4*>(prow + pchunk[jj]) =
-                make_uint4(pk[4 * jj], pk[4 * jj + 1], pk[4 * jj + 2], pk[4 * jj + 3]);
+          st_shared_v4(pa0 + sb * 16384u, pk[0], pk[1], pk[2], pk[3]);
+          st_shared_v4((pa0 ^ 16u) + sb * 16384u, pk[4], pk[5], pk[6], pk[7]);
           fence_async_smem();
           tc_fence_before();
           __syncwarp();
