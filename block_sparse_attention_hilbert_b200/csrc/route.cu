@@ -24,10 +24,12 @@
 // * 64 / n_J.
 //
 // Warp 0 issues the TMA copies (qbar tile per item; K_J and V_J per tile into
-// a 2-stage ring), warp 1 issues the MMAs (S of tile t+1 ahead of the E.V of
-// tile t) and owns TMEM, warps 2-5 hold one proxy per thread: exponentials,
-// the E split into shared memory, and the error epilogue of the previous
-// tile while the tensor core works on the next one.  Every wait is bounded.
+// a 2-stage ring; the fp32 centroid value row vbar_J per tile into a 4-deep
+// ring that the error epilogue releases), warp 1 issues the MMAs (S of tile
+// t+1 ahead of the E.V of tile t) and owns TMEM, warps 2-5 hold one proxy per
+// thread: exponentials, the E split into shared memory, and the error
+// epilogue of the previous tile while the tensor core works on the next one.
+// Every wait is bounded.
 #include "tcgen05.cuh"
 
 namespace svsa {
@@ -36,7 +38,7 @@ namespace route {
 
 constexpr int kThreads = 192;
 constexpr int kRows = 128;                   // proxies per item
-constexpr int kStages = 2, kSBufs = 2, kEBufs = 2, kOBufs = 2;
+constexpr int kStages = 2, kSBufs = 2, kEBufs = 2, kOBufs = 2, kVbBufs = 4;
 constexpr uint32_t kBoxQ = kRows * 128;      // 128 rows x 64 bf16 (16 KB)
 constexpr uint32_t kBoxK = kBlock * 128;     // 64 rows x 64 elements (8 KB)
 constexpr uint32_t kEPart = kRows * 128;     // E hi or lo: 128 proxies x 64 fp16 (16 KB)
@@ -49,7 +51,9 @@ struct Smem {
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffKV = kQ;
   static constexpr uint32_t kOffE = kOffKV + kStages * kStage;
-  static constexpr uint32_t kOffMisc = kOffE + kEBufs * 2 * kEPart;
+  static constexpr uint32_t kVb = D * 4;                      // one fp32 centroid value row
+  static constexpr uint32_t kOffVb = kOffE + kEBufs * 2 * kEPart;
+  static constexpr uint32_t kOffMisc = kOffVb + kVbBufs * kVb;
   static constexpr uint32_t kBytes = kOffMisc + 512 + 1024;
   static_assert(kBytes <= 232448, "shared memory per CTA");
   // TMEM: S buffers (64 columns each), then O buffers (D columns each)
@@ -61,7 +65,8 @@ enum : uint32_t {
   BAR_Q_FULL = 0, BAR_Q_EMPTY, BAR_KV_FULL, BAR_KV_EMPTY = BAR_KV_FULL + kStages,
   BAR_S_FULL = BAR_KV_EMPTY + kStages, BAR_S_EMPTY = BAR_S_FULL + kSBufs,
   BAR_E_FULL = BAR_S_EMPTY + kSBufs, BAR_E_EMPTY = BAR_E_FULL + kEBufs,
-  BAR_O_FULL = BAR_E_EMPTY + kEBufs, BAR_O_EMPTY = BAR_O_FULL + kOBufs, BAR_FINAL = BAR_O_EMPTY + kOBufs,
+  BAR_O_FULL = BAR_E_EMPTY + kEBufs, BAR_O_EMPTY = BAR_O_FULL + kOBufs,
+  BAR_VB_FULL = BAR_O_EMPTY + kOBufs, BAR_VB_EMPTY = BAR_VB_FULL + kVbBufs, BAR_FINAL = BAR_VB_EMPTY + kVbBufs,
   NUM_BARS
 };
 
@@ -119,6 +124,10 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(const __grid_cons
       mbar_init(bar(BAR_O_FULL + i), 1);
       mbar_init(bar(BAR_O_EMPTY + i), 4);
     }
+    for (int i = 0; i < kVbBufs; ++i) {
+      mbar_init(bar(BAR_VB_FULL + i), 1);
+      mbar_init(bar(BAR_VB_EMPTY + i), 4);
+    }
     mbar_init(bar(BAR_FINAL), 1);
     ms->abort = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -170,6 +179,13 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(const __grid_cons
             tma_load_2d(dst + c * kBoxK, &tmK, c * 64, yk, bar(BAR_KV_FULL + stg));
             tma_load_2d(dst + (NCH + c) * kBoxK, &tmV, c * 64, yk, bar(BAR_KV_FULL + stg));
           }
+          // the centroid value row of block J for this tile's error epilogue
+          const uint32_t vs = kn % kVbBufs;
+          ok = wait_bar(bar(BAR_VB_EMPTY + vs), ((kn / kVbBufs) & 1u) ^ 1u, abort_flag, 64);
+          if (!ok) break;
+          mbar_expect_tx(bar(BAR_VB_FULL + vs), L::kVb);
+          bulk_load(sbase + L::kOffVb + vs * L::kVb, a.vbar + (bh * nb + J) * (long long)D, L::kVb,
+                    bar(BAR_VB_FULL + vs));
           ++kn;
         }
       }
@@ -178,6 +194,10 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(const __grid_cons
       for (uint32_t j = 1; j <= (uint32_t)kStages && j <= kn; ++j) {
         const uint32_t n = kn - j;
         wait_bar(bar(BAR_KV_FULL + n % kStages), (n / kStages) & 1u, &no_abort, 61);
+      }
+      for (uint32_t j = 1; j <= (uint32_t)kVbBufs && j <= kn; ++j) {
+        const uint32_t n = kn - j;
+        wait_bar(bar(BAR_VB_FULL + n % kVbBufs), (n / kVbBufs) & 1u, &no_abort, 65);
       }
     }
   } else if (warp == 1) {
@@ -274,16 +294,19 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(const __grid_cons
       }
       const long long rbase = (bh * nb + (row_ok ? I : 0)) * (long long)nb;
       float m = -INFINITY, Z = 0.f;
-      float m_prev = 0.f;
+      float m_prev = 0.f, L_prev = 0.f;
       int J_prev = -1;
-      // error epilogue of tile n (block J, weights against m_used)
-      auto epilogue = [&](uint32_t n, int J, float m_used) -> bool {
-        const uint32_t ob = n % kOBufs;
-        if (!wait_bar(bar(BAR_O_FULL + ob), (n / kOBufs) & 1u, abort_flag, 58)) return false;
+      // error epilogue of tile n (block J, weights against m_used; LJ = the
+      // proxy's centroid logit of block J, loaded one tile earlier)
+      auto epilogue = [&](uint32_t n, int J, float m_used, float LJ) -> bool {
+        const uint32_t ob = n % kOBufs, vs = n % kVbBufs;
+        if (!wait_bar(bar(BAR_O_FULL + ob), (n / kOBufs) & 1u, abort_flag, 58) ||
+            !wait_bar(bar(BAR_VB_FULL + vs), (n / kVbBufs) & 1u, abort_flag, 66))
+          return false;
         tc_fence_after();
         const int nJ = J == nb - 1 ? n_in_last : kBlock;
-        const float cw = row_ok ? (float)nJ * ex2(a.L[rbase + J] - m_used) : 0.f;
-        const float4* vb = reinterpret_cast<const float4*>(a.vbar + (bh * nb + J) * (long long)D);
+        const float cw = row_ok ? (float)nJ * ex2(LJ - m_used) : 0.f;
+        const float4* vb = reinterpret_cast<const float4*>(smem + L::kOffVb + vs * L::kVb);
         float err2 = 0.f;
 #pragma unroll 1
         for (int ch = 0; ch < D / 32; ++ch) {
@@ -292,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(const __grid_cons
           tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < 32; c += 4) {
-            const float4 v4 = __ldg(vb + ch * 8 + c / 4);
+            const float4 v4 = vb[ch * 8 + c / 4];       // same address in every lane: broadcast
             const float d0 = fmaf(-cw, v4.x, o[c]), d1 = fmaf(-cw, v4.y, o[c + 1]);
             const float d2 = fmaf(-cw, v4.z, o[c + 2]), d3 = fmaf(-cw, v4.w, o[c + 3]);
             err2 = fmaf(d0, d0, fmaf(d1, d1, fmaf(d2, d2, fmaf(d3, d3, err2))));
@@ -300,7 +323,10 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(const __grid_cons
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(BAR_O_EMPTY + ob));
+        if (lane == 0) {
+          mbar_arrive(bar(BAR_O_EMPTY + ob));
+          mbar_arrive(bar(BAR_VB_EMPTY + vs));
+        }
         if (row_ok) {
           a.R[rbase + J] = sqrtf(err2);
           a.Rm[rbase + J] = m_used;
@@ -309,6 +335,8 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(const __grid_cons
       };
       for (int J = j0; J < j1; ++J) {
         const uint32_t sb = sn % kSBufs, eb = sn % kEBufs;
+        // this tile's centroid logit, used by its epilogue one tile later
+        const float L_cur = row_ok ? __ldg(a.L + rbase + J) : 0.f;
         if (!wait_bar(bar(BAR_S_FULL + sb), (sn / kSBufs) & 1u, abort_flag, 59)) { stop = true; break; }
         tc_fence_after();
         float x[64];
@@ -353,13 +381,14 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(const __grid_cons
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(BAR_E_FULL + eb));
-        if (J_prev >= 0 && !epilogue(sn - 1, J_prev, m_prev)) { stop = true; break; }
+        if (J_prev >= 0 && !epilogue(sn - 1, J_prev, m_prev, L_prev)) { stop = true; break; }
         J_prev = J;
         m_prev = m;
+        L_prev = L_cur;
         ++sn;
       }
       if (stop) break;
-      if (J_prev >= 0 && !epilogue(sn - 1, J_prev, m_prev)) break;
+      if (J_prev >= 0 && !epilogue(sn - 1, J_prev, m_prev, L_prev)) break;
       if (row_ok) {
         const long long p = (bh * nb + I) * (long long)a.nsplit + it % a.nsplit;
         a.Mp[p] = m;

@@ -16,10 +16,12 @@
 // the candidates' counts and masses per digit, and a suffix scan over the 256
 // digits locates the digit holding the crossing element.  After the 4th pass
 // the crossing value v* is known exactly; everything above v* is kept, and of
-// the elements equal to v* the first t in index order.  One warp per row
-// (histogram updates aggregated over the lanes that share a digit, so the
-// shared-memory atomics do not contend); output lists are ascending by
-// construction (ballot-based compaction in index order).
+// the elements equal to v* the first t in index order.  Short rows: one warp
+// per row, its keys staged in shared memory once for all passes; long rows:
+// one CTA per row.  Histogram updates are plain per-lane shared-memory
+// atomics (measured faster than aggregating the lanes that share a digit with
+// match / reduce).  Output lists are ascending by construction (ballot-based
+// compaction in index order).
 #include "common.cuh"
 
 namespace svsa {
@@ -85,7 +87,6 @@ __device__ void compact_row(int n, KeepFn keep, int32_t* idx_out, int32_t* cnt_o
 // partial sum is exact and independent of the order it is taken in, so the
 // crossing digit found in one pass is consistent with the next, and the sums
 // differ from fp64 cumulative sums by < nb * 2^-48.
-constexpr int kSelWarps = 8;                 // rows per CTA
 constexpr double kFix = 281474976710656.0;   // 2^48
 
 __device__ __forceinline__ unsigned long long fix48(uint32_t key) {
@@ -102,15 +103,14 @@ struct Cut {
   uint32_t take;        // how many keys equal to vstar (first in index order) are kept
 };
 
-// Radix select over one row by a single warp: keys are re-read from `row`
-// (through `key_of`) in every pass.  by_mass: the shortest prefix of the
-// (key desc, index asc) order whose mass reaches tau_fx; else the first k.
-// The target must be reachable (the caller handles "keep all").
+// Radix select over one row by a single warp: every pass reads the keys
+// through `key_of` (the row staged in shared memory).  by_mass: the shortest
+// prefix of the (key desc, index asc) order whose mass reaches tau_fx; else
+// the first k.  The target must be reachable (the caller handles "keep all").
 template <typename KeyOf>
 __device__ Cut warp_radix_cut(KeyOf key_of, int n, bool by_mass, unsigned long long tau_fx, uint32_t k,
                               WarpHist& h) {
   const int lane = threadIdx.x & 31;
-  const uint32_t lt = (1u << lane) - 1u;
   uint32_t prefix = 0u, pmask = 0u, above_c = 0u, eq_c = 0u;
   unsigned long long above_m = 0ull;
   for (int shift = 24; shift >= 0; shift -= 8) {
@@ -124,18 +124,10 @@ __device__ Cut warp_radix_cut(KeyOf key_of, int n, bool by_mass, unsigned long l
       const int j = base + lane;
       const uint32_t key = j < n ? key_of(j) : 0u;
       const bool cand = j < n && (key & pmask) == prefix;
-      const uint32_t cmask = __ballot_sync(0xffffffffu, cand);
       if (cand) {
         const uint32_t dg = (key >> shift) & 255u;
-        const uint32_t peers = __match_any_sync(cmask, dg);
-        const bool leader = (peers & lt) == 0u;
-        if (by_mass) {
-          const unsigned long long m = fix48(key);
-          const uint32_t hi = __reduce_add_sync(peers, (uint32_t)(m >> 24));
-          const uint32_t lo = __reduce_add_sync(peers, (uint32_t)(m & 0xFFFFFFull));
-          if (leader) atomicAdd(&h.mass[dg], ((unsigned long long)hi << 24) + lo);
-        }
-        if (leader) atomicAdd(&h.cnt[dg], (uint32_t)__popc(peers));
+        if (by_mass) atomicAdd(&h.mass[dg], fix48(key));
+        atomicAdd(&h.cnt[dg], 1u);
       }
     }
     __syncwarp();
@@ -202,25 +194,46 @@ __device__ Cut warp_radix_cut(KeyOf key_of, int n, bool by_mass, unsigned long l
   return cut;
 }
 
-__global__ void __launch_bounds__(kSelWarps * 32) select_kernel(
+// One warp per row, blockDim.x / 32 rows per CTA.  The row's keys are copied
+// once into this warp's slice of dynamic shared memory and every pass reads
+// them there, so the row is read from global memory once, not once per pass.
+// Dynamic shared memory: one histogram per warp, then one row of nb keys per
+// warp.
+constexpr int kSelMaxWarps = 4;
+constexpr size_t kSelMaxSmem = 227 * 1024;   // opt-in dynamic shared memory per CTA
+
+__global__ void __launch_bounds__(kSelMaxWarps * 32) select_kernel(
     const float* __restrict__ S, const float* __restrict__ R, long long rows, int nb, int mode, float tau, int k,
     int cap, int32_t* __restrict__ kv_idx, int32_t* __restrict__ kv_cnt, uint32_t* __restrict__ bits) {
-  __shared__ WarpHist hist[kSelWarps];
+  extern __shared__ __align__(16) unsigned char sel_smem[];
+  const int warps = (int)(blockDim.x >> 5);
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const long long row = (long long)blockIdx.x * kSelWarps + wid;
+  const long long row = (long long)blockIdx.x * warps + wid;
   if (row >= rows) return;
-  WarpHist& h = hist[wid];
+  WarpHist& h = reinterpret_cast<WarpHist*>(sel_smem)[wid];
+  uint32_t* const kbuf = reinterpret_cast<uint32_t*>(sel_smem + warps * sizeof(WarpHist)) + (size_t)wid * nb;
   const uint32_t lt = (1u << lane) - 1u;
   const int words = (nb + 31) / 32;
   const float* srow = S + row * (long long)nb;
-  auto skey = [&](int j) { return score_key(__ldg(srow + j)); };
+  const float* rrow = R != nullptr ? R + row * (long long)nb : nullptr;
+  // stage a row's keys; returns the lane's part of the fixed-point mass
+  auto stage = [&](const float* src, bool mass) -> unsigned long long {
+    unsigned long long part = 0ull;
+    for (int j = lane; j < nb; j += 32) {
+      const uint32_t key = score_key(__ldg(src + j));
+      kbuf[j] = key;
+      if (mass) part += fix48(key);
+    }
+    __syncwarp();
+    return part;
+  };
+  auto key_at = [&](int j) { return kbuf[j]; };
 
   bool keep_all = false;
   uint32_t budget = 0u;
   Cut cut{0u, 0u};
   if (mode == SEL_THRESHOLD || mode == SEL_ROUTING) {
-    unsigned long long part = 0ull;
-    for (int j = lane; j < nb; j += 32) part += fix48(skey(j));
+    unsigned long long part = stage(srow, true);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
     const unsigned long long tau_fx = (unsigned long long)((double)tau * kFix);
@@ -228,13 +241,13 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(
       keep_all = true;
       budget = (uint32_t)nb;
     } else if (tau_fx == 0ull) {
-      cut = warp_radix_cut(skey, nb, false, 0ull, 1u, h);       // the shortest prefix is one block
+      cut = warp_radix_cut(key_at, nb, false, 0ull, 1u, h);     // the shortest prefix is one block
       budget = 1u;
     } else {
-      cut = warp_radix_cut(skey, nb, true, tau_fx, 0u, h);
+      cut = warp_radix_cut(key_at, nb, true, tau_fx, 0u, h);
       // budget = kept count: keys above vstar plus `take`
       uint32_t above = 0u;
-      for (int j = lane; j < nb; j += 32) above += skey(j) > cut.vstar ? 1u : 0u;
+      for (int j = lane; j < nb; j += 32) above += key_at(j) > cut.vstar ? 1u : 0u;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
       budget = above + cut.take;
@@ -242,14 +255,19 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(
   } else {  // TOPK
     budget = (uint32_t)k;
     if (k >= nb) keep_all = true;
-    else cut = warp_radix_cut(skey, nb, false, 0ull, (uint32_t)k, h);
+    else {
+      stage(srow, false);
+      cut = warp_radix_cut(key_at, nb, false, 0ull, (uint32_t)k, h);
+    }
   }
-  const float* rrow = R != nullptr ? R + row * (long long)nb : nullptr;
-  auto rkey = [&](int j) { return score_key(__ldg(rrow + j)); };
   const bool by_ratio = mode == SEL_ROUTING && !keep_all;
   if (by_ratio) {
     if (budget >= (uint32_t)nb) keep_all = true;
-    else cut = warp_radix_cut(rkey, nb, false, 0ull, budget, h);
+    else {
+      __syncwarp();                      // every lane is done with the score keys
+      stage(rrow, false);                // the cut and the compaction below read the ratios
+      cut = warp_radix_cut(key_at, nb, false, 0ull, budget, h);
+    }
   }
 
   int32_t* idx_out = kv_idx + row * (long long)cap;
@@ -260,7 +278,7 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(
     bool f = j < nb;
     bool eq = false;
     if (!keep_all && f) {
-      const uint32_t key = by_ratio ? rkey(j) : skey(j);
+      const uint32_t key = key_at(j);
       eq = key == cut.vstar;
       f = key > cut.vstar;
     }
@@ -273,6 +291,224 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_kernel(
     run += (uint32_t)__popc(fb);
   }
   if (lane == 0) kv_cnt[row] = (int32_t)run;
+}
+
+// ---------------------------------------------------------------- one CTA per row
+// Long rows (nb > kRowNbMin): a CTA of kRowThreads threads per row, the row's
+// keys staged in shared memory once.  Same radix cut as the warp version: a
+// 256-bin histogram per digit (one copy per warp, merged per bin, so that the
+// shared-memory atomics of different warps never meet on one address), a
+// block scan over the bins in descending digit order, and the one bin where
+// the cumulative count or mass reaches its target.
+constexpr int kRowThreads = 256;
+constexpr int kRowWarps = kRowThreads / 32;
+constexpr int kRowNbMin = 1024;
+static_assert(kRowThreads == 256, "one histogram bin per thread");
+
+struct RowShared {
+  uint32_t cnt[kRowWarps][256];                 // one histogram per warp
+  unsigned long long mass[kRowWarps][256];
+  uint32_t wc[kRowWarps];
+  unsigned long long wm[kRowWarps];
+  int hit_digit;
+  uint32_t hit_above_c, hit_c;
+  unsigned long long hit_above_m;
+  uint32_t run, eq_run;
+};
+
+// Inclusive block scan of (c, m) over threadIdx.x (all kRowThreads threads call it).
+__device__ __forceinline__ void row_scan(uint32_t& c, unsigned long long& m, RowShared& sh) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t yc = __shfl_up_sync(0xffffffffu, c, o);
+    const unsigned long long ym = __shfl_up_sync(0xffffffffu, m, o);
+    if (lane >= o) { c += yc; m += ym; }
+  }
+  if (lane == 31) { sh.wc[wid] = c; sh.wm[wid] = m; }
+  __syncthreads();
+  uint32_t oc = 0u;
+  unsigned long long om = 0ull;
+  for (int w = 0; w < wid; ++w) { oc += sh.wc[w]; om += sh.wm[w]; }
+  c += oc;
+  m += om;
+  __syncthreads();
+}
+
+struct RowCut {
+  uint32_t vstar;       // the crossing key
+  uint32_t take;        // keys equal to vstar kept (first in index order)
+  uint32_t above;       // keys strictly above vstar
+};
+
+// by_mass: the shortest prefix of the (key desc, index asc) order whose mass
+// reaches tau_fx (reachable: the caller checked the row's total); else the
+// first k (1 <= k < nb).
+__device__ RowCut row_radix_cut(const uint32_t* keys, int nb, bool by_mass, unsigned long long tau_fx, uint32_t k,
+                                RowShared& sh) {
+  const int tid = threadIdx.x, wid = tid >> 5;
+  uint32_t prefix = 0u, pmask = 0u, above_c = 0u, eq_c = 0u;
+  unsigned long long above_m = 0ull;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+#pragma unroll
+    for (int w = 0; w < kRowWarps; ++w) {   // bin tid of every warp's histogram
+      sh.cnt[w][tid] = 0u;
+      sh.mass[w][tid] = 0ull;
+    }
+    if (tid == 0) {                    // (a reachable target always overwrites these)
+      sh.hit_digit = 0;
+      sh.hit_above_c = above_c;
+      sh.hit_above_m = above_m;
+      sh.hit_c = 0u;
+    }
+    __syncthreads();
+    for (int base = 0; base < nb; base += kRowThreads) {
+      const int j = base + tid;
+      const uint32_t key = j < nb ? keys[j] : 0u;
+      const bool cand = j < nb && (key & pmask) == prefix;
+      if (cand) {                      // this warp's own histogram
+        const uint32_t dg = (key >> shift) & 255u;
+        if (by_mass) atomicAdd(&sh.mass[wid][dg], fix48(key));
+        atomicAdd(&sh.cnt[wid][dg], 1u);
+      }
+    }
+    __syncthreads();
+    // thread t owns digit 255 - t: scan in descending digit order
+    uint32_t c = 0u;
+    unsigned long long m = 0ull;
+#pragma unroll
+    for (int w = 0; w < kRowWarps; ++w) {
+      c += sh.cnt[w][255 - tid];
+      m += sh.mass[w][255 - tid];
+    }
+    uint32_t sc = c;
+    unsigned long long sm = m;
+    row_scan(sc, sm, sh);
+    const uint32_t ex_c = above_c + sc - c;
+    const unsigned long long ex_m = above_m + sm - m;
+    const bool reach = by_mass ? (ex_m + m >= tau_fx && ex_m < tau_fx) : (ex_c + c >= k && ex_c < k);
+    if (reach && c > 0u) {             // exact sums: exactly one thread
+      sh.hit_digit = 255 - tid;
+      sh.hit_above_c = ex_c;
+      sh.hit_above_m = ex_m;
+      sh.hit_c = c;
+    }
+    __syncthreads();
+    const int dg = sh.hit_digit;
+    above_c = sh.hit_above_c;
+    above_m = sh.hit_above_m;
+    eq_c = sh.hit_c;
+    prefix |= (uint32_t)dg << shift;
+    pmask |= 255u << shift;
+    __syncthreads();                   // the hit is read before the next pass clears the bins
+  }
+  RowCut cut;
+  cut.vstar = prefix;
+  cut.above = above_c;
+  if (by_mass) {
+    const unsigned long long v = fix48(prefix);
+    const unsigned long long need = tau_fx - above_m;           // > 0 by construction
+    unsigned long long t = v > 0ull ? (need + v - 1ull) / v : (unsigned long long)eq_c;
+    if (t < 1ull) t = 1ull;
+    if (t > eq_c) t = eq_c;
+    cut.take = (uint32_t)t;
+  } else {
+    cut.take = k - above_c;
+  }
+  return cut;
+}
+
+// Stage a row's keys; returns the row's fixed-point mass (every thread).
+__device__ unsigned long long row_stage(const float* __restrict__ src, int nb, uint32_t* keys, bool mass,
+                                        RowShared& sh) {
+  unsigned long long part = 0ull;
+  for (int j = threadIdx.x; j < nb; j += kRowThreads) {
+    const uint32_t key = score_key(__ldg(src + j));
+    keys[j] = key;
+    if (mass) part += fix48(key);
+  }
+  uint32_t c = 0u;
+  row_scan(c, part, sh);               // (also orders the staging stores before later reads)
+  if (threadIdx.x == kRowThreads - 1) sh.hit_above_m = part;
+  __syncthreads();
+  const unsigned long long total = sh.hit_above_m;
+  __syncthreads();
+  return total;
+}
+
+__global__ void __launch_bounds__(kRowThreads, 4) select_row_kernel(
+    const float* __restrict__ S, const float* __restrict__ R, int nb, int mode, float tau, int k, int cap,
+    int32_t* __restrict__ kv_idx, int32_t* __restrict__ kv_cnt, uint32_t* __restrict__ bits) {
+  extern __shared__ __align__(16) uint32_t row_keys[];
+  __shared__ RowShared sh;
+  const long long row = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int words = (nb + 31) / 32;
+  bool keep_all = false;
+  uint32_t budget = 0u;
+  RowCut cut{0u, 0u, 0u};
+  if (mode == SEL_THRESHOLD || mode == SEL_ROUTING) {
+    const unsigned long long total = row_stage(S + row * (long long)nb, nb, row_keys, true, sh);
+    const unsigned long long tau_fx = (unsigned long long)((double)tau * kFix);
+    if ((double)tau >= 1.0 || total < tau_fx) {
+      keep_all = true;
+      budget = (uint32_t)nb;
+    } else if (tau_fx == 0ull) {
+      cut = row_radix_cut(row_keys, nb, false, 0ull, 1u, sh);   // the shortest prefix is one block
+      budget = 1u;
+    } else {
+      cut = row_radix_cut(row_keys, nb, true, tau_fx, 0u, sh);
+      budget = cut.above + cut.take;
+    }
+  } else {  // TOPK
+    budget = (uint32_t)k;
+    if (k >= nb) keep_all = true;
+    else {
+      row_stage(S + row * (long long)nb, nb, row_keys, false, sh);
+      cut = row_radix_cut(row_keys, nb, false, 0ull, (uint32_t)k, sh);
+    }
+  }
+  if (mode == SEL_ROUTING && !keep_all) {
+    if (budget >= (uint32_t)nb) keep_all = true;
+    else {
+      row_stage(R + row * (long long)nb, nb, row_keys, false, sh);   // the ratios replace the scores
+      cut = row_radix_cut(row_keys, nb, false, 0ull, budget, sh);
+    }
+  }
+
+  // compaction in index order: keys above vstar, then the first `take` equal to it
+  int32_t* idx_out = kv_idx + row * (long long)cap;
+  uint32_t* bits_out = bits ? bits + row * (long long)words : nullptr;
+  if (tid == 0) { sh.run = 0u; sh.eq_run = 0u; }
+  __syncthreads();
+  for (int base = 0; base < nb; base += kRowThreads) {
+    const int j = base + tid;
+    const uint32_t key = (j < nb && !keep_all) ? row_keys[j] : 0u;
+    const bool gt = j < nb && (keep_all || key > cut.vstar);
+    const bool eq = j < nb && !keep_all && key == cut.vstar;
+    // one scan of (above count, equal count): both fit 16 bits per chunk
+    uint32_t packed = (gt ? 1u : 0u) | (eq ? 0x10000u : 0u);
+    unsigned long long unused = 0ull;
+    row_scan(packed, unused, sh);
+    const uint32_t own = (gt ? 1u : 0u) | (eq ? 0x10000u : 0u);
+    const uint32_t ex = packed - own;                   // exclusive prefix
+    const uint32_t run = sh.run, eq_run = sh.eq_run;
+    const uint32_t eq_left = cut.take > eq_run ? cut.take - eq_run : 0u;   // equal keys still to keep
+    const uint32_t ex_gt = ex & 0xFFFFu, ex_eq = ex >> 16;
+    const bool f = gt || (eq && ex_eq < eq_left);
+    const uint32_t pos = run + ex_gt + (ex_eq < eq_left ? ex_eq : eq_left);
+    if (f) idx_out[pos] = j;
+    const uint32_t fb = __ballot_sync(0xffffffffu, f);
+    if (bits_out != nullptr && lane == 0 && base + wid * 32 < nb) bits_out[(base >> 5) + wid] = fb;
+    __syncthreads();                                    // every thread has read run / eq_run
+    if (tid == kRowThreads - 1) {
+      const uint32_t tot_gt = packed & 0xFFFFu, tot_eq = packed >> 16;
+      sh.run = run + tot_gt + (tot_eq < eq_left ? tot_eq : eq_left);
+      sh.eq_run = eq_run + tot_eq;
+    }
+    __syncthreads();
+  }
+  if (tid == 0) kv_cnt[row] = (int32_t)sh.run;
 }
 
 // STRUCTURED: block coordinates from the raster id of each block's first token.
@@ -309,9 +545,31 @@ __global__ void __launch_bounds__(kSelThreads) structured_kernel(
 cudaError_t launch_select(const float* S, const float* R, long long rows, int nb, int mode, float tau,
                           int k, int cap, int32_t* kv_idx, int32_t* kv_cnt, uint32_t* bits,
                           cudaStream_t st) {
-  const long long blocks = (rows + kSelWarps - 1) / kSelWarps;
-  select_kernel<<<(unsigned)blocks, kSelWarps * 32, 0, st>>>(S, R, rows, nb, mode, tau, k, cap, kv_idx, kv_cnt,
-                                                             bits);
+  if (nb > kRowNbMin) {
+    // long rows: one CTA per row, its keys staged in shared memory
+    const size_t smem = (size_t)nb * sizeof(uint32_t);
+    if (smem + sizeof(RowShared) > kSelMaxSmem) return cudaErrorInvalidValue;
+    if (smem > 48 * 1024 - sizeof(RowShared)) {
+      const cudaError_t e = cudaFuncSetAttribute(select_row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)smem);
+      if (e != cudaSuccess) return e;
+    }
+    select_row_kernel<<<(unsigned)rows, kRowThreads, smem, st>>>(S, R, nb, mode, tau, k, cap, kv_idx, kv_cnt, bits);
+    return cudaGetLastError();
+  }
+  // short rows: one warp per row, as many rows per CTA (up to 4) as fit in
+  // shared memory with their keys
+  const size_t per_warp = sizeof(WarpHist) + (size_t)nb * sizeof(uint32_t);
+  const int warps = (int)std::min<size_t>(kSelMaxWarps, kSelMaxSmem / per_warp);
+  if (warps < 1) return cudaErrorInvalidValue;
+  const size_t smem = (size_t)warps * per_warp;
+  if (smem > 48 * 1024) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  const long long blocks = (rows + warps - 1) / warps;
+  select_kernel<<<(unsigned)blocks, warps * 32, smem, st>>>(S, R, rows, nb, mode, tau, k, cap, kv_idx, kv_cnt, bits);
   return cudaGetLastError();
 }
 

@@ -161,6 +161,32 @@ def test_routing_masks(sub, d, grid, heads):
     _run_and_compare_masks(w)
 
 
+@pytest.mark.parametrize("select,kw", [
+    ("threshold", dict(tau=0.9)),
+    ("threshold", dict(tau=0.5)),
+    ("threshold", dict(tau=0.0)),                   # shortest prefix: one block
+    ("topk", dict(keep_frac=0.3)),
+    ("threshold", dict(tau=0.9, routing=True)),
+    ("threshold", dict(tau=0.9, sub_block=16)),
+])
+def test_long_row_selection(select, kw):
+    """nb = 1129 (> 1024): rows selected by one CTA each; sampled rows against
+    the oracle, every row's list and bit row checked for consistency."""
+    sub = kw.pop("sub_block", 64)
+    w = _small(select, sub, grid=(10, 20, 361), heads=1, d=64, **kw)
+    q, k, v = (t.cuda() for t in workloads.make_qkv(w, seed=3))
+    attn = gpu_layer(w, q, k, v)
+    assert attn.nb == 1129
+    keep = gpu_keep(attn)
+    perm, _ = oracle.build_perm(w.T, w.H, w.W, w.order)
+    qp, kp, vp = (oracle.reorder(to_np(t)[0].astype(np.float64), perm) for t in (q, k, v))
+    rows = sorted(set(range(0, attn.nb, 61)) | {attn.nb - 1})
+    kept, near = oracle_rows(w, qp[0], kp[0], vp[0], perm, rows)
+    compare_mask_rows(keep[0][rows], kept, near)
+    if select == "threshold" and kw.get("tau") == 0.0:
+        assert np.all(keep[0].sum(axis=1) == 1)
+
+
 @pytest.mark.parametrize("select,start,end", [("threshold", 0.97, 0.7), ("topk", 0.6, 0.25)])
 def test_schedule_run_matches_oracle(select, start, end):
     """An 8-step run under the step schedule (2 dense steps, mask rebuilt every 3
