@@ -23,22 +23,23 @@
 // kernel combines the key ranges and rescales: r_IJ = e_IJ 2^(m_IJ - M) / Z
 // * 64 / n_J.
 //
-// Warp 0 issues the TMA copies (qbar tile per item; K_J and V_J per tile into
-// a 2-stage ring; the fp32 centroid value row vbar_J per tile into a 4-deep
-// ring that the error epilogue releases), warp 1 issues the MMAs (S of tile
-// t+1 ahead of the E.V of tile t) and owns TMEM, warps 2-5 hold one proxy per
-// thread: exponentials, the E split into shared memory, and the error
-// epilogue of the previous tile while the tensor core works on the next one.
-// Every wait is bounded.
+// Warp 0 issues the TMA copies of the qbar tile per item and of K_J per tile
+// (3-stage ring, freed when S_J is done); warp 10 those of V_J (2-stage ring,
+// freed when E.V_J is done) and the fp32 centroid value row vbar_J (4-deep
+// ring, freed by the error epilogue).  Warp 1 issues the MMAs (S of tile t+1
+// ahead of the E.V of tile t) and owns TMEM.  Two warpgroups hold one
+// proxy per thread: warps 2-5 take the exponentials and the E split of every
+// tile, warps 6-9 the error epilogue of the tiles whose E.V has finished, so
+// the two run side by side on different tiles.  Every wait is bounded.
 #include "tcgen05.cuh"
 
 namespace svsa {
 namespace tc {
 namespace route {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 352;
 constexpr int kRows = 128;                   // proxies per item
-constexpr int kStages = 2, kSBufs = 2, kEBufs = 2, kOBufs = 2, kVbBufs = 4;
+constexpr int kKStages = 3, kVStages = 2, kSBufs = 2, kEBufs = 2, kOBufs = 2, kVbBufs = 4, kMBufs = 4;
 constexpr uint32_t kBoxQ = kRows * 128;      // 128 rows x 64 bf16 (16 KB)
 constexpr uint32_t kBoxK = kBlock * 128;     // 64 rows x 64 elements (8 KB)
 constexpr uint32_t kEPart = kRows * 128;     // E hi or lo: 128 proxies x 64 fp16 (16 KB)
@@ -47,13 +48,15 @@ template <int D>
 struct Smem {
   static constexpr int NCH = D / 64;
   static constexpr uint32_t kQ = 2 * NCH * kBoxQ;          // qbar hi and lo
-  static constexpr uint32_t kStage = 2 * NCH * kBoxK;      // K_J then V_J
+  static constexpr uint32_t kStage = NCH * kBoxK;          // one K_J or V_J tile
   static constexpr uint32_t kOffQ = 0;
-  static constexpr uint32_t kOffKV = kQ;
-  static constexpr uint32_t kOffE = kOffKV + kStages * kStage;
+  static constexpr uint32_t kOffK = kQ;
+  static constexpr uint32_t kOffV = kOffK + kKStages * kStage;
+  static constexpr uint32_t kOffE = kOffV + kVStages * kStage;
   static constexpr uint32_t kVb = D * 4;                      // one fp32 centroid value row
   static constexpr uint32_t kOffVb = kOffE + kEBufs * 2 * kEPart;
-  static constexpr uint32_t kOffMisc = kOffVb + kVbBufs * kVb;
+  static constexpr uint32_t kOffM = kOffVb + kVbBufs * kVb;     // per-tile maxima, kMBufs x kRows floats
+  static constexpr uint32_t kOffMisc = kOffM + kMBufs * kRows * 4;
   static constexpr uint32_t kBytes = kOffMisc + 512 + 1024;
   static_assert(kBytes <= 232448, "shared memory per CTA");
   // TMEM: S buffers (64 columns each), then O buffers (D columns each)
@@ -62,11 +65,13 @@ struct Smem {
 };
 
 enum : uint32_t {
-  BAR_Q_FULL = 0, BAR_Q_EMPTY, BAR_KV_FULL, BAR_KV_EMPTY = BAR_KV_FULL + kStages,
-  BAR_S_FULL = BAR_KV_EMPTY + kStages, BAR_S_EMPTY = BAR_S_FULL + kSBufs,
+  BAR_Q_FULL = 0, BAR_Q_EMPTY, BAR_K_FULL, BAR_K_EMPTY = BAR_K_FULL + kKStages,
+  BAR_V_FULL = BAR_K_EMPTY + kKStages, BAR_V_EMPTY = BAR_V_FULL + kVStages,
+  BAR_S_FULL = BAR_V_EMPTY + kVStages, BAR_S_EMPTY = BAR_S_FULL + kSBufs,
   BAR_E_FULL = BAR_S_EMPTY + kSBufs, BAR_E_EMPTY = BAR_E_FULL + kEBufs,
   BAR_O_FULL = BAR_E_EMPTY + kEBufs, BAR_O_EMPTY = BAR_O_FULL + kOBufs,
-  BAR_VB_FULL = BAR_O_EMPTY + kOBufs, BAR_VB_EMPTY = BAR_VB_FULL + kVbBufs, BAR_FINAL = BAR_VB_EMPTY + kVbBufs,
+  BAR_VB_FULL = BAR_O_EMPTY + kOBufs, BAR_VB_EMPTY = BAR_VB_FULL + kVbBufs,
+  BAR_M_FULL = BAR_VB_EMPTY + kVbBufs, BAR_M_EMPTY = BAR_M_FULL + kMBufs, BAR_FINAL = BAR_M_EMPTY + kMBufs,
   NUM_BARS
 };
 
@@ -108,9 +113,13 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(const __grid_cons
   if (tid == 0) {
     mbar_init(bar(BAR_Q_FULL), 1);
     mbar_init(bar(BAR_Q_EMPTY), 1);
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(bar(BAR_KV_FULL + i), 1);
-      mbar_init(bar(BAR_KV_EMPTY + i), 1);
+    for (int i = 0; i < kKStages; ++i) {
+      mbar_init(bar(BAR_K_FULL + i), 1);
+      mbar_init(bar(BAR_K_EMPTY + i), 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(bar(BAR_V_FULL + i), 1);
+      mbar_init(bar(BAR_V_EMPTY + i), 1);
     }
     for (int i = 0; i < kSBufs; ++i) {
       mbar_init(bar(BAR_S_FULL + i), 1);
@@ -127,6 +136,10 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(const __grid_cons
     for (int i = 0; i < kVbBufs; ++i) {
       mbar_init(bar(BAR_VB_FULL + i), 1);
       mbar_init(bar(BAR_VB_EMPTY + i), 4);
+    }
+    for (int i = 0; i < kMBufs; ++i) {
+      mbar_init(bar(BAR_M_FULL + i), 4);
+      mbar_init(bar(BAR_M_EMPTY + i), 4);
     }
     mbar_init(bar(BAR_FINAL), 1);
     ms->abort = 0u;
@@ -152,9 +165,14 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(const __grid_cons
     j1 = min(nb, j0 + a.per);
   };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp == 0 || warp == 10) {
+    // ------------------------------------------------------------ TMA producers
+    // warp 0: the qbar tile of each item and K_J per tile (freed when S_J is
+    // done); warp 10: V_J per tile (freed when E.V_J is done) and the fp32
+    // centroid value row vbar_J (freed by the error epilogue).  Separate rings
+    // let the K loads run ahead of the slower V turnover.
     if (lane == 0) {
+      const bool is_k = warp == 0;
       uint32_t qit = 0, kn = 0;
       bool ok = true;
       for (long long it = blockIdx.x; it < a.items && ok; it += gridDim.x) {
@@ -162,43 +180,54 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(const __grid_cons
         int qt, j0, j1;
         decode(it, bh, qt, j0, j1);
         if (j0 >= j1) continue;
-        ok = wait_bar(bar(BAR_Q_EMPTY), (qit & 1u) ^ 1u, abort_flag, 51);
-        if (!ok) break;
-        mbar_expect_tx(bar(BAR_Q_FULL), L::kQ);
-        const int yq = (int)(bh * nb + (long long)qt * kRows);
-        for (int c = 0; c < 2 * NCH; ++c) tma_load_2d(sbase + L::kOffQ + c * kBoxQ, &tmQ, c * 64, yq, bar(BAR_Q_FULL));
-        ++qit;
+        if (is_k) {
+          ok = wait_bar(bar(BAR_Q_EMPTY), (qit & 1u) ^ 1u, abort_flag, 51);
+          if (!ok) break;
+          mbar_expect_tx(bar(BAR_Q_FULL), L::kQ);
+          const int yq = (int)(bh * nb + (long long)qt * kRows);
+          for (int c = 0; c < 2 * NCH; ++c)
+            tma_load_2d(sbase + L::kOffQ + c * kBoxQ, &tmQ, c * 64, yq, bar(BAR_Q_FULL));
+          ++qit;
+        }
         for (int J = j0; J < j1 && ok; ++J) {
-          const uint32_t stg = kn % kStages;
-          ok = wait_bar(bar(BAR_KV_EMPTY + stg), ((kn / kStages) & 1u) ^ 1u, abort_flag, 52);
-          if (!ok) break;
-          mbar_expect_tx(bar(BAR_KV_FULL + stg), L::kStage);
           const int yk = (int)(bh * a.Npad + (long long)J * kBlock);
-          const uint32_t dst = sbase + L::kOffKV + stg * L::kStage;
-          for (int c = 0; c < NCH; ++c) {
-            tma_load_2d(dst + c * kBoxK, &tmK, c * 64, yk, bar(BAR_KV_FULL + stg));
-            tma_load_2d(dst + (NCH + c) * kBoxK, &tmV, c * 64, yk, bar(BAR_KV_FULL + stg));
+          if (is_k) {
+            const uint32_t stg = kn % kKStages;
+            ok = wait_bar(bar(BAR_K_EMPTY + stg), ((kn / kKStages) & 1u) ^ 1u, abort_flag, 52);
+            if (!ok) break;
+            mbar_expect_tx(bar(BAR_K_FULL + stg), L::kStage);
+            for (int c = 0; c < NCH; ++c)
+              tma_load_2d(sbase + L::kOffK + stg * L::kStage + c * kBoxK, &tmK, c * 64, yk, bar(BAR_K_FULL + stg));
+          } else {
+            const uint32_t stg = kn % kVStages;
+            ok = wait_bar(bar(BAR_V_EMPTY + stg), ((kn / kVStages) & 1u) ^ 1u, abort_flag, 69);
+            if (!ok) break;
+            mbar_expect_tx(bar(BAR_V_FULL + stg), L::kStage);
+            for (int c = 0; c < NCH; ++c)
+              tma_load_2d(sbase + L::kOffV + stg * L::kStage + c * kBoxK, &tmV, c * 64, yk, bar(BAR_V_FULL + stg));
+            const uint32_t vs = kn % kVbBufs;
+            ok = wait_bar(bar(BAR_VB_EMPTY + vs), ((kn / kVbBufs) & 1u) ^ 1u, abort_flag, 64);
+            if (!ok) break;
+            mbar_expect_tx(bar(BAR_VB_FULL + vs), L::kVb);
+            bulk_load(sbase + L::kOffVb + vs * L::kVb, a.vbar + (bh * nb + J) * (long long)D, L::kVb,
+                      bar(BAR_VB_FULL + vs));
           }
-          // the centroid value row of block J for this tile's error epilogue
-          const uint32_t vs = kn % kVbBufs;
-          ok = wait_bar(bar(BAR_VB_EMPTY + vs), ((kn / kVbBufs) & 1u) ^ 1u, abort_flag, 64);
-          if (!ok) break;
-          mbar_expect_tx(bar(BAR_VB_FULL + vs), L::kVb);
-          bulk_load(sbase + L::kOffVb + vs * L::kVb, a.vbar + (bh * nb + J) * (long long)D, L::kVb,
-                    bar(BAR_VB_FULL + vs));
           ++kn;
         }
       }
+      // never leave with copies in flight: wait (bounded) for the last fill of every ring slot
       volatile uint32_t no_abort = 0u;
       if (qit > 0) wait_bar(bar(BAR_Q_FULL), (qit - 1) & 1u, &no_abort, 60);
-      for (uint32_t j = 1; j <= (uint32_t)kStages && j <= kn; ++j) {
+      const uint32_t stages = is_k ? (uint32_t)kKStages : (uint32_t)kVStages;
+      for (uint32_t j = 1; j <= stages && j <= kn; ++j) {
         const uint32_t n = kn - j;
-        wait_bar(bar(BAR_KV_FULL + n % kStages), (n / kStages) & 1u, &no_abort, 61);
+        wait_bar(bar((is_k ? BAR_K_FULL : BAR_V_FULL) + n % stages), (n / stages) & 1u, &no_abort, 61);
       }
-      for (uint32_t j = 1; j <= (uint32_t)kVbBufs && j <= kn; ++j) {
-        const uint32_t n = kn - j;
-        wait_bar(bar(BAR_VB_FULL + n % kVbBufs), (n / kVbBufs) & 1u, &no_abort, 65);
-      }
+      if (!is_k)
+        for (uint32_t j = 1; j <= (uint32_t)kVbBufs && j <= kn; ++j) {
+          const uint32_t n = kn - j;
+          wait_bar(bar(BAR_VB_FULL + n % kVbBufs), (n / kVbBufs) & 1u, &no_abort, 65);
+        }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -206,30 +235,32 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(const __grid_cons
       constexpr uint32_t ID_S = idesc_f16(true, false, false, 64, kRows);     // bf16 Qbar . K^T
       constexpr uint32_t ID_O = idesc_f16(false, false, true, D, kRows);      // fp16 E . V (V MN-major)
       const uint64_t dQ = sdesc(sbase + L::kOffQ, 16, 1024);
-      const uint64_t dKV = sdesc(sbase + L::kOffKV, 16, 1024);
-      const uint64_t dVm = sdesc(sbase + L::kOffKV + NCH * kBoxK, kBoxK, 1024);
+      const uint64_t dK = sdesc(sbase + L::kOffK, 16, 1024);
+      const uint64_t dVm = sdesc(sbase + L::kOffV, kBoxK, 1024);
       const uint64_t dE = sdesc(sbase + L::kOffE, 16, 1024);
-      uint32_t qit = 0, kn = 0, pn = 0;     // K/V ring position of the next S, of the next E.V
+      uint32_t qit = 0, kn = 0, pn = 0;     // tile index of the next S, of the next E.V
       bool ok = true;
       auto issue_s = [&](uint32_t n) -> bool {
-        const uint32_t stg = n % kStages, sb = n % kSBufs;
-        if (!wait_bar(bar(BAR_KV_FULL + stg), (n / kStages) & 1u, abort_flag, 53) ||
+        const uint32_t stg = n % kKStages, sb = n % kSBufs;
+        if (!wait_bar(bar(BAR_K_FULL + stg), (n / kKStages) & 1u, abort_flag, 53) ||
             !wait_bar(bar(BAR_S_EMPTY + sb), ((n / kSBufs) & 1u) ^ 1u, abort_flag, 54))
           return false;
         tc_fence_after();
-        const uint64_t k0 = dKV + ((stg * L::kStage) >> 4);
+        const uint64_t k0 = dK + ((stg * L::kStage) >> 4);
 #pragma unroll
         for (int part = 0; part < 2; ++part)
 #pragma unroll
           for (int kk = 0; kk < KSTEPS; ++kk)
             umma_f16(tmem + L::kColS + sb * 64, dQ + ((((part * NCH) + (kk >> 2)) * kBoxQ + (kk & 3) * 32) >> 4),
                      k0 + ((((kk >> 2)) * kBoxK + (kk & 3) * 32) >> 4), ID_S, (part > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(bar(BAR_K_EMPTY + stg));
         umma_commit(bar(BAR_S_FULL + sb));
         return true;
       };
       auto issue_o = [&](uint32_t n) -> bool {
-        const uint32_t stg = n % kStages, eb = n % kEBufs, ob = n % kOBufs;
-        if (!wait_bar(bar(BAR_E_FULL + eb), (n / kEBufs) & 1u, abort_flag, 55) ||
+        const uint32_t stg = n % kVStages, eb = n % kEBufs, ob = n % kOBufs;
+        if (!wait_bar(bar(BAR_V_FULL + stg), (n / kVStages) & 1u, abort_flag, 70) ||
+            !wait_bar(bar(BAR_E_FULL + eb), (n / kEBufs) & 1u, abort_flag, 55) ||
             !wait_bar(bar(BAR_O_EMPTY + ob), ((n / kOBufs) & 1u) ^ 1u, abort_flag, 56))
           return false;
         tc_fence_after();
@@ -241,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(const __grid_cons
           for (int kk = 0; kk < 4; ++kk)
             umma_f16(tmem + L::kColO + ob * D, e0 + ((part * kEPart + kk * 32) >> 4), v0 + ((kk * 2048) >> 4), ID_O,
                      (part > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(bar(BAR_KV_EMPTY + stg));
+        umma_commit(bar(BAR_V_EMPTY + stg));
         umma_commit(bar(BAR_E_EMPTY + eb));
         umma_commit(bar(BAR_O_FULL + ob));
         return true;
@@ -266,8 +297,11 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(const __grid_cons
       volatile uint32_t no_abort = 0u;
       wait_bar(bar(BAR_FINAL), 0u, &no_abort, 62);
     }
-  } else {
-    // ------------------------------------------------------------ one proxy per thread
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ proxies: exponentials
+    // One proxy per thread (warps 2-5): the tile's exponentials against the
+    // running maximum, the E split into shared memory, and the maximum used
+    // for the tile into the M ring for the error warps.
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
@@ -275,6 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(const __grid_cons
     const int n_in_last = (int)(a.N - (long long)(nb - 1) * kBlock);
     // this thread's E row in the K-major 128-byte-swizzled layout
     unsigned char* const erow0 = smem + L::kOffE + (row >> 3) * 1024 + (row & 7) * 128;
+    float* const mring = reinterpret_cast<float*>(smem + L::kOffM);
     uint32_t sn = 0;
     bool stop = false;
     for (long long it = blockIdx.x; it < a.items && !stop; it += gridDim.x) {
@@ -292,51 +327,9 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(const __grid_cons
         }
         continue;
       }
-      const long long rbase = (bh * nb + (row_ok ? I : 0)) * (long long)nb;
       float m = -INFINITY, Z = 0.f;
-      float m_prev = 0.f, L_prev = 0.f;
-      int J_prev = -1;
-      // error epilogue of tile n (block J, weights against m_used; LJ = the
-      // proxy's centroid logit of block J, loaded one tile earlier)
-      auto epilogue = [&](uint32_t n, int J, float m_used, float LJ) -> bool {
-        const uint32_t ob = n % kOBufs, vs = n % kVbBufs;
-        if (!wait_bar(bar(BAR_O_FULL + ob), (n / kOBufs) & 1u, abort_flag, 58) ||
-            !wait_bar(bar(BAR_VB_FULL + vs), (n / kVbBufs) & 1u, abort_flag, 66))
-          return false;
-        tc_fence_after();
-        const int nJ = J == nb - 1 ? n_in_last : kBlock;
-        const float cw = row_ok ? (float)nJ * ex2(LJ - m_used) : 0.f;
-        const float4* vb = reinterpret_cast<const float4*>(smem + L::kOffVb + vs * L::kVb);
-        float err2 = 0.f;
-#pragma unroll 1
-        for (int ch = 0; ch < D / 32; ++ch) {
-          float o[32];
-          tmem_ld32(tmem + lane_off + L::kColO + ob * D + ch * 32, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 32; c += 4) {
-            const float4 v4 = vb[ch * 8 + c / 4];       // same address in every lane: broadcast
-            const float d0 = fmaf(-cw, v4.x, o[c]), d1 = fmaf(-cw, v4.y, o[c + 1]);
-            const float d2 = fmaf(-cw, v4.z, o[c + 2]), d3 = fmaf(-cw, v4.w, o[c + 3]);
-            err2 = fmaf(d0, d0, fmaf(d1, d1, fmaf(d2, d2, fmaf(d3, d3, err2))));
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(bar(BAR_O_EMPTY + ob));
-          mbar_arrive(bar(BAR_VB_EMPTY + vs));
-        }
-        if (row_ok) {
-          a.R[rbase + J] = sqrtf(err2);
-          a.Rm[rbase + J] = m_used;
-        }
-        return true;
-      };
       for (int J = j0; J < j1; ++J) {
-        const uint32_t sb = sn % kSBufs, eb = sn % kEBufs;
-        // this tile's centroid logit, used by its epilogue one tile later
-        const float L_cur = row_ok ? __ldg(a.L + rbase + J) : 0.f;
+        const uint32_t sb = sn % kSBufs, eb = sn % kEBufs, mb = sn % kMBufs;
         if (!wait_bar(bar(BAR_S_FULL + sb), (sn / kSBufs) & 1u, abort_flag, 59)) { stop = true; break; }
         tc_fence_after();
         float x[64];
@@ -368,7 +361,11 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(const __grid_cons
         }
         Z = (m == -INFINITY ? 0.f : Z * ex2(m - mn)) + sum;
         m = mn;
-        if (!wait_bar(bar(BAR_E_EMPTY + eb), ((sn / kEBufs) & 1u) ^ 1u, abort_flag, 63)) { stop = true; break; }
+        if (!wait_bar(bar(BAR_E_EMPTY + eb), ((sn / kEBufs) & 1u) ^ 1u, abort_flag, 63) ||
+            !wait_bar(bar(BAR_M_EMPTY + mb), ((sn / kMBufs) & 1u) ^ 1u, abort_flag, 67)) {
+          stop = true;
+          break;
+        }
         unsigned char* erow = erow0 + eb * 2 * kEPart;
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
@@ -377,22 +374,85 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(const __grid_cons
           *reinterpret_cast<uint4*>(erow + kEPart + off) =
               make_uint4(lo[4 * ch], lo[4 * ch + 1], lo[4 * ch + 2], lo[4 * ch + 3]);
         }
+        mring[mb * kRows + row] = m;
         fence_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(BAR_E_FULL + eb));
-        if (J_prev >= 0 && !epilogue(sn - 1, J_prev, m_prev, L_prev)) { stop = true; break; }
-        J_prev = J;
-        m_prev = m;
-        L_prev = L_cur;
+        if (lane == 0) {
+          mbar_arrive(bar(BAR_E_FULL + eb));
+          mbar_arrive(bar(BAR_M_FULL + mb));
+        }
         ++sn;
       }
       if (stop) break;
-      if (J_prev >= 0 && !epilogue(sn - 1, J_prev, m_prev, L_prev)) break;
       if (row_ok) {
         const long long p = (bh * nb + I) * (long long)a.nsplit + it % a.nsplit;
         a.Mp[p] = m;
         a.Zp[p] = Z;
+      }
+    }
+  } else if (warp < 10) {
+    // ------------------------------------------------------------ proxies: error epilogue
+    // One proxy per thread (warps 6-9, same TMEM lane quadrants as 2-5): for
+    // every tile, in the same order, e_IJ = || O_I - n_J 2^(L_IJ - m) vbar_J ||
+    // against the maximum m the exponential warps used for that tile.
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const int n_in_last = (int)(a.N - (long long)(nb - 1) * kBlock);
+    const float* const mring = reinterpret_cast<const float*>(smem + L::kOffM);
+    uint32_t n = 0;
+    bool stop = false;
+    for (long long it = blockIdx.x; it < a.items && !stop; it += gridDim.x) {
+      long long bh;
+      int qt, j0, j1;
+      decode(it, bh, qt, j0, j1);
+      if (j0 >= j1) continue;
+      const int I = qt * kRows + row;
+      const bool row_ok = I < nb;
+      const long long rbase = (bh * nb + (row_ok ? I : 0)) * (long long)nb;
+      float L_next = row_ok ? __ldg(a.L + rbase + j0) : 0.f;     // centroid logits, one tile ahead
+      for (int J = j0; J < j1; ++J) {
+        const float LJ = L_next;
+        if (J + 1 < j1) L_next = row_ok ? __ldg(a.L + rbase + J + 1) : 0.f;
+        const uint32_t ob = n % kOBufs, vs = n % kVbBufs, mb = n % kMBufs;
+        if (!wait_bar(bar(BAR_M_FULL + mb), (n / kMBufs) & 1u, abort_flag, 68) ||
+            !wait_bar(bar(BAR_O_FULL + ob), (n / kOBufs) & 1u, abort_flag, 58) ||
+            !wait_bar(bar(BAR_VB_FULL + vs), (n / kVbBufs) & 1u, abort_flag, 66)) {
+          stop = true;
+          break;
+        }
+        tc_fence_after();
+        const float m_used = mring[mb * kRows + row];
+        const int nJ = J == nb - 1 ? n_in_last : kBlock;
+        const float cw = row_ok ? (float)nJ * ex2(LJ - m_used) : 0.f;
+        const float4* vb = reinterpret_cast<const float4*>(smem + L::kOffVb + vs * L::kVb);
+        float err2 = 0.f;
+#pragma unroll 1
+        for (int ch = 0; ch < D / 32; ++ch) {
+          float o[32];
+          tmem_ld32(tmem + lane_off + L::kColO + ob * D + ch * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; c += 4) {
+            const float4 v4 = vb[ch * 8 + c / 4];       // same address in every lane: broadcast
+            const float d0 = fmaf(-cw, v4.x, o[c]), d1 = fmaf(-cw, v4.y, o[c + 1]);
+            const float d2 = fmaf(-cw, v4.z, o[c + 2]), d3 = fmaf(-cw, v4.w, o[c + 3]);
+            err2 = fmaf(d0, d0, fmaf(d1, d1, fmaf(d2, d2, fmaf(d3, d3, err2))));
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(bar(BAR_O_EMPTY + ob));
+          mbar_arrive(bar(BAR_VB_EMPTY + vs));
+          mbar_arrive(bar(BAR_M_EMPTY + mb));
+        }
+        if (row_ok) {
+          a.R[rbase + J] = sqrtf(err2);
+          a.Rm[rbase + J] = m_used;
+        }
+        ++n;
       }
     }
   }
