@@ -26,8 +26,8 @@
 // Warp 0 issues the TMA copies of the qbar tile per item and of K_J per tile
 // (3-stage ring, freed when S_J is done); warp 10 those of V_J (2-stage ring,
 // freed when E.V_J is done) and the fp32 centroid value row vbar_J (4-deep
-// ring, freed by the error epilogue).  Warp 1 issues the MMAs (S of tile t+1
-// ahead of the E.V of tile t) and owns TMEM.  Two warpgroups hold one
+// ring, freed by the error epilogue).  Warp 1 issues the S MMAs and owns
+// TMEM, warp 11 the E.V MMAs.  Two warpgroups hold one
 // proxy per thread: warps 2-5 take the exponentials and the E split of every
 // tile, warps 6-9 the error epilogue of the tiles whose E.V has finished, so
 // the two run side by side on different tiles.  Every wait is bounded.
@@ -37,7 +37,7 @@ namespace svsa {
 namespace tc {
 namespace route {
 
-constexpr int kThreads = 352;
+constexpr int kThreads = 384;
 constexpr int kRows = 128;                   // proxies per item
 constexpr int kKStages = 3, kVStages = 2, kSBufs = 2, kEBufs = 2, kOBufs = 2, kVbBufs = 4, kMBufs = 4;
 constexpr uint32_t kBoxQ = kRows * 128;      // 128 rows x 64 bf16 (16 KB)
@@ -72,7 +72,7 @@ enum : uint32_t {
   BAR_O_FULL = BAR_E_EMPTY + kEBufs, BAR_O_EMPTY = BAR_O_FULL + kOBufs,
   BAR_VB_FULL = BAR_O_EMPTY + kOBufs, BAR_VB_EMPTY = BAR_VB_FULL + kVbBufs,
   BAR_M_FULL = BAR_VB_EMPTY + kVbBufs, BAR_M_EMPTY = BAR_M_FULL + kMBufs, BAR_FINAL = BAR_M_EMPTY + kMBufs,
-  NUM_BARS
+  BAR_FINAL2, NUM_BARS
 };
 
 struct Misc {
@@ -142,6 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(const __grid_cons
       mbar_init(bar(BAR_M_EMPTY + i), 4);
     }
     mbar_init(bar(BAR_FINAL), 1);
+    mbar_init(bar(BAR_FINAL2), 1);
     ms->abort = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
@@ -229,16 +230,20 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(const __grid_cons
           wait_bar(bar(BAR_VB_FULL + n % kVbBufs), (n / kVbBufs) & 1u, &no_abort, 65);
         }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 11) {
+    // ------------------------------------------------------------ MMA issuers
+    // warp 1: S = Qbar . K_J^T of every tile (runs ahead as far as the S ring
+    // allows); warp 11: O = E . V_J.  Two issuing threads keep the tensor core
+    // fed, and each commits (hence waits for) only its own MMAs.
     if (lane == 0) {
+      const bool s_issuer = warp == 1;
       constexpr uint32_t ID_S = idesc_f16(true, false, false, 64, kRows);     // bf16 Qbar . K^T
       constexpr uint32_t ID_O = idesc_f16(false, false, true, D, kRows);      // fp16 E . V (V MN-major)
       const uint64_t dQ = sdesc(sbase + L::kOffQ, 16, 1024);
       const uint64_t dK = sdesc(sbase + L::kOffK, 16, 1024);
       const uint64_t dVm = sdesc(sbase + L::kOffV, kBoxK, 1024);
       const uint64_t dE = sdesc(sbase + L::kOffE, 16, 1024);
-      uint32_t qit = 0, kn = 0, pn = 0;     // tile index of the next S, of the next E.V
+      uint32_t qit = 0, n = 0;              // this issuer's next tile
       bool ok = true;
       auto issue_s = [&](uint32_t n) -> bool {
         const uint32_t stg = n % kKStages, sb = n % kSBufs;
@@ -282,20 +287,21 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(const __grid_cons
         int qt, j0, j1;
         decode(it, bh, qt, j0, j1);
         if (j0 >= j1) continue;
-        ok = wait_bar(bar(BAR_Q_FULL), qit & 1u, abort_flag, 57);
-        ++qit;
-        const uint32_t first = kn;
-        for (int J = j0; J < j1 && ok; ++J) {
-          ok = issue_s(kn);
-          ++kn;
-          if (ok && kn - first >= 2) ok = issue_o(pn++);    // E.V of the previous tile
+        if (s_issuer) {
+          ok = wait_bar(bar(BAR_Q_FULL), qit & 1u, abort_flag, 57);
+          ++qit;
         }
-        if (ok) ok = issue_o(pn++);                         // the last tile of the item
-        if (ok) umma_commit(bar(BAR_Q_EMPTY));
+        for (int J = j0; J < j1 && ok; ++J) {
+          ok = s_issuer ? issue_s(n) : issue_o(n);
+          ++n;
+        }
+        if (s_issuer && ok) umma_commit(bar(BAR_Q_EMPTY));   // the item's S products have read qbar
       }
-      umma_commit(bar(BAR_FINAL));
+      // every MMA this thread issued has finished before TMEM is released
+      const uint32_t fin = s_issuer ? BAR_FINAL : BAR_FINAL2;
+      umma_commit(bar(fin));
       volatile uint32_t no_abort = 0u;
-      wait_bar(bar(BAR_FINAL), 0u, &no_abort, 62);
+      wait_bar(bar(fin), 0u, &no_abort, 62);
     }
   } else if (warp < 6) {
     // ------------------------------------------------------------ proxies: exponentials
