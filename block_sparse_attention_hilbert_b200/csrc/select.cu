@@ -310,10 +310,10 @@ struct RowShared {
   unsigned long long mass[kRowWarps][256];
   uint32_t wc[kRowWarps];
   unsigned long long wm[kRowWarps];
+  uint32_t eq_w[kRowWarps];
   int hit_digit;
   uint32_t hit_above_c, hit_c;
   unsigned long long hit_above_m;
-  uint32_t run, eq_run;
 };
 
 // Inclusive block scan of (c, m) over threadIdx.x (all kRowThreads threads call it).
@@ -476,39 +476,54 @@ __global__ void __launch_bounds__(kRowThreads, 4) select_row_kernel(
     }
   }
 
-  // compaction in index order: keys above vstar, then the first `take` equal to it
+  // compaction in index order: keys above vstar, then the first `take` equal
+  // to it.  Warp w owns the 32-aligned segment [w * seg, (w + 1) * seg): it
+  // counts its keys above / equal, one barrier publishes the per-warp counts,
+  // and each warp writes its kept indices at its offset.
   int32_t* idx_out = kv_idx + row * (long long)cap;
   uint32_t* bits_out = bits ? bits + row * (long long)words : nullptr;
-  if (tid == 0) { sh.run = 0u; sh.eq_run = 0u; }
-  __syncthreads();
-  for (int base = 0; base < nb; base += kRowThreads) {
-    const int j = base + tid;
-    const uint32_t key = (j < nb && !keep_all) ? row_keys[j] : 0u;
-    const bool gt = j < nb && (keep_all || key > cut.vstar);
-    const bool eq = j < nb && !keep_all && key == cut.vstar;
-    // one scan of (above count, equal count): both fit 16 bits per chunk
-    uint32_t packed = (gt ? 1u : 0u) | (eq ? 0x10000u : 0u);
-    unsigned long long unused = 0ull;
-    row_scan(packed, unused, sh);
-    const uint32_t own = (gt ? 1u : 0u) | (eq ? 0x10000u : 0u);
-    const uint32_t ex = packed - own;                   // exclusive prefix
-    const uint32_t run = sh.run, eq_run = sh.eq_run;
-    const uint32_t eq_left = cut.take > eq_run ? cut.take - eq_run : 0u;   // equal keys still to keep
-    const uint32_t ex_gt = ex & 0xFFFFu, ex_eq = ex >> 16;
-    const bool f = gt || (eq && ex_eq < eq_left);
-    const uint32_t pos = run + ex_gt + (ex_eq < eq_left ? ex_eq : eq_left);
-    if (f) idx_out[pos] = j;
-    const uint32_t fb = __ballot_sync(0xffffffffu, f);
-    if (bits_out != nullptr && lane == 0 && base + wid * 32 < nb) bits_out[(base >> 5) + wid] = fb;
-    __syncthreads();                                    // every thread has read run / eq_run
-    if (tid == kRowThreads - 1) {
-      const uint32_t tot_gt = packed & 0xFFFFu, tot_eq = packed >> 16;
-      sh.run = run + tot_gt + (tot_eq < eq_left ? tot_eq : eq_left);
-      sh.eq_run = eq_run + tot_eq;
-    }
-    __syncthreads();
+  const uint32_t lt = (1u << lane) - 1u;
+  const int seg = ((nb + kRowThreads - 1) / kRowThreads) * 32;
+  const int s0 = wid * seg, s1 = min(nb, s0 + seg);
+  auto flags = [&](int j, bool& gt, bool& eq) {
+    const uint32_t key = (j < s1 && !keep_all) ? row_keys[j] : 0u;
+    gt = j < s1 && (keep_all || key > cut.vstar);
+    eq = j < s1 && !keep_all && key == cut.vstar;
+  };
+  uint32_t n_gt = 0u, n_eq = 0u;
+  for (int base = s0; base < s1; base += 32) {
+    bool gt, eq;
+    flags(base + lane, gt, eq);
+    n_gt += (uint32_t)__popc(__ballot_sync(0xffffffffu, gt));
+    n_eq += (uint32_t)__popc(__ballot_sync(0xffffffffu, eq));
   }
-  if (tid == 0) kv_cnt[row] = (int32_t)sh.run;
+  if (lane == 0) {
+    sh.wc[wid] = n_gt;
+    sh.eq_w[wid] = n_eq;
+  }
+  __syncthreads();
+  uint32_t gt_before = 0u, eq_before = 0u, gt_all = 0u, eq_all = 0u;
+#pragma unroll
+  for (int w = 0; w < kRowWarps; ++w) {
+    const uint32_t g = sh.wc[w], e = sh.eq_w[w];
+    if (w < wid) { gt_before += g; eq_before += e; }
+    gt_all += g;
+    eq_all += e;
+  }
+  uint32_t run = gt_before + min(eq_before, cut.take);     // kept entries before this segment
+  uint32_t eq_run = eq_before;                              // equal keys before the current word
+  for (int base = s0; base < s1; base += 32) {
+    bool gt, eq;
+    flags(base + lane, gt, eq);
+    const uint32_t eb = __ballot_sync(0xffffffffu, eq);
+    const bool f = gt || (eq && eq_run + (uint32_t)__popc(eb & lt) < cut.take);
+    eq_run += (uint32_t)__popc(eb);
+    const uint32_t fb = __ballot_sync(0xffffffffu, f);
+    if (f) idx_out[run + (uint32_t)__popc(fb & lt)] = base + lane;
+    if (bits_out != nullptr && lane == 0) bits_out[base >> 5] = fb;
+    run += (uint32_t)__popc(fb);
+  }
+  if (tid == 0) kv_cnt[row] = (int32_t)(gt_all + min(eq_all, cut.take));
 }
 
 // STRUCTURED: block coordinates from the raster id of each block's first token.
