@@ -79,8 +79,10 @@ class SparseVideoAttention:
         kept until `rebuild_order()`).  schedule: optional (n_steps, dense_steps,
         start, end, refresh_every) -- a timestep-adaptive rule for `step()`.
         attn_passes: key-range passes of the attention (svsa_attn_fwd_split); by
-        default 1 while a head's reordered K and V (Npad * d * 4 bytes) fit in
-        48 MB of L2, else enough passes for at most 64 MB each (at most 8)."""
+        default 1 for the structured rule (its windows keep the key blocks of
+        neighbouring query blocks close together, so they share L2 already)
+        and while a head's reordered K and V (Npad * d * 4 bytes) fit in 48 MB
+        of L2, else enough passes for at most 32 MB each (at most 8)."""
         self.B, self.heads, self.T, self.H, self.W, self.d = B, heads, T, H, W, d
         self.N = T * H * W
         self.nb = -(-self.N // BLOCK)
@@ -107,7 +109,8 @@ class SparseVideoAttention:
         self._mask = self.buf.mask()
         kv_bytes = self.Npad * d * 4
         if attn_passes is None:
-            attn_passes = 1 if kv_bytes <= 48 * 2**20 else min(8, -(-kv_bytes // (64 * 2**20)))
+            local = self.select == SEL_STRUCTURED
+            attn_passes = 1 if (local or kv_bytes <= 48 * 2**20) else min(8, -(-kv_bytes // (32 * 2**20)))
         self.attn_passes = int(attn_passes)
         self.buf.split_ws = (torch.empty(svsa_attn_split_workspace_bytes(self.shape, self.attn_passes),
                                          dtype=torch.uint8, device=self.buf.qp.device)
