@@ -213,7 +213,7 @@ class SparseVideoAttention:
                       b.nvalid, self._rows(b.cbar, r0, r1))
         return sh, m
 
-    def forward_host(self, q, k, v, out, *, anchor_offset: int = 0, reuse_mask: bool = False, groups: int = 8):
+    def forward_host(self, q, k, v, out, *, anchor_offset: int = 0, reuse_mask: bool = False, groups: int = 12):
         """q, k, v, out: pinned host bf16 [B, heads, N, d] (raster order).  The rows
         are processed in `groups` groups; each group's inputs are copied in on one
         stream, its four library calls run on the current stream once they have
