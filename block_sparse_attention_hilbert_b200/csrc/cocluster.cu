@@ -400,8 +400,17 @@ __global__ void __launch_bounds__(kThreads, 1) assign_tc_kernel(const __grid_con
       const long long bh = it / a.nxt;
       const int xt = (int)(it % a.nxt);
       const long long t = (long long)xt * kRows + row;
-      float best = -INFINITY, second = -INFINITY;
-      int bi = 0;
+      // running (best, second, index of best) over the even and the odd
+      // columns separately (two independent dependency chains), merged at the
+      // end; branch-free updates, strict > keeps the first index on ties
+      float best0 = -INFINITY, second0 = -INFINITY, best1 = -INFINITY, second1 = -INFINITY;
+      int bi0 = 0x7fffffff, bi1 = 0x7fffffff;
+      auto update = [](float x, int j, float& b, float& s, int& bi) {
+        const bool gt = x > b;
+        s = gt ? b : fmaxf(s, x);
+        bi = gt ? j : bi;
+        b = gt ? x : b;
+      };
       for (int ct = 0; ct < a.nct; ++ct) {
         const uint32_t sb = cn % kSBufs;
         if (!wait_bar(bar(BAR_S_FULL + sb), (cn / kSBufs) & 1u, abort_flag, 76)) { stop = true; break; }
@@ -417,22 +426,26 @@ __global__ void __launch_bounds__(kThreads, 1) assign_tc_kernel(const __grid_con
             if (lane == 0) mbar_arrive(bar(BAR_S_EMPTY + sb));
           }
           const int j0 = ct * kCent + ch * 32;
+          if (j0 + 32 > a.C) {               // the ragged last centroid tile
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            if (j0 + c < a.C) {
-              if (v[c] > best) {
-                second = best;
-                best = v[c];
-                bi = j0 + c;
-              } else if (v[c] > second) {
-                second = v[c];
-              }
-            }
+            for (int c = 0; c < 32; ++c)
+              if (j0 + c >= a.C) v[c] = -INFINITY;
+          }
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            update(v[c], j0 + c, best0, second0, bi0);
+            update(v[c + 1], j0 + c + 1, best1, second1, bi1);
           }
         }
         ++cn;
       }
       if (stop) break;
+      // merge: the larger best (the lower index on equal values); the second
+      // is the larger of the two seconds and the smaller best
+      const bool one = best1 > best0 || (best1 == best0 && bi1 < bi0);
+      const float best = one ? best1 : best0;
+      const int bi = min(one ? bi1 : bi0, a.C - 1);        // (no comparable score at all: NaN input)
+      const float second = fmaxf(fmaxf(second0, second1), one ? best0 : best1);
       if (t < a.N) {
         const long long tok = bh * a.N + t;
         a.assign[tok] = bi;
