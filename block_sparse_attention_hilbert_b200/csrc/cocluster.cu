@@ -20,7 +20,10 @@
 //     at most 3d * 2^-20 * sum|x_c c_c| <= 3d * 2^-20 * |x| |c| (a bound with
 //     a 16x margin over round-to-nearest, for the accumulator's alignment);
 //   * a token whose best and second-best affinities lie within twice that
-//     bound of each other is recomputed in fp64 against every centroid.
+//     bound of each other is decided again in fp64: fp32 scores of every
+//     centroid narrow it to those within twice the bound of the best, and
+//     their fp64 dot products decide (every centroid's, when a lane's list of
+//     its four best cannot hold them all).
 // Centroids are the float32 rounding of fp64 sums of bf16 values.
 #include "tcgen05.cuh"
 
@@ -104,14 +107,43 @@ __global__ void means_kernel(const __nv_bfloat16* __restrict__ x, const int32_t*
   if (lane == 0) atomicMax(&cmax[bh], __float_as_uint(sqrtf(ss) * (1.f + 9.5367431640625e-7f)));
 }
 
-// Exact argmax for the tokens the tensor-core pass could not separate: fp64
-// dot products against every centroid of the head, first index on ties.  A
-// warp takes one token; lanes split the head dimension (coalesced centroid
-// rows), 32 centroids are accumulated at a time and a transpose-reduction
-// leaves lane L with centroid L's dot product.
+// The five largest values a lane has seen (t[0] >= ... >= t[4]) and the
+// indices of the first four (-1 while empty).  Strict comparisons keep the
+// earlier of equal values in front; insertion is branch-free and taken only
+// by a value above t[4].
+struct Top5 {
+  float t[5] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  int id[4] = {-1, -1, -1, -1};
+  __device__ __forceinline__ void push(float x, int j) {
+    if (!(x > t[4])) return;
+    const bool c0 = x > t[0], c1 = x > t[1], c2 = x > t[2], c3 = x > t[3];
+    t[4] = c3 ? t[3] : x;
+    t[3] = c3 ? (c2 ? t[2] : x) : t[3];
+    id[3] = c3 ? (c2 ? id[2] : j) : id[3];
+    t[2] = c2 ? (c1 ? t[1] : x) : t[2];
+    id[2] = c2 ? (c1 ? id[1] : j) : id[2];
+    t[1] = c1 ? (c0 ? t[0] : x) : t[1];
+    id[1] = c1 ? (c0 ? id[0] : j) : id[1];
+    t[0] = c0 ? x : t[0];
+    id[0] = c0 ? j : id[0];
+  }
+};
+
+// Exact argmax for the tokens the tensor-core pass could not separate, first
+// index on ties.  A warp takes one token; lanes split the head dimension
+// (coalesced centroid rows); 32 centroids are accumulated at a time and a
+// transpose-reduction leaves lane L with centroid L's dot product.
+//   1. fp32 scores s_j of every centroid (error far below the tensor-core
+//      bound gamma |x| |c_j|), each lane keeping the five largest of its own;
+//   2. with s1 the largest and thr = 2 gamma |x| max|c|, the exact maximum is
+//      among the centroids with s_j >= s1 - thr.  When no lane's fifth value
+//      reaches that line, those are all in the lanes' first four: fp64 dot
+//      products of just them decide.  Otherwise every centroid is scored in
+//      fp64.
 template <int D>
 __global__ void fix_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ cent,
                            const int32_t* __restrict__ list, const unsigned int* __restrict__ count,
+                           const float* __restrict__ xnorm, const unsigned int* __restrict__ cmax, float gamma,
                            int32_t* __restrict__ assign, long long N, int C) {
   constexpr int U = D / 32;
   const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -120,11 +152,67 @@ __global__ void fix_kernel(const __nv_bfloat16* __restrict__ x, const float* __r
        i += (long long)gridDim.x * kWarpsPerBlock) {
     const long long tok = list[i];                   // bh * N + t
     const long long bh = tok / N;
+    float xf[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) xf[u] = __bfloat162float(x[tok * D + lane + 32 * u]);
+    // 1. fp32 scores, five best per lane
+    Top5 top;
+    for (int j0 = 0; j0 < C; j0 += 32) {
+      float acc[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        acc[c] = 0.f;
+        if (j0 + c < C) {
+          const float* row = cent + (bh * C + j0 + c) * D;
+#pragma unroll
+          for (int u = 0; u < U; ++u) acc[c] = fmaf(xf[u], row[lane + 32 * u], acc[c]);
+        }
+      }
+#pragma unroll
+      for (int w = 16; w >= 1; w >>= 1) {
+        const bool hi = (lane & w) != 0;
+#pragma unroll
+        for (int c = 0; c < w; ++c) {
+          const float keep = hi ? acc[c + w] : acc[c];
+          const float send = hi ? acc[c] : acc[c + w];
+          acc[c] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+        }
+      }
+      if (j0 + lane < C) top.push(acc[0], j0 + lane);
+    }
+    float s1 = top.t[0];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s1 = fmaxf(s1, __shfl_xor_sync(0xffffffffu, s1, o));
+    const double line = (double)s1 - 2.0 * (double)gamma * (double)xnorm[tok] * (double)__uint_as_float(cmax[bh]);
+    const bool complete = !__any_sync(0xffffffffu, (double)top.t[4] >= line);
     double xv[U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) xv[u] = (double)__bfloat162float(x[tok * D + lane + 32 * u]);
+    for (int u = 0; u < U; ++u) xv[u] = (double)xf[u];
     double best = -INFINITY;
     int bi = 0x7fffffff;
+    if (complete) {
+      // 2a. fp64 dot products of the candidates only
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        uint32_t m = __ballot_sync(0xffffffffu, top.id[k] >= 0 && (double)top.t[k] >= line);
+        while (m) {
+          const int src = __ffs(m) - 1;
+          m &= m - 1u;
+          const int j = __shfl_sync(0xffffffffu, top.id[k], src);
+          const float* row = cent + (bh * C + j) * D;
+          double acc = 0.0;
+#pragma unroll
+          for (int u = 0; u < U; ++u) acc = fma(xv[u], (double)row[lane + 32 * u], acc);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+          acc = __shfl_sync(0xffffffffu, acc, 0);    // one value for every lane
+          if (acc > best || (acc == best && j < bi)) { best = acc; bi = j; }
+        }
+      }
+      if (lane == 0) assign[tok] = bi;
+      continue;
+    }
+    // 2b. fp64 dot products of every centroid
     for (int j0 = 0; j0 < C; j0 += 32) {
       double acc[32];
 #pragma unroll
@@ -565,7 +653,7 @@ cudaError_t launch_cocluster(const void* q, const void* k, long long BH, long lo
       assign_tc_kernel<128><<<grid, kThreads, Smem<128>::kBytes, st>>>(mx, mc, a);
       SVSA_CLU_CHECK();
       fix_kernel<128><<<(unsigned)(tc::sm_count() * 4), 32 * kWarpsPerBlock, 0, st>>>(
-          x, cent, I(w.list), U(w.count), I(w.assign), N, C);
+          x, cent, I(w.list), U(w.count), xnorm, cmax, a.gamma, I(w.assign), N, C);
       SVSA_CLU_CHECK();
     } else {
       e = cudaFuncSetAttribute(assign_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Smem<64>::kBytes);
@@ -573,7 +661,7 @@ cudaError_t launch_cocluster(const void* q, const void* k, long long BH, long lo
       assign_tc_kernel<64><<<grid, kThreads, Smem<64>::kBytes, st>>>(mx, mc, a);
       SVSA_CLU_CHECK();
       fix_kernel<64><<<(unsigned)(tc::sm_count() * 4), 32 * kWarpsPerBlock, 0, st>>>(
-          x, cent, I(w.list), U(w.count), I(w.assign), N, C);
+          x, cent, I(w.list), U(w.count), xnorm, cmax, a.gamma, I(w.assign), N, C);
       SVSA_CLU_CHECK();
     }
     // as many segment warps as 200 KB of counters allow, at most 32

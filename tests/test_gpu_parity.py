@@ -390,6 +390,18 @@ def test_cocluster_exact_ties_take_the_lower_cluster():
     _cocluster_case(w, q, k, rounds=2)
 
 
+def test_cocluster_all_centroids_tied_recompute_every_centroid():
+    """Identical tokens make all 8 centroids equal: every affinity ties across
+    more than four centroids, so the fix-up scores every centroid in fp64 and
+    keeps cluster 0, as the oracle does."""
+    w = _small("topk", 64, grid=(4, 8, 16), heads=1, d=128, keep_frac=0.3)
+    g = torch.Generator().manual_seed(11)
+    row = (torch.randn(128, generator=g) * 2).to(torch.bfloat16)
+    q = row.expand(w.N, 128).contiguous()[None, None].cuda()
+    k = (row * 0.5).to(torch.bfloat16).expand(w.N, 128).contiguous()[None, None].cuda()
+    _cocluster_case(w, q, k, rounds=2)
+
+
 @pytest.mark.parametrize("select", ["topk", "threshold"])
 def test_cocluster_layer_matches_oracle(select):
     """The whole layer on the co-clustering order: masks bit-exact outside the
