@@ -130,16 +130,23 @@ struct Top5 {
 };
 
 // Exact argmax for the tokens the tensor-core pass could not separate, first
-// index on ties.  A warp takes one token; lanes split the head dimension
-// (coalesced centroid rows); 32 centroids are accumulated at a time and a
-// transpose-reduction leaves lane L with centroid L's dot product.
-//   1. fp32 scores s_j of every centroid (error far below the tensor-core
-//      bound gamma |x| |c_j|), each lane keeping the five largest of its own;
-//   2. with s1 the largest and thr = 2 gamma |x| max|c|, the exact maximum is
-//      among the centroids with s_j >= s1 - thr.  When no lane's fifth value
-//      reaches that line, those are all in the lanes' first four: fp64 dot
-//      products of just them decide.  Otherwise every centroid is scored in
-//      fp64.
+// index on ties.  Per head, list[bh * N + i] (i < count[bh]) holds those
+// tokens.  A warp takes kFixTok tokens of one head, so that every centroid row
+// it loads serves kFixTok dot products; lanes split the head dimension
+// (U = D / 32 consecutive values each).
+//   1. fp32 scores s_j of every centroid, kFixCent centroids at a time: the
+//      kFixCent x kFixTok partial sums of a lane go through a transpose-
+//      reduction that leaves lane L with the full score of centroid
+//      j0 + L / kFixTok for token L % kFixTok.  Each lane keeps the five best
+//      it has seen (its token, every kFixCent-th centroid).  The fp32 error is
+//      far below the tensor-core bound gamma |x| |c_j|.
+//   2. With s1 a token's largest score and thr = 2 gamma |x| max|c|, its exact
+//      maximum is among the centroids with s_j >= s1 - thr.  When no lane of
+//      the token has a fifth value reaching that line, they are all in its
+//      lanes' first four: fp64 dot products of just them decide.  Otherwise
+//      every centroid is scored in fp64 for that token.
+constexpr int kFixTok = 8, kFixCent = 32 / kFixTok;
+
 template <int D>
 __global__ void fix_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ cent,
                            const int32_t* __restrict__ list, const unsigned int* __restrict__ count,
@@ -147,27 +154,44 @@ __global__ void fix_kernel(const __nv_bfloat16* __restrict__ x, const float* __r
                            int32_t* __restrict__ assign, long long N, int C) {
   constexpr int U = D / 32;
   const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const unsigned int n = *count;
-  for (long long i = (long long)blockIdx.x * kWarpsPerBlock + wid; i < n;
-       i += (long long)gridDim.x * kWarpsPerBlock) {
-    const long long tok = list[i];                   // bh * N + t
-    const long long bh = tok / N;
-    float xf[U];
+  const long long bh = blockIdx.y;
+  const int n = (int)count[bh];
+  const int32_t* lst = list + bh * N;
+  const float* ch = cent + bh * (long long)C * D;
+  const int my = lane % kFixTok;                     // the token this lane scores
+  for (int g = (blockIdx.x * kWarpsPerBlock + wid) * kFixTok; g < n; g += gridDim.x * kWarpsPerBlock * kFixTok) {
+    // the group's tokens (a short last group repeats its last token)
+    long long tk[kFixTok];
+    float xf[kFixTok][U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) xf[u] = __bfloat162float(x[tok * D + lane + 32 * u]);
+    for (int t = 0; t < kFixTok; ++t) {
+      tk[t] = bh * N + lst[min(g + t, n - 1)];
+#pragma unroll
+      for (int u = 0; u < U; ++u) xf[t][u] = __bfloat162float(x[tk[t] * D + lane * U + u]);
+    }
     // 1. fp32 scores, five best per lane
     Top5 top;
-    for (int j0 = 0; j0 < C; j0 += 32) {
-      float acc[32];
+    for (int j0 = 0; j0 < C; j0 += kFixCent) {
+      float acc[kFixCent * kFixTok];                 // [centroid c][token t] at c * kFixTok + t
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        acc[c] = 0.f;
+      for (int c = 0; c < kFixCent; ++c) {
+        float cv[U];
         if (j0 + c < C) {
-          const float* row = cent + (bh * C + j0 + c) * D;
 #pragma unroll
-          for (int u = 0; u < U; ++u) acc[c] = fmaf(xf[u], row[lane + 32 * u], acc[c]);
+          for (int u = 0; u < U; ++u) cv[u] = ch[(long long)(j0 + c) * D + lane * U + u];
+        } else {
+#pragma unroll
+          for (int u = 0; u < U; ++u) cv[u] = 0.f;
+        }
+#pragma unroll
+        for (int t = 0; t < kFixTok; ++t) {
+          float v = 0.f;
+#pragma unroll
+          for (int u = 0; u < U; ++u) v = fmaf(xf[t][u], cv[u], v);
+          acc[c * kFixTok + t] = v;
         }
       }
+      // halving exchanges: lane L ends with the full sum of value L
 #pragma unroll
       for (int w = 16; w >= 1; w >>= 1) {
         const bool hi = (lane & w) != 0;
@@ -178,73 +202,61 @@ __global__ void fix_kernel(const __nv_bfloat16* __restrict__ x, const float* __r
           acc[c] = keep + __shfl_xor_sync(0xffffffffu, send, w);
         }
       }
-      if (j0 + lane < C) top.push(acc[0], j0 + lane);
+      const int j = j0 + lane / kFixTok;
+      if (j < C) top.push(acc[0], j);
     }
+    // per token (lanes my, my + kFixTok, ...): the largest score and the line
     float s1 = top.t[0];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s1 = fmaxf(s1, __shfl_xor_sync(0xffffffffu, s1, o));
+    for (int o = kFixTok; o < 32; o <<= 1) s1 = fmaxf(s1, __shfl_xor_sync(0xffffffffu, s1, o));
+    long long tok = tk[0];                           // this lane's token (static indices only)
+#pragma unroll
+    for (int t = 1; t < kFixTok; ++t) tok = my == t ? tk[t] : tok;
     const double line = (double)s1 - 2.0 * (double)gamma * (double)xnorm[tok] * (double)__uint_as_float(cmax[bh]);
-    const bool complete = !__any_sync(0xffffffffu, (double)top.t[4] >= line);
-    double xv[U];
+    bool reach = (double)top.t[4] >= line;
 #pragma unroll
-    for (int u = 0; u < U; ++u) xv[u] = (double)xf[u];
-    double best = -INFINITY;
-    int bi = 0x7fffffff;
-    if (complete) {
-      // 2a. fp64 dot products of the candidates only
+    for (int o = kFixTok; o < 32; o <<= 1) reach |= __shfl_xor_sync(0xffffffffu, reach ? 1 : 0, o) != 0;
+    // 2. token by token: fp64 dot products of the candidates (or of all centroids)
+#pragma unroll 1
+    for (int t = 0; t < kFixTok && g + t < n; ++t) {
+      const long long tt = bh * N + lst[g + t];     // (reloaded: no dynamic index into registers)
+      double xv[U];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        uint32_t m = __ballot_sync(0xffffffffu, top.id[k] >= 0 && (double)top.t[k] >= line);
-        while (m) {
-          const int src = __ffs(m) - 1;
-          m &= m - 1u;
-          const int j = __shfl_sync(0xffffffffu, top.id[k], src);
-          const float* row = cent + (bh * C + j) * D;
-          double acc = 0.0;
+      for (int u = 0; u < U; ++u) xv[u] = (double)__bfloat162float(x[tt * D + lane * U + u]);
+      const bool full = __shfl_sync(0xffffffffu, reach ? 1 : 0, t) != 0;
+      double best = -INFINITY;
+      int bi = 0x7fffffff;
+      auto score = [&](int j) -> double {             // warp-wide fp64 dot product, one value in every lane
+        const float* row = ch + (long long)j * D;
+        double a = 0.0;
 #pragma unroll
-          for (int u = 0; u < U; ++u) acc = fma(xv[u], (double)row[lane + 32 * u], acc);
+        for (int u = 0; u < U; ++u) a = fma(xv[u], (double)row[lane * U + u], a);
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-          acc = __shfl_sync(0xffffffffu, acc, 0);    // one value for every lane
-          if (acc > best || (acc == best && j < bi)) { best = acc; bi = j; }
+        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        return __shfl_sync(0xffffffffu, a, 0);
+      };
+      if (!full) {
+        const double ln = __shfl_sync(0xffffffffu, line, t);
+        const uint32_t mine = my == t ? 0xffffffffu : 0u;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint32_t m = __ballot_sync(0xffffffffu, top.id[k] >= 0 && (double)top.t[k] >= ln) & __ballot_sync(0xffffffffu, mine != 0u);
+          while (m) {
+            const int src = __ffs(m) - 1;
+            m &= m - 1u;
+            const int j = __shfl_sync(0xffffffffu, top.id[k], src);
+            const double v = score(j);
+            if (v > best || (v == best && j < bi)) { best = v; bi = j; }
+          }
+        }
+      } else {
+        for (int j = 0; j < C; ++j) {
+          const double v = score(j);
+          if (v > best) { best = v; bi = j; }      // increasing j: the first index on ties
         }
       }
-      if (lane == 0) assign[tok] = bi;
-      continue;
+      if (lane == 0) assign[tt] = bi;
     }
-    // 2b. fp64 dot products of every centroid
-    for (int j0 = 0; j0 < C; j0 += 32) {
-      double acc[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        acc[c] = 0.0;
-        if (j0 + c < C) {
-          const float* row = cent + (bh * C + j0 + c) * D;
-#pragma unroll
-          for (int u = 0; u < U; ++u) acc[c] = fma(xv[u], (double)row[lane + 32 * u], acc[c]);
-        }
-      }
-      // halving exchanges: lane L ends with the full sum of centroid j0 + L
-#pragma unroll
-      for (int w = 16; w >= 1; w >>= 1) {
-        const bool hi = (lane & w) != 0;
-#pragma unroll
-        for (int c = 0; c < w; ++c) {
-          const double keep = hi ? acc[c + w] : acc[c];
-          const double send = hi ? acc[c] : acc[c + w];
-          acc[c] = keep + __shfl_xor_sync(0xffffffffu, send, w);
-        }
-      }
-      const int j = j0 + lane;
-      if (j < C && acc[0] > best) { best = acc[0]; bi = j; }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const double ob = __shfl_xor_sync(0xffffffffu, best, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
-    }
-    if (lane == 0) assign[tok] = bi;
   }
 }
 
@@ -360,8 +372,8 @@ struct Args {
   const float* xnorm;           // [BH * N] token norms (upper bounds)
   const unsigned int* cmax;     // [BH] largest centroid norm (float bits, upper bound)
   int32_t* assign;              // [BH * N]
-  int32_t* fix_list;            // tokens to recompute exactly
-  unsigned int* fix_count;
+  int32_t* fix_list;            // [BH, N] per head: tokens to decide exactly
+  unsigned int* fix_count;      // [BH] their counts
   long long N;
   int C, nxt, nct;              // clusters, token tiles and centroid tiles per head
   long long items;
@@ -538,7 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1) assign_tc_kernel(const __grid_con
         const long long tok = bh * a.N + t;
         a.assign[tok] = bi;
         const float thr = 2.f * a.gamma * a.xnorm[tok] * __uint_as_float(a.cmax[bh]);
-        if (best - second <= thr) a.fix_list[atomicAdd(a.fix_count, 1u)] = (int32_t)tok;
+        if (best - second <= thr) a.fix_list[bh * a.N + atomicAdd(a.fix_count + bh, 1u)] = (int32_t)t;
       }
     }
   }
@@ -578,7 +590,7 @@ CluWs clu_layout(long long BH, long long N, int C, int d) {
   w.starts = take(BH * C * 4);
   w.counts = take(BH * C * 4);
   w.list = take(BH * N * 4);
-  w.count = take(4);
+  w.count = take(BH * 4);
   w.total = off;
   return w;
 }
@@ -608,6 +620,8 @@ cudaError_t launch_cocluster(const void* q, const void* k, long long BH, long lo
 #define SVSA_CLU_CHECK() do { e = cudaGetLastError(); if (e != cudaSuccess) return e; ++n_launch; } while (0)
 
   const unsigned row_blocks = (unsigned)((BH * N + kWarpsPerBlock - 1) / kWarpsPerBlock);
+  // fix-up: about four CTAs per SM over all heads, at least one per head
+  const dim3 fix_grid((unsigned)std::max<long long>(1, (tc::sm_count() * 4 + BH - 1) / BH), (unsigned)BH);
   const unsigned cent_blocks = (unsigned)((BH * C + kWarpsPerBlock - 1) / kWarpsPerBlock);
   auto norms = [&](const __nv_bfloat16* x, float* out) -> cudaError_t {
     if (d == 128) tc::clu::norms_kernel<128><<<row_blocks, 32 * kWarpsPerBlock, 0, st>>>(x, out, BH * N);
@@ -639,7 +653,7 @@ cudaError_t launch_cocluster(const void* q, const void* k, long long BH, long lo
     if (!tc::make_map_2d(&mx, x, BH * N, d, kRows, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) ||
         !tc::make_map_2d(&mc, c3, BH * C, 3 * d, kCent, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16))
       return cudaErrorInvalidValue;
-    e = cudaMemsetAsync(U(w.count), 0, 4, st);
+    e = cudaMemsetAsync(U(w.count), 0, BH * 4, st);
     if (e != cudaSuccess) return e;
     Args a;
     a.xnorm = xnorm; a.cmax = cmax; a.assign = I(w.assign); a.fix_list = I(w.list); a.fix_count = U(w.count);
@@ -652,7 +666,7 @@ cudaError_t launch_cocluster(const void* q, const void* k, long long BH, long lo
       if (e != cudaSuccess) return e;
       assign_tc_kernel<128><<<grid, kThreads, Smem<128>::kBytes, st>>>(mx, mc, a);
       SVSA_CLU_CHECK();
-      fix_kernel<128><<<(unsigned)(tc::sm_count() * 4), 32 * kWarpsPerBlock, 0, st>>>(
+      fix_kernel<128><<<fix_grid, 32 * kWarpsPerBlock, 0, st>>>(
           x, cent, I(w.list), U(w.count), xnorm, cmax, a.gamma, I(w.assign), N, C);
       SVSA_CLU_CHECK();
     } else {
@@ -660,7 +674,7 @@ cudaError_t launch_cocluster(const void* q, const void* k, long long BH, long lo
       if (e != cudaSuccess) return e;
       assign_tc_kernel<64><<<grid, kThreads, Smem<64>::kBytes, st>>>(mx, mc, a);
       SVSA_CLU_CHECK();
-      fix_kernel<64><<<(unsigned)(tc::sm_count() * 4), 32 * kWarpsPerBlock, 0, st>>>(
+      fix_kernel<64><<<fix_grid, 32 * kWarpsPerBlock, 0, st>>>(
           x, cent, I(w.list), U(w.count), xnorm, cmax, a.gamma, I(w.assign), N, C);
       SVSA_CLU_CHECK();
     }
