@@ -79,9 +79,26 @@ __global__ void means_kernel(const __nv_bfloat16* __restrict__ x, const int32_t*
   double acc[U];
 #pragma unroll
   for (int u = 0; u < U; ++u) acc[u] = 0.0;
-  for (int i = 0; i < n; ++i) {
-    const long long t = order == nullptr ? (long long)(s0 + i) : (long long)order[bh * N + s0 + i];
-    const __nv_bfloat16* row = x + (bh * N + t) * D;
+  // members in order; four rows are loaded ahead of their (ordered) adds
+  auto member = [&](int i) -> long long {
+    return order == nullptr ? (long long)(s0 + i) : (long long)order[bh * N + s0 + i];
+  };
+  int i = 0;
+  for (; i + 4 <= n; i += 4) {
+    float r[4][U];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const __nv_bfloat16* row = x + (bh * N + member(i + m)) * D;
+#pragma unroll
+      for (int u = 0; u < U; ++u) r[m][u] = __bfloat162float(row[lane + 32 * u]);
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+#pragma unroll
+      for (int u = 0; u < U; ++u) acc[u] += (double)r[m][u];
+  }
+  for (; i < n; ++i) {
+    const __nv_bfloat16* row = x + (bh * N + member(i)) * D;
 #pragma unroll
     for (int u = 0; u < U; ++u) acc[u] += (double)__bfloat162float(row[lane + 32 * u]);
   }
