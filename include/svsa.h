@@ -196,8 +196,8 @@ size_t svsa_mask_workspace_bytes(svsa_shape s, const svsa_mask_params* p);
  * Outputs: m->kv_idx, m->kv_cnt, and m->bits / kbar / vbar / nvalid when those
  * are non-NULL (kbar, vbar, nvalid required for routing).  perm may be NULL
  * unless select = STRUCTURED.  vp may be NULL unless routing = 1.
- * THRESHOLD / TOPK / routing stage one mask row in shared memory: nb up to
- * 57,000 blocks (3.6 M tokens per head); longer rows return SVSA_ERR_CUDA. */
+ * THRESHOLD / TOPK / routing stage each mask row's keys in shared memory
+ * (within the nb <= 16384 limit above). */
 svsa_status svsa_build_mask(const void* qp, const void* kp, const void* vp, const int32_t* perm,
                             svsa_shape s, const svsa_mask_params* p, const svsa_mask* m,
                             void* ws, size_t ws_bytes, void* stream);
