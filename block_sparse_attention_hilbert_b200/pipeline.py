@@ -69,6 +69,18 @@ class LayerBuffers:
                          self.cbar)
 
 
+def default_attn_passes(select: int, Npad: int, d: int) -> int:
+    """Key-range passes of the attention for a head of Npad reordered tokens:
+    one for the structured rule (its windows keep the key blocks of
+    neighbouring query blocks together, so they share L2 already) and while
+    the head's K and V (Npad * d * 4 bytes) fit in 48 MB of L2, else enough
+    passes for at most 32 MB each, at most 8."""
+    kv_bytes = Npad * d * 4
+    if select == SEL_STRUCTURED or kv_bytes <= 48 * 2**20:
+        return 1
+    return min(8, -(-kv_bytes // (32 * 2**20)))
+
+
 class SparseVideoAttention:
     def __init__(self, B, heads, T, H, W, d, *, order="hilbert", select="threshold", tau=0.9,
                  keep_frac=0.25, sub_block=64, win_t=2, win_rows=1, n_anchors=0, routing=False,
@@ -107,10 +119,8 @@ class SparseVideoAttention:
                                 perm_ws_bytes=svsa_perm_workspace_bytes(self.shape, self.order),
                                 device=device, compensate=self.compensate)
         self._mask = self.buf.mask()
-        kv_bytes = self.Npad * d * 4
         if attn_passes is None:
-            local = self.select == SEL_STRUCTURED
-            attn_passes = 1 if (local or kv_bytes <= 48 * 2**20) else min(8, -(-kv_bytes // (32 * 2**20)))
+            attn_passes = default_attn_passes(self.select, self.Npad, d)
         self.attn_passes = int(attn_passes)
         self.buf.split_ws = (torch.empty(svsa_attn_split_workspace_bytes(self.shape, self.attn_passes),
                                          dtype=torch.uint8, device=self.buf.qp.device)

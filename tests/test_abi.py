@@ -171,3 +171,17 @@ def test_schedule_step_rejects():
     assert lib.svsa_schedule_step(ctypes.byref(bad), 0, ctypes.byref(base), ctypes.byref(out), ctypes.byref(r)) == 1
     bad = svsa.schedule(10, 2, 0.9, 0.5, 0)
     assert lib.svsa_schedule_step(ctypes.byref(bad), 0, ctypes.byref(base), ctypes.byref(out), ctypes.byref(r)) == 1
+
+
+def test_default_attention_passes():
+    """Key-range passes by rule and head size: one while K and V of a head
+    fit in 48 MB (and always for the structured rule), else 32 MB each."""
+    from block_sparse_attention_hilbert_b200.pipeline import default_attn_passes
+    mb = 2**20
+    rows = lambda nbytes, d=128: nbytes // (d * 4)          # Npad giving that many K+V bytes
+    assert default_attn_passes(svsa.SEL_TOPK, 512 * 64, 128) == 1          # the wan13b layer, 16.8 MB
+    assert default_attn_passes(svsa.SEL_THRESHOLD, rows(48 * mb), 128) == 1
+    assert default_attn_passes(svsa.SEL_THRESHOLD, rows(48 * mb) + 64, 128) == 2
+    assert default_attn_passes(svsa.SEL_THRESHOLD, 3488 * 64, 128) == 4     # HunyuanVideo, 114 MB
+    assert default_attn_passes(svsa.SEL_STRUCTURED, 3072 * 64, 128) == 1    # the 6x Wan layer, 101 MB
+    assert default_attn_passes(svsa.SEL_TOPK, rows(1024 * mb), 128) == 8    # capped
