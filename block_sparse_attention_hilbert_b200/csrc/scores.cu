@@ -19,8 +19,12 @@
 // logits, normalises, and writes S (SIZE = 16: the 4 x 4 sub-pairs of each
 // block pair are added first, columns in-thread and rows by warp shuffles).
 // Warp 0 issues the TMA copies (Q tile once per item, K tiles into a 2-stage
-// ring), warp 1 issues the MMAs into a 2-deep TMEM ring and owns the TMEM
-// allocation, warps 2-5 hold one query row per thread.  Every wait is bounded.
+// ring); the MMAs go into a 2-deep TMEM ring (warp 1 owns the allocation).
+// SIZE = 16: warps 1 and 10 issue the MMAs of the even and the odd tiles,
+// warps 2-5 and 6-9 hold one query row per thread for the first and the
+// second 64 keys of every tile and merge their pass-1 maxima and sums once
+// per item.  SIZE = 64: warp 1 issues every tile, warps 2-5 take whole tiles.
+// Every wait is bounded.
 //
 // SIZE = 64 can also write the raw logits L_IJ = qbar_I . kbar_J / sqrt(d) *
 // log2(e) (the centroid logits of the error-aware routing); with S = NULL
@@ -31,7 +35,16 @@ namespace svsa {
 namespace tc {
 namespace scores {
 
-constexpr int kThreads = 192;
+// Thread layout by sub-block size.  SIZE = 16 (many tiles per item): warps
+// 0 TMA, 1 and 10 MMA, 2-5 and 6-9 the two key halves of every tile.
+// SIZE = 64 (few items, short rows): warps 0 TMA, 1 MMA, 2-5 whole tiles.
+template <int SIZE> struct Layout {
+  static constexpr int kHalves = SIZE == 16 ? 2 : 1;
+  static constexpr int kIssuers = kHalves;
+  static constexpr int kRowThreads = 128 * kHalves;
+  static constexpr int kThreads = 64 + kRowThreads + 32 * (kIssuers - 1);
+};
+constexpr uint32_t kMergeBar = 1;           // named barrier of the row warps
 constexpr int kRows = 128;                  // pooled query rows per item
 constexpr int kKeys = 128;                  // pooled keys per tile
 constexpr int kKStages = 2, kSBufs = 2;
@@ -45,21 +58,23 @@ struct Smem {
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffK = kTile;
   static constexpr uint32_t kOffMisc = kOffK + kKStages * kTile;
-  static constexpr uint32_t kBytes = kOffMisc + 256 + 1024;    // + alignment slack
+  static constexpr uint32_t kBytes = kOffMisc + 2560 + 1024;   // Misc + alignment slack
   static_assert(kBytes <= 232448, "shared memory per CTA");
 };
 
 enum : uint32_t {
   BAR_Q_FULL = 0, BAR_Q_EMPTY, BAR_K_FULL, BAR_K_EMPTY = BAR_K_FULL + kKStages,
   BAR_S_FULL = BAR_K_EMPTY + kKStages, BAR_S_EMPTY = BAR_S_FULL + kSBufs, BAR_FINAL = BAR_S_EMPTY + kSBufs,
-  NUM_BARS
+  BAR_FINAL2, NUM_BARS
 };
 
 struct Misc {
   uint64_t bar[NUM_BARS];
   uint32_t tmem_base;
   uint32_t abort;
+  float pm[2][kRows], pl[2][kRows];          // pass-1 (max, sum) of each half, merged per item
 };
+static_assert(sizeof(Misc) <= 2560, "Misc fits its reservation");
 
 struct Args {
   float* S;            // nullable: normalised scores
@@ -75,12 +90,13 @@ struct Args {
 };
 
 template <int D, int SIZE>
-__global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+__global__ void __launch_bounds__(Layout<SIZE>::kThreads, 1) scores_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                                 const __grid_constant__ CUtensorMap tmK,
                                                                 const Args a) {
   constexpr int NCH = D / 64;
   constexpr int KSTEPS = D / 16;
   using L = Smem<D>;
+  using Y = Layout<SIZE>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   Misc* ms = reinterpret_cast<Misc*>(smem + L::kOffMisc);
@@ -91,16 +107,17 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
 
   if (tid == 0) {
     mbar_init(bar(BAR_Q_FULL), 1);
-    mbar_init(bar(BAR_Q_EMPTY), 1);
+    mbar_init(bar(BAR_Q_EMPTY), Y::kIssuers);      // every MMA issuer
     for (int i = 0; i < kKStages; ++i) {
       mbar_init(bar(BAR_K_FULL + i), 1);
       mbar_init(bar(BAR_K_EMPTY + i), 1);
     }
     for (int i = 0; i < kSBufs; ++i) {
       mbar_init(bar(BAR_S_FULL + i), 1);
-      mbar_init(bar(BAR_S_EMPTY + i), 4);
+      mbar_init(bar(BAR_S_EMPTY + i), 4 * Y::kHalves);   // every row warp
     }
     mbar_init(bar(BAR_FINAL), 1);
+    mbar_init(bar(BAR_FINAL2), 1);
     ms->abort = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
@@ -149,21 +166,28 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
         wait_bar(bar(BAR_K_FULL + n % kKStages), (n / kKStages) & 1u, &no_abort, 41);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || (Y::kIssuers == 2 && warp == 10)) {
+    // ------------------------------------------------------------ MMA issuers
+    // tile n (counted over this CTA's items) uses K stage and S buffer n % 2.
+    // With two issuers warp 1 issues the even tiles and warp 10 the odd ones;
+    // both wait for every item's Q tile and release it after their tiles.
+    static_assert(kKStages == 2 && kSBufs == 2, "one K stage and one S buffer per issuer");
     if (lane == 0) {
+      const uint32_t parity = warp == 1 ? 0u : 1u;
+      const uint32_t stride_mask = Y::kIssuers == 2 ? 1u : 0u;   // tiles this issuer skips
       constexpr uint32_t ID = idesc_f16(false, false, false, kKeys, kRows);   // fp16, K-major A and B
       const uint64_t dQ = sdesc(sbase + L::kOffQ, 16, 1024);
       const uint64_t dK = sdesc(sbase + L::kOffK, 16, 1024);
-      uint32_t qit = 0, kn = 0, sn = 0;
+      uint32_t qit = 0, n = 0;
       bool ok = true;
       for (long long it = blockIdx.x; it < a.items && ok; it += gridDim.x) {
         ok = wait_bar(bar(BAR_Q_FULL), qit & 1u, abort_flag, 33);
         ++qit;
-        for (int t = 0; t < ntiles && ok; ++t) {
-          const uint32_t ks = kn % kKStages, sb = sn % kSBufs;
-          ok = wait_bar(bar(BAR_K_FULL + ks), (kn / kKStages) & 1u, abort_flag, 34) &&
-               wait_bar(bar(BAR_S_EMPTY + sb), ((sn / kSBufs) & 1u) ^ 1u, abort_flag, 35);
+        for (int t = 0; t < ntiles && ok; ++t, ++n) {
+          if ((n & stride_mask) != parity) continue;
+          const uint32_t ks = n & 1u, sb = n & 1u, ph = (n >> 1) & 1u;
+          ok = wait_bar(bar(BAR_K_FULL + ks), ph, abort_flag, 34) &&
+               wait_bar(bar(BAR_S_EMPTY + sb), ph ^ 1u, abort_flag, 35);
           if (!ok) break;
           tc_fence_after();
           const uint64_t k0 = dK + ((ks * L::kTile) >> 4);
@@ -181,17 +205,20 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
           }
           umma_commit(bar(BAR_K_EMPTY + ks));
           umma_commit(bar(BAR_S_FULL + sb));
-          ++kn;
-          ++sn;
         }
         if (ok) umma_commit(bar(BAR_Q_EMPTY));
       }
-      umma_commit(bar(BAR_FINAL));
+      // every MMA this thread issued has finished before TMEM is released
+      const uint32_t fin = parity == 0u ? BAR_FINAL : BAR_FINAL2;
+      umma_commit(bar(fin));
       volatile uint32_t no_abort = 0u;
-      wait_bar(bar(BAR_FINAL), 0u, &no_abort, 42);
+      wait_bar(bar(fin), 0u, &no_abort, 42);
     }
   } else {
     // ------------------------------------------------------------ one pooled query row per thread
+    // warps 2-5 take keys 0-63 of every tile, warps 6-9 keys 64-127
+    const int half = Y::kHalves == 2 && warp >= 6 ? 1 : 0;
+    constexpr int kChunks = kKeys / 32 / Y::kHalves;   // 32-key chunks of a tile per warp
     const int quad = warp & 3;                      // TMEM lane quadrant of this warp
     const int row = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
@@ -214,21 +241,41 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
       }
       const long long roff = (bh * a.nb + (I < a.nb ? I : 0)) * (long long)a.nb;   // row I of S / L
       float* srow = a.S != nullptr ? a.S + roff : nullptr;
-      for (int t = 0; t < ntiles; ++t) {
+      // a failed wait only marks the item: the warp keeps meeting the other
+      // row warps at their barriers, and they all leave after the item's vote
+      bool bad = false;
+      for (int t = 0; t < ntiles; ++t, ++sn) {
         const uint32_t sb = sn % kSBufs;
-        if (!wait_bar(bar(BAR_S_FULL + sb), (sn / kSBufs) & 1u, abort_flag, 36)) { stop = true; break; }
-        tc_fence_after();
         const bool pass2 = t >= a.nkt || a.passes == 1;
+        if (a.passes == 2 && t == a.nkt) {
+          if (Y::kHalves == 2) {
+            // merge the two halves' running (max, sum) of pass 1
+            ms->pm[half][row] = m;
+            ms->pl[half][row] = l;
+            named_bar(kMergeBar, Y::kRowThreads);
+            const float m0 = ms->pm[0][row], m1 = ms->pm[1][row];
+            const float l0 = ms->pl[0][row], l1 = ms->pl[1][row];
+            m = fmaxf(m0, m1);
+            l = m == -INFINITY ? 0.f
+                               : (m0 == -INFINITY ? 0.f : l0 * ex2(m0 - m)) + (m1 == -INFINITY ? 0.f : l1 * ex2(m1 - m));
+            named_bar(kMergeBar, Y::kRowThreads);    // both halves have read before the next item writes
+          }
+          inv = (row_ok && l > 0.f) ? 1.f / l : 0.f;
+        }
+        if (bad || !wait_bar(bar(BAR_S_FULL + sb), (sn / kSBufs) & 1u, abort_flag, 36)) {
+          bad = true;
+          continue;
+        }
+        tc_fence_after();
         const int kt = t >= a.nkt ? t - a.nkt : t;
         const int c0 = kt * kKeys;
-        if (pass2 && t == a.nkt) inv = (row_ok && l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll 1
-        for (int ch = 0; ch < kKeys / 32; ++ch) {
+        for (int ch = kChunks * half; ch < kChunks * half + kChunks; ++ch) {
           float x[32];
           tmem_ld32(tmem + lane_off + sb * kKeys + ch * 32, x);
           tmem_wait_ld();
-          if (ch == kKeys / 32 - 1) {
-            // the whole S tile is in registers: hand the buffer back
+          if (ch == kChunks * half + kChunks - 1) {
+            // this half of the S tile is in registers: hand it back
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(BAR_S_EMPTY + sb));
@@ -287,8 +334,8 @@ __global__ void __launch_bounds__(kThreads, 1) scores_tc_kernel(const __grid_con
             }
           }
         }
-        ++sn;
       }
+      stop = named_bar_or(kMergeBar, Y::kRowThreads, bad);
     }
   }
 
@@ -325,16 +372,16 @@ cudaError_t launch_scores(const void* qsplit, const void* ksplit, float* S, floa
   a.items = BH * a.nqt;
   a.scale_log2 = 1.4426950408889634f / sqrtf((float)d);
   const long long grid = std::min<long long>(a.items, tc::sm_count());
-  auto go = [&](auto kernel, uint32_t smem) -> cudaError_t {
+  auto go = [&](auto kernel, uint32_t smem, int threads) -> cudaError_t {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kernel<<<(unsigned)grid, kThreads, smem, st>>>(mq, mk, a);
+    kernel<<<(unsigned)grid, threads, smem, st>>>(mq, mk, a);
     return cudaGetLastError();
   };
-  if (d == 128 && size == 64) return go(scores_tc_kernel<128, 64>, Smem<128>::kBytes);
-  if (d == 128 && size == 16) return go(scores_tc_kernel<128, 16>, Smem<128>::kBytes);
-  if (d == 64 && size == 64) return go(scores_tc_kernel<64, 64>, Smem<64>::kBytes);
-  if (d == 64 && size == 16) return go(scores_tc_kernel<64, 16>, Smem<64>::kBytes);
+  if (d == 128 && size == 64) return go(scores_tc_kernel<128, 64>, Smem<128>::kBytes, Layout<64>::kThreads);
+  if (d == 128 && size == 16) return go(scores_tc_kernel<128, 16>, Smem<128>::kBytes, Layout<16>::kThreads);
+  if (d == 64 && size == 64) return go(scores_tc_kernel<64, 64>, Smem<64>::kBytes, Layout<64>::kThreads);
+  if (d == 64 && size == 16) return go(scores_tc_kernel<64, 16>, Smem<64>::kBytes, Layout<16>::kThreads);
   return cudaErrorInvalidValue;
 }
 
