@@ -13,19 +13,22 @@
 //     granularity is 64 queries:
 //        S^T [128 keys x 64 queries] = K_pair [128 x d] . Q^T      (A, B: K-major)
 //        O^T [d x 64 queries]       += V_pair^T [d x 128] . P^T    (A, B: MN-major)
-//     Both accumulate in TMEM (S^T double-buffered, O^T resident).
-//   * Warp roles: warp 0 issues TMA copies (Q once per item; K and V of each
-//     pair into 2-stage rings, 64-row boxes with 128-byte swizzle), warp 1
-//     issues the MMAs from one thread and owns the TMEM allocation, warps 2-9
-//     (two warpgroups, one thread per key / head-dim lane, 32 query columns
-//     per group) run the softmax and the epilogue.  All hand-offs are mbarriers; every wait is bounded in time
-//     and a timeout sets an error word read by svsa_sync_status.
-//   * Softmax: thread k holds key k's 64 scores.  A column (query) maximum
-//     needs all 128 threads, so the running maximum is lazy: a tile only
-//     updates it (warp transpose-reduction + shared memory, then an in-TMEM
-//     rescale of O^T and of the partial sums) when some score exceeds the
-//     current maximum by more than 2^12; otherwise exp2(x - m) is taken against
-//     the stale maximum, which is exact up to the final normalisation.  The
+//     Both accumulate in TMEM (S^T in a 3-deep ring, O^T resident).
+//   * Warp roles: warp 0 issues the TMA copies of Q (once per item) and of
+//     the K pairs, warp 2 those of the V pairs (separate 2-stage rings, 64-row
+//     boxes, 128-byte swizzle); warp 1 issues the S^T MMAs and owns the TMEM
+//     allocation, warp 3 the O^T MMAs; warps 4-19 are four softmax warpgroups,
+//     one thread per key / head-dim lane, 16 query columns per group.  All
+//     hand-offs are mbarriers; every wait is bounded in time and a timeout
+//     sets an error word read by svsa_sync_status.
+//   * Softmax: thread k holds key k's scores for its group's 16 columns.  A
+//     column (query) maximum needs all 128 threads, so the running maximum is
+//     lazy: a tile only updates it (a group vote, a warp transpose-reduction
+//     + shared memory, then an in-TMEM rescale of O^T and of the partial
+//     sums) when some score exceeds the current reference by more than 2^12;
+//     otherwise exp2(x - m) is taken against the stale reference, which is
+//     exact up to the final normalisation.  The exponentials are computed
+//     before the vote, so the wait for the slowest warp overlaps them.  The
 //     row sums stay per-thread partial sums until the epilogue.
 //   * Compensation ("SVG-EAR" 2.A): after the kept pairs, an item walks
 //     ceil(nb / 128) centroid tiles -- 128 key-block means as keys and value
