@@ -12,7 +12,8 @@
 //
 // The ordered prefix is found without sorting: scores are non-negative
 // floats, so their bit patterns order like the values.  A most-significant-
-// digit-first radix select over the 32 bits (4 passes of 8 bits) histograms
+// digit-first radix select over the 31 bits below the sign (4 passes: the
+// 8 exponent bits, then 8, 8 and 7 significand bits) histograms
 // the candidates' counts and masses per digit, and a suffix scan over the 256
 // digits locates the digit holding the crossing element.  After the 4th pass
 // the crossing value v* is known exactly; everything above v* is kept, and of
@@ -113,7 +114,11 @@ __device__ Cut warp_radix_cut(KeyOf key_of, int n, bool by_mass, unsigned long l
   const int lane = threadIdx.x & 31;
   uint32_t prefix = 0u, pmask = 0u, above_c = 0u, eq_c = 0u;
   unsigned long long above_m = 0ull;
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  // digits below the (always clear) sign bit: bits 30-23 (the exponent, one
+  // binade per bin), 22-15, 14-7 and 6-0
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = pass < 3 ? 23 - 8 * pass : 0;
+    const uint32_t dmask = pass < 3 ? 255u : 127u;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       h.cnt[lane * 8 + i] = 0u;
@@ -125,7 +130,7 @@ __device__ Cut warp_radix_cut(KeyOf key_of, int n, bool by_mass, unsigned long l
       const uint32_t key = j < n ? key_of(j) : 0u;
       const bool cand = j < n && (key & pmask) == prefix;
       if (cand) {
-        const uint32_t dg = (key >> shift) & 255u;
+        const uint32_t dg = (key >> shift) & dmask;
         if (by_mass) atomicAdd(&h.mass[dg], fix48(key));
         atomicAdd(&h.cnt[dg], 1u);
       }
@@ -176,7 +181,7 @@ __device__ Cut warp_radix_cut(KeyOf key_of, int n, bool by_mass, unsigned long l
     above_m = __shfl_sync(0xffffffffu, hit_above_m, src);
     eq_c = __shfl_sync(0xffffffffu, hit_c, src);
     prefix |= (uint32_t)(dg < 0 ? 0 : dg) << shift;
-    pmask |= 255u << shift;
+    pmask |= dmask << shift;
     __syncwarp();
   }
   Cut cut;
@@ -349,7 +354,11 @@ __device__ RowCut row_radix_cut(const uint32_t* keys, int nb, bool by_mass, unsi
   const int tid = threadIdx.x, wid = tid >> 5;
   uint32_t prefix = 0u, pmask = 0u, above_c = 0u, eq_c = 0u;
   unsigned long long above_m = 0ull;
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  // digits below the (always clear) sign bit: bits 30-23 (the exponent, one
+  // binade per bin), 22-15, 14-7 and 6-0
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = pass < 3 ? 23 - 8 * pass : 0;
+    const uint32_t dmask = pass < 3 ? 255u : 127u;
 #pragma unroll
     for (int w = 0; w < kRowWarps; ++w) {   // bin tid of every warp's histogram
       sh.cnt[w][tid] = 0u;
@@ -367,7 +376,7 @@ __device__ RowCut row_radix_cut(const uint32_t* keys, int nb, bool by_mass, unsi
       const uint32_t key = j < nb ? keys[j] : 0u;
       const bool cand = j < nb && (key & pmask) == prefix;
       if (cand) {                      // this warp's own histogram
-        const uint32_t dg = (key >> shift) & 255u;
+        const uint32_t dg = (key >> shift) & dmask;
         if (by_mass) atomicAdd(&sh.mass[wid][dg], fix48(key));
         atomicAdd(&sh.cnt[wid][dg], 1u);
       }
@@ -399,7 +408,7 @@ __device__ RowCut row_radix_cut(const uint32_t* keys, int nb, bool by_mass, unsi
     above_m = sh.hit_above_m;
     eq_c = sh.hit_c;
     prefix |= (uint32_t)dg << shift;
-    pmask |= 255u << shift;
+    pmask |= dmask << shift;
     __syncthreads();                   // the hit is read before the next pass clears the bins
   }
   RowCut cut;
