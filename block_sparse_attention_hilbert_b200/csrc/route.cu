@@ -346,25 +346,35 @@ __global__ void __launch_bounds__(kThreads, 1) route_tc_kernel(const __grid_cons
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(BAR_S_EMPTY + sb));
         const int nval = J == nb - 1 ? n_in_last : kBlock;
-        float tmax = -INFINITY;
+        // short dependency chains (one warp per scheduler runs this): packed
+        // scaling, a tree of 3-input maxima, four partial sums
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          x[c] = c < nval ? x[c] * sl2 : -INFINITY;
-          tmax = fmaxf(tmax, x[c]);
+        for (int c = 0; c < 64; c += 2) fma2(x[c], x[c + 1], sl2, 0.f, 0.f);
+        if (nval < 64) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c >= nval) x[c] = -INFINITY;
         }
+        float t16[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) t16[i] = max3(x[4 * i], x[4 * i + 1], fmaxf(x[4 * i + 2], x[4 * i + 3]));
+#pragma unroll
+        for (int i = 0; i < 5; ++i) t16[i] = max3(t16[3 * i], t16[3 * i + 1], t16[3 * i + 2]);
+        const float tmax = max3(max3(t16[0], t16[1], t16[2]), max3(t16[3], t16[4], t16[15]), -INFINITY);
         const float mn = fmaxf(m, tmax);
-        float sum = 0.f;
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t hi[32], lo[32];
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
           const float e0 = ex2(x[c] - mn), e1 = ex2(x[c + 1] - mn);
-          sum += e0 + e1;
+          s4[(c >> 1) & 3] += e0 + e1;
           const __half2 h = __floats2half2_rn(e0, e1);
           const float2 hf = __half22float2(h);
           const __half2 l = __floats2half2_rn(e0 - hf.x, e1 - hf.y);
           hi[c / 2] = *reinterpret_cast<const uint32_t*>(&h);
           lo[c / 2] = *reinterpret_cast<const uint32_t*>(&l);
         }
+        const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
         Z = (m == -INFINITY ? 0.f : Z * ex2(m - mn)) + sum;
         m = mn;
         if (!wait_bar(bar(BAR_E_EMPTY + eb), ((sn / kEBufs) & 1u) ^ 1u, abort_flag, 63) ||
