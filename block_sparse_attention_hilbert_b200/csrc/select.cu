@@ -27,60 +27,9 @@
 
 namespace svsa {
 
-constexpr int kSelThreads = 256;
-
 enum { SEL_THRESHOLD = 0, SEL_TOPK = 1, SEL_STRUCTURED = 2, SEL_ROUTING = 3 };
 
-struct SelShared {
-  uint32_t scan_cnt[kSelThreads / 32];
-  double scan_mass[kSelThreads / 32];
-  uint32_t run;                     // running output position (compaction)
-};
-
 __device__ __forceinline__ uint32_t score_key(float x) { return x > 0.f ? __float_as_uint(x) : 0u; }
-
-// Block-wide inclusive scan of (count, mass) over threadIdx.x.
-__device__ __forceinline__ void block_scan2(uint32_t& c, double& m, SelShared& sh) {
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t yc = __shfl_up_sync(0xffffffffu, c, o);
-    const double ym = __shfl_up_sync(0xffffffffu, m, o);
-    if (lane >= o) { c += yc; m += ym; }
-  }
-  if (lane == 31) { sh.scan_cnt[wid] = c; sh.scan_mass[wid] = m; }
-  __syncthreads();
-  uint32_t oc = 0; double om = 0.0;
-  for (int w = 0; w < wid; ++w) { oc += sh.scan_cnt[w]; om += sh.scan_mass[w]; }
-  c += oc; m += om;
-  __syncthreads();
-}
-
-// Write the kept list: flag(j) computed by `keep`; returns nothing, writes
-// kv_idx (ascending), kv_cnt and the optional bit row.
-template <typename KeepFn>
-__device__ void compact_row(int n, KeepFn keep, int32_t* idx_out, int32_t* cnt_out,
-                            uint32_t* bits_out, SelShared& sh) {
-  const int tid = threadIdx.x;
-  if (tid == 0) sh.run = 0u;
-  __syncthreads();
-  for (int base = 0; base < n; base += kSelThreads) {
-    const int j = base + tid;
-    const bool f = j < n && keep(j);
-    const uint32_t ballot = __ballot_sync(0xffffffffu, f);
-    if (bits_out != nullptr && (tid & 31) == 0 && base + (tid & ~31) < n)
-      bits_out[(base + tid) >> 5] = ballot;
-    uint32_t c = f ? 1u : 0u;
-    double dummy = 0.0;
-    const uint32_t own = c;
-    block_scan2(c, dummy, sh);
-    if (f) idx_out[sh.run + c - own] = j;
-    __syncthreads();
-    if (tid == kSelThreads - 1) sh.run += c;
-    __syncthreads();
-  }
-  if (tid == 0) *cnt_out = (int32_t)sh.run;
-}
 
 // ---------------------------------------------------------------- one warp per row
 // Masses are exact 48-bit fixed-point integers (x * 2^48 truncated; scores are
@@ -535,35 +484,56 @@ __global__ void __launch_bounds__(kRowThreads, 4) select_row_kernel(
   if (tid == 0) kv_cnt[row] = (int32_t)(gt_all + min(eq_all, cut.take));
 }
 
-// STRUCTURED: block coordinates from the raster id of each block's first token.
-__global__ void __launch_bounds__(kSelThreads) structured_kernel(
-    const int32_t* __restrict__ perm, int nb, int H, int W, int win_t, int R, int n_anchors,
-    int anchor_offset, int heads_rows, int cap, int32_t* __restrict__ kv_idx,
-    int32_t* __restrict__ kv_cnt, uint32_t* __restrict__ bits) {
-  __shared__ SelShared sh;
-  const long long row = blockIdx.x;                    // (bh, I)
-  const int I = (int)(row % nb);
+// STRUCTURED: block coordinates from the raster id of each block's first
+// token.  A CTA takes kStructRows rows (one warp each); it first builds, in
+// shared memory, every key block's (t, h) coordinate and a bitmap of the
+// anchor columns, then each warp walks its row 32 blocks at a time and
+// compacts with ballots (ascending lists, no block barriers).
+constexpr int kStructRows = 8;
+
+__global__ void __launch_bounds__(kStructRows * 32) structured_kernel(
+    const int32_t* __restrict__ perm, long long rows, int nb, int H, int W, int win_t, int R, int n_anchors,
+    int anchor_offset, int cap, int32_t* __restrict__ kv_idx, int32_t* __restrict__ kv_cnt,
+    uint32_t* __restrict__ bits) {
+  extern __shared__ __align__(16) unsigned char st_smem[];
+  int2* const crd = reinterpret_cast<int2*>(st_smem);                         // [nb] (t, h)
+  uint32_t* const anchor = reinterpret_cast<uint32_t*>(st_smem + (size_t)nb * sizeof(int2));   // [words]
   const int words = (nb + 31) / 32;
   const long long HW = (long long)H * W;
-  auto coord = [&](int J, int& t, int& h) {
+  for (int J = threadIdx.x; J < nb; J += blockDim.x) {
     const long long r = perm[(long long)J * kBlock];
-    t = (int)(r / HW);
-    h = (int)((r % HW) / W);
-  };
-  int tI, hI;
-  coord(I, tI, hI);
+    crd[J] = make_int2((int)(r / HW), (int)((r % HW) / W));
+  }
+  for (int w = threadIdx.x; w < words; w += blockDim.x) anchor[w] = 0u;
+  __syncthreads();
   const int stride = n_anchors > 0 ? (nb / n_anchors > 0 ? nb / n_anchors : 1) : 1;
-  auto keep = [&](int J) {
-    int tJ, hJ;
-    coord(J, tJ, hJ);
-    if (abs(tI - tJ) <= win_t || abs(hI - hJ) <= R) return true;
-    for (int m = 0; m < n_anchors; ++m)
-      if (((long long)anchor_offset + (long long)m * stride) % nb == J) return true;
-    return false;
-  };
-  compact_row(nb, keep, kv_idx + row * (long long)cap, kv_cnt + row,
-              bits ? bits + row * (long long)words : nullptr, sh);
-  (void)heads_rows;
+  for (int m = threadIdx.x; m < n_anchors; m += blockDim.x) {
+    const int J = (int)(((long long)anchor_offset + (long long)m * stride) % nb);
+    atomicOr(&anchor[J >> 5], 1u << (J & 31));
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  const long long row = (long long)blockIdx.x * kStructRows + (threadIdx.x >> 5);    // (bh, I)
+  if (row >= rows) return;
+  const int I = (int)(row % nb);
+  const int2 cI = crd[I];
+  int32_t* idx_out = kv_idx + row * (long long)cap;
+  uint32_t* bits_out = bits ? bits + row * (long long)words : nullptr;
+  uint32_t run = 0u;
+  for (int base = 0; base < nb; base += 32) {
+    const int J = base + lane;
+    bool f = false;
+    if (J < nb) {
+      const int2 cJ = crd[J];
+      f = abs(cI.x - cJ.x) <= win_t || abs(cI.y - cJ.y) <= R || ((anchor[J >> 5] >> (J & 31)) & 1u);
+    }
+    const uint32_t fb = __ballot_sync(0xffffffffu, f);
+    if (bits_out != nullptr && lane == 0) bits_out[base >> 5] = fb;
+    if (f) idx_out[run + (uint32_t)__popc(fb & lt)] = J;
+    run += (uint32_t)__popc(fb);
+  }
+  if (lane == 0) kv_cnt[row] = (int32_t)run;
 }
 
 cudaError_t launch_select(const float* S, const float* R, long long rows, int nb, int mode, float tau,
@@ -600,8 +570,13 @@ cudaError_t launch_select(const float* S, const float* R, long long rows, int nb
 cudaError_t launch_structured(const int32_t* perm, long long rows, int nb, int H, int W, int win_t,
                               int R, int n_anchors, int anchor_offset, int cap, int32_t* kv_idx,
                               int32_t* kv_cnt, uint32_t* bits, cudaStream_t st) {
-  structured_kernel<<<(unsigned)rows, kSelThreads, 0, st>>>(perm, nb, H, W, win_t, R, n_anchors,
-                                                            anchor_offset, 0, cap, kv_idx, kv_cnt, bits);
+  const size_t smem = (size_t)nb * sizeof(int2) + (size_t)((nb + 31) / 32) * sizeof(uint32_t);
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(structured_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  structured_kernel<<<(unsigned)((rows + kStructRows - 1) / kStructRows), kStructRows * 32, smem, st>>>(
+      perm, rows, nb, H, W, win_t, R, n_anchors, anchor_offset, cap, kv_idx, kv_cnt, bits);
   return cudaGetLastError();
 }
 
