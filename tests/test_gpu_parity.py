@@ -428,13 +428,15 @@ def test_cocluster_layer_matches_oracle(select):
 
 
 @pytest.mark.parametrize("grid", [(1, 1, 1), (1, 1, 64), (1, 1, 65), (2, 3, 5), (1, 8, 8)])
-@pytest.mark.parametrize("case", ["topk", "threshold", "threshold16", "routing_comp", "cocluster"])
+@pytest.mark.parametrize("case", ["topk", "threshold", "threshold16", "routing_comp", "cocluster", "structured"])
 def test_degenerate_grids(grid, case):
     """One token, exactly one block, one token past a block, tiny ragged grids:
     the whole layer through every rule, masks and outputs against the oracle."""
     d = 64 if case == "threshold16" else 128
-    sel = "topk" if case in ("topk", "cocluster") else "threshold"
+    sel = {"topk": "topk", "cocluster": "topk", "structured": "structured"}.get(case, "threshold")
     kw = {"routing": True, "compensate": True} if case == "routing_comp" else {}
+    if case == "structured":
+        kw = {"n_anchors": 1}                                  # at most nb anchor columns
     w = _small(sel, 16 if case == "threshold16" else 64, grid=grid, heads=2, d=d, tau=0.9, keep_frac=0.3, **kw)
     q, k, v = (t.cuda() for t in workloads.make_qkv(w, seed=9))
     if case == "cocluster":
