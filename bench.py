@@ -47,6 +47,7 @@ def _args():
     ap.add_argument("--order", default=None, choices=["raster", "hilbert", "cocluster"])
     ap.add_argument("--heads", type=int, default=None, help="override the layer's head count (profiling captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay of the step")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--schedule", default=None, metavar="N,DENSE,START,END,EVERY",
                     help="time whole denoising runs of the layer under the step schedule "
@@ -381,6 +382,29 @@ def run_svsa(args):
     h2d = 3 * q.numel() * q.element_size()
     d2h = out.numel() * out.element_size()
 
+    # the same step replayed from a CUDA graph (no host launch per kernel);
+    # reported beside the eager step, whose per-phase events the graph cannot hold
+    graph_ms, graph_err = None, None
+    layer = None
+    if not args.no_graph:
+        try:
+            layer = attn.capture(q, k, v, out, anchor_offset=off, with_order=True)
+        except Exception as exc:                       # reported, not fatal: the eager step is the measure
+            graph_err = f"capture failed: {exc}"[:200]
+    if layer is not None:
+        gtimes = []
+        for i in range(args.warmup + args.steps):
+            flush.fill_(1.0)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            layer.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if i >= args.warmup:
+                gtimes.append(e0.elapsed_time(e1))
+        del layer
+        graph_ms = _max_over_ranks(statistics.mean(gtimes), ws)
+
     peaks, peak_src = _peaks()
     # a kernel inside steps of 100 ms or more runs seconds-long loops under the
     # power cap: its denominator is the sustained GEMM rate, else the burst one
@@ -411,6 +435,8 @@ def run_svsa(args):
             "dense_ms": dense_ms, "dense_tflops": dense_flops / (dense_ms * 1e-3) / 1e12,
             "speedup_vs_dense": dense_ms / attn_ms, "density": density,
             "kept_tflop_per_step": kflops / 1e12,
+            "graph": ({"ms_per_step": graph_ms, "value": ws * kflops / (graph_ms * 1e-3) / 1e12}
+                      if graph_ms is not None else ({"unavailable": graph_err} if graph_err else None)),
             "phase_ms": {p: statistics.mean(times[p]) for p in phases},
             "reorder_gbs": reorder_bytes / (reorder_ms * 1e-3) / 1e9,
             "inverse_gbs": inverse_bytes / (inverse_ms * 1e-3) / 1e9,

@@ -261,4 +261,4 @@ def svsa_sync_status(stream=None) -> None:
     _check(lib().svsa_sync_status(_stream(stream)), "svsa_sync_status")
 
 
-from .pipeline import SparseVideoAttention, LayerBuffers  # noqa: E402,F401
+from .pipeline import CapturedLayer, SparseVideoAttention, LayerBuffers  # noqa: E402,F401

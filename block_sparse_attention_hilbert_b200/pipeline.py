@@ -69,6 +69,17 @@ class LayerBuffers:
                          self.cbar)
 
 
+class CapturedLayer:
+    """A layer call captured by SparseVideoAttention.capture()."""
+
+    def __init__(self, graph):
+        self.graph = graph
+
+    def replay(self):
+        """Run the captured layer on the current stream (asynchronous)."""
+        self.graph.replay()
+
+
 def default_attn_passes(select: int, Npad: int, d: int) -> int:
     """Key-range passes of the attention for a head of Npad reordered tokens:
     one for the structured rule (its windows keep the key blocks of
@@ -292,6 +303,36 @@ class SparseVideoAttention:
         return out
 
     # ---- whole layer ----------------------------------------------------
+    # ---- the layer as one CUDA graph ---------------------------------------
+    def capture(self, q, k, v, out, *, anchor_offset: int = 0, with_order: bool = False) -> "CapturedLayer":
+        """Capture one layer call on these device buffers (reorder, block mask,
+        attention, inverse reorder; the token order too with with_order) into
+        a CUDA graph.  replay() re-runs it on whatever q, k and v then hold and
+        writes `out`, without a host launch per kernel.  The buffers, the
+        shape and the mask parameters (anchor_offset included) are fixed at
+        capture."""
+        if self.cocluster and not with_order and not self._perm_ready:
+            raise ValueError("build the co-clustering order first, or capture it with with_order=True")
+
+        def body():
+            if with_order or not self._perm_ready:
+                self.build_perm(q=q, k=k)
+            self.reorder(q, k, v)
+            self.build_mask(anchor_offset)
+            self.attend()
+            self.inverse(out)
+
+        # allocator-safe warm-up on a side stream, then the capture
+        side = torch.cuda.Stream(q.device)
+        side.wait_stream(torch.cuda.current_stream(q.device))
+        with torch.cuda.stream(side):
+            body()
+        torch.cuda.current_stream(q.device).wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            body()
+        return CapturedLayer(graph)
+
     def __call__(self, q, k, v, *, out=None, anchor_offset: int = 0, reuse_mask: bool = False, stream=None):
         if out is None:
             out = torch.empty_like(q)

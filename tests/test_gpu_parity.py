@@ -509,3 +509,25 @@ def test_split_attention_matches_single_pass_and_oracle(passes, select, kw):
             ref = oracle.masked_attention(qp[eta], kp[eta], vp[eta], w.N, keep[eta])
         gout = np.concatenate([ap[eta][I * 64:min(I * 64 + 64, w.N)] for I in range(many.nb)])
         check_attention(gout, np.concatenate([ref[I] for I in range(many.nb)]), f"passes={passes} head {eta}")
+
+
+@pytest.mark.parametrize("select,kw", [("topk", {}), ("threshold", dict(routing=True, compensate=True)),
+                                       ("structured", dict(n_anchors=2))])
+def test_captured_layer_replays_the_eager_call(select, kw):
+    """A layer captured in a CUDA graph, replayed on new contents of its input
+    buffers, gives the eager call's output bit for bit."""
+    w = _small(select, 64, grid=(6, 12, 20), heads=2, tau=0.9, keep_frac=0.3, **kw)
+    q, k, v = (t.cuda() for t in workloads.make_qkv(w, seed=1))
+    layer = gpu_layer(w, q, k, v)                         # builds the order, sizes the buffers
+    out = torch.empty_like(q)
+    g = layer.capture(q, k, v, out)
+    for seed in (2, 3):
+        q2, k2, v2 = (t.cuda() for t in workloads.make_qkv(w, seed=seed))
+        q.copy_(q2)
+        k.copy_(k2)
+        v.copy_(v2)
+        g.replay()
+        torch.cuda.synchronize()
+        ref = gpu_layer(w, q2, k2, v2).out                 # a fresh layer, eager
+        assert torch.equal(out, ref), f"seed {seed}: replay differs from the eager call"
+    svsa.svsa_sync_status()
