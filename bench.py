@@ -351,6 +351,30 @@ def run_svsa(args):
     attn_ms_local = statistics.mean(times["attn"])
     attn_ms = _max_over_ranks(attn_ms_local, ws)
 
+    # the same step replayed from a CUDA graph (no host launch per kernel),
+    # right after the eager steps so that both see the same clocks; reported
+    # beside the eager step, whose per-phase events a graph cannot hold
+    graph_ms, graph_err = None, None
+    layer = None
+    if not args.no_graph:
+        try:
+            layer = attn.capture(q, k, v, out, anchor_offset=off, with_order=True)
+        except Exception as exc:                       # reported, not fatal: the eager step is the measure
+            graph_err = f"capture failed: {exc}"[:200]
+    if layer is not None:
+        gtimes = []
+        for i in range(args.warmup + args.steps):
+            flush.fill_(1.0)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            layer.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if i >= args.warmup:
+                gtimes.append(e0.elapsed_time(e1))
+        del layer
+        graph_ms = _max_over_ranks(statistics.mean(gtimes), ws)
+
     # dense denominator: same arithmetic over every key block
     dtimes = []
     for i in range(args.warmup + args.steps):
@@ -381,29 +405,6 @@ def run_svsa(args):
     e2e_ms = _max_over_ranks(statistics.mean(e2e_times), ws)
     h2d = 3 * q.numel() * q.element_size()
     d2h = out.numel() * out.element_size()
-
-    # the same step replayed from a CUDA graph (no host launch per kernel);
-    # reported beside the eager step, whose per-phase events the graph cannot hold
-    graph_ms, graph_err = None, None
-    layer = None
-    if not args.no_graph:
-        try:
-            layer = attn.capture(q, k, v, out, anchor_offset=off, with_order=True)
-        except Exception as exc:                       # reported, not fatal: the eager step is the measure
-            graph_err = f"capture failed: {exc}"[:200]
-    if layer is not None:
-        gtimes = []
-        for i in range(args.warmup + args.steps):
-            flush.fill_(1.0)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            layer.replay()
-            e1.record(stream)
-            torch.cuda.synchronize()
-            if i >= args.warmup:
-                gtimes.append(e0.elapsed_time(e1))
-        del layer
-        graph_ms = _max_over_ranks(statistics.mean(gtimes), ws)
 
     peaks, peak_src = _peaks()
     # a kernel inside steps of 100 ms or more runs seconds-long loops under the
