@@ -84,8 +84,8 @@ constexpr uint32_t kColS0 = 0, kColO = 192;
 enum : uint32_t {
   BAR_Q_FULL = 0, BAR_Q_EMPTY, BAR_K_FULL, BAR_K_EMPTY = BAR_K_FULL + kKStages,
   BAR_V_FULL = BAR_K_EMPTY + kKStages, BAR_V_EMPTY = BAR_V_FULL + kVStages,
-  BAR_S_FULL = BAR_V_EMPTY + kVStages, BAR_S_EMPTY = BAR_S_FULL + kSBufs,
-  BAR_P_FULL = BAR_S_EMPTY + kSBufs, BAR_P_EMPTY = BAR_P_FULL + kPBufs, BAR_O_FULL = BAR_P_EMPTY + kPBufs,
+  BAR_S_FULL = BAR_V_EMPTY + kVStages,
+  BAR_P_FULL = BAR_S_FULL + kSBufs, BAR_P_EMPTY = BAR_P_FULL + kPBufs, BAR_O_FULL = BAR_P_EMPTY + kPBufs,
   BAR_O_EMPTY, BAR_FINAL, BAR_FINAL2, NUM_BARS
 };
 
@@ -174,10 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       mbar_init(bar(BAR_V_FULL + i), 1);
       mbar_init(bar(BAR_V_EMPTY + i), 1);
     }
-    for (int i = 0; i < kSBufs; ++i) {
-      mbar_init(bar(BAR_S_FULL + i), 1);
-      mbar_init(bar(BAR_S_EMPTY + i), 4 * kGroups);
-    }
+    for (int i = 0; i < kSBufs; ++i) mbar_init(bar(BAR_S_FULL + i), 1);
     for (int i = 0; i < kPBufs; ++i) {
       mbar_init(bar(BAR_P_FULL + i), 4 * kGroups);
       mbar_init(bar(BAR_P_EMPTY + i), 1);
@@ -290,7 +287,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     // ------------------------------------------------------------ MMA issuers
     // Warp 1 issues the first product S^T = K_pair . Q^T of every tile into
     // the kSBufs-deep S ring (it runs ahead as far as the softmax frees S
-    // buffers); warp 3 issues the second product O^T += V^T . P^T.  Two
+    // buffers: the P hand-off of a slot also frees the S buffer of that slot,
+    // whose scores the softmax has read by then, so one arrive per warp and
+    // tile serves both rings); warp 3 issues the second product
+    // O^T += V^T . P^T.  Two
     // issuing threads keep the tensor core fed, and each commits (hence
     // waits for) only its own MMAs.  Descriptors are base values plus
     // compile-time offsets (the 14-bit address field never carries).
@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           for (int t = 0; t < npairs && ok; ++t) {
             const uint32_t ks = ring % kKStages, sb = tiles % kSBufs;
             ok = wait_bar(bar(BAR_K_FULL + ks), (ring / kKStages) & 1u, abort_flag, 5) &&
-                 wait_bar(bar(BAR_S_EMPTY + sb), ((tiles / kSBufs) & 1u) ^ 1u, abort_flag, 6);
+                 wait_bar(bar(BAR_P_FULL + sb), ((tiles / kSBufs) & 1u) ^ 1u, abort_flag, 6);
             if (!ok) break;
             tc_fence_after();
             const uint64_t a0 = dK + ((ks * 32768u) >> 4);
@@ -534,10 +534,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
               tmem_wait_st();
             }
           }
-          // S slot free (this warp's reads of it are done)
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(BAR_S_EMPTY + sb));
           // P^T row k, this group's columns: exp2(y), fp16, 128-byte swizzled MN-major layout
           uint32_t pk[kCols / 2];
 #pragma unroll
@@ -549,6 +545,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           st_shared_v4(pa0 + sb * 16384u, pk[0], pk[1], pk[2], pk[3]);
           st_shared_v4((pa0 ^ 16u) + sb * 16384u, pk[4], pk[5], pk[6], pk[7]);
           fence_async_smem();
+          // P tile ready, and the S slot free: this warp's TMEM reads of it
+          // (and any rescale of O^T) are complete and ordered before the arrive
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(BAR_P_FULL + sb));
