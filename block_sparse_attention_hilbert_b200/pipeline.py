@@ -236,10 +236,12 @@ class SparseVideoAttention:
 
     def forward_host(self, q, k, v, out, *, anchor_offset: int = 0, reuse_mask: bool = False, groups: int = 12):
         """q, k, v, out: pinned host bf16 [B, heads, N, d] (raster order).  The rows
-        are processed in `groups` groups; each group's inputs are copied in on one
-        stream, its four library calls run on the current stream once they have
-        arrived, and its output is copied out on a third stream.  The current
-        stream waits for the last copy, so synchronising it covers the layer."""
+        are processed in `groups` groups.  Every group's input copies are queued
+        first, on one stream, each group ending in an event, so the link stays
+        busy whatever the host's launch rate; each group's four library calls
+        run on the current stream once its event has fired, and its output is
+        copied out on a third stream.  The current stream waits for the last
+        copy, so synchronising it covers the layer."""
         b = self.buf
         rows = self.B * self.heads
         if getattr(self, "_stage", None) is None:
@@ -265,11 +267,17 @@ class SparseVideoAttention:
         # the copy streams start after what the current stream has already queued
         self._h2d.wait_stream(compute)
         self._d2h.wait_stream(compute)
-        for r0, r1 in zip(bounds[:-1], bounds[1:]):
-            with torch.cuda.stream(self._h2d):
+        spans = list(zip(bounds[:-1], bounds[1:]))
+        arrived = []
+        with torch.cuda.stream(self._h2d):
+            for r0, r1 in spans:
                 for h, d_ in ((hq, dq), (hk, dk), (hv, dv)):
                     d_[r0:r1].copy_(h[r0:r1], non_blocking=True)
-            compute.wait_stream(self._h2d)
+                ev = torch.cuda.Event()
+                ev.record(self._h2d)
+                arrived.append(ev)
+        for (r0, r1), ev in zip(spans, arrived):
+            compute.wait_event(ev)
             sh, m = self._group(r0, r1)
             if self.cocluster:
                 svsa_reorder_heads(dq[r0:r1], self._rows(b.qp, r0, r1), b.perm_q[r0:r1], sh, compute)
