@@ -134,7 +134,7 @@ svsa_status svsa_build_perm(svsa_shape s, int32_t order, int32_t* perm, int32_t*
                             void* ws, size_t ws_bytes, void* stream);
 
 /* Permutation build for callers that cannot allocate device memory.
- * (An addition of this library with no counterpart on the pages.)  Some
+ * (An addition of this library: the method descriptions have no counterpart.)  Some
  * callers have no way to provide the scratch svsa_build_perm needs: code that
  * runs where cudaMalloc is not allowed or not reachable -- a plain-C host
  * that owns no allocator, or a component whose device memory is entirely

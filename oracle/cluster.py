@@ -13,7 +13,7 @@ Sources (page title, section):
   * "SVG-EAR", 2.A: tokens are grouped semantically and permuted so that
     similar tokens are contiguous in memory, forming the block structure.
 
-Readings where the pages leave a step open (also listed in the design doc):
+Readings taken where the method description leaves a step open:
   * per (batch, head), C = nb clusters (as many as 64-token blocks);
   * affinity = the dot product q . k (the attention logit up to its 1/sqrt(d)
     scale), taken exactly: bf16 token values and float32 centroids, products

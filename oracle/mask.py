@@ -16,7 +16,7 @@ Sources (page title, section):
     individual queries, compensation error estimated per block, greedy pick by
     estimated error divided by block size under a fixed density budget.
 
-Readings where the pages leave a step open (also listed in the design doc):
+Readings taken where the method description leaves a step open:
   * pooled scores P_IJ = softmax_J(qbar_I . kbar_J / sqrt(d)) over all key
     blocks, one entry per block (no block-size weighting);
   * threshold rule: sort a row by (score desc, block index asc), keep the
