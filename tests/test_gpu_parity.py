@@ -427,6 +427,48 @@ def test_cocluster_layer_matches_oracle(select):
         check_attention(on[eta], ref_raster, f"head {eta}")
 
 
+@pytest.mark.parametrize("case", ["topk", "threshold16", "routing_comp", "structured", "cocluster"])
+def test_batch_rows_are_independent(case):
+    """B = 2: every step treats the (batch, head) rows independently, so the
+    two-batch layer equals two one-batch layers (each checked against the
+    oracle elsewhere) bit for bit: permutations, masks and outputs."""
+    sel = {"topk": "topk", "cocluster": "topk", "structured": "structured"}.get(case, "threshold")
+    kw = {"routing": True, "compensate": True} if case == "routing_comp" else {}
+    if case == "structured":
+        kw = {"n_anchors": 2}
+    sub = 16 if case == "threshold16" else 64
+    T, H, W = 5, 12, 20
+    w2 = workloads.Workload("batch2", 2, 2, 128, T, H, W, select=sel, sub_block=sub, tau=0.9, keep_frac=0.3, **kw)
+    q, k, v = (t.cuda() for t in workloads.make_qkv(w2, seed=11))
+    w1 = workloads.Workload("batch1", 1, 2, 128, T, H, W, select=sel, sub_block=sub, tau=0.9, keep_frac=0.3, **kw)
+
+    def run(w, q, k, v):
+        if case == "cocluster":
+            attn = _cocluster_case(w, q, k) if w.B == 1 else svsa.SparseVideoAttention(
+                w.B, w.heads, T, H, W, w.d, order="cocluster", select=w.select, tau=w.tau, keep_frac=w.keep_frac,
+                cluster_rounds=3, device="cuda")
+            if w.B != 1:
+                attn.build_perm(q=q, k=k)
+            out = attn(q, k, v)
+        else:
+            attn = gpu_layer(w, q, k, v, anchor_offset=1)
+            out = attn.out
+        torch.cuda.synchronize()
+        return attn, out
+
+    a2, o2 = run(w2, q, k, v)
+    rows = w2.heads
+    for bi in range(2):
+        a1, o1 = run(w1, *(t[bi:bi + 1].contiguous() for t in (q, k, v)))
+        assert torch.equal(o2[bi].view(torch.int16), o1[0].view(torch.int16)), f"batch {bi}: outputs differ"
+        assert torch.equal(a2.buf.kv_cnt.view(2 * rows, -1)[bi * rows:(bi + 1) * rows],
+                           a1.buf.kv_cnt.view(rows, -1)), f"batch {bi}: kept counts differ"
+        assert np.array_equal(gpu_keep(a2)[bi * rows:(bi + 1) * rows], gpu_keep(a1)), f"batch {bi}: masks differ"
+        if case == "cocluster":
+            assert torch.equal(a2.buf.perm_q[bi * rows:(bi + 1) * rows], a1.buf.perm_q)
+            assert torch.equal(a2.buf.perm_k[bi * rows:(bi + 1) * rows], a1.buf.perm_k)
+
+
 @pytest.mark.parametrize("grid", [(1, 1, 1), (1, 1, 64), (1, 1, 65), (2, 3, 5), (1, 8, 8)])
 @pytest.mark.parametrize("case", ["topk", "threshold", "threshold16", "routing_comp", "cocluster", "structured"])
 def test_degenerate_grids(grid, case):
