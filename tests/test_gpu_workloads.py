@@ -138,3 +138,18 @@ def test_hunyuan_2x_subblock_mask_reuse():
         for I in rows:
             check_attention(op[I * 64:min(I * 64 + 64, w.N)], ref[I], f"step {step} block {I}")
         del out
+
+
+def test_largest_block_count_topk():
+    """The largest grid the boundary accepts in blocks (nb <= 16384): a ragged
+    61 x 133 x 129 latent (1,046,577 tokens, nb = 16,353, Hilbert cube side
+    256), one head, d = 64; every row keeps exactly k blocks and sampled rows
+    match the oracle (the CTA-per-row selection and the long kept lists).
+    At this size the pooled scores of one row are close together, so about a
+    third of its blocks sit within the rounding bound of the cut and are
+    checked only through the exact count and the outputs."""
+    w = workloads.Workload("largest_nb", 1, 1, 64, 61, 133, 129, order="hilbert", select="topk", keep_frac=0.25)
+    assert w.nb == 16353
+    q, k, v = workloads.make_qkv(w, device="cuda")
+    attn = _check_layer(w, q, k, v, n_rows=5, heads=[0])
+    assert torch.all(attn.buf.kv_cnt == oracle.topk_count(w.keep_frac, attn.nb))
