@@ -153,3 +153,14 @@ def test_largest_block_count_topk():
     q, k, v = workloads.make_qkv(w, device="cuda")
     attn = _check_layer(w, q, k, v, n_rows=5, heads=[0])
     assert torch.all(attn.buf.kv_cnt == oracle.topk_count(w.keep_frac, attn.nb))
+
+
+def test_largest_block_count_threshold():
+    """The same largest grid under the cumulative-mass rule (tau = 0.5): the
+    mass-based radix selection over 16,353-entry rows, sampled rows against
+    the oracle."""
+    w = workloads.Workload("largest_nb_tau", 1, 1, 64, 61, 133, 129, order="hilbert", select="threshold", tau=0.5)
+    q, k, v = workloads.make_qkv(w, device="cuda")
+    attn = _check_layer(w, q, k, v, n_rows=3, heads=[0])
+    cnt = attn.buf.kv_cnt.cpu().numpy()
+    assert cnt.min() >= 1 and cnt.max() <= attn.nb
