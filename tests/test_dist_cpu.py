@@ -53,3 +53,43 @@ def test_kept_flops_from_lists():
     n = np.array([64, 64, 8])
     expect = 4 * 128 * (64 * 64 + 64 * (64 + 8) + 8 * (64 + 8))
     assert bench.kept_flops_from_lists(idx, cnt, n, 128) == expect
+
+
+def test_traffic_is_reported_only_for_the_profiled_kernel_source(tmp_path, monkeypatch):
+    """roofline.traffic comes from a committed ncu figure only while the
+    attention sources still hash to the value recorded with it; any edit of
+    them turns it into null (the counters no longer describe the kernel)."""
+    import hashlib
+    srcs = []
+    for name, body in (("attn_tc.cu", b"kernel v1\n"), ("tcgen05.cuh", b"helpers\n")):
+        p = tmp_path / name
+        p.write_bytes(body)
+        srcs.append(str(p))
+    h = hashlib.sha256()
+    for p in srcs:
+        h.update(open(p, "rb").read())
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "attn_demo.traffic.txt").write_text(
+        f"# comment: 1\ndram_bytes_per_launch: 12345\nkernel_sha256_16: {h.hexdigest()[:16]}\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "ATTN_KERNEL_SRCS", srcs)
+    assert bench._attn_traffic("demo") == 12345.0
+    assert bench._attn_traffic("missing") is None
+    (tmp_path / "attn_tc.cu").write_bytes(b"kernel v2\n")
+    assert bench._attn_traffic("demo") is None
+
+
+def test_committed_traffic_file_is_well_formed():
+    """The committed wan13b figure parses and is at least the algorithmic
+    Q, K, V, O bytes of a launch within 5% (DRAM bytes below the algorithmic
+    ones would mean a capture of some other launch)."""
+    path = os.path.join(bench.ROOT, "profiles", "attn_wan13b.traffic.txt")
+    kv = {}
+    for line in open(path):
+        if ":" in line and not line.startswith("#"):
+            a, b = line.split(":", 1)
+            kv[a.strip()] = b.strip()
+    assert len(kv["kernel_sha256_16"]) == 16
+    algorithmic = 4 * 12 * 32768 * 128 * 2
+    assert 0.95 * algorithmic <= float(kv["dram_bytes_per_launch"]) <= 1.25 * algorithmic
