@@ -1,15 +1,19 @@
 """Benchmark of the block-sparse video attention hot path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload wan13b] [--order hilbert]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload hunyuan_2x] [--order hilbert]
     python bench.py --impl reference ...      # the fp64 CPU oracle as the reference arm
 
-One step = the whole path over one synthetic layer already resident in HBM:
-svsa_build_perm, svsa_reorder (Q, K), svsa_reorder_values (V), svsa_build_mask, svsa_attn_fwd,
-svsa_inverse_reorder.  Each timed step is bracketed by CUDA events on the
-launching stream, with an L2 flush (a 512 MiB write) between steps, outside
-the events.  `value` = kept-block attention FLOPs of all ranks / the slowest
-rank's time (TFLOP/s).  Ranks run independent layers (weak scaling, no
-collective on the data path; only the timing max is reduced).
+One step = the whole path over one synthetic layer already resident in HBM,
+for one mask cycle of the layer: svsa_build_perm, then at each of the layer's
+reuse_steps denoising steps svsa_reorder (Q, K), svsa_reorder_values (V),
+svsa_attn_fwd and svsa_inverse_reorder, with svsa_build_mask at the first of
+them (the HunyuanVideo layer reuses its mask over 4 steps while Q and K
+drift; the other layers build a mask every step).  Each timed step is
+bracketed by CUDA events on the launching stream, with an L2 flush (a
+512 MiB write) between steps, outside the events.  `value` = kept-block
+attention FLOPs of all ranks / the slowest rank's time (TFLOP/s).  Ranks run
+independent layers (weak scaling, no collective on the data path; only the
+timing max is reduced).
 """
 from __future__ import annotations
 
@@ -40,10 +44,13 @@ ATTN_KERNEL_SRCS = [os.path.join(ROOT, "block_sparse_attention_hilbert_b200", "c
 def _args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="svsa", choices=["svsa", "reference"])
-    ap.add_argument("--workload", default="wan13b", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--workload", default="hunyuan_2x", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--secondary", default="wan13b",
+                    help="a second, short layer whose attention / dense figures ride along in the line ('' = none)")
+    ap.add_argument("--scorer", default=None, choices=["pooled", "sics"])
     ap.add_argument("--order", default=None, choices=["raster", "hilbert", "cocluster"])
     ap.add_argument("--heads", type=int, default=None, help="override the layer's head count (profiling captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -101,6 +108,8 @@ def _workload(args):
         w = w.with_(order=args.order)
     if args.heads:
         w = w.with_(heads=args.heads)
+    if args.scorer:
+        w = w.with_(scorer=args.scorer, sub_block=64 if args.scorer == "sics" else w.sub_block)
     return w
 
 
@@ -217,7 +226,7 @@ def _oracle_sample(w, q, k, v, seconds: float, perm_cache=None):
     heads_done = 0
     nb = w.nb
     k_keep = oracle.topk_count(w.keep_frac, nb)
-    for eta in range(w.heads):
+    for eta in range(min(w.heads, q.shape[1])):
         qp, kp, vp = (oracle.reorder(t[0, eta].float().cpu().numpy().astype(np.float64), perm) for t in (q, k, v))
         qb, nv = oracle.pool(qp, w.N)
         kb, _ = oracle.pool(kp, w.N)
@@ -225,9 +234,13 @@ def _oracle_sample(w, q, k, v, seconds: float, perm_cache=None):
         for I in range(nb):
             if w.select == "structured":
                 keep_row = oracle.structured_mask(perm, w.T, w.H, w.W, win_t=w.win_t, win_rows=w.win_rows,
-                                                  n_anchors=w.n_anchors, anchor_offset=0)[I]
+                                                  n_anchors=w.n_anchors, seed=0, step=0)[I]
             else:
-                if w.sub_block == 64:
+                if w.scorer == "sics":
+                    if I == 0:
+                        S_head = oracle.sics_scores(kp, w.N)
+                    S = S_head
+                elif w.sub_block == 64:
                     S = oracle.block_scores(qb[I:I + 1], kb)[0]
                 else:
                     S = oracle.subblock_scores(qp, kp, w.N, w.sub_block, rows=[I])[0]
@@ -258,7 +271,9 @@ def run_reference(args):
         return
     import oracle
     w = _workload(args)
-    q, k, v = workloads.make_qkv(w, device="cpu")
+    # the sample covers a head or two: generate two heads of the layer's shape
+    # (every head has the same shape and input distribution)
+    q, k, v = workloads.make_qkv(w.with_(heads=min(w.heads, 2)), device="cpu")
     if w.order not in ("raster", "hilbert"):
         raise SystemExit("the oracle arm samples the geometric orders (raster, hilbert) only")
     perm_cache = oracle.build_perm(w.T, w.H, w.W, w.order)
@@ -284,6 +299,58 @@ def run_reference(args):
 
 
 # --------------------------------------------------------------------------- GPU arm
+def _layer(svsa, w, dev, seed=0):
+    return svsa.SparseVideoAttention(w.B, w.heads, w.T, w.H, w.W, w.d, order=w.order, select=w.select,
+                                     tau=w.tau, keep_frac=w.keep_frac, sub_block=w.sub_block,
+                                     win_t=w.win_t, win_rows=w.win_rows,
+                                     n_anchors=w.n_anchors if w.select == "structured" else 0,
+                                     routing=w.routing, compensate=w.compensate, seed=seed, scorer=w.scorer,
+                                     device=dev)
+
+
+def _timed(fn, stream, flush, warmup, iters):
+    """Mean CUDA-event time (ms) of fn() on `stream`, L2 flushed before each call."""
+    times = []
+    for i in range(warmup + iters):
+        flush.fill_(1.0)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i >= warmup:
+            times.append(e0.elapsed_time(e1))
+    return statistics.mean(times)
+
+
+def _secondary(svsa, name, dev, stream, flush, peaks, steps):
+    """Attention and dense figures of a second, short layer (one mask per step)."""
+    w = workloads.WORKLOADS[name]
+    q, k, v = workloads.make_qkv(w, device=dev)
+    attn = _layer(svsa, w, dev)
+    out = torch.empty_like(q)
+    attn(q, k, v, out=out)
+    torch.cuda.synchronize()
+    nvalid = np.minimum(64, w.N - 64 * np.arange(w.nb)).astype(np.int64)
+    kflops = kept_flops_from_lists(attn.buf.kv_idx.cpu().numpy(), attn.buf.kv_cnt.cpu().numpy(), nvalid, w.d)
+    dense_flops = 4.0 * w.d * float(w.N) ** 2 * w.heads * w.B
+    step_ms = _timed(lambda: attn(q, k, v, out=out), stream, flush, 3, steps)
+    attn_ms = _timed(attn.attend, stream, flush, 3, steps)
+    dense_ms = _timed(attn.attend_dense, stream, flush, 3, steps)
+    peak = float(peaks["bf16_tflops"])
+    res = {"workload": name, "heads": w.heads, "grid": [w.T, w.H, w.W], "select": w.select,
+           "keep_frac": w.keep_frac, "step_ms": step_ms, "attn_ms": attn_ms,
+           "attn_tflops": kflops / (attn_ms * 1e-3) / 1e12, "dense_ms": dense_ms,
+           "dense_tflops": dense_flops / (dense_ms * 1e-3) / 1e12, "speedup_vs_dense": dense_ms / attn_ms,
+           "density": kflops / dense_flops}
+    res["attn_frac_of_peak"] = res["attn_tflops"] / peak
+    res["dense_frac_of_peak"] = res["dense_tflops"] / peak
+    res["peak"] = "bf16_tflops (burst)"
+    del attn, q, k, v, out
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_svsa(args):
     rank, ws, local = _dist()
     import block_sparse_attention_hilbert_b200 as svsa
@@ -293,118 +360,140 @@ def run_svsa(args):
     svsa.lib()
     w = _workload(args)
     stream = torch.cuda.current_stream()
-    q, k, v = workloads.make_qkv(w, seed=rank, device=dev)
-    attn = svsa.SparseVideoAttention(w.B, w.heads, w.T, w.H, w.W, w.d, order=w.order, select=w.select,
-                                     tau=w.tau, keep_frac=w.keep_frac, sub_block=w.sub_block,
-                                     win_t=w.win_t, win_rows=w.win_rows,
-                                     n_anchors=w.n_anchors if w.select == "structured" else 0,
-                                     routing=w.routing, compensate=w.compensate, device=dev)
-    out = torch.empty_like(q)
+    # one bench step = the layer's mask cycle: the mask is built at the first
+    # denoising step and reused for the next reuse_steps - 1, while Q and K
+    # drift by sigma * N(0, 1) per step (V does not)
+    cycle = max(1, w.reuse_steps)
+    q0, k0, v = workloads.make_qkv(w, seed=rank, device=dev)
+    qs, ks = [q0], [k0]
+    for st in range(1, cycle):
+        qs.append(workloads.perturb(qs[-1], sigma=w.sigma, seed=rank, step=st, tensor=workloads.TENSOR_Q))
+        ks.append(workloads.perturb(ks[-1], sigma=w.sigma, seed=rank, step=st, tensor=workloads.TENSOR_K))
+    attn = _layer(svsa, w, dev)
+    out = torch.empty_like(q0)
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
-    off = workloads.anchor_offset(seed=0, step=0, nkb=w.nb, n_anchors=w.n_anchors) if w.select == "structured" else 0
 
-    def step(evs=None):
-        if evs is not None:
-            evs[0].record(stream)
-        attn.build_perm(q=q, k=k)
-        if evs is not None:
-            evs[1].record(stream)
-        attn.reorder(q, k, v)
-        if evs is not None:
-            evs[2].record(stream)
-        attn.build_mask(off)
-        if evs is not None:
-            evs[3].record(stream)
-        attn.attend()
-        if evs is not None:
-            evs[4].record(stream)
-        attn.inverse(out)
-        if evs is not None:
-            evs[5].record(stream)
+    phases = ["perm", "reorder", "mask", "attn", "inverse"]
+
+    def cycle_body(acc=None):
+        def mark():
+            if acc is None:
+                return None
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(stream)
+            return e
+
+        def close(phase, e0):
+            if acc is not None:
+                acc.append((phase, e0, mark()))
+
+        e = mark()
+        attn.build_perm(q=q0, k=k0)
+        close("perm", e)
+        for st in range(cycle):
+            e = mark()
+            attn.reorder(qs[st], ks[st], v)
+            close("reorder", e)
+            if st == 0:
+                e = mark()
+                attn.build_mask(0)
+                close("mask", e)
+            e = mark()
+            attn.attend()
+            close("attn", e)
+            e = mark()
+            attn.inverse(out)
+            close("inverse", e)
 
     for _ in range(max(args.warmup, 3)):
-        step()
+        cycle_body()
     torch.cuda.synchronize()
     nvalid = np.minimum(64, w.N - 64 * np.arange(w.nb)).astype(np.int64)
     kflops = kept_flops_from_lists(attn.buf.kv_idx.cpu().numpy(), attn.buf.kv_cnt.cpu().numpy(), nvalid, w.d)
     dense_flops = 4.0 * w.d * float(w.N) ** 2 * w.heads * w.B
     density = kflops / dense_flops
 
-    phases = ["perm", "reorder", "mask", "attn", "inverse"]
     times = {p: [] for p in phases}
+    attn_launch = []
     launches0 = svsa.svsa_launch_count()
     _barrier(ws)
     torch.cuda.synchronize()
     with ClockSampler(dev.index) as clk:
         for _ in range(args.steps):
             flush.fill_(1.0)
-            evs = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
-            step(evs)
+            acc = []
+            cycle_body(acc)
             torch.cuda.synchronize()
-            for i, p in enumerate(phases):
-                times[p].append(evs[i].elapsed_time(evs[i + 1]))
+            per = {p: 0.0 for p in phases}
+            for phase, e0, e1 in acc:
+                ms = e0.elapsed_time(e1)
+                per[phase] += ms
+                if phase == "attn":
+                    attn_launch.append(ms)
+            for p in phases:
+                times[p].append(per[p])
     torch.cuda.synchronize()
     _barrier(ws)
     launches = svsa.svsa_launch_count() - launches0
     step_ms_local = sum(sum(times[p]) for p in phases) / args.steps
     step_ms = _max_over_ranks(step_ms_local, ws)
-    attn_ms_local = statistics.mean(times["attn"])
-    attn_ms = _max_over_ranks(attn_ms_local, ws)
+    attn_ms = _max_over_ranks(statistics.mean(attn_launch), ws)      # one attention launch
 
-    # the same step replayed from a CUDA graph (no host launch per kernel),
+    # the same cycle replayed from a CUDA graph (no host launch per kernel),
     # right after the eager steps so that both see the same clocks; reported
     # beside the eager step, whose per-phase events a graph cannot hold
     graph_ms, graph_err = None, None
-    layer = None
     if not args.no_graph:
         try:
-            layer = attn.capture(q, k, v, out, anchor_offset=off, with_order=True)
+            side = torch.cuda.Stream(dev)
+            side.wait_stream(stream)
+            with torch.cuda.stream(side):
+                cycle_body()
+            stream.wait_stream(side)
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                cycle_body()
+            graph_ms = _max_over_ranks(_timed(graph.replay, stream, flush, args.warmup, args.steps), ws)
+            del graph
         except Exception as exc:                       # reported, not fatal: the eager step is the measure
             graph_err = f"capture failed: {exc}"[:200]
-    if layer is not None:
-        gtimes = []
-        for i in range(args.warmup + args.steps):
-            flush.fill_(1.0)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            layer.replay()
-            e1.record(stream)
-            torch.cuda.synchronize()
-            if i >= args.warmup:
-                gtimes.append(e0.elapsed_time(e1))
-        del layer
-        graph_ms = _max_over_ranks(statistics.mean(gtimes), ws)
 
-    # dense denominator: same arithmetic over every key block
-    dtimes = []
-    for i in range(args.warmup + args.steps):
-        flush.fill_(1.0)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        attn.attend_dense()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        if i >= args.warmup:
-            dtimes.append(e0.elapsed_time(e1))
-    dense_ms = _max_over_ranks(statistics.mean(dtimes), ws)
+    # pooling on its own (svsa_pool of Q and K at the rule's group size): one HBM pass each
+    size = w.sub_block if w.select != "structured" else 64
+    pq = torch.empty(w.B, w.heads, w.Npad // size, w.d, dtype=torch.float32, device=dev)
+    pk = torch.empty_like(pq)
 
-    # end to end through the public API: pinned host Q, K, V in, O back to the host,
-    # the copies of one group of heads overlapping the compute of another
-    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    def pool_both():
+        svsa.svsa_pool(attn.buf.qp, pq, attn.shape, size)
+        svsa.svsa_pool(attn.buf.kp, pk, attn.shape, size)
+
+    pool_ms = _max_over_ranks(_timed(pool_both, stream, flush, 3, args.steps), ws)
+    pool_bytes = 2 * (w.B * w.heads * w.Npad * w.d * 2 + w.B * w.heads * (w.Npad // size) * w.d * 4)
+    del pq, pk
+
+    # dense denominator: same arithmetic over every key block (seconds per launch on
+    # the long layers, so at most 3 timed launches there)
+    long_layer = attn_ms >= LONG_STEP_MS / 2
+    dense_ms = _max_over_ranks(_timed(attn.attend_dense, stream, flush, 1 if long_layer else args.warmup,
+                                      min(args.steps, 3) if long_layer else args.steps), ws)
+
+    # end to end through the public API: pinned host Q, K, V of every step of the
+    # cycle in, O of every step back to the host, the copies of one group of
+    # heads overlapping the compute of another
+    hq = [t.cpu().pin_memory() for t in qs]
+    hk = [t.cpu().pin_memory() for t in ks]
+    hv = v.cpu().pin_memory()
     hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    e2e_times = []
-    for i in range(args.warmup + args.steps):
-        flush.fill_(1.0)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        attn.forward_host(hq, hk, hv, hout, anchor_offset=off)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        if i >= args.warmup:
-            e2e_times.append(e0.elapsed_time(e1))
-    e2e_ms = _max_over_ranks(statistics.mean(e2e_times), ws)
-    h2d = 3 * q.numel() * q.element_size()
-    d2h = out.numel() * out.element_size()
+
+    def e2e_cycle():
+        for st in range(cycle):
+            attn.forward_host(hq[st], hk[st], hv, hout, step=0, reuse_mask=st > 0)
+
+    e2e_ms = _max_over_ranks(_timed(e2e_cycle, stream, flush, args.warmup, args.steps), ws)
+    h2d = cycle * 3 * q0.numel() * q0.element_size()
+    d2h = cycle * out.numel() * out.element_size()
+    del hq, hk, hv, hout
 
     peaks, peak_src = _peaks()
     # a kernel inside steps of 100 ms or more runs seconds-long loops under the
@@ -412,15 +501,19 @@ def run_svsa(args):
     sustained = step_ms >= LONG_STEP_MS
     peak = float(peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"])
     attn_tflops = kflops / (attn_ms * 1e-3) / 1e12
-    value = ws * kflops / (step_ms * 1e-3) / 1e12
+    cycle_flops = cycle * kflops
+    value = ws * cycle_flops / (step_ms * 1e-3) / 1e12
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        f, t, desc, threads = _oracle_sample(w, q, k, v, args.cpu_seconds)
+        f, t, desc, threads = _oracle_sample(w, q0, k0, v, args.cpu_seconds)
         cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
+    secondary = None
+    if rank == 0 and ws == 1 and args.secondary and args.secondary != w.name:
+        secondary = _secondary(svsa, args.secondary, dev, stream, flush, peaks, args.steps)
 
     if rank == 0:
-        reorder_bytes = 3 * (w.B * w.heads * (w.N + w.Npad) * w.d * 2)
-        inverse_bytes = w.B * w.heads * (w.N + w.Npad) * w.d * 2
+        reorder_bytes = cycle * 3 * (w.B * w.heads * (w.N + w.Npad) * w.d * 2)
+        inverse_bytes = cycle * w.B * w.heads * (w.N + w.Npad) * w.d * 2
         reorder_ms = statistics.mean(times["reorder"])
         inverse_ms = statistics.mean(times["inverse"])
         line = {
@@ -430,27 +523,38 @@ def run_svsa(args):
             "config": {"workload": w.name, "B": w.B, "heads": w.heads, "d": w.d, "grid": [w.T, w.H, w.W],
                        "N": w.N, "order": w.order, "select": w.select, "keep_frac": w.keep_frac,
                        "tau": w.tau, "sub_block": w.sub_block, "routing": w.routing,
-                       "compensate": w.compensate, "l2": "flushed (512 MiB write) between timed steps",
+                       "compensate": w.compensate, "scorer": w.scorer,
+                       "step": (f"one mask cycle: perm, mask at the first of {cycle} denoising steps, then "
+                                f"reorder + attention + inverse at each of the {cycle} steps (Q, K drift by "
+                                f"sigma={w.sigma} between steps)") if cycle > 1 else
+                               "perm + reorder + mask + attention + inverse",
+                       "l2": "flushed (512 MiB write) between timed steps",
                        "parallelism": f"independent layer per GPU x{ws}"},
             "attn_ms": attn_ms, "attn_tflops": attn_tflops, "attn_frac_of_peak": attn_tflops / peak,
+            "attn_passes": attn.attn_passes,
             "dense_ms": dense_ms, "dense_tflops": dense_flops / (dense_ms * 1e-3) / 1e12,
+            "dense_frac_of_peak": dense_flops / (dense_ms * 1e-3) / 1e12 / peak,
             "speedup_vs_dense": dense_ms / attn_ms, "density": density,
-            "kept_tflop_per_step": kflops / 1e12,
-            "graph": ({"ms_per_step": graph_ms, "value": ws * kflops / (graph_ms * 1e-3) / 1e12}
+            "kept_tflop_per_attention": kflops / 1e12, "kept_tflop_per_step": cycle_flops / 1e12,
+            "graph": ({"ms_per_step": graph_ms, "value": ws * cycle_flops / (graph_ms * 1e-3) / 1e12}
                       if graph_ms is not None else ({"unavailable": graph_err} if graph_err else None)),
             "phase_ms": {p: statistics.mean(times[p]) for p in phases},
             "reorder_gbs": reorder_bytes / (reorder_ms * 1e-3) / 1e9,
             "inverse_gbs": inverse_bytes / (inverse_ms * 1e-3) / 1e9,
+            "pool": {"ms": pool_ms, "gbs": pool_bytes / (pool_ms * 1e-3) / 1e9,
+                     "frac_of_hbm": pool_bytes / (pool_ms * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),
+                     "what": f"svsa_pool of Q and K ({size}-token groups), read bf16 + write fp32 means"},
             "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
                          "frac": attn_tflops / peak, "traffic": _attn_traffic(w.name),
                          "kernel": "svsa attention (kept-block FLOPs / launch time)",
                          "peak_source": f"{peak_src} " + ("bf16_tflops_sustained (step >= 100 ms)" if sustained
                                                            else "bf16_tflops (burst)")},
-            "e2e": {"value": ws * kflops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+            "e2e": {"value": ws * cycle_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
+            "secondary": secondary,
         }
         print(json.dumps(line), flush=True)
     if ws > 1:

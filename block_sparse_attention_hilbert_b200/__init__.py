@@ -19,9 +19,11 @@ LIB_PATH = os.path.join(_PKG, "lib", "libsvsa.so")
 
 ORDER_RASTER, ORDER_HILBERT = 0, 1
 SEL_THRESHOLD, SEL_TOPK, SEL_STRUCTURED = 0, 1, 2
+SCORE_POOLED, SCORE_SICS = 0, 1
 BLOCK = 64
 
-STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: "CUDA", 5: "TIMEOUT"}
+STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: "CUDA", 5: "TIMEOUT", 6: "RANGE",
+          7: "MASK"}
 
 
 class SvsaError(RuntimeError):
@@ -38,14 +40,14 @@ class Shape(ctypes.Structure):
 class MaskParams(ctypes.Structure):
     _fields_ = [("select", ctypes.c_int32), ("tau", ctypes.c_float), ("keep_frac", ctypes.c_float),
                 ("sub_block", ctypes.c_int32), ("win_t", ctypes.c_int32), ("win_rows", ctypes.c_int32),
-                ("n_anchors", ctypes.c_int32), ("anchor_offset", ctypes.c_int32),
-                ("routing", ctypes.c_int32)]
+                ("n_anchors", ctypes.c_int32), ("step", ctypes.c_int32), ("seed", ctypes.c_uint64),
+                ("routing", ctypes.c_int32), ("scorer", ctypes.c_int32)]
 
 
 class Mask(ctypes.Structure):
     _fields_ = [("kv_idx", ctypes.c_void_p), ("kv_cnt", ctypes.c_void_p), ("cap", ctypes.c_int32),
                 ("bits", ctypes.c_void_p), ("kbar", ctypes.c_void_p), ("vbar", ctypes.c_void_p),
-                ("nvalid", ctypes.c_void_p), ("cbar", ctypes.c_void_p)]
+                ("nvalid", ctypes.c_void_p), ("cbar", ctypes.c_void_p), ("check", ctypes.c_int32)]
 
 
 class Schedule(ctypes.Structure):
@@ -65,6 +67,7 @@ _SIGS = {
                                     ctypes.c_void_p]),
     "svsa_reorder_values": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, Shape,
                                            ctypes.c_void_p]),
+    "svsa_pool": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, Shape, ctypes.c_int32, ctypes.c_void_p]),
     "svsa_mask_workspace_bytes": (ctypes.c_size_t, [Shape, ctypes.POINTER(MaskParams)]),
     "svsa_build_mask": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                        ctypes.c_void_p, Shape, ctypes.POINTER(MaskParams),
@@ -94,6 +97,8 @@ _SIGS = {
                                                   ctypes.c_void_p]),
     "svsa_schedule_step": (ctypes.c_int, [ctypes.POINTER(Schedule), ctypes.c_int32, ctypes.POINTER(MaskParams),
                                           ctypes.POINTER(MaskParams), ctypes.POINTER(ctypes.c_int32)]),
+    "svsa_anchor_offset": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                          ctypes.POINTER(ctypes.c_int32)]),
     "svsa_selftest_timeout": (ctypes.c_int, [ctypes.c_int32, ctypes.c_void_p]),
     "svsa_sync_status": (ctypes.c_int, [ctypes.c_void_p]),
     "svsa_last_error": (ctypes.c_char_p, []),
@@ -146,13 +151,22 @@ def shape(B: int, heads: int, T: int, H: int, W: int, d: int) -> Shape:
 
 def mask_params(select: int = SEL_THRESHOLD, tau: float = 0.9, keep_frac: float = 0.25,
                 sub_block: int = 64, win_t: int = 2, win_rows: int = 1, n_anchors: int = 0,
-                anchor_offset: int = 0, routing: bool = False) -> MaskParams:
-    return MaskParams(select, tau, keep_frac, sub_block, win_t, win_rows, n_anchors, anchor_offset,
-                      int(routing))
+                step: int = 0, seed: int = 0, routing: bool = False, scorer: int = SCORE_POOLED) -> MaskParams:
+    return MaskParams(select, tau, keep_frac, sub_block, win_t, win_rows, n_anchors, step,
+                      seed & 0xFFFFFFFFFFFFFFFF, int(routing), scorer)
 
 
-def make_mask(kv_idx, kv_cnt, cap: int, bits=None, kbar=None, vbar=None, nvalid=None, cbar=None) -> Mask:
-    return Mask(_p(kv_idx), _p(kv_cnt), cap, _p(bits), _p(kbar), _p(vbar), _p(nvalid), _p(cbar))
+def make_mask(kv_idx, kv_cnt, cap: int, bits=None, kbar=None, vbar=None, nvalid=None, cbar=None,
+              check: bool = False) -> Mask:
+    return Mask(_p(kv_idx), _p(kv_cnt), cap, _p(bits), _p(kbar), _p(vbar), _p(nvalid), _p(cbar), int(check))
+
+
+def svsa_anchor_offset(seed: int, step: int, nb: int, n_anchors: int) -> int:
+    """The anchor rotation of step `step` for a run seeded `seed` (host-only)."""
+    out = ctypes.c_int32(0)
+    _check(lib().svsa_anchor_offset(seed & 0xFFFFFFFFFFFFFFFF, step, nb, n_anchors, ctypes.byref(out)),
+           "svsa_anchor_offset")
+    return int(out.value)
 
 
 def version() -> str:
@@ -217,6 +231,10 @@ def svsa_reorder(x, xp, perm, s: Shape, stream=None) -> None:
 
 def svsa_reorder_values(v, vp, perm, s: Shape, stream=None) -> None:
     _check(lib().svsa_reorder_values(_p(v), _p(vp), _p(perm), s, _stream(stream)), "svsa_reorder_values")
+
+
+def svsa_pool(xp, out, s: Shape, size: int, stream=None) -> None:
+    _check(lib().svsa_pool(_p(xp), _p(out), s, size, _stream(stream)), "svsa_pool")
 
 
 def svsa_mask_workspace_bytes(s: Shape, p: MaskParams) -> int:

@@ -61,6 +61,15 @@ cudaError_t launch_combine(const float* o_p, const float* lse_p, long long rows,
 cudaError_t attn_tc_error(unsigned int* code, cudaStream_t st);
 cudaError_t launch_selftest_timeout(unsigned long long budget_ns, cudaStream_t st);
 cudaError_t scores_tc_error(unsigned int* code, cudaStream_t st);
+cudaError_t launch_sics(const void* kp, float* coh, float* S, long long BH, long long N, int nb, int d,
+                        cudaStream_t st);
+cudaError_t launch_broadcast(const int32_t* hidx, const int32_t* hcnt, int hcap, long long BH, int nb, int cap,
+                             int32_t* kv_idx, int32_t* kv_cnt, uint32_t* bits, cudaStream_t st);
+cudaError_t launch_check_mask(const int32_t* kv_idx, const int32_t* kv_cnt, long long rows, int cap, int nb,
+                              cudaStream_t st);
+cudaError_t sics_flags(unsigned int* v, cudaStream_t st);
+cudaError_t reorder_flags(unsigned int* v, cudaStream_t st);
+cudaError_t pool_flags(unsigned int* v, cudaStream_t st);
 }  // namespace svsa
 
 using namespace svsa;
@@ -127,7 +136,7 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // Workspace layout of svsa_build_mask.
 struct MaskWs {
-  size_t qsplit, ksplit, S, R, Rm, qbf, L, Mp, Zp, q64, k64, total;
+  size_t qsplit, ksplit, S, R, Rm, qbf, L, Mp, Zp, q64, k64, coh, hidx, hcnt, total;
 };
 
 MaskWs mask_ws_layout(const Dims& g, const svsa_mask_params& p, bool have_kbar) {
@@ -139,6 +148,17 @@ MaskWs mask_ws_layout(const Dims& g, const svsa_mask_params& p, bool have_kbar) 
     w.total = 0;
     return w;
   }
+  if (p.scorer == SVSA_SCORE_SICS) {
+    // per-head coherences, their normalised scores, and one selected list per head
+    w.qsplit = w.ksplit = w.R = w.Rm = w.qbf = w.L = w.Mp = w.Zp = w.q64 = w.k64 = SIZE_MAX;
+    w.coh = take((size_t)g.BH * g.nb * f);
+    w.S = take((size_t)g.BH * g.nb * f);
+    w.hidx = take((size_t)g.BH * g.nb * 4);
+    w.hcnt = take((size_t)g.BH * 4);
+    w.total = off;
+    return w;
+  }
+  w.coh = w.hidx = w.hcnt = SIZE_MAX;
   const int sub = p.sub_block;
   const long long ng = g.Npad / sub;
   (void)have_kbar;
@@ -176,17 +196,56 @@ svsa_status check_params(const svsa_mask_params* p, const Dims& g) {
     return fail(SVSA_ERR_INVALID_ARG, "keep_frac=%g must be >= 0", (double)p->keep_frac);
   if (p->routing && p->select != SVSA_SEL_THRESHOLD)
     return fail(SVSA_ERR_INVALID_ARG, "routing needs select = THRESHOLD (its budget)");
+  if (p->scorer != SVSA_SCORE_POOLED && p->scorer != SVSA_SCORE_SICS)
+    return fail(SVSA_ERR_INVALID_ARG, "scorer=%d unknown", p->scorer);
+  if (p->scorer == SVSA_SCORE_SICS) {
+    if (p->select == SVSA_SEL_STRUCTURED)
+      return fail(SVSA_ERR_INVALID_ARG, "the SICS scorer ranks blocks for THRESHOLD / TOPK, not STRUCTURED");
+    if (p->sub_block != 64 || p->routing)
+      return fail(SVSA_ERR_UNSUPPORTED, "the SICS scorer works on 64-token blocks without routing");
+  }
   if (p->select == SVSA_SEL_STRUCTURED) {
     if (p->win_t < 0 || p->win_rows < 0 || p->n_anchors < 0 || p->n_anchors > g.nb)
       return fail(SVSA_ERR_INVALID_ARG, "structured window/anchors out of range");
-    if (p->n_anchors > 0) {
-      const int stride = std::max(g.nb / p->n_anchors, 1);
-      if (p->anchor_offset < 0 || p->anchor_offset >= stride)
-        return fail(SVSA_ERR_INVALID_ARG, "anchor_offset=%d not in [0, %d)", p->anchor_offset, stride);
-    }
+    if (p->step < 0) return fail(SVSA_ERR_INVALID_ARG, "step=%d must be >= 0", p->step);
   }
   if (g.nb > kMaxBlocks) return fail(SVSA_ERR_UNSUPPORTED, "nb=%d blocks exceeds %d", g.nb, kMaxBlocks);
   return SVSA_OK;
+}
+
+// Philox4x32-10 (J. K. Salmon, M. A. Moraes, R. O. Dror, D. E. Shaw,
+// "Parallel random numbers: as easy as 1, 2, 3", SC'11): ten rounds, each two
+// 32x32 -> 64-bit products of counter words with the round multipliers, the
+// high halves XORed with the other counter words and the key; the key is
+// bumped by the two Weyl increments before every round after the first.
+void philox4x32_10(const uint32_t in[4], uint32_t k0, uint32_t k1, uint32_t out[4]) {
+  uint32_t c0 = in[0], c1 = in[1], c2 = in[2], c3 = in[3];
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+    const uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+    const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0;
+    const uint32_t n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1;
+    c0 = n0;
+    c1 = (uint32_t)p1;
+    c2 = n2;
+    c3 = (uint32_t)p0;
+  }
+  out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+// Rotation of the anchor columns at step `step` (>= 0): the first Philox word
+// of counter (step, 0, 0, 0) under key (seed low, seed high), mod the stride.
+int anchor_rotation(uint64_t seed, int32_t step, int nb, int n_anchors) {
+  if (n_anchors <= 0 || nb <= 0) return 0;
+  const uint32_t stride = (uint32_t)std::max(nb / n_anchors, 1);
+  const uint32_t ctr[4] = {(uint32_t)step, 0u, 0u, 0u};
+  uint32_t out[4];
+  philox4x32_10(ctr, (uint32_t)seed, (uint32_t)(seed >> 32), out);
+  return (int)(out[0] % stride);
 }
 
 int topk_count(float keep_frac, int nb) {
@@ -340,6 +399,19 @@ svsa_status svsa_build_perm_cocluster(const void* q, const void* k, svsa_shape s
   return cuda_status(counted(e, launches), "cocluster launch");
 }
 
+svsa_status svsa_pool(const void* xp, float* out, svsa_shape s, int32_t size, void* stream) {
+  NvtxRange nvtx_("svsa_pool");
+  g_last_error.clear();
+  SVSA_TRY(check_shape(s, true));
+  SVSA_PTR(xp, "xp");
+  SVSA_PTR(out, "out");
+  if (size != 64 && size != 16) return fail(SVSA_ERR_UNSUPPORTED, "size=%d (supported: 64, 16)", size);
+  const Dims g = make_dims(s.B, s.heads, s.T, s.H, s.W, s.d);
+  return cuda_status(counted(launch_pool(xp, out, nullptr, nullptr, nullptr, g.BH, g.N, g.Npad, g.d, size,
+                                         (cudaStream_t)stream), 1),
+                     "pool launch");
+}
+
 size_t svsa_mask_workspace_bytes(svsa_shape s, const svsa_mask_params* p) {
   if (p == nullptr || s.T < 1 || s.H < 1 || s.W < 1 || s.B < 1 || s.heads < 1) return 0;
   if (p->select != SVSA_SEL_STRUCTURED && p->sub_block != 64 && p->sub_block != 16) return 0;
@@ -368,7 +440,7 @@ svsa_status svsa_build_mask(const void* qp, const void* kp, const void* vp, cons
   if (m->cap < need_cap) return fail(SVSA_ERR_INVALID_ARG, "mask.cap=%d < %d", m->cap, need_cap);
   const bool structured = p->select == SVSA_SEL_STRUCTURED;
   if (!structured) {
-    SVSA_PTR(qp, "qp");
+    if (p->scorer != SVSA_SCORE_SICS) SVSA_PTR(qp, "qp");
     SVSA_PTR(kp, "kp");
   }
   if (structured) SVSA_PTR(perm, "perm");
@@ -393,7 +465,7 @@ svsa_status svsa_build_mask(const void* qp, const void* kp, const void* vp, cons
 
   // block-level outputs the caller asked for (compensation / routing inputs)
   if (nvalid != nullptr) SVSA_TRY(cuda_status(counted(launch_nvalid(nvalid, g.N, g.nb, st), 1), "nvalid"));
-  if (m->kbar != nullptr && (structured || p->sub_block != kBlock))
+  if (m->kbar != nullptr && (structured || p->sub_block != kBlock || p->scorer == SVSA_SCORE_SICS))
     SVSA_TRY(cuda_status(counted(launch_pool(kp, m->kbar, nullptr, nullptr, nullptr, g.BH, g.N, g.Npad, g.d, kBlock, st), 1),
                          "pool K"));
   if (m->vbar != nullptr)
@@ -402,10 +474,25 @@ svsa_status svsa_build_mask(const void* qp, const void* kp, const void* vp, cons
 
   if (structured) {
     const int R = p->win_rows * ((kBlock + g.W - 1) / g.W);
-    return cuda_status(counted(launch_structured(perm, rows, g.nb, g.H, g.W, p->win_t, R, p->n_anchors,
-                                                 p->anchor_offset, m->cap, m->kv_idx, m->kv_cnt, m->bits,
-                                                 st), 1),
+    const int offset = anchor_rotation(p->seed, p->step, g.nb, p->n_anchors);
+    return cuda_status(counted(launch_structured(perm, rows, g.nb, g.H, g.W, p->win_t, R, p->n_anchors, offset,
+                                                 m->cap, m->kv_idx, m->kv_cnt, m->bits, st), 1),
                        "structured mask");
+  }
+
+  if (p->scorer == SVSA_SCORE_SICS) {
+    // per-head coherence scores -> one selected list per head -> every row of the head
+    float* coh = at(w.coh);
+    float* S1 = at(w.S);
+    int32_t* hidx = reinterpret_cast<int32_t*>(base + w.hidx);
+    int32_t* hcnt = reinterpret_cast<int32_t*>(base + w.hcnt);
+    SVSA_TRY(cuda_status(counted(launch_sics(kp, coh, S1, g.BH, g.N, g.nb, g.d, st), 2), "SICS scores"));
+    SVSA_TRY(cuda_status(counted(launch_select(S1, nullptr, g.BH, g.nb, p->select == SVSA_SEL_TOPK ? 1 : 0, p->tau,
+                                               k, g.nb, hidx, hcnt, nullptr, st), 1),
+                         "SICS select"));
+    return cuda_status(counted(launch_broadcast(hidx, hcnt, g.nb, g.BH, g.nb, m->cap, m->kv_idx, m->kv_cnt, m->bits,
+                                                st), 1),
+                       "SICS lists");
   }
 
   const int sub = p->sub_block;
@@ -473,6 +560,10 @@ svsa_status svsa_attn_fwd(const void* qp, const void* kp, const void* vp, const 
     SVSA_PTR(m->cbar, "mask.cbar (compensation)");
   }
   if (op == qp || op == kp || op == vp) return fail(SVSA_ERR_INVALID_ARG, "op must not alias an input");
+  if (m->check)
+    SVSA_TRY(cuda_status(counted(launch_check_mask(m->kv_idx, m->kv_cnt, g.BH * g.nb, m->cap, g.nb,
+                                                   (cudaStream_t)stream), 1),
+                         "mask check"));
   if (compensate)
     SVSA_TRY(cuda_status(counted(launch_centroid16(m->kbar, m->vbar, m->cbar, g.BH * g.nb, g.d,
                                                    (cudaStream_t)stream), 1),
@@ -545,6 +636,8 @@ svsa_status svsa_attn_fwd_split(const void* qp, const void* kp, const void* vp, 
   float* lse_p = reinterpret_cast<float*>(base + w.lse);
   const long long rows = g.BH * g.nb;
   const int R = (g.nb + passes - 1) / passes;
+  if (m->check)
+    SVSA_TRY(cuda_status(counted(launch_check_mask(m->kv_idx, m->kv_cnt, rows, m->cap, g.nb, st), 1), "mask check"));
   if (compensate)
     SVSA_TRY(cuda_status(counted(launch_centroid16(m->kbar, m->vbar, m->cbar, g.BH * g.nb, g.d, st), 1),
                          "centroid copies"));
@@ -612,6 +705,16 @@ svsa_status svsa_schedule_step(const svsa_schedule* sch, int32_t step, const svs
   return SVSA_OK;
 }
 
+svsa_status svsa_anchor_offset(uint64_t seed, int32_t step, int32_t nb, int32_t n_anchors, int32_t* offset) {
+  g_last_error.clear();
+  if (offset == nullptr) return fail(SVSA_ERR_INVALID_ARG, "offset is NULL");
+  if (step < 0) return fail(SVSA_ERR_INVALID_ARG, "step=%d must be >= 0", step);
+  if (nb < 1 || n_anchors < 0 || n_anchors > nb)
+    return fail(SVSA_ERR_INVALID_ARG, "nb=%d, n_anchors=%d: need nb >= 1 and n_anchors in [0, nb]", nb, n_anchors);
+  *offset = anchor_rotation(seed, step, nb, n_anchors);
+  return SVSA_OK;
+}
+
 svsa_status svsa_selftest_timeout(int32_t wait_us, void* stream) {
   NvtxRange nvtx_("svsa_selftest_timeout");
   g_last_error.clear();
@@ -642,8 +745,22 @@ svsa_status svsa_sync_status(void* stream) {
       first_name = names[i];
     }
   }
+  // status bits of the data checks (reading clears them)
+  unsigned int fl[3] = {0u, 0u, 0u};
+  cudaError_t (*flag_readers[3])(unsigned int*, cudaStream_t) = {reorder_flags, pool_flags, sics_flags};
+  for (int i = 0; i < 3; ++i) {
+    e = flag_readers[i](&fl[i], (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_status(e, "reading a status word");
+  }
+  const unsigned int bits = fl[0] | fl[1] | fl[2];
   if (first_name != nullptr)
     return fail(SVSA_ERR_TIMEOUT, "%s kernel: a bounded wait gave up (site %u)", first_name, first_code);
+  if (bits & kFlagMask)
+    return fail(SVSA_ERR_MASK, "a mask list checked before the attention was malformed "
+                               "(kv_cnt outside [0, cap], an index outside [0, nb) or not strictly ascending)");
+  if (bits & (kFlagRangeValue | kFlagRangeMean))
+    return fail(SVSA_ERR_RANGE, "%s beyond the fp16 range (+-65504) or not finite; the result saturated",
+                (bits & kFlagRangeValue) ? "a value given to svsa_reorder_values" : "a block mean of the scores");
   return SVSA_OK;
 }
 

@@ -49,4 +49,26 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
+// Status bits that kernels OR into a word of their translation unit (each
+// unit that raises one keeps a static word and a reader): bit 0 = a value
+// beyond the fp16 range in a bf16 -> fp16 conversion, bit 1 = a block mean
+// beyond the fp16 range in the scores' split, bit 2 = a malformed mask list.
+constexpr unsigned int kFlagRangeValue = 1u, kFlagRangeMean = 2u, kFlagMask = 4u;
+
+// Read a status word of the calling translation unit and clear it.
+template <typename Word>
+inline cudaError_t read_and_clear_flags(const Word& word, unsigned int* v, cudaStream_t st) {
+  unsigned int zero = 0u;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(v, word, sizeof(unsigned int), 0, cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return e;
+  e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return e;
+  if (*v != 0u) {
+    e = cudaMemcpyToSymbolAsync(word, &zero, sizeof(unsigned int), 0, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return e;
+    e = cudaStreamSynchronize(st);
+  }
+  return e;
+}
+
 }  // namespace svsa

@@ -10,8 +10,6 @@
 // The sort of the N valid cells by curve index is a rank by bitmap: one bit
 // per cube cell, a per-word prefix count and a per-chunk prefix count give
 // each cell its rank with no comparison sort, deterministically.
-#include <mutex>
-
 #include "common.cuh"
 
 namespace svsa {
@@ -218,27 +216,17 @@ static __device__ __align__(256) unsigned char g_perm_scratch[kNoAllocScratchByt
 int perm_noalloc_max_bits() { return kNoAllocMaxBits; }
 size_t perm_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
 
-namespace {
-std::mutex g_scratch_mu;
-void* g_scratch_addr[128] = {};   // per device ordinal, resolved once
-}  // namespace
-
-// Device address of g_perm_scratch on the current device.  The first call on
-// a device resolves it (cudaGetSymbolAddress, with that device current); later
-// calls reuse the cached value.
+// Device address of g_perm_scratch in the current context.  It is looked up
+// on every call (cudaGetSymbolAddress, a host-side query once the module is
+// loaded) rather than cached: a cached address would go stale if the
+// device's primary context were reset and the module loaded again.  The
+// first call on a device loads the module, so make it before any stream
+// capture.
 cudaError_t perm_noalloc_scratch(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_perm_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_perm_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return cudaSuccess;
 }
 

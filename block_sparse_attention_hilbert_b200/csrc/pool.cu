@@ -23,6 +23,10 @@ namespace svsa {
 
 constexpr int kPoolThreads = 256;
 
+// Status bits of this translation unit (kFlagRangeMean: a mean that the fp16
+// split of the scores saturated, or a non-finite one).
+static __device__ unsigned int g_pool_flags;
+
 __device__ __forceinline__ float2 pair_to_float2(const __nv_bfloat162& v) { return __bfloat1622float2(v); }
 __device__ __forceinline__ float2 pair_to_float2(const __half2& v) { return __half22float2(v); }
 
@@ -86,6 +90,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(
     const long long row = bh * (Npad / SIZE) + gidx;
     if (out != nullptr) out[row * D + c] = mean;
     if (split != nullptr) {
+      if (!(fabsf(mean) <= 65504.f)) atomicOr(&g_pool_flags, kFlagRangeMean);
       const __half hi = __float2half_rn(fminf(fmaxf(mean, -65504.f), 65504.f));
       split[row * 2 * D + c] = hi;
       split[row * 2 * D + D + c] = __float2half_rn(fminf(fmaxf(mean - __half2float(hi), -65504.f), 65504.f));
@@ -165,5 +170,7 @@ cudaError_t launch_centroid16(const float* kbar, const float* vbar, void* cbar, 
                                             rows, d / 4);
   return cudaGetLastError();
 }
+
+cudaError_t pool_flags(unsigned int* v, cudaStream_t st) { return read_and_clear_flags(g_pool_flags, v, st); }
 
 }  // namespace svsa

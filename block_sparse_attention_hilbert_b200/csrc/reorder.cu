@@ -57,6 +57,21 @@ __global__ void __launch_bounds__(kGatherThreads) gather_rows_kernel(
   }
 }
 
+// Status bits of this translation unit (kFlagRangeValue: a value given to the
+// fp16 gather lies beyond the fp16 range or is not finite).
+static __device__ unsigned int g_reorder_flags;
+
+// True when one of the 8 bf16 values of a chunk is beyond fp16's range or
+// not finite: |x| >= 65536 (the bf16 value after 65280 is 65536) is an
+// exponent field >= 143, i.e. magnitude bits > 0x477F.
+__device__ __forceinline__ bool bf16x8_out_of_f16(uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  bool bad = false;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) bad |= (w[e] & 0x7FFFu) > 0x477Fu || ((w[e] >> 16) & 0x7FFFu) > 0x477Fu;
+  return bad;
+}
+
 // bf16 -> fp16 conversion of one 16-byte chunk (8 values), saturating at
 // +-65504; exact for every bf16 value in fp16's normal range.
 __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
@@ -94,11 +109,14 @@ __global__ void __launch_bounds__(kGatherThreads) gather_rows_f16_kernel(
         if (srow >= 0) v[u] = ld_stream(s_base + (long long)srow * CPR + (c % CPR));
       }
     }
+    bool bad = false;
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const long long c = base + u * kGatherThreads + threadIdx.x;
       if (c < total) d_base[c] = bf16x8_to_f16x8(v[u]);
+      bad |= bf16x8_out_of_f16(v[u]);          // (zero chunks never flag)
     }
+    if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(&g_reorder_flags, kFlagRangeValue);
   }
 }
 
@@ -135,5 +153,7 @@ cudaError_t launch_gather_rows(const void* src, void* dst, const int32_t* map, l
     return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
+
+cudaError_t reorder_flags(unsigned int* v, cudaStream_t st) { return read_and_clear_flags(g_reorder_flags, v, st); }
 
 }  // namespace svsa

@@ -21,7 +21,7 @@ import math
 
 import torch
 
-from . import (ORDER_HILBERT, ORDER_RASTER, SEL_STRUCTURED, SEL_THRESHOLD, SEL_TOPK, BLOCK,
+from . import (ORDER_HILBERT, ORDER_RASTER, SEL_STRUCTURED, SEL_THRESHOLD, SEL_TOPK, SCORE_POOLED, SCORE_SICS, BLOCK,
                make_mask, mask_params, schedule as make_schedule, shape, svsa_attn_dense_fwd, svsa_attn_fwd,
                svsa_build_mask, svsa_build_perm, svsa_build_perm_cocluster, svsa_cocluster_workspace_bytes,
                svsa_inverse_reorder, svsa_inverse_reorder_heads, svsa_mask_workspace_bytes,
@@ -31,6 +31,7 @@ from . import (ORDER_HILBERT, ORDER_RASTER, SEL_STRUCTURED, SEL_THRESHOLD, SEL_T
 
 _ORDERS = {"raster": ORDER_RASTER, "hilbert": ORDER_HILBERT}
 _SELECTS = {"threshold": SEL_THRESHOLD, "topk": SEL_TOPK, "structured": SEL_STRUCTURED}
+_SCORERS = {"pooled": SCORE_POOLED, "sics": SCORE_SICS}
 
 
 class LayerBuffers:
@@ -96,7 +97,7 @@ class SparseVideoAttention:
     def __init__(self, B, heads, T, H, W, d, *, order="hilbert", select="threshold", tau=0.9,
                  keep_frac=0.25, sub_block=64, win_t=2, win_rows=1, n_anchors=0, routing=False,
                  compensate=False, keep_bits=False, schedule=None, cluster_rounds=3, attn_passes=None,
-                 device="cuda"):
+                 seed=0, scorer="pooled", check_mask=False, device="cuda"):
         """order: "raster", "hilbert" or "cocluster" (a per-head semantic order from
         bidirectional query-key co-clustering, built from the first inputs and
         kept until `rebuild_order()`).  schedule: optional (n_steps, dense_steps,
@@ -105,7 +106,12 @@ class SparseVideoAttention:
         default 1 for the structured rule (its windows keep the key blocks of
         neighbouring query blocks close together, so they share L2 already)
         and while a head's reordered K and V (Npad * d * 4 bytes) fit in 48 MB
-        of L2, else enough passes for at most 32 MB each (at most 8)."""
+        of L2, else enough passes for at most 32 MB each (at most 8).
+        seed: the run's seed of the structured rule's anchor rotation (the
+        step index of each call picks the rotation).  scorer: "pooled" (block
+        scores) or "sics" (per-head block coherence).  check_mask: validate
+        the lists before every attention call (svsa_sync_status reports a
+        malformed one)."""
         self.B, self.heads, self.T, self.H, self.W, self.d = B, heads, T, H, W, d
         self.N = T * H * W
         self.nb = -(-self.N // BLOCK)
@@ -119,8 +125,8 @@ class SparseVideoAttention:
         self.compensate = bool(compensate)
         self.routing = bool(routing)
         self.shape = shape(B, heads, T, H, W, d)
-        self.params = mask_params(self.select, tau, keep_frac, sub_block, win_t, win_rows, n_anchors, 0,
-                                  routing)
+        self.params = mask_params(self.select, tau, keep_frac, sub_block, win_t, win_rows, n_anchors, 0, seed,
+                                  routing, _SCORERS[scorer])
         k = max(1, min(self.nb, math.ceil(float(torch.tensor(keep_frac, dtype=torch.float32)) * self.nb)))
         self.schedule = make_schedule(*schedule) if schedule is not None else None
         # a scheduled top-k rule reaches keep_frac = 1 on its dense steps
@@ -130,6 +136,7 @@ class SparseVideoAttention:
                                 perm_ws_bytes=svsa_perm_workspace_bytes(self.shape, self.order),
                                 device=device, compensate=self.compensate)
         self._mask = self.buf.mask()
+        self._mask.check = int(bool(check_mask))
         if attn_passes is None:
             attn_passes = default_attn_passes(self.select, self.Npad, d)
         self.attn_passes = int(attn_passes)
@@ -176,9 +183,11 @@ class SparseVideoAttention:
         svsa_reorder(k, b.kp, b.perm, self.shape, stream)
         svsa_reorder_values(v, b.vp, b.perm, self.shape, stream)
 
-    def build_mask(self, anchor_offset: int = 0, stream=None):
+    def build_mask(self, step: int = 0, stream=None):
+        """The block mask for denoising step `step` (the structured rule's
+        anchors rotate with it; the other rules do not depend on it)."""
         b = self.buf
-        self.params.anchor_offset = int(anchor_offset)
+        self.params.step = int(step)
         svsa_build_mask(b.qp, b.kp, b.vp, None if self.cocluster else b.perm, self.shape, self.params, self._mask,
                         b.ws, b.ws.numel(), stream)
         self.mask_ready = True
@@ -202,7 +211,7 @@ class SparseVideoAttention:
             svsa_inverse_reorder(self.buf.op, out, self.buf.iperm, self.shape, stream)
 
     # ---- one denoising step under the schedule ----------------------------
-    def step(self, q, k, v, step: int, *, out=None, anchor_offset: int = 0, stream=None):
+    def step(self, q, k, v, step: int, *, out=None, stream=None):
         """The layer at denoising step `step` of the schedule: the step's rule
         parameter, and a new mask only on the schedule's rebuild steps (the
         others reuse the last mask).  Returns (out, rebuilt)."""
@@ -216,7 +225,7 @@ class SparseVideoAttention:
         build = rebuild or not self.mask_ready
         self.reorder(q, k, v, stream)
         if build:
-            self.build_mask(anchor_offset, stream)
+            self.build_mask(step, stream)
         self.attend(stream=stream)
         self.inverse(out, stream)
         return out, build
@@ -231,10 +240,10 @@ class SparseVideoAttention:
         sh = shape(1, r1 - r0, self.T, self.H, self.W, self.d)
         m = make_mask(self._rows(b.kv_idx, r0, r1), self._rows(b.kv_cnt, r0, r1), b.cap,
                       self._rows(b.bits, r0, r1), self._rows(b.kbar, r0, r1), self._rows(b.vbar, r0, r1),
-                      b.nvalid, self._rows(b.cbar, r0, r1))
+                      b.nvalid, self._rows(b.cbar, r0, r1), check=bool(self._mask.check))
         return sh, m
 
-    def forward_host(self, q, k, v, out, *, anchor_offset: int = 0, reuse_mask: bool = False, groups: int = 12):
+    def forward_host(self, q, k, v, out, *, step: int = 0, reuse_mask: bool = False, groups: int = 12):
         """q, k, v, out: pinned host bf16 [B, heads, N, d] (raster order).  The rows
         are processed in `groups` groups.  Every group's input copies are queued
         first, on one stream, each group ending in an event, so the link stays
@@ -258,7 +267,7 @@ class SparseVideoAttention:
             self.build_perm()
         build = not (reuse_mask and self.mask_ready)
         if build:
-            self.params.anchor_offset = int(anchor_offset)
+            self.params.step = int(step)
         # group bounds keep every per-row mask slice 16-byte aligned (the ABI's
         # pointer rule): rows of nb int32 counts must start at a multiple of 4 words
         unit = 4 // math.gcd(self.nb, 4)
@@ -312,12 +321,12 @@ class SparseVideoAttention:
 
     # ---- whole layer ----------------------------------------------------
     # ---- the layer as one CUDA graph ---------------------------------------
-    def capture(self, q, k, v, out, *, anchor_offset: int = 0, with_order: bool = False) -> "CapturedLayer":
+    def capture(self, q, k, v, out, *, step: int = 0, with_order: bool = False) -> "CapturedLayer":
         """Capture one layer call on these device buffers (reorder, block mask,
         attention, inverse reorder; the token order too with with_order) into
         a CUDA graph.  replay() re-runs it on whatever q, k and v then hold and
         writes `out`, without a host launch per kernel.  The buffers, the
-        shape and the mask parameters (anchor_offset included) are fixed at
+        shape and the mask parameters (the step index included) are fixed at
         capture."""
         if self.cocluster and not with_order and not self._perm_ready:
             raise ValueError("build the co-clustering order first, or capture it with with_order=True")
@@ -326,7 +335,7 @@ class SparseVideoAttention:
             if with_order or not self._perm_ready:
                 self.build_perm(q=q, k=k)
             self.reorder(q, k, v)
-            self.build_mask(anchor_offset)
+            self.build_mask(step)
             self.attend()
             self.inverse(out)
 
@@ -341,12 +350,12 @@ class SparseVideoAttention:
             body()
         return CapturedLayer(graph)
 
-    def __call__(self, q, k, v, *, out=None, anchor_offset: int = 0, reuse_mask: bool = False, stream=None):
+    def __call__(self, q, k, v, *, out=None, step: int = 0, reuse_mask: bool = False, stream=None):
         if out is None:
             out = torch.empty_like(q)
         self.reorder(q, k, v, stream)
         if not (reuse_mask and self.mask_ready):
-            self.build_mask(anchor_offset, stream)
+            self.build_mask(step, stream)
         self.attend(stream=stream)
         self.inverse(out, stream)
         return out

@@ -60,7 +60,14 @@ typedef enum {
   SVSA_ERR_UNSUPPORTED = 2,   /* valid request outside the supported range */
   SVSA_ERR_WORKSPACE = 3,     /* workspace smaller than the *_workspace_bytes query */
   SVSA_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed */
-  SVSA_ERR_TIMEOUT = 5        /* a bounded device-side wait gave up (svsa_sync_status) */
+  SVSA_ERR_TIMEOUT = 5,       /* a bounded device-side wait gave up (svsa_sync_status) */
+  SVSA_ERR_RANGE = 6,         /* an input left the range the fp16 paths hold: a value
+                                 given to svsa_reorder_values, or a block / sub-block mean
+                                 of the scores, beyond +-65504 or not finite; the result
+                                 saturated (svsa_sync_status) */
+  SVSA_ERR_MASK = 7           /* svsa_attn_fwd with mask.check set found a malformed list:
+                                 kv_cnt outside [0, cap], an index outside [0, nb) or a
+                                 row not strictly ascending (svsa_sync_status) */
 } svsa_status;
 
 typedef enum { SVSA_ORDER_RASTER = 0, SVSA_ORDER_HILBERT = 1 } svsa_order;
@@ -70,6 +77,13 @@ typedef enum {
   SVSA_SEL_TOPK = 1,          /* k = ceil(keep_frac * nb) highest scores */
   SVSA_SEL_STRUCTURED = 2     /* temporal/spatial window OR rotating anchors */
 } svsa_select;
+
+/* What the THRESHOLD / TOPK rules rank. */
+typedef enum {
+  SVSA_SCORE_POOLED = 0,      /* pooled block scores P_IJ (per query block) */
+  SVSA_SCORE_SICS = 1         /* block coherence from the sum of intra-block cosine
+                                 similarities of the keys (per head; see svsa_build_mask) */
+} svsa_scorer;
 
 /* One attention layer: batch, heads, latent grid (frames T, rows H, columns W)
  * and head dimension d.  N = T*H*W tokens. */
@@ -87,12 +101,14 @@ typedef struct {
   int32_t win_t;          /* STRUCTURED: keep |t_I - t_J| <= win_t (frames) */
   int32_t win_rows;       /* STRUCTURED: or |h_I - h_J| <= win_rows * ceil(64 / W) */
   int32_t n_anchors;      /* STRUCTURED: anchor key-block columns kept for all rows */
-  int32_t anchor_offset;  /* STRUCTURED: this step's rotation, in [0, nb / n_anchors);
-                             anchors are (anchor_offset + m * floor(nb / n_anchors)) mod nb */
+  int32_t step;           /* STRUCTURED: denoising step index s >= 0; the anchors
+                             rotate with it (see svsa_anchor_offset) */
+  uint64_t seed;          /* STRUCTURED: seed of the run's anchor rotation */
   int32_t routing;        /* THRESHOLD only: 1 = keep, per row, as many blocks as the
                              threshold rule would, chosen by largest estimated
                              compensation error per token (SVG-EAR 2.B); needs vp,
                              mask.kbar, mask.vbar and mask.nvalid */
+  int32_t scorer;         /* THRESHOLD / TOPK: svsa_scorer (0 = pooled scores) */
 } svsa_mask_params;
 
 /* Block mask, written by svsa_build_mask and read by svsa_attn_fwd.  All
@@ -113,6 +129,12 @@ typedef struct {
                              svsa_attn_fwd(compensate = 1), which first writes each
                              block's kbar (bf16, first d) and vbar (fp16, last d)
                              there; 16-byte aligned; not read by svsa_build_mask */
+  int32_t check;          /* svsa_attn_fwd only: nonzero = first validate every list
+                             (kv_cnt in [0, cap], indices in [0, nb), strictly
+                             ascending) in a kernel of its own and record a malformed
+                             one for svsa_sync_status (SVSA_ERR_MASK).  The attention
+                             still runs, and clamps counts and indices to the tensors,
+                             so a bad list gives a wrong output but no stray access. */
 } svsa_mask;
 
 /* ---- step 1: token order ------------------------------------------------ */
@@ -147,9 +169,10 @@ svsa_status svsa_build_perm(svsa_shape s, int32_t order, int32_t* perm, int32_t*
  *     process exits).  Larger grids return SVSA_ERR_UNSUPPORTED with a
  *     message; use svsa_build_perm with a workspace for them.  Raster order
  *     needs no scratch and has no limit.
- *   - The first call on a device looks up the array's device address once
- *     (with that device current); make that first call before any stream
- *     capture.
+ *   - Every call looks up the array's device address in the current
+ *     context (a host-side query, nothing is cached across contexts); the
+ *     first call on a device also loads the library's device code, so make
+ *     that first call before any stream capture.
  *   - Every call shares the one array: two calls whose kernels overlap on
  *     the GPU (different streams, no ordering between them) race and may both
  *     produce wrong permutations.  Order them on one stream or with events.
@@ -175,6 +198,17 @@ svsa_status svsa_reorder_values(const void* v, void* vp, const int32_t* perm, sv
 
 /* ---- step 2: block mask ------------------------------------------------- */
 
+/* Block (or sub-block) means of a reordered tensor -- the pooling that
+ * svsa_build_mask starts with, as a call of its own ("DFSAttn", trick 2: a
+ * block is represented by its average; "SVG-EAR" 2.A: a centroid is the mean
+ * of its tokens):
+ *   out[b, h, g, :] = mean of the valid rows (position < N) of group g, the
+ *   rows [g * size, (g + 1) * size); 0 for a group with no valid row.
+ * xp: bf16 [B, heads, Npad, d] (from svsa_reorder); out: fp32
+ * [B, heads, Npad / size, d]; size in {64, 16}.  The sums are fp32 in a fixed
+ * order, so the result is deterministic. */
+svsa_status svsa_pool(const void* xp, float* out, svsa_shape s, int32_t size, void* stream);
+
 /* Workspace bytes svsa_build_mask needs for this shape and rule. */
 size_t svsa_mask_workspace_bytes(svsa_shape s, const svsa_mask_params* p);
 
@@ -188,7 +222,22 @@ size_t svsa_mask_workspace_bytes(svsa_shape s, const svsa_mask_params* p);
  *   whose fp64 cumulative sum reaches tau, or the first k.
  * STRUCTURED: keep (I, J) iff |t_I - t_J| <= win_t or |h_I - h_J| <=
  *   win_rows * ceil(64 / W) or J is an anchor column, where (t, h) is the
- *   coordinate of the block's first token (perm required).
+ *   coordinate of the block's first token (perm required).  The anchor
+ *   columns of step p->step are (o + m * floor(nb / n_anchors)) mod nb,
+ *   m < n_anchors, with o = svsa_anchor_offset(p->seed, p->step, ...): the
+ *   anchors rotate with the step index ("LVSA", abstract: rotating global
+ *   anchors remove the fixed-grid bias).
+ * scorer = SVSA_SCORE_SICS ("SPADE: An Input-Adaptive Sparse Attention Engine
+ *   for Fast Video Diffusion Models Inference", part 2: the sum of intra-block
+ *   cosine similarities decides, per head and per step, which blocks attention
+ *   focuses on; a block whose tokens agree is kept, one whose tokens disagree
+ *   is skipped).  Reading: for key block J of a head, with n_J valid keys,
+ *   SICS_J = sum_{i, j in J} cos(k_i, k_j) (a zero key has cosine 0 with
+ *   everything), the coherence c_J = SICS_J / n_J^2 in [0, 1], and the score
+ *   S_J = c_J / sum_J' c_J' is the same for every query block of the head;
+ *   THRESHOLD / TOPK then keep blocks as above, so every query block of a
+ *   head gets the same list.  No pooled scores are computed (qp unused);
+ *   sub_block and routing must be 64 and 0.
  * routing = 1: with the threshold rule's count m_I as the budget, keep the
  *   m_I blocks with the largest r_IJ = e_IJ / Z_I * 64 / n_J, where e_IJ is the
  *   l2 norm of the change of the un-normalised output of the proxy query
@@ -201,6 +250,17 @@ size_t svsa_mask_workspace_bytes(svsa_shape s, const svsa_mask_params* p);
 svsa_status svsa_build_mask(const void* qp, const void* kp, const void* vp, const int32_t* perm,
                             svsa_shape s, const svsa_mask_params* p, const svsa_mask* m,
                             void* ws, size_t ws_bytes, void* stream);
+
+/* The rotation of the anchor columns at denoising step `step` of a run seeded
+ * `seed`: with stride = max(floor(nb / n_anchors), 1),
+ *   *offset = Philox4x32-10(counter = (step, 0, 0, 0),
+ *                           key = (seed mod 2^32, floor(seed / 2^32)))[0] mod stride,
+ * the first output word of the counter-based generator of J. K. Salmon et al.,
+ * "Parallel random numbers: as easy as 1, 2, 3" (SC'11); 0 when n_anchors is
+ * 0.  The same (seed, step) always gives the same anchors, and consecutive
+ * steps give independent rotations ("LVSA", abstract).  Host-only, no device
+ * work.  step >= 0, nb >= 1, n_anchors in [0, nb]. */
+svsa_status svsa_anchor_offset(uint64_t seed, int32_t step, int32_t nb, int32_t n_anchors, int32_t* offset);
 
 /* ---- step 3: attention -------------------------------------------------- */
 

@@ -23,7 +23,11 @@ Sources (page title, section):
     (SVOO) -- technical summary 2.A (density needed to cover a cumulative
     attention mass such as 95%).
   * "LVSA: Training-Free Sparse Attention for Long Video Diffusion" --
-    abstract (structured window pattern with rotating global anchors).
+    abstract (structured window pattern with rotating global anchors; the
+    rotation by step index is a Philox4x32-10 draw, Salmon et al., SC'11).
+  * "SPADE: An Input-Adaptive Sparse Attention Engine for Fast Video
+    Diffusion Models Inference", part 2 -- the SICS coherence scorer (sum of
+    intra-block cosine similarities).
   * DFSAttn trick 3 and SVOO 2.B -- a step schedule: dense early steps, a
     sparser rule as the video clears, the mask rebuilt every few steps
     (`schedule.py`).
@@ -38,8 +42,8 @@ docstring.  At the time of writing every function is pinned.
 from .order import (hilbert_key_3d, perm_raster, perm_hilbert, build_perm, reorder, inverse_reorder,
                     locality_stats)
 from .mask import (pool, block_scores, subblock_scores, select_threshold, select_topk, topk_count,
-                   select_rows, structured_mask, anchor_blocks, route_ratios, select_routing,
-                   mask_from_rows)
+                   select_rows, structured_mask, anchor_blocks, anchor_offset, philox4x32_10, route_ratios,
+                   select_routing, mask_from_rows, sics_coherence, sics_scores)
 from .attention import (masked_attention, compensated_attention, dense_attention,
                         online_block_attention, kept_flops)
 from .schedule import step_param, rebuilds, mask_steps
@@ -48,8 +52,9 @@ from .cluster import cocluster, perm_from_clusters, initial_centroids
 __all__ = [
     "hilbert_key_3d", "perm_raster", "perm_hilbert", "build_perm", "reorder", "inverse_reorder",
     "locality_stats", "pool", "block_scores", "subblock_scores", "select_threshold", "select_topk",
-    "topk_count", "select_rows", "structured_mask", "anchor_blocks", "route_ratios",
+    "topk_count", "select_rows", "structured_mask", "anchor_blocks", "anchor_offset", "philox4x32_10",
+    "route_ratios",
     "select_routing", "mask_from_rows", "masked_attention", "compensated_attention",
     "dense_attention", "online_block_attention", "kept_flops", "step_param", "rebuilds", "mask_steps",
-    "cocluster", "perm_from_clusters", "initial_centroids",
+    "cocluster", "perm_from_clusters", "initial_centroids", "sics_coherence", "sics_scores",
 ]

@@ -51,25 +51,33 @@ def _means(x: np.ndarray, assign: np.ndarray, C: int, fallback: np.ndarray) -> n
 
 
 def _assign(x: np.ndarray, cent: np.ndarray):
-    """argmax_j x . c_j (first index on ties) and the top-2 gap.  The products
-    of a bf16 and a float32 value are exact in float64; rows whose best
-    candidates lie within 1e-9 of each other (relative) are re-decided on the
-    correctly rounded exact sums (math.fsum), so that equal centroids always
-    give equal affinities."""
+    """argmax_j x . c_j (first index on ties) and the top-2 gap, decided on the
+    exact affinities.  The products of a bf16 and a float32 value are exact in
+    float64, so only the summation rounds: whatever its order, an fp64 dot
+    product of length d is within gamma_d * sum_i |x_i c_i| of the exact value
+    (gamma_d = d u / (1 - d u), u = 2^-53).  Every centroid whose interval
+    reaches the best one's is a candidate; rows with two or more candidates
+    are re-decided on the correctly rounded exact sums (math.fsum), so that
+    equal centroids always give equal affinities and a cancellation cannot
+    flip the argmax."""
     c64 = cent.astype(np.float64)
     a = x @ c64.T
+    d = x.shape[1]
+    u = 2.0 ** -53
+    # twice the a-priori bound: the bound itself is evaluated in fp64
+    err = 2.0 * (d * u / (1.0 - d * u)) * (np.abs(x) @ np.abs(c64).T)
     best = np.argmax(a, axis=1)
-    top = a[np.arange(a.shape[0]), best]
-    close = a >= (top - 1e-9 * np.maximum(np.abs(top), 1.0))[:, None]
+    rows = np.arange(a.shape[0])
+    close = (a + err) >= (a[rows, best] - err[rows, best])[:, None]
     for t in np.nonzero(close.sum(axis=1) > 1)[0]:
         cand = np.nonzero(close[t])[0]
         exact = [math.fsum(x[t] * c64[j]) for j in cand]
         a[t, cand] = exact
         best[t] = cand[int(np.argmax(exact))]
-    top = a[np.arange(a.shape[0]), best]
+    top = a[rows, best]
     if a.shape[1] > 1:
         a2 = a.copy()
-        a2[np.arange(a.shape[0]), best] = -np.inf
+        a2[rows, best] = -np.inf
         gap = top - a2.max(axis=1)
     else:
         gap = np.full(a.shape[0], np.inf)

@@ -30,8 +30,17 @@ Readings taken where the method description leaves a step open:
   * structured window: block coordinates are the (t, h) of the block's first
     token; keep (I, J) iff |t_I - t_J| <= win_t or |h_I - h_J| <= win_rows *
     ceil(64 / W) token rows; anchors are n_anchors evenly spaced key-block
-    columns (stride floor(nkb / n_anchors)) shifted by a per-step offset that
-    the caller draws;
+    columns (stride floor(nkb / n_anchors)) shifted by a per-step offset
+    o_s = Philox4x32-10(counter = (s, 0, 0, 0), key = (seed mod 2^32,
+    seed div 2^32)), first output word, mod stride -- a counter-based draw, so
+    the anchors rotate with the step index s and repeat for the same seed;
+  * SICS scorer (SPADE, part 2: a coherence check -- the sum of the cosine
+    similarities inside a block -- decides per head and step which blocks
+    are focused on; blocks whose tokens agree are kept, blocks whose tokens
+    disagree are skipped): per head, key block J scores S_J = c_J / sum c with
+    c_J = (sum of cos(k_i, k_j) over the pairs of J's valid keys) / n_J^2; the
+    same score row serves every query block of the head, and the threshold /
+    top-k rules select from it as from pooled scores;
   * routing budget m_I = the count the threshold rule keeps in row I; error
     e_IJ = || sum_{j in J} e^{s_j - M} v_j - n_J e^{qbar.kbar_J/sqrt(d) - M} vbar_J ||_2
     with s_j = qbar_I . k_j / sqrt(d), M = max_j s_j; ratio
@@ -190,6 +199,40 @@ def select_rows(S: np.ndarray, mode: str, *, tau: float = 0.9, keep_frac: float 
     return kept.reshape(S.shape), near.reshape(S.shape)
 
 
+# Philox4x32-10 (J. K. Salmon, M. A. Moraes, R. O. Dror, D. E. Shaw, "Parallel
+# random numbers: as easy as 1, 2, 3", SC'11): ten rounds of two 32x32->64-bit
+# multiplications on a 4-word counter, the 2-word key bumped by the Weyl
+# constants between rounds.
+_PHILOX_M = (0xD2511F53, 0xCD9E8D57)
+_PHILOX_W = (0x9E3779B9, 0xBB67AE85)
+_U32 = 0xFFFFFFFF
+
+
+def philox4x32_10(counter, key):
+    """The four 32-bit output words for a 4-word counter and a 2-word key."""
+    c0, c1, c2, c3 = (int(x) & _U32 for x in counter)
+    k0, k1 = (int(x) & _U32 for x in key)
+    for r in range(10):
+        if r > 0:
+            k0 = (k0 + _PHILOX_W[0]) & _U32
+            k1 = (k1 + _PHILOX_W[1]) & _U32
+        p0 = _PHILOX_M[0] * c0
+        p1 = _PHILOX_M[1] * c2
+        c0, c1, c2, c3 = ((p1 >> 32) ^ c1 ^ k0, p1 & _U32, (p0 >> 32) ^ c3 ^ k1, p0 & _U32)
+    return c0, c1, c2, c3
+
+
+def anchor_offset(seed: int, step: int, nkb: int, n_anchors: int) -> int:
+    """Rotation of the anchor columns at denoising step `step`, in [0, stride),
+    stride = floor(nkb / n_anchors) (at least 1); 0 without anchors."""
+    if n_anchors <= 0 or nkb <= 0:
+        return 0
+    stride = max(nkb // n_anchors, 1)
+    seed = int(seed) & 0xFFFFFFFFFFFFFFFF
+    word = philox4x32_10((int(step), 0, 0, 0), (seed & _U32, seed >> 32))[0]
+    return word % stride
+
+
 def anchor_blocks(nkb: int, n_anchors: int, offset: int) -> np.ndarray:
     """Key-block columns of the rotating anchors for one step."""
     if n_anchors <= 0:
@@ -199,8 +242,9 @@ def anchor_blocks(nkb: int, n_anchors: int, offset: int) -> np.ndarray:
 
 
 def structured_mask(perm: np.ndarray, T: int, H: int, W: int, *, win_t: int, win_rows: int,
-                    n_anchors: int, anchor_offset: int, mode: str = "union") -> np.ndarray:
-    """bool [nb, nb]: temporal band OR spatial band (OR anchors) on 64-token blocks.
+                    n_anchors: int, seed: int = 0, step: int = 0, mode: str = "union") -> np.ndarray:
+    """bool [nb, nb]: temporal band OR spatial band (OR anchors) on 64-token blocks,
+    the anchors rotated for denoising step `step` of the run seeded `seed`.
 
     mode="union" is the reading used by the library; mode="intersection" keeps
     only pairs inside both bands (reported for comparison, not built on GPU).
@@ -214,8 +258,49 @@ def structured_mask(perm: np.ndarray, T: int, H: int, W: int, *, win_t: int, win
     dh = np.abs(h[:, None] - h[None, :]) <= R
     keep = (dt | dh) if mode == "union" else (dt & dh)
     keep = keep.copy()
-    keep[:, anchor_blocks(nb, n_anchors, anchor_offset)] = True
+    keep[:, anchor_blocks(nb, n_anchors, anchor_offset(seed, step, nb, n_anchors))] = True
     return keep
+
+
+def sics_coherence(kp: np.ndarray, N: int) -> np.ndarray:
+    """Block coherence c [nb] of one head's keys ([Npad, d], reordered).
+
+    SPADE, part 2: the sum of intra-block cosine similarities.  Written out as
+    the definition: SICS_J = sum over all ordered pairs (i, j) of valid keys of
+    block J of cos(k_i, k_j) (the i = j terms included; a zero key has cosine
+    0 with every key), and c_J = SICS_J / n_J^2; a block with no valid key has
+    c = 0.
+    """
+    Npad = kp.shape[-2]
+    nb = Npad // BLOCK
+    x = np.asarray(kp, dtype=np.float64)
+    out = np.zeros(nb)
+    for J in range(nb):
+        rows = [r for r in range(J * BLOCK, min(J * BLOCK + BLOCK, N))]
+        n = len(rows)
+        if n == 0:
+            continue
+        blk = x[rows]
+        norms = np.sqrt((blk * blk).sum(axis=1))
+        total = 0.0
+        for i in range(n):
+            if norms[i] == 0.0:
+                continue
+            # cos(k_i, k_j) for every j of the block (zero keys contribute 0)
+            dots = blk @ blk[i]
+            ok = norms > 0.0
+            total += float((dots[ok] / (norms[i] * norms[ok])).sum())
+        out[J] = total / (n * n)
+    return out
+
+
+def sics_scores(kp: np.ndarray, N: int) -> np.ndarray:
+    """S [nb] = c_J / sum_J' c_J' for one head (all zero if every c is 0): the
+    score every query block of the head ranks the key blocks by under the
+    SICS scorer."""
+    c = sics_coherence(kp, N)
+    tot = c.sum()
+    return c / tot if tot > 0 else np.zeros_like(c)
 
 
 def route_ratios(qp: np.ndarray, kp: np.ndarray, vp: np.ndarray, N: int, rows=None) -> np.ndarray:

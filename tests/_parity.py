@@ -17,14 +17,16 @@ def to_np(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy()
 
 
-def gpu_layer(w: workloads.Workload, q, k, v, *, anchor_offset=0, keep_bits=True, compensate=None):
-    """Run the four library calls for workload `w` on cuda tensors; return the object."""
+def gpu_layer(w: workloads.Workload, q, k, v, *, step=0, seed=0, keep_bits=True, compensate=None):
+    """Run the four library calls for workload `w` on cuda tensors at denoising
+    step `step` of a run seeded `seed`; return the object."""
     comp = w.compensate if compensate is None else compensate
     attn = SparseVideoAttention(w.B, w.heads, w.T, w.H, w.W, w.d, order=w.order, select=w.select,
                                 tau=w.tau, keep_frac=w.keep_frac, sub_block=w.sub_block, win_t=w.win_t,
                                 win_rows=w.win_rows, n_anchors=w.n_anchors if w.select == "structured" else 0,
-                                routing=w.routing, compensate=comp, keep_bits=keep_bits, device="cuda")
-    out = attn(q, k, v, anchor_offset=anchor_offset)
+                                routing=w.routing, compensate=comp, keep_bits=keep_bits, seed=seed,
+                                scorer=w.scorer, device="cuda")
+    out = attn(q, k, v, step=step)
     torch.cuda.synchronize()
     attn.out = out
     return attn
@@ -51,13 +53,16 @@ def gpu_keep(attn) -> np.ndarray:
     return keep
 
 
-def oracle_rows(w: workloads.Workload, qp, kp, vp, perm, rows, anchor_offset=0):
+def oracle_rows(w: workloads.Workload, qp, kp, vp, perm, rows, step=0, seed=0):
     """Oracle (kept, near) for query-block rows `rows` of one head ([Npad, d] fp64)."""
     N = w.N
     if w.select == "structured":
         keep = oracle.structured_mask(perm, w.T, w.H, w.W, win_t=w.win_t, win_rows=w.win_rows,
-                                      n_anchors=w.n_anchors, anchor_offset=anchor_offset)
+                                      n_anchors=w.n_anchors, seed=seed, step=step)
         return keep[rows], np.zeros((len(rows), keep.shape[1]), dtype=bool)
+    if w.scorer == "sics":
+        S = np.tile(oracle.sics_scores(kp, N), (len(rows), 1))
+        return oracle.select_rows(S, w.select, tau=w.tau, keep_frac=w.keep_frac)
     if w.sub_block == 64:
         qb, _ = oracle.pool(qp, N)
         kb, _ = oracle.pool(kp, N)

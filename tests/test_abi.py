@@ -36,8 +36,58 @@ def test_library_exports_every_declared_symbol():
 
 def test_struct_sizes_match_header():
     assert ctypes.sizeof(Shape) == 24
-    assert ctypes.sizeof(MaskParams) == 36
-    assert ctypes.sizeof(Mask) == 64
+    assert ctypes.sizeof(MaskParams) == 48
+    assert ctypes.sizeof(Mask) == 72
+
+
+def test_struct_layouts_match_the_c_compiler(tmp_path):
+    # every field offset of the binding's structures equals the C compiler's
+    # for include/svsa.h (a C probe built with gcc)
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    structs = {"svsa_shape": Shape, "svsa_mask_params": MaskParams, "svsa_mask": Mask}
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "svsa.h"', "int main(void) {"]
+    for cname, cls in structs.items():
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for fname, _ in cls._fields_:
+            lines.append(f'  printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "probe.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "probe"
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    seen = 0
+    for line in out:
+        if not line:
+            continue
+        cname, field, val = line.split()
+        cls = structs[cname]
+        want = ctypes.sizeof(cls) if field == "size" else getattr(cls, field).offset
+        assert int(val) == want, (cname, field, val, want)
+        seen += 1
+    assert seen == sum(len(c._fields_) + 1 for c in structs.values())
+
+
+def test_anchor_offset_entry_point_matches_the_oracle():
+    # the library's host-side Philox4x32-10 draw against the oracle's, bit for bit
+    import oracle
+    rng = np.random.default_rng(2024)
+    for i in range(1000):
+        seed = int(rng.integers(0, 2**63)) * (2 if i % 3 else 1) % 2**64
+        step = int(rng.integers(0, 2**31)) if i % 2 else i
+        nb = int(rng.integers(1, 16385))
+        n = int(rng.integers(0, min(nb, 16) + 1))
+        assert svsa.svsa_anchor_offset(seed, step, nb, n) == oracle.anchor_offset(seed, step, nb, n), (seed, step, nb, n)
+    # rejections
+    lib = svsa.lib()
+    out = ctypes.c_int32(0)
+    assert lib.svsa_anchor_offset(0, -1, 512, 4, ctypes.byref(out)) == 1
+    assert lib.svsa_anchor_offset(0, 0, 0, 0, ctypes.byref(out)) == 1
+    assert lib.svsa_anchor_offset(0, 0, 4, 5, ctypes.byref(out)) == 1
+    assert lib.svsa_anchor_offset(0, 0, 4, 1, None) == 1
 
 
 def test_version():
@@ -88,7 +138,7 @@ def test_reorder_and_attention_reject_before_launch():
     assert lib.svsa_inverse_reorder(None, 32, 48, s, None) == 1
     m = Mask(None, None, 4, None, None, None, None, None)
     assert lib.svsa_attn_fwd(16, 32, 48, ctypes.byref(m), 0, 64, None, s, None) == 1
-    m = Mask(16, 32, 4, None, None, None, None, None)
+    m = Mask(16, 32, 4, None, None, None, None, None, 0)
     assert lib.svsa_attn_fwd(16, 32, 48, ctypes.byref(m), 1, 64, None, s, None) == 1   # comp w/o means
     assert "kbar" in _err()
     kb = 80
@@ -105,10 +155,10 @@ def test_reorder_and_attention_reject_before_launch():
 def test_build_mask_rejects_before_launch():
     lib = _raw()
     s = svsa.shape(1, 2, 4, 8, 8, 128)                                    # nb = 4
-    m = Mask(16, 32, 4, None, None, None, None, None)
+    m = Mask(16, 32, 4, None, None, None, None, None, 0)
     ok = svsa.mask_params(svsa.SEL_THRESHOLD)
     # capacity below nb for a threshold rule
-    small = Mask(16, 32, 3, None, None, None, None, None)
+    small = Mask(16, 32, 3, None, None, None, None, None, 0)
     assert lib.svsa_build_mask(16, 32, None, None, s, ctypes.byref(ok), ctypes.byref(small), 64, 1 << 20, None) == 1
     # routing without V / means
     r = svsa.mask_params(svsa.SEL_THRESHOLD, routing=True)
@@ -117,11 +167,28 @@ def test_build_mask_rejects_before_launch():
     r2 = svsa.mask_params(svsa.SEL_TOPK, routing=True)
     assert lib.svsa_build_mask(16, 32, 48, None, s, ctypes.byref(r2), ctypes.byref(m), 64, 1 << 20, None) == 1
     # structured without perm
-    st = svsa.mask_params(svsa.SEL_STRUCTURED, n_anchors=2, anchor_offset=0)
+    st = svsa.mask_params(svsa.SEL_STRUCTURED, n_anchors=2, step=0)
     assert lib.svsa_build_mask(None, None, None, None, s, ctypes.byref(st), ctypes.byref(m), None, 0, None) == 1
-    # anchor offset outside [0, nb / n_anchors)
-    st2 = svsa.mask_params(svsa.SEL_STRUCTURED, n_anchors=2, anchor_offset=5)
+    # a negative step index
+    st2 = svsa.mask_params(svsa.SEL_STRUCTURED, n_anchors=2, step=-3)
     assert lib.svsa_build_mask(None, None, None, 16, s, ctypes.byref(st2), ctypes.byref(m), None, 0, None) == 1
+    # more anchors than blocks
+    st3 = svsa.mask_params(svsa.SEL_STRUCTURED, n_anchors=5)
+    assert lib.svsa_build_mask(None, None, None, 16, s, ctypes.byref(st3), ctypes.byref(m), None, 0, None) == 1
+    # the SICS scorer: not for the structured rule, only 64-token blocks, no routing, unknown scorer
+    sx = svsa.mask_params(svsa.SEL_STRUCTURED, scorer=svsa.SCORE_SICS)
+    assert lib.svsa_build_mask(None, 32, None, 16, s, ctypes.byref(sx), ctypes.byref(m), 64, 1 << 20, None) == 1
+    sx = svsa.mask_params(svsa.SEL_TOPK, sub_block=16, scorer=svsa.SCORE_SICS)
+    assert lib.svsa_build_mask(None, 32, None, None, s, ctypes.byref(sx), ctypes.byref(m), 64, 1 << 20, None) == 2
+    sx = svsa.mask_params(svsa.SEL_THRESHOLD, routing=True, scorer=svsa.SCORE_SICS)
+    assert lib.svsa_build_mask(16, 32, 48, None, s, ctypes.byref(sx), ctypes.byref(m), 64, 1 << 20, None) == 2
+    sx = svsa.mask_params(svsa.SEL_TOPK, scorer=7)
+    assert lib.svsa_build_mask(16, 32, None, None, s, ctypes.byref(sx), ctypes.byref(m), 64, 1 << 20, None) == 1
+    # the SICS scorer needs no queries but its workspace
+    sx = svsa.mask_params(svsa.SEL_TOPK, scorer=svsa.SCORE_SICS)
+    need = svsa.svsa_mask_workspace_bytes(s, sx)
+    assert need > 0
+    assert lib.svsa_build_mask(None, 32, None, None, s, ctypes.byref(sx), ctypes.byref(m), 64, need - 1, None) == 3
     # workspace too small
     assert lib.svsa_build_mask(16, 32, None, None, s, ctypes.byref(ok), ctypes.byref(m), 64, 16, None) == 3
     # unknown selection rule / sub-block size
@@ -135,7 +202,8 @@ def test_status_codes_are_stable():
     # values are part of the ABI
     text = open(os.path.join(ROOT, "include", "svsa.h")).read()
     for name, val in [("SVSA_OK", 0), ("SVSA_ERR_INVALID_ARG", 1), ("SVSA_ERR_UNSUPPORTED", 2),
-                      ("SVSA_ERR_WORKSPACE", 3), ("SVSA_ERR_CUDA", 4), ("SVSA_ERR_TIMEOUT", 5)]:
+                      ("SVSA_ERR_WORKSPACE", 3), ("SVSA_ERR_CUDA", 4), ("SVSA_ERR_TIMEOUT", 5),
+                      ("SVSA_ERR_RANGE", 6), ("SVSA_ERR_MASK", 7)]:
         assert re.search(rf"{name}\s*=\s*{val}\b", text)
 
 

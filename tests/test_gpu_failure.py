@@ -58,3 +58,91 @@ def test_two_runs_are_bit_identical(kw):
     assert torch.equal(runs[0][0], runs[1][0])
     assert np.array_equal(runs[0][1], runs[1][1])
     assert all(torch.equal(a, b) for a, b in zip(runs[0][2], runs[1][2]))
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def test_values_beyond_fp16_are_reported_as_range():
+    """A bf16 value of 7e4 given to the fp16 value gather saturates; the call
+    succeeds but svsa_sync_status reports SVSA_ERR_RANGE once, then clears."""
+    lib = svsa.lib()
+    w = workloads.WORKLOADS["tiny"]
+    q, k, v = (t.cuda() for t in workloads.make_qkv(w))
+    s = svsa.shape(1, 1, w.T, w.H, w.W, w.d)
+    perm = torch.arange(w.Npad, dtype=torch.int32, device="cuda")
+    vp = torch.empty(1, 1, w.Npad, w.d, dtype=torch.float16, device="cuda")
+    svsa.svsa_reorder_values(v, vp, perm, s)
+    assert lib.svsa_sync_status(_stream()) == 0                   # in range: nothing recorded
+    v2 = v.clone()
+    v2[0, 0, 17, 5] = 7.0e4
+    svsa.svsa_reorder_values(v2, vp, perm, s)
+    assert lib.svsa_sync_status(_stream()) == 6                   # SVSA_ERR_RANGE
+    assert "svsa_reorder_values" in lib.svsa_last_error().decode()
+    assert float(vp[0, 0, 17, 5]) == 65504.0                       # saturated, as documented
+    assert lib.svsa_sync_status(_stream()) == 0                   # reported once
+    v2[0, 0, 3, 0] = float("inf")
+    v2[0, 0, 17, 5] = 0.0
+    svsa.svsa_reorder_values(v2, vp, perm, s)
+    assert lib.svsa_sync_status(_stream()) == 6
+
+
+def test_block_means_beyond_fp16_are_reported_as_range():
+    """Queries whose block mean exceeds the fp16 range of the scores' split."""
+    lib = svsa.lib()
+    w = workloads.WORKLOADS["tiny"]
+    q, k, v = (t.cuda() for t in workloads.make_qkv(w))
+    q2 = q.clone()
+    q2[0, 0, :64, 3] = 9.0e4                                      # a whole block: its mean is 9e4
+    attn = svsa.SparseVideoAttention(w.B, w.heads, w.T, w.H, w.W, w.d, order=w.order, select=w.select, tau=w.tau)
+    attn(q, k, v)
+    assert lib.svsa_sync_status(_stream()) == 0
+    attn(q2, k, v)
+    assert lib.svsa_sync_status(_stream()) == 6
+    assert "block mean" in lib.svsa_last_error().decode()
+    assert lib.svsa_sync_status(_stream()) == 0
+
+
+@pytest.mark.parametrize("defect", ["descending", "out_of_range", "negative", "count_above_cap", "duplicate"])
+def test_malformed_masks_are_reported(defect):
+    """mask.check validates caller-built lists before the attention; the
+    attention still clamps every count and index to the tensors, so the run
+    touches nothing outside them and returns, and svsa_sync_status reports
+    SVSA_ERR_MASK."""
+    lib = svsa.lib()
+    B, heads, T, H, W, d = 1, 2, 4, 8, 16, 128                    # nb = 8
+    N = T * H * W
+    nb = N // 64
+    s = svsa.shape(B, heads, T, H, W, d)
+    g = torch.Generator(device="cuda").manual_seed(5)
+    qp = torch.randn(B, heads, nb * 64, d, generator=g, device="cuda").to(torch.bfloat16)
+    kp = torch.randn(B, heads, nb * 64, d, generator=g, device="cuda").to(torch.bfloat16)
+    vp = torch.randn(B, heads, nb * 64, d, generator=g, device="cuda").to(torch.float16)
+    op = torch.empty_like(qp)
+    cap = nb
+    kv_idx = torch.arange(cap, dtype=torch.int32, device="cuda").repeat(B * heads * nb, 1).reshape(B, heads, nb, cap)
+    kv_cnt = torch.full((B, heads, nb), 4, dtype=torch.int32, device="cuda")
+    good = svsa.make_mask(kv_idx, kv_cnt, cap, check=True)
+    svsa.svsa_attn_fwd(qp, kp, vp, good, False, op, None, s)
+    assert lib.svsa_sync_status(_stream()) == 0
+    bad_idx, bad_cnt = kv_idx.clone(), kv_cnt.clone()
+    if defect == "descending":
+        bad_idx[0, 1, 3, :4] = torch.tensor([5, 3, 2, 0], dtype=torch.int32)
+    elif defect == "out_of_range":
+        bad_idx[0, 0, 2, 3] = nb + 5
+    elif defect == "negative":
+        bad_idx[0, 0, 0, 0] = -1
+    elif defect == "count_above_cap":
+        bad_cnt[0, 1, 7] = cap + 3
+    else:
+        bad_idx[0, 0, 6, :4] = torch.tensor([1, 2, 2, 3], dtype=torch.int32)
+    bad = svsa.make_mask(bad_idx, bad_cnt, cap, check=True)
+    svsa.svsa_attn_fwd(qp, kp, vp, bad, False, op, None, s)
+    assert lib.svsa_sync_status(_stream()) == 7                   # SVSA_ERR_MASK
+    assert "malformed" in lib.svsa_last_error().decode()
+    assert lib.svsa_sync_status(_stream()) == 0
+    # without the check the same call is not validated (and still stays in bounds)
+    unchecked = svsa.make_mask(bad_idx, bad_cnt, cap)
+    svsa.svsa_attn_fwd(qp, kp, vp, unchecked, False, op, None, s)
+    assert lib.svsa_sync_status(_stream()) == 0

@@ -85,16 +85,16 @@ def _small(select, sub=64, grid=(5, 7, 9), heads=2, d=128, **kw):
     return workloads.Workload("small", 1, heads, d, T, H, W, select=select, sub_block=sub, **kw)
 
 
-def _run_and_compare_masks(w, anchor_offset=0, seed=0):
+def _run_and_compare_masks(w, step=0, seed=0, run_seed=0):
     q, k, v = (t.cuda() for t in workloads.make_qkv(w, seed=seed))
-    attn = gpu_layer(w, q, k, v, anchor_offset=anchor_offset)
+    attn = gpu_layer(w, q, k, v, step=step, seed=run_seed)
     keep = gpu_keep(attn)
     perm, _ = oracle.build_perm(w.T, w.H, w.W, w.order)
     qp, kp, vp = (oracle.reorder(to_np(t)[0].astype(np.float64), perm) for t in (q, k, v))
     near_total = 0
     rows = list(range(attn.nb))
     for eta in range(w.heads):
-        kept, near = oracle_rows(w, qp[eta], kp[eta], vp[eta], perm, rows, anchor_offset)
+        kept, near = oracle_rows(w, qp[eta], kp[eta], vp[eta], perm, rows, step=step, seed=run_seed)
         n, _ = compare_mask_rows(keep[eta], kept, near)
         near_total += n
     return attn, keep, (q, k, v), (qp, kp, vp), perm, near_total
@@ -114,6 +114,76 @@ def test_mask_and_attention_small(order, select, sub, grid):
         assert np.all(op[eta][w.N:] == 0)
 
 
+@pytest.mark.parametrize("order", ["raster", "hilbert"])
+@pytest.mark.parametrize("select", ["topk", "threshold"])
+@pytest.mark.parametrize("grid,d", [((5, 7, 9), 128), ((6, 12, 20), 64), ((4, 8, 8), 128)])
+def test_sics_mask_and_attention_small(order, select, grid, d):
+    """The SICS scorer: per-head coherence scores, one list per head copied to
+    every query block, against the oracle's definition (the double sum of
+    cosines); outputs on that mask within tolerance."""
+    T, H, W = grid
+    w = workloads.Workload("sics", 1, 2, d, T, H, W, order=order, select=select, tau=0.6, keep_frac=0.3,
+                           scorer="sics")
+    attn, keep, _, (qp, kp, vp), _, near = _run_and_compare_masks(w)
+    for eta in range(w.heads):
+        assert np.all(keep[eta] == keep[eta][:1])              # the same list for every query block
+    op = to_np(attn.buf.op)[0]
+    for eta in range(w.heads):
+        ref = oracle.masked_attention(qp[eta], kp[eta], vp[eta], w.N, keep[eta])
+        gout = np.concatenate([op[eta][I * 64:min(I * 64 + 64, w.N)] for I in range(attn.nb)])
+        check_attention(gout, np.concatenate([ref[I] for I in range(attn.nb)]), f"head {eta}")
+
+
+def test_sics_zero_keys_and_compensation():
+    """All-zero keys: every coherence is 0, so the threshold rule keeps every
+    block and top-k the first k; with compensation on a SICS mask, the means
+    come from the same call."""
+    w = workloads.Workload("sics0", 1, 2, 128, 6, 12, 20, order="hilbert", select="threshold", tau=0.9,
+                           scorer="sics")
+    q, k, v = (t.cuda() for t in workloads.make_qkv(w, seed=3))
+    attn = gpu_layer(w, q, torch.zeros_like(k), v)
+    assert gpu_keep(attn).all()
+    wk = w.with_(select="topk", keep_frac=0.25)
+    attn = gpu_layer(wk, q, torch.zeros_like(k), v)
+    keep = gpu_keep(attn)
+    kk = oracle.topk_count(wk.keep_frac, attn.nb)
+    assert np.all(keep[:, :, :kk]) and not keep[:, :, kk:].any()
+    wc = w.with_(select="topk", keep_frac=0.3, compensate=True)
+    attn = gpu_layer(wc, q, k, v)
+    keep = gpu_keep(attn)
+    perm, _ = oracle.build_perm(wc.T, wc.H, wc.W, wc.order)
+    qp, kp, vp = (oracle.reorder(to_np(t)[0].astype(np.float64), perm) for t in (q, k, v))
+    op = to_np(attn.buf.op)[0]
+    for eta in range(wc.heads):
+        kb, nv = oracle.pool(kp[eta], wc.N)
+        vb, _ = oracle.pool(vp[eta], wc.N)
+        ref = oracle.compensated_attention(qp[eta], kp[eta], vp[eta], wc.N, keep[eta], kb, vb, nv)
+        gout = np.concatenate([op[eta][I * 64:min(I * 64 + 64, wc.N)] for I in range(attn.nb)])
+        check_attention(gout, np.concatenate([ref[I] for I in range(attn.nb)]), f"head {eta}")
+
+
+@pytest.mark.parametrize("size,d,grid", [(64, 128, (5, 7, 9)), (16, 128, (6, 12, 20)), (16, 64, (2, 9, 13)),
+                                         (64, 64, (1, 1, 65))])
+def test_pool_entry_point(size, d, grid):
+    """svsa_pool: fp32 means of the valid rows of every group, pads never
+    counted, against the oracle's fp64 means (fp32 sums of <= 64 bf16 values)."""
+    T, H, W = grid
+    N = T * H * W
+    nb = -(-N // 64)
+    g = torch.Generator(device="cuda").manual_seed(9)
+    xp = torch.zeros(1, 3, nb * 64, d, dtype=torch.bfloat16, device="cuda")
+    xp[:, :, :N] = (2.0 * torch.randn(1, 3, N, d, generator=g, device="cuda")).to(torch.bfloat16)
+    xp[:, :, N:] = 7.0                                          # pads must not count
+    out = torch.empty(1, 3, nb * 64 // size, d, dtype=torch.float32, device="cuda")
+    svsa.svsa_pool(xp, out, svsa.shape(1, 3, T, H, W, d), size)
+    torch.cuda.synchronize()
+    for eta in range(3):
+        ref, cnt = oracle.pool(to_np(xp)[0, eta].astype(np.float64), N, size)
+        got = out[0, eta].cpu().numpy().astype(np.float64)
+        assert np.abs(got - ref).max() <= 1e-5
+        assert np.all(got[cnt == 0] == 0.0)
+
+
 @pytest.mark.parametrize("tau", [0.5, 0.95, 1.0])
 def test_threshold_extremes(tau):
     w = _small("threshold", 64, grid=(6, 12, 20), tau=tau)
@@ -125,9 +195,14 @@ def test_threshold_extremes(tau):
 def test_structured_bit_exact():
     w = workloads.Workload("s", 1, 2, 64, 12, 10, 20, order="raster", select="structured",
                            win_t=2, win_rows=1, n_anchors=4)
-    for off in (0, 3, 7):
-        _, keep, *_ = _run_and_compare_masks(w, anchor_offset=off)
+    # the anchors rotate with the step index (computed in the library from
+    # (seed, step)); each step's mask must equal the oracle's bit for bit
+    cols = []
+    for run_seed, step in ((0, 0), (0, 1), (0, 2), (0, 3), (12345, 3), (2**40 + 1, 0)):
+        _, keep, *_ = _run_and_compare_masks(w, step=step, run_seed=run_seed)
         assert np.array_equal(keep[0], keep[1])          # structure is per layer, not per head
+        cols.append(tuple(np.nonzero(keep[0].all(axis=0))[0]))
+    assert len(set(cols[:4])) > 1                        # the always-kept columns move with the step
     w0 = w.with_(win_t=0, win_rows=0, n_anchors=0, T=3, H=8, W=16)
     _run_and_compare_masks(w0)
 
@@ -240,11 +315,11 @@ def test_forward_host_matches_device_call(select, groups, kw):
     mk = lambda: svsa.SparseVideoAttention(w.B, w.heads, w.T, w.H, w.W, w.d, order=w.order, select=w.select,
                                            tau=w.tau, keep_frac=w.keep_frac, n_anchors=w.n_anchors,
                                            routing=w.routing, compensate=w.compensate, device="cuda")
-    ref = mk()(q, k, v, anchor_offset=1)
+    ref = mk()(q, k, v, step=1)
     hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
     hout = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
     attn = mk()
-    attn.forward_host(hq, hk, hv, hout, anchor_offset=1, groups=groups)
+    attn.forward_host(hq, hk, hv, hout, step=1, groups=groups)
     torch.cuda.synchronize()
     assert torch.equal(hout, ref.cpu())
     # a second call reusing the cached mask gives the same output again
@@ -451,7 +526,7 @@ def test_batch_rows_are_independent(case):
                 attn.build_perm(q=q, k=k)
             out = attn(q, k, v)
         else:
-            attn = gpu_layer(w, q, k, v, anchor_offset=1)
+            attn = gpu_layer(w, q, k, v, step=1)
             out = attn.out
         torch.cuda.synchronize()
         return attn, out

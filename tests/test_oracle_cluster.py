@@ -71,3 +71,27 @@ def test_one_round_fixed_point_on_separated_data():
     a3 = cluster.cocluster(q, k, N, rounds=3)
     a5 = cluster.cocluster(q, k, N, rounds=5)
     assert np.array_equal(a3[0], a5[0]) and np.array_equal(a3[1], a5[1])
+
+
+def test_assignment_survives_cancellation_in_the_fp64_sums():
+    # Exact affinities that fp64 summation gets wrong in any usual order: with
+    # x = (1, 1, 1) and a centroid holding +-2^60, adding 1 to 2^60 first loses
+    # the 1.  The oracle must decide on the exact sums (math.fsum over the
+    # exact bf16 x float32 products), so a plain fp64 argmax, or a near-tie
+    # window that is relative to the (cancelled) result, fails here.
+    big = 2.0 ** 60
+    x = np.ones((2, 3))
+    # row 0: every permutation of (2^60, 1, -2^60): all exactly 1 -> tie -> index 0
+    perms = [(1.0, big, -big), (big, -big, 1.0), (big, 1.0, -big), (-big, big, 1.0), (1.0, -big, big),
+             (-big, 1.0, big)]
+    c = np.array(perms, dtype=np.float32)
+    best, gap = cluster._assign(x[:1], c)
+    assert best.tolist() == [0] and gap.tolist() == [0.0]
+    # row 1: exactly 1 (cancelling) against exactly 0.5 (plain): the first wins by 0.5
+    c2 = np.array([(1.0, big, -big), (0.5, 0.0, 0.0)], dtype=np.float32)
+    best, gap = cluster._assign(x[1:], c2)
+    assert best.tolist() == [0] and gap.tolist() == [0.5]
+    # the candidates' exact values are what decide: swapping the two centroids
+    # moves the winner with them
+    best, _ = cluster._assign(x[1:], c2[::-1].copy())
+    assert best.tolist() == [1]

@@ -145,18 +145,18 @@ def test_near_threshold_flags():
 def test_structured_hand_case(golden):
     expect = np.array(golden("structured_3x8x16.txt"), dtype=bool)
     perm, _ = oracle.perm_raster(3, 8, 16)
-    keep = oracle.structured_mask(perm, 3, 8, 16, win_t=0, win_rows=0, n_anchors=0, anchor_offset=0)
+    keep = oracle.structured_mask(perm, 3, 8, 16, win_t=0, win_rows=0, n_anchors=0)
     assert np.array_equal(keep, expect)
 
 
 def test_structured_symmetry_and_anchors():
     perm, _ = oracle.perm_raster(12, 10, 20)
-    base = oracle.structured_mask(perm, 12, 10, 20, win_t=2, win_rows=1, n_anchors=0, anchor_offset=0)
+    base = oracle.structured_mask(perm, 12, 10, 20, win_t=2, win_rows=1, n_anchors=0)
     assert np.array_equal(base, base.T)
     nb = base.shape[0]
-    for off in (0, 3, 7):
-        keep = oracle.structured_mask(perm, 12, 10, 20, win_t=2, win_rows=1, n_anchors=4, anchor_offset=off)
-        cols = oracle.anchor_blocks(nb, 4, off)
+    for seed, step in ((0, 0), (0, 1), (5, 3), (2**40 + 7, 11)):
+        keep = oracle.structured_mask(perm, 12, 10, 20, win_t=2, win_rows=1, n_anchors=4, seed=seed, step=step)
+        cols = oracle.anchor_blocks(nb, 4, oracle.anchor_offset(seed, step, nb, 4))
         assert keep[:, cols].all()
         extra = keep & ~base
         assert set(np.nonzero(extra.any(axis=0))[0]) <= set(cols.tolist())
@@ -165,13 +165,65 @@ def test_structured_symmetry_and_anchors():
     assert a.tolist() == [2, 11, 20, 29]
 
 
+def _hex_rows(name):
+    import os
+    rows = []
+    with open(os.path.join(os.path.dirname(__file__), "golden", name)) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                rows.append([int(x, 16) for x in line.split()])
+    return rows
+
+
+def test_philox_known_answers():
+    # Random123's published philox4x32-10 vectors: a dropped round, a wrong
+    # multiplier, Weyl constant or word order fails at least one of them
+    for row in _hex_rows("philox4x32_10_kat.txt"):
+        ctr, key, out = row[:4], row[4:6], row[6:]
+        assert list(oracle.philox4x32_10(ctr, key)) == out
+
+
+def test_anchor_offset_closed_form_and_range():
+    # seed 0, step 0: counter and key all zero, so the offset is the first
+    # known-answer word 0x6627e8d5 = 1713891541 modulo the stride
+    assert oracle.anchor_offset(0, 0, 3072, 4) == 1713891541 % 768 == 469
+    assert oracle.anchor_offset(0, 0, 512, 4) == 1713891541 % 128
+    assert oracle.anchor_offset(0, 0, 3, 4) == 0          # stride clamps to 1
+    assert oracle.anchor_offset(9, 9, 512, 0) == 0        # no anchors
+    rng = np.random.default_rng(3)
+    for _ in range(300):
+        nkb = int(rng.integers(1, 5000))
+        n = int(rng.integers(1, 9))
+        off = oracle.anchor_offset(int(rng.integers(0, 2**63)), int(rng.integers(0, 2**31)), nkb, n)
+        assert 0 <= off < max(nkb // n, 1)
+
+
+def test_anchors_rotate_with_the_step_and_repeat_for_the_seed():
+    nkb, n = 3072, 4
+    stride = nkb // n
+    offs = [oracle.anchor_offset(0, s, nkb, n) for s in range(64)]
+    # a counter-based draw: the same (seed, step) gives the same anchors ...
+    assert offs == [oracle.anchor_offset(0, s, nkb, n) for s in range(64)]
+    # ... the anchors move from step to step (64 draws from 768 values) ...
+    assert len(set(offs)) > 55
+    assert all(offs[s] != offs[s + 1] for s in range(8))
+    # ... each step's columns stay evenly spaced, one per stride ...
+    for s in range(4):
+        cols = oracle.anchor_blocks(nkb, n, offs[s])
+        assert np.all(np.diff(cols) == stride) and cols[0] == offs[s]
+    # ... and another seed gives another rotation
+    assert [oracle.anchor_offset(1, s, nkb, n) for s in range(8)] != offs[:8]
+    # the 64-bit seed enters both key words
+    assert oracle.anchor_offset(2**32, 0, nkb, n) != oracle.anchor_offset(0, 0, nkb, n)
+    assert oracle.anchor_offset(1, 0, nkb, n) != oracle.anchor_offset(0, 0, nkb, n)
+
+
 def test_structured_density_readings():
     # the long-horizon grid: union reading ~19%, intersection far sparser
     T, H, W = 126, 30, 52
     perm, _ = oracle.perm_raster(T, H, W)
-    u = oracle.structured_mask(perm, T, H, W, win_t=2, win_rows=1, n_anchors=0, anchor_offset=0)
-    x = oracle.structured_mask(perm, T, H, W, win_t=2, win_rows=1, n_anchors=0, anchor_offset=0,
-                               mode="intersection")
+    u = oracle.structured_mask(perm, T, H, W, win_t=2, win_rows=1, n_anchors=0)
+    x = oracle.structured_mask(perm, T, H, W, win_t=2, win_rows=1, n_anchors=0, mode="intersection")
     assert 0.17 < u.mean() < 0.22
     assert x.mean() < 0.02
 
@@ -250,3 +302,69 @@ def test_mask_from_rows():
     kept = np.array([[True, False, True], [False, False, True]])
     idx, cnt = oracle.mask_from_rows(kept)
     assert cnt.tolist() == [2, 1] and idx[0].tolist() == [0, 2] and idx[1].tolist() == [2]
+
+
+# ---- SICS coherence (SPADE, part 2) -------------------------------------------------
+def test_sics_constant_block_is_fully_coherent():
+    # n identical keys: every cosine is 1, SICS = n^2, c = 1
+    kp = np.zeros((128, 8))
+    kp[:64] = np.array([1.0, -2.0, 0.5, 3.0, 0.0, 1.0, 1.0, -1.0])
+    kp[64:128] = 0.25
+    c = oracle.sics_coherence(kp, 128)
+    assert np.allclose(c, [1.0, 1.0], atol=1e-12)
+
+
+def test_sics_orthogonal_keys_give_one_over_n():
+    # n mutually orthogonal keys (scaled basis vectors): only the n diagonal
+    # terms survive, SICS = n, c = 1 / n
+    d = 64
+    kp = np.zeros((64, d))
+    kp[np.arange(64), np.arange(64)] = np.linspace(0.5, 3.0, 64)
+    assert abs(oracle.sics_coherence(kp, 64)[0] - 1.0 / 64) < 1e-14
+
+
+def test_sics_antipodal_keys_cancel_and_scale_does_not_matter():
+    # keys s_i * x with s_i = +-1 in equal numbers: SICS = (sum s_i)^2 = 0
+    x = np.array([0.3, -1.0, 2.0, 0.7])
+    kp = np.tile(x, (64, 1)) * np.repeat([1.0, -1.0], 32)[:, None]
+    assert abs(oracle.sics_coherence(kp, 64)[0]) < 1e-12
+    # 48 keys along +x and 16 along -x: SICS = (48 - 16)^2 = 1024, c = 1/4;
+    # positive rescaling of individual keys changes nothing
+    s = np.where(np.arange(64) < 48, 1.0, -1.0) * np.linspace(0.1, 5.0, 64)
+    assert abs(oracle.sics_coherence(np.outer(s, x), 64)[0] - 0.25) < 1e-12
+
+
+def test_sics_zero_key_ragged_block_and_closed_form():
+    rng = np.random.default_rng(11)
+    N, d = 64 + 40, 16                                 # second block: 40 valid keys, 24 pads
+    kp = np.zeros((128, d))
+    kp[:N] = rng.standard_normal((N, d))
+    kp[5] = 0.0                                        # a zero key counts in n, adds nothing
+    kp[N:] = 9.0                                       # pads must be ignored
+    c = oracle.sics_coherence(kp, N)
+    # identity: sum_{i,j} cos(k_i, k_j) = || sum_i k_i / ||k_i|| ||^2 over nonzero keys
+    for J, (lo, hi) in enumerate([(0, 64), (64, N)]):
+        blk = kp[lo:hi]
+        nrm = np.linalg.norm(blk, axis=1)
+        u = (blk[nrm > 0] / nrm[nrm > 0, None]).sum(axis=0)
+        assert abs(c[J] - (u @ u) / (hi - lo) ** 2) < 1e-12
+    # one zero key among n - 1 identical ones: SICS = (n - 1)^2
+    kq = np.zeros((64, d))
+    kq[1:] = 2.0
+    assert abs(oracle.sics_coherence(kq, 64)[0] - (63 / 64) ** 2) < 1e-14
+    # an empty block (all pads) scores 0
+    assert oracle.sics_coherence(np.ones((128, 4)), 64)[1] == 0.0
+
+
+def test_sics_scores_rank_the_coherent_blocks():
+    rng = np.random.default_rng(12)
+    d, nb = 16, 6
+    kp = rng.standard_normal((nb * 64, d))
+    # blocks 1 and 4 made coherent: a shared direction plus a little noise
+    for J, a in ((1, 0.1), (4, 0.3)):
+        kp[J * 64:(J + 1) * 64] = rng.standard_normal(d) + a * rng.standard_normal((64, d))
+    S = oracle.sics_scores(kp, nb * 64)
+    assert abs(S.sum() - 1.0) < 1e-12 and np.all(S >= 0)
+    kept, _ = oracle.select_topk(S, 2)
+    assert np.nonzero(kept)[0].tolist() == [1, 4]
+    assert np.all(oracle.sics_scores(np.zeros((128, 4)), 128) == 0.0)

@@ -64,3 +64,33 @@ def test_rejects_grids_beyond_the_fixed_scratch():
     status = svsa.lib().svsa_build_perm_noalloc(s, svsa.ORDER_HILBERT, perm.data_ptr(), iperm.data_ptr(), stream)
     assert status == 2
     assert "128" in svsa.lib().svsa_last_error().decode()
+
+
+def test_two_streams_ordered_by_an_event():
+    # The calls share one scratch array: on two streams they are correct only
+    # when ordered.  Both calls are queued back to back with no host
+    # synchronisation between them; stream b waits for an event recorded
+    # after the call on stream a, so both results must equal the workspace
+    # variant's.
+    T, H, W = 21, 30, 52
+    s = svsa.shape(1, 1, T, H, W, 128)
+    N = T * H * W
+    Npad = -(-N // 64) * 64
+    ref = _with_workspace(s, svsa.ORDER_HILBERT, N, Npad)
+    outs = [(torch.full((Npad,), -7, dtype=torch.int32, device="cuda"),
+             torch.full((N,), -7, dtype=torch.int32, device="cuda")) for _ in range(2)]
+    torch.cuda.synchronize()
+    sa, sb = torch.cuda.Stream(), torch.cuda.Stream()
+    done = torch.cuda.Event()
+    for n, ((perm, iperm), stream) in enumerate(zip(outs, (sa, sb))):
+        if n == 1:
+            stream.wait_event(done)
+        status = svsa.lib().svsa_build_perm_noalloc(s, svsa.ORDER_HILBERT, perm.data_ptr(), iperm.data_ptr(),
+                                                    ctypes.c_void_p(stream.cuda_stream))
+        assert status == 0, svsa.lib().svsa_last_error().decode()
+        if n == 0:
+            done.record(stream)
+    torch.cuda.synchronize()
+    svsa.svsa_sync_status()
+    for perm, iperm in outs:
+        assert torch.equal(perm, ref[0]) and torch.equal(iperm, ref[1])

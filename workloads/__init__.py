@@ -16,9 +16,9 @@ drawn per (tensor, batch, head, channel, f), eps ~ N(0, 1) per element, and the
 sum rounded to bf16 (round-to-nearest-even).  Every draw comes from a torch
 generator seeded with (seed, tensor id); the field is evaluated in fp32.
 
-Random numbers that the method itself draws (the per-step offset of the
-rotating anchor blocks) are also produced here and handed to both sides as an
-input.
+The method's own random draw (the per-step rotation of the anchor blocks of
+the structured rule) is not made here: the library and the oracle each
+implement the counter-based generator it is defined by.
 """
 from __future__ import annotations
 
@@ -54,6 +54,7 @@ class Workload:
     n_anchors: int = 4
     routing: bool = False
     compensate: bool = False
+    scorer: str = "pooled"            # "pooled" | "sics" (per-head block coherence)
     reuse_steps: int = 1              # mask reused over this many denoising steps
     sigma: float = 0.05               # Q/K perturbation between reused steps
     notes: str = ""
@@ -147,19 +148,6 @@ def qk_at_step(q0: torch.Tensor, k0: torch.Tensor, *, sigma: float, seed: int, s
         q = perturb(q, sigma=sigma, seed=seed, step=s, tensor=TENSOR_Q)
         k = perturb(k, sigma=sigma, seed=seed, step=s, tensor=TENSOR_K)
     return q, k
-
-
-def anchor_offset(*, seed: int, step: int, nkb: int, n_anchors: int) -> int:
-    """Per-step rotation offset of the global anchor blocks, in [0, nkb // n_anchors).
-
-    This is the one random draw the mask rule makes; it is passed to the
-    library and to the oracle as an input.
-    """
-    if n_anchors <= 0 or nkb <= 0:
-        return 0
-    stride = max(nkb // n_anchors, 1)
-    rng = np.random.Generator(np.random.Philox(key=[seed & 0xFFFFFFFFFFFFFFFF, step & 0xFFFFFFFFFFFFFFFF]))
-    return int(rng.integers(0, stride))
 
 
 def random_mask_lists(nb: int, rows: int, *, density: float, seed: int):
