@@ -47,7 +47,8 @@ class MaskParams(ctypes.Structure):
 class Mask(ctypes.Structure):
     _fields_ = [("kv_idx", ctypes.c_void_p), ("kv_cnt", ctypes.c_void_p), ("cap", ctypes.c_int32),
                 ("bits", ctypes.c_void_p), ("kbar", ctypes.c_void_p), ("vbar", ctypes.c_void_p),
-                ("nvalid", ctypes.c_void_p), ("cbar", ctypes.c_void_p), ("check", ctypes.c_int32)]
+                ("nvalid", ctypes.c_void_p), ("cbar", ctypes.c_void_p), ("pairs", ctypes.c_void_p),
+                ("check", ctypes.c_int32)]
 
 
 class Schedule(ctypes.Structure):
@@ -157,8 +158,9 @@ def mask_params(select: int = SEL_THRESHOLD, tau: float = 0.9, keep_frac: float 
 
 
 def make_mask(kv_idx, kv_cnt, cap: int, bits=None, kbar=None, vbar=None, nvalid=None, cbar=None,
-              check: bool = False) -> Mask:
-    return Mask(_p(kv_idx), _p(kv_cnt), cap, _p(bits), _p(kbar), _p(vbar), _p(nvalid), _p(cbar), int(check))
+              check: bool = False, pairs=None) -> Mask:
+    return Mask(_p(kv_idx), _p(kv_cnt), cap, _p(bits), _p(kbar), _p(vbar), _p(nvalid), _p(cbar), _p(pairs),
+                int(check))
 
 
 def svsa_anchor_offset(seed: int, step: int, nb: int, n_anchors: int) -> int:

@@ -54,6 +54,14 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, const in
                            const int32_t* kv_cnt, int cap, const uint32_t* bits, const void* cbar, void* o,
                            float* lse, long long BH, long long N, int nb, int d, bool dense, cudaStream_t st,
                            float* o32 = nullptr, float lse_empty = 0.f);
+cudaError_t launch_attn_fa(const void* q, const void* k, const void* v, const int32_t* kv_idx,
+                           const int32_t* kv_cnt, int cap, const uint32_t* bits, const void* cbar, void* o,
+                           float* lse, long long BH, long long N, int nb, int d, bool dense, cudaStream_t st,
+                           float* o32 = nullptr, float lse_empty = 0.f, const int32_t* pairs = nullptr);
+cudaError_t attn_fa_error(unsigned int* code, cudaStream_t st);
+size_t pair_table_bytes(long long BH, int nb);
+cudaError_t launch_pair(const uint32_t* bits, long long BH, int nb, int16_t* tab, int32_t* pairs,
+                        cudaStream_t st);
 cudaError_t launch_split_mask(const int32_t* kv_idx, const int32_t* kv_cnt, int cap, long long rows, int nb, int P,
                               int R, int32_t* idx_p, int32_t* cnt_p, cudaStream_t st);
 cudaError_t launch_combine(const float* o_p, const float* lse_p, long long rows, int P, int d, void* out,
@@ -67,6 +75,7 @@ cudaError_t launch_broadcast(const int32_t* hidx, const int32_t* hcnt, int hcap,
                              int32_t* kv_idx, int32_t* kv_cnt, uint32_t* bits, cudaStream_t st);
 cudaError_t launch_check_mask(const int32_t* kv_idx, const int32_t* kv_cnt, long long rows, int cap, int nb,
                               cudaStream_t st);
+cudaError_t launch_check_pairs(const int32_t* pairs, long long BH, int nb, cudaStream_t st);
 cudaError_t sics_flags(unsigned int* v, cudaStream_t st);
 cudaError_t reorder_flags(unsigned int* v, cudaStream_t st);
 cudaError_t pool_flags(unsigned int* v, cudaStream_t st);
@@ -136,7 +145,7 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // Workspace layout of svsa_build_mask.
 struct MaskWs {
-  size_t qsplit, ksplit, S, R, Rm, qbf, L, Mp, Zp, q64, k64, coh, hidx, hcnt, total;
+  size_t qsplit, ksplit, S, R, Rm, qbf, L, Mp, Zp, q64, k64, coh, hidx, hcnt, ptab, total;
 };
 
 MaskWs mask_ws_layout(const Dims& g, const svsa_mask_params& p, bool have_kbar) {
@@ -144,8 +153,12 @@ MaskWs mask_ws_layout(const Dims& g, const svsa_mask_params& p, bool have_kbar) 
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o = off; off += align256(bytes); return o; };
   const size_t f = sizeof(float);
+  // the query-block pairing's intersection table (used when mask.pairs is given)
+  w.ptab = take(pair_table_bytes(g.BH, g.nb));
   if (p.select == SVSA_SEL_STRUCTURED) {
-    w.total = 0;
+    w.qsplit = w.ksplit = w.S = w.R = w.Rm = w.qbf = w.L = w.Mp = w.Zp = w.q64 = w.k64 = SIZE_MAX;
+    w.coh = w.hidx = w.hcnt = SIZE_MAX;
+    w.total = off;
     return w;
   }
   if (p.scorer == SVSA_SCORE_SICS) {
@@ -420,11 +433,10 @@ size_t svsa_mask_workspace_bytes(svsa_shape s, const svsa_mask_params* p) {
   return mask_ws_layout(g, *p, false).total;
 }
 
-svsa_status svsa_build_mask(const void* qp, const void* kp, const void* vp, const int32_t* perm,
-                            svsa_shape s, const svsa_mask_params* p, const svsa_mask* m, void* ws,
-                            size_t ws_bytes, void* stream) {
-  NvtxRange nvtx_("svsa_build_mask");
-  g_last_error.clear();
+// The kept lists of svsa_build_mask (everything but the pairing).
+static svsa_status build_mask_lists(const void* qp, const void* kp, const void* vp, const int32_t* perm,
+                                    svsa_shape s, const svsa_mask_params* p, const svsa_mask* m, void* ws,
+                                    size_t ws_bytes, void* stream) {
   SVSA_TRY(check_shape(s, true));
   const Dims g = make_dims(s.B, s.heads, s.T, s.H, s.W, s.d);
   SVSA_TRY(check_params(p, g));
@@ -432,6 +444,10 @@ svsa_status svsa_build_mask(const void* qp, const void* kp, const void* vp, cons
   SVSA_PTR(m->kv_idx, "mask.kv_idx");
   SVSA_PTR(m->kv_cnt, "mask.kv_cnt");
   if (m->bits != nullptr && !aligned16(m->bits)) return fail(SVSA_ERR_INVALID_ARG, "mask.bits misaligned");
+  if (m->pairs != nullptr) {
+    if (!aligned16(m->pairs)) return fail(SVSA_ERR_INVALID_ARG, "mask.pairs misaligned");
+    if (m->bits == nullptr) return fail(SVSA_ERR_INVALID_ARG, "mask.pairs needs mask.bits (the pairing reads it)");
+  }
   if (m->kbar != nullptr && !aligned16(m->kbar)) return fail(SVSA_ERR_INVALID_ARG, "mask.kbar misaligned");
   if (m->vbar != nullptr && !aligned16(m->vbar)) return fail(SVSA_ERR_INVALID_ARG, "mask.vbar misaligned");
   if (m->nvalid != nullptr && !aligned16(m->nvalid)) return fail(SVSA_ERR_INVALID_ARG, "mask.nvalid misaligned");
@@ -453,7 +469,8 @@ svsa_status svsa_build_mask(const void* qp, const void* kp, const void* vp, cons
   if (m->vbar != nullptr) SVSA_PTR(vp, "vp (mask.vbar requested)");
   if (m->kbar != nullptr) SVSA_PTR(kp, "kp (mask.kbar requested)");
   const MaskWs w = mask_ws_layout(g, *p, m->kbar != nullptr);
-  if (w.total > 0) {
+  // (the structured rule uses the workspace only for the pairing table)
+  if (w.total > 0 && !(structured && m->pairs == nullptr)) {
     SVSA_PTR(ws, "ws");
     if (ws_bytes < w.total) return fail(SVSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, w.total);
   }
@@ -537,6 +554,19 @@ svsa_status svsa_build_mask(const void* qp, const void* kp, const void* vp, cons
                                            m->kv_cnt, m->bits, st), 1), "select");
 }
 
+svsa_status svsa_build_mask(const void* qp, const void* kp, const void* vp, const int32_t* perm,
+                            svsa_shape s, const svsa_mask_params* p, const svsa_mask* m, void* ws,
+                            size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_("svsa_build_mask");
+  g_last_error.clear();
+  SVSA_TRY(build_mask_lists(qp, kp, vp, perm, s, p, m, ws, ws_bytes, stream));
+  if (m->pairs == nullptr) return SVSA_OK;
+  const Dims g = make_dims(s.B, s.heads, s.T, s.H, s.W, s.d);
+  int16_t* tab = reinterpret_cast<int16_t*>(reinterpret_cast<char*>(ws) + mask_ws_layout(g, *p, false).ptab);
+  return cuda_status(counted(launch_pair(m->bits, g.BH, g.nb, tab, m->pairs, (cudaStream_t)stream), 2),
+                     "query-block pairing");
+}
+
 svsa_status svsa_attn_fwd(const void* qp, const void* kp, const void* vp, const svsa_mask* m,
                           int32_t compensate, void* op, float* lse, svsa_shape s, void* stream) {
   NvtxRange nvtx_("svsa_attn_fwd");
@@ -551,6 +581,7 @@ svsa_status svsa_attn_fwd(const void* qp, const void* kp, const void* vp, const 
   SVSA_PTR(m->kv_idx, "mask.kv_idx");
   SVSA_PTR(m->kv_cnt, "mask.kv_cnt");
   if (m->cap < 1) return fail(SVSA_ERR_INVALID_ARG, "mask.cap=%d", m->cap);
+  if (m->pairs != nullptr && !aligned16(m->pairs)) return fail(SVSA_ERR_INVALID_ARG, "mask.pairs misaligned");
   if (lse != nullptr && !aligned16(lse)) return fail(SVSA_ERR_INVALID_ARG, "lse misaligned");
   if (g.nb > kMaxBlocks) return fail(SVSA_ERR_UNSUPPORTED, "nb=%d exceeds %d", g.nb, kMaxBlocks);
   if (compensate) {
@@ -560,17 +591,21 @@ svsa_status svsa_attn_fwd(const void* qp, const void* kp, const void* vp, const 
     SVSA_PTR(m->cbar, "mask.cbar (compensation)");
   }
   if (op == qp || op == kp || op == vp) return fail(SVSA_ERR_INVALID_ARG, "op must not alias an input");
-  if (m->check)
+  if (m->check) {
     SVSA_TRY(cuda_status(counted(launch_check_mask(m->kv_idx, m->kv_cnt, g.BH * g.nb, m->cap, g.nb,
                                                    (cudaStream_t)stream), 1),
                          "mask check"));
+    if (m->pairs != nullptr)
+      SVSA_TRY(cuda_status(counted(launch_check_pairs(m->pairs, g.BH, g.nb, (cudaStream_t)stream), 1),
+                           "pairing check"));
+  }
   if (compensate)
     SVSA_TRY(cuda_status(counted(launch_centroid16(m->kbar, m->vbar, m->cbar, g.BH * g.nb, g.d,
                                                    (cudaStream_t)stream), 1),
                          "centroid copies"));
-  return cuda_status(counted(launch_attn_tc(qp, kp, vp, m->kv_idx, m->kv_cnt, m->cap, compensate ? m->bits : nullptr,
+  return cuda_status(counted(launch_attn_fa(qp, kp, vp, m->kv_idx, m->kv_cnt, m->cap, compensate ? m->bits : nullptr,
                                             compensate ? m->cbar : nullptr, op, lse, g.BH, g.N, g.nb, g.d, false,
-                                            (cudaStream_t)stream), 1),
+                                            (cudaStream_t)stream, nullptr, 0.f, m->pairs), 1),
                      "attn_fwd launch");
 }
 
@@ -617,6 +652,7 @@ svsa_status svsa_attn_fwd_split(const void* qp, const void* kp, const void* vp, 
   SVSA_PTR(m->kv_idx, "mask.kv_idx");
   SVSA_PTR(m->kv_cnt, "mask.kv_cnt");
   if (m->cap < 1) return fail(SVSA_ERR_INVALID_ARG, "mask.cap=%d", m->cap);
+  if (m->pairs != nullptr && !aligned16(m->pairs)) return fail(SVSA_ERR_INVALID_ARG, "mask.pairs misaligned");
   if (lse != nullptr && !aligned16(lse)) return fail(SVSA_ERR_INVALID_ARG, "lse misaligned");
   if (g.nb > kMaxBlocks) return fail(SVSA_ERR_UNSUPPORTED, "nb=%d exceeds %d", g.nb, kMaxBlocks);
   if (compensate) {
@@ -636,8 +672,11 @@ svsa_status svsa_attn_fwd_split(const void* qp, const void* kp, const void* vp, 
   float* lse_p = reinterpret_cast<float*>(base + w.lse);
   const long long rows = g.BH * g.nb;
   const int R = (g.nb + passes - 1) / passes;
-  if (m->check)
+  if (m->check) {
     SVSA_TRY(cuda_status(counted(launch_check_mask(m->kv_idx, m->kv_cnt, rows, m->cap, g.nb, st), 1), "mask check"));
+    if (m->pairs != nullptr)
+      SVSA_TRY(cuda_status(counted(launch_check_pairs(m->pairs, g.BH, g.nb, st), 1), "pairing check"));
+  }
   if (compensate)
     SVSA_TRY(cuda_status(counted(launch_centroid16(m->kbar, m->vbar, m->cbar, g.BH * g.nb, g.d, st), 1),
                          "centroid copies"));
@@ -647,10 +686,10 @@ svsa_status svsa_attn_fwd_split(const void* qp, const void* kp, const void* vp, 
   for (int p = 0; p < passes; ++p) {
     // the centroid tiles of the skipped blocks go with the last pass
     const bool comp = compensate && p + 1 == passes;
-    SVSA_TRY(cuda_status(counted(launch_attn_tc(qp, kp, vp, idx_p + (long long)p * rows * R, cnt_p + (long long)p * rows,
+    SVSA_TRY(cuda_status(counted(launch_attn_fa(qp, kp, vp, idx_p + (long long)p * rows * R, cnt_p + (long long)p * rows,
                                                  R, comp ? m->bits : nullptr, comp ? m->cbar : nullptr, nullptr,
                                                  lse_p + (long long)p * g.BH * g.Npad, g.BH, g.N, g.nb, g.d, false, st,
-                                                 o_p + (long long)p * g.BH * g.Npad * g.d, -INFINITY), 1),
+                                                 o_p + (long long)p * g.BH * g.Npad * g.d, -INFINITY, m->pairs), 1),
                          "attn_fwd pass launch"));
   }
   return cuda_status(counted(launch_combine(o_p, lse_p, g.BH * g.Npad, passes, g.d, op, lse, st), 1),
@@ -669,7 +708,7 @@ svsa_status svsa_attn_dense_fwd(const void* qp, const void* kp, const void* vp, 
   SVSA_PTR(op, "op");
   if (lse != nullptr && !aligned16(lse)) return fail(SVSA_ERR_INVALID_ARG, "lse misaligned");
   if (op == qp || op == kp || op == vp) return fail(SVSA_ERR_INVALID_ARG, "op must not alias an input");
-  return cuda_status(counted(launch_attn_tc(qp, kp, vp, nullptr, nullptr, 1, nullptr, nullptr, op, lse, g.BH, g.N,
+  return cuda_status(counted(launch_attn_fa(qp, kp, vp, nullptr, nullptr, 1, nullptr, nullptr, op, lse, g.BH, g.N,
                                             g.nb, g.d, true, (cudaStream_t)stream), 1),
                      "attn_dense_fwd launch");
 }
@@ -731,12 +770,12 @@ svsa_status svsa_sync_status(void* stream) {
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_status(e, "asynchronous error");
   // every tensor-core translation unit keeps its own error word; read (and clear) all of them
-  cudaError_t (*readers[4])(unsigned int*, cudaStream_t) = {attn_tc_error, scores_tc_error, route_tc_error,
-                                                           cocluster_tc_error};
-  const char* names[4] = {"attention", "scores", "routing", "co-clustering"};
+  cudaError_t (*readers[5])(unsigned int*, cudaStream_t) = {attn_fa_error, attn_tc_error, scores_tc_error,
+                                                           route_tc_error, cocluster_tc_error};
+  const char* names[5] = {"attention", "self-test", "scores", "routing", "co-clustering"};
   unsigned int first_code = 0u;
   const char* first_name = nullptr;
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < 5; ++i) {
     unsigned int code = 0u;
     e = readers[i](&code, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_status(e, "reading the device error word");
@@ -757,7 +796,8 @@ svsa_status svsa_sync_status(void* stream) {
     return fail(SVSA_ERR_TIMEOUT, "%s kernel: a bounded wait gave up (site %u)", first_name, first_code);
   if (bits & kFlagMask)
     return fail(SVSA_ERR_MASK, "a mask list checked before the attention was malformed "
-                               "(kv_cnt outside [0, cap], an index outside [0, nb) or not strictly ascending)");
+                               "(kv_cnt outside [0, cap], an index outside [0, nb), not strictly ascending, "
+                               "or a pairing table that is not a permutation)");
   if (bits & (kFlagRangeValue | kFlagRangeMean))
     return fail(SVSA_ERR_RANGE, "%s beyond the fp16 range (+-65504) or not finite; the result saturated",
                 (bits & kFlagRangeValue) ? "a value given to svsa_reorder_values" : "a block mean of the scores");

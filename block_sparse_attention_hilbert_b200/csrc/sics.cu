@@ -202,6 +202,33 @@ cudaError_t launch_check_mask(const int32_t* kv_idx, const int32_t* kv_cnt, long
   return cudaGetLastError();
 }
 
+// One CTA per head: the pairing table must be a permutation of 0..nb-1 (every
+// entry in range, none twice); a bit per block in shared memory catches a
+// repeat.  A bad table ORs kFlagMask into the status word.
+__global__ void __launch_bounds__(256) check_pairs_kernel(const int32_t* __restrict__ pairs, int nb) {
+  extern __shared__ uint32_t seen[];          // ceil(nb / 32) words
+  const int words = (nb + 31) / 32;
+  for (int w = threadIdx.x; w < words; w += 256) seen[w] = 0u;
+  __syncthreads();
+  const int32_t* row = pairs + (long long)blockIdx.x * nb;
+  bool bad = false;
+  for (int i = threadIdx.x; i < nb; i += 256) {
+    const int J = row[i];
+    if (J < 0 || J >= nb) {
+      bad = true;
+    } else {
+      const uint32_t bit = 1u << (J & 31);
+      bad |= (atomicOr(&seen[J >> 5], bit) & bit) != 0u;
+    }
+  }
+  if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(&g_sics_flags, kFlagMask);
+}
+
+cudaError_t launch_check_pairs(const int32_t* pairs, long long BH, int nb, cudaStream_t st) {
+  check_pairs_kernel<<<(unsigned)BH, 256, (size_t)((nb + 31) / 32) * sizeof(uint32_t), st>>>(pairs, nb);
+  return cudaGetLastError();
+}
+
 cudaError_t sics_flags(unsigned int* v, cudaStream_t st) { return read_and_clear_flags(g_sics_flags, v, st); }
 
 }  // namespace svsa

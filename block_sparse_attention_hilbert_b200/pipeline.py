@@ -38,7 +38,7 @@ class LayerBuffers:
     """Device buffers of one layer shape (all caller-owned, as the ABI requires)."""
 
     def __init__(self, B, heads, T, H, W, d, *, cap, need_means, keep_bits, ws_bytes, perm_ws_bytes,
-                 device, compensate=False):
+                 device, compensate=False, pair_blocks=False):
         N = T * H * W
         nb = -(-N // BLOCK)
         Npad = nb * BLOCK
@@ -56,18 +56,20 @@ class LayerBuffers:
         self.kbar = torch.empty(B, heads, nb, d, dtype=torch.float32, device=dev) if need_means else None
         self.vbar = torch.empty_like(self.kbar) if need_means else None
         self.nvalid = torch.empty(nb, dtype=torch.int32, device=dev) if need_means else None
-        # compensation: kept-block bitmap and the 16-bit centroid scratch of the attention
-        if compensate:
+        # compensation: kept-block bitmap and the 16-bit centroid scratch of the attention;
+        # the query-block pairing reads the bitmap too
+        if compensate or pair_blocks:
             keep_bits = True
         self.bits = (torch.empty(B, heads, nb, -(-nb // 32), dtype=torch.int32, device=dev)
                      if keep_bits else None)
         self.cbar = torch.empty(B, heads, nb, 2 * d, dtype=torch.int16, device=dev) if compensate else None
+        self.pairs = torch.empty(B, heads, nb, dtype=torch.int32, device=dev) if pair_blocks else None
         self.ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
         self.cap = cap
 
     def mask(self):
         return make_mask(self.kv_idx, self.kv_cnt, self.cap, self.bits, self.kbar, self.vbar, self.nvalid,
-                         self.cbar)
+                         self.cbar, pairs=self.pairs)
 
 
 class CapturedLayer:
@@ -97,7 +99,7 @@ class SparseVideoAttention:
     def __init__(self, B, heads, T, H, W, d, *, order="hilbert", select="threshold", tau=0.9,
                  keep_frac=0.25, sub_block=64, win_t=2, win_rows=1, n_anchors=0, routing=False,
                  compensate=False, keep_bits=False, schedule=None, cluster_rounds=3, attn_passes=None,
-                 seed=0, scorer="pooled", check_mask=False, device="cuda"):
+                 seed=0, scorer="pooled", check_mask=False, pair_blocks=True, device="cuda"):
         """order: "raster", "hilbert" or "cocluster" (a per-head semantic order from
         bidirectional query-key co-clustering, built from the first inputs and
         kept until `rebuild_order()`).  schedule: optional (n_steps, dense_steps,
@@ -111,7 +113,9 @@ class SparseVideoAttention:
         step index of each call picks the rotation).  scorer: "pooled" (block
         scores) or "sics" (per-head block coherence).  check_mask: validate
         the lists before every attention call (svsa_sync_status reports a
-        malformed one)."""
+        malformed one).  pair_blocks: let svsa_build_mask pair the query
+        blocks by kept-list overlap for the attention's 128-row items (else
+        blocks 2p and 2p + 1 go together)."""
         self.B, self.heads, self.T, self.H, self.W, self.d = B, heads, T, H, W, d
         self.N = T * H * W
         self.nb = -(-self.N // BLOCK)
@@ -134,7 +138,7 @@ class SparseVideoAttention:
         self.buf = LayerBuffers(B, heads, T, H, W, d, cap=cap, need_means=self.compensate or self.routing,
                                 keep_bits=keep_bits, ws_bytes=svsa_mask_workspace_bytes(self.shape, self.params),
                                 perm_ws_bytes=svsa_perm_workspace_bytes(self.shape, self.order),
-                                device=device, compensate=self.compensate)
+                                device=device, compensate=self.compensate, pair_blocks=pair_blocks)
         self._mask = self.buf.mask()
         self._mask.check = int(bool(check_mask))
         if attn_passes is None:
@@ -240,7 +244,8 @@ class SparseVideoAttention:
         sh = shape(1, r1 - r0, self.T, self.H, self.W, self.d)
         m = make_mask(self._rows(b.kv_idx, r0, r1), self._rows(b.kv_cnt, r0, r1), b.cap,
                       self._rows(b.bits, r0, r1), self._rows(b.kbar, r0, r1), self._rows(b.vbar, r0, r1),
-                      b.nvalid, self._rows(b.cbar, r0, r1), check=bool(self._mask.check))
+                      b.nvalid, self._rows(b.cbar, r0, r1), check=bool(self._mask.check),
+                      pairs=self._rows(b.pairs, r0, r1))
         return sh, m
 
     def forward_host(self, q, k, v, out, *, step: int = 0, reuse_mask: bool = False, groups: int = 12):

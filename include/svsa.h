@@ -129,10 +129,20 @@ typedef struct {
                              svsa_attn_fwd(compensate = 1), which first writes each
                              block's kbar (bf16, first d) and vbar (fp16, last d)
                              there; 16-byte aligned; not read by svsa_build_mask */
+  int32_t* pairs;         /* nullable [B, heads, nb]: the query blocks of each head in
+                             the order the attention takes them, two at a time (each
+                             item is 128 query rows walking the union of two kept
+                             lists, so partners that share kept blocks waste less).
+                             When non-NULL, svsa_build_mask fills it (a greedy pairing
+                             by kept-list overlap; needs bits) and svsa_attn_fwd reads
+                             it; it must be a permutation of 0..nb-1 per head (a caller
+                             that writes kv_idx itself passes NULL or its own table).
+                             NULL: the attention pairs blocks 2p and 2p + 1. */
   int32_t check;          /* svsa_attn_fwd only: nonzero = first validate every list
                              (kv_cnt in [0, cap], indices in [0, nb), strictly
-                             ascending) in a kernel of its own and record a malformed
-                             one for svsa_sync_status (SVSA_ERR_MASK).  The attention
+                             ascending) and the pairing table when given (a
+                             permutation per head) in kernels of their own and record
+                             a malformed one for svsa_sync_status (SVSA_ERR_MASK).  The attention
                              still runs, and clamps counts and indices to the tensors,
                              so a bad list gives a wrong output but no stray access. */
 } svsa_mask;

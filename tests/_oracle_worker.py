@@ -1,6 +1,5 @@
-"""Whole-head oracle evaluation for the full-size parity tests, run in a
-`spawn` process pool (one head per task).  Imports only numpy and `oracle/`:
-the workers never touch torch or the GPU."""
+"""Whole-head oracle evaluation for the full-size parity tests (one head per
+call).  Imports only numpy and `oracle/`: it never touches torch or the GPU."""
 from __future__ import annotations
 
 import numpy as np

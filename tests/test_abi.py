@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol():
 def test_struct_sizes_match_header():
     assert ctypes.sizeof(Shape) == 24
     assert ctypes.sizeof(MaskParams) == 48
-    assert ctypes.sizeof(Mask) == 72
+    assert ctypes.sizeof(Mask) == 80
 
 
 def test_struct_layouts_match_the_c_compiler(tmp_path):
@@ -102,7 +102,8 @@ def test_workspace_queries():
     nb = 512
     p = svsa.mask_params(svsa.SEL_TOPK)
     assert svsa.svsa_mask_workspace_bytes(s, p) >= 12 * nb * nb * 4
-    assert svsa.svsa_mask_workspace_bytes(s, svsa.mask_params(svsa.SEL_STRUCTURED)) == 0
+    # the structured rule needs workspace only for the query-block pairing table ([BH, nb, 32] int16)
+    assert svsa.svsa_mask_workspace_bytes(s, svsa.mask_params(svsa.SEL_STRUCTURED)) >= 12 * nb * 32 * 2
     p16 = svsa.mask_params(svsa.SEL_THRESHOLD, sub_block=16)
     assert svsa.svsa_mask_workspace_bytes(s, p16) > svsa.svsa_mask_workspace_bytes(s, p)
     assert svsa.svsa_mask_workspace_bytes(s, svsa.mask_params(sub_block=32)) == 0
@@ -138,7 +139,7 @@ def test_reorder_and_attention_reject_before_launch():
     assert lib.svsa_inverse_reorder(None, 32, 48, s, None) == 1
     m = Mask(None, None, 4, None, None, None, None, None)
     assert lib.svsa_attn_fwd(16, 32, 48, ctypes.byref(m), 0, 64, None, s, None) == 1
-    m = Mask(16, 32, 4, None, None, None, None, None, 0)
+    m = Mask(16, 32, 4, None, None, None, None, None, None, 0)
     assert lib.svsa_attn_fwd(16, 32, 48, ctypes.byref(m), 1, 64, None, s, None) == 1   # comp w/o means
     assert "kbar" in _err()
     kb = 80
@@ -155,10 +156,10 @@ def test_reorder_and_attention_reject_before_launch():
 def test_build_mask_rejects_before_launch():
     lib = _raw()
     s = svsa.shape(1, 2, 4, 8, 8, 128)                                    # nb = 4
-    m = Mask(16, 32, 4, None, None, None, None, None, 0)
+    m = Mask(16, 32, 4, None, None, None, None, None, None, 0)
     ok = svsa.mask_params(svsa.SEL_THRESHOLD)
     # capacity below nb for a threshold rule
-    small = Mask(16, 32, 3, None, None, None, None, None, 0)
+    small = Mask(16, 32, 3, None, None, None, None, None, None, 0)
     assert lib.svsa_build_mask(16, 32, None, None, s, ctypes.byref(ok), ctypes.byref(small), 64, 1 << 20, None) == 1
     # routing without V / means
     r = svsa.mask_params(svsa.SEL_THRESHOLD, routing=True)

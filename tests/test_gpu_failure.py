@@ -94,7 +94,7 @@ def test_block_means_beyond_fp16_are_reported_as_range():
     w = workloads.WORKLOADS["tiny"]
     q, k, v = (t.cuda() for t in workloads.make_qkv(w))
     q2 = q.clone()
-    q2[0, 0, :64, 3] = 9.0e4                                      # a whole block: its mean is 9e4
+    q2[0, 0, :, 3] = 9.0e4                                        # every block's mean is 9e4 in this channel
     attn = svsa.SparseVideoAttention(w.B, w.heads, w.T, w.H, w.W, w.d, order=w.order, select=w.select, tau=w.tau)
     attn(q, k, v)
     assert lib.svsa_sync_status(_stream()) == 0
@@ -142,6 +142,15 @@ def test_malformed_masks_are_reported(defect):
     assert lib.svsa_sync_status(_stream()) == 7                   # SVSA_ERR_MASK
     assert "malformed" in lib.svsa_last_error().decode()
     assert lib.svsa_sync_status(_stream()) == 0
+    # a pairing table that is not a permutation
+    pairs = torch.arange(nb, dtype=torch.int32, device="cuda").repeat(B * heads, 1).reshape(B, heads, nb)
+    goodp = svsa.make_mask(kv_idx, kv_cnt, cap, check=True, pairs=pairs)
+    svsa.svsa_attn_fwd(qp, kp, vp, goodp, False, op, None, s)
+    assert lib.svsa_sync_status(_stream()) == 0
+    badp = pairs.clone()
+    badp[0, 1, 5] = badp[0, 1, 2]
+    svsa.svsa_attn_fwd(qp, kp, vp, svsa.make_mask(kv_idx, kv_cnt, cap, check=True, pairs=badp), False, op, None, s)
+    assert lib.svsa_sync_status(_stream()) == 7
     # without the check the same call is not validated (and still stays in bounds)
     unchecked = svsa.make_mask(bad_idx, bad_cnt, cap)
     svsa.svsa_attn_fwd(qp, kp, vp, unchecked, False, op, None, s)

@@ -7,6 +7,7 @@ import torch
 import oracle
 import workloads
 import block_sparse_attention_hilbert_b200 as svsa
+from block_sparse_attention_hilbert_b200 import SparseVideoAttention
 from _parity import (check_attention, compare_mask_rows, gpu_keep, gpu_layer, oracle_rows, to_np)
 
 pytestmark = pytest.mark.gpu
@@ -73,6 +74,10 @@ def test_reorder_values_fp16_bit_exact(d):
     attn.build_perm()
     b = attn.buf
     svsa.svsa_reorder_values(v, b.vp, b.perm, attn.shape)
+    # the two saturating values are reported (SVSA_ERR_RANGE), and the status clears
+    with pytest.raises(svsa.SvsaError) as err:
+        svsa.svsa_sync_status()
+    assert err.value.status == 6
     svsa.svsa_sync_status()
     perm, _ = oracle.build_perm(T, H, W, "hilbert")
     vf16 = v.float().clamp(-65504, 65504).to(torch.float16).cpu()
@@ -334,7 +339,10 @@ def test_dense_and_random_masks(d):
     T, H, W = 5, 7, 9
     w = _small("topk", 64, grid=(T, H, W), heads=2, d=d)
     q, k, v = (t.cuda() for t in workloads.make_qkv(w, seed=4))
-    attn = svsa.SparseVideoAttention(1, 2, T, H, W, d, order="hilbert", select="threshold", tau=1.0)
+    # the lists are written here, not by svsa_build_mask, so no pairing table
+    # (the attention then pairs query blocks 2p and 2p + 1)
+    attn = svsa.SparseVideoAttention(1, 2, T, H, W, d, order="hilbert", select="threshold", tau=1.0,
+                                     pair_blocks=False)
     attn.reorder(q, k, v)
     b = attn.buf
     perm, _ = oracle.build_perm(T, H, W, "hilbert")
@@ -648,3 +656,43 @@ def test_captured_layer_replays_the_eager_call(select, kw):
         ref = gpu_layer(w, q2, k2, v2).out                 # a fresh layer, eager
         assert torch.equal(out, ref), f"seed {seed}: replay differs from the eager call"
     svsa.svsa_sync_status()
+
+
+@pytest.mark.parametrize("select,kw", [("topk", {}), ("threshold", dict(sub=16)),
+                                       ("threshold", dict(routing=True, compensate=True))])
+def test_query_block_pairing(select, kw):
+    """The pairing svsa_build_mask writes (mask.pairs) is a permutation of the
+    query blocks of every head, pairs blocks that share kept key blocks at
+    least as well as the plain adjacent pairs do, and the attention on it
+    matches both the unpaired call and the oracle."""
+    w = _small(select, grid=(7, 13, 21), heads=2, tau=0.9, keep_frac=0.3, **kw)   # nb = 30
+    q, k, v = (t.cuda() for t in workloads.make_qkv(w, seed=4))
+    mk = lambda pair: SparseVideoAttention(w.B, w.heads, w.T, w.H, w.W, w.d, order=w.order, select=w.select,
+                                           tau=w.tau, keep_frac=w.keep_frac, sub_block=w.sub_block,
+                                           routing=w.routing, compensate=w.compensate, pair_blocks=pair,
+                                           keep_bits=True, device="cuda")
+    paired, plain = mk(True), mk(False)
+    out_p, out_u = paired(q, k, v), plain(q, k, v)
+    torch.cuda.synchronize()
+    nb = paired.nb
+    pairs = paired.buf.pairs.cpu().numpy().reshape(w.heads, nb)
+    keep = gpu_keep(paired)
+    assert np.array_equal(keep, gpu_keep(plain))
+    for eta in range(w.heads):
+        assert np.array_equal(np.sort(pairs[eta]), np.arange(nb))
+        shared = sum((keep[eta, pairs[eta, i]] & keep[eta, pairs[eta, i + 1]]).sum() for i in range(0, nb - 1, 2))
+        adjacent = sum((keep[eta, i] & keep[eta, i + 1]).sum() for i in range(0, nb - 1, 2))
+        assert shared >= adjacent
+    check_attention(to_np(out_p), to_np(out_u), "paired vs unpaired")
+    perm, _ = oracle.build_perm(w.T, w.H, w.W, w.order)
+    qp, kp, vp = (oracle.reorder(to_np(t)[0].astype(np.float64), perm) for t in (q, k, v))
+    op = to_np(paired.buf.op)[0]
+    for eta in range(w.heads):
+        if w.compensate:
+            kb, nv = oracle.pool(kp[eta], w.N)
+            vb, _ = oracle.pool(vp[eta], w.N)
+            ref = oracle.compensated_attention(qp[eta], kp[eta], vp[eta], w.N, keep[eta], kb, vb, nv)
+        else:
+            ref = oracle.masked_attention(qp[eta], kp[eta], vp[eta], w.N, keep[eta])
+        gout = np.concatenate([op[eta][I * 64:min(I * 64 + 64, w.N)] for I in range(nb)])
+        check_attention(gout, np.concatenate([ref[I] for I in range(nb)]), f"head {eta}")
