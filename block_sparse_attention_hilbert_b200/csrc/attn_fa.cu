@@ -17,8 +17,9 @@
 //        S [128 q x 128 k]  = Q [128 x d] . K_pair^T        (A, B from smem, K-major)
 //        O [128 q x d]     += P [128 x 128] . V_pair [128 x d]
 //     with P in tensor memory (the A operand), V from smem (MN-major).
-//   * TMEM: three S buffers of 128 columns, P written over the first 64
-//     columns of its own S buffer (fp16 pairs), and O (d columns).
+//   * TMEM: two S buffers of 128 columns; each half of a tile (64 keys) writes
+//     its P as fp16 pairs over the first 32 of its own 64 S columns; two
+//     accumulators O_A, O_B (d columns each), one per half.
 //   * Warp roles: warp 0 TMA of Q (once per item) and of the K tiles, warp 1
 //     TMA of the V tiles, warp 2 issues the S products and owns TMEM, warp 3
 //     issues the P.V products, warps 4-7 are the softmax warpgroup: thread t
@@ -51,7 +52,7 @@ namespace fa {
 using namespace tc;
 
 constexpr int kThreads = 384;                 // 4 role warps + 2 softmax warpgroups
-constexpr int kQBufs = 1, kKStages = 3, kVStages = 2, kSBufs = 3;
+constexpr int kQBufs = 1, kKStages = 3, kVStages = 2, kSBufs = 2;
 constexpr uint32_t kBox = 8192;                 // one 64-row x 128-byte TMA box
 constexpr uint32_t kSlot = 32768;               // one 128-row tile (d = 128; d = 64 uses half)
 constexpr float kLazyTh = 12.0f;                // log2 headroom before a rescale (fp16 P <= 2^12)
@@ -64,13 +65,14 @@ constexpr uint32_t kSmemBytes = kOffMisc + 4096 + 1024;     // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 384;                 // S buffers at 0, 128, 256
+constexpr uint32_t kColO = 256;                 // S buffers at 0, 128; O_A at 256, O_B at 256 + d
 
 enum : uint32_t {
   BAR_Q_FULL = 0, BAR_Q_EMPTY = BAR_Q_FULL + kQBufs,
   BAR_K_FULL = BAR_Q_EMPTY + kQBufs, BAR_K_EMPTY = BAR_K_FULL + kKStages,
   BAR_V_FULL = BAR_K_EMPTY + kKStages, BAR_V_EMPTY = BAR_V_FULL + kVStages,
-  BAR_S_FULL = BAR_V_EMPTY + kVStages, BAR_P_FULL = BAR_S_FULL + kSBufs, BAR_SP_FREE = BAR_P_FULL + kSBufs,
+  BAR_S_FULL = BAR_V_EMPTY + kVStages, BAR_P_FULL = BAR_S_FULL + kSBufs,   // P_FULL: [2 halves][kSBufs]
+  BAR_SP_FREE = BAR_P_FULL + 2 * kSBufs,
   BAR_O_FULL = BAR_SP_FREE + kSBufs, BAR_O_EMPTY, BAR_FINAL, BAR_FINAL2, NUM_BARS
 };
 
@@ -78,8 +80,8 @@ struct Misc {
   uint64_t bar[NUM_BARS];
   uint32_t tmem_base;
   uint32_t abort;
-  float xch[6 * 128];               // exchanged by the two threads of a row: half maxima of even /
-                                    // odd tiles, then the item's partial row sums
+  float xch[4 * 128];               // exchanged by the two threads of a row at the end of an item:
+                                    // [m, l] of each half
 };
 static_assert(sizeof(Misc) <= 4096, "misc region");
 
@@ -193,6 +195,15 @@ struct Tiles {
     ncent = nc;
   }
   __device__ __forceinline__ bool empty() const { return J1 < 0 && ncent == 0; }
+  // the next union tile only (false once the union is done)
+  __device__ __forceinline__ bool next_union(int& j1, int& j2, uint32_t& fl1, uint32_t& fl2) {
+    if (J1 < 0) return false;
+    j1 = J1;
+    fl1 = f1;
+    j2 = m.next(fl2);
+    J1 = j2 >= 0 ? m.next(f1) : -1;
+    return true;
+  }
   // false when the item is done; c = -1 for a union tile, else the centroid tile index
   __device__ __forceinline__ bool next(int& j1, int& j2, uint32_t& fl1, uint32_t& fl2, int& c) {
     if (J1 >= 0) {
@@ -296,7 +307,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fa_kernel(const __grid_const
     }
     for (int i = 0; i < kSBufs; ++i) {
       mbar_init(bar(BAR_S_FULL + i), 1);
-      mbar_init(bar(BAR_P_FULL + i), 8);
+      mbar_init(bar(BAR_P_FULL + i), 4);               // the first half's warpgroup
+      mbar_init(bar(BAR_P_FULL + kSBufs + i), 4);      // the second half's
       mbar_init(bar(BAR_SP_FREE + i), 1);
     }
     mbar_init(bar(BAR_O_FULL), 1);
@@ -449,15 +461,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fa_kernel(const __grid_const
           while (ok && ti.next(j1, j2, fl1, fl2, cix)) {
             const uint32_t vs = ring % kVStages, sb = j % kSBufs;
             ok = wait_bar(bar(BAR_V_FULL + vs), (ring / kVStages) & 1u, abort_flag, 7) &&
-                 wait_bar(bar(BAR_P_FULL + sb), (j / kSBufs) & 1u, abort_flag, 8) &&
                  (t > 0 || wait_bar(bar(BAR_O_EMPTY), (oit & 1u) ^ 1u, abort_flag, 9));
-            if (!ok) break;
-            tc_fence_after();
             const uint64_t b0 = dV + ((vs * kSlot) >> 4);
+            // each half's keys (64) into that half's accumulator, as soon as its P is ready
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              umma_f16_ts(tmem + kColO, tmem + sb * 128 + kk * 8, b0 + ((kk * 2048) >> 4), ID_O,
-                          (t > 0 || kk > 0) ? 1u : 0u);
+            for (int h = 0; h < 2 && ok; ++h) {
+              ok = wait_bar(bar(BAR_P_FULL + h * kSBufs + sb), (j / kSBufs) & 1u, abort_flag, 8);
+              if (!ok) break;
+              tc_fence_after();
+              // (half h's P sits over the first 32 columns of its own 64 S columns)
+#pragma unroll
+              for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
+                umma_f16_ts(tmem + kColO + h * D, tmem + sb * 128 + 64 * h + (kk - 4 * h) * 8,
+                            b0 + ((kk * 2048) >> 4), ID_O, (t > 0 || kk > 4 * h) ? 1u : 0u);
+            }
+            if (!ok) break;
             umma_commit(bar(BAR_V_EMPTY + vs));
             umma_commit(bar(BAR_SP_FREE + sb));
             ++ring;
@@ -479,25 +497,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fa_kernel(const __grid_const
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     // Query row `row` (0..127) is shared by two threads: warp 4 + q of the
-    // first warpgroup takes the tile's first key block (columns 0-63), warp
-    // 8 + q of the second the second block (columns 64-127), both on TMEM
-    // lane quadrant q.  Rows 0-63 are block I0, rows 64-127 block I1, so every
-    // validity decision is uniform across a warp.  The two threads of a row
-    // exchange their half maxima through shared memory (double-buffered by
-    // tile parity, a 64-thread named barrier per quadrant), so both take the
-    // same reference-maximum decisions; each keeps a partial row sum and
-    // rescales / stores its own half of the O row.
+    // first warpgroup takes the first key block of every tile (columns 0-63
+    // of S, accumulator O_A), warp 8 + q of the second the second block
+    // (columns 64-127, O_B), both on TMEM lane quadrant q.  Each half runs an
+    // online softmax of its own -- reference maximum, row sum, accumulator --
+    // so the two never synchronise inside an item; at the item's end the two
+    // partial results are merged as O = (O_A 2^(m_A - m) + O_B 2^(m_B - m)) /
+    // (l_A 2^(m_A - m) + l_B 2^(m_B - m)), m = max(m_A, m_B), the softmax over
+    // the union of two disjoint key sets.  Rows 0-63 are block I0, rows
+    // 64-127 block I1, so every validity decision is uniform across a warp.
     const int wq = warp & 3;                       // TMEM lane quadrant
-    const int half = warp >= 8 ? 1 : 0;            // which key block of the tile, which half of O
+    const int half = warp >= 8 ? 1 : 0;            // which key block of the tile, which accumulator
     const int row = wq * 32 + lane;
     const uint32_t mine = row < 64 ? 0u : 1u;      // bit of the union flags for this row's block
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t qbar = 1u + (uint32_t)wq;       // named barrier of the quadrant's two warps
-    constexpr int DH = D / 2;                      // O columns per thread
+    constexpr int DH = D / 2;                      // output columns this thread stores
+    const uint32_t col_own = kColO + half * D;     // this half's accumulator
     const float sl2 = a.scale_log2;
     const int n_last = (int)(a.N - (long long)(nb - 1) * kBlock);   // valid keys of block nb - 1
     const float bias_last = __log2f((float)n_last);
-    float* xch = ms->xch;                          // [3 uses][2 halves][128 rows]
+    float* xch = ms->xch;                          // [m, l][2 halves][128 rows]
     uint32_t j = 0, oit = 0;
     bool stop = false;
     for (long long it = blockIdx.x; it < items && !stop; it += gridDim.x) {
@@ -510,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fa_kernel(const __grid_const
       Tiles ti;
       ti.init(a, bh, I0, I1, ncent);
       if (ti.empty()) {
-        // nothing kept by either block: zero output rows (each thread its half)
+        // nothing kept by either block: zero output rows (each thread its half of the columns)
         if (q >= 0) {
           if (O32) {
             float4* og = reinterpret_cast<float4*>(a.o32 + (bh * a.Npad + q) * D + half * DH);
@@ -523,206 +543,231 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fa_kernel(const __grid_const
         }
         continue;
       }
+      // (the reference stays finite before the first valid score, so that a
+      // fully masked tile gives exp2(-inf - 0) = 0, never -inf - (-inf))
       bool have_ref = false;
       float mref = 0.f, l = 0.f;
-      int j1, j2, cix;
-      uint32_t fl1, fl2;
-      while (ti.next(j1, j2, fl1, fl2, cix)) {
-        const uint32_t sb = j % kSBufs;
-        const int Jh = half ? j2 : j1;
-        const uint32_t flh = half ? fl2 : fl1;
-        // centroid tile: this row's block's kept bits for this half's 64 means
-        uint32_t kw[2] = {0u, 0u};
-        if (COMP && cix >= 0 && Im >= 0) {
+      // the union tiles, then (with compensation) the centroid tiles: the
+      // phase loop is unrolled so that each phase's tile loop is compiled for
+      // its own kind of tile and the union loop carries no centroid code
+      int cnext = 0;
 #pragma unroll
-          for (int w = 0; w < 2; ++w) {
-            const int word = cix * 4 + half * 2 + w;
-            kw[w] = word < a.nwords ? a.bits[(bh * nb + Im) * a.nwords + word] : ~0u;
-          }
-        }
-        // (every decision that guards a TMEM access or a warp sync is made
-        // warp-uniform -- tcgen05.ld / st are warp-collective -- and every
-        // exit is agreed by the row's two warps at an OR-barrier that both
-        // reach, so neither waits at a named barrier the other has left)
-        const bool ok = __all_sync(0xffffffffu, wait_bar(bar(BAR_S_FULL + sb), (j / kSBufs) & 1u, abort_flag, 10));
+      for (int phase = 0; phase < (COMP ? 2 : 1); ++phase) {
+        const bool cent = phase == 1;
         float s[64];
-        float hmax = -INFINITY;
-        bool cheap = false, dead = true;
-        if (ok) {
+        while (true) {
+          int j1 = -1, j2 = -1, cix = -1;
+          uint32_t fl1 = 0u, fl2 = 0u;
+          if (!cent) {
+            if (!ti.next_union(j1, j2, fl1, fl2)) break;
+          } else {
+            if (cnext >= ncent) break;
+            cix = cnext++;
+          }
+          const uint32_t sb = j % kSBufs;
+          const int Jh = half ? j2 : j1;
+          const uint32_t flh = half ? fl2 : fl1;
+          // centroid tile: this row's block's kept bits for this half's 64 means
+          uint32_t kw[2] = {0u, 0u};
+          if (COMP && cent && Im >= 0) {
+#pragma unroll
+            for (int w = 0; w < 2; ++w) {
+              const int word = cix * 4 + half * 2 + w;
+              kw[w] = word < a.nwords ? a.bits[(bh * nb + Im) * a.nwords + word] : ~0u;
+            }
+          }
+          // (every decision that guards a TMEM access or a warp sync is made
+          // warp-uniform: tcgen05.ld / st are warp-collective)
+          if (!__all_sync(0xffffffffu, wait_bar(bar(BAR_S_FULL + sb), (j / kSBufs) & 1u, abort_flag, 10))) {
+            stop = true;
+            break;
+          }
           tc_fence_after();
           tmem_ld32(tmem + lane_off + sb * 128 + 64 * half, s);
           tmem_ld32(tmem + lane_off + sb * 128 + 64 * half + 32, s + 32);
           tmem_wait_ld();
-        }
-        // scaled scores (log2 units) with masked columns at -inf, and their maximum
-        if (!ok) {
-        } else if (COMP && cix >= 0) {
-#pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const int J = cix * 128 + 64 * half + c;
-            const bool ok_c = Im >= 0 && J < nb && ((kw[c >> 5] >> (c & 31)) & 1u) == 0u;
-            const float bias = J == nb - 1 ? bias_last : 6.0f;        // log2 n_J
-            s[c] = ok_c ? fmaf(s[c], sl2, bias) : -INFINITY;
-            hmax = fmaxf(hmax, s[c]);
-          }
-          dead = false;
-        } else if (Jh >= 0 && ((flh >> mine) & 1u) != 0u && Im >= 0) {
-          dead = false;
-          if (Jh != nb - 1 || n_last == kBlock) {
-            cheap = true;
-            float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 64; c += 8) {
-              m0 = max3(m0, s[c], s[c + 1]);
-              m1 = max3(m1, s[c + 2], s[c + 3]);
-              m2 = max3(m2, s[c + 4], s[c + 5]);
-              m3 = max3(m3, s[c + 6], s[c + 7]);
-            }
-            hmax = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * sl2;
-          } else {
-            // the ragged last block: keys past n_last are pads
+          // scaled scores (log2 units) with masked columns at -inf, and their maximum
+          float tmax = -INFINITY;
+          bool cheap = false, dead = true;
+          if (COMP && cent) {
 #pragma unroll
             for (int c = 0; c < 64; ++c) {
-              s[c] = c < n_last ? s[c] * sl2 : -INFINITY;
-              hmax = fmaxf(hmax, s[c]);
+              const int J = cix * 128 + 64 * half + c;
+              const bool ok_c = Im >= 0 && J < nb && ((kw[c >> 5] >> (c & 31)) & 1u) == 0u;
+              const float bias = J == nb - 1 ? bias_last : 6.0f;        // log2 n_J
+              s[c] = ok_c ? fmaf(s[c], sl2, bias) : -INFINITY;
+              tmax = fmaxf(tmax, s[c]);
             }
-          }
-        }
-        // the row's maximum over both halves (and the two warps' exit decision)
-        xch[((j & 1u) * 2 + half) * 128 + row] = hmax;
-        if (named_bar_or(qbar, 64, stop || !ok)) {
-          stop = true;
-          break;
-        }
-        const float tmax = fmaxf(hmax, xch[((j & 1u) * 2 + (half ^ 1)) * 128 + row]);
-        // the reference maximum: set by the first tile with a valid score,
-        // raised (with a rescale of the row sum and of the O row) only when a
-        // score exceeds it by more than 2^kLazyTh; both threads of a row see
-        // the same tmax and make the same decisions
-        float alpha = 1.f;
-        if (tmax > -INFINITY) {
-          if (!have_ref) {
-            mref = tmax;
-            have_ref = true;
-          } else if (tmax > mref + kLazyTh) {
-            alpha = ex2(mref - tmax);
-            l *= alpha;
-            mref = tmax;
-          }
-        }
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
-          // the whole warp rescales its half of the O rows (factor 1 where
-          // nothing changed) once the previous P.V has finished: O holds the
-          // previous tiles' sum then (its slot barrier; the same item, since
-          // a raised reference needs an earlier tile)
-          const uint32_t jp = j - 1u, sp = jp % kSBufs;
-          if (!__all_sync(0xffffffffu, wait_bar(bar(BAR_SP_FREE + sp), (jp / kSBufs) & 1u, abort_flag, 11))) {
-            stop = true;
-          } else {
-            tc_fence_after();
+            dead = false;
+          } else if (Jh >= 0 && ((flh >> mine) & 1u) != 0u && Im >= 0) {
+            dead = false;
+            if (Jh != nb - 1 || n_last == kBlock) {
+              cheap = true;
+              float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-            for (int c0 = 0; c0 < DH; c0 += 32) {
-              float o[32];
-              tmem_ld32(tmem + lane_off + kColO + half * DH + c0, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int c = 0; c < 32; ++c) o[c] *= alpha;
-              tmem_st32(tmem + lane_off + kColO + half * DH + c0, o);
-            }
-            tmem_wait_st();
-          }
-        }
-        // P = exp2(y - m) as fp16 pairs: this half's 32 columns of the S buffer's P region
-        uint32_t pk[32];
-        float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
-        const float nm = -mref;
-        if (dead) {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) pk[c] = 0u;
-        } else if (cheap) {
-#pragma unroll
-          for (int c = 0; c < 64; c += 4) {
-            float y0 = s[c], y1 = s[c + 1], y2 = s[c + 2], y3 = s[c + 3];
-            fma2(y0, y1, sl2, nm, nm);
-            fma2(y2, y3, sl2, nm, nm);
-            float p0, p1, p2, p3;
-            if (SVSA_FA_POLY_EVERY > 0 && (c >> 2) % (SVSA_FA_POLY_EVERY > 0 ? SVSA_FA_POLY_EVERY : 1) ==
-                                              (SVSA_FA_POLY_EVERY > 0 ? SVSA_FA_POLY_EVERY - 1 : 0)) {
-              p0 = y0; p1 = y1;
-              exp2_fma2(p0, p1);
+              for (int c = 0; c < 64; c += 8) {
+                m0 = max3(m0, s[c], s[c + 1]);
+                m1 = max3(m1, s[c + 2], s[c + 3]);
+                m2 = max3(m2, s[c + 4], s[c + 5]);
+                m3 = max3(m3, s[c + 6], s[c + 7]);
+              }
+              tmax = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * sl2;
             } else {
-              p0 = ex2(y0);
-              p1 = ex2(y1);
-            }
-            p2 = ex2(y2);
-            p3 = ex2(y3);
-            add2(ls0, ls1, p0, p1);
-            add2(ls2, ls3, p2, p3);
-            pk[c >> 1] = pack_f16x2(p0, p1);
-            pk[(c >> 1) + 1] = pack_f16x2(p2, p3);
-          }
-        } else {
+              // the ragged last block: keys past n_last are pads
 #pragma unroll
-          for (int c = 0; c < 64; c += 2) {
-            const float p0 = ex2(s[c] + nm), p1 = ex2(s[c + 1] + nm);
-            add2(ls0, ls1, p0, p1);
-            pk[c >> 1] = pack_f16x2(p0, p1);
+              for (int c = 0; c < 64; ++c) {
+                s[c] = c < n_last ? s[c] * sl2 : -INFINITY;
+                tmax = fmaxf(tmax, s[c]);
+              }
+            }
           }
+          // this half's reference maximum: set by its first tile with a valid
+          // score, raised (with a rescale of its row sum and accumulator row)
+          // only when a score exceeds it by more than 2^kLazyTh
+          float alpha = 1.f;
+          if (tmax > -INFINITY) {
+            if (!have_ref) {
+              mref = tmax;
+              have_ref = true;
+            } else if (tmax > mref + kLazyTh) {
+              alpha = ex2(mref - tmax);
+              l *= alpha;
+              mref = tmax;
+            }
+          }
+          if (__any_sync(0xffffffffu, alpha != 1.f)) {
+            // the warp rescales its rows of this half's accumulator (factor 1
+            // where nothing changed) once the previous P.V products have
+            // finished: the accumulator holds the previous tiles' sum then
+            // (their slot barrier; the same item, since a raised reference
+            // needs an earlier tile)
+            const uint32_t jp = j - 1u, sp = jp % kSBufs;
+            if (!__all_sync(0xffffffffu, wait_bar(bar(BAR_SP_FREE + sp), (jp / kSBufs) & 1u, abort_flag, 11))) {
+              stop = true;
+            } else {
+              tc_fence_after();
+#pragma unroll
+              for (int c0 = 0; c0 < D; c0 += 32) {
+                float o[32];
+                tmem_ld32(tmem + lane_off + col_own + c0, o);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; ++c) o[c] *= alpha;
+                tmem_st32(tmem + lane_off + col_own + c0, o);
+              }
+              tmem_wait_st();
+            }
+          }
+          // P = exp2(y - m) as fp16 pairs over the first 32 of this half's own 64 S
+          // columns (never over the other half's scores, which may not be read yet)
+          uint32_t pk[32];
+          float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
+          const float nm = -mref;
+          if (dead) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) pk[c] = 0u;
+          } else if (cheap) {
+            // packed fp32 pairs (sm_100 f32x2 instructions, each rounding as its scalar form)
+            const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(nm, nm);
+            float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int c = 0; c < 64; c += 4) {
+              const float2 y01 = __ffma2_rn(make_float2(s[c], s[c + 1]), sc2, nm2);
+              const float2 y23 = __ffma2_rn(make_float2(s[c + 2], s[c + 3]), sc2, nm2);
+              float2 p01, p23;
+              if (SVSA_FA_POLY_EVERY > 0 && (c >> 2) % (SVSA_FA_POLY_EVERY > 0 ? SVSA_FA_POLY_EVERY : 1) ==
+                                                (SVSA_FA_POLY_EVERY > 0 ? SVSA_FA_POLY_EVERY - 1 : 0)) {
+                p01 = y01;
+                exp2_fma2(p01.x, p01.y);
+              } else {
+                p01 = make_float2(ex2(y01.x), ex2(y01.y));
+              }
+              p23 = make_float2(ex2(y23.x), ex2(y23.y));
+              acc0 = __fadd2_rn(acc0, p01);
+              acc1 = __fadd2_rn(acc1, p23);
+              pk[c >> 1] = pack_f16x2(p01.x, p01.y);
+              pk[(c >> 1) + 1] = pack_f16x2(p23.x, p23.y);
+            }
+            ls0 = acc0.x;
+            ls1 = acc0.y;
+            ls2 = acc1.x;
+            ls3 = acc1.y;
+          } else {
+#pragma unroll
+            for (int c = 0; c < 64; c += 2) {
+              const float p0 = ex2(s[c] + nm), p1 = ex2(s[c + 1] + nm);
+              add2(ls0, ls1, p0, p1);
+              pk[c >> 1] = pack_f16x2(p0, p1);
+            }
+          }
+          l += (ls0 + ls1) + (ls2 + ls3);
+          tmem_st32u(tmem + lane_off + sb * 128 + 64 * half, pk);
+          tmem_wait_st();
+          // this half's P ready (and this warp's reads of S and any rescale complete)
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(BAR_P_FULL + half * kSBufs + sb));
+          ++j;
+          if (stop) break;
         }
-        l += (ls0 + ls1) + (ls2 + ls3);
-        tmem_st32u(tmem + lane_off + sb * 128 + 32 * half, pk);
-        tmem_wait_st();
-        // P ready (and this warp's reads of S and any rescale of O complete)
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(BAR_P_FULL + sb));
-        ++j;
+        if (stop) break;
       }
-      // (a stop is decided below, at an OR-barrier both warps of the quadrant reach)
 
-      // ---- epilogue: the row sum over both halves, normalise this half of the O row, store it
-      const bool ok_o = __all_sync(0xffffffffu, wait_bar(bar(BAR_O_FULL), oit & 1u, abort_flag, 13));
-      xch[(4 + half) * 128 + row] = l;              // slots of their own: the last tile's maxima may still be read
-      if (named_bar_or(qbar, 64, stop || !ok_o)) {
+      // ---- epilogue: merge the two halves, normalise this thread's half of the columns, store
+      // (every exit is agreed by the row's two warps at an OR-barrier both
+      // reach, so neither waits at a named barrier the other has left)
+      const bool ok_o = !stop && __all_sync(0xffffffffu, wait_bar(bar(BAR_O_FULL), oit & 1u, abort_flag, 13));
+      xch[(0 + half) * 128 + row] = mref;
+      xch[(2 + half) * 128 + row] = l;
+      if (named_bar_or(qbar, 64, !ok_o)) {
         stop = true;
         break;
       }
-      const float lt = l + xch[(4 + (half ^ 1)) * 128 + row];
-      named_bar(qbar, 64);                          // both read before the next tile writes the slot
+      const float m_o = xch[(0 + (half ^ 1)) * 128 + row], l_o = xch[(2 + (half ^ 1)) * 128 + row];
+      named_bar(qbar, 64);                          // both read before the next item writes the slots
       ++oit;
       tc_fence_after();
+      const float mA = half ? m_o : mref, mB = half ? mref : m_o;
+      const float lA = half ? l_o : l, lB = half ? l : l_o;
+      // (a half with no valid key has l = 0 and takes no part)
+      const float mx = fmaxf(lA > 0.f ? mA : -INFINITY, lB > 0.f ? mB : -INFINITY);
+      const float sA = lA > 0.f ? ex2(mA - mx) : 0.f, sB = lB > 0.f ? ex2(mB - mx) : 0.f;
+      const float lt = lA * sA + lB * sB;
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      const float wA = sA * inv, wB = sB * inv;
       if (a.lse != nullptr && q >= 0 && half == 0) {
         const float ln2 = 0.6931471805599453f;
-        a.lse[bh * a.Npad + q] = (row_ok && lt > 0.f) ? (mref + __log2f(lt)) * ln2 : a.lse_empty;
+        a.lse[bh * a.Npad + q] = (row_ok && lt > 0.f) ? (mx + __log2f(lt)) * ln2 : a.lse_empty;
       }
 #pragma unroll
-      for (int c0 = 0; c0 < DH; c0 += 32) {
-        float o[32];
-        tmem_ld32(tmem + lane_off + kColO + half * DH + c0, o);
+      for (int c0 = 0; c0 < DH; c0 += 16) {
+        float oa[16], ob[16];
+        tmem_ld16(tmem + lane_off + kColO + half * DH + c0, oa);
+        tmem_ld16(tmem + lane_off + kColO + D + half * DH + c0, ob);
         tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 16; ++c) oa[c] = oa[c] * wA + ob[c] * wB;
         if (q >= 0) {
           if (O32) {
             float4* og = reinterpret_cast<float4*>(a.o32 + (bh * a.Npad + q) * D + half * DH + c0);
 #pragma unroll
-            for (int c = 0; c < 32; c += 4)
-              og[c >> 2] = row_ok ? make_float4(o[c] * inv, o[c + 1] * inv, o[c + 2] * inv, o[c + 3] * inv)
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int c = 0; c < 16; c += 4)
+              og[c >> 2] = row_ok ? make_float4(oa[c], oa[c + 1], oa[c + 2], oa[c + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
           } else {
             uint4* og = reinterpret_cast<uint4*>(a.o + (bh * a.Npad + q) * D + half * DH + c0);
 #pragma unroll
-            for (int c = 0; c < 32; c += 8) {
+            for (int c = 0; c < 16; c += 8) {
               uint4 v;
-              v.x = row_ok ? pack_bf16x2(o[c] * inv, o[c + 1] * inv) : 0u;
-              v.y = row_ok ? pack_bf16x2(o[c + 2] * inv, o[c + 3] * inv) : 0u;
-              v.z = row_ok ? pack_bf16x2(o[c + 4] * inv, o[c + 5] * inv) : 0u;
-              v.w = row_ok ? pack_bf16x2(o[c + 6] * inv, o[c + 7] * inv) : 0u;
+              v.x = row_ok ? pack_bf16x2(oa[c], oa[c + 1]) : 0u;
+              v.y = row_ok ? pack_bf16x2(oa[c + 2], oa[c + 3]) : 0u;
+              v.z = row_ok ? pack_bf16x2(oa[c + 4], oa[c + 5]) : 0u;
+              v.w = row_ok ? pack_bf16x2(oa[c + 6], oa[c + 7]) : 0u;
               og[c >> 3] = v;
             }
           }
         }
       }
-      // the O accumulator is free for the next item
+      // the accumulators are free for the next item
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(BAR_O_EMPTY));

@@ -683,7 +683,10 @@ def test_query_block_pairing(select, kw):
         shared = sum((keep[eta, pairs[eta, i]] & keep[eta, pairs[eta, i + 1]]).sum() for i in range(0, nb - 1, 2))
         adjacent = sum((keep[eta, i] & keep[eta, i + 1]).sum() for i in range(0, nb - 1, 2))
         assert shared >= adjacent
-    check_attention(to_np(out_p), to_np(out_u), "paired vs unpaired")
+    # two independently rounded bf16 outputs may differ by a rounding step
+    # (2^-7 relative); each is checked against the oracle below
+    a, b = to_np(out_p), to_np(out_u)
+    assert np.all(np.abs(a - b) <= 2.0 ** -7 * np.maximum(np.abs(a), np.abs(b)) + 2e-3)
     perm, _ = oracle.build_perm(w.T, w.H, w.W, w.order)
     qp, kp, vp = (oracle.reorder(to_np(t)[0].astype(np.float64), perm) for t in (q, k, v))
     op = to_np(paired.buf.op)[0]
