@@ -51,6 +51,8 @@ def _args():
     ap.add_argument("--secondary", default="wan13b",
                     help="a second, short layer whose attention / dense figures ride along in the line ('' = none)")
     ap.add_argument("--scorer", default=None, choices=["pooled", "sics"])
+    ap.add_argument("--attn", default="transposed", choices=["paired", "transposed"],
+                    help="sparse attention: the 64-row kernel alone (default) or the paired-block split")
     ap.add_argument("--order", default=None, choices=["raster", "hilbert", "cocluster"])
     ap.add_argument("--heads", type=int, default=None, help="override the layer's head count (profiling captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -103,6 +105,7 @@ def _max_over_ranks(x: float, ws: int) -> float:
 
 
 def _workload(args):
+    _LAYER_OPTS["paired_split"] = _LAYER_OPTS["pair_blocks"] = getattr(args, "attn", "transposed") == "paired"
     w = workloads.WORKLOADS[args.workload]
     if args.order:
         w = w.with_(order=args.order)
@@ -299,13 +302,17 @@ def run_reference(args):
 
 
 # --------------------------------------------------------------------------- GPU arm
+# layer options every GPU arm shares (set from the command line)
+_LAYER_OPTS = {"paired_split": False, "pair_blocks": False}
+
+
 def _layer(svsa, w, dev, seed=0):
     return svsa.SparseVideoAttention(w.B, w.heads, w.T, w.H, w.W, w.d, order=w.order, select=w.select,
                                      tau=w.tau, keep_frac=w.keep_frac, sub_block=w.sub_block,
                                      win_t=w.win_t, win_rows=w.win_rows,
                                      n_anchors=w.n_anchors if w.select == "structured" else 0,
                                      routing=w.routing, compensate=w.compensate, seed=seed, scorer=w.scorer,
-                                     device=dev)
+                                     device=dev, **_LAYER_OPTS)
 
 
 def _timed(fn, stream, flush, warmup, iters):
@@ -524,6 +531,7 @@ def run_svsa(args):
                        "N": w.N, "order": w.order, "select": w.select, "keep_frac": w.keep_frac,
                        "tau": w.tau, "sub_block": w.sub_block, "routing": w.routing,
                        "compensate": w.compensate, "scorer": w.scorer,
+                       "attention": "paired-block split" if _LAYER_OPTS["paired_split"] else "64-row kernel",
                        "step": (f"one mask cycle: perm, mask at the first of {cycle} denoising steps, then "
                                 f"reorder + attention + inverse at each of the {cycle} steps (Q, K drift by "
                                 f"sigma={w.sigma} between steps)") if cycle > 1 else
@@ -581,7 +589,8 @@ def run_schedule(args):
     q, k, v = workloads.make_qkv(w, seed=rank, device=dev)
     attn = svsa.SparseVideoAttention(w.B, w.heads, w.T, w.H, w.W, w.d, order=w.order, select=w.select,
                                      tau=w.tau, keep_frac=w.keep_frac, sub_block=w.sub_block,
-                                     routing=w.routing, compensate=w.compensate, schedule=sched, device=dev)
+                                     routing=w.routing, compensate=w.compensate, schedule=sched, device=dev,
+                                     **_LAYER_OPTS)
     out = torch.empty_like(q)
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     nvalid = np.minimum(64, w.N - 64 * np.arange(w.nb)).astype(np.int64)

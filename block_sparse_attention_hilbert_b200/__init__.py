@@ -82,6 +82,11 @@ _SIGS = {
                                            ctypes.POINTER(Mask), ctypes.c_int32, ctypes.c_void_p,
                                            ctypes.c_void_p, Shape, ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t,
                                            ctypes.c_void_p]),
+    "svsa_attn_paired_workspace_bytes": (ctypes.c_size_t, [Shape, ctypes.c_int32]),
+    "svsa_attn_fwd_paired": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                            ctypes.POINTER(Mask), ctypes.c_int32, ctypes.c_void_p,
+                                            ctypes.c_void_p, Shape, ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t,
+                                            ctypes.c_void_p]),
     "svsa_attn_dense_fwd": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                            ctypes.c_void_p, ctypes.c_void_p, Shape, ctypes.c_void_p]),
     "svsa_inverse_reorder": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, Shape,
@@ -262,6 +267,16 @@ def svsa_attn_fwd_split(qp, kp, vp, m: Mask, compensate: bool, op, lse, s: Shape
                         stream=None) -> None:
     _check(lib().svsa_attn_fwd_split(_p(qp), _p(kp), _p(vp), ctypes.byref(m), int(compensate), _p(op), _p(lse), s,
                                      passes, _p(ws), ws_bytes, _stream(stream)), "svsa_attn_fwd_split")
+
+
+def svsa_attn_paired_workspace_bytes(s: Shape, passes: int) -> int:
+    return int(lib().svsa_attn_paired_workspace_bytes(s, passes))
+
+
+def svsa_attn_fwd_paired(qp, kp, vp, m: Mask, compensate: bool, op, lse, s: Shape, passes: int, ws, ws_bytes: int,
+                         stream=None) -> None:
+    _check(lib().svsa_attn_fwd_paired(_p(qp), _p(kp), _p(vp), ctypes.byref(m), int(compensate), _p(op), _p(lse), s,
+                                      passes, _p(ws), ws_bytes, _stream(stream)), "svsa_attn_fwd_paired")
 
 
 def svsa_attn_dense_fwd(qp, kp, vp, op, lse, s: Shape, stream=None) -> None:

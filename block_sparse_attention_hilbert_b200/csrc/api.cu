@@ -1,6 +1,7 @@
 // C ABI of libsvsa: argument validation, workspace layout, kernel launches.
 // Every entry point validates before launching anything, returns a status
 // and never throws across the boundary.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdarg>
@@ -57,7 +58,11 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, const in
 cudaError_t launch_attn_fa(const void* q, const void* k, const void* v, const int32_t* kv_idx,
                            const int32_t* kv_cnt, int cap, const uint32_t* bits, const void* cbar, void* o,
                            float* lse, long long BH, long long N, int nb, int d, bool dense, cudaStream_t st,
-                           float* o32 = nullptr, float lse_empty = 0.f, const int32_t* pairs = nullptr);
+                           float* o32 = nullptr, float lse_empty = 0.f, const int32_t* pairs = nullptr,
+                           int inter_only = 0, const float* m_in = nullptr, const float* lse_in = nullptr);
+cudaError_t launch_exclusive(const int32_t* kv_idx, const int32_t* kv_cnt, int cap, const uint32_t* bits,
+                             const int32_t* pairs, long long BH, int nb, int32_t* x_idx, int xcap, int32_t* x_cnt,
+                             cudaStream_t st);
 cudaError_t attn_fa_error(unsigned int* code, cudaStream_t st);
 size_t pair_table_bytes(long long BH, int nb);
 cudaError_t launch_pair(const uint32_t* bits, long long BH, int nb, int16_t* tab, int32_t* pairs,
@@ -603,42 +608,59 @@ svsa_status svsa_attn_fwd(const void* qp, const void* kp, const void* vp, const 
     SVSA_TRY(cuda_status(counted(launch_centroid16(m->kbar, m->vbar, m->cbar, g.BH * g.nb, g.d,
                                                    (cudaStream_t)stream), 1),
                          "centroid copies"));
-  return cuda_status(counted(launch_attn_fa(qp, kp, vp, m->kv_idx, m->kv_cnt, m->cap, compensate ? m->bits : nullptr,
+  return cuda_status(counted(launch_attn_tc(qp, kp, vp, m->kv_idx, m->kv_cnt, m->cap, compensate ? m->bits : nullptr,
                                             compensate ? m->cbar : nullptr, op, lse, g.BH, g.N, g.nb, g.d, false,
-                                            (cudaStream_t)stream, nullptr, 0.f, m->pairs), 1),
+                                            (cudaStream_t)stream), 1),
                      "attn_fwd launch");
 }
 
 namespace {
 struct SplitWs {
-  size_t idx, cnt, o, lse, total;
+  size_t idx, cnt, o, lse, xidx, xcnt, part, plse, total;
 };
-SplitWs split_layout(const Dims& g, int P) {
+// Workspace of svsa_attn_fwd_split / svsa_attn_fwd_paired: the P range lists
+// and per-pass outputs (P > 1), then (paired) the exclusive lists and the
+// fp32 partial of the paired-block split.
+SplitWs split_layout(const Dims& g, int P, bool paired) {
   SplitWs w{};
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o = off; off += (bytes + 255) & ~(size_t)255; return o; };
   const long long rows = g.BH * g.nb;
   const int R = (g.nb + P - 1) / P;
-  w.idx = take((size_t)P * rows * R * 4);
-  w.cnt = take((size_t)P * rows * 4);
-  w.o = take((size_t)P * g.BH * g.Npad * g.d * 4);
-  w.lse = take((size_t)P * g.BH * g.Npad * 4);
+  w.idx = w.cnt = w.o = w.lse = w.xidx = w.xcnt = w.part = w.plse = SIZE_MAX;
+  if (P > 1) {
+    w.idx = take((size_t)P * rows * R * 4);
+    w.cnt = take((size_t)P * rows * 4);
+    w.o = take((size_t)P * g.BH * g.Npad * g.d * 4);
+    w.lse = take((size_t)P * g.BH * g.Npad * 4);
+  }
+  if (paired) {
+    w.xidx = take((size_t)rows * std::min(R, g.nb) * 4);
+    w.xcnt = take((size_t)rows * 4);
+    w.part = take((size_t)g.BH * g.Npad * g.d * 4);
+    w.plse = take((size_t)g.BH * g.Npad * 4);
+  }
   w.total = off;
   return w;
 }
 }  // namespace
 
 size_t svsa_attn_split_workspace_bytes(svsa_shape s, int32_t passes) {
-  if (passes < 2 || passes > 8 || s.T < 1 || s.H < 1 || s.W < 1 || s.B < 1 || s.heads < 1) return 0;
+  if (passes < 1 || passes > 8 || s.T < 1 || s.H < 1 || s.W < 1 || s.B < 1 || s.heads < 1) return 0;
   const Dims g = make_dims(s.B, s.heads, s.T, s.H, s.W, s.d);
-  return split_layout(g, passes).total;
+  return split_layout(g, passes, false).total;
 }
 
-svsa_status svsa_attn_fwd_split(const void* qp, const void* kp, const void* vp, const svsa_mask* m,
-                                int32_t compensate, void* op, float* lse, svsa_shape s, int32_t passes, void* ws,
-                                size_t ws_bytes, void* stream) {
-  if (passes == 1) return svsa_attn_fwd(qp, kp, vp, m, compensate, op, lse, s, stream);
-  NvtxRange nvtx_("svsa_attn_fwd_split");
+size_t svsa_attn_paired_workspace_bytes(svsa_shape s, int32_t passes) {
+  if (passes < 1 || passes > 8 || s.T < 1 || s.H < 1 || s.W < 1 || s.B < 1 || s.heads < 1) return 0;
+  const Dims g = make_dims(s.B, s.heads, s.T, s.H, s.W, s.d);
+  return split_layout(g, passes, true).total;
+}
+
+namespace {
+svsa_status attn_split(const void* qp, const void* kp, const void* vp, const svsa_mask* m, int32_t compensate,
+                       void* op, float* lse, svsa_shape s, int32_t passes, void* ws, size_t ws_bytes, void* stream,
+                       bool hybrid) {
   g_last_error.clear();
   if (passes < 1 || passes > 8) return fail(SVSA_ERR_INVALID_ARG, "passes=%d outside [1, 8]", passes);
   SVSA_TRY(check_shape(s, true));
@@ -661,15 +683,21 @@ svsa_status svsa_attn_fwd_split(const void* qp, const void* kp, const void* vp, 
     SVSA_PTR(m->bits, "mask.bits (compensation)");
     SVSA_PTR(m->cbar, "mask.cbar (compensation)");
   }
+  if (hybrid) SVSA_PTR(m->bits, "mask.bits (paired-block split)");
   if (op == qp || op == kp || op == vp) return fail(SVSA_ERR_INVALID_ARG, "op must not alias an input");
-  const SplitWs w = split_layout(g, passes);
+  const SplitWs w = split_layout(g, passes, hybrid);
   if (ws_bytes < w.total) return fail(SVSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, w.total);
   cudaStream_t st = (cudaStream_t)stream;
   char* base = reinterpret_cast<char*>(ws);
-  int32_t* idx_p = reinterpret_cast<int32_t*>(base + w.idx);
-  int32_t* cnt_p = reinterpret_cast<int32_t*>(base + w.cnt);
-  float* o_p = reinterpret_cast<float*>(base + w.o);
-  float* lse_p = reinterpret_cast<float*>(base + w.lse);
+  auto at = [&](size_t off) { return off == SIZE_MAX ? nullptr : base + off; };
+  int32_t* idx_p = reinterpret_cast<int32_t*>(at(w.idx));
+  int32_t* cnt_p = reinterpret_cast<int32_t*>(at(w.cnt));
+  float* o_p = reinterpret_cast<float*>(at(w.o));
+  float* lse_p = reinterpret_cast<float*>(at(w.lse));
+  int32_t* xidx = reinterpret_cast<int32_t*>(at(w.xidx));
+  int32_t* xcnt = reinterpret_cast<int32_t*>(at(w.xcnt));
+  float* part = reinterpret_cast<float*>(at(w.part));
+  float* plse = reinterpret_cast<float*>(at(w.plse));
   const long long rows = g.BH * g.nb;
   const int R = (g.nb + passes - 1) / passes;
   if (m->check) {
@@ -680,20 +708,64 @@ svsa_status svsa_attn_fwd_split(const void* qp, const void* kp, const void* vp, 
   if (compensate)
     SVSA_TRY(cuda_status(counted(launch_centroid16(m->kbar, m->vbar, m->cbar, g.BH * g.nb, g.d, st), 1),
                          "centroid copies"));
-  SVSA_TRY(cuda_status(counted(launch_split_mask(m->kv_idx, m->kv_cnt, m->cap, rows, g.nb, passes, R, idx_p, cnt_p,
-                                                 st), 1),
-                       "split mask"));
+  if (passes > 1)
+    SVSA_TRY(cuda_status(counted(launch_split_mask(m->kv_idx, m->kv_cnt, m->cap, rows, g.nb, passes, R, idx_p, cnt_p,
+                                                   st), 1),
+                         "split mask"));
+  const long long rows_o = g.BH * g.Npad;
   for (int p = 0; p < passes; ++p) {
-    // the centroid tiles of the skipped blocks go with the last pass
+    // this pass's lists; the centroid tiles of the skipped blocks go with the last pass
+    const int32_t* L_idx = passes > 1 ? idx_p + (long long)p * rows * R : m->kv_idx;
+    const int32_t* L_cnt = passes > 1 ? cnt_p + (long long)p * rows : m->kv_cnt;
+    const int L_cap = passes > 1 ? R : m->cap;
     const bool comp = compensate && p + 1 == passes;
-    SVSA_TRY(cuda_status(counted(launch_attn_fa(qp, kp, vp, idx_p + (long long)p * rows * R, cnt_p + (long long)p * rows,
-                                                 R, comp ? m->bits : nullptr, comp ? m->cbar : nullptr, nullptr,
-                                                 lse_p + (long long)p * g.BH * g.Npad, g.BH, g.N, g.nb, g.d, false, st,
-                                                 o_p + (long long)p * g.BH * g.Npad * g.d, -INFINITY, m->pairs), 1),
-                         "attn_fwd pass launch"));
+    float* out32 = passes > 1 ? o_p + (long long)p * rows_o * g.d : nullptr;
+    float* out_lse = passes > 1 ? lse_p + (long long)p * rows_o : lse;
+    if (!hybrid) {
+      SVSA_TRY(cuda_status(counted(launch_attn_tc(qp, kp, vp, L_idx, L_cnt, L_cap, comp ? m->bits : nullptr,
+                                                   comp ? m->cbar : nullptr, nullptr, out_lse, g.BH, g.N, g.nb, g.d,
+                                                   false, st, out32, -INFINITY), 1),
+                           "attn_fwd pass launch"));
+      continue;
+    }
+    // The paired-block split: every pair of query blocks (the pairing table,
+    // else blocks 2p, 2p + 1) shares the key blocks both keep -- the 128-row
+    // kernel takes those with no masked quarter -- and each block keeps the
+    // ones its partner does not -- the transposed 64-query kernel takes those,
+    // with the centroid tiles, into an fp32 partial that the 128-row kernel
+    // then merges (log-sum-exp) into its output rows.
+    const int xcap = std::min(L_cap, g.nb);
+    SVSA_TRY(cuda_status(counted(launch_exclusive(L_idx, L_cnt, L_cap, m->bits, m->pairs, g.BH, g.nb, xidx, xcap,
+                                                  xcnt, st), 1),
+                         "exclusive lists"));
+    SVSA_TRY(cuda_status(counted(launch_attn_tc(qp, kp, vp, xidx, xcnt, xcap, comp ? m->bits : nullptr,
+                                                 comp ? m->cbar : nullptr, nullptr, plse, g.BH, g.N, g.nb, g.d, false,
+                                                 st, part, -INFINITY), 1),
+                         "attn_fwd exclusive launch"));
+    SVSA_TRY(cuda_status(counted(launch_attn_fa(qp, kp, vp, L_idx, L_cnt, L_cap, nullptr, nullptr,
+                                                 passes > 1 ? nullptr : op, out_lse, g.BH, g.N, g.nb, g.d, false, st,
+                                                 out32, passes > 1 ? -INFINITY : 0.f, m->pairs, 1, part, plse), 1),
+                         "attn_fwd shared launch"));
   }
+  if (passes == 1) return SVSA_OK;
   return cuda_status(counted(launch_combine(o_p, lse_p, g.BH * g.Npad, passes, g.d, op, lse, st), 1),
                      "combine launch");
+}
+}  // namespace
+
+svsa_status svsa_attn_fwd_split(const void* qp, const void* kp, const void* vp, const svsa_mask* m,
+                                int32_t compensate, void* op, float* lse, svsa_shape s, int32_t passes, void* ws,
+                                size_t ws_bytes, void* stream) {
+  if (passes == 1) return svsa_attn_fwd(qp, kp, vp, m, compensate, op, lse, s, stream);
+  NvtxRange nvtx_("svsa_attn_fwd_split");
+  return attn_split(qp, kp, vp, m, compensate, op, lse, s, passes, ws, ws_bytes, stream, false);
+}
+
+svsa_status svsa_attn_fwd_paired(const void* qp, const void* kp, const void* vp, const svsa_mask* m,
+                                 int32_t compensate, void* op, float* lse, svsa_shape s, int32_t passes, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_("svsa_attn_fwd_paired");
+  return attn_split(qp, kp, vp, m, compensate, op, lse, s, passes, ws, ws_bytes, stream, true);
 }
 
 svsa_status svsa_attn_dense_fwd(const void* qp, const void* kp, const void* vp, void* op, float* lse,

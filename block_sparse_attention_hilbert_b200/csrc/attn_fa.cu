@@ -103,6 +103,9 @@ struct Args {
   float scale_log2;
   int dense;
   const int32_t* pairs;    // nullable [BH, nb]: query blocks in item order (default: 0, 1, 2, ...)
+  int inter_only;          // 1: walk only the key blocks both query blocks keep (their intersection)
+  const float* m_in;       // nullable fp32 [BH * Npad, D]: a partial result over other keys (normalised) ...
+  const float* lse_in;     // ... and its natural-log sum-exp, merged into this launch's rows
 };
 
 // The ascending union of the kept lists of the item's two query blocks,
@@ -113,7 +116,7 @@ struct Merge {
   const int32_t* la;
   const int32_t* lb;
   int na, nb2, ia, ib, ca, cb, nkb;
-  bool dense;
+  bool dense, inter;
   __device__ __forceinline__ int load(const int32_t* l, int i, int n) const {
     if (i >= n) return INT_MAX;
     if (dense) return i;
@@ -123,6 +126,9 @@ struct Merge {
   __device__ __forceinline__ void init(const Args& a, long long bh, int I0, int I1) {
     nkb = a.nb;
     dense = a.dense != 0;
+    // (a block without a partner has an empty intersection: its whole list
+    // goes to the 64-row pass)
+    inter = a.inter_only != 0;
     const long long r0 = bh * a.nb + I0;
     if (dense) {
       na = a.nb;
@@ -146,17 +152,20 @@ struct Merge {
     ca = load(la, 0, na);
     cb = load(lb, 0, nb2);
   }
-  // next union element (-1 when both lists are exhausted)
+  // next union element (-1 when both lists are exhausted); with `inter`, the
+  // next element of the intersection
   __device__ __forceinline__ int next(uint32_t& fl) {
-    const int J = ca < cb ? ca : cb;
-    if (J == INT_MAX) {
-      fl = 0u;
-      return -1;
+    while (true) {
+      const int J = ca < cb ? ca : cb;
+      if (J == INT_MAX) {
+        fl = 0u;
+        return -1;
+      }
+      fl = (ca == J ? 1u : 0u) | (cb == J ? 2u : 0u);
+      if (ca == J) ca = load(la, ++ia, na);
+      if (cb == J) cb = load(lb, ++ib, nb2);
+      if (!inter || fl == 3u) return J;
     }
-    fl = (ca == J ? 1u : 0u) | (cb == J ? 2u : 0u);
-    if (ca == J) ca = load(la, ++ia, na);
-    if (cb == J) cb = load(lb, ++ib, nb2);
-    return J;
   }
 };
 
@@ -530,16 +539,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fa_kernel(const __grid_const
       Tiles ti;
       ti.init(a, bh, I0, I1, ncent);
       if (ti.empty()) {
-        // nothing kept by either block: zero output rows (each thread its half of the columns)
+        // no tile: the incoming partial as it is (merge mode), else zero rows
+        // (each thread its half of the columns)
         if (q >= 0) {
+          const bool pin = a.m_in != nullptr && row_ok && a.lse_in[bh * a.Npad + q] > -INFINITY;
+          const float* src = a.m_in != nullptr ? a.m_in + (bh * a.Npad + q) * D + half * DH : nullptr;
           if (O32) {
             float4* og = reinterpret_cast<float4*>(a.o32 + (bh * a.Npad + q) * D + half * DH);
-            for (int i = 0; i < DH / 4; ++i) og[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int i = 0; i < DH / 4; ++i)
+              og[i] = pin ? reinterpret_cast<const float4*>(src)[i] : make_float4(0.f, 0.f, 0.f, 0.f);
           } else {
             uint4* og = reinterpret_cast<uint4*>(a.o + (bh * a.Npad + q) * D + half * DH);
-            for (int i = 0; i < DH / 8; ++i) og[i] = make_uint4(0u, 0u, 0u, 0u);
+            for (int i = 0; i < DH / 8; ++i) {
+              uint4 v = make_uint4(0u, 0u, 0u, 0u);
+              if (pin) {
+                const float4 f0 = reinterpret_cast<const float4*>(src)[2 * i];
+                const float4 f1 = reinterpret_cast<const float4*>(src)[2 * i + 1];
+                v = make_uint4(pack_bf16x2(f0.x, f0.y), pack_bf16x2(f0.z, f0.w), pack_bf16x2(f1.x, f1.y),
+                               pack_bf16x2(f1.z, f1.w));
+              }
+              og[i] = v;
+            }
           }
-          if (a.lse != nullptr && half == 0) a.lse[bh * a.Npad + q] = a.lse_empty;
+          if (a.lse != nullptr && half == 0) a.lse[bh * a.Npad + q] = pin ? a.lse_in[bh * a.Npad + q] : a.lse_empty;
         }
         continue;
       }
@@ -733,12 +755,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fa_kernel(const __grid_const
       const float mx = fmaxf(lA > 0.f ? mA : -INFINITY, lB > 0.f ? mB : -INFINITY);
       const float sA = lA > 0.f ? ex2(mA - mx) : 0.f, sB = lB > 0.f ? ex2(mB - mx) : 0.f;
       const float lt = lA * sA + lB * sB;
-      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      const float ln2 = 0.6931471805599453f, log2e = 1.4426950408889634f;
+      // this launch's log2 sum-exp, and (merge mode) the incoming partial's:
+      // out = (o_here 2^(L_here - L) + o_in 2^(L_in - L)) / (2^(L_here - L) + 2^(L_in - L))
+      const float L2h = lt > 0.f ? mx + __log2f(lt) : -INFINITY;
+      float L2i = -INFINITY;
+      if (a.m_in != nullptr && q >= 0 && row_ok) L2i = a.lse_in[bh * a.Npad + q] * log2e;
+      const float L2m = fmaxf(L2h, L2i);
+      const float eh = L2h > -INFINITY ? ex2(L2h - L2m) : 0.f, ei = L2i > -INFINITY ? ex2(L2i - L2m) : 0.f;
+      const float es = eh + ei;
+      const float wh = es > 0.f ? eh / es : 0.f, wi = es > 0.f ? ei / es : 0.f;
+      const float inv = lt > 0.f ? wh / lt : 0.f;
       const float wA = sA * inv, wB = sB * inv;
-      if (a.lse != nullptr && q >= 0 && half == 0) {
-        const float ln2 = 0.6931471805599453f;
-        a.lse[bh * a.Npad + q] = (row_ok && lt > 0.f) ? (mx + __log2f(lt)) * ln2 : a.lse_empty;
-      }
+      const float* pin = (a.m_in != nullptr && q >= 0) ? a.m_in + (bh * a.Npad + q) * D + half * DH : nullptr;
+      if (a.lse != nullptr && q >= 0 && half == 0)
+        a.lse[bh * a.Npad + q] = (row_ok && es > 0.f) ? (L2m + __log2f(es)) * ln2 : a.lse_empty;
 #pragma unroll
       for (int c0 = 0; c0 < DH; c0 += 16) {
         float oa[16], ob[16];
@@ -747,6 +778,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fa_kernel(const __grid_const
         tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < 16; ++c) oa[c] = oa[c] * wA + ob[c] * wB;
+        if (pin != nullptr && wi > 0.f) {
+#pragma unroll
+          for (int c = 0; c < 16; c += 4) {
+            const float4 f = reinterpret_cast<const float4*>(pin + c0 + c)[0];
+            oa[c] = fmaf(f.x, wi, oa[c]);
+            oa[c + 1] = fmaf(f.y, wi, oa[c + 1]);
+            oa[c + 2] = fmaf(f.z, wi, oa[c + 2]);
+            oa[c + 3] = fmaf(f.w, wi, oa[c + 3]);
+          }
+        }
         if (q >= 0) {
           if (O32) {
             float4* og = reinterpret_cast<float4*>(a.o32 + (bh * a.Npad + q) * D + half * DH + c0);
@@ -797,7 +838,8 @@ bool make_map_fa(CUtensorMap* m, const void* base, long long rows, int d, bool f
 cudaError_t launch_attn_fa(const void* q, const void* k, const void* v, const int32_t* kv_idx,
                            const int32_t* kv_cnt, int cap, const uint32_t* bits, const void* cbar, void* o,
                            float* lse, long long BH, long long N, int nb, int d, bool dense, cudaStream_t st,
-                           float* o32, float lse_empty, const int32_t* pairs) {
+                           float* o32, float lse_empty, const int32_t* pairs, int inter_only, const float* m_in,
+                           const float* lse_in) {
   CUtensorMap mq, mk, mv, mc;
   const long long rows = BH * (long long)nb * kBlock;
   if (!make_map_fa(&mq, q, rows, d, false) || !make_map_fa(&mk, k, rows, d, false) ||
@@ -818,6 +860,9 @@ cudaError_t launch_attn_fa(const void* q, const void* k, const void* v, const in
   a.scale_log2 = 1.4426950408889634f / sqrtf((float)d);
   a.dense = dense ? 1 : 0;
   a.pairs = dense ? nullptr : pairs;
+  a.inter_only = inter_only;
+  a.m_in = m_in;
+  a.lse_in = lse_in;
   const long long grid = std::min<long long>(a.items, tc::sm_count());
   const bool comp = a.ncent > 0;
   auto go = [&](auto kernel) -> cudaError_t {

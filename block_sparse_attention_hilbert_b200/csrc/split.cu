@@ -91,7 +91,70 @@ __global__ void combine_kernel(const float* __restrict__ o_p, const float* __res
   if (lse_out != nullptr && lane == 0) lse_out[row] = wsum > 0.f ? m + __logf(wsum) : 0.f;
 }
 
+// One warp per pair item p of a head: the query blocks I0 = pairs[2p] and
+// I1 = pairs[2p + 1] (2p and 2p + 1 without a table).  Writes the blocks of
+// each list that the partner does not keep -- A \ B for I0, B \ A for I1 --
+// as ascending lists (ballot compaction in list order); the partner's kept
+// set is read from its bitmap row.  A block without a partner (odd nb) keeps
+// its whole list.  Entries are clamped to [0, nb), counts to [0, cap]; the
+// output rows have xcap = min(cap, nb) entries (more than nb only for a list
+// with repeats, whose excess is dropped).
+__global__ void exclusive_kernel(const int32_t* __restrict__ kv_idx, const int32_t* __restrict__ kv_cnt, int cap,
+                                 const uint32_t* __restrict__ bits, const int32_t* __restrict__ pairs, long long BH,
+                                 int nb, int npairs, int32_t* __restrict__ x_idx, int xcap,
+                                 int32_t* __restrict__ x_cnt) {
+  const long long item = (long long)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (item >= BH * npairs) return;
+  const long long bh = item / npairs;
+  const int p = (int)(item % npairs);
+  const int words = (nb + 31) / 32;
+  int blk[2] = {2 * p, 2 * p + 1 < nb ? 2 * p + 1 : -1};
+  if (pairs != nullptr) {
+    for (int h = 0; h < 2; ++h)
+      if (blk[h] >= 0) {
+        const int x = pairs[bh * nb + blk[h]];
+        blk[h] = x < 0 ? 0 : (x >= nb ? nb - 1 : x);
+      }
+  }
+  for (int h = 0; h < 2; ++h) {
+    const int I = blk[h], Ip = blk[h ^ 1];
+    if (I < 0) continue;
+    const long long row = bh * nb + I;
+    const int c0 = kv_cnt[row];
+    const int cnt = c0 < 0 ? 0 : (c0 > cap ? cap : c0);
+    const int32_t* lst = kv_idx + row * (long long)cap;
+    const uint32_t* pb = Ip >= 0 ? bits + (bh * nb + Ip) * (long long)words : nullptr;
+    int out = 0;
+    for (int base = 0; base < cnt; base += 32) {
+      const int e = base + lane;
+      int J = 0;
+      bool keep = false;
+      if (e < cnt) {
+        J = lst[e];
+        J = J < 0 ? 0 : (J >= nb ? nb - 1 : J);
+        keep = pb == nullptr || ((pb[J >> 5] >> (J & 31)) & 1u) == 0u;
+      }
+      const uint32_t m = __ballot_sync(0xffffffffu, keep);
+      const int at = out + __popc(m & ((1u << lane) - 1u));
+      if (keep && at < xcap) x_idx[row * (long long)xcap + at] = J;
+      out += __popc(m);
+    }
+    if (lane == 0) x_cnt[row] = out < xcap ? out : xcap;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_exclusive(const int32_t* kv_idx, const int32_t* kv_cnt, int cap, const uint32_t* bits,
+                             const int32_t* pairs, long long BH, int nb, int32_t* x_idx, int xcap, int32_t* x_cnt,
+                             cudaStream_t st) {
+  const int npairs = (nb + 1) / 2;
+  const long long items = BH * npairs;
+  exclusive_kernel<<<(unsigned)((items + kWarps - 1) / kWarps), 32 * kWarps, 0, st>>>(
+      kv_idx, kv_cnt, cap, bits, pairs, BH, nb, npairs, x_idx, xcap, x_cnt);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_split_mask(const int32_t* kv_idx, const int32_t* kv_cnt, int cap, long long rows, int nb, int P,
                               int R, int32_t* idx_p, int32_t* cnt_p, cudaStream_t st) {

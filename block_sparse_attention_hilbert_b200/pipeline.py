@@ -27,7 +27,7 @@ from . import (ORDER_HILBERT, ORDER_RASTER, SEL_STRUCTURED, SEL_THRESHOLD, SEL_T
                svsa_inverse_reorder, svsa_inverse_reorder_heads, svsa_mask_workspace_bytes,
                svsa_perm_workspace_bytes, svsa_reorder, svsa_reorder_heads, svsa_reorder_values,
                svsa_reorder_values_heads, svsa_schedule_step, svsa_attn_fwd_split,
-               svsa_attn_split_workspace_bytes)
+               svsa_attn_split_workspace_bytes, svsa_attn_fwd_paired, svsa_attn_paired_workspace_bytes)
 
 _ORDERS = {"raster": ORDER_RASTER, "hilbert": ORDER_HILBERT}
 _SELECTS = {"threshold": SEL_THRESHOLD, "topk": SEL_TOPK, "structured": SEL_STRUCTURED}
@@ -99,7 +99,7 @@ class SparseVideoAttention:
     def __init__(self, B, heads, T, H, W, d, *, order="hilbert", select="threshold", tau=0.9,
                  keep_frac=0.25, sub_block=64, win_t=2, win_rows=1, n_anchors=0, routing=False,
                  compensate=False, keep_bits=False, schedule=None, cluster_rounds=3, attn_passes=None,
-                 seed=0, scorer="pooled", check_mask=False, pair_blocks=True, device="cuda"):
+                 seed=0, scorer="pooled", check_mask=False, pair_blocks=False, paired_split=False, device="cuda"):
         """order: "raster", "hilbert" or "cocluster" (a per-head semantic order from
         bidirectional query-key co-clustering, built from the first inputs and
         kept until `rebuild_order()`).  schedule: optional (n_steps, dense_steps,
@@ -113,9 +113,13 @@ class SparseVideoAttention:
         step index of each call picks the rotation).  scorer: "pooled" (block
         scores) or "sics" (per-head block coherence).  check_mask: validate
         the lists before every attention call (svsa_sync_status reports a
-        malformed one).  pair_blocks: let svsa_build_mask pair the query
-        blocks by kept-list overlap for the attention's 128-row items (else
-        blocks 2p and 2p + 1 go together)."""
+        malformed one).  paired_split: run the attention as
+        svsa_attn_fwd_paired (the key blocks both query blocks of a pair keep
+        on the 128-row kernel, the rest on the 64-row one; it keeps the
+        kept-block bitmap).  pair_blocks: let svsa_build_mask pair the query
+        blocks by kept-list overlap for that split (else blocks 2p and 2p + 1
+        go together).  Both are off by default: on B200 the 64-row kernel
+        alone is the faster one on the sparse masks measured."""
         self.B, self.heads, self.T, self.H, self.W, self.d = B, heads, T, H, W, d
         self.N = T * H * W
         self.nb = -(-self.N // BLOCK)
@@ -136,7 +140,7 @@ class SparseVideoAttention:
         # a scheduled top-k rule reaches keep_frac = 1 on its dense steps
         cap = k if (self.select == SEL_TOPK and self.schedule is None) else self.nb
         self.buf = LayerBuffers(B, heads, T, H, W, d, cap=cap, need_means=self.compensate or self.routing,
-                                keep_bits=keep_bits, ws_bytes=svsa_mask_workspace_bytes(self.shape, self.params),
+                                keep_bits=keep_bits or paired_split, ws_bytes=svsa_mask_workspace_bytes(self.shape, self.params),
                                 perm_ws_bytes=svsa_perm_workspace_bytes(self.shape, self.order),
                                 device=device, compensate=self.compensate, pair_blocks=pair_blocks)
         self._mask = self.buf.mask()
@@ -144,9 +148,11 @@ class SparseVideoAttention:
         if attn_passes is None:
             attn_passes = default_attn_passes(self.select, self.Npad, d)
         self.attn_passes = int(attn_passes)
-        self.buf.split_ws = (torch.empty(svsa_attn_split_workspace_bytes(self.shape, self.attn_passes),
-                                         dtype=torch.uint8, device=self.buf.qp.device)
-                             if self.attn_passes > 1 else None)
+        self.paired_split = bool(paired_split)
+        ws_bytes = (svsa_attn_paired_workspace_bytes if self.paired_split
+                    else svsa_attn_split_workspace_bytes)(self.shape, self.attn_passes)
+        self.buf.split_ws = (torch.empty(ws_bytes, dtype=torch.uint8, device=self.buf.qp.device)
+                             if self.attn_passes > 1 or self.paired_split else None)
         if self.cocluster:
             rows, dev = B * heads, self.buf.qp.device
             b = self.buf
@@ -198,7 +204,10 @@ class SparseVideoAttention:
 
     def attend(self, lse=None, stream=None):
         b = self.buf
-        if self.attn_passes > 1:
+        if self.paired_split:
+            svsa_attn_fwd_paired(b.qp, b.kp, b.vp, self._mask, self.compensate, b.op, lse, self.shape,
+                                 self.attn_passes, b.split_ws, b.split_ws.numel(), stream)
+        elif self.attn_passes > 1:
             svsa_attn_fwd_split(b.qp, b.kp, b.vp, self._mask, self.compensate, b.op, lse, self.shape,
                                 self.attn_passes, b.split_ws, b.split_ws.numel(), stream)
         else:
@@ -305,7 +314,11 @@ class SparseVideoAttention:
                 svsa_build_mask(self._rows(b.qp, r0, r1), self._rows(b.kp, r0, r1), self._rows(b.vp, r0, r1),
                                 None if self.cocluster else b.perm, sh, self.params, m, b.ws, b.ws.numel(),
                                 compute)
-            if self.attn_passes > 1:
+            if self.paired_split:
+                svsa_attn_fwd_paired(self._rows(b.qp, r0, r1), self._rows(b.kp, r0, r1), self._rows(b.vp, r0, r1),
+                                     m, self.compensate, self._rows(b.op, r0, r1), None, sh, self.attn_passes,
+                                     b.split_ws, b.split_ws.numel(), compute)
+            elif self.attn_passes > 1:
                 svsa_attn_fwd_split(self._rows(b.qp, r0, r1), self._rows(b.kp, r0, r1), self._rows(b.vp, r0, r1), m,
                                     self.compensate, self._rows(b.op, r0, r1), None, sh, self.attn_passes,
                                     b.split_ws, b.split_ws.numel(), compute)

@@ -305,6 +305,23 @@ svsa_status svsa_attn_fwd_split(const void* qp, const void* kp, const void* vp, 
                                 int32_t compensate, void* op, float* lse, svsa_shape s, int32_t passes, void* ws,
                                 size_t ws_bytes, void* stream);
 
+/* svsa_attn_fwd as the paired-block split, same result up to rounding.  The
+ * query blocks go in pairs (m->pairs entries 2p, 2p + 1 when given, else
+ * blocks 2p, 2p + 1; an odd last block alone).  The key blocks that both
+ * blocks of a pair keep are attended by 128 query rows at once (both blocks
+ * share every key tile, so no tensor work is spent on a masked quarter); the
+ * key blocks that only one of them keeps, and the compensation terms, are
+ * attended by 64 query rows into an fp32 partial output with its
+ * log-sum-exp, which the 128-row pass then merges into its rows by the same
+ * rule as svsa_attn_fwd_split's passes.  Needs m->bits (the kept set; it
+ * must agree with kv_idx / kv_cnt).  passes in [1, 8] as for
+ * svsa_attn_fwd_split (each key-range pass is split this way); ws: device
+ * memory of svsa_attn_paired_workspace_bytes(s, passes) bytes. */
+size_t svsa_attn_paired_workspace_bytes(svsa_shape s, int32_t passes);
+svsa_status svsa_attn_fwd_paired(const void* qp, const void* kp, const void* vp, const svsa_mask* m,
+                                 int32_t compensate, void* op, float* lse, svsa_shape s, int32_t passes, void* ws,
+                                 size_t ws_bytes, void* stream);
+
 /* Dense attention over all N keys, same arithmetic and layouts as
  * svsa_attn_fwd; the denominator of the speedup the benchmark reports. */
 svsa_status svsa_attn_dense_fwd(const void* qp, const void* kp, const void* vp, void* op,

@@ -107,6 +107,21 @@ def test_workspace_queries():
     p16 = svsa.mask_params(svsa.SEL_THRESHOLD, sub_block=16)
     assert svsa.svsa_mask_workspace_bytes(s, p16) > svsa.svsa_mask_workspace_bytes(s, p)
     assert svsa.svsa_mask_workspace_bytes(s, svsa.mask_params(sub_block=32)) == 0
+    # attention: one plain pass needs none; the paired-block split needs at
+    # least its fp32 partial output [BH, Npad, d] and lse, the exclusive lists
+    # [BH, nb, nb] and counts; key-range passes add their lists and outputs
+    rows, npad = 12 * nb, nb * 64
+    assert svsa.svsa_attn_split_workspace_bytes(s, 1) == 0
+    need1 = 12 * npad * 128 * 4 + 12 * npad * 4 + rows * nb * 4 + rows * 4
+    assert svsa.svsa_attn_paired_workspace_bytes(s, 1) >= need1
+    for P in (2, 3, 8):
+        R = -(-nb // P)
+        split = svsa.svsa_attn_split_workspace_bytes(s, P)
+        assert split >= P * (rows * R * 4 + rows * 4 + 12 * npad * 128 * 4 + 12 * npad * 4)
+        assert svsa.svsa_attn_paired_workspace_bytes(s, P) >= split + 12 * npad * 128 * 4 + rows * R * 4
+    for P in (0, 9):
+        assert svsa.svsa_attn_split_workspace_bytes(s, P) == 0
+        assert svsa.svsa_attn_paired_workspace_bytes(s, P) == 0
 
 
 def _raw():

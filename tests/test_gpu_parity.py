@@ -601,16 +601,20 @@ def test_degenerate_grids(grid, case):
     (3, "threshold", {"routing": True, "compensate": True}),
     (5, "threshold", {"sub": 16}),
 ])
-def test_split_attention_matches_single_pass_and_oracle(passes, select, kw):
-    """Key-range passes merged by log-sum-exp: the output and the lse agree with
-    the single-pass call (up to rounding) and with the oracle."""
+@pytest.mark.parametrize("paired", [False, True])
+def test_split_attention_matches_single_pass_and_oracle(passes, select, kw, paired):
+    """Key-range passes merged by log-sum-exp (svsa_attn_fwd_split, or each
+    pass as the paired-block split): the output and the lse agree with the
+    single-pass call (up to rounding) and with the oracle."""
+    kw = dict(kw)
     sub = kw.pop("sub", 64)
     w = _small(select, sub, grid=(6, 12, 20), heads=2, tau=0.9, keep_frac=0.3, **kw)
     q, k, v = (t.cuda() for t in workloads.make_qkv(w, seed=12))
-    mk = lambda p: svsa.SparseVideoAttention(w.B, w.heads, w.T, w.H, w.W, w.d, order=w.order, select=select,
-                                             tau=w.tau, keep_frac=w.keep_frac, sub_block=sub, routing=w.routing,
-                                             compensate=w.compensate, keep_bits=True, attn_passes=p, device="cuda")
-    one, many = mk(1), mk(passes)
+    mk = lambda p, ps: svsa.SparseVideoAttention(w.B, w.heads, w.T, w.H, w.W, w.d, order=w.order, select=select,
+                                                 tau=w.tau, keep_frac=w.keep_frac, sub_block=sub,
+                                                 routing=w.routing, compensate=w.compensate, keep_bits=True,
+                                                 attn_passes=p, paired_split=ps, device="cuda")
+    one, many = mk(1, False), mk(passes, paired)
     one.reorder(q, k, v); one.build_mask()
     many.reorder(q, k, v); many.build_mask()
     lse1 = torch.empty(1, w.heads, one.Npad, dtype=torch.float32, device="cuda")
@@ -670,7 +674,7 @@ def test_query_block_pairing(select, kw):
     mk = lambda pair: SparseVideoAttention(w.B, w.heads, w.T, w.H, w.W, w.d, order=w.order, select=w.select,
                                            tau=w.tau, keep_frac=w.keep_frac, sub_block=w.sub_block,
                                            routing=w.routing, compensate=w.compensate, pair_blocks=pair,
-                                           keep_bits=True, device="cuda")
+                                           keep_bits=True, paired_split=True, device="cuda")
     paired, plain = mk(True), mk(False)
     out_p, out_u = paired(q, k, v), plain(q, k, v)
     torch.cuda.synchronize()
@@ -699,3 +703,91 @@ def test_query_block_pairing(select, kw):
             ref = oracle.masked_attention(qp[eta], kp[eta], vp[eta], w.N, keep[eta])
         gout = np.concatenate([op[eta][I * 64:min(I * 64 + 64, w.N)] for I in range(nb)])
         check_attention(gout, np.concatenate([ref[I] for I in range(nb)]), f"head {eta}")
+
+
+def _write_lists(attn, keep):
+    """Kept sets keep [heads, nb, nb] (bool) into the layer's kv lists and bitmap."""
+    heads, nb = keep.shape[0], keep.shape[1]
+    b = attn.buf
+    idx = np.zeros((1, heads, nb, b.cap), dtype=np.int32)
+    for eta in range(heads):
+        for I in range(nb):
+            lst = np.nonzero(keep[eta, I])[0]
+            idx[0, eta, I, :len(lst)] = lst
+    words = -(-nb // 32)
+    bits = np.zeros((1, heads, nb, words), dtype=np.uint32)
+    for J in range(nb):
+        bits[..., J >> 5] |= keep[None, :, :, J].astype(np.uint32) << np.uint32(J & 31)
+    b.kv_idx.copy_(torch.from_numpy(idx))
+    b.kv_cnt.copy_(torch.from_numpy(keep.sum(-1).astype(np.int32)[None]))
+    b.bits.copy_(torch.from_numpy(bits.view(np.int32)))
+
+
+@pytest.mark.parametrize("passes", [1, 2, 3])
+@pytest.mark.parametrize("table", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_paired_split_on_written_masks(passes, table, d):
+    """svsa_attn_fwd_paired on lists written here, with every shape a pair can
+    take: identical lists (all shared), disjoint lists (all exclusive), one
+    empty list, both empty, a full row, and (odd nb) the lone last block;
+    with and without a pairing table.  Output and lse agree with
+    svsa_attn_fwd up to rounding and with the oracle."""
+    T, H, W = 7, 13, 20                                   # N = 1820: nb = 29, last block 28 tokens
+    heads = 2
+    w = _small("topk", 64, grid=(T, H, W), heads=heads, d=d)
+    q, k, v = (t.cuda() for t in workloads.make_qkv(w, seed=21))
+    nb = -(-w.N // 64)
+    rng = np.random.default_rng(5 + passes)
+    keep = rng.random((heads, nb, nb)) < 0.35
+    keep[:, 4] = keep[:, 5]                               # identical
+    keep[:, 6] = ~keep[:, 7]                              # disjoint
+    keep[:, 8] = False                                    # one empty
+    keep[:, 10] = keep[:, 11] = False                     # both empty
+    keep[:, 12] = True                                    # full
+    mk = lambda ps: SparseVideoAttention(1, heads, T, H, W, d, order="hilbert", select="threshold", tau=1.0,
+                                         keep_bits=True, pair_blocks=table, attn_passes=passes,
+                                         paired_split=ps, device="cuda")
+    paired, plain = mk(True), mk(False)
+    for a in (paired, plain):
+        a.reorder(q, k, v)
+        _write_lists(a, keep)
+    if table:
+        # a random order of the query blocks per head, so pairs are far apart
+        pt = np.stack([rng.permutation(nb) for _ in range(heads)]).astype(np.int32)
+        paired.buf.pairs.copy_(torch.from_numpy(pt)[None])
+    lse_p = torch.empty(1, heads, paired.Npad, dtype=torch.float32, device="cuda")
+    lse_u = torch.empty_like(lse_p)
+    paired.attend(lse=lse_p)
+    plain.attend(lse=lse_u)
+    torch.cuda.synchronize()
+    svsa.svsa_sync_status()
+    a, b = to_np(paired.buf.op)[0], to_np(plain.buf.op)[0]
+    assert np.all(np.abs(a - b) <= 2.0 ** -7 * np.maximum(np.abs(a), np.abs(b)) + 2e-3)
+    valid = np.arange(paired.Npad) < w.N
+    assert np.allclose(to_np(lse_p)[0][:, valid], to_np(lse_u)[0][:, valid], atol=1e-4)
+    assert np.all(a[:, ~valid] == 0)
+    lp = to_np(lse_p)[0]
+    for eta in range(heads):
+        for I in (8, 10, 11):                             # no kept key: zero rows, lse 0
+            rows = slice(I * 64, I * 64 + 64)
+            assert np.all(a[eta, rows] == 0) and np.all(lp[eta, rows] == 0)
+    perm, _ = oracle.build_perm(T, H, W, "hilbert")
+    qp, kp, vp = (oracle.reorder(to_np(t)[0].astype(np.float64), perm) for t in (q, k, v))
+    for eta in range(heads):
+        # (the softmax over no key is undefined; those rows were checked above)
+        blocks = [I for I in range(nb) if keep[eta, I].any()]
+        ref = oracle.masked_attention(qp[eta], kp[eta], vp[eta], w.N, keep[eta], q_blocks=blocks)
+        gout = np.concatenate([a[eta][I * 64:min(I * 64 + 64, w.N)] for I in blocks])
+        check_attention(gout, np.concatenate([ref[I] for I in blocks]), f"passes={passes} head {eta}")
+
+
+def test_paired_split_needs_the_bitmap():
+    w = _small("topk", 64, grid=(5, 7, 9), heads=1)
+    attn = SparseVideoAttention(1, 1, 5, 7, 9, w.d, select="topk", keep_frac=0.3, device="cuda")
+    assert attn.buf.bits is None
+    ws = torch.empty(svsa.svsa_attn_paired_workspace_bytes(attn.shape, 1), dtype=torch.uint8, device="cuda")
+    b = attn.buf
+    with pytest.raises(svsa.SvsaError):
+        svsa.svsa_attn_fwd_paired(b.qp, b.kp, b.vp, attn._mask, False, b.op, None, attn.shape, 1, ws, ws.numel())
+    assert SparseVideoAttention(1, 1, 5, 7, 9, w.d, select="topk", paired_split=True,
+                                device="cuda").buf.bits is not None
