@@ -485,19 +485,33 @@ def run_svsa(args):
     dense_ms = _max_over_ranks(_timed(attn.attend_dense, stream, flush, 1 if long_layer else args.warmup,
                                       min(args.steps, 3) if long_layer else args.steps), ws)
 
-    # end to end through the public API: pinned host Q, K, V of every step of the
-    # cycle in, O of every step back to the host, the copies of one group of
-    # heads overlapping the compute of another
+    # end to end through the C entry point on host buffers (svsa_layer_forward_host):
+    # pinned host Q, K, V of every step of the cycle in, O of every step back to
+    # the host, the copies of one group of heads overlapping the compute of another
     hq = [t.cpu().pin_memory() for t in qs]
     hk = [t.cpu().pin_memory() for t in ks]
     hv = v.cpu().pin_memory()
     hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    e2e_groups = min(12, w.B * w.heads)
+    # (the co-clustering order is built from the layer's device tensors: that
+    # order streams through the Python layer object instead)
+    layer = None if attn.cocluster else svsa.svsa_layer_create(attn.shape, svsa.layer_config(
+        attn.order, attn.params, compensate=w.compensate, attn_passes=attn.attn_passes,
+        paired=attn.paired_split, groups=e2e_groups))
 
     def e2e_cycle():
         for st in range(cycle):
-            attn.forward_host(hq[st], hk[st], hv, hout, step=0, reuse_mask=st > 0)
+            if layer is None:
+                attn.forward_host(hq[st], hk[st], hv, hout, step=0, reuse_mask=st > 0, groups=e2e_groups)
+            else:
+                svsa.svsa_layer_forward_host(layer, hq[st], hk[st], hv, hout, step=0,
+                                             flags=svsa.LAYER_REUSE_MASK if st > 0 else 0, stream=stream)
 
-    e2e_ms = _max_over_ranks(_timed(e2e_cycle, stream, flush, args.warmup, args.steps), ws)
+    try:
+        e2e_ms = _max_over_ranks(_timed(e2e_cycle, stream, flush, args.warmup, args.steps), ws)
+    finally:
+        if layer is not None:
+            svsa.svsa_layer_destroy(layer)
     h2d = cycle * 3 * q0.numel() * q0.element_size()
     d2h = cycle * out.numel() * out.element_size()
     del hq, hk, hv, hout
@@ -558,7 +572,10 @@ def run_svsa(args):
                          "peak_source": f"{peak_src} " + ("bf16_tflops_sustained (step >= 100 ms)" if sustained
                                                            else "bf16_tflops (burst)")},
             "e2e": {"value": ws * cycle_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "path": (f"svsa_layer_forward_host (C entry point, pinned host buffers, {e2e_groups} row "
+                             "groups; the token order built once at svsa_layer_create)") if not attn.cocluster else
+                            f"SparseVideoAttention.forward_host (pinned host buffers, {e2e_groups} row groups)"},
             "gpu_launches": launches,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,

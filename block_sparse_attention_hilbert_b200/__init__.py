@@ -51,6 +51,14 @@ class Mask(ctypes.Structure):
                 ("check", ctypes.c_int32)]
 
 
+class LayerConfig(ctypes.Structure):
+    _fields_ = [("order", ctypes.c_int32), ("mask", MaskParams), ("compensate", ctypes.c_int32),
+                ("attn_passes", ctypes.c_int32), ("paired", ctypes.c_int32), ("groups", ctypes.c_int32)]
+
+
+LAYER_REUSE_MASK = 1
+
+
 class Schedule(ctypes.Structure):
     _fields_ = [("n_steps", ctypes.c_int32), ("dense_steps", ctypes.c_int32), ("start", ctypes.c_float),
                 ("end", ctypes.c_float), ("refresh_every", ctypes.c_int32)]
@@ -82,6 +90,11 @@ _SIGS = {
                                            ctypes.POINTER(Mask), ctypes.c_int32, ctypes.c_void_p,
                                            ctypes.c_void_p, Shape, ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t,
                                            ctypes.c_void_p]),
+    "svsa_layer_device_bytes": (ctypes.c_size_t, [Shape, ctypes.POINTER(LayerConfig)]),
+    "svsa_layer_create": (ctypes.c_int, [Shape, ctypes.POINTER(LayerConfig), ctypes.POINTER(ctypes.c_void_p)]),
+    "svsa_layer_forward_host": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                               ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p]),
+    "svsa_layer_destroy": (ctypes.c_int, [ctypes.c_void_p]),
     "svsa_attn_paired_workspace_bytes": (ctypes.c_size_t, [Shape, ctypes.c_int32]),
     "svsa_attn_fwd_paired": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                             ctypes.POINTER(Mask), ctypes.c_int32, ctypes.c_void_p,
@@ -267,6 +280,32 @@ def svsa_attn_fwd_split(qp, kp, vp, m: Mask, compensate: bool, op, lse, s: Shape
                         stream=None) -> None:
     _check(lib().svsa_attn_fwd_split(_p(qp), _p(kp), _p(vp), ctypes.byref(m), int(compensate), _p(op), _p(lse), s,
                                      passes, _p(ws), ws_bytes, _stream(stream)), "svsa_attn_fwd_split")
+
+
+def layer_config(order: int, mask: MaskParams, compensate: bool = False, attn_passes: int = 1,
+                 paired: bool = False, groups: int = 1) -> LayerConfig:
+    return LayerConfig(order, mask, int(compensate), attn_passes, int(paired), groups)
+
+
+def svsa_layer_device_bytes(s: Shape, cfg: LayerConfig) -> int:
+    return int(lib().svsa_layer_device_bytes(s, ctypes.byref(cfg)))
+
+
+def svsa_layer_create(s: Shape, cfg: LayerConfig) -> int:
+    """A host-buffer layer (an opaque handle; free it with svsa_layer_destroy)."""
+    h = ctypes.c_void_p(0)
+    _check(lib().svsa_layer_create(s, ctypes.byref(cfg), ctypes.byref(h)), "svsa_layer_create")
+    return int(h.value)
+
+
+def svsa_layer_forward_host(layer: int, q, k, v, o, step: int = 0, flags: int = 0, stream=None) -> None:
+    """q, k, v, o: host bf16 [B, heads, N, d] (pinned for overlap)."""
+    _check(lib().svsa_layer_forward_host(layer, _p(q), _p(k), _p(v), _p(o), step, flags, _stream(stream)),
+           "svsa_layer_forward_host")
+
+
+def svsa_layer_destroy(layer: int) -> None:
+    _check(lib().svsa_layer_destroy(layer), "svsa_layer_destroy")
 
 
 def svsa_attn_paired_workspace_bytes(s: Shape, passes: int) -> int:

@@ -84,6 +84,7 @@ cudaError_t launch_check_pairs(const int32_t* pairs, long long BH, int nb, cudaS
 cudaError_t sics_flags(unsigned int* v, cudaStream_t st);
 cudaError_t reorder_flags(unsigned int* v, cudaStream_t st);
 cudaError_t pool_flags(unsigned int* v, cudaStream_t st);
+svsa_status record_error(svsa_status st, const char* msg);
 }  // namespace svsa
 
 using namespace svsa;
@@ -108,6 +109,13 @@ svsa_status fail(svsa_status st, const char* fmt, ...) {
   g_last_error = buf;
   return st;
 }
+
+}  // namespace
+
+// For the library's other host-side files: record a failure message.
+svsa_status svsa::record_error(svsa_status st, const char* msg) { return fail(st, "%s", msg); }
+
+namespace {
 
 svsa_status cuda_status(cudaError_t e, const char* what) {
   if (e == cudaSuccess) return SVSA_OK;

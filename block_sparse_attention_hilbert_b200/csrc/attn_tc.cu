@@ -62,7 +62,7 @@ constexpr int kThreads = 32 * (4 + 4 * kGroups);
 #ifndef SVSA_TC_PBUFS
 #define SVSA_TC_PBUFS 3
 #endif
-constexpr int kKStages = SVSA_TC_KSTAGES, kVStages = 2, kSBufs = 3, kPBufs = SVSA_TC_PBUFS;
+constexpr int kKStages = SVSA_TC_KSTAGES, kVStages = 2, kSBufs = SVSA_TC_PBUFS, kPBufs = SVSA_TC_PBUFS;
 constexpr int kSoftmaxThreads = 128;             // one softmax warpgroup
 constexpr uint32_t kBox = 8192;                  // one 64-row x 128-byte TMA box
 constexpr float kLazyTh = 12.0f;                 // log2 headroom before a rescale (fp16 P <= 2^12)
@@ -76,9 +76,11 @@ constexpr uint32_t kOffMisc = kOffP + kPBufs * 16384;
 constexpr uint32_t kSmemBytes = kOffMisc + 2048 + 1024;     // + alignment slack
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
-// TMEM columns: three S^T buffers and O^T
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS0 = 0, kColO = 192;
+// TMEM columns: the S^T ring (64 columns a buffer), then O^T; the allocation
+// is the next power of two
+constexpr uint32_t kColS0 = 0, kColO = 64u * kSBufs;
+constexpr uint32_t kTmemCols = kColO + 64u <= 256u ? 256u : 512u;
+static_assert(kColO + 64u <= 512u, "TMEM columns");
 
 
 enum : uint32_t {

@@ -130,14 +130,15 @@ typedef struct {
                              block's kbar (bf16, first d) and vbar (fp16, last d)
                              there; 16-byte aligned; not read by svsa_build_mask */
   int32_t* pairs;         /* nullable [B, heads, nb]: the query blocks of each head in
-                             the order the attention takes them, two at a time (each
-                             item is 128 query rows walking the union of two kept
-                             lists, so partners that share kept blocks waste less).
-                             When non-NULL, svsa_build_mask fills it (a greedy pairing
-                             by kept-list overlap; needs bits) and svsa_attn_fwd reads
-                             it; it must be a permutation of 0..nb-1 per head (a caller
-                             that writes kv_idx itself passes NULL or its own table).
-                             NULL: the attention pairs blocks 2p and 2p + 1. */
+                             the order svsa_attn_fwd_paired takes them, two at a time
+                             (partners that share kept blocks leave more of the work
+                             to its 128-row pass).  When non-NULL, svsa_build_mask
+                             fills it (a greedy pairing by kept-list overlap; needs
+                             bits) and svsa_attn_fwd_paired reads it; it must be a
+                             permutation of 0..nb-1 per head (a caller that writes
+                             kv_idx itself passes NULL or its own table).  NULL: blocks
+                             2p and 2p + 1 go together.  svsa_attn_fwd and
+                             svsa_attn_fwd_split do not read it (beyond the check). */
   int32_t check;          /* svsa_attn_fwd only: nonzero = first validate every list
                              (kv_cnt in [0, cap], indices in [0, nb), strictly
                              ascending) and the pairing table when given (a
@@ -394,6 +395,51 @@ typedef struct {
  * out may alias base. */
 svsa_status svsa_schedule_step(const svsa_schedule* sch, int32_t step, const svsa_mask_params* base,
                                svsa_mask_params* out, int32_t* rebuild);
+
+/* ---- the whole layer on host buffers ------------------------------------ */
+
+/* A layer object that owns every device buffer of the four steps, for
+ * callers whose q, k, v and output live in host memory.  Configuration: */
+typedef struct {
+  int32_t order;          /* svsa_order (RASTER or HILBERT) */
+  svsa_mask_params mask;  /* the selection rule; mask.step is set by each call */
+  int32_t compensate;     /* 1: centroid compensation of the skipped blocks */
+  int32_t attn_passes;    /* key-range passes of the attention, [1, 8] */
+  int32_t paired;         /* 1: the attention as svsa_attn_fwd_paired */
+  int32_t groups;         /* row groups the host path streams, [1, B * heads] */
+} svsa_layer_config;
+
+typedef struct svsa_layer svsa_layer;
+
+/* Allocate the layer's device memory on the current device (about
+ * B * heads * Npad * d * 18 bytes plus the mask and workspaces) and build its
+ * token order.  Synchronous.  *out is NULL on failure. */
+svsa_status svsa_layer_create(svsa_shape s, const svsa_layer_config* cfg, svsa_layer** out);
+
+/* Device bytes a layer of this shape and configuration holds (0 for an
+ * invalid request). */
+size_t svsa_layer_device_bytes(svsa_shape s, const svsa_layer_config* cfg);
+
+/* One layer call on host buffers: q, k, v, o are bf16 [B, heads, N, d] in
+ * raster order (host memory; pinned memory lets the copies overlap the
+ * work).  The rows (batch, head) go in cfg->groups groups: each group's
+ * inputs are copied in on one stream, each group's reorder, block mask,
+ * attention and inverse reorder run on `stream` once its inputs have
+ * arrived, and its output is copied out on a third stream, so the copies of
+ * one group overlap the work of another.  Asynchronous with respect to the
+ * host: o is complete when `stream` reaches the point of this call, and the
+ * inputs must stay unchanged until then.  step: the denoising step (the
+ * structured rule's anchor rotation).  flags: SVSA_LAYER_REUSE_MASK keeps the
+ * mask of the previous call (built if there is none).  Calls on one layer
+ * must be made from one stream.  The result equals the device-side sequence
+ * of svsa_reorder / svsa_reorder_values, svsa_build_mask, the attention entry
+ * point and svsa_inverse_reorder on the whole layer. */
+enum { SVSA_LAYER_REUSE_MASK = 1 };
+svsa_status svsa_layer_forward_host(svsa_layer* layer, const void* q, const void* k, const void* v, void* o,
+                                    int32_t step, int32_t flags, void* stream);
+
+/* Free the layer (after the work queued on it has completed).  NULL is a no-op. */
+svsa_status svsa_layer_destroy(svsa_layer* layer);
 
 /* ---- status ------------------------------------------------------------- */
 

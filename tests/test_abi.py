@@ -47,7 +47,8 @@ def test_struct_layouts_match_the_c_compiler(tmp_path):
     import subprocess
     if shutil.which("gcc") is None:
         pytest.skip("gcc not available")
-    structs = {"svsa_shape": Shape, "svsa_mask_params": MaskParams, "svsa_mask": Mask}
+    structs = {"svsa_shape": Shape, "svsa_mask_params": MaskParams, "svsa_mask": Mask,
+               "svsa_layer_config": svsa.LayerConfig}
     lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "svsa.h"', "int main(void) {"]
     for cname, cls in structs.items():
         lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
@@ -269,3 +270,32 @@ def test_default_attention_passes():
     assert default_attn_passes(svsa.SEL_THRESHOLD, 3488 * 64, 128) == 4     # HunyuanVideo, 114 MB
     assert default_attn_passes(svsa.SEL_STRUCTURED, 3072 * 64, 128) == 1    # the 6x Wan layer, 101 MB
     assert default_attn_passes(svsa.SEL_TOPK, rows(1024 * mb), 128) == 8    # capped
+
+
+def test_layer_configuration_checks_need_no_gpu():
+    # the host-buffer layer validates its configuration before any CUDA call
+    lib = svsa.lib()
+    s = svsa.shape(1, 12, 21, 30, 52, 128)
+    mp = svsa.mask_params(svsa.SEL_THRESHOLD)
+    good = svsa.layer_config(svsa.ORDER_HILBERT, mp, groups=12)
+    nb, npad, N = 512, 512 * 64, 21 * 30 * 52
+    # at least: four reordered and four raster token tensors, the lists at cap = nb
+    need = 12 * (4 * npad + 4 * N) * 128 * 2 + 12 * nb * nb * 4
+    assert svsa.svsa_layer_device_bytes(s, good) >= need
+    comp = svsa.layer_config(svsa.ORDER_HILBERT, mp, compensate=True, attn_passes=2, groups=3)
+    assert svsa.svsa_layer_device_bytes(s, comp) > svsa.svsa_layer_device_bytes(s, good)
+    h = ctypes.c_void_p(1)
+    bad = [(svsa.layer_config(2, mp), 2),                          # the co-clustering order: unsupported
+           (svsa.layer_config(svsa.ORDER_RASTER, mp, groups=0), 1),
+           (svsa.layer_config(svsa.ORDER_RASTER, mp, groups=13), 1),
+           (svsa.layer_config(svsa.ORDER_RASTER, mp, attn_passes=9), 1)]
+    for cfg, status in bad:
+        assert svsa.svsa_layer_device_bytes(s, cfg) == 0
+        assert lib.svsa_layer_create(s, ctypes.byref(cfg), ctypes.byref(h)) == status
+        assert h.value is None
+        assert lib.svsa_last_error()
+    assert lib.svsa_layer_create(svsa.shape(1, 12, 21, 30, 52, 96), ctypes.byref(good), ctypes.byref(h)) == 2
+    assert lib.svsa_layer_create(s, None, ctypes.byref(h)) == 1
+    assert lib.svsa_layer_create(s, ctypes.byref(good), None) == 1
+    assert lib.svsa_layer_forward_host(None, 16, 16, 16, 16, 0, 0, None) == 1
+    assert lib.svsa_layer_destroy(None) == 0

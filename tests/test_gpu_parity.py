@@ -334,6 +334,43 @@ def test_forward_host_matches_device_call(select, groups, kw):
     assert torch.equal(hout2, hout)
 
 
+@pytest.mark.parametrize("select,groups,kw", [
+    ("topk", 1, dict(order="raster")),
+    ("threshold", 3, dict(routing=True, compensate=True)),
+    ("threshold", 8, dict(sub=16, passes=2)),
+    ("structured", 2, dict(n_anchors=2)),
+    ("topk", 4, dict(paired=True, d=64)),
+])
+def test_layer_entry_point_on_host_buffers(select, groups, kw):
+    """svsa_layer_forward_host (the C entry point on host buffers, with its own
+    copy streams) gives bit for bit the device pipeline's output, over steps
+    that rebuild the mask and steps that reuse it."""
+    kw = dict(kw)
+    sub, passes, paired = kw.pop("sub", 64), kw.pop("passes", 1), kw.pop("paired", False)
+    w = _small(select, sub, grid=(6, 12, 20), heads=8, tau=0.9, keep_frac=0.3, **kw)
+    mk = lambda: svsa.SparseVideoAttention(w.B, w.heads, w.T, w.H, w.W, w.d, order=w.order, select=w.select,
+                                           tau=w.tau, keep_frac=w.keep_frac, sub_block=sub, n_anchors=w.n_anchors,
+                                           routing=w.routing, compensate=w.compensate, attn_passes=passes,
+                                           paired_split=paired, device="cuda")
+    ref_layer = mk()
+    cfg = svsa.layer_config(svsa.ORDER_HILBERT if w.order == "hilbert" else svsa.ORDER_RASTER, ref_layer.params,
+                            compensate=w.compensate, attn_passes=passes, paired=paired, groups=groups)
+    h = svsa.svsa_layer_create(ref_layer.shape, cfg)
+    try:
+        for step, reuse in ((0, False), (1, True), (2, False)):
+            q, k, v = (t.cuda() for t in workloads.make_qkv(w, seed=10 + step))
+            ref = ref_layer(q, k, v, step=step, reuse_mask=reuse).cpu()
+            hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+            hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+            svsa.svsa_layer_forward_host(h, hq, hk, hv, hout, step=step,
+                                         flags=svsa.LAYER_REUSE_MASK if reuse else 0)
+            torch.cuda.synchronize()
+            assert torch.equal(hout, ref), f"step {step}"
+        svsa.svsa_sync_status()
+    finally:
+        svsa.svsa_layer_destroy(h)
+
+
 @pytest.mark.parametrize("d", [64, 128])
 def test_dense_and_random_masks(d):
     T, H, W = 5, 7, 9
