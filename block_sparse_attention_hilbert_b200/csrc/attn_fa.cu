@@ -8,32 +8,42 @@
 //
 // Design:
 //   * Work item = two query blocks I0, I1 of one head (128 query rows, the
-//     M of a full-rate MMA).  The item walks the ascending union of their
-//     kept lists, two key blocks (128 keys) per tile; a 64 x 64 quarter whose
-//     key block the row's own query block does not keep is masked (and costs
-//     no exponentials).  The union costs extra tensor work where the two
-//     lists differ; in exchange every product is M = 128 x N = 128 and the
-//     softmax needs no cross-thread reduction.
+//     M of a full-rate MMA; the blocks 2p, 2p + 1, or entries 2p, 2p + 1 of
+//     a pairing table).  The item walks the ascending union of their kept
+//     lists -- or, for the shared pass of the paired-block split, only
+//     their intersection -- two key blocks (128 keys) per tile; a 64 x 64
+//     quarter whose key block the row's own query block does not keep is
+//     masked (and costs no exponentials).
 //        S [128 q x 128 k]  = Q [128 x d] . K_pair^T        (A, B from smem, K-major)
-//        O [128 q x d]     += P [128 x 128] . V_pair [128 x d]
+//        O [128 q x d]     += P [128 x 64] . V_block [64 x d]   (one per key block)
 //     with P in tensor memory (the A operand), V from smem (MN-major).
-//   * TMEM: two S buffers of 128 columns; each half of a tile (64 keys) writes
-//     its P as fp16 pairs over the first 32 of its own 64 S columns; two
-//     accumulators O_A, O_B (d columns each), one per half.
+//   * The two key blocks of a tile are two independent halves: softmax
+//     warpgroup h (warps 4-7 for the first block, 8-11 for the second)
+//     keeps, for every row, its own running maximum, row sum and output
+//     accumulator O_h in TMEM, and the halves are merged once per item by
+//     the log-sum-exp rule.  Neither half waits for the other inside a tile.
+//   * TMEM: two S buffers of 128 columns; half h writes its P as fp16 pairs
+//     over the first 32 of its own 64 S columns; O_A, O_B (d columns each).
 //   * Warp roles: warp 0 TMA of Q (once per item) and of the K tiles, warp 1
 //     TMA of the V tiles, warp 2 issues the S products and owns TMEM, warp 3
-//     issues the P.V products, warps 4-7 are the softmax warpgroup: thread t
-//     owns query row t (TMEM lane t) -- its scores, running maximum, row sum
-//     and output row.
+//     issues the P.V products, warps 4-11 the two softmax warpgroups; thread
+//     t of a group owns query row t (TMEM lane t) of its half.
 //   * Softmax: the row maximum is thread-local.  The reference maximum m is
 //     lazy: a tile only raises it when a score exceeds m by more than 2^12
 //     (fp16 P then stays <= 2^12); raising it rescales the row sum and the
-//     thread's O row in TMEM, after the previous P.V product has finished
-//     (its slot barrier).  Otherwise exp2(x - m) is taken against the stale
-//     m, exact up to the final normalisation.
+//     half's O row in TMEM, after that half's previous P.V product has
+//     finished.  Otherwise exp2(x - m) is taken against the stale m, exact
+//     up to the final normalisation.  Every decision that guards a TMEM
+//     access or a warp sync is warp-uniform (tcgen05.ld / st are
+//     warp-collective).
+//   * Merge mode (m_in, lse_in): the epilogue also folds in a partial result
+//     over other keys -- normalised fp32 rows and their log-sum-exp, as the
+//     64-row kernel writes them for the paired-block split -- by the same
+//     rule; an item with no tile copies that partial.
 //   * Every role walks the same merged list itself, so no schedule is
 //     stored; all hand-offs are mbarriers, every wait is bounded in time and
-//     a timeout sets an error word read by svsa_sync_status.
+//     a timeout sets an error word read by svsa_sync_status; exits are agreed
+//     by the two warps of a row at an OR-barrier.
 //   * Compensation ("SVG-EAR" 2.A): after the union tiles an item walks
 //     ceil(nb / 128) centroid tiles (128 block means as keys, value means as
 //     values, 16-bit copies of the fp32 means); a row's centroid column J
@@ -41,6 +51,10 @@
 //     it keeps J.
 //   * Counts and indices read from the mask are clamped to the tensors, so a
 //     malformed list gives a wrong result, never an access outside them.
+//
+// This kernel serves the dense denominator (every key block, no list) and
+// the shared pass of svsa_attn_fwd_paired; the sparse entry points use the
+// 64-row kernel (attn_tc.cu), which is faster on sparse lists.
 #include <climits>
 #include <cstddef>
 

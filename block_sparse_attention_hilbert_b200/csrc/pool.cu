@@ -6,8 +6,11 @@
 //
 // One CTA reads one 64-row block (d*128 bytes) with 16-byte loads: 16 (d=128)
 // or 32 (d=64) row lanes x CPR chunk lanes; each thread keeps fp32 partial
-// sums of its rows per group, and the row lanes are added in a fixed order
-// through shared memory, so the result is deterministic.
+// sums of its rows per group, the row lanes of a warp are added by shuffles
+// and the warps' partials in a fixed order through shared memory, so the
+// result is deterministic.  (Adding in the warp first keeps the shared
+// buffer at one row of partials per warp, which lets more CTAs, and so more
+// loads, be resident on an SM.)
 //
 // Optional second output for the tensor-core scores: each mean m as an fp16
 // pair, split[bh, g, :] = [hi (d) | lo (d)] with hi = fp16(m) and
@@ -39,7 +42,8 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(
   constexpr int RL = kPoolThreads / CPR;     // row lanes
   constexpr int RPT = kBlock / RL;           // rows per thread
   constexpr int G = kBlock / SIZE;           // groups per 64-row block
-  __shared__ float red[RL][G][D];
+  constexpr int NW = kPoolThreads / 32;      // warps; a warp holds 32 / CPR row lanes
+  __shared__ float red[NW][G][D];
 
   const int blk = blockIdx.x;
   const long long bh = blockIdx.y;
@@ -73,16 +77,26 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(
       }
     }
   }
+  // the warp's row lanes (lanes ch, ch + CPR, ...) into its first CPR lanes
 #pragma unroll
-  for (int g = 0; g < G; ++g)
+  for (int o = CPR; o < 32; o <<= 1)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) red[rl][g][ch * 8 + e] = acc[g][e];
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[g][e] += __shfl_xor_sync(0xffffffffu, acc[g][e], o);
+  const int warp = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) < CPR) {
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) red[warp][g][ch * 8 + e] = acc[g][e];
+  }
   __syncthreads();
   for (int o = threadIdx.x; o < G * D; o += kPoolThreads) {
     const int g = o / D, c = o % D;
     float s = 0.f;
-#pragma unroll 8
-    for (int l = 0; l < RL; ++l) s += red[l][g][c];
+#pragma unroll
+    for (int l = 0; l < NW; ++l) s += red[l][g][c];
     const long long grow = row0 + (long long)g * SIZE;
     const long long n = std::max<long long>(0, std::min<long long>(SIZE, N - grow));
     const long long gidx = (long long)blk * G + g;
