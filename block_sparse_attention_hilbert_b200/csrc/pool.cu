@@ -4,13 +4,14 @@
 // 2.A (a cluster centroid is its mean).  out[bh, g, :] = mean of the valid
 // rows (position < N) of group g = rows [g*SIZE, g*SIZE + SIZE); 0 if none.
 //
-// One CTA reads one 64-row block (d*128 bytes) with 16-byte loads: 16 (d=128)
-// or 32 (d=64) row lanes x CPR chunk lanes; each thread keeps fp32 partial
-// sums of its rows per group, the row lanes of a warp are added by shuffles
-// and the warps' partials in a fixed order through shared memory, so the
-// result is deterministic.  (Adding in the warp first keeps the shared
-// buffer at one row of partials per warp, which lets more CTAs, and so more
-// loads, be resident on an SM.)
+// One CTA reads one 64-row block (d*128 bytes) with 16-byte loads: CPR chunk
+// lanes x 256 / CPR row lanes, row lane l taking the consecutive rows
+// [l * RPT, l * RPT + RPT), so a warp covers 8 consecutive rows and lies in
+// one group (groups are 16 or 64 rows).  Each thread sums its rows in fp32,
+// the row lanes of a warp are added by shuffles, and the warps of a group in
+// a fixed order through shared memory, so the result is deterministic.  One
+// accumulator row per thread and one partial row per warp keep registers and
+// shared memory small, so many CTAs -- and their loads -- are resident.
 //
 // Optional second output for the tensor-core scores: each mean m as an fp16
 // pair, split[bh, g, :] = [hi (d) | lo (d)] with hi = fp16(m) and
@@ -40,10 +41,12 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(
     __nv_bfloat16* __restrict__ split_bf, int32_t* __restrict__ nvalid, long long N, long long Npad) {
   constexpr int CPR = D / 8;                 // 16-byte chunks per row
   constexpr int RL = kPoolThreads / CPR;     // row lanes
-  constexpr int RPT = kBlock / RL;           // rows per thread
+  constexpr int RPT = kBlock / RL;           // consecutive rows per thread
   constexpr int G = kBlock / SIZE;           // groups per 64-row block
-  constexpr int NW = kPoolThreads / 32;      // warps; a warp holds 32 / CPR row lanes
-  __shared__ float red[NW][G][D];
+  constexpr int NW = kPoolThreads / 32;      // warps
+  constexpr int WR = kBlock / NW;            // rows per warp (8)
+  static_assert(WR * NW == kBlock && SIZE % WR == 0, "a warp's rows lie in one group");
+  __shared__ float red[NW][D];
 
   const int blk = blockIdx.x;
   const long long bh = blockIdx.y;
@@ -51,52 +54,42 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(
   const long long row0 = (long long)blk * kBlock;
   const T2* base = xp + (bh * Npad + row0) * (D / 2);
 
-  float acc[G][8];
+  float acc[8];
 #pragma unroll
-  for (int g = 0; g < G; ++g)
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  uint4 v[RPT];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
-
+  for (int u = 0; u < RPT; ++u) {            // all loads first
+    const int r = rl * RPT + u;
+    v[u] = row0 + r < N ? __ldg(reinterpret_cast<const uint4*>(base + (long long)r * (D / 2)) + ch)
+                        : make_uint4(0u, 0u, 0u, 0u);
+  }
 #pragma unroll
   for (int u = 0; u < RPT; ++u) {
-    const int r = rl + RL * u;
-    if (row0 + r < N) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(base + (long long)r * (D / 2)) + ch);
-      const T2* p = reinterpret_cast<const T2*>(&v);
-      const int g = r / SIZE;
+    const T2* p = reinterpret_cast<const T2*>(&v[u]);
 #pragma unroll
-      for (int gg = 0; gg < G; ++gg) {
-        if (gg == g) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = pair_to_float2(p[e]);
-            acc[gg][2 * e] += f.x;
-            acc[gg][2 * e + 1] += f.y;
-          }
-        }
-      }
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = pair_to_float2(p[e]);
+      acc[2 * e] += f.x;
+      acc[2 * e + 1] += f.y;
     }
   }
   // the warp's row lanes (lanes ch, ch + CPR, ...) into its first CPR lanes
 #pragma unroll
   for (int o = CPR; o < 32; o <<= 1)
 #pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[g][e] += __shfl_xor_sync(0xffffffffu, acc[g][e], o);
+    for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
   const int warp = threadIdx.x >> 5;
   if ((threadIdx.x & 31) < CPR) {
 #pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) red[warp][g][ch * 8 + e] = acc[g][e];
+    for (int e = 0; e < 8; ++e) red[warp][ch * 8 + e] = acc[e];
   }
   __syncthreads();
   for (int o = threadIdx.x; o < G * D; o += kPoolThreads) {
     const int g = o / D, c = o % D;
-    float s = 0.f;
+    float s = 0.f;                           // the group's warps, in order
 #pragma unroll
-    for (int l = 0; l < NW; ++l) s += red[l][g][c];
+    for (int l = 0; l < SIZE / WR; ++l) s += red[g * (SIZE / WR) + l][c];
     const long long grow = row0 + (long long)g * SIZE;
     const long long n = std::max<long long>(0, std::min<long long>(SIZE, N - grow));
     const long long gidx = (long long)blk * G + g;
