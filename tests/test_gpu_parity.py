@@ -366,6 +366,13 @@ def test_layer_entry_point_on_host_buffers(select, groups, kw):
                                          flags=svsa.LAYER_REUSE_MASK if reuse else 0)
             torch.cuda.synchronize()
             assert torch.equal(hout, ref), f"step {step}"
+        # pageable host memory: the copies no longer overlap, the result is the same
+        pq, pk, pv = (t.clone() for t in (hq, hk, hv))
+        pout = torch.empty(q.shape, dtype=q.dtype)
+        assert not pq.is_pinned() and not pout.is_pinned()
+        svsa.svsa_layer_forward_host(h, pq, pk, pv, pout, step=2, flags=svsa.LAYER_REUSE_MASK)
+        torch.cuda.synchronize()
+        assert torch.equal(pout, ref)
         svsa.svsa_sync_status()
     finally:
         svsa.svsa_layer_destroy(h)
