@@ -492,7 +492,7 @@ def run_svsa(args):
     hk = [t.cpu().pin_memory() for t in ks]
     hv = v.cpu().pin_memory()
     hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    e2e_groups = min(24, w.B * w.heads)
+    e2e_groups = min(12, w.B * w.heads)
     # (the co-clustering order is built from the layer's device tensors: that
     # order streams through the Python layer object instead)
     layer = None if attn.cocluster else svsa.svsa_layer_create(attn.shape, svsa.layer_config(
