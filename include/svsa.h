@@ -26,6 +26,10 @@
  *      block centroid).
  *   4. svsa_inverse_reorder -- put the output back in raster order.
  *
+ * svsa_layer_create / svsa_layer_forward_host run the four steps on host
+ * buffers (a layer object that owns its device memory and streams the rows
+ * through the entry points above).
+ *
  * Conventions shared by every entry point
  *   - Tensors are row-major and contiguous.  Q, K, V and O in raster order are
  *     bf16 [B, heads, N, d] with N = T*H*W; the reordered ("p") tensors are
@@ -33,7 +37,9 @@
  *     N..Npad-1 of a reordered tensor are zero pads; they never count in a
  *     mean, a softmax or an output.
  *   - Every pointer is a device pointer owned by the caller, and must be
- *     16-byte aligned.  The library allocates no memory and keeps no state.
+ *     16-byte aligned.  The library allocates no memory and keeps no state
+ *     (the svsa_layer_* object excepted: it owns its arena, and its
+ *     forward call takes host pointers).
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream) and returns after enqueueing its kernels.
  *   - Arguments are validated before anything is launched.  A failed
