@@ -54,7 +54,11 @@ cudaError_t launch_centroid16(const float* kbar, const float* vbar, void* cbar, 
 cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, const int32_t* kv_idx,
                            const int32_t* kv_cnt, int cap, const uint32_t* bits, const void* cbar, void* o,
                            float* lse, long long BH, long long N, int nb, int d, bool dense, cudaStream_t st,
-                           float* o32 = nullptr, float lse_empty = 0.f);
+                           float* o32 = nullptr, float lse_empty = 0.f, const int32_t* sched = nullptr,
+                           long long nwaves = 0);
+long long attn_tc_grid(long long items);
+cudaError_t launch_sched(const int32_t* cnt_p, long long items, int cap, int P, int G, long long nwaves,
+                         int32_t* sched, cudaStream_t st);
 cudaError_t launch_attn_fa(const void* q, const void* k, const void* v, const int32_t* kv_idx,
                            const int32_t* kv_cnt, int cap, const uint32_t* bits, const void* cbar, void* o,
                            float* lse, long long BH, long long N, int nb, int d, bool dense, cudaStream_t st,
@@ -624,24 +628,26 @@ svsa_status svsa_attn_fwd(const void* qp, const void* kp, const void* vp, const 
 
 namespace {
 struct SplitWs {
-  size_t idx, cnt, o, lse, xidx, xcnt, part, plse, total;
+  size_t idx, cnt, o, lse, sched, xidx, xcnt, part, plse, total;
 };
+constexpr int kSchedMaxCtas = 256;   // the item schedule serves grids of up to this many CTAs
 // Workspace of svsa_attn_fwd_split / svsa_attn_fwd_paired: the P range lists
-// and per-pass outputs (P > 1), then (paired) the exclusive lists and the
-// fp32 partial of the paired-block split.
+// and per-pass outputs (P > 1), the item schedule of every pass (split), then
+// (paired) the exclusive lists and the fp32 partial of the paired-block split.
 SplitWs split_layout(const Dims& g, int P, bool paired) {
   SplitWs w{};
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o = off; off += (bytes + 255) & ~(size_t)255; return o; };
   const long long rows = g.BH * g.nb;
   const int R = (g.nb + P - 1) / P;
-  w.idx = w.cnt = w.o = w.lse = w.xidx = w.xcnt = w.part = w.plse = SIZE_MAX;
+  w.idx = w.cnt = w.o = w.lse = w.sched = w.xidx = w.xcnt = w.part = w.plse = SIZE_MAX;
   if (P > 1) {
     w.idx = take((size_t)P * rows * R * 4);
     w.cnt = take((size_t)P * rows * 4);
     w.o = take((size_t)P * g.BH * g.Npad * g.d * 4);
     w.lse = take((size_t)P * g.BH * g.Npad * 4);
   }
+  if (!paired) w.sched = take((size_t)P * (rows + kSchedMaxCtas) * 4);     // [P][waves][grid]
   if (paired) {
     w.xidx = take((size_t)rows * std::min(R, g.nb) * 4);
     w.xcnt = take((size_t)rows * 4);
@@ -706,6 +712,7 @@ svsa_status attn_split(const void* qp, const void* kp, const void* vp, const svs
   int32_t* xcnt = reinterpret_cast<int32_t*>(at(w.xcnt));
   float* part = reinterpret_cast<float*>(at(w.part));
   float* plse = reinterpret_cast<float*>(at(w.plse));
+  int32_t* sched = reinterpret_cast<int32_t*>(at(w.sched));
   const long long rows = g.BH * g.nb;
   const int R = (g.nb + passes - 1) / passes;
   if (m->check) {
@@ -720,6 +727,14 @@ svsa_status attn_split(const void* qp, const void* kp, const void* vp, const svs
     SVSA_TRY(cuda_status(counted(launch_split_mask(m->kv_idx, m->kv_cnt, m->cap, rows, g.nb, passes, R, idx_p, cnt_p,
                                                    st), 1),
                          "split mask"));
+  // every pass's items balanced over the attention's persistent CTAs
+  const long long grid = attn_tc_grid(rows);
+  const long long nwaves = (rows + grid - 1) / grid;
+  const bool use_sched = sched != nullptr && grid <= kSchedMaxCtas;
+  if (use_sched)
+    SVSA_TRY(cuda_status(counted(launch_sched(passes > 1 ? cnt_p : m->kv_cnt, rows, passes > 1 ? R : m->cap, passes,
+                                              (int)grid, nwaves, sched, st), 1),
+                         "item schedule"));
   const long long rows_o = g.BH * g.Npad;
   for (int p = 0; p < passes; ++p) {
     // this pass's lists; the centroid tiles of the skipped blocks go with the last pass
@@ -731,8 +746,11 @@ svsa_status attn_split(const void* qp, const void* kp, const void* vp, const svs
     float* out_lse = passes > 1 ? lse_p + (long long)p * rows_o : lse;
     if (!hybrid) {
       SVSA_TRY(cuda_status(counted(launch_attn_tc(qp, kp, vp, L_idx, L_cnt, L_cap, comp ? m->bits : nullptr,
-                                                   comp ? m->cbar : nullptr, nullptr, out_lse, g.BH, g.N, g.nb, g.d,
-                                                   false, st, out32, -INFINITY), 1),
+                                                   comp ? m->cbar : nullptr, passes > 1 ? nullptr : op, out_lse,
+                                                   g.BH, g.N, g.nb, g.d, false, st, out32,
+                                                   passes > 1 ? -INFINITY : 0.f,
+                                                   use_sched ? sched + (long long)p * nwaves * grid : nullptr,
+                                                   nwaves), 1),
                            "attn_fwd pass launch"));
       continue;
     }
@@ -764,7 +782,8 @@ svsa_status attn_split(const void* qp, const void* kp, const void* vp, const svs
 svsa_status svsa_attn_fwd_split(const void* qp, const void* kp, const void* vp, const svsa_mask* m,
                                 int32_t compensate, void* op, float* lse, svsa_shape s, int32_t passes, void* ws,
                                 size_t ws_bytes, void* stream) {
-  if (passes == 1) return svsa_attn_fwd(qp, kp, vp, m, compensate, op, lse, s, stream);
+  // one pass without a workspace: the plain call (no item schedule)
+  if (passes == 1 && (ws == nullptr || ws_bytes == 0)) return svsa_attn_fwd(qp, kp, vp, m, compensate, op, lse, s, stream);
   NvtxRange nvtx_("svsa_attn_fwd_split");
   return attn_split(qp, kp, vp, m, compensate, op, lse, s, passes, ws, ws_bytes, stream, false);
 }

@@ -119,7 +119,24 @@ struct Args {
   long long items;
   float scale_log2;
   int dense;
+  const int32_t* sched;    // nullable [nwaves][gridDim.x]: each wave's item per CTA (-1 = none)
+  long long nwaves;
 };
+
+// The j-th item of this CTA: wave j's entry of the schedule (-1 = none in
+// that wave), or without one item blockIdx.x + j * gridDim.x.  False once
+// the CTA has no further wave.  Every role of the CTA walks the same
+// sequence.
+__device__ __forceinline__ bool cta_item(const Args& a, long long j, long long& it) {
+  if (a.sched == nullptr) {
+    it = (long long)blockIdx.x + j * gridDim.x;
+    return it < a.items;
+  }
+  if (j >= a.nwaves) return false;
+  const int v = a.sched[j * gridDim.x + blockIdx.x];
+  it = (v >= 0 && (long long)v < a.items) ? v : -1;
+  return true;
+}
 
 // Column reduction of v[0..NC-1] across the 32 lanes of a warp: halving
 // exchanges over lane bits log2(NC)-1 .. 0 leave lane l with column l % NC
@@ -205,7 +222,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ms->tmem_base;
-  const long long items = a.items;
   const int nb = a.nb;
   const int ncent = COMP ? a.ncent : 0;          // centroid tiles per item
 
@@ -229,7 +245,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const bool is_k = warp == 0;
       uint32_t qit = 0, it_n = 0;
       bool ok = true;
-      for (long long it = blockIdx.x; it < items && ok; it += gridDim.x) {
+      for (long long j = 0; ok; ++j) {
+        long long it;
+        if (!cta_item(a, j, it)) break;
+        if (it < 0) continue;
         const int cnt = item_count(it);
         const int npairs = (cnt + 1) >> 1;
         const int ntiles = npairs + ncent;
@@ -306,7 +325,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const uint64_t dP = sdesc(sbase + kOffP, 16384, 1024);
       uint32_t ring = 0, tiles = 0, qit = 0, oit = 0;
       bool ok = true;
-      for (long long it = blockIdx.x; it < items && ok; it += gridDim.x) {
+      for (long long j = 0; ok; ++j) {
+        long long it;
+        if (!cta_item(a, j, it)) break;
+        if (it < 0) continue;
         const int cnt = item_count(it);
         const int npairs = ((cnt + 1) >> 1) + ncent;       // pair tiles, then centroid tiles
         if (npairs == 0) continue;
@@ -394,7 +416,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const uint32_t pa0 = sbase + kOffP + (uint32_t)((k >> 3) * 1024 + (k & 7) * 128) +
                          (uint32_t)(((2 * wg) ^ (k & 7)) << 4);
     bool stop = false;
-    for (long long it = blockIdx.x; it < items && !stop; it += gridDim.x) {
+    for (long long j = 0; !stop; ++j) {
+      long long it;
+      if (!cta_item(a, j, it)) break;
+      if (it < 0) continue;
       const int cnt = item_count(it);
       const long long bh = it / nb;
       const int I = (int)(it % nb);
@@ -628,10 +653,13 @@ bool make_map(CUtensorMap* m, const void* base, long long rows, int d, bool f16)
 
 }  // namespace
 
+// Persistent grid of the 64-row kernel for `items` work items: one CTA per SM.
+long long attn_tc_grid(long long items) { return std::min<long long>(items, tc::sm_count()); }
+
 cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, const int32_t* kv_idx,
                            const int32_t* kv_cnt, int cap, const uint32_t* bits, const void* cbar, void* o,
                            float* lse, long long BH, long long N, int nb, int d, bool dense, cudaStream_t st,
-                           float* o32, float lse_empty) {
+                           float* o32, float lse_empty, const int32_t* sched, long long nwaves) {
   CUtensorMap mq, mk, mv, mc;
   const long long rows = BH * (long long)nb * kBlock;
   if (!make_map(&mq, q, rows, d, false) || !make_map(&mk, k, rows, d, false) || !make_map(&mv, v, rows, d, true))
@@ -649,7 +677,10 @@ cudaError_t launch_attn_tc(const void* q, const void* k, const void* v, const in
   a.items = BH * nb;
   a.scale_log2 = 1.4426950408889634f / sqrtf((float)d);
   a.dense = dense ? 1 : 0;
-  const long long grid = std::min<long long>(a.items, tc::sm_count());
+  const long long grid = attn_tc_grid(a.items);
+  a.sched = sched;
+  a.nwaves = nwaves;
+  if (sched != nullptr && nwaves < (a.items + grid - 1) / grid) return cudaErrorInvalidValue;
   const bool comp = a.ncent > 0;
   auto go = [&](auto kernel) -> cudaError_t {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kSmemBytes);

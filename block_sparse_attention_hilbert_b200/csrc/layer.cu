@@ -264,11 +264,9 @@ svsa_status svsa_layer_forward_host(svsa_layer* L, const void* q, const void* k,
     if (L->cfg.paired)
       LTRY(svsa_attn_fwd_paired(gq, gk, gv, &m, L->cfg.compensate, go, nullptr, gs, L->cfg.attn_passes,
                                 L->attn_ws, L->attn_ws_bytes, cs));
-    else if (L->cfg.attn_passes > 1)
+    else
       LTRY(svsa_attn_fwd_split(gq, gk, gv, &m, L->cfg.compensate, go, nullptr, gs, L->cfg.attn_passes,
                                L->attn_ws, L->attn_ws_bytes, cs));
-    else
-      LTRY(svsa_attn_fwd(gq, gk, gv, &m, L->cfg.compensate, go, nullptr, gs, cs));
     LTRY(svsa_inverse_reorder(go, rawm(L->so, r0), L->iperm, gs, cs));
     LTRY(cuda_err(cudaEventRecord(L->ev_out[gi], cs), "event record"));
     LTRY(cuda_err(cudaStreamWaitEvent(L->d2h, L->ev_out[gi], 0), "stream wait"));

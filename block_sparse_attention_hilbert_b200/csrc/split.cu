@@ -12,7 +12,8 @@
 //
 // split_mask_kernel cuts every ascending kept list into its P range lists
 // (each at most R long, so the P masks together take the room of one);
-// combine_kernel merges the passes.
+// sched_kernel balances each pass's items over the attention's persistent
+// CTAs; combine_kernel merges the passes.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -144,7 +145,78 @@ __global__ void exclusive_kernel(const int32_t* __restrict__ kv_idx, const int32
   }
 }
 
+// Wave-by-wave longest-first assignment of one pass's items to the G
+// persistent CTAs of the attention (one CTA of this kernel per pass).  Wave w
+// holds items [w G, w G + G) -- neighbouring query blocks, which share their
+// keys in L2, so they still run together.  Its items, ranked by estimated
+// cost (descending, ties to the lower index), go to the CTAs ranked by the
+// cost already given to them (ascending, ties to the lower index), so after
+// every wave the CTAs' totals stay within about one item of each other.
+// Cost of an item: its pair tiles ((count + 1) / 2) plus 2 for the per-item
+// work; an empty item 1.  sched[p][w][b] = item index, or -1 (the last wave
+// of a pass whose items are not a multiple of G).
+constexpr int kSchedMaxG = 256;
+
+__global__ void __launch_bounds__(2 * kSchedMaxG) sched_kernel(const int32_t* __restrict__ cnt_p, long long items,
+                                                               int cap, int G, long long nwaves,
+                                                               int32_t* __restrict__ sched) {
+  __shared__ int cost[kSchedMaxG];
+  __shared__ long long load[kSchedMaxG];
+  __shared__ int16_t item_at[kSchedMaxG], cta_at[kSchedMaxG];
+  const int t = threadIdx.x;
+  const int32_t* cnt = cnt_p + (long long)blockIdx.x * items;
+  int32_t* out = sched + (long long)blockIdx.x * nwaves * G;
+  if (t < G) load[t] = 0;
+  for (long long w = 0; w < nwaves; ++w) {
+    const long long base = w * G;
+    if (t < G) {
+      int c = -1;                                  // no item in this slot
+      if (base + t < items) {
+        int k = cnt[base + t];
+        k = k < 0 ? 0 : (k > cap ? cap : k);
+        const int tiles = (k + 1) >> 1;
+        c = tiles > 0 ? tiles + 2 : 1;
+      }
+      cost[t] = c;
+    }
+    __syncthreads();
+    if (t < G) {                                   // rank of item t: cost descending
+      const int c = cost[t];
+      int r = 0;
+      for (int u = 0; u < G; ++u) {
+        const int cu = cost[u];
+        r += (cu > c) | ((cu == c) & (u < t));
+      }
+      item_at[r] = (int16_t)t;
+    } else if (t >= kSchedMaxG && t - kSchedMaxG < G) {   // rank of CTA b: load ascending
+      const int b = t - kSchedMaxG;
+      const long long L = load[b];
+      int r = 0;
+      for (int u = 0; u < G; ++u) {
+        const long long lu = load[u];
+        r += (lu < L) | ((lu == L) & (u < b));
+      }
+      cta_at[r] = (int16_t)b;
+    }
+    __syncthreads();
+    if (t < G) {
+      const int i = item_at[t], b = cta_at[t];
+      const int c = cost[i];
+      out[w * G + b] = c >= 0 ? (int32_t)(base + i) : -1;
+      if (c > 0) load[b] += c;
+    }
+    __syncthreads();
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_sched(const int32_t* cnt_p, long long items, int cap, int P, int G, long long nwaves,
+                         int32_t* sched, cudaStream_t st) {
+  if (G < 1 || G > kSchedMaxG || P < 1 || nwaves * G < items) return cudaErrorInvalidValue;
+  sched_kernel<<<(unsigned)P, 2 * kSchedMaxG, 0, st>>>(cnt_p, items, cap, G, nwaves, sched);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_exclusive(const int32_t* kv_idx, const int32_t* kv_cnt, int cap, const uint32_t* bits,
                              const int32_t* pairs, long long BH, int nb, int32_t* x_idx, int xcap, int32_t* x_cnt,

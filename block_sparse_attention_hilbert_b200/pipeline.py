@@ -151,8 +151,8 @@ class SparseVideoAttention:
         self.paired_split = bool(paired_split)
         ws_bytes = (svsa_attn_paired_workspace_bytes if self.paired_split
                     else svsa_attn_split_workspace_bytes)(self.shape, self.attn_passes)
-        self.buf.split_ws = (torch.empty(ws_bytes, dtype=torch.uint8, device=self.buf.qp.device)
-                             if self.attn_passes > 1 or self.paired_split else None)
+        # (every path has a workspace: at one pass it holds the item schedule)
+        self.buf.split_ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=self.buf.qp.device)
         if self.cocluster:
             rows, dev = B * heads, self.buf.qp.device
             b = self.buf
@@ -207,11 +207,9 @@ class SparseVideoAttention:
         if self.paired_split:
             svsa_attn_fwd_paired(b.qp, b.kp, b.vp, self._mask, self.compensate, b.op, lse, self.shape,
                                  self.attn_passes, b.split_ws, b.split_ws.numel(), stream)
-        elif self.attn_passes > 1:
+        else:
             svsa_attn_fwd_split(b.qp, b.kp, b.vp, self._mask, self.compensate, b.op, lse, self.shape,
                                 self.attn_passes, b.split_ws, b.split_ws.numel(), stream)
-        else:
-            svsa_attn_fwd(b.qp, b.kp, b.vp, self._mask, self.compensate, b.op, lse, self.shape, stream)
 
     def attend_dense(self, lse=None, stream=None):
         b = self.buf
@@ -318,13 +316,10 @@ class SparseVideoAttention:
                 svsa_attn_fwd_paired(self._rows(b.qp, r0, r1), self._rows(b.kp, r0, r1), self._rows(b.vp, r0, r1),
                                      m, self.compensate, self._rows(b.op, r0, r1), None, sh, self.attn_passes,
                                      b.split_ws, b.split_ws.numel(), compute)
-            elif self.attn_passes > 1:
+            else:
                 svsa_attn_fwd_split(self._rows(b.qp, r0, r1), self._rows(b.kp, r0, r1), self._rows(b.vp, r0, r1), m,
                                     self.compensate, self._rows(b.op, r0, r1), None, sh, self.attn_passes,
                                     b.split_ws, b.split_ws.numel(), compute)
-            else:
-                svsa_attn_fwd(self._rows(b.qp, r0, r1), self._rows(b.kp, r0, r1), self._rows(b.vp, r0, r1), m,
-                              self.compensate, self._rows(b.op, r0, r1), None, sh, compute)
             if self.cocluster:
                 svsa_inverse_reorder_heads(self._rows(b.op, r0, r1), dout[r0:r1], b.iperm_q[r0:r1], sh, compute)
             else:
