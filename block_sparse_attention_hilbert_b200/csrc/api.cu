@@ -631,8 +631,8 @@ struct SplitWs {
   size_t idx, cnt, o, lse, sched, xidx, xcnt, part, plse, total;
 };
 constexpr int kSchedMaxCtas = 256;   // the item schedule serves grids of up to this many CTAs
-// Workspace of svsa_attn_fwd_split / svsa_attn_fwd_paired: the P range lists
-// and per-pass outputs (P > 1), the item schedule of every pass (split), then
+// Workspace of svsa_attn_fwd_split / svsa_attn_fwd_paired: the P range lists,
+// per-pass outputs and the item schedule of every pass (P > 1, split), then
 // (paired) the exclusive lists and the fp32 partial of the paired-block split.
 SplitWs split_layout(const Dims& g, int P, bool paired) {
   SplitWs w{};
@@ -647,7 +647,7 @@ SplitWs split_layout(const Dims& g, int P, bool paired) {
     w.o = take((size_t)P * g.BH * g.Npad * g.d * 4);
     w.lse = take((size_t)P * g.BH * g.Npad * 4);
   }
-  if (!paired) w.sched = take((size_t)P * (rows + kSchedMaxCtas) * 4);     // [P][waves][grid]
+  if (!paired && P > 1) w.sched = take((size_t)P * (rows + kSchedMaxCtas) * 4);   // [P][waves][grid]
   if (paired) {
     w.xidx = take((size_t)rows * std::min(R, g.nb) * 4);
     w.xcnt = take((size_t)rows * 4);
@@ -782,8 +782,8 @@ svsa_status attn_split(const void* qp, const void* kp, const void* vp, const svs
 svsa_status svsa_attn_fwd_split(const void* qp, const void* kp, const void* vp, const svsa_mask* m,
                                 int32_t compensate, void* op, float* lse, svsa_shape s, int32_t passes, void* ws,
                                 size_t ws_bytes, void* stream) {
-  // one pass without a workspace: the plain call (no item schedule)
-  if (passes == 1 && (ws == nullptr || ws_bytes == 0)) return svsa_attn_fwd(qp, kp, vp, m, compensate, op, lse, s, stream);
+  // one pass: the plain call (measured, the item schedule does not pay for itself there)
+  if (passes == 1) return svsa_attn_fwd(qp, kp, vp, m, compensate, op, lse, s, stream);
   NvtxRange nvtx_("svsa_attn_fwd_split");
   return attn_split(qp, kp, vp, m, compensate, op, lse, s, passes, ws, ws_bytes, stream, false);
 }

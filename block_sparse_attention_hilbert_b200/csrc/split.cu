@@ -14,6 +14,8 @@
 // (each at most R long, so the P masks together take the room of one);
 // sched_kernel balances each pass's items over the attention's persistent
 // CTAs; combine_kernel merges the passes.
+#include <climits>
+
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -160,13 +162,19 @@ constexpr int kSchedMaxG = 256;
 __global__ void __launch_bounds__(2 * kSchedMaxG) sched_kernel(const int32_t* __restrict__ cnt_p, long long items,
                                                                int cap, int G, long long nwaves,
                                                                int32_t* __restrict__ sched) {
-  __shared__ int cost[kSchedMaxG];
-  __shared__ long long load[kSchedMaxG];
+  // slots G.. hold values that never rank before a real one (read in 16-byte vectors)
+  __shared__ __align__(16) int cost[kSchedMaxG];
+  __shared__ __align__(16) long long load[kSchedMaxG];
   __shared__ int16_t item_at[kSchedMaxG], cta_at[kSchedMaxG];
   const int t = threadIdx.x;
   const int32_t* cnt = cnt_p + (long long)blockIdx.x * items;
   int32_t* out = sched + (long long)blockIdx.x * nwaves * G;
-  if (t < G) load[t] = 0;
+  const int G4 = (G + 3) >> 2, G2 = (G + 1) >> 1;
+  if (t < kSchedMaxG) {
+    load[t] = t < G ? 0 : LLONG_MAX;
+    cost[t] = INT_MIN;
+  }
+  __syncthreads();
   for (long long w = 0; w < nwaves; ++w) {
     const long long base = w * G;
     if (t < G) {
@@ -180,23 +188,31 @@ __global__ void __launch_bounds__(2 * kSchedMaxG) sched_kernel(const int32_t* __
       cost[t] = c;
     }
     __syncthreads();
-    if (t < G) {                                   // rank of item t: cost descending
+    if (t < G) {                                   // rank of item t: cost descending, ties to the lower index
       const int c = cost[t];
-      int r = 0;
-      for (int u = 0; u < G; ++u) {
-        const int cu = cost[u];
-        r += (cu > c) | ((cu == c) & (u < t));
+      int r0 = 0, r1 = 0;
+#pragma unroll 4
+      for (int u4 = 0; u4 < G4; ++u4) {
+        const int4 v = reinterpret_cast<const int4*>(cost)[u4];
+        const int u = 4 * u4;
+        r0 += (v.x > c) | ((v.x == c) & (u < t));
+        r1 += (v.y > c) | ((v.y == c) & (u + 1 < t));
+        r0 += (v.z > c) | ((v.z == c) & (u + 2 < t));
+        r1 += (v.w > c) | ((v.w == c) & (u + 3 < t));
       }
-      item_at[r] = (int16_t)t;
-    } else if (t >= kSchedMaxG && t - kSchedMaxG < G) {   // rank of CTA b: load ascending
+      item_at[r0 + r1] = (int16_t)t;
+    } else if (t >= kSchedMaxG && t - kSchedMaxG < G) {   // rank of CTA b: load ascending, ties to the lower index
       const int b = t - kSchedMaxG;
       const long long L = load[b];
-      int r = 0;
-      for (int u = 0; u < G; ++u) {
-        const long long lu = load[u];
-        r += (lu < L) | ((lu == L) & (u < b));
+      int r0 = 0, r1 = 0;
+#pragma unroll 4
+      for (int u2 = 0; u2 < G2; ++u2) {
+        const longlong2 v = reinterpret_cast<const longlong2*>(load)[u2];
+        const int u = 2 * u2;
+        r0 += (v.x < L) | ((v.x == L) & (u < b));
+        r1 += (v.y < L) | ((v.y == L) & (u + 1 < b));
       }
-      cta_at[r] = (int16_t)b;
+      cta_at[r0 + r1] = (int16_t)b;
     }
     __syncthreads();
     if (t < G) {

@@ -304,13 +304,13 @@ svsa_status svsa_attn_fwd(const void* qp, const void* kp, const void* vp, const 
  * O = sum_p exp(lse_p - lse) O_p, lse = log sum_p exp(lse_p) (the softmax over
  * the union of disjoint key sets), so the result is svsa_attn_fwd's up to
  * rounding.  Compensation terms go with the last pass.  kv_idx rows must be
- * ascending (as svsa_build_mask writes them).  Every pass's work items
- * (query blocks) are assigned to the kernel's persistent CTAs by a schedule
- * computed on the device from the kept counts: wave by wave, the costliest
- * item of a wave to the least loaded CTA; the result is the same bit for bit
- * as without it, only the load is balanced.  passes in [1, 8]; ws: device
- * memory of svsa_attn_split_workspace_bytes(s, passes) bytes (with passes = 1
- * and ws = NULL or ws_bytes = 0 this is a plain svsa_attn_fwd call). */
+ * ascending (as svsa_build_mask writes them).  With passes > 1, every pass's
+ * work items (query blocks) are assigned to the kernel's persistent CTAs by
+ * a schedule computed on the device from the kept counts: wave by wave, the
+ * costliest item of a wave to the least loaded CTA; the result is the same
+ * bit for bit as without it, only the load is balanced.  passes in [1, 8]
+ * (1 = a plain svsa_attn_fwd call, no workspace needed); ws: device memory of
+ * svsa_attn_split_workspace_bytes(s, passes) bytes. */
 size_t svsa_attn_split_workspace_bytes(svsa_shape s, int32_t passes);
 svsa_status svsa_attn_fwd_split(const void* qp, const void* kp, const void* vp, const svsa_mask* m,
                                 int32_t compensate, void* op, float* lse, svsa_shape s, int32_t passes, void* ws,

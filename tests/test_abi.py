@@ -112,14 +112,14 @@ def test_workspace_queries():
     # least its fp32 partial output [BH, Npad, d] and lse, the exclusive lists
     # [BH, nb, nb] and counts; key-range passes add their lists and outputs
     rows, npad = 12 * nb, nb * 64
-    # one pass: only the item schedule (an int32 per query block and a wave's slack)
-    assert rows * 4 <= svsa.svsa_attn_split_workspace_bytes(s, 1) <= (rows + 256) * 4 + 256
+    assert svsa.svsa_attn_split_workspace_bytes(s, 1) == 0
     need1 = 12 * npad * 128 * 4 + 12 * npad * 4 + rows * nb * 4 + rows * 4
     assert svsa.svsa_attn_paired_workspace_bytes(s, 1) >= need1
     for P in (2, 3, 8):
         R = -(-nb // P)
         split = svsa.svsa_attn_split_workspace_bytes(s, P)
-        assert split >= P * (rows * R * 4 + rows * 4 + 12 * npad * 128 * 4 + 12 * npad * 4)
+        # range lists and counts, fp32 outputs and lse, the item schedule
+        assert split >= P * (rows * R * 4 + rows * 4 + 12 * npad * 128 * 4 + 12 * npad * 4 + rows * 4)
         assert svsa.svsa_attn_paired_workspace_bytes(s, P) >= split + 12 * npad * 128 * 4 + rows * R * 4
     for P in (0, 9):
         assert svsa.svsa_attn_split_workspace_bytes(s, P) == 0
