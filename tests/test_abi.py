@@ -170,6 +170,29 @@ def test_reorder_and_attention_reject_before_launch():
     assert lib.svsa_attn_fwd(16, 32, 48, None, 0, 64, None, s, None) == 1
 
 
+def test_split_and_paired_attention_reject_before_launch():
+    lib = _raw()
+    s = svsa.shape(1, 2, 4, 8, 8, 128)                                    # nb = 4
+    m = Mask(16, 32, 4, None, None, None, None, None, None, 0)
+    ws_need = svsa.svsa_attn_split_workspace_bytes(s, 2)
+    assert ws_need > 0
+    # passes outside [1, 8]
+    for P in (0, 9):
+        assert lib.svsa_attn_fwd_split(16, 32, 48, ctypes.byref(m), 0, 64, None, s, P, 80, 1 << 30, None) == 1
+        assert lib.svsa_attn_fwd_paired(16, 32, 48, ctypes.byref(m), 0, 64, None, s, P, 80, 1 << 30, None) == 1
+    # a workspace smaller than the query
+    assert lib.svsa_attn_fwd_split(16, 32, 48, ctypes.byref(m), 0, 64, None, s, 2, 80, ws_need - 1, None) == 3
+    assert lib.svsa_attn_fwd_split(16, 32, 48, ctypes.byref(m), 0, 64, None, s, 2, None, ws_need, None) == 1
+    # the paired split needs the kept-block bitmap, and its own (larger) workspace
+    assert lib.svsa_attn_fwd_paired(16, 32, 48, ctypes.byref(m), 0, 64, None, s, 1, 80, 1 << 30, None) == 1
+    assert "bits" in _err()
+    mb = Mask(16, 32, 4, 96, None, None, None, None, None, 0)
+    need_p = svsa.svsa_attn_paired_workspace_bytes(s, 1)
+    assert lib.svsa_attn_fwd_paired(16, 32, 48, ctypes.byref(mb), 0, 64, None, s, 1, 80, need_p - 1, None) == 3
+    # the output may not alias an input
+    assert lib.svsa_attn_fwd_paired(16, 32, 48, ctypes.byref(mb), 0, 16, None, s, 1, 80, need_p, None) == 1
+
+
 def test_build_mask_rejects_before_launch():
     lib = _raw()
     s = svsa.shape(1, 2, 4, 8, 8, 128)                                    # nb = 4
