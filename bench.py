@@ -504,8 +504,10 @@ def run_svsa(args):
             if layer is None:
                 attn.forward_host(hq[st], hk[st], hv, hout, step=0, reuse_mask=st > 0, groups=e2e_groups)
             else:
+                # (the pinned inputs are ready: each step's copies may overlap the previous step's work)
                 svsa.svsa_layer_forward_host(layer, hq[st], hk[st], hv, hout, step=0,
-                                             flags=svsa.LAYER_REUSE_MASK if st > 0 else 0, stream=stream)
+                                             flags=svsa.LAYER_INPUTS_READY | (svsa.LAYER_REUSE_MASK if st > 0 else 0),
+                                             stream=stream)
 
     try:
         e2e_ms = _max_over_ranks(_timed(e2e_cycle, stream, flush, args.warmup, args.steps), ws)

@@ -57,6 +57,7 @@ class LayerConfig(ctypes.Structure):
 
 
 LAYER_REUSE_MASK = 1
+LAYER_INPUTS_READY = 2
 
 
 class Schedule(ctypes.Structure):

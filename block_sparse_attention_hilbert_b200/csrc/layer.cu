@@ -1,6 +1,7 @@
 // The whole layer on host buffers (svsa_layer_*): a layer object owns one
-// device arena holding every buffer of the four steps, plus two copy streams
-// and the events that chain them to the caller's stream.  A call streams the
+// device arena holding every buffer of the four steps (with two sets of input
+// staging, used in turn), plus two copy streams and the events that chain
+// them to the caller's stream.  A call streams the
 // (batch, head) rows in groups -- inputs in on one stream, the four steps on
 // the caller's stream, the output out on another -- through the library's
 // own entry points, one group's copies overlapping another group's work.
@@ -26,14 +27,17 @@ struct svsa_layer {
   void *perm_ws = nullptr, *mask_ws = nullptr, *attn_ws = nullptr;
   size_t perm_ws_bytes = 0, mask_ws_bytes = 0, attn_ws_bytes = 0;
   void *qp = nullptr, *kp = nullptr, *vp = nullptr, *op = nullptr;
-  void *sq = nullptr, *sk = nullptr, *sv = nullptr, *so = nullptr;   // raster staging
+  void *sq[2] = {}, *sk[2] = {}, *sv[2] = {};   // raster input staging, two sets used in turn
+  void* so = nullptr;                           // raster output staging
   int32_t *kv_idx = nullptr, *kv_cnt = nullptr, *nvalid = nullptr;
   uint32_t* bits = nullptr;
   float *kbar = nullptr, *vbar = nullptr;
   void* cbar = nullptr;
   cudaStream_t h2d = nullptr, d2h = nullptr;
   cudaEvent_t ev_start = nullptr, ev_done = nullptr;
-  std::vector<cudaEvent_t> ev_in, ev_out;
+  cudaEvent_t ev_free[2] = {};                  // the caller's stream has read input set i
+  std::vector<cudaEvent_t> ev_in[2], ev_out;    // per group: inputs of set i arrived / output ready
+  unsigned long long calls = 0;
   std::vector<long long> bounds;   // row group bounds
   bool mask_ready = false;
 };
@@ -68,7 +72,7 @@ bool needs_bits(const svsa_layer_config& c) { return c.compensate != 0 || c.pair
 
 // Offsets of every buffer in the arena (256-byte aligned).
 struct Arena {
-  size_t perm, iperm, perm_ws, qp, kp, vp, op, sq, sk, sv, so, kv_idx, kv_cnt, nvalid, bits, kbar, vbar,
+  size_t perm, iperm, perm_ws, qp, kp, vp, op, sq[2], sk[2], sv[2], so, kv_idx, kv_cnt, nvalid, bits, kbar, vbar,
       cbar, mask_ws, attn_ws, total;
 };
 
@@ -99,7 +103,10 @@ svsa_status layout(const svsa_shape& s, const svsa_layer_config& c, Arena& A, si
   A.iperm = take((size_t)g.N * 4);
   A.perm_ws = take(perm_ws_bytes);
   A.qp = take(tok); A.kp = take(tok); A.vp = take(tok); A.op = take(tok);
-  A.sq = take(raw); A.sk = take(raw); A.sv = take(raw); A.so = take(raw);
+  for (int i = 0; i < 2; ++i) {
+    A.sq[i] = take(raw); A.sk[i] = take(raw); A.sv[i] = take(raw);
+  }
+  A.so = take(raw);
   A.kv_idx = take(rows * nb * nb * 4);            // cap = nb
   A.kv_cnt = take(rows * nb * 4);
   A.nvalid = take(needs_means(c) ? nb * 4 : 0);
@@ -114,7 +121,10 @@ svsa_status layout(const svsa_shape& s, const svsa_layer_config& c, Arena& A, si
 }
 
 void release(svsa_layer* L) {
-  for (cudaEvent_t e : L->ev_in) if (e) cudaEventDestroy(e);
+  for (int i = 0; i < 2; ++i) {
+    for (cudaEvent_t e : L->ev_in[i]) if (e) cudaEventDestroy(e);
+    if (L->ev_free[i]) cudaEventDestroy(L->ev_free[i]);
+  }
   for (cudaEvent_t e : L->ev_out) if (e) cudaEventDestroy(e);
   if (L->ev_start) cudaEventDestroy(L->ev_start);
   if (L->ev_done) cudaEventDestroy(L->ev_done);
@@ -175,7 +185,10 @@ svsa_status svsa_layer_create(svsa_shape s, const svsa_layer_config* cfg, svsa_l
   L->perm_ws = perm_ws ? at(A.perm_ws) : nullptr;
   L->perm_ws_bytes = perm_ws;
   L->qp = at(A.qp); L->kp = at(A.kp); L->vp = at(A.vp); L->op = at(A.op);
-  L->sq = at(A.sq); L->sk = at(A.sk); L->sv = at(A.sv); L->so = at(A.so);
+  for (int i = 0; i < 2; ++i) {
+    L->sq[i] = at(A.sq[i]); L->sk[i] = at(A.sk[i]); L->sv[i] = at(A.sv[i]);
+  }
+  L->so = at(A.so);
   L->kv_idx = static_cast<int32_t*>(at(A.kv_idx));
   L->kv_cnt = static_cast<int32_t*>(at(A.kv_cnt));
   L->nvalid = needs_means(*cfg) ? static_cast<int32_t*>(at(A.nvalid)) : nullptr;
@@ -200,10 +213,14 @@ svsa_status svsa_layer_create(svsa_shape s, const svsa_layer_config* cfg, svsa_l
   if (st == SVSA_OK) st = cuda_err(cudaStreamCreateWithFlags(&L->d2h, cudaStreamNonBlocking), "copy stream");
   if (st == SVSA_OK) st = cuda_err(cudaEventCreateWithFlags(&L->ev_start, cudaEventDisableTiming), "event");
   if (st == SVSA_OK) st = cuda_err(cudaEventCreateWithFlags(&L->ev_done, cudaEventDisableTiming), "event");
-  L->ev_in.assign(ng, nullptr);
+  for (int k = 0; k < 2; ++k) {
+    L->ev_in[k].assign(ng, nullptr);
+    if (st == SVSA_OK) st = cuda_err(cudaEventCreateWithFlags(&L->ev_free[k], cudaEventDisableTiming), "event");
+  }
   L->ev_out.assign(ng, nullptr);
   for (size_t i = 0; i < ng && st == SVSA_OK; ++i) {
-    st = cuda_err(cudaEventCreateWithFlags(&L->ev_in[i], cudaEventDisableTiming), "event");
+    st = cuda_err(cudaEventCreateWithFlags(&L->ev_in[0][i], cudaEventDisableTiming), "event");
+    if (st == SVSA_OK) st = cuda_err(cudaEventCreateWithFlags(&L->ev_in[1][i], cudaEventDisableTiming), "event");
     if (st == SVSA_OK) st = cuda_err(cudaEventCreateWithFlags(&L->ev_out[i], cudaEventDisableTiming), "event");
   }
   if (st != SVSA_OK) return fail_free(st);
@@ -221,7 +238,8 @@ svsa_status svsa_layer_forward_host(svsa_layer* L, const void* q, const void* k,
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr)
     return err(SVSA_ERR_INVALID_ARG, "a host buffer is NULL");
   if (step < 0) return err(SVSA_ERR_INVALID_ARG, "step=%lld < 0", step);
-  if (flags & ~(int32_t)SVSA_LAYER_REUSE_MASK) return err(SVSA_ERR_INVALID_ARG, "unknown flags %lld", flags);
+  if (flags & ~(int32_t)(SVSA_LAYER_REUSE_MASK | SVSA_LAYER_INPUTS_READY))
+    return err(SVSA_ERR_INVALID_ARG, "unknown flags %lld", flags);
   int dev = -1;
   LTRY(cuda_err(cudaGetDevice(&dev), "cudaGetDevice"));
   if (dev != L->device) return err(SVSA_ERR_INVALID_ARG, "current device %lld, layer on %lld", dev, L->device);
@@ -235,19 +253,25 @@ svsa_status svsa_layer_forward_host(svsa_layer* L, const void* q, const void* k,
   auto raw = [&](const void* base, long long r) { return static_cast<const char*>(base) + r * row_raw; };
   auto rawm = [&](void* base, long long r) { return static_cast<char*>(base) + r * row_raw; };
   auto tokm = [&](void* base, long long r) { return static_cast<char*>(base) + r * row_tok; };
-  // the copy streams start after what the caller's stream has queued (which
-  // includes the previous call's last output copy)
+  // Input set of this call (the two sets alternate).  The output copies start
+  // after what the caller's stream has queued (which includes the previous
+  // call's last output copy); so do the input copies, unless the caller
+  // declares its host inputs ready -- then they wait only until the call two
+  // back has read this set, and overlap the previous call's work.
+  const int set = (int)(L->calls++ & 1ull);
   LTRY(cuda_err(cudaEventRecord(L->ev_start, cs), "event record"));
-  LTRY(cuda_err(cudaStreamWaitEvent(L->h2d, L->ev_start, 0), "stream wait"));
+  LTRY(cuda_err(cudaStreamWaitEvent(L->h2d, (flags & SVSA_LAYER_INPUTS_READY) ? L->ev_free[set] : L->ev_start, 0),
+                "stream wait"));
   LTRY(cuda_err(cudaStreamWaitEvent(L->d2h, L->ev_start, 0), "stream wait"));
+  void *sq = L->sq[set], *sk = L->sk[set], *sv = L->sv[set];
   // every group's inputs first, so the link stays busy whatever the host's launch rate
   for (size_t gi = 0; gi < ng; ++gi) {
     const long long r0 = L->bounds[gi], r1 = L->bounds[gi + 1];
     const size_t bytes = (size_t)(r1 - r0) * row_raw;
-    LTRY(cuda_err(cudaMemcpyAsync(rawm(L->sq, r0), raw(q, r0), bytes, cudaMemcpyHostToDevice, L->h2d), "copy in"));
-    LTRY(cuda_err(cudaMemcpyAsync(rawm(L->sk, r0), raw(k, r0), bytes, cudaMemcpyHostToDevice, L->h2d), "copy in"));
-    LTRY(cuda_err(cudaMemcpyAsync(rawm(L->sv, r0), raw(v, r0), bytes, cudaMemcpyHostToDevice, L->h2d), "copy in"));
-    LTRY(cuda_err(cudaEventRecord(L->ev_in[gi], L->h2d), "event record"));
+    LTRY(cuda_err(cudaMemcpyAsync(rawm(sq, r0), raw(q, r0), bytes, cudaMemcpyHostToDevice, L->h2d), "copy in"));
+    LTRY(cuda_err(cudaMemcpyAsync(rawm(sk, r0), raw(k, r0), bytes, cudaMemcpyHostToDevice, L->h2d), "copy in"));
+    LTRY(cuda_err(cudaMemcpyAsync(rawm(sv, r0), raw(v, r0), bytes, cudaMemcpyHostToDevice, L->h2d), "copy in"));
+    LTRY(cuda_err(cudaEventRecord(L->ev_in[set][gi], L->h2d), "event record"));
   }
   for (size_t gi = 0; gi < ng; ++gi) {
     const long long r0 = L->bounds[gi], r1 = L->bounds[gi + 1];
@@ -256,10 +280,10 @@ svsa_status svsa_layer_forward_host(svsa_layer* L, const void* q, const void* k,
     gs.heads = (int32_t)(r1 - r0);
     svsa_mask m = group_mask(L, r0);
     void *gq = tokm(L->qp, r0), *gk = tokm(L->kp, r0), *gv = tokm(L->vp, r0), *go = tokm(L->op, r0);
-    LTRY(cuda_err(cudaStreamWaitEvent(cs, L->ev_in[gi], 0), "stream wait"));
-    LTRY(svsa_reorder(rawm(L->sq, r0), gq, L->perm, gs, cs));
-    LTRY(svsa_reorder(rawm(L->sk, r0), gk, L->perm, gs, cs));
-    LTRY(svsa_reorder_values(rawm(L->sv, r0), gv, L->perm, gs, cs));
+    LTRY(cuda_err(cudaStreamWaitEvent(cs, L->ev_in[set][gi], 0), "stream wait"));
+    LTRY(svsa_reorder(rawm(sq, r0), gq, L->perm, gs, cs));
+    LTRY(svsa_reorder(rawm(sk, r0), gk, L->perm, gs, cs));
+    LTRY(svsa_reorder_values(rawm(sv, r0), gv, L->perm, gs, cs));
     if (build) LTRY(svsa_build_mask(gq, gk, gv, L->perm, gs, &p, &m, L->mask_ws, L->mask_ws_bytes, cs));
     if (L->cfg.paired)
       LTRY(svsa_attn_fwd_paired(gq, gk, gv, &m, L->cfg.compensate, go, nullptr, gs, L->cfg.attn_passes,
@@ -274,6 +298,7 @@ svsa_status svsa_layer_forward_host(svsa_layer* L, const void* q, const void* k,
                                   cudaMemcpyDeviceToHost, L->d2h), "copy out"));
   }
   if (build) L->mask_ready = true;
+  LTRY(cuda_err(cudaEventRecord(L->ev_free[set], cs), "event record"));   // this call's reads of the set
   LTRY(cuda_err(cudaEventRecord(L->ev_done, L->d2h), "event record"));
   return cuda_err(cudaStreamWaitEvent(cs, L->ev_done, 0), "stream wait");
 }

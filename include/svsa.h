@@ -422,7 +422,7 @@ typedef struct {
 typedef struct svsa_layer svsa_layer;
 
 /* Allocate the layer's device memory on the current device (about
- * B * heads * Npad * d * 18 bytes plus the mask and workspaces) and build its
+ * B * heads * Npad * d * 22 bytes plus the mask and workspaces) and build its
  * token order.  Synchronous.  *out is NULL on failure. */
 svsa_status svsa_layer_create(svsa_shape s, const svsa_layer_config* cfg, svsa_layer** out);
 
@@ -440,11 +440,15 @@ size_t svsa_layer_device_bytes(svsa_shape s, const svsa_layer_config* cfg);
  * host: o is complete when `stream` reaches the point of this call, and the
  * inputs must stay unchanged until then.  step: the denoising step (the
  * structured rule's anchor rotation).  flags: SVSA_LAYER_REUSE_MASK keeps the
- * mask of the previous call (built if there is none).  Calls on one layer
- * must be made from one stream.  The result equals the device-side sequence
- * of svsa_reorder / svsa_reorder_values, svsa_build_mask, the attention entry
- * point and svsa_inverse_reorder on the whole layer. */
-enum { SVSA_LAYER_REUSE_MASK = 1 };
+ * mask of the previous call (built if there is none); SVSA_LAYER_INPUTS_READY
+ * declares that q, k, v are not produced by work still pending on `stream`
+ * (for instance not the o of a call not yet complete), so their copies may
+ * start at once and overlap the previous call's work (the calls alternate
+ * between two input staging sets).  Calls on one layer must be made from one
+ * stream.  The result equals the device-side sequence of svsa_reorder /
+ * svsa_reorder_values, svsa_build_mask, the attention entry point and
+ * svsa_inverse_reorder on the whole layer. */
+enum { SVSA_LAYER_REUSE_MASK = 1, SVSA_LAYER_INPUTS_READY = 2 };
 svsa_status svsa_layer_forward_host(svsa_layer* layer, const void* q, const void* k, const void* v, void* o,
                                     int32_t step, int32_t flags, void* stream);
 

@@ -366,11 +366,28 @@ def test_layer_entry_point_on_host_buffers(select, groups, kw):
                                          flags=svsa.LAYER_REUSE_MASK if reuse else 0)
             torch.cuda.synchronize()
             assert torch.equal(hout, ref), f"step {step}"
+        # three calls queued back to back with their inputs declared ready (the
+        # next call's copies overlap this one's work, the input staging
+        # alternates between two sets), one synchronisation at the end
+        ins, refs, outs = [], [], []
+        for step in (3, 4, 5):
+            q3, k3, v3 = (t.cuda() for t in workloads.make_qkv(w, seed=20 + step))
+            refs.append(ref_layer(q3, k3, v3, step=step, reuse_mask=step > 3).cpu())
+            ins.append(tuple(t.cpu().pin_memory() for t in (q3, k3, v3)))
+            outs.append(torch.empty(q3.shape, dtype=q3.dtype).pin_memory())
+        torch.cuda.synchronize()
+        for i, step in enumerate((3, 4, 5)):
+            svsa.svsa_layer_forward_host(h, *ins[i], outs[i], step=step,
+                                         flags=svsa.LAYER_INPUTS_READY | (svsa.LAYER_REUSE_MASK if step > 3 else 0))
+        torch.cuda.synchronize()
+        for i in range(3):
+            assert torch.equal(outs[i], refs[i]), f"queued call {i}"
+        (hq, hk, hv), ref = ins[2], refs[2]
         # pageable host memory: the copies no longer overlap, the result is the same
         pq, pk, pv = (t.clone() for t in (hq, hk, hv))
-        pout = torch.empty(q.shape, dtype=q.dtype)
+        pout = torch.empty(hq.shape, dtype=hq.dtype)
         assert not pq.is_pinned() and not pout.is_pinned()
-        svsa.svsa_layer_forward_host(h, pq, pk, pv, pout, step=2, flags=svsa.LAYER_REUSE_MASK)
+        svsa.svsa_layer_forward_host(h, pq, pk, pv, pout, step=5, flags=svsa.LAYER_REUSE_MASK)
         torch.cuda.synchronize()
         assert torch.equal(pout, ref)
         svsa.svsa_sync_status()
