@@ -4,16 +4,21 @@
     o = attn(q, k, v)               # q, k, v: bf16 [B, heads, T*H*W, d] on the GPU, raster order
 
 A call runs svsa_reorder (Q, K), svsa_reorder_values (V), svsa_build_mask (unless the cached mask is
-reused across denoising steps -- "DFSAttn" trick 3), svsa_attn_fwd and
-svsa_inverse_reorder on the current stream.  The permutation is built once per
-object.  Buffers are allocated once with torch (the library allocates nothing).
+reused across denoising steps -- "DFSAttn" trick 3), the attention
+(svsa_attn_fwd_split: one pass is a plain svsa_attn_fwd, more passes run over
+key ranges with a balanced item schedule; svsa_attn_fwd_paired with
+paired_split) and svsa_inverse_reorder on the current stream.  The
+permutation is built once per object.  Buffers are allocated once with torch
+(the library allocates nothing).
 
     attn.forward_host(q_h, k_h, v_h, o_h)   # pinned host tensors in and out
 
 runs the same calls on groups of (batch, head) rows, with the host->device
 copies of one group, the library calls of the previous group and the
 device->host copy of the one before overlapping on three streams (every
-(batch, head) row is independent in all four steps).
+(batch, head) row is independent in all four steps).  The library's own
+host-buffer entry point (svsa_layer_create / svsa_layer_forward_host) does the
+same in C with a device arena of its own.
 """
 from __future__ import annotations
 
